@@ -1,0 +1,429 @@
+#!/usr/bin/env python
+"""Forward-pass throughput of the GPT-2 124M decoder (B 12, T 1024, bf16) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one gpt_forward call with targets: embedding, 12 Blocks, ln_f, the tied lm_head
+with the fused cross-entropy, and (with N > 1) the all-reduce of {sum of row losses, count}
+that forms the global loss of a batch-sharded run (weak scaling: every rank runs B 12).
+Inputs (weights, token ids, targets) are resident in HBM before timing; the step touches
+well over the 126 MB L2 (0.25 GB of weights, 1.24 GB of logits), so no flush is needed.
+Rank 0 prints one JSON line.
+
+--impl reference times the fp64 CPU oracle on the host cores on a bounded sample of the
+same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import seeded  # noqa: E402
+
+WORKLOAD = "gpt2"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-kernels", action="store_true", help="skip the per-kernel timings")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------- workload accounting
+def forward_flops(w) -> float:
+    """Algorithmic FLOPs of one forward: 4 GEMMs per layer, the head, and causal attention
+    counted over unmasked (i, j) pairs only."""
+    N, C, L, V, T, B = w.batch * w.seq_len, w.n_embd, w.n_layer, w.vocab_size, w.seq_len, w.batch
+    gemm = 2 * N * (3 * C * C + C * C + 4 * C * C + 4 * C * C) * L
+    head = 2 * N * C * V
+    attn = 2 * B * C * T * (T + 1) * L
+    return float(gemm + head + attn)
+
+
+def attention_flops(B, nh, T, hs) -> float:
+    return float(2 * B * nh * hs * T * (T + 1))
+
+
+def launches_per_forward(w) -> int:
+    return 1 + 7 * w.n_layer + 1 + 3
+
+
+def workload_desc(w) -> str:
+    return (f"GPT-2 124M forward+loss: {w.n_layer} layers, {w.n_head} heads, width {w.n_embd}, "
+            f"vocab {w.vocab_size}, B {w.batch}, T {w.seq_len}, bf16")
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while the timed region runs."""
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.02):
+        self.samples, self.reasons, self.ok = [], set(), False
+        self.period = period_s
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:  # noqa: BLE001
+            self.max_mhz = None
+
+    def _run(self):
+        nv = self.nv
+        get_r = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = get_r(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": len(self.samples)}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------- CPU oracle timing
+def oracle_sample(w, T_sample: int, budget_s: float, max_reps: int = 1000):
+    """Times the fp64 oracle on one sequence of T_sample tokens of the workload (full depth,
+    full width, full vocabulary), repeated until budget_s has passed."""
+    import numpy as np  # noqa: F401
+    import oracle
+    from threadpoolctl import threadpool_info
+    cfg = w.model_dict()
+    W = seeded.to_f64(seeded.make_weights(cfg))
+    idx, tgt = seeded.make_tokens(1, T_sample, w.token_high)
+    idx, tgt = idx.numpy(), tgt.numpy()
+    times = []
+    t_end = time.perf_counter() + budget_s
+    while len(times) < max_reps:
+        t0 = time.perf_counter()
+        oracle.forward(W, cfg, idx, tgt, keep_logits=False)
+        times.append(time.perf_counter() - t0)
+        if time.perf_counter() > t_end:
+            break
+    threads = max([d.get("num_threads", 1) for d in threadpool_info()] + [1])
+    return times, threads
+
+
+# ---------------------------------------------------------------- reference arm
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = seeded.WORKLOADS[WORKLOAD]
+    T_sample = 64
+    import oracle
+    from threadpoolctl import threadpool_info
+    cfg = w.model_dict()
+    W = seeded.to_f64(seeded.make_weights(cfg))
+    idx, tgt = seeded.make_tokens(1, T_sample, w.token_high)
+    idx, tgt = idx.numpy(), tgt.numpy()
+    for _ in range(args.warmup):
+        oracle.forward(W, cfg, idx, tgt, keep_logits=False)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.forward(W, cfg, idx, tgt, keep_logits=False)
+    dt = time.perf_counter() - t0
+    threads = max([d.get("num_threads", 1) for d in threadpool_info()] + [1])
+    value = T_sample * args.steps / dt
+    sample = (f"one sequence of {T_sample} tokens of the workload (all {w.n_layer} layers, width "
+              f"{w.n_embd}, vocab {w.vocab_size}) per step, fp64 numpy oracle")
+    line = {
+        "impl": "reference", "metric": "forward tokens/sec (GPT-2 124M, T=1024, bf16)",
+        "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1000 * dt / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": workload_desc(w), "global_batch": w.batch, "seq_len": w.seq_len,
+                   "parallelism": "none (host cores)", "sample_seq_len": T_sample},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- our arm
+def time_region(fn, iters: int, stream) -> float:
+    """Average ms per call of fn() over iters calls, CUDA events on `stream`."""
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    start.record(stream)
+    for _ in range(iters):
+        fn()
+    end.record(stream)
+    torch.cuda.synchronize()
+    return start.elapsed_time(end) / iters
+
+
+def kernel_timings(w, model, native, dev, stream):
+    """Average duration of each kernel of the forward pass, launched alone through the C ABI
+    on the shapes the forward uses (inputs > L2 for the GEMMs on the token dimension)."""
+    N, C, V = w.batch * w.seq_len, w.n_embd, w.vocab_size
+    g = torch.Generator(device=dev).manual_seed(7)
+    bf = torch.bfloat16
+    u = torch.randn((N, C), generator=g, device=dev).to(bf)
+    hbuf = torch.randn((N, 4 * C), generator=g, device=dev).to(bf)
+    Wa = (0.02 * torch.randn((3 * C, C), generator=g, device=dev)).to(bf)
+    Wp = (0.02 * torch.randn((C, C), generator=g, device=dev)).to(bf)
+    Wf = (0.02 * torch.randn((4 * C, C), generator=g, device=dev)).to(bf)
+    W2 = (0.02 * torch.randn((C, 4 * C), generator=g, device=dev)).to(bf)
+    b3, b1, b4 = (torch.zeros(n, device=dev, dtype=bf) for n in (3 * C, C, 4 * C))
+    qkv_out = torch.empty((N, 3 * C), device=dev, dtype=bf)
+    x = torch.zeros((N, C), device=dev)
+    h_out = torch.empty((N, 4 * C), device=dev, dtype=bf)
+    q, k, v = (torch.randn((w.batch, w.n_head, w.seq_len, C // w.n_head), generator=g, device=dev).to(bf)
+               for _ in range(3))
+    y = torch.empty_like(q)
+    wte = (0.02 * torch.randn((V, C), generator=g, device=dev)).to(bf)
+    _, tgt = seeded.make_tokens(1, N, w.token_high)
+    tgt = tgt.reshape(-1).to(dev)
+    logits = torch.empty((N, V), device=dev, dtype=bf)
+    loss = torch.empty((), device=dev)
+    lm_ws = native.alloc_workspace(native.lm_head_workspace_bytes(N, V), dev)
+    xf = torch.randn((N, C), generator=g, device=dev)
+    ln_w, ln_b = torch.ones(C, device=dev, dtype=bf), torch.zeros(C, device=dev, dtype=bf)
+    ln_out = torch.empty((N, C), device=dev, dtype=bf)
+    ops = {
+        "gemm_c_attn": (lambda: native.linear(u, Wa, b3, out=qkv_out, stream=stream), 2.0 * N * 3 * C * C, "tensor", w.n_layer),
+        "attention": (lambda: native.attention(q, k, v, y=y, stream=stream),
+                      attention_flops(w.batch, w.n_head, w.seq_len, C // w.n_head), "tensor", w.n_layer),
+        "gemm_attn_proj_resid": (lambda: native.linear(u, Wp, b1, out=x, epilogue=native.GPT_EPI_RESID, stream=stream),
+                                 2.0 * N * C * C, "tensor", w.n_layer),
+        "gemm_c_fc_gelu": (lambda: native.linear(u, Wf, b4, out=h_out, epilogue=native.GPT_EPI_GELU, stream=stream),
+                           2.0 * N * 4 * C * C, "tensor", w.n_layer),
+        "gemm_mlp_proj_resid": (lambda: native.linear(hbuf, W2, b1, out=x, epilogue=native.GPT_EPI_RESID, stream=stream),
+                                2.0 * N * 4 * C * C, "tensor", w.n_layer),
+        "lm_head_ce": (lambda: native.lm_head_loss(u, wte, tgt, workspace=lm_ws, logits=logits, loss=loss, stream=stream),
+                       2.0 * N * C * V, "tensor", 1),
+        "layernorm": (lambda: native.layernorm(xf, ln_w, ln_b, out=ln_out, stream=stream), N * C * (4 + 2) + 4 * C,
+                      "hbm", 2 * w.n_layer + 1),
+    }
+    out = {}
+    for name, (fn, work, bound, per_fwd) in ops.items():
+        for _ in range(3):
+            fn()
+        iters = 20
+        ms = time_region(fn, iters, stream)
+        out[name] = {"ms": ms, "work": work, "bound": bound, "per_forward": per_fwd}
+    return out
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    assert args.warmup >= 3, "at least 3 warm-up steps"
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+
+    from decoder_only_transformer_causal_b200 import GPT, GPTConfig, native
+
+    w = seeded.WORKLOADS[WORKLOAD]
+    cfg = GPTConfig.from_dict(w.model_dict())
+    model = GPT(cfg, seeded.make_weights(w.model_dict(), seed=seeded.BASE_SEED + 17 * rank, device=str(dev)), dev)
+    idx_h, tgt_h = seeded.make_tokens(w.batch, w.seq_len, w.token_high, seed=seeded.BASE_SEED + 100_000 + rank)
+    idx, tgt = idx_h.to(dev), tgt_h.to(dev)
+    ws = model.workspace(w.batch, w.seq_len)
+    logits = torch.empty((w.batch, w.seq_len, w.vocab_size), dtype=torch.bfloat16, device=dev)
+    loss = torch.empty((), dtype=torch.float32, device=dev)
+    sc = torch.empty(2, dtype=torch.float64, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        native.forward(cfg, model.weights, idx, tgt, ws, logits=logits, loss=loss, loss_sum_count=sc,
+                       stream=stream)
+        if dist is not None:
+            dist.all_reduce(sc)          # global {sum of row losses, count}
+
+    # correctness guard before timing: the status word must be clean
+    native.forward(cfg, model.weights, idx, tgt, ws, logits=logits, loss=loss, sync_check=True)
+    for _ in range(args.warmup):
+        step()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks:
+        start.record(stream)
+        for _ in range(args.steps):
+            step()
+        end.record(stream)
+        torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    ms_total = start.elapsed_time(end)
+    t = torch.tensor([ms_total], device=dev)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_total = float(t)
+    status = native.check_status(ws)
+    tokens = world * w.batch * w.seq_len * args.steps
+    value = tokens / (ms_total / 1000.0)
+    ms_step = ms_total / args.steps
+
+    # end to end through the public call with host buffers (pinned), loss read back each step
+    idx_p, tgt_p = idx_h.pin_memory(), tgt_h.pin_memory()
+    for _ in range(3):
+        model.forward_host(idx_p, tgt_p)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_steps = max(3, args.steps // 2)
+    e_start.record(stream)
+    for _ in range(e_steps):
+        model.forward_host(idx_p, tgt_p)
+    e_end.record(stream)
+    torch.cuda.synchronize()
+    te = torch.tensor([e_start.elapsed_time(e_end)], device=dev)
+    if dist is not None:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_value = world * w.batch * w.seq_len * e_steps / (float(te) / 1000.0)
+
+    peaks, peak_src = load_peaks()
+    line = None
+    if rank == 0:
+        fwd_fl = forward_flops(w)
+        line = {
+            "metric": "forward tokens/sec (GPT-2 124M, T=1024, bf16)",
+            "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded GPT-2-init weights, uniform token ids)",
+            "config": {"workload": workload_desc(w), "global_batch": w.batch * world, "seq_len": w.seq_len,
+                       "parallelism": f"dp{world}",
+                       "l2": "no flush: each step touches > 1.4 GB (weights 0.25 GB, logits 1.24 GB) vs 126 MB L2"},
+            "status": native.status_string(status),
+            "e2e": {"value": e2e_value, "unit": "tokens/s",
+                    "h2d_bytes_per_step": int(idx_h.numel() * 8 + tgt_h.numel() * 8),
+                    "d2h_bytes_per_step": 4},
+            "gpu_launches": launches_per_forward(w) * args.steps,
+            "forward": {"tflops": fwd_fl / (ms_step / 1000.0) / 1e12 * world,
+                        "flops_per_step_per_gpu": fwd_fl,
+                        "frac_of_sustained_bf16": fwd_fl / (ms_step / 1000.0) / 1e12 /
+                        peaks["bf16_tflops_sustained"], "peak_source": peak_src},
+            "clocks": clocks.summary(),
+        }
+    if not args.no_kernels and rank == 0:
+        kt = kernel_timings(w, model, native, dev, stream)
+        # dominant kernel: largest time share of one forward
+        share = {k: v["ms"] * v["per_forward"] for k, v in kt.items()}
+        dom = max(share, key=share.get)
+        d = kt[dom]
+        if d["bound"] == "tensor":
+            achieved = d["work"] / (d["ms"] / 1000.0) / 1e12
+            peak = peaks["bf16_tflops"]
+            unit = "TFLOP/s"
+        else:
+            achieved = d["work"] / (d["ms"] / 1000.0) / 1e9
+            peak = peaks["hbm_gbs"]
+            unit = "GB/s"
+        line["roofline"] = {"kernel": dom, "bound": d["bound"], "achieved": achieved, "peak": peak,
+                            "unit": unit, "frac": achieved / peak, "traffic": traffic_for(dom),
+                            "peak_source": f"{peak_src} (burst, kernel timed alone)",
+                            "work_per_launch": d["work"], "ms_per_launch": d["ms"]}
+        a = kt["attention"]
+        a_tf = a["work"] / (a["ms"] / 1000.0) / 1e12
+        line["attention"] = {"workload": "causal attention B 12, 12 heads, T 1024, hs 64, bf16",
+                             "tflops": a_tf, "ms": a["ms"], "frac_of_bf16_peak": a_tf / peaks["bf16_tflops"],
+                             "flops": a["work"], "peak_source": peak_src}
+        line["kernels_ms_per_forward"] = {k: round(v, 4) for k, v in share.items()}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        times, threads = oracle_sample(w, 256, budget_s=12.0)
+        tok_s = 256 * len(times) / sum(times)
+        line["cpu_baseline"] = {"value": tok_s, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                                "sample": f"{len(times)} x one sequence of 256 tokens of the workload (all "
+                                          f"{w.n_layer} layers, full vocab), fp64 numpy oracle"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def traffic_for(kernel: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, if it was taken on the
+    current source of that kernel; else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(kernel)
+    if not e:
+        return None
+    src = os.path.join(ROOT, e["source"])
+    if not os.path.exists(src):
+        return None
+    with open(src, "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()[:16]
+    return e["bytes_per_launch"] if sha == e.get("source_sha") else None
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,68 @@
+"""B200-native GPT-2 / nanoGPT causal decoder forward pass.
+
+The compute lives in libgptb200.so (hand-written sm_100a CUDA behind the C ABI of
+include/gpt.h); this package is its ctypes binding (``native``) plus a small model wrapper
+that owns the packed weights and a workspace.  Importing the package loads the library and
+raises if it is missing: there is no CPU path.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import native
+from .native import GPTConfig, GPTError  # noqa: F401
+
+__all__ = ["GPT", "GPTConfig", "GPTError", "native"]
+
+
+class GPT:
+    """A model instance: packed device weights + a cached workspace.
+
+    ``model(idx, targets)`` is GPT.forward(idx, targets) of the pages ("nanoGPT 全局流程图",
+    §3.2) on device tensors: (logits [B, T, V], loss) with targets, (logits [B, 1, V], None)
+    without.  ``forward_host`` takes CPU tensors and returns the loss as a Python float,
+    copying inputs in and the result out (the end-to-end call).
+    """
+
+    def __init__(self, cfg: GPTConfig, tensors: dict, device="cuda"):
+        self.cfg = cfg
+        self.device = torch.device(device)
+        self.weights = native.pack_weights(cfg, tensors, self.device)
+        self._ws = None
+        self._ws_bt = None
+        self._host = {}
+
+    def workspace(self, B: int, T: int) -> torch.Tensor:
+        need = native.workspace_bytes(self.cfg, B, T)
+        if need == 0:
+            raise native.GPTError(native.GPT_ERR_BAD_SHAPE, "gpt_workspace_bytes")
+        if self._ws is None or self._ws.numel() < need:
+            self._ws = native.alloc_workspace(need, self.device)
+        return self._ws
+
+    def __call__(self, idx, targets=None, **kw):
+        B, T = idx.shape
+        return native.forward(self.cfg, self.weights, idx, targets, self.workspace(B, T), **kw)
+
+    def block(self, layer: int, x: torch.Tensor, **kw) -> torch.Tensor:
+        B, T, _ = x.shape
+        return native.block(self.cfg, self.weights, layer, x, self.workspace(B, T), **kw)
+
+    def forward_host(self, idx_cpu: torch.Tensor, targets_cpu: torch.Tensor) -> float:
+        """End-to-end: pinned host inputs -> device, forward, loss -> host."""
+        B, T = idx_cpu.shape
+        key = (B, T)
+        if key not in self._host:
+            self._host[key] = (torch.empty((B, T), dtype=torch.int64, device=self.device),
+                               torch.empty((B, T), dtype=torch.int64, device=self.device),
+                               torch.empty((B, T, self.cfg.vocab_size), dtype=self.cfg.torch_dtype,
+                                           device=self.device),
+                               torch.empty((), dtype=torch.float32, device=self.device),
+                               torch.empty((), dtype=torch.float32).pin_memory())
+        d_idx, d_tgt, logits, loss, h_loss = self._host[key]
+        d_idx.copy_(idx_cpu, non_blocking=True)
+        d_tgt.copy_(targets_cpu, non_blocking=True)
+        native.forward(self.cfg, self.weights, d_idx, d_tgt, self.workspace(B, T), logits=logits, loss=loss)
+        h_loss.copy_(loss, non_blocking=True)
+        torch.cuda.current_stream(self.device).synchronize()
+        return float(h_loss)

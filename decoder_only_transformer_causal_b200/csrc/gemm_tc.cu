@@ -1,0 +1,66 @@
+// Host launcher of the tensor-core GEMM (kernel in gemm_tc.cuh).
+#include "gemm_tc.cuh"
+#include "internal.h"
+
+namespace gpt {
+
+namespace {
+
+constexpr int kBN = 256;
+
+template <int EPI, int NEPI>
+int launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const gemm::Params& p, cudaStream_t s) {
+    using L = gemm::Cfg<kBN, NEPI>;
+    auto kern = gemm::gemm_bf16_tc<kBN, EPI, NEPI>;
+    static bool configured = false;
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_BYTES);
+        if (e != cudaSuccess) return cuda_status(e);
+        configured = true;
+    }
+    const int tiles = ((p.M + gemm::BM - 1) / gemm::BM) * ((p.N + kBN - 1) / kBN);
+    const int grid = tiles < num_sms() ? tiles : num_sms();
+    kern<<<grid, L::THREADS, L::SMEM_BYTES, s>>>(ta, tb, p);
+    return cuda_status(cudaGetLastError());
+}
+
+}  // namespace
+
+int gemm_ce_parts(int N) { return ((N + kBN - 1) / kBN) * gemm::Cfg<kBN, 8>::PARTS_PER_TILE; }
+
+int launch_gemm_bf16(const bf16* A, long long lda, const bf16* W, long long ldw, const bf16* bias,
+                     void* out, long long ldo, int M, int N, int K, int epilogue, int gelu,
+                     const CeArgs* ce, int32_t* status, cudaStream_t s) {
+    if (M == 0 || N == 0) return GPT_OK;
+    CUtensorMap ta, tb;
+    int rc = make_tmap_bf16_2d(&ta, A, static_cast<uint64_t>(K), static_cast<uint64_t>(M),
+                               static_cast<uint64_t>(lda) * 2, gemm::BK, gemm::BM);
+    if (rc) return rc;
+    rc = make_tmap_bf16_2d(&tb, W, static_cast<uint64_t>(K), static_cast<uint64_t>(N),
+                           static_cast<uint64_t>(ldw) * 2, gemm::BK, kBN);
+    if (rc) return rc;
+    gemm::Params p{};
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    p.bias = bias;
+    p.out = out;
+    p.ldo = ldo;
+    p.gelu_tanh = gelu == GPT_GELU_TANH;
+    p.status = status;
+    switch (epilogue) {
+        case GPT_EPI_STORE: return launch_one<gemm::EPI_STORE, 4>(ta, tb, p, s);
+        case GPT_EPI_GELU: return launch_one<gemm::EPI_GELU, 8>(ta, tb, p, s);
+        case GPT_EPI_RESID: return launch_one<gemm::EPI_RESID, 4>(ta, tb, p, s);
+        case gemm::EPI_CE:
+            if (!ce) return GPT_ERR_NULL;
+            p.targets = ce->targets;
+            p.part = ce->part;
+            p.tlogit = ce->tlogit;
+            p.n_part = ce->n_part;
+            return launch_one<gemm::EPI_CE, 8>(ta, tb, p, s);
+        default: return GPT_ERR_UNSUPPORTED;
+    }
+}
+
+}  // namespace gpt

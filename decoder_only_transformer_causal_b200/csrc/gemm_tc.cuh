@@ -1,0 +1,334 @@
+// Tensor-core GEMM for sm_100a: Y[M, N] = epilogue(A[M, K] * W[N, K]^T), bf16 operands,
+// fp32 accumulation in tensor memory.
+//
+// Used for every nn.Linear of the forward pass ("nanoGPT 全局流程图", §2.5: c_attn, attn
+// c_proj, c_fc, mlp c_proj) and for the tied lm_head (§3.2 ④), each with its epilogue fused:
+//   EPI_STORE  out_bf16 = acc + b                 (c_attn)
+//   EPI_GELU   out_bf16 = gelu(acc + b)           (c_fc; "nanoGPT架构逐步详解", 4. MLP)
+//   EPI_RESID  x_fp32  += acc + b                 (both c_proj: the residual add of Block)
+//   EPI_CE     logits_bf16 = acc, plus per (row, column slice) the running maximum and the sum
+//              of exp(z - max) and, in the slice holding the row's target, z[target] in fp32:
+//              the pieces of F.cross_entropy's logsumexp (§3.3), reduced by ce_reduce.
+//
+// Design: one persistent CTA per SM walks the output tiles (128 x BN) in m-fastest order so
+// concurrently running CTAs share the same W columns in L2.  Warp 0 streams 128x64 A and
+// BNx64 W tiles with TMA (128-byte swizzle) through a kStages-deep shared-memory ring; one
+// thread of warp 1 issues tcgen05.mma (M=128, N=BN, K=16) into one of two TMEM accumulators;
+// the epilogue warps drain the other accumulator (tcgen05.ld) while the next tile's MMAs
+// run.  Every wait is bounded (common.cuh).
+#pragma once
+
+#include "common.cuh"
+
+namespace gpt {
+namespace gemm {
+
+constexpr int BM = 128;
+constexpr int BK = 64;  // one 128-byte swizzle row of bf16
+constexpr int kStages = 4;
+
+enum Epi { EPI_STORE = 0, EPI_GELU = 1, EPI_RESID = 2, EPI_CE = 3 };
+
+struct Params {
+    int M, N, K;
+    const bf16* bias;  // [N] or nullptr
+    void* out;         // bf16 [M, ldo] (STORE / GELU / CE logits) or fp32 [M, ldo] (RESID)
+    long long ldo;
+    int gelu_tanh;
+    const int64_t* targets;  // EPI_CE: [M]
+    float2* part;            // EPI_CE: [M, n_part] of (max, sum exp(z - max))
+    float* tlogit;           // EPI_CE: [M], z[target] in fp32
+    int n_part;
+    int32_t* status;
+};
+
+template <int BN, int NEPI>
+struct Cfg {
+    static_assert(BN == 128 || BN == 256, "BN");
+    static_assert(NEPI == 4 || NEPI == 8, "NEPI");
+    static constexpr int A_BYTES = BM * BK * 2;
+    static constexpr int B_BYTES = BN * BK * 2;
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int BAR_OFF = kStages * STAGE_BYTES;
+    static constexpr int SMEM_BYTES = BAR_OFF + 256 + 1024;  // barriers + alignment slack
+    static constexpr int TMEM_COLS = 2 * BN;                  // two accumulators
+    static constexpr int THREADS = 64 + NEPI * 32;
+    static constexpr int COLS_PER_WARP = BN / (NEPI / 4);
+    static constexpr int PARTS_PER_TILE = NEPI / 4;
+};
+
+GPT_DEVINL float gelu_f(float v, int tanh_mode) {
+    if (tanh_mode) {
+        const float k0 = 0.7978845608028654f;  // sqrt(2/pi)
+        return 0.5f * v * (1.0f + tanhf(k0 * (v + 0.044715f * v * v * v)));
+    }
+    return 0.5f * v * (1.0f + erff(v * 0.7071067811865476f));
+}
+
+template <int BN, int EPI, int NEPI>
+__global__ void __launch_bounds__(Cfg<BN, NEPI>::THREADS, 1)
+    gemm_bf16_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                 const Params p) {
+    using L = Cfg<BN, NEPI>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
+    uint64_t* empty = full + kStages;
+    uint64_t* tfull = empty + kStages;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* drain = tempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int num_m = (p.M + BM - 1) / BM;
+    const int num_n = (p.N + BN - 1) / BN;
+    const int num_tiles = num_m * num_n;
+    const int num_kb = (p.K + BK - 1) / BK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&tfull[a], 1);
+            mbar_init(&tempty[a], NEPI * 32);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, L::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t ph = 0;
+            long long issued = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+                const int m0 = (tile % num_m) * BM;
+                const int n0 = (tile / num_m) * BN;
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!mbar_wait(&empty[stage], ph ^ 1u, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* st = smem + stage * L::STAGE_BYTES;
+                    mbar_arrive_expect_tx(&full[stage], L::STAGE_BYTES);
+                    tma_load_2d(st, &tmA, &full[stage], kb * BK, m0);
+                    tma_load_2d(st + L::A_BYTES, &tmB, &full[stage], kb * BK, n0);
+                    ++issued;
+                    if (++stage == kStages) {
+                        stage = 0;
+                        ph ^= 1u;
+                    }
+                }
+            }
+            // Make sure no bulk copy is still writing shared memory when the CTA exits: wait
+            // for the latest load issued into each stage (already complete on the normal path).
+            const long long n_check = issued < kStages ? issued : kStages;
+            for (long long i = 1; i <= n_check; ++i) {
+                const long long idx = issued - i;
+                mbar_drain(&full[idx % kStages], static_cast<uint32_t>((idx / kStages) & 1));
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = make_idesc_bf16(BM, BN, false);
+            int stage = 0;
+            uint32_t ph = 0;
+            int acc = 0;
+            uint32_t acc_ph = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+                if (!mbar_wait(&tempty[acc], acc_ph ^ 1u, abort_flag)) break;
+                tc_fence_after();
+                const uint32_t d = tmem_base + static_cast<uint32_t>(acc * BN);
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!mbar_wait(&full[stage], ph, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_addr(smem + stage * L::STAGE_BYTES);
+                    const uint32_t b_addr = a_addr + L::A_BYTES;
+#pragma unroll
+                    for (int k = 0; k < BK / 16; ++k) {
+                        umma_ss(d, make_sdesc_sw128(a_addr + k * 32), make_sdesc_sw128(b_addr + k * 32),
+                                idesc, (kb | k) != 0 ? 1u : 0u);
+                    }
+                    umma_commit(&empty[stage]);
+                    if (++stage == kStages) {
+                        stage = 0;
+                        ph ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                umma_commit(&tfull[acc]);
+                acc ^= 1;
+                if (acc == 0) acc_ph ^= 1u;
+            }
+            // All MMAs issued by this thread must be finished before TMEM is released.
+            umma_commit(drain);
+            mbar_drain(drain, 0);
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue warps
+        const int ew = warp - 2;
+        const int quarter = warp & 3;        // TMEM lanes this warp may access
+        const int half = ew >> 2;            // column slice (NEPI == 8 splits BN in two)
+        int acc = 0;
+        uint32_t acc_ph = 0;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+            const int n_blk = tile / num_m;
+            const int m0 = (tile % num_m) * BM;
+            const int n0 = n_blk * BN;
+            const bool got = mbar_wait(&tfull[acc], acc_ph, abort_flag);
+            __syncwarp();  // tcgen05.ld below is warp-collective
+            if (!__all_sync(0xffffffffu, got)) break;
+            tc_fence_after();
+            const int row = m0 + quarter * 32 + lane;
+            const bool row_ok = row < p.M;
+            const uint32_t tbase = tmem_base + static_cast<uint32_t>(acc * BN + half * L::COLS_PER_WARP) +
+                                   (static_cast<uint32_t>(quarter * 32) << 16);
+            const int nw0 = n0 + half * L::COLS_PER_WARP;  // first column of this warp's slice
+
+            float run_max = -INFINITY, run_sum = 0.f;
+            long long tgt = -1;
+            if (EPI == EPI_CE && row_ok) tgt = p.targets[row];
+
+#pragma unroll 1
+            for (int c = 0; c < L::COLS_PER_WARP; c += 32) {
+                uint32_t r[32];
+                tmem_ld32(tbase + c, r);
+                const int n = nw0 + c;
+                if (n >= p.N) continue;  // slice past the right edge (warp-uniform)
+                const bool full_chunk = (n + 32 <= p.N);
+                float v[32];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+
+                if (EPI == EPI_STORE || EPI == EPI_GELU || EPI == EPI_RESID) {
+                    if (p.bias) {
+                        if (full_chunk) {
+                            const uint4* bp = reinterpret_cast<const uint4*>(p.bias + n);
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) {
+                                uint4 w = __ldg(bp + q);
+                                const bf16* wb = reinterpret_cast<const bf16*>(&w);
+#pragma unroll
+                                for (int e = 0; e < 8; ++e) v[q * 8 + e] += __bfloat162float(wb[e]);
+                            }
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 32; ++j)
+                                if (n + j < p.N) v[j] += __bfloat162float(p.bias[n + j]);
+                        }
+                    }
+                }
+                if (EPI == EPI_GELU) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) v[j] = gelu_f(v[j], p.gelu_tanh);
+                }
+                if (EPI == EPI_STORE || EPI == EPI_GELU || EPI == EPI_CE) {
+                    if (row_ok) {
+                        bf16* o = static_cast<bf16*>(p.out) + static_cast<size_t>(row) * p.ldo + n;
+                        if (full_chunk && (p.ldo % 8) == 0) {
+                            uint4* op = reinterpret_cast<uint4*>(o);
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) {
+                                uint4 w;
+                                w.x = pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]);
+                                w.y = pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]);
+                                w.z = pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]);
+                                w.w = pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]);
+                                op[q] = w;
+                            }
+                        } else {
+                            for (int j = 0; j < 32; ++j)
+                                if (n + j < p.N) o[j] = __float2bfloat16_rn(v[j]);
+                        }
+                    }
+                }
+                if (EPI == EPI_RESID) {
+                    if (row_ok) {
+                        float* o = static_cast<float*>(p.out) + static_cast<size_t>(row) * p.ldo + n;
+                        if (full_chunk && (p.ldo % 4) == 0) {
+                            float4* op = reinterpret_cast<float4*>(o);
+#pragma unroll
+                            for (int q = 0; q < 8; ++q) {
+                                float4 x = op[q];
+                                x.x += v[q * 4 + 0];
+                                x.y += v[q * 4 + 1];
+                                x.z += v[q * 4 + 2];
+                                x.w += v[q * 4 + 3];
+                                op[q] = x;
+                            }
+                        } else {
+                            for (int j = 0; j < 32; ++j)
+                                if (n + j < p.N) o[j] += v[j];
+                        }
+                    }
+                }
+                if (EPI == EPI_CE) {
+                    constexpr float kLog2e = 1.4426950408889634f;
+                    float cmax = -INFINITY;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        if (full_chunk || n + j < p.N) cmax = fmaxf(cmax, v[j]);
+                    const float new_max = fmaxf(run_max, cmax);
+                    float s = 0.f;
+                    const float off = new_max * kLog2e;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        if (full_chunk || n + j < p.N) s += exp2_approx(fmaf(v[j], kLog2e, -off));
+                    run_sum = run_sum * exp2_approx((run_max - new_max) * kLog2e) + s;
+                    run_max = new_max;
+                    const long long rel = tgt - n;
+                    if (rel >= 0 && rel < 32) {
+                        float zt = 0.f;
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            if (j == rel) zt = v[j];
+                        if (row_ok) p.tlogit[row] = zt;
+                    }
+                }
+            }
+            if (EPI == EPI_CE && row_ok) {
+                p.part[static_cast<size_t>(row) * p.n_part + n_blk * L::PARTS_PER_TILE + half] =
+                    make_float2(run_max, run_sum);
+            }
+            tc_fence_before();
+            mbar_arrive(&tempty[acc]);
+            acc ^= 1;
+            if (acc == 0) acc_ph ^= 1u;
+        }
+    }
+
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem_base, L::TMEM_COLS);
+    }
+    if (threadIdx.x == 0 && *abort_flag) set_status(p.status, GPT_ERR_TIMEOUT);
+}
+
+}  // namespace gemm
+}  // namespace gpt

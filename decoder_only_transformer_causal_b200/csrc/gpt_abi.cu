@@ -1,0 +1,518 @@
+// The C ABI declared in include/gpt.h: argument validation, the packed-weight layout, the
+// workspace plan and the launch sequence of the forward pass.  All work runs in the
+// kernels of this library; nothing here computes on the host.
+#include <math.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "internal.h"
+
+#define GPT_API extern "C" __attribute__((visibility("default")))
+
+namespace gpt {
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? GPT_OK : GPT_ERR_CUDA; }
+
+int num_sms() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    static int cached[64] = {0};
+    if (dev < 0 || dev >= 64) dev = 0;
+    if (cached[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
+// ------------------------------------------------------------------ TMA descriptors
+namespace {
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = []() -> EncodeTiledFn {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        return reinterpret_cast<EncodeTiledFn>(p);
+    }();
+    return fn;
+}
+
+int encode(CUtensorMap* m, const void* base, cuuint32_t rank, const cuuint64_t* dims, const cuuint64_t* strides,
+           const cuuint32_t* box) {
+    if (reinterpret_cast<uintptr_t>(base) & 15) return GPT_ERR_BAD_ALIGN;
+    for (cuuint32_t i = 0; i + 1 < rank; ++i)
+        if (strides[i] & 15) return GPT_ERR_BAD_ALIGN;
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return GPT_ERR_CUDA;
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? GPT_OK : GPT_ERR_CUDA;
+}
+}  // namespace
+
+int make_tmap_bf16_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
+                      uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer) {
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {row_stride_bytes};
+    const cuuint32_t box[2] = {box_inner, box_outer};
+    return encode(m, base, 2, dims, strides, box);
+}
+
+int make_tmap_bf16_4d(CUtensorMap* m, const void* base, const uint64_t dims[4], const uint64_t strides_bytes[3],
+                      const uint32_t box[4]) {
+    const cuuint64_t d[4] = {dims[0], dims[1], dims[2], dims[3]};
+    const cuuint64_t s[3] = {strides_bytes[0], strides_bytes[1], strides_bytes[2]};
+    const cuuint32_t b[4] = {box[0], box[1], box[2], box[3]};
+    return encode(m, base, 4, d, s, b);
+}
+
+}  // namespace gpt
+
+using namespace gpt;
+
+namespace {
+
+constexpr int kTensorsPerLayer = 12;
+enum {
+    W_LN1_W = 0, W_LN1_B, W_ATTN_W, W_ATTN_B, W_PROJ_W, W_PROJ_B,
+    W_LN2_W, W_LN2_B, W_FC_W, W_FC_B, W_FC2_W, W_FC2_B
+};
+
+size_t a256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int elem_size(const gpt_config_t* c) { return c->dtype == GPT_DTYPE_BF16 ? 2 : 4; }
+
+int validate(const gpt_config_t* c) {
+    if (!c) return GPT_ERR_NULL;
+    if (c->n_layer < 0 || c->n_head <= 0 || c->n_embd <= 0 || c->block_size <= 0 || c->vocab_size <= 0)
+        return GPT_ERR_BAD_SHAPE;
+    if (c->n_embd % c->n_head) return GPT_ERR_BAD_SHAPE;
+    if (c->dtype != GPT_DTYPE_F32 && c->dtype != GPT_DTYPE_BF16) return GPT_ERR_BAD_SHAPE;
+    if (c->gelu != GPT_GELU_ERF && c->gelu != GPT_GELU_TANH) return GPT_ERR_BAD_SHAPE;
+    if (c->n_embd % 4) return GPT_ERR_UNSUPPORTED;       // 16-byte rows in the row kernels
+    if (c->n_embd > 2048) return GPT_ERR_UNSUPPORTED;    // LayerNorm keeps a row in registers
+    const int hs = c->n_embd / c->n_head;
+    if (c->dtype == GPT_DTYPE_BF16) {
+        if (hs != 64) return GPT_ERR_UNSUPPORTED;        // tensor-core attention tile
+        if (c->n_embd % 8) return GPT_ERR_UNSUPPORTED;   // 16-byte TMA rows
+    } else if (hs > 128) {
+        return GPT_ERR_UNSUPPORTED;
+    }
+    return GPT_OK;
+}
+
+// Offsets (bytes) and element counts of the packed weights, in the documented order.
+int layout(const gpt_config_t* c, size_t* offs, size_t* numels, int n) {
+    const size_t C = c->n_embd, V = c->vocab_size, bs = c->block_size, es = elem_size(c);
+    const int count = 2 + kTensorsPerLayer * c->n_layer + 2;
+    size_t off = 0;
+    int k = 0;
+    auto put = [&](size_t numel) {
+        if (k < n) {
+            if (offs) offs[k] = off;
+            if (numels) numels[k] = numel;
+        }
+        off += a256(numel * es);
+        ++k;
+    };
+    put(V * C);
+    put(bs * C);
+    for (int l = 0; l < c->n_layer; ++l) {
+        put(C); put(C);
+        put(3 * C * C); put(3 * C);
+        put(C * C); put(C);
+        put(C); put(C);
+        put(4 * C * C); put(4 * C);
+        put(4 * C * C); put(C);
+    }
+    put(C);
+    put(C);
+    (void)count;
+    return k;
+}
+
+size_t weights_total(const gpt_config_t* c) {
+    const size_t C = c->n_embd, V = c->vocab_size, bs = c->block_size, es = elem_size(c);
+    size_t per_layer = a256(C * es) * 6 + a256(3 * C * C * es) + a256(3 * C * es) + a256(C * C * es) +
+                       a256(4 * C * C * es) + a256(4 * C * es) + a256(4 * C * C * es);
+    return a256(V * C * es) + a256(bs * C * es) + per_layer * c->n_layer + 2 * a256(C * es);
+}
+
+// Pointers into the packed weight buffer, computed from the same layout as layout().
+struct Weights {
+    const uint8_t* base;
+    const gpt_config_t* c;
+    size_t head, layer_bytes, in_layer[kTensorsPerLayer], tail;
+    const void* wte() const { return base; }
+    const void* wpe() const { return base + a256(static_cast<size_t>(c->vocab_size) * c->n_embd * elem_size(c)); }
+    const void* layer(int l, int which) const { return base + head + layer_bytes * l + in_layer[which]; }
+    const void* bias(int l, int which) const { return c->bias ? layer(l, which) : nullptr; }
+    const void* lnf_w() const { return base + tail; }
+    const void* lnf_b() const {
+        return c->bias ? base + tail + a256(static_cast<size_t>(c->n_embd) * elem_size(c)) : nullptr;
+    }
+};
+
+struct Plan {
+    size_t ctrl, x, u, qkv, y, h, part, tlogit, rowloss, total;
+    int n_part;
+};
+
+Plan plan_ws(const gpt_config_t* c, long long B, long long T) {
+    Plan P{};
+    const size_t N = static_cast<size_t>(B * T), C = c->n_embd, es = elem_size(c);
+    size_t off = 0;
+    P.ctrl = off; off += 256;
+    P.x = off; off += a256(N * C * 4);
+    P.u = off; off += a256(N * C * es);
+    P.qkv = off; off += a256(N * 3 * C * es);
+    P.y = off; off += a256(N * C * es);
+    P.h = off; off += a256(N * 4 * C * es);
+    P.n_part = c->dtype == GPT_DTYPE_BF16 ? gemm_ce_parts(c->vocab_size) : 0;
+    P.part = off; off += a256(N * static_cast<size_t>(P.n_part) * 8);
+    P.tlogit = off; off += a256(N * 4);
+    P.rowloss = off; off += a256(N * 4);
+    P.total = off;
+    return P;
+}
+
+int32_t* status_word(void* ws) { return static_cast<int32_t*>(ws); }
+
+int sync_and_read_status(void* ws, cudaStream_t s) {
+    if (cudaStreamSynchronize(s) != cudaSuccess) return GPT_ERR_CUDA;
+    int32_t st = 0;
+    if (cudaMemcpy(&st, ws, sizeof(st), cudaMemcpyDeviceToHost) != cudaSuccess) return GPT_ERR_CUDA;
+    if (cudaMemset(ws, 0, sizeof(st)) != cudaSuccess) return GPT_ERR_CUDA;
+    return st;
+}
+
+#define GPT_TRY(expr)               \
+    do {                            \
+        int _rc = (expr);           \
+        if (_rc != GPT_OK) return _rc; \
+    } while (0)
+
+// One pre-LN Block ("nanoGPT 全局流程图", §2.5): x += attn(ln_1(x)); x += mlp(ln_2(x)).
+int run_block(const gpt_config_t* c, const Weights& W, int l, float* x, int B, int T, uint8_t* ws,
+              const Plan& P, cudaStream_t s) {
+    const int C = c->n_embd, nh = c->n_head, hs = C / nh;
+    const int N = B * T;
+    int32_t* status = status_word(ws);
+    void* u = ws + P.u;
+    void* qkv = ws + P.qkv;
+    void* y = ws + P.y;
+    void* h = ws + P.h;
+    GPT_TRY(launch_layernorm(x, W.layer(l, W_LN1_W), W.bias(l, W_LN1_B), u, N, C, c->dtype, s));
+    if (c->dtype == GPT_DTYPE_BF16) {
+        const bf16* ub = static_cast<const bf16*>(u);
+        bf16* qkvb = static_cast<bf16*>(qkv);
+        GPT_TRY(launch_gemm_bf16(ub, C, static_cast<const bf16*>(W.layer(l, W_ATTN_W)), C,
+                                 static_cast<const bf16*>(W.bias(l, W_ATTN_B)), qkv, 3LL * C, N, 3 * C, C,
+                                 GPT_EPI_STORE, c->gelu, nullptr, status, s));
+        AttnLayout L{};
+        L.q = qkvb;
+        L.k = qkvb + C;
+        L.v = qkvb + 2 * C;
+        L.sb = 3LL * C * T;
+        L.sh = hs;
+        L.st = 3LL * C;
+        L.y = static_cast<bf16*>(y);
+        L.y_sb = static_cast<long long>(C) * T;
+        L.y_sh = hs;
+        L.y_st = C;
+        GPT_TRY(launch_attention_bf16(L, B, nh, T, status, s));
+        GPT_TRY(launch_gemm_bf16(static_cast<const bf16*>(y), C, static_cast<const bf16*>(W.layer(l, W_PROJ_W)), C,
+                                 static_cast<const bf16*>(W.bias(l, W_PROJ_B)), x, C, N, C, C, GPT_EPI_RESID,
+                                 c->gelu, nullptr, status, s));
+        GPT_TRY(launch_layernorm(x, W.layer(l, W_LN2_W), W.bias(l, W_LN2_B), u, N, C, c->dtype, s));
+        GPT_TRY(launch_gemm_bf16(ub, C, static_cast<const bf16*>(W.layer(l, W_FC_W)), C,
+                                 static_cast<const bf16*>(W.bias(l, W_FC_B)), h, 4LL * C, N, 4 * C, C,
+                                 GPT_EPI_GELU, c->gelu, nullptr, status, s));
+        GPT_TRY(launch_gemm_bf16(static_cast<const bf16*>(h), 4LL * C, static_cast<const bf16*>(W.layer(l, W_FC2_W)),
+                                 4LL * C, static_cast<const bf16*>(W.bias(l, W_FC2_B)), x, C, N, C, 4 * C,
+                                 GPT_EPI_RESID, c->gelu, nullptr, status, s));
+    } else {
+        const float* uf = static_cast<const float*>(u);
+        float* qkvf = static_cast<float*>(qkv);
+        GPT_TRY(launch_linear_f32(uf, C, static_cast<const float*>(W.layer(l, W_ATTN_W)),
+                                  static_cast<const float*>(W.bias(l, W_ATTN_B)), qkvf, 3LL * C, N, 3 * C, C,
+                                  GPT_EPI_STORE, c->gelu, s));
+        AttnLayoutF32 L{};
+        L.q = qkvf;
+        L.k = qkvf + C;
+        L.v = qkvf + 2 * C;
+        L.sb = 3LL * C * T;
+        L.sh = hs;
+        L.st = 3LL * C;
+        L.y = static_cast<float*>(y);
+        L.y_sb = static_cast<long long>(C) * T;
+        L.y_sh = hs;
+        L.y_st = C;
+        GPT_TRY(launch_attention_f32(L, B, nh, T, hs, s));
+        GPT_TRY(launch_linear_f32(static_cast<const float*>(y), C, static_cast<const float*>(W.layer(l, W_PROJ_W)),
+                                  static_cast<const float*>(W.bias(l, W_PROJ_B)), x, C, N, C, C, GPT_EPI_RESID,
+                                  c->gelu, s));
+        GPT_TRY(launch_layernorm(x, W.layer(l, W_LN2_W), W.bias(l, W_LN2_B), u, N, C, c->dtype, s));
+        GPT_TRY(launch_linear_f32(uf, C, static_cast<const float*>(W.layer(l, W_FC_W)),
+                                  static_cast<const float*>(W.bias(l, W_FC_B)), static_cast<float*>(h), 4LL * C, N,
+                                  4 * C, C, GPT_EPI_GELU, c->gelu, s));
+        GPT_TRY(launch_linear_f32(static_cast<const float*>(h), 4LL * C, static_cast<const float*>(W.layer(l, W_FC2_W)),
+                                  static_cast<const float*>(W.bias(l, W_FC2_B)), x, C, N, C, 4 * C, GPT_EPI_RESID,
+                                  c->gelu, s));
+    }
+    return GPT_OK;
+}
+
+void fill_weights(Weights& W, const gpt_config_t* c, const void* base) {
+    W.base = static_cast<const uint8_t*>(base);
+    W.c = c;
+    size_t offs[2 + kTensorsPerLayer + 2];
+    gpt_config_t one = *c;
+    one.n_layer = 1;
+    layout(&one, offs, nullptr, 2 + kTensorsPerLayer + 2);
+    W.head = offs[2];
+    for (int i = 0; i < kTensorsPerLayer; ++i) W.in_layer[i] = offs[2 + i] - W.head;
+    W.layer_bytes = offs[2 + kTensorsPerLayer] - W.head;
+    W.tail = W.head + W.layer_bytes * static_cast<size_t>(c->n_layer);
+}
+
+int check_common(const gpt_config_t* c, const void* weights, int B, int T, void* ws, size_t ws_bytes,
+                 Plan* P) {
+    GPT_TRY(validate(c));
+    if (!weights || !ws) return GPT_ERR_NULL;
+    if (B < 1 || T < 1 || T > c->block_size) return GPT_ERR_BAD_SHAPE;
+    if (static_cast<long long>(B) * T > 0x7fffffffLL / 4 / c->n_embd) return GPT_ERR_UNSUPPORTED;
+    if (!aligned(weights, 256) || !aligned(ws, 256)) return GPT_ERR_BAD_ALIGN;
+    *P = plan_ws(c, B, T);
+    if (ws_bytes < P->total) return GPT_ERR_WS_TOO_SMALL;
+    return GPT_OK;
+}
+
+}  // namespace
+
+// =================================================================== exported ABI
+GPT_API const char* gpt_status_string(int status) {
+    switch (status) {
+        case GPT_OK: return "ok";
+        case GPT_ERR_NULL: return "a required pointer is NULL";
+        case GPT_ERR_BAD_SHAPE: return "inconsistent sizes";
+        case GPT_ERR_BAD_ALIGN: return "pointer not aligned";
+        case GPT_ERR_WS_TOO_SMALL: return "workspace too small";
+        case GPT_ERR_INDEX: return "token id or target out of range";
+        case GPT_ERR_TIMEOUT: return "device pipeline wait timed out";
+        case GPT_ERR_UNSUPPORTED: return "unsupported configuration";
+        case GPT_ERR_CUDA: return "CUDA runtime error";
+        default: return "unknown status";
+    }
+}
+
+GPT_API int gpt_abi_version(void) { return GPT_ABI_VERSION; }
+
+GPT_API int gpt_validate_config(const gpt_config_t* cfg) { return validate(cfg); }
+
+GPT_API size_t gpt_weights_bytes(const gpt_config_t* cfg) {
+    if (validate(cfg) != GPT_OK) return 0;
+    return weights_total(cfg);
+}
+
+GPT_API int gpt_weights_count(const gpt_config_t* cfg) {
+    const int rc = validate(cfg);
+    if (rc != GPT_OK) return rc;
+    return 2 + kTensorsPerLayer * cfg->n_layer + 2;
+}
+
+GPT_API int gpt_weights_layout(const gpt_config_t* cfg, size_t* offsets, size_t* numels, int n) {
+    const int rc = validate(cfg);
+    if (rc != GPT_OK) return rc;
+    return layout(cfg, offsets, numels, n < 0 ? 0 : n);
+}
+
+GPT_API size_t gpt_workspace_bytes(const gpt_config_t* cfg, int B, int T) {
+    if (validate(cfg) != GPT_OK || B < 1 || T < 1 || T > cfg->block_size) return 0;
+    return plan_ws(cfg, B, T).total;
+}
+
+GPT_API int gpt_check_status(void* workspace, void* stream) {
+    if (!workspace) return GPT_ERR_NULL;
+    return sync_and_read_status(workspace, static_cast<cudaStream_t>(stream));
+}
+
+GPT_API int gpt_forward(const gpt_config_t* cfg, const void* weights, const int64_t* idx, const int64_t* targets,
+                        int B, int T, void* logits, float* loss, float* row_loss, double* loss_sum_count,
+                        void* workspace, size_t workspace_bytes, void* stream, int flags) {
+    Plan P;
+    GPT_TRY(check_common(cfg, weights, B, T, workspace, workspace_bytes, &P));
+    if (!idx || !logits) return GPT_ERR_NULL;
+    if (!aligned(logits, 16)) return GPT_ERR_BAD_ALIGN;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    Weights W;
+    fill_weights(W, cfg, weights);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    int32_t* status = status_word(ws);
+    const int C = cfg->n_embd, V = cfg->vocab_size, N = B * T;
+    float* x = reinterpret_cast<float*>(ws + P.x);
+    void* u = ws + P.u;
+
+    GPT_TRY(cuda_status(cudaMemsetAsync(status, 0, sizeof(int32_t), s)));
+    GPT_TRY(launch_embed(W.wte(), W.wpe(), idx, x, B, T, C, V, cfg->dtype, status, s));
+    for (int l = 0; l < cfg->n_layer; ++l) GPT_TRY(run_block(cfg, W, l, x, B, T, ws, P, s));
+    GPT_TRY(launch_layernorm(x, W.lnf_w(), W.lnf_b(), u, N, C, cfg->dtype, s));
+
+    if (targets) {
+        float* rl = row_loss ? row_loss : reinterpret_cast<float*>(ws + P.rowloss);
+        if (cfg->dtype == GPT_DTYPE_BF16) {
+            CeArgs ce{targets, reinterpret_cast<float2*>(ws + P.part), reinterpret_cast<float*>(ws + P.tlogit),
+                      P.n_part};
+            GPT_TRY(launch_gemm_bf16(static_cast<const bf16*>(u), C, static_cast<const bf16*>(W.wte()), C, nullptr,
+                                     logits, V, N, V, C, 3 /* EPI_CE */, cfg->gelu, &ce, status, s));
+            GPT_TRY(launch_ce_rows_from_parts(ce.part, P.n_part, ce.tlogit, targets, N, V, rl, status, s));
+        } else {
+            GPT_TRY(launch_linear_f32(static_cast<const float*>(u), C, static_cast<const float*>(W.wte()), nullptr,
+                                      static_cast<float*>(logits), V, N, V, C, GPT_EPI_STORE, cfg->gelu, s));
+            GPT_TRY(launch_ce_rows_from_logits(static_cast<const float*>(logits), targets, N, V, rl, status, s));
+        }
+        GPT_TRY(launch_loss_finalize(rl, targets, N, V, loss, loss_sum_count, s));
+    } else {
+        // Inference branch: only the last position's logits, [B, 1, V] (§3.2 ④).
+        const long long lda = static_cast<long long>(T) * C;
+        if (cfg->dtype == GPT_DTYPE_BF16) {
+            const bf16* ulast = static_cast<const bf16*>(u) + static_cast<long long>(T - 1) * C;
+            GPT_TRY(launch_gemm_bf16(ulast, lda, static_cast<const bf16*>(W.wte()), C, nullptr, logits, V, B, V, C,
+                                     GPT_EPI_STORE, cfg->gelu, nullptr, status, s));
+        } else {
+            const float* ulast = static_cast<const float*>(u) + static_cast<long long>(T - 1) * C;
+            GPT_TRY(launch_linear_f32(ulast, lda, static_cast<const float*>(W.wte()), nullptr,
+                                      static_cast<float*>(logits), V, B, V, C, GPT_EPI_STORE, cfg->gelu, s));
+        }
+    }
+    if (flags & GPT_FLAG_SYNC_CHECK) return sync_and_read_status(ws, s);
+    return GPT_OK;
+}
+
+GPT_API int gpt_block(const gpt_config_t* cfg, const void* weights, int layer, float* x, int B, int T,
+                      void* workspace, size_t workspace_bytes, void* stream, int flags) {
+    Plan P;
+    GPT_TRY(check_common(cfg, weights, B, T, workspace, workspace_bytes, &P));
+    if (!x) return GPT_ERR_NULL;
+    if (layer < 0 || layer >= cfg->n_layer) return GPT_ERR_BAD_SHAPE;
+    if (!aligned(x, 16)) return GPT_ERR_BAD_ALIGN;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    Weights W;
+    fill_weights(W, cfg, weights);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    GPT_TRY(cuda_status(cudaMemsetAsync(status_word(ws), 0, sizeof(int32_t), s)));
+    GPT_TRY(run_block(cfg, W, layer, x, B, T, ws, P, s));
+    if (flags & GPT_FLAG_SYNC_CHECK) return sync_and_read_status(ws, s);
+    return GPT_OK;
+}
+
+GPT_API int gpt_attention(const void* q, const void* k, const void* v, void* y, int B, int nh, int T, int hs,
+                          int dtype, int32_t* status, void* stream) {
+    if (!q || !k || !v || !y) return GPT_ERR_NULL;
+    if (B < 0 || nh < 0 || T < 0 || hs <= 0) return GPT_ERR_BAD_SHAPE;
+    if (dtype != GPT_DTYPE_BF16 && dtype != GPT_DTYPE_F32) return GPT_ERR_BAD_SHAPE;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(y, 16)) return GPT_ERR_BAD_ALIGN;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const long long sh = static_cast<long long>(T) * hs, sb = sh * nh;
+    if (dtype == GPT_DTYPE_BF16) {
+        if (hs != 64) return GPT_ERR_UNSUPPORTED;
+        AttnLayout L{static_cast<const bf16*>(q), static_cast<const bf16*>(k), static_cast<const bf16*>(v), sb, sh, hs,
+                     static_cast<bf16*>(y), sb, sh, hs};
+        return launch_attention_bf16(L, B, nh, T, status, s);
+    }
+    if (hs > 128) return GPT_ERR_UNSUPPORTED;
+    AttnLayoutF32 L{static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v), sb, sh, hs,
+                    static_cast<float*>(y), sb, sh, hs};
+    return launch_attention_f32(L, B, nh, T, hs, s);
+}
+
+GPT_API int gpt_embed(const void* wte, const void* wpe, const int64_t* idx, float* x, int B, int T, int C, int V,
+                      int dtype, int32_t* status, void* stream) {
+    if (!wte || !wpe || !idx || !x) return GPT_ERR_NULL;
+    if (B < 0 || T < 0 || C <= 0 || V <= 0 || (C % 4)) return GPT_ERR_BAD_SHAPE;
+    if (dtype != GPT_DTYPE_BF16 && dtype != GPT_DTYPE_F32) return GPT_ERR_BAD_SHAPE;
+    if (!aligned(wte, 16) || !aligned(wpe, 16) || !aligned(x, 16)) return GPT_ERR_BAD_ALIGN;
+    return launch_embed(wte, wpe, idx, x, B, T, C, V, dtype, status, static_cast<cudaStream_t>(stream));
+}
+
+GPT_API int gpt_layernorm(const float* x, const void* w, const void* b, void* out, int rows, int C, int dtype,
+                          void* stream) {
+    if (!x || !w || !out) return GPT_ERR_NULL;
+    if (rows < 0 || C <= 0 || (C % 4)) return GPT_ERR_BAD_SHAPE;
+    if (dtype != GPT_DTYPE_BF16 && dtype != GPT_DTYPE_F32) return GPT_ERR_BAD_SHAPE;
+    if (!aligned(x, 16) || !aligned(w, 16) || !aligned(out, 16) || (b && !aligned(b, 16))) return GPT_ERR_BAD_ALIGN;
+    return launch_layernorm(x, w, b, out, rows, C, dtype, static_cast<cudaStream_t>(stream));
+}
+
+GPT_API int gpt_linear(const void* x, const void* W, const void* b, void* out, int M, int N, int K, int dtype,
+                       int epilogue, int gelu, int32_t* status, void* stream) {
+    if (!x || !W || !out) return GPT_ERR_NULL;
+    if (M < 0 || N <= 0 || K <= 0) return GPT_ERR_BAD_SHAPE;
+    if (epilogue != GPT_EPI_STORE && epilogue != GPT_EPI_GELU && epilogue != GPT_EPI_RESID) return GPT_ERR_BAD_SHAPE;
+    if (gelu != GPT_GELU_ERF && gelu != GPT_GELU_TANH) return GPT_ERR_BAD_SHAPE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (dtype == GPT_DTYPE_BF16) {
+        if ((K % 8) || (N % 8)) return GPT_ERR_UNSUPPORTED;
+        if (!aligned(x, 16) || !aligned(W, 16) || !aligned(out, 16) || (b && !aligned(b, 16))) return GPT_ERR_BAD_ALIGN;
+        return launch_gemm_bf16(static_cast<const bf16*>(x), K, static_cast<const bf16*>(W), K,
+                                static_cast<const bf16*>(b), out, N, M, N, K, epilogue, gelu, nullptr, status, s);
+    }
+    if (dtype != GPT_DTYPE_F32) return GPT_ERR_BAD_SHAPE;
+    return launch_linear_f32(static_cast<const float*>(x), K, static_cast<const float*>(W),
+                             static_cast<const float*>(b), static_cast<float*>(out), N, M, N, K, epilogue, gelu, s);
+}
+
+GPT_API size_t gpt_lm_head_workspace_bytes(int rows, int V) {
+    if (rows < 1 || V < 1) return 0;
+    const size_t n = rows;
+    return 256 + a256(n * static_cast<size_t>(gemm_ce_parts(V)) * 8) + a256(n * 4) + a256(n * 4);
+}
+
+GPT_API int gpt_lm_head_loss(const void* u, const void* wte, const int64_t* targets, int rows, int C, int V,
+                             int dtype, void* logits, float* loss, float* row_loss, double* loss_sum_count,
+                             void* workspace, size_t workspace_bytes, void* stream, int flags) {
+    if (!u || !wte || !targets || !logits || !workspace) return GPT_ERR_NULL;
+    if (rows < 1 || C <= 0 || V <= 0) return GPT_ERR_BAD_SHAPE;
+    if (workspace_bytes < gpt_lm_head_workspace_bytes(rows, V)) return GPT_ERR_WS_TOO_SMALL;
+    if (!aligned(workspace, 256) || !aligned(u, 16) || !aligned(wte, 16) || !aligned(logits, 16))
+        return GPT_ERR_BAD_ALIGN;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    int32_t* status = status_word(ws);
+    const size_t n = rows;
+    const int n_part = gemm_ce_parts(V);
+    float2* part = reinterpret_cast<float2*>(ws + 256);
+    float* tlogit = reinterpret_cast<float*>(ws + 256 + a256(n * n_part * 8));
+    float* rl_ws = reinterpret_cast<float*>(ws + 256 + a256(n * n_part * 8) + a256(n * 4));
+    float* rl = row_loss ? row_loss : rl_ws;
+    GPT_TRY(cuda_status(cudaMemsetAsync(status, 0, sizeof(int32_t), s)));
+    if (dtype == GPT_DTYPE_BF16) {
+        if ((C % 8) || (V % 8)) return GPT_ERR_UNSUPPORTED;
+        CeArgs ce{targets, part, tlogit, n_part};
+        GPT_TRY(launch_gemm_bf16(static_cast<const bf16*>(u), C, static_cast<const bf16*>(wte), C, nullptr, logits, V,
+                                 rows, V, C, 3 /* EPI_CE */, GPT_GELU_ERF, &ce, status, s));
+        GPT_TRY(launch_ce_rows_from_parts(part, n_part, tlogit, targets, rows, V, rl, status, s));
+    } else if (dtype == GPT_DTYPE_F32) {
+        GPT_TRY(launch_linear_f32(static_cast<const float*>(u), C, static_cast<const float*>(wte), nullptr,
+                                  static_cast<float*>(logits), V, rows, V, C, GPT_EPI_STORE, GPT_GELU_ERF, s));
+        GPT_TRY(launch_ce_rows_from_logits(static_cast<const float*>(logits), targets, rows, V, rl, status, s));
+    } else {
+        return GPT_ERR_BAD_SHAPE;
+    }
+    GPT_TRY(launch_loss_finalize(rl, targets, rows, V, loss, loss_sum_count, s));
+    if (flags & GPT_FLAG_SYNC_CHECK) return sync_and_read_status(ws, s);
+    return GPT_OK;
+}

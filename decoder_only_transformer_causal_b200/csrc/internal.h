@@ -1,0 +1,74 @@
+// Host-side launchers shared by the C ABI (gpt_abi.cu) and the kernel files.  Every
+// launcher validates nothing beyond what its kernel needs; argument checking against the
+// public contract happens in gpt_abi.cu.  All return a GPT_* status.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/gpt.h"
+
+namespace gpt {
+
+typedef __nv_bfloat16 bf16;
+
+int num_sms();
+int cuda_status(cudaError_t e);
+
+// ---- TMA descriptors (cuTensorMapEncodeTiled through the runtime's driver entry point)
+int make_tmap_bf16_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
+                      uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer);
+int make_tmap_bf16_4d(CUtensorMap* m, const void* base, const uint64_t dims[4],
+                      const uint64_t strides_bytes[3], const uint32_t box[4]);
+
+// ---- row-wise kernels (rowwise.cu)
+int launch_embed(const void* wte, const void* wpe, const int64_t* idx, float* x, int B, int T,
+                 int C, int V, int dtype, int32_t* status, cudaStream_t s);
+int launch_layernorm(const float* x, const void* w, const void* b, void* out, int rows, int C,
+                     int dtype, cudaStream_t s);
+// bf16 path: combine the lm_head epilogue's partials into per-row losses.
+int launch_ce_rows_from_parts(const float2* part, int n_part, const float* tlogit,
+                              const int64_t* targets, int rows, int V, float* row_loss,
+                              int32_t* status, cudaStream_t s);
+// fp32 path: per-row losses straight from fp32 logits.
+int launch_ce_rows_from_logits(const float* logits, const int64_t* targets, int rows, int V,
+                               float* row_loss, int32_t* status, cudaStream_t s);
+// Fixed-order sum of the counted rows' losses -> loss, {sum, count}.
+int launch_loss_finalize(const float* row_loss, const int64_t* targets, int rows, int V,
+                         float* loss, double* sum_count, cudaStream_t s);
+
+// ---- tensor-core GEMM (gemm_tc.cu)
+struct CeArgs {
+    const int64_t* targets;
+    float2* part;
+    float* tlogit;
+    int n_part;
+};
+int gemm_ce_parts(int N);  // partial slots per row of the lm_head epilogue
+int launch_gemm_bf16(const bf16* A, long long lda, const bf16* W, long long ldw, const bf16* bias,
+                     void* out, long long ldo, int M, int N, int K, int epilogue, int gelu,
+                     const CeArgs* ce, int32_t* status, cudaStream_t s);
+
+// ---- tensor-core attention (attention_tc.cu); strides in elements
+struct AttnLayout {
+    const bf16 *q, *k, *v;
+    long long sb, sh, st;  // strides of q/k/v for batch, head, position (hs contiguous)
+    bf16* y;
+    long long y_sb, y_sh, y_st;
+};
+int launch_attention_bf16(const AttnLayout& L, int B, int nh, int T, int32_t* status, cudaStream_t s);
+
+// ---- fp32 SIMT path (simt_f32.cu)
+int launch_linear_f32(const float* A, long long lda, const float* W, const float* bias, float* out,
+                      long long ldo, int M, int N, int K, int epilogue, int gelu, cudaStream_t s);
+struct AttnLayoutF32 {
+    const float *q, *k, *v;
+    long long sb, sh, st;
+    float* y;
+    long long y_sb, y_sh, y_st;
+};
+int launch_attention_f32(const AttnLayoutF32& L, int B, int nh, int T, int hs, cudaStream_t s);
+
+}  // namespace gpt

@@ -1,0 +1,302 @@
+"""ctypes binding of libgptb200.so (include/gpt.h).
+
+Argument marshalling only: every function here checks Python-side types, turns tensors into
+raw device pointers and calls the C entry point of the same name.  PyTorch supplies device
+memory and streams; all arithmetic runs in the library's CUDA kernels.  There is no fallback:
+if the library cannot be loaded, importing this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "_lib", "libgptb200.so")
+
+GPT_OK = 0
+GPT_ERR_NULL = -1
+GPT_ERR_BAD_SHAPE = -2
+GPT_ERR_BAD_ALIGN = -3
+GPT_ERR_WS_TOO_SMALL = -4
+GPT_ERR_INDEX = -5
+GPT_ERR_TIMEOUT = -6
+GPT_ERR_UNSUPPORTED = -7
+GPT_ERR_CUDA = -8
+
+GPT_DTYPE_F32 = 0
+GPT_DTYPE_BF16 = 1
+GPT_GELU_ERF = 0
+GPT_GELU_TANH = 1
+GPT_FLAG_SYNC_CHECK = 1
+GPT_EPI_STORE, GPT_EPI_GELU, GPT_EPI_RESID = 0, 1, 2
+
+DTYPES = {"f32": GPT_DTYPE_F32, "bf16": GPT_DTYPE_BF16}
+TORCH_DTYPES = {GPT_DTYPE_F32: torch.float32, GPT_DTYPE_BF16: torch.bfloat16}
+GELUS = {"erf": GPT_GELU_ERF, "tanh": GPT_GELU_TANH}
+
+
+class GPTError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+class gpt_config_t(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in
+                ("n_layer", "n_head", "n_embd", "block_size", "vocab_size", "bias", "dtype", "gelu")]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m decoder_only_transformer_causal_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, Z, D = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_int
+    CFG = ctypes.POINTER(gpt_config_t)
+    sig = {
+        "gpt_status_string": (ctypes.c_char_p, [I]),
+        "gpt_abi_version": (I, []),
+        "gpt_validate_config": (I, [CFG]),
+        "gpt_weights_bytes": (Z, [CFG]),
+        "gpt_weights_count": (I, [CFG]),
+        "gpt_weights_layout": (I, [CFG, P, P, I]),
+        "gpt_workspace_bytes": (Z, [CFG, I, I]),
+        "gpt_check_status": (I, [P, P]),
+        "gpt_forward": (I, [CFG, P, P, P, I, I, P, P, P, P, P, Z, P, I]),
+        "gpt_block": (I, [CFG, P, I, P, I, I, P, Z, P, I]),
+        "gpt_attention": (I, [P, P, P, P, I, I, I, I, D, P, P]),
+        "gpt_embed": (I, [P, P, P, P, I, I, I, I, D, P, P]),
+        "gpt_layernorm": (I, [P, P, P, P, I, I, D, P]),
+        "gpt_linear": (I, [P, P, P, P, I, I, I, D, I, I, P, P]),
+        "gpt_lm_head_workspace_bytes": (Z, [I, I]),
+        "gpt_lm_head_loss": (I, [P, P, P, I, I, I, D, P, P, P, P, P, Z, P, I]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    return lib
+
+
+LIB = _load()
+
+EXPORTED = ("gpt_status_string", "gpt_abi_version", "gpt_validate_config", "gpt_weights_bytes",
+            "gpt_weights_count", "gpt_weights_layout", "gpt_workspace_bytes", "gpt_check_status",
+            "gpt_forward", "gpt_block", "gpt_attention", "gpt_embed", "gpt_layernorm", "gpt_linear",
+            "gpt_lm_head_workspace_bytes", "gpt_lm_head_loss")
+
+
+def status_string(status: int) -> str:
+    return LIB.gpt_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != GPT_OK:
+        raise GPTError(status, where)
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, torch.Tensor):
+        if t.numel() and not t.is_contiguous():
+            raise ValueError("tensors passed to the library must be contiguous")
+        return t.data_ptr() or None
+    return int(t)
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        if torch.cuda.is_available():
+            return torch.cuda.current_stream().cuda_stream or None
+        return None
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream or None
+    return int(stream) or None
+
+
+@dataclass(frozen=True)
+class GPTConfig:
+    """GPTConfig of the pages ("nanoGPT 全局流程图", §2.1) plus storage dtype and GELU form."""
+    n_layer: int = 12
+    n_head: int = 12
+    n_embd: int = 768
+    block_size: int = 1024
+    vocab_size: int = 50304
+    bias: bool = True
+    dtype: str = "bf16"
+    gelu: str = "erf"
+
+    def c(self) -> gpt_config_t:
+        return gpt_config_t(self.n_layer, self.n_head, self.n_embd, self.block_size,
+                            self.vocab_size, int(bool(self.bias)), DTYPES[self.dtype],
+                            GELUS[self.gelu])
+
+    @property
+    def torch_dtype(self):
+        return TORCH_DTYPES[DTYPES[self.dtype]]
+
+    @classmethod
+    def from_dict(cls, d: dict) -> "GPTConfig":
+        keys = cls.__dataclass_fields__
+        return cls(**{k: v for k, v in d.items() if k in keys})
+
+
+def packed_names(n_layer: int) -> list[str]:
+    """Tensor names in the packed order documented in gpt.h."""
+    names = ["wte", "wpe"]
+    for l in range(n_layer):
+        p = f"h.{l}."
+        names += [p + s for s in ("ln_1.weight", "ln_1.bias", "attn.c_attn.weight", "attn.c_attn.bias",
+                                  "attn.c_proj.weight", "attn.c_proj.bias", "ln_2.weight", "ln_2.bias",
+                                  "mlp.c_fc.weight", "mlp.c_fc.bias", "mlp.c_proj.weight",
+                                  "mlp.c_proj.bias")]
+    return names + ["ln_f.weight", "ln_f.bias"]
+
+
+def validate_config(cfg: GPTConfig) -> int:
+    return LIB.gpt_validate_config(ctypes.byref(cfg.c()))
+
+
+def weights_layout(cfg: GPTConfig) -> tuple[list[tuple[str, int, int]], int]:
+    """[(name, byte offset, numel)] in packed order, and the buffer size in bytes."""
+    c = cfg.c()
+    n = LIB.gpt_weights_count(ctypes.byref(c))
+    _check(n if n < 0 else GPT_OK, "gpt_weights_count")
+    offs = (ctypes.c_size_t * n)()
+    nums = (ctypes.c_size_t * n)()
+    got = LIB.gpt_weights_layout(ctypes.byref(c), offs, nums, n)
+    _check(got if got < 0 else GPT_OK, "gpt_weights_layout")
+    total = LIB.gpt_weights_bytes(ctypes.byref(c))
+    return [(nm, offs[i], nums[i]) for i, nm in enumerate(packed_names(cfg.n_layer))], total
+
+
+def pack_weights(cfg: GPTConfig, tensors: dict, device="cuda") -> torch.Tensor:
+    """Copies named parameter tensors into one packed device buffer (bias slots stay zero
+    when absent or when cfg.bias is False)."""
+    entries, total = weights_layout(cfg)
+    buf = torch.zeros(total, dtype=torch.uint8, device=device)
+    dt = cfg.torch_dtype
+    for name, off, numel in entries:
+        t = tensors.get(name)
+        if t is None:
+            if name.endswith(".bias"):
+                continue
+            raise KeyError(name)
+        if t.numel() != numel:
+            raise ValueError(f"{name}: {t.numel()} elements, layout expects {numel}")
+        esz = torch.finfo(dt).bits // 8
+        buf[off:off + numel * esz].view(dt).copy_(t.reshape(-1).to(dt))
+    return buf
+
+
+def workspace_bytes(cfg: GPTConfig, B: int, T: int) -> int:
+    return LIB.gpt_workspace_bytes(ctypes.byref(cfg.c()), B, T)
+
+
+def alloc_workspace(nbytes: int, device="cuda") -> torch.Tensor:
+    return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+
+
+def check_status(workspace: torch.Tensor, stream=None) -> int:
+    return LIB.gpt_check_status(_ptr(workspace), _stream(stream))
+
+
+def forward(cfg: GPTConfig, weights: torch.Tensor, idx: torch.Tensor, targets: torch.Tensor | None,
+            workspace: torch.Tensor, logits: torch.Tensor | None = None, loss: torch.Tensor | None = None,
+            row_loss: torch.Tensor | None = None, loss_sum_count: torch.Tensor | None = None,
+            stream=None, sync_check: bool = False):
+    """gpt_forward.  Returns (logits, loss) device tensors (loss None without targets)."""
+    B, T = idx.shape
+    dt = cfg.torch_dtype
+    if logits is None:
+        shape = (B, T, cfg.vocab_size) if targets is not None else (B, 1, cfg.vocab_size)
+        logits = torch.empty(shape, dtype=dt, device=idx.device)
+    if targets is not None and loss is None:
+        loss = torch.empty((), dtype=torch.float32, device=idx.device)
+    rc = LIB.gpt_forward(ctypes.byref(cfg.c()), _ptr(weights), _ptr(idx), _ptr(targets), B, T,
+                         _ptr(logits), _ptr(loss) if targets is not None else None, _ptr(row_loss),
+                         _ptr(loss_sum_count), _ptr(workspace), workspace.numel(), _stream(stream),
+                         GPT_FLAG_SYNC_CHECK if sync_check else 0)
+    _check(rc, "gpt_forward")
+    return logits, (loss if targets is not None else None)
+
+
+def block(cfg: GPTConfig, weights: torch.Tensor, layer: int, x: torch.Tensor, workspace: torch.Tensor,
+          stream=None, sync_check: bool = False) -> torch.Tensor:
+    B, T, _ = x.shape
+    rc = LIB.gpt_block(ctypes.byref(cfg.c()), _ptr(weights), layer, _ptr(x), B, T, _ptr(workspace),
+                       workspace.numel(), _stream(stream), GPT_FLAG_SYNC_CHECK if sync_check else 0)
+    _check(rc, "gpt_block")
+    return x
+
+
+def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, y: torch.Tensor | None = None,
+              status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    B, nh, T, hs = q.shape
+    dtype = {torch.bfloat16: GPT_DTYPE_BF16, torch.float32: GPT_DTYPE_F32}[q.dtype]
+    if y is None:
+        y = torch.empty_like(q)
+    rc = LIB.gpt_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(y), B, nh, T, hs, dtype, _ptr(status),
+                           _stream(stream))
+    _check(rc, "gpt_attention")
+    return y
+
+
+def embed(wte, wpe, idx, x=None, status=None, stream=None):
+    B, T = idx.shape
+    V, C = wte.shape
+    dtype = {torch.bfloat16: GPT_DTYPE_BF16, torch.float32: GPT_DTYPE_F32}[wte.dtype]
+    if x is None:
+        x = torch.empty((B, T, C), dtype=torch.float32, device=idx.device)
+    _check(LIB.gpt_embed(_ptr(wte), _ptr(wpe), _ptr(idx), _ptr(x), B, T, C, V, dtype, _ptr(status),
+                         _stream(stream)), "gpt_embed")
+    return x
+
+
+def layernorm(x, w, b=None, out=None, stream=None):
+    C = x.shape[-1]
+    rows = x.numel() // C
+    dtype = {torch.bfloat16: GPT_DTYPE_BF16, torch.float32: GPT_DTYPE_F32}[w.dtype]
+    if out is None:
+        out = torch.empty(x.shape, dtype=w.dtype, device=x.device)
+    _check(LIB.gpt_layernorm(_ptr(x), _ptr(w), _ptr(b), _ptr(out), rows, C, dtype, _stream(stream)),
+           "gpt_layernorm")
+    return out
+
+
+def linear(x, W, b=None, out=None, epilogue=GPT_EPI_STORE, gelu=GPT_GELU_ERF, status=None, stream=None):
+    M, K = x.shape
+    N = W.shape[0]
+    dtype = {torch.bfloat16: GPT_DTYPE_BF16, torch.float32: GPT_DTYPE_F32}[x.dtype]
+    if out is None:
+        odt = torch.float32 if epilogue == GPT_EPI_RESID else x.dtype
+        out = torch.zeros((M, N), dtype=odt, device=x.device)
+    _check(LIB.gpt_linear(_ptr(x), _ptr(W), _ptr(b), _ptr(out), M, N, K, dtype, epilogue, gelu,
+                          _ptr(status), _stream(stream)), "gpt_linear")
+    return out
+
+
+def lm_head_workspace_bytes(rows: int, V: int) -> int:
+    return LIB.gpt_lm_head_workspace_bytes(rows, V)
+
+
+def lm_head_loss(u, wte, targets, workspace=None, logits=None, loss=None, row_loss=None,
+                 loss_sum_count=None, stream=None, sync_check=False):
+    rows, C = u.shape
+    V = wte.shape[0]
+    dtype = {torch.bfloat16: GPT_DTYPE_BF16, torch.float32: GPT_DTYPE_F32}[u.dtype]
+    if workspace is None:
+        workspace = alloc_workspace(lm_head_workspace_bytes(rows, V), u.device)
+    if logits is None:
+        logits = torch.empty((rows, V), dtype=u.dtype, device=u.device)
+    if loss is None:
+        loss = torch.empty((), dtype=torch.float32, device=u.device)
+    _check(LIB.gpt_lm_head_loss(_ptr(u), _ptr(wte), _ptr(targets), rows, C, V, dtype, _ptr(logits),
+                                _ptr(loss), _ptr(row_loss), _ptr(loss_sum_count), _ptr(workspace),
+                                workspace.numel(), _stream(stream),
+                                GPT_FLAG_SYNC_CHECK if sync_check else 0), "gpt_lm_head_loss")
+    return logits, loss

@@ -1,0 +1,202 @@
+/*
+ * gpt.h - C ABI of the B200 (sm_100a) GPT-2 / nanoGPT causal decoder forward pass.
+ *
+ * What the library computes is the forward pass the nanoGPT pages describe:
+ *   - "nanoGPT 全局流程图" (devpress.csdn.net), §3.2 前向传播: tok_emb + pos_emb, the Blocks,
+ *     ln_f, then logits = lm_head(x) and F.cross_entropy(..., ignore_index=-1) when targets
+ *     are given, or lm_head(x[:, [-1], :]) and no loss when they are not;
+ *   - same page §2.5: the pre-LN Block x = x + attn(ln_1(x)); x = x + mlp(ln_2(x)),
+ *     CausalSelfAttention (c_attn C->3C, heads, softmax(mask(q k^T / sqrt(hs))) v, c_proj),
+ *     MLP (c_fc C->4C, GELU, c_proj 4C->C), LayerNorm with eps 1e-5;
+ *   - same page §2.3: the head is tied to the token embedding (one [V, C] table);
+ *   - "nanoGPT 核心代码速查表" (pgsm.cn), 七、关键函数签名: forward(idx, targets=None) ->
+ *     (logits, loss).
+ *
+ * Conventions that hold for every entry point:
+ *   - Every pointer is a DEVICE pointer unless stated otherwise.  The caller owns and
+ *     allocates every buffer; no entry point allocates or frees device memory.
+ *   - Tensors are dense and row-major; shapes are given outermost first.
+ *   - Work is enqueued on `stream` (a cudaStream_t passed as void*, NULL = legacy default
+ *     stream) and runs asynchronously, except where GPT_FLAG_SYNC_CHECK asks for a
+ *     synchronising error check.
+ *   - Every entry point returns an int status: GPT_OK (0) or a negative GPT_ERR_* code.
+ *     Argument errors are detected on the host before anything is enqueued.  Device-side
+ *     conditions (an out-of-range token id or target, a pipeline wait that exceeded its
+ *     time limit) are recorded in a device status word and reported by gpt_check_status()
+ *     or by a call made with GPT_FLAG_SYNC_CHECK.  No kernel traps or asserts.
+ *   - Results are deterministic: every reduction runs in a fixed order.
+ *   - Storage precision: GPT_DTYPE_BF16 stores weights, activations between kernels and
+ *     logits in bf16, accumulates in fp32 and keeps the residual stream, LayerNorm
+ *     statistics, softmax and cross-entropy in fp32.  GPT_DTYPE_F32 is fp32 throughout.
+ */
+#ifndef GPT_B200_H
+#define GPT_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define GPT_ABI_VERSION 1
+
+/* ---- status codes ------------------------------------------------------------------ */
+#define GPT_OK                 0
+#define GPT_ERR_NULL          -1  /* a required pointer is NULL */
+#define GPT_ERR_BAD_SHAPE     -2  /* inconsistent sizes: T > block_size, C % n_head != 0, ... */
+#define GPT_ERR_BAD_ALIGN     -3  /* a pointer is not 16-byte aligned */
+#define GPT_ERR_WS_TOO_SMALL  -4  /* workspace_bytes < gpt_workspace_bytes(...) */
+#define GPT_ERR_INDEX         -5  /* device: a token id outside [0, V) or a target outside [0, V) and != -1 */
+#define GPT_ERR_TIMEOUT       -6  /* device: a pipeline wait exceeded its time limit; results invalid */
+#define GPT_ERR_UNSUPPORTED   -7  /* valid request this build does not implement (e.g. bf16 with hs != 64) */
+#define GPT_ERR_CUDA          -8  /* a CUDA runtime call failed (launch error, no device, ...) */
+
+/* ---- configuration ------------------------------------------------------------------ */
+#define GPT_DTYPE_F32   0
+#define GPT_DTYPE_BF16  1
+
+#define GPT_GELU_ERF    0   /* x * Phi(x), nn.GELU()'s default ("nanoGPT架构逐步详解", 4. MLP) */
+#define GPT_GELU_TANH   1   /* 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))) */
+
+#define GPT_FLAG_SYNC_CHECK 1  /* synchronise `stream` at the end and return the device status */
+
+/* GPTConfig ("nanoGPT 全局流程图", §2.1 模型配置).  Dropout is not a field: it is 0.0 there
+ * and the identity in a forward pass. */
+typedef struct gpt_config {
+    int32_t n_layer;
+    int32_t n_head;
+    int32_t n_embd;       /* C; head size hs = C / n_head */
+    int32_t block_size;   /* rows of wpe; T must not exceed it */
+    int32_t vocab_size;   /* V; rows of the tied wte / lm_head table */
+    int32_t bias;         /* 1: Linear and LayerNorm layers carry biases; 0: none are read */
+    int32_t dtype;        /* GPT_DTYPE_F32 or GPT_DTYPE_BF16 */
+    int32_t gelu;         /* GPT_GELU_ERF or GPT_GELU_TANH */
+} gpt_config_t;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* gpt_status_string(int status);
+
+/* GPT_ABI_VERSION of the loaded library. */
+int gpt_abi_version(void);
+
+/* Checks a configuration: positive sizes, C % n_head == 0, dtype and gelu in range,
+ * and, for GPT_DTYPE_BF16, hs == 64 and C % 8 == 0 (the tensor-core kernels' layout).
+ * Returns GPT_OK, GPT_ERR_NULL, GPT_ERR_BAD_SHAPE or GPT_ERR_UNSUPPORTED. */
+int gpt_validate_config(const gpt_config_t* cfg);
+
+/* ---- packed weights ------------------------------------------------------------------
+ * All parameters live in ONE device buffer of gpt_weights_bytes(cfg) bytes, each tensor at
+ * a 256-byte aligned offset, stored in the config's dtype, in this order (the nanoGPT
+ * module tree of "nanoGPT 全局流程图" §2.2 and §2.5):
+ *   0 wte [V, C]            (also the lm_head weight: tied, §2.3)
+ *   1 wpe [block_size, C]
+ *   then for each layer l:  ln_1.weight [C], ln_1.bias [C],
+ *                           attn.c_attn.weight [3C, C], attn.c_attn.bias [3C],
+ *                           attn.c_proj.weight [C, C],  attn.c_proj.bias [C],
+ *                           ln_2.weight [C], ln_2.bias [C],
+ *                           mlp.c_fc.weight [4C, C],    mlp.c_fc.bias [4C],
+ *                           mlp.c_proj.weight [C, 4C],  mlp.c_proj.bias [C]
+ *   then ln_f.weight [C], ln_f.bias [C].
+ * Linear weights are [out, in] (nn.Linear).  Bias slots exist even when cfg->bias == 0;
+ * they are then never read. */
+size_t gpt_weights_bytes(const gpt_config_t* cfg);   /* 0 on an invalid config */
+int    gpt_weights_count(const gpt_config_t* cfg);   /* 2 + 12 * n_layer + 2, or < 0 */
+/* Fills offsets[i] (bytes) and numels[i] (elements) for i < min(n, count).  Either array
+ * may be NULL.  Returns the tensor count or a negative status. */
+int    gpt_weights_layout(const gpt_config_t* cfg, size_t* offsets, size_t* numels, int n);
+
+/* ---- workspace ----------------------------------------------------------------------
+ * Bytes of device scratch gpt_forward / gpt_block need for a [B, T] batch (activations,
+ * cross-entropy partials and the device status word).  0 on invalid arguments.  The
+ * workspace must be 256-byte aligned; its contents need no initialisation and are
+ * overwritten by each call, so calls that share a workspace must be serialised on one
+ * stream. */
+size_t gpt_workspace_bytes(const gpt_config_t* cfg, int B, int T);
+
+/* Synchronises `stream`, reads and clears the device status word in `workspace`, and
+ * returns it (GPT_OK, GPT_ERR_INDEX or GPT_ERR_TIMEOUT), or GPT_ERR_CUDA. */
+int gpt_check_status(void* workspace, void* stream);
+
+/* ---- the forward pass ---------------------------------------------------------------
+ * GPT.forward(idx, targets) ("nanoGPT 全局流程图", §3.2; "nanoGPT 代码解析", forward).
+ *   weights  packed buffer described above.
+ *   idx      int64 [B, T], token ids in [0, V).
+ *   targets  int64 [B, T] in [0, V) or -1 (ignored), or NULL.
+ *   logits   with targets: [B, T, V]; without: [B, 1, V], the last position only.
+ *            bf16 for GPT_DTYPE_BF16, fp32 for GPT_DTYPE_F32.  Must be 16-byte aligned.
+ *   loss     fp32 scalar: mean of logsumexp(z) - z[target] over rows whose target != -1;
+ *            NaN when every target is -1.  May be NULL.  Untouched when targets == NULL.
+ *   row_loss fp32 [B, T]: per-position loss, 0 at ignored positions.  May be NULL.
+ *   loss_sum_count  fp64 [2]: {sum of counted row losses, number of counted rows}, the
+ *            terms a batch-sharded caller adds across devices.  May be NULL.
+ *   Requires 1 <= T <= block_size and B >= 1.  With bf16, the cross-entropy is taken from
+ *   the fp32 accumulators, before the logits are rounded for storage.
+ * The device status word in `workspace` is cleared at the start of every gpt_forward and
+ * gpt_block call.
+ * Returns GPT_OK once enqueued (or, with GPT_FLAG_SYNC_CHECK, once finished and checked). */
+int gpt_forward(const gpt_config_t* cfg, const void* weights,
+                const int64_t* idx, const int64_t* targets, int B, int T,
+                void* logits, float* loss, float* row_loss, double* loss_sum_count,
+                void* workspace, size_t workspace_bytes, void* stream, int flags);
+
+/* One pre-LN Block in place ("nanoGPT 全局流程图", §2.5 Block.forward):
+ *   x = x + attn(ln_1(x)); x = x + mlp(ln_2(x))  for layer `layer` of `weights`.
+ *   x  fp32 [B, T, C] (the residual stream is fp32 for both dtypes), updated in place.
+ *   workspace as for gpt_forward (gpt_workspace_bytes(cfg, B, T) bytes). */
+int gpt_block(const gpt_config_t* cfg, const void* weights, int layer, float* x, int B, int T,
+              void* workspace, size_t workspace_bytes, void* stream, int flags);
+
+/* Causal self-attention of one batch of heads ("nanoGPT 全局流程图", §2.5 (B) 步骤3-6;
+ * "nanoGPT架构逐步详解", 3. 因果自注意力):
+ *   y[b, h, i] = sum_{j <= i} softmax_j(q[b,h,i] . k[b,h,j] / sqrt(hs)) v[b,h,j]
+ *   q, k, v, y  [B, nh, T, hs], 16-byte aligned, dtype GPT_DTYPE_BF16 (hs must be 64) or
+ *               GPT_DTYPE_F32 (1 <= hs <= 128).
+ *   status      optional device int32 (NULL allowed); a pipeline time-out writes
+ *               GPT_ERR_TIMEOUT there.  It is never cleared by the library. */
+int gpt_attention(const void* q, const void* k, const void* v, void* y,
+                  int B, int nh, int T, int hs, int dtype, int32_t* status, void* stream);
+
+/* ---- single kernels of the forward pass (same kernels gpt_forward launches) ----------- */
+
+/* x[b, t, :] = wte[idx[b, t], :] + wpe[t, :]  ("nanoGPT 全局流程图", §3.2 ①).
+ *   wte [V, C], wpe [>= T, C] in `dtype`; x fp32 [B, T, C].  An id outside [0, V) reads
+ *   row 0 instead and writes GPT_ERR_INDEX to *status (optional device int32). */
+int gpt_embed(const void* wte, const void* wpe, const int64_t* idx, float* x,
+              int B, int T, int C, int V, int dtype, int32_t* status, void* stream);
+
+/* out = (x - mean) / sqrt(var + 1e-5) * w + b per row, var the population variance
+ * ("nanoGPT 全局流程图", §2.5 (A)).  x fp32 [rows, C]; w, b [C] in `dtype` (b may be NULL);
+ * out [rows, C] in `dtype`.  C <= 2048 and C % 4 == 0. */
+int gpt_layernorm(const float* x, const void* w, const void* b, void* out,
+                  int rows, int C, int dtype, void* stream);
+
+#define GPT_EPI_STORE   0  /* out = x W^T + b                       (out in dtype)      */
+#define GPT_EPI_GELU    1  /* out = gelu(x W^T + b)                 (out in dtype)      */
+#define GPT_EPI_RESID   2  /* out += x W^T + b, out fp32            (residual stream)   */
+
+/* nn.Linear with a fused epilogue: x [M, K], W [N, K] (nn.Linear layout), b [N] or NULL,
+ * all in `dtype`; out [M, N] as the epilogue says.  gelu = GPT_GELU_*.  With bf16,
+ * K % 8 == 0 and N % 8 == 0.  status: optional device int32 that receives GPT_ERR_TIMEOUT
+ * if a pipeline wait of the tensor-core kernel expires (never cleared by the library). */
+int gpt_linear(const void* x, const void* W, const void* b, void* out, int M, int N, int K,
+               int dtype, int epilogue, int gelu, int32_t* status, void* stream);
+
+/* Tied head with fused cross-entropy ("nanoGPT 全局流程图", §3.2 ④ and §3.3):
+ *   logits = u wte^T ([rows, V] in `dtype`), then per row logsumexp - logit[target] over all
+ *   V columns, averaged over rows whose target != -1 (fixed-order reduction).
+ *   u [rows, C] in `dtype` (the ln_f output), wte [V, C], targets int64 [rows].
+ *   loss / row_loss / loss_sum_count as in gpt_forward (each may be NULL).
+ *   workspace: gpt_lm_head_workspace_bytes(rows, V) bytes, 256-byte aligned; its status word
+ *   is read by gpt_check_status(). */
+size_t gpt_lm_head_workspace_bytes(int rows, int V);
+int gpt_lm_head_loss(const void* u, const void* wte, const int64_t* targets, int rows, int C,
+                     int V, int dtype, void* logits, float* loss, float* row_loss,
+                     double* loss_sum_count, void* workspace, size_t workspace_bytes,
+                     void* stream, int flags);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GPT_B200_H */

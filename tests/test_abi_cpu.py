@@ -1,0 +1,127 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports every function
+include/gpt.h declares, and rejects bad arguments on the host before anything is enqueued."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle
+import seeded
+from decoder_only_transformer_causal_b200 import native
+from decoder_only_transformer_causal_b200.native import GPTConfig
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "gpt.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(gpt_\w+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared_functions()
+    assert len(names) >= 16
+    lib = ctypes.CDLL(native.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(native.EXPORTED)
+
+
+def test_abi_version_and_status_strings():
+    assert native.LIB.gpt_abi_version() == 1
+    for code in range(-8, 1):
+        s = native.status_string(code)
+        assert s and s != "unknown status"
+    assert native.status_string(-99) == "unknown status"
+
+
+def _cfg(name, **kw):
+    return GPTConfig.from_dict(dict(seeded.WORKLOADS[name].model_dict(), **kw))
+
+
+@pytest.mark.parametrize("name", sorted(seeded.WORKLOADS))
+def test_presets_validate(name):
+    assert native.validate_config(_cfg(name)) == native.GPT_OK
+
+
+def test_validate_rejects():
+    assert native.validate_config(_cfg("gpt2", n_head=7)) == native.GPT_ERR_BAD_SHAPE      # C % nh
+    assert native.validate_config(_cfg("gpt2", n_head=24)) == native.GPT_ERR_UNSUPPORTED   # bf16 hs 32
+    assert native.validate_config(_cfg("tiny", n_head=8)) == native.GPT_OK                 # fp32 hs 16
+    assert native.validate_config(_cfg("gpt2", n_layer=-1)) == native.GPT_ERR_BAD_SHAPE
+    bad = native.gpt_config_t(1, 1, 64, 8, 10, 1, 5, 0)
+    assert native.LIB.gpt_validate_config(ctypes.byref(bad)) == native.GPT_ERR_BAD_SHAPE
+    assert native.LIB.gpt_validate_config(None) == native.GPT_ERR_NULL
+
+
+@pytest.mark.parametrize("name", sorted(seeded.WORKLOADS))
+def test_weights_layout_counts(name):
+    cfg = _cfg(name)
+    entries, total = native.weights_layout(cfg)
+    # every parameter exactly once (tied head): the element count is get_num_params
+    assert sum(n for _, _, n in entries) == oracle.num_params(seeded.WORKLOADS[name].model_dict(), False)
+    offs = [o for _, o, _ in entries]
+    assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
+    esz = 2 if cfg.dtype == "bf16" else 4
+    last_name, last_off, last_n = entries[-1]
+    assert total >= last_off + last_n * esz
+    shapes = seeded.weight_shapes(seeded.WORKLOADS[name].model_dict())
+    for nm, _, n in entries:
+        numel = 1
+        for d in shapes[nm]:
+            numel *= d
+        assert numel == n, nm
+
+
+def test_workspace_bytes():
+    cfg = _cfg("gpt2")
+    ws = native.workspace_bytes(cfg, 12, 1024)
+    N, C = 12 * 1024, 768
+    # x fp32 + ln out + qkv + y + h (bf16) at least
+    assert ws >= N * C * 4 + N * C * 2 * (1 + 3 + 1 + 4)
+    assert native.workspace_bytes(cfg, 12, 1025) == 0       # T > block_size
+    assert native.workspace_bytes(cfg, 0, 16) == 0
+    assert native.lm_head_workspace_bytes(12288, 50304) > 12288 * 4
+
+
+FAKE = 1 << 20  # an aligned non-null address; the calls below must fail before using it
+
+
+def _fwd(cfg, B, T, weights=FAKE, ws=FAKE, ws_bytes=1 << 40, logits=FAKE, idx=FAKE):
+    return native.LIB.gpt_forward(ctypes.byref(cfg.c()), weights, idx, None, B, T, logits, None, None,
+                                  None, ws, ws_bytes, None, 0)
+
+
+def test_forward_host_validation():
+    cfg = _cfg("gpt2")
+    assert _fwd(cfg, 2, 1025) == native.GPT_ERR_BAD_SHAPE        # T > block_size
+    assert _fwd(cfg, 0, 16) == native.GPT_ERR_BAD_SHAPE
+    assert _fwd(cfg, 2, 16, weights=None) == native.GPT_ERR_NULL
+    assert _fwd(cfg, 2, 16, idx=None) == native.GPT_ERR_NULL
+    assert _fwd(cfg, 2, 16, weights=FAKE + 8) == native.GPT_ERR_BAD_ALIGN
+    assert _fwd(cfg, 2, 16, ws_bytes=1024) == native.GPT_ERR_WS_TOO_SMALL
+    assert _fwd(_cfg("gpt2", n_head=24), 2, 16) == native.GPT_ERR_UNSUPPORTED
+    rc = native.LIB.gpt_block(ctypes.byref(cfg.c()), FAKE, 12, FAKE, 1, 8, FAKE, 1 << 40, None, 0)
+    assert rc == native.GPT_ERR_BAD_SHAPE                          # layer out of range
+
+
+def test_kernel_entry_validation():
+    L = native.LIB
+    assert L.gpt_attention(FAKE, FAKE, FAKE, FAKE, 1, 1, 8, 32, native.GPT_DTYPE_BF16, None, None) \
+        == native.GPT_ERR_UNSUPPORTED                              # bf16 needs hs 64
+    assert L.gpt_attention(FAKE, FAKE, FAKE, FAKE + 4, 1, 1, 8, 64, native.GPT_DTYPE_BF16, None, None) \
+        == native.GPT_ERR_BAD_ALIGN
+    assert L.gpt_attention(None, FAKE, FAKE, FAKE, 1, 1, 8, 64, native.GPT_DTYPE_BF16, None, None) \
+        == native.GPT_ERR_NULL
+    assert L.gpt_linear(FAKE, FAKE, None, FAKE, 8, 12, 64, native.GPT_DTYPE_BF16, 0, 0, None, None) \
+        == native.GPT_ERR_UNSUPPORTED                              # N % 8
+    assert L.gpt_linear(FAKE, FAKE, None, FAKE, 8, 16, 64, native.GPT_DTYPE_BF16, 9, 0, None, None) \
+        == native.GPT_ERR_BAD_SHAPE
+    assert L.gpt_layernorm(FAKE, FAKE, None, FAKE, 4, 6, native.GPT_DTYPE_F32, None) == native.GPT_ERR_BAD_SHAPE
+    assert L.gpt_embed(FAKE, FAKE, FAKE, FAKE, 1, 1, 6, 10, native.GPT_DTYPE_F32, None, None) \
+        == native.GPT_ERR_BAD_SHAPE
+    assert L.gpt_lm_head_loss(FAKE, FAKE, FAKE, 4, 64, 128, native.GPT_DTYPE_BF16, FAKE, None, None, None,
+                              FAKE, 16, None, 0) == native.GPT_ERR_WS_TOO_SMALL
+    assert L.gpt_check_status(None, None) == native.GPT_ERR_NULL

@@ -1,0 +1,149 @@
+"""The whole forward pass (gpt_forward) and single Blocks (gpt_block) through the C ABI
+against the fp64 oracle, from the tiny fp32 model to GPT-2 XL at full size.
+
+Full-size bf16 workloads run on the GPU exactly as the benchmark launches them; the oracle
+then recomputes sampled sequences (sequences are independent) and, for the two largest
+models, a prefix of one sequence (logits at position t depend only on positions <= t)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import seeded
+from gpu_helpers import BF16_ATOL, F32_ATOL, LOSS_RTOL, f64, max_abs, model_inputs, needs_gpu
+
+pytestmark = [pytest.mark.gpu, needs_gpu]
+
+
+def gpu_model(cfg, W, gelu="erf"):
+    from decoder_only_transformer_causal_b200 import GPT, GPTConfig
+    return GPT(GPTConfig.from_dict(dict(cfg, gelu=gelu)), W)
+
+
+# ------------------------------------------------------------------ tiny fp32 model
+@pytest.mark.parametrize("stress,gelu,ign", [(False, "erf", 0.0), (True, "erf", 0.15), (True, "tanh", 0.0)])
+def test_tiny_fp32_forward(stress, gelu, ign):
+    cfg, W, W64, idx, tgt = model_inputs("tiny", stress=stress, ignore_frac=ign)
+    m = gpu_model(cfg, W, gelu)
+    row = torch.empty(idx.shape, device="cuda")
+    logits, loss = m(idx.cuda(), tgt.cuda(), row_loss=row, sync_check=True)
+    ref = oracle.forward(W64, cfg, idx.numpy(), tgt.numpy(), gelu_mode=gelu)
+    assert max_abs(f64(logits), ref["logits"]) <= F32_ATOL
+    assert abs(float(loss) - ref["loss"]) <= LOSS_RTOL * abs(ref["loss"])
+    assert max_abs(f64(row), ref["row_loss"]) <= 1e-4
+    last, none = m(idx.cuda(), None, sync_check=True)
+    assert none is None and last.shape == (idx.shape[0], 1, cfg["vocab_size"])
+    assert max_abs(f64(last)[:, 0], ref["logits"][:, -1]) <= F32_ATOL
+
+
+def test_tiny_fp32_short_sequences():
+    cfg, W, W64, idx, tgt = model_inputs("tiny", stress=True, B=3, T=17)
+    m = gpu_model(cfg, W)
+    logits, loss = m(idx.cuda(), tgt.cuda(), sync_check=True)
+    ref = oracle.forward(W64, cfg, idx.numpy(), tgt.numpy())
+    assert max_abs(f64(logits), ref["logits"]) <= F32_ATOL
+
+
+# ------------------------------------------------------------------ one Block
+@pytest.mark.parametrize("name,B,T", [("gpt2", 2, 300), ("gpt2-xl", 1, 200), ("tiny", 4, 64)])
+def test_block(name, B, T):
+    cfg, W, W64, _, _ = model_inputs(name, stress=True, n_layer=2)
+    m = gpu_model(cfg, W)
+    x = seeded.make_residual(B, T, cfg["n_embd"])
+    xg = x.clone().cuda()
+    m.block(1, xg, sync_check=True)
+    ref = oracle.block(f64(x), W64, 1, cfg["n_head"])
+    tol = F32_ATOL if cfg["dtype"] == "f32" else BF16_ATOL
+    err = max_abs(f64(xg), ref)
+    assert err <= tol, err
+
+
+# ------------------------------------------------------------------ bf16 models, reduced depth
+@pytest.mark.parametrize("stress", [False, True])
+def test_gpt2_width_two_layers(stress):
+    cfg, W, W64, idx, tgt = model_inputs("gpt2", stress=stress, n_layer=2, B=2, T=333, ignore_frac=0.1)
+    m = gpu_model(cfg, W)
+    row = torch.empty(idx.shape, device="cuda")
+    logits, loss = m(idx.cuda(), tgt.cuda(), row_loss=row, sync_check=True)
+    ref = oracle.forward(W64, cfg, idx.numpy(), tgt.numpy())
+    assert max_abs(f64(logits), ref["logits"]) <= BF16_ATOL
+    assert abs(float(loss) - ref["loss"]) <= LOSS_RTOL * abs(ref["loss"])
+    assert max_abs(f64(row), ref["row_loss"]) <= BF16_ATOL
+
+
+# ------------------------------------------------------------------ full-size workloads
+def _full_size(name, sample_b, prefix=None):
+    w = seeded.WORKLOADS[name]
+    cfg, W, W64, idx, tgt = model_inputs(name)
+    m = gpu_model(cfg, W)
+    row = torch.empty(idx.shape, device="cuda")
+    sc = torch.empty(2, dtype=torch.float64, device="cuda")
+    logits, loss = m(idx.cuda(), tgt.cuda(), row_loss=row, loss_sum_count=sc, sync_check=True)
+    # whole-batch properties: the loss is the mean of the row losses, and equals the loss of
+    # the returned (bf16-rounded) logits within the rounding of the logits
+    rows = f64(row)
+    assert float(sc[1]) == w.batch * w.seq_len
+    assert abs(float(loss) - rows.mean()) <= 1e-6 * abs(rows.mean())
+    # sampled sequences against the oracle
+    for b in sample_b:
+        T = prefix or w.seq_len
+        ref = oracle.forward(W64, cfg, idx[b:b + 1, :T].numpy(), tgt[b:b + 1, :T].numpy())
+        got = f64(logits[b:b + 1, :T])
+        err = max_abs(got, ref["logits"])
+        assert err <= BF16_ATOL, (b, err)
+        assert max_abs(rows[b, :T], ref["row_loss"][0]) <= BF16_ATOL
+        assert abs(rows[b, :T].mean() - ref["loss"]) <= LOSS_RTOL * abs(ref["loss"])
+        if b == sample_b[0]:
+            z = got[0]
+            _, lrow, _ = oracle.cross_entropy(z, tgt[b, :T].numpy())
+            assert max_abs(lrow, rows[b, :T]) <= 2e-2   # loss of the stored logits
+    return m, idx, logits
+
+
+def test_gpt2_full_size():
+    _full_size("gpt2", sample_b=[0, 11])
+
+
+def test_gpt2_medium_full_size():
+    _full_size("gpt2-medium", sample_b=[5], prefix=384)
+
+
+def test_gpt2_xl_full_size_and_last_position():
+    m, idx, logits = _full_size("gpt2-xl", sample_b=[2], prefix=256)
+    last, _ = m(idx.cuda(), None, sync_check=True)
+    assert last.shape == (4, 1, 50304)
+    assert max_abs(f64(last)[:, 0], f64(logits[:, -1])) <= BF16_ATOL
+
+
+def test_loss_at_init_band():
+    """GPT-2 init: loss near ln V + 0.02^2 C / 2 (a band, not parity)."""
+    cfg, W, _, idx, tgt = model_inputs("gpt2", B=2, T=256)
+    _, loss = gpu_model(cfg, W)(idx.cuda(), tgt.cuda(), sync_check=True)
+    assert abs(float(loss) - (math.log(50304) + 0.02 ** 2 * 768 / 2)) < 0.1
+
+
+# ------------------------------------------------------------------ device-side errors
+def test_bad_token_id_reports_index():
+    from decoder_only_transformer_causal_b200 import native
+    cfg, W, _, idx, tgt = model_inputs("gpt2", n_layer=1, B=1, T=64)
+    m = gpu_model(cfg, W)
+    idx[0, 5] = 60000
+    with pytest.raises(native.GPTError) as e:
+        m(idx.cuda(), tgt.cuda(), sync_check=True)
+    assert e.value.status == native.GPT_ERR_INDEX
+    idx[0, 5] = 1
+    tgt[0, 9] = -7
+    with pytest.raises(native.GPTError) as e:
+        m(idx.cuda(), tgt.cuda(), sync_check=True)
+    assert e.value.status == native.GPT_ERR_INDEX
+    tgt[0, 9] = 3
+    m(idx.cuda(), tgt.cuda(), sync_check=True)   # the context is still usable
+
+
+def test_e2e_host_call_matches_device_call():
+    cfg, W, _, idx, tgt = model_inputs("gpt2", n_layer=2, B=2, T=128)
+    m = gpu_model(cfg, W)
+    _, loss = m(idx.cuda(), tgt.cuda(), sync_check=True)
+    assert m.forward_host(idx, tgt) == float(loss)
