@@ -45,6 +45,9 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-kernels", action="store_true", help="skip the per-kernel timings")
+    ap.add_argument("--profile-kernel", default=None,
+                    help="launch only this kernel of the forward (names as in kernels_ms_per_forward): "
+                         "--warmup untimed then --steps timed launches; for profiler captures")
     return ap.parse_args()
 
 
@@ -211,49 +214,75 @@ def time_region(fn, iters: int, stream) -> float:
     return start.elapsed_time(end) / iters
 
 
-def kernel_timings(w, model, native, dev, stream):
-    """Average duration of each kernel of the forward pass, launched alone through the C ABI
-    on the shapes the forward uses (inputs > L2 for the GEMMs on the token dimension)."""
-    N, C, V = w.batch * w.seq_len, w.n_embd, w.vocab_size
+def kernel_ops(w, native, dev, stream, only=None):
+    """Each kernel of the forward pass as a closure launching it alone through the C ABI on the
+    shapes the forward uses: name -> (fn, algorithmic work per launch, bound, launches per
+    forward).  Inputs are allocated per kernel (only the one asked for when `only` is set)."""
+    N, C, V, L = w.batch * w.seq_len, w.n_embd, w.vocab_size, w.n_layer
+    hs = C // w.n_head
     g = torch.Generator(device=dev).manual_seed(7)
     bf = torch.bfloat16
-    u = torch.randn((N, C), generator=g, device=dev).to(bf)
-    hbuf = torch.randn((N, 4 * C), generator=g, device=dev).to(bf)
-    Wa = (0.02 * torch.randn((3 * C, C), generator=g, device=dev)).to(bf)
-    Wp = (0.02 * torch.randn((C, C), generator=g, device=dev)).to(bf)
-    Wf = (0.02 * torch.randn((4 * C, C), generator=g, device=dev)).to(bf)
-    W2 = (0.02 * torch.randn((C, 4 * C), generator=g, device=dev)).to(bf)
-    b3, b1, b4 = (torch.zeros(n, device=dev, dtype=bf) for n in (3 * C, C, 4 * C))
-    qkv_out = torch.empty((N, 3 * C), device=dev, dtype=bf)
-    x = torch.zeros((N, C), device=dev)
-    h_out = torch.empty((N, 4 * C), device=dev, dtype=bf)
-    q, k, v = (torch.randn((w.batch, w.n_head, w.seq_len, C // w.n_head), generator=g, device=dev).to(bf)
-               for _ in range(3))
-    y = torch.empty_like(q)
-    wte = (0.02 * torch.randn((V, C), generator=g, device=dev)).to(bf)
-    _, tgt = seeded.make_tokens(1, N, w.token_high)
-    tgt = tgt.reshape(-1).to(dev)
-    logits = torch.empty((N, V), device=dev, dtype=bf)
-    loss = torch.empty((), device=dev)
-    lm_ws = native.alloc_workspace(native.lm_head_workspace_bytes(N, V), dev)
-    xf = torch.randn((N, C), generator=g, device=dev)
-    ln_w, ln_b = torch.ones(C, device=dev, dtype=bf), torch.zeros(C, device=dev, dtype=bf)
-    ln_out = torch.empty((N, C), device=dev, dtype=bf)
-    ops = {
-        "gemm_c_attn": (lambda: native.linear(u, Wa, b3, out=qkv_out, stream=stream), 2.0 * N * 3 * C * C, "tensor", w.n_layer),
-        "attention": (lambda: native.attention(q, k, v, y=y, stream=stream),
-                      attention_flops(w.batch, w.n_head, w.seq_len, C // w.n_head), "tensor", w.n_layer),
-        "gemm_attn_proj_resid": (lambda: native.linear(u, Wp, b1, out=x, epilogue=native.GPT_EPI_RESID, stream=stream),
-                                 2.0 * N * C * C, "tensor", w.n_layer),
-        "gemm_c_fc_gelu": (lambda: native.linear(u, Wf, b4, out=h_out, epilogue=native.GPT_EPI_GELU, stream=stream),
-                           2.0 * N * 4 * C * C, "tensor", w.n_layer),
-        "gemm_mlp_proj_resid": (lambda: native.linear(hbuf, W2, b1, out=x, epilogue=native.GPT_EPI_RESID, stream=stream),
-                                2.0 * N * 4 * C * C, "tensor", w.n_layer),
-        "lm_head_ce": (lambda: native.lm_head_loss(u, wte, tgt, workspace=lm_ws, logits=logits, loss=loss, stream=stream),
-                       2.0 * N * C * V, "tensor", 1),
-        "layernorm": (lambda: native.layernorm(xf, ln_w, ln_b, out=ln_out, stream=stream), N * C * (4 + 2) + 4 * C,
-                      "hbm", 2 * w.n_layer + 1),
+
+    def rnd(shape, std=1.0, dtype=bf):
+        return (std * torch.randn(shape, generator=g, device=dev)).to(dtype)
+
+    def gemm(K, Nout, epi, out_dtype):
+        a, Wt, bias = rnd((N, K)), rnd((Nout, K), 0.02), torch.zeros(Nout, device=dev, dtype=bf)
+        out = torch.zeros((N, Nout), device=dev, dtype=out_dtype)
+        return lambda: native.linear(a, Wt, bias, out=out, epilogue=epi, stream=stream)
+
+    def attention():
+        q, k, v = (rnd((w.batch, w.n_head, w.seq_len, hs)) for _ in range(3))
+        y = torch.empty_like(q)
+        return lambda: native.attention(q, k, v, y=y, stream=stream)
+
+    def lm_head():
+        u, wte = rnd((N, C)), rnd((V, C), 0.02)
+        _, tgt = seeded.make_tokens(1, N, w.token_high)
+        tgt = tgt.reshape(-1).to(dev)
+        logits = torch.empty((N, V), device=dev, dtype=bf)
+        loss = torch.empty((), device=dev)
+        ws = native.alloc_workspace(native.lm_head_workspace_bytes(N, V), dev)
+        return lambda: native.lm_head_loss(u, wte, tgt, workspace=ws, logits=logits, loss=loss, stream=stream)
+
+    def layernorm():
+        x = rnd((N, C), 1.0, torch.float32)
+        lw, lb = torch.ones(C, device=dev, dtype=bf), torch.zeros(C, device=dev, dtype=bf)
+        out = torch.empty((N, C), device=dev, dtype=bf)
+        return lambda: native.layernorm(x, lw, lb, out=out, stream=stream)
+
+    # name -> (factory, work per launch, bound, launches per forward, kernel function)
+    specs = {
+        "gemm_c_attn": (lambda: gemm(C, 3 * C, native.GPT_EPI_STORE, bf), 2.0 * N * 3 * C * C, "tensor", L),
+        "attention": (attention, attention_flops(w.batch, w.n_head, w.seq_len, hs), "tensor", L),
+        "gemm_attn_proj_resid": (lambda: gemm(C, C, native.GPT_EPI_RESID, torch.float32), 2.0 * N * C * C,
+                                 "tensor", L),
+        "gemm_c_fc_gelu": (lambda: gemm(C, 4 * C, native.GPT_EPI_GELU, bf), 2.0 * N * 4 * C * C, "tensor", L),
+        "gemm_mlp_proj_resid": (lambda: gemm(4 * C, C, native.GPT_EPI_RESID, torch.float32), 2.0 * N * 4 * C * C,
+                                "tensor", L),
+        "lm_head_ce": (lm_head, 2.0 * N * C * V, "tensor", 1),
+        "layernorm": (layernorm, float(N * C * (4 + 2) + 4 * C), "hbm", 2 * L + 1),
     }
+    return {k: (make(), work, bound, per) for k, (make, work, bound, per) in specs.items()
+            if only is None or k == only}
+
+
+# The kernel function (as ncu names it) behind each op of kernel_ops: ops sharing a function
+# are one kernel for the roofline, whose work and time add up.
+KERNEL_OF = {
+    "gemm_c_attn": "gemm_bf16_tc<256, EPI_STORE, 4>",
+    "gemm_attn_proj_resid": "gemm_bf16_tc<256, EPI_RESID, 4>",
+    "gemm_mlp_proj_resid": "gemm_bf16_tc<256, EPI_RESID, 4>",
+    "gemm_c_fc_gelu": "gemm_bf16_tc<256, EPI_GELU, 8>",
+    "lm_head_ce": "gemm_bf16_tc<256, EPI_CE, 8> (+ ce_rows, loss_finalize)",
+    "attention": "attention_fwd_tc",
+    "layernorm": "layernorm_kernel<bf16>",
+}
+
+
+def kernel_timings(w, native, dev, stream):
+    """Average duration of each kernel of the forward pass launched alone."""
+    ops = kernel_ops(w, native, dev, stream)
     out = {}
     for name, (fn, work, bound, per_fwd) in ops.items():
         for _ in range(3):
@@ -268,6 +297,8 @@ def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.profile_kernel:
+        return profile_kernel(args)
     assert args.warmup >= 3, "at least 3 warm-up steps"
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -369,23 +400,33 @@ def main():
             "clocks": clocks.summary(),
         }
     if not args.no_kernels and rank == 0:
-        kt = kernel_timings(w, model, native, dev, stream)
-        # dominant kernel: largest time share of one forward
+        kt = kernel_timings(w, native, dev, stream)
+        # dominant kernel: the kernel function with the largest time share of one forward
         share = {k: v["ms"] * v["per_forward"] for k, v in kt.items()}
-        dom = max(share, key=share.get)
-        d = kt[dom]
+        by_fn = {}
+        for k, v in kt.items():
+            f = by_fn.setdefault(KERNEL_OF[k], {"ms": 0.0, "work": 0.0, "launches": 0, "bound": v["bound"]})
+            f["ms"] += v["ms"] * v["per_forward"]
+            f["work"] += v["work"] * v["per_forward"]
+            f["launches"] += v["per_forward"]
+        dom = max(by_fn, key=lambda f: by_fn[f]["ms"])
+        d = by_fn[dom]
+        ms_launch = d["ms"] / d["launches"]
+        work_launch = d["work"] / d["launches"]
         if d["bound"] == "tensor":
-            achieved = d["work"] / (d["ms"] / 1000.0) / 1e12
+            achieved = work_launch / (ms_launch / 1000.0) / 1e12
             peak = peaks["bf16_tflops"]
             unit = "TFLOP/s"
         else:
-            achieved = d["work"] / (d["ms"] / 1000.0) / 1e9
+            achieved = work_launch / (ms_launch / 1000.0) / 1e9
             peak = peaks["hbm_gbs"]
             unit = "GB/s"
         line["roofline"] = {"kernel": dom, "bound": d["bound"], "achieved": achieved, "peak": peak,
                             "unit": unit, "frac": achieved / peak, "traffic": traffic_for(dom),
                             "peak_source": f"{peak_src} (burst, kernel timed alone)",
-                            "work_per_launch": d["work"], "ms_per_launch": d["ms"]}
+                            "work_per_launch": work_launch, "ms_per_launch": ms_launch,
+                            "launches_per_forward": d["launches"],
+                            "share_of_forward": d["ms"] / sum(share.values())}
         a = kt["attention"]
         a_tf = a["work"] / (a["ms"] / 1000.0) / 1e12
         line["attention"] = {"workload": "causal attention B 12, 12 heads, T 1024, hs 64, bf16",
@@ -403,6 +444,21 @@ def main():
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
+    return 0
+
+
+def profile_kernel(args):
+    """Launches one kernel of the forward alone (for an ncu capture of a single kernel)."""
+    from decoder_only_transformer_causal_b200 import native
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream(dev)
+    w = seeded.WORKLOADS[WORKLOAD]
+    fn, work, bound, _ = kernel_ops(w, native, dev, stream, only=args.profile_kernel)[args.profile_kernel]
+    for _ in range(args.warmup):
+        fn()
+    ms = time_region(fn, args.steps, stream)
+    print(json.dumps({"kernel": args.profile_kernel, "ms": ms, "work": work, "bound": bound}))
     return 0
 
 

@@ -57,12 +57,33 @@ struct Cfg {
     static constexpr int PARTS_PER_TILE = NEPI / 4;
 };
 
-GPT_DEVINL float gelu_f(float v, int tanh_mode) {
+// GELU for the epilogue, cheap enough to hide under the next tile's MMAs.
+//  erf form:  x * Phi(x), Phi(x) = (1 + erf(x / sqrt 2)) / 2, with erf from Abramowitz & Stegun,
+//             Handbook of Mathematical Functions (1964), formula 7.1.26:
+//             erf(z) = 1 - t (a1 + t (a2 + t (a3 + t (a4 + t a5)))) exp(-z^2), t = 1 / (1 + p z),
+//             z >= 0, absolute error <= 1.5e-7; odd symmetry gives z < 0.
+//  tanh form: 0.5 x (1 + tanh(u)) = x / (1 + exp(-2u)), u = sqrt(2/pi) (x + 0.044715 x^3).
+GPT_DEVINL float rcp_approx(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+GPT_DEVINL float gelu_f(float x, int tanh_mode) {
+    constexpr float kLog2e = 1.4426950408889634f;
     if (tanh_mode) {
-        const float k0 = 0.7978845608028654f;  // sqrt(2/pi)
-        return 0.5f * v * (1.0f + tanhf(k0 * (v + 0.044715f * v * v * v)));
+        const float u2 = -2.0f * 0.7978845608028654f * x * fmaf(0.044715f * x, x, 1.0f);
+        return x * rcp_approx(1.0f + exp2_approx(u2 * kLog2e));
     }
-    return 0.5f * v * (1.0f + erff(v * 0.7071067811865476f));
+    const float z = fabsf(x) * 0.7071067811865476f;
+    const float t = rcp_approx(fmaf(0.3275911f, z, 1.0f));
+    float q = fmaf(t, 1.061405429f, -1.453152027f);
+    q = fmaf(t, q, 1.421413741f);
+    q = fmaf(t, q, -0.284496736f);
+    q = fmaf(t, q, 0.254829592f);
+    q *= t;
+    const float erf_abs = fmaf(-q, exp2_approx(-z * z * kLog2e), 1.0f);
+    return 0.5f * x * (1.0f + copysignf(erf_abs, x));
 }
 
 template <int BN, int EPI, int NEPI>
