@@ -52,7 +52,7 @@ class gpt_config_t(ctypes.Structure):
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"{LIB_PATH} is missing: build it with "
-                          "`python -m decoder_only_transformer_causal_b200.build`")
+                          "`python decoder_only_transformer_causal_b200/build.py`")
     lib = ctypes.CDLL(LIB_PATH)
     P, I, Z, D = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_int
     CFG = ctypes.POINTER(gpt_config_t)
@@ -73,6 +73,7 @@ def _load() -> ctypes.CDLL:
         "gpt_linear": (I, [P, P, P, P, I, I, I, D, I, I, P, P]),
         "gpt_lm_head_workspace_bytes": (Z, [I, I]),
         "gpt_lm_head_loss": (I, [P, P, P, I, I, I, D, P, P, P, P, P, Z, P, I]),
+        "gpt_lm_head_loss_noalloc": (I, [P, P, P, I, I, I, D, P, P, P, P, P, I]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -86,7 +87,7 @@ LIB = _load()
 EXPORTED = ("gpt_status_string", "gpt_abi_version", "gpt_validate_config", "gpt_weights_bytes",
             "gpt_weights_count", "gpt_weights_layout", "gpt_workspace_bytes", "gpt_check_status",
             "gpt_forward", "gpt_block", "gpt_attention", "gpt_embed", "gpt_layernorm", "gpt_linear",
-            "gpt_lm_head_workspace_bytes", "gpt_lm_head_loss")
+            "gpt_lm_head_workspace_bytes", "gpt_lm_head_loss", "gpt_lm_head_loss_noalloc")
 
 
 def status_string(status: int) -> str:
@@ -282,6 +283,23 @@ def linear(x, W, b=None, out=None, epilogue=GPT_EPI_STORE, gelu=GPT_GELU_ERF, st
 
 def lm_head_workspace_bytes(rows: int, V: int) -> int:
     return LIB.gpt_lm_head_workspace_bytes(rows, V)
+
+
+def lm_head_loss_noalloc(u, wte, targets, logits=None, loss=None, row_loss=None, loss_sum_count=None,
+                         stream=None, sync_check=False):
+    """gpt_lm_head_loss_noalloc: the head and loss with the library's static scratch (no
+    workspace); for callers that cannot allocate device memory at this point."""
+    rows, C = u.shape
+    V = wte.shape[0]
+    dtype = {torch.bfloat16: GPT_DTYPE_BF16, torch.float32: GPT_DTYPE_F32}[u.dtype]
+    if logits is None:
+        logits = torch.empty((rows, V), dtype=u.dtype, device=u.device)
+    if loss is None:
+        loss = torch.empty((), dtype=torch.float32, device=u.device)
+    _check(LIB.gpt_lm_head_loss_noalloc(_ptr(u), _ptr(wte), _ptr(targets), rows, C, V, dtype, _ptr(logits),
+                                        _ptr(loss), _ptr(row_loss), _ptr(loss_sum_count), _stream(stream),
+                                        GPT_FLAG_SYNC_CHECK if sync_check else 0), "gpt_lm_head_loss_noalloc")
+    return logits, loss
 
 
 def lm_head_loss(u, wte, targets, workspace=None, logits=None, loss=None, row_loss=None,

@@ -195,6 +195,25 @@ int gpt_lm_head_loss(const void* u, const void* wte, const int64_t* targets, int
                      double* loss_sum_count, void* workspace, size_t workspace_bytes,
                      void* stream, int flags);
 
+/* gpt_lm_head_loss without a workspace argument.  The pages have no counterpart: this exists
+ * for callers that cannot allocate device memory when they need the loss (a serving process
+ * that gave all of its GPU memory to a fixed pool at start-up, a plugin inside another
+ * framework whose allocator it may not bypass, a latency-critical loop that cannot pay for
+ * cudaMalloc and its implicit device synchronisation).  Arguments and results are those of
+ * gpt_lm_head_loss.
+ *   Scratch: a static 16 MiB device array inside this library, held by every GPU that uses the
+ *   library until the process exits.  A request needing more than that
+ *   (gpt_lm_head_workspace_bytes(rows, V) > 16 MiB; about 5,300 rows at V = 50304) returns
+ *   GPT_ERR_WS_TOO_SMALL before anything is enqueued.  Nothing is allocated or freed.
+ *   The first call on each device looks up the array's device address (cudaGetSymbolAddress)
+ *   with that device current; make that first call before any stream capture begins.
+ *   All calls on a device share the array and it keeps the last call's contents (the status
+ *   word is cleared at the start of each call): calls whose work overlaps on the GPU race, so
+ *   order them on one stream.  With GPT_FLAG_SYNC_CHECK the status word is read from the array. */
+int gpt_lm_head_loss_noalloc(const void* u, const void* wte, const int64_t* targets, int rows,
+                             int C, int V, int dtype, void* logits, float* loss, float* row_loss,
+                             double* loss_sum_count, void* stream, int flags);
+
 #ifdef __cplusplus
 }
 #endif
