@@ -1,6 +1,8 @@
 """Builds the CUDA library libgptb200.so in-tree (sm_100a only).
 
-    python -m decoder_only_transformer_causal_b200.build [--force] [--verbose]
+    python decoder_only_transformer_causal_b200/build.py [--force] [--verbose]
+
+(run by path: importing the package would load the library before it is built)
 
 Each csrc/*.cu is compiled by nvcc for ``-gencode arch=compute_100a,code=sm_100a`` into
 _build/, then linked into decoder_only_transformer_causal_b200/_lib/libgptb200.so with the
