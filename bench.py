@@ -269,12 +269,14 @@ def kernel_ops(w, native, dev, stream, only=None):
 
 # The kernel function (as ncu names it) behind each op of kernel_ops: ops sharing a function
 # are one kernel for the roofline, whose work and time add up.
+# Template arguments as ncu prints them: <BN, epilogue (0 store, 1 GELU, 2 residual add,
+# 3 cross-entropy partials), GELU tanh form>.
 KERNEL_OF = {
-    "gemm_c_attn": "gemm_bf16_tc<256, EPI_STORE, 4>",
-    "gemm_attn_proj_resid": "gemm_bf16_tc<256, EPI_RESID, 4>",
-    "gemm_mlp_proj_resid": "gemm_bf16_tc<256, EPI_RESID, 4>",
-    "gemm_c_fc_gelu": "gemm_bf16_tc<256, EPI_GELU, 8>",
-    "lm_head_ce": "gemm_bf16_tc<256, EPI_CE, 8> (+ ce_rows, loss_finalize)",
+    "gemm_c_attn": "gemm_bf16_tc<256, 0, 0>",
+    "gemm_attn_proj_resid": "gemm_bf16_tc<256, 2, 0>",
+    "gemm_mlp_proj_resid": "gemm_bf16_tc<256, 2, 0>",
+    "gemm_c_fc_gelu": "gemm_bf16_tc<256, 1, 0>",
+    "lm_head_ce": "gemm_bf16_tc<256, 3, 0> (+ ce_rows, loss_finalize)",
     "attention": "attention_fwd_tc",
     "layernorm": "layernorm_kernel<bf16>",
 }
@@ -465,7 +467,7 @@ def profile_kernel(args):
 def traffic_for(kernel: str):
     """DRAM bytes per launch of `kernel` from the committed ncu summary, if it was taken on the
     current source of that kernel; else None."""
-    p = os.path.join(ROOT, "profiles", "traffic.json")
+    p = os.path.join(ROOT, "profiles", "traffic.json")  # written from an ncu capture of the current source
     if not os.path.exists(p):
         return None
     with open(p) as f:

@@ -197,13 +197,15 @@ __global__ void __launch_bounds__(THREADS, 2)
                 break;
             }
             tc_fence_after();
+            // S row -> registers (raw scores; the 1/sqrt(hs) * log2(e) scale is folded into the
+            // exponent below).  8 independent partial maxima / sums keep the dependency chains short.
             float s[BKV];
 #pragma unroll
-            for (int c = 0; c < BKV; c += 32) {
-                uint32_t u[32];
-                tmem_ld32(tS + c, u);
+            for (int c = 0; c < BKV; c += 64) {
+                uint32_t u[64];
+                tmem_ld64(tS + c, u);
 #pragma unroll
-                for (int e = 0; e < 32; ++e) s[c + e] = __uint_as_float(u[e]) * p.scale_log2;
+                for (int e = 0; e < 64; ++e) s[c + e] = __uint_as_float(u[e]);
             }
             tc_fence_before();
             mbar_arrive(s_free);
@@ -213,24 +215,30 @@ __global__ void __launch_bounds__(THREADS, 2)
                 for (int c = 0; c < BKV; ++c)
                     if (c > r) s[c] = -INFINITY;
             }
-            float mx = s[0];
+            float m8[8];
 #pragma unroll
-            for (int c = 1; c < BKV; ++c) mx = fmaxf(mx, s[c]);
+            for (int e = 0; e < 8; ++e) m8[e] = s[e];
+#pragma unroll
+            for (int c = 8; c < BKV; ++c) m8[c & 7] = fmaxf(m8[c & 7], s[c]);
+            const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                                   fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * p.scale_log2;
             float alpha = 1.f;
             if (mx > m_used + kRescaleThreshold || m_used == -INFINITY) {
                 alpha = exp2_approx(m_used - mx);  // 0 on the first tile
                 m_used = mx;
             }
-            float rs = 0.f;
+            const float neg_m = -m_used;
+            float r8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
             uint32_t pk0[32], pk1[32];
 #pragma unroll
             for (int c = 0; c < BKV; c += 2) {
-                const float p0 = exp2_approx(s[c] - m_used);
-                const float p1 = exp2_approx(s[c + 1] - m_used);
-                rs += p0 + p1;
+                const float p0 = exp2_approx(fmaf(s[c], p.scale_log2, neg_m));
+                const float p1 = exp2_approx(fmaf(s[c + 1], p.scale_log2, neg_m));
+                r8[(c >> 1) & 7] += p0 + p1;
                 if (c < 64) pk0[c / 2] = pack_bf16x2(p0, p1);
                 else pk1[(c - 64) / 2] = pack_bf16x2(p0, p1);
             }
+            const float rs = ((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7]));
             l = l * alpha + rs;
             // P_j may overwrite P_{j-1} and O may be rescaled only after O += P_{j-1} V_{j-1}.
             if (j > 0) {

@@ -8,10 +8,11 @@ namespace {
 
 constexpr int kBN = 256;
 
-template <int EPI, int NEPI>
-int launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const gemm::Params& p, cudaStream_t s) {
-    using L = gemm::Cfg<kBN, NEPI>;
-    auto kern = gemm::gemm_bf16_tc<kBN, EPI, NEPI>;
+template <int EPI, int GELU_TANH>
+int launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, const gemm::Params& p,
+               cudaStream_t s) {
+    using L = gemm::Cfg<kBN>;
+    auto kern = gemm::gemm_bf16_tc<kBN, EPI, GELU_TANH>;
     static bool configured = false;
     if (!configured) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_BYTES);
@@ -20,13 +21,13 @@ int launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const gemm::Params&
     }
     const int tiles = ((p.M + gemm::BM - 1) / gemm::BM) * ((p.N + kBN - 1) / kBN);
     const int grid = tiles < num_sms() ? tiles : num_sms();
-    kern<<<grid, L::THREADS, L::SMEM_BYTES, s>>>(ta, tb, p);
+    kern<<<grid, L::THREADS, L::SMEM_BYTES, s>>>(ta, tb, tc, p);
     return cuda_status(cudaGetLastError());
 }
 
 }  // namespace
 
-int gemm_ce_parts(int N) { return ((N + kBN - 1) / kBN) * gemm::Cfg<kBN, 8>::PARTS_PER_TILE; }
+int gemm_ce_parts(int N) { return ((N + kBN - 1) / kBN) * gemm::Cfg<kBN>::PARTS_PER_TILE; }
 
 int launch_gemm_bf16(const bf16* A, long long lda, const bf16* W, long long ldw, const bf16* bias,
                      void* out, long long ldo, int M, int N, int K, int epilogue, int gelu,
@@ -39,6 +40,12 @@ int launch_gemm_bf16(const bf16* A, long long lda, const bf16* W, long long ldw,
     rc = make_tmap_bf16_2d(&tb, W, static_cast<uint64_t>(K), static_cast<uint64_t>(N),
                            static_cast<uint64_t>(ldw) * 2, gemm::BK, kBN);
     if (rc) return rc;
+    // Output map for the epilogue's TMA stores: 32-row boxes of 64 bytes (32 bf16 or 16 fp32).
+    CUtensorMap tc;
+    const bool out_f32 = epilogue == GPT_EPI_RESID;
+    rc = make_tmap_2d_sw64(&tc, out, out_f32, static_cast<uint64_t>(N), static_cast<uint64_t>(M),
+                           static_cast<uint64_t>(ldo) * (out_f32 ? 4 : 2), out_f32 ? 16 : 32, 32);
+    if (rc) return rc;
     gemm::Params p{};
     p.M = M;
     p.N = N;
@@ -46,19 +53,22 @@ int launch_gemm_bf16(const bf16* A, long long lda, const bf16* W, long long ldw,
     p.bias = bias;
     p.out = out;
     p.ldo = ldo;
-    p.gelu_tanh = gelu == GPT_GELU_TANH;
+    // Visit tiles so that the larger operand streams from memory once (see gemm_tc.cuh).
+    p.n_fastest = static_cast<long long>(M) >= static_cast<long long>(N) ? 1 : 0;
     p.status = status;
     switch (epilogue) {
-        case GPT_EPI_STORE: return launch_one<gemm::EPI_STORE, 4>(ta, tb, p, s);
-        case GPT_EPI_GELU: return launch_one<gemm::EPI_GELU, 8>(ta, tb, p, s);
-        case GPT_EPI_RESID: return launch_one<gemm::EPI_RESID, 4>(ta, tb, p, s);
+        case GPT_EPI_STORE: return launch_one<gemm::EPI_STORE, 0>(ta, tb, tc, p, s);
+        case GPT_EPI_GELU:
+            return gelu == GPT_GELU_TANH ? launch_one<gemm::EPI_GELU, 1>(ta, tb, tc, p, s)
+                                         : launch_one<gemm::EPI_GELU, 0>(ta, tb, tc, p, s);
+        case GPT_EPI_RESID: return launch_one<gemm::EPI_RESID, 0>(ta, tb, tc, p, s);
         case gemm::EPI_CE:
             if (!ce) return GPT_ERR_NULL;
             p.targets = ce->targets;
             p.part = ce->part;
             p.tlogit = ce->tlogit;
             p.n_part = ce->n_part;
-            return launch_one<gemm::EPI_CE, 8>(ta, tb, p, s);
+            return launch_one<gemm::EPI_CE, 0>(ta, tb, tc, p, s);
         default: return GPT_ERR_UNSUPPORTED;
     }
 }

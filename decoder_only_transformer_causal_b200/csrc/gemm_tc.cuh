@@ -8,14 +8,21 @@
 //   EPI_RESID  x_fp32  += acc + b                 (both c_proj: the residual add of Block)
 //   EPI_CE     logits_bf16 = acc, plus per (row, column slice) the running maximum and the sum
 //              of exp(z - max) and, in the slice holding the row's target, z[target] in fp32:
-//              the pieces of F.cross_entropy's logsumexp (§3.3), reduced by ce_reduce.
+//              the pieces of F.cross_entropy's logsumexp (§3.3), reduced by ce_rows.
 //
-// Design: one persistent CTA per SM walks the output tiles (128 x BN) in m-fastest order so
-// concurrently running CTAs share the same W columns in L2.  Warp 0 streams 128x64 A and
-// BNx64 W tiles with TMA (128-byte swizzle) through a kStages-deep shared-memory ring; one
-// thread of warp 1 issues tcgen05.mma (M=128, N=BN, K=16) into one of two TMEM accumulators;
-// the epilogue warps drain the other accumulator (tcgen05.ld) while the next tile's MMAs
-// run.  Every wait is bounded (common.cuh).
+// Design: one persistent CTA per SM walks the output tiles (128 x BN).  Tiles are visited so
+// that the larger operand is streamed from HBM once: n-fastest when A is the larger (the CTAs
+// sharing an A row-block run together), m-fastest when W is (the head: the CTAs of a wave share
+// W columns).  Warp 0 streams 128x64 A and BNx64 W tiles with TMA (128-byte swizzle) through a
+// kStages-deep shared-memory ring; one thread of warp 1 issues tcgen05.mma (M=128, N=BN, K=16)
+// into one of two TMEM accumulators; 8 epilogue warps drain the other accumulator while the
+// next tile's MMAs run.  Each epilogue warp owns 32 rows (its TMEM lane quarter) and half of the
+// tile's columns; it turns 32 columns at a time into a 32 x 64-byte tile in a private shared-
+// memory buffer (64-byte swizzle: conflict-free from one-row-per-thread writes) and one lane hands
+// that tile to TMA: a tile store for the bf16 outputs, a tile reduce-add for the residual stream
+// (x += acc + b happens at the destination; x never travels to the SM).  TMA clips the ragged
+// edges.  The tile's bias is staged in shared memory before the accumulator wait.  Every wait is
+// bounded (common.cuh).
 #pragma once
 
 #include "common.cuh"
@@ -26,15 +33,16 @@ namespace gemm {
 constexpr int BM = 128;
 constexpr int BK = 64;  // one 128-byte swizzle row of bf16
 constexpr int kStages = 4;
+constexpr int NEPI = 8;  // epilogue warps: two per TMEM lane quarter, each half of BN
 
 enum Epi { EPI_STORE = 0, EPI_GELU = 1, EPI_RESID = 2, EPI_CE = 3 };
 
 struct Params {
     int M, N, K;
+    int n_fastest;     // tile order: 1 = n fastest (A-heavy), 0 = m fastest (W-heavy)
     const bf16* bias;  // [N] or nullptr
     void* out;         // bf16 [M, ldo] (STORE / GELU / CE logits) or fp32 [M, ldo] (RESID)
     long long ldo;
-    int gelu_tanh;
     const int64_t* targets;  // EPI_CE: [M]
     float2* part;            // EPI_CE: [M, n_part] of (max, sum exp(z - max))
     float* tlogit;           // EPI_CE: [M], z[target] in fp32
@@ -42,18 +50,20 @@ struct Params {
     int32_t* status;
 };
 
-template <int BN, int NEPI>
+template <int BN>
 struct Cfg {
-    static_assert(BN == 128 || BN == 256, "BN");
-    static_assert(NEPI == 4 || NEPI == 8, "NEPI");
+    static_assert(BN == 256, "BN");
     static constexpr int A_BYTES = BM * BK * 2;
     static constexpr int B_BYTES = BN * BK * 2;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-    static constexpr int BAR_OFF = kStages * STAGE_BYTES;
+    static constexpr int BIAS_OFF = kStages * STAGE_BYTES;    // one bias slice per epilogue warp
+    static constexpr int STG_OFF = BIAS_OFF + NEPI * (BN / (NEPI / 4)) * 4;
+    static constexpr int STG_BYTES = 32 * 64;                 // 32 rows x 64 bytes per warp
+    static constexpr int BAR_OFF = STG_OFF + NEPI * STG_BYTES;
     static constexpr int SMEM_BYTES = BAR_OFF + 256 + 1024;  // barriers + alignment slack
     static constexpr int TMEM_COLS = 2 * BN;                  // two accumulators
     static constexpr int THREADS = 64 + NEPI * 32;
-    static constexpr int COLS_PER_WARP = BN / (NEPI / 4);
+    static constexpr int COLS_PER_WARP = BN / (NEPI / 4);     // 128
     static constexpr int PARTS_PER_TILE = NEPI / 4;
 };
 
@@ -69,9 +79,10 @@ GPT_DEVINL float rcp_approx(float x) {
     return y;
 }
 
-GPT_DEVINL float gelu_f(float x, int tanh_mode) {
+template <int TANH>
+GPT_DEVINL float gelu_f(float x) {
     constexpr float kLog2e = 1.4426950408889634f;
-    if (tanh_mode) {
+    if (TANH) {
         const float u2 = -2.0f * 0.7978845608028654f * x * fmaf(0.044715f * x, x, 1.0f);
         return x * rcp_approx(1.0f + exp2_approx(u2 * kLog2e));
     }
@@ -86,14 +97,16 @@ GPT_DEVINL float gelu_f(float x, int tanh_mode) {
     return 0.5f * x * (1.0f + copysignf(erf_abs, x));
 }
 
-template <int BN, int EPI, int NEPI>
-__global__ void __launch_bounds__(Cfg<BN, NEPI>::THREADS, 1)
+template <int BN, int EPI, int GELU_TANH>
+__global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)  // 10 warps: <= 168 registers per thread
     gemm_bf16_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                 const Params p) {
-    using L = Cfg<BN, NEPI>;
+                 const __grid_constant__ CUtensorMap tmC, const Params p) {
+    using L = Cfg<BN>;
+    constexpr int COLS = L::COLS_PER_WARP;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
+    float* sbias = reinterpret_cast<float*>(smem + L::BIAS_OFF);  // [NEPI][COLS]
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
     uint64_t* empty = full + kStages;
     uint64_t* tfull = empty + kStages;
@@ -108,6 +121,15 @@ __global__ void __launch_bounds__(Cfg<BN, NEPI>::THREADS, 1)
     const int num_n = (p.N + BN - 1) / BN;
     const int num_tiles = num_m * num_n;
     const int num_kb = (p.K + BK - 1) / BK;
+    auto tile_mn = [&](int tile, int& m_blk, int& n_blk) {
+        if (p.n_fastest) {
+            n_blk = tile % num_n;
+            m_blk = tile / num_n;
+        } else {
+            m_blk = tile % num_m;
+            n_blk = tile / num_m;
+        }
+    };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -124,6 +146,7 @@ __global__ void __launch_bounds__(Cfg<BN, NEPI>::THREADS, 1)
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
+        tma_prefetch_desc(&tmC);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, L::TMEM_COLS);
@@ -142,8 +165,9 @@ __global__ void __launch_bounds__(Cfg<BN, NEPI>::THREADS, 1)
             long long issued = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-                const int m0 = (tile % num_m) * BM;
-                const int n0 = (tile / num_m) * BN;
+                int m_blk, n_blk;
+                tile_mn(tile, m_blk, n_blk);
+                const int m0 = m_blk * BM, n0 = n_blk * BN;
                 for (int kb = 0; kb < num_kb; ++kb) {
                     if (!mbar_wait(&empty[stage], ph ^ 1u, abort_flag)) {
                         ok = false;
@@ -213,121 +237,149 @@ __global__ void __launch_bounds__(Cfg<BN, NEPI>::THREADS, 1)
         // ------------------------------------------------------------ epilogue warps
         const int ew = warp - 2;
         const int quarter = warp & 3;        // TMEM lanes this warp may access
-        const int half = ew >> 2;            // column slice (NEPI == 8 splits BN in two)
+        const int half = ew >> 2;            // which BN/2 columns of the tile
         int acc = 0;
         uint32_t acc_ph = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-            const int n_blk = tile / num_m;
-            const int m0 = (tile % num_m) * BM;
-            const int n0 = n_blk * BN;
+            int m_blk, n_blk;
+            tile_mn(tile, m_blk, n_blk);
+            const int m0 = m_blk * BM, n0 = n_blk * BN;
+            const int row = m0 + quarter * 32 + lane;
+            const bool row_ok = row < p.M;
+            const int nw0 = n0 + half * COLS;  // first column of this warp's slice
+            float* sb = sbias + ew * COLS;  // this warp's private bias slice
+            uint8_t* stg = smem + L::STG_OFF + ew * L::STG_BYTES;  // this warp's staging tile
+
+            // Before the accumulator is ready: this warp's bias slice into shared memory.
+            if (EPI != EPI_CE) {
+                __syncwarp();  // the previous tile's reads of sb are done
+                for (int c = lane; c < COLS; c += 32) {
+                    const int n = nw0 + c;
+                    sb[c] = (p.bias && n < p.N) ? __bfloat162float(p.bias[n]) : 0.f;
+                }
+                __syncwarp();
+            }
+            long long tgt = -1;
+            if (EPI == EPI_CE && row_ok) tgt = p.targets[row];
+
             const bool got = mbar_wait(&tfull[acc], acc_ph, abort_flag);
             __syncwarp();  // tcgen05.ld below is warp-collective
             if (!__all_sync(0xffffffffu, got)) break;
             tc_fence_after();
-            const int row = m0 + quarter * 32 + lane;
-            const bool row_ok = row < p.M;
-            const uint32_t tbase = tmem_base + static_cast<uint32_t>(acc * BN + half * L::COLS_PER_WARP) +
+            const uint32_t tbase = tmem_base + static_cast<uint32_t>(acc * BN + half * COLS) +
                                    (static_cast<uint32_t>(quarter * 32) << 16);
-            const int nw0 = n0 + half * L::COLS_PER_WARP;  // first column of this warp's slice
+            const int row0 = m0 + quarter * 32;      // first row of this warp's band
+            const bool band_ok = row0 < p.M;         // warp-uniform
+            // Row `lane` of the staging tile; its four 16-byte chunks are swizzled by bits 1-2 of
+            // the row (the 64-byte TMA swizzle).
+            uint4* srow = reinterpret_cast<uint4*>(stg + lane * 64);
+            const int swz = (lane >> 1) & 3;
 
             float run_max = -INFINITY, run_sum = 0.f;
-            long long tgt = -1;
-            if (EPI == EPI_CE && row_ok) tgt = p.targets[row];
+            constexpr float kLog2e = 1.4426950408889634f;
 
+            if (EPI == EPI_RESID) {
 #pragma unroll 1
-            for (int c = 0; c < L::COLS_PER_WARP; c += 32) {
-                uint32_t r[32];
-                tmem_ld32(tbase + c, r);
-                const int n = nw0 + c;
-                if (n >= p.N) continue;  // slice past the right edge (warp-uniform)
-                const bool full_chunk = (n + 32 <= p.N);
-                float v[32];
+                for (int c = 0; c < COLS; c += 32) {
+                    uint32_t r[32];
+                    tmem_ld32(tbase + c, r);
 #pragma unroll
-                for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-
-                if (EPI == EPI_STORE || EPI == EPI_GELU || EPI == EPI_RESID) {
-                    if (p.bias) {
-                        if (full_chunk) {
-                            const uint4* bp = reinterpret_cast<const uint4*>(p.bias + n);
+                    for (int sub = 0; sub < 2; ++sub) {
+                        const int n = nw0 + c + 16 * sub;
+                        if (n >= p.N || !band_ok) continue;  // warp-uniform
+                        float v[16];
 #pragma unroll
-                            for (int q = 0; q < 4; ++q) {
-                                uint4 w = __ldg(bp + q);
-                                const bf16* wb = reinterpret_cast<const bf16*>(&w);
+                        for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r[16 * sub + j]) + sb[c + 16 * sub + j];
+                        if (lane == 0) bulk_wait_read_all();  // the buffer's previous tile was read
+                        __syncwarp();
 #pragma unroll
-                                for (int e = 0; e < 8; ++e) v[q * 8 + e] += __bfloat162float(wb[e]);
-                            }
-                        } else {
-#pragma unroll
-                            for (int j = 0; j < 32; ++j)
-                                if (n + j < p.N) v[j] += __bfloat162float(p.bias[n + j]);
+                        for (int q = 0; q < 4; ++q)
+                            srow[q ^ swz] = make_uint4(__float_as_uint(v[4 * q]), __float_as_uint(v[4 * q + 1]),
+                                                       __float_as_uint(v[4 * q + 2]), __float_as_uint(v[4 * q + 3]));
+                        fence_proxy_async_shared();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_reduce_add_2d(&tmC, stg, n, row0);
+                            bulk_commit();
                         }
                     }
                 }
-                if (EPI == EPI_GELU) {
+            } else {
+#pragma unroll 1
+                for (int c = 0; c < COLS; c += 64) {
+                    uint32_t r[64];
+                    tmem_ld64(tbase + c, r);
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) v[j] = gelu_f(v[j], p.gelu_tanh);
-                }
-                if (EPI == EPI_STORE || EPI == EPI_GELU || EPI == EPI_CE) {
-                    if (row_ok) {
-                        bf16* o = static_cast<bf16*>(p.out) + static_cast<size_t>(row) * p.ldo + n;
-                        if (full_chunk && (p.ldo % 8) == 0) {
-                            uint4* op = reinterpret_cast<uint4*>(o);
+                    for (int h = 0; h < 2; ++h) {
+                        const int cc = c + 32 * h;
+                        const int n = nw0 + cc;
+                        if (n >= p.N) continue;  // warp-uniform
+                        const bool full_chunk = (n + 32 <= p.N);
+                        float v[32];
 #pragma unroll
-                            for (int q = 0; q < 4; ++q) {
-                                uint4 w;
-                                w.x = pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]);
-                                w.y = pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]);
-                                w.z = pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]);
-                                w.w = pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]);
-                                op[q] = w;
-                            }
-                        } else {
-                            for (int j = 0; j < 32; ++j)
-                                if (n + j < p.N) o[j] = __float2bfloat16_rn(v[j]);
-                        }
-                    }
-                }
-                if (EPI == EPI_RESID) {
-                    if (row_ok) {
-                        float* o = static_cast<float*>(p.out) + static_cast<size_t>(row) * p.ldo + n;
-                        if (full_chunk && (p.ldo % 4) == 0) {
-                            float4* op = reinterpret_cast<float4*>(o);
+                        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[32 * h + j]);
+                        if (EPI == EPI_STORE || EPI == EPI_GELU) {
 #pragma unroll
                             for (int q = 0; q < 8; ++q) {
-                                float4 x = op[q];
-                                x.x += v[q * 4 + 0];
-                                x.y += v[q * 4 + 1];
-                                x.z += v[q * 4 + 2];
-                                x.w += v[q * 4 + 3];
-                                op[q] = x;
+                                const float4 b4 = *reinterpret_cast<const float4*>(sb + cc + 4 * q);
+                                v[4 * q + 0] += b4.x;
+                                v[4 * q + 1] += b4.y;
+                                v[4 * q + 2] += b4.z;
+                                v[4 * q + 3] += b4.w;
                             }
-                        } else {
-                            for (int j = 0; j < 32; ++j)
-                                if (n + j < p.N) o[j] += v[j];
                         }
-                    }
-                }
-                if (EPI == EPI_CE) {
-                    constexpr float kLog2e = 1.4426950408889634f;
-                    float cmax = -INFINITY;
+                        if (EPI == EPI_GELU) {
 #pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        if (full_chunk || n + j < p.N) cmax = fmaxf(cmax, v[j]);
-                    const float new_max = fmaxf(run_max, cmax);
-                    float s = 0.f;
-                    const float off = new_max * kLog2e;
+                            for (int j = 0; j < 32; ++j) v[j] = gelu_f<GELU_TANH>(v[j]);
+                        }
+                        if (EPI == EPI_CE) {
+                            float cmax = -INFINITY;
+                            if (full_chunk) {
+                                float m4[4] = {v[0], v[1], v[2], v[3]};
 #pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        if (full_chunk || n + j < p.N) s += exp2_approx(fmaf(v[j], kLog2e, -off));
-                    run_sum = run_sum * exp2_approx((run_max - new_max) * kLog2e) + s;
-                    run_max = new_max;
-                    const long long rel = tgt - n;
-                    if (rel >= 0 && rel < 32) {
-                        float zt = 0.f;
+                                for (int j = 4; j < 32; ++j) m4[j & 3] = fmaxf(m4[j & 3], v[j]);
+                                cmax = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+                            } else {
+                                for (int j = 0; j < 32; ++j)
+                                    if (n + j < p.N) cmax = fmaxf(cmax, v[j]);
+                            }
+                            const float new_max = fmaxf(run_max, cmax);
+                            const float off = new_max * kLog2e;
+                            float s4[4] = {0.f, 0.f, 0.f, 0.f};
+                            if (full_chunk) {
 #pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            if (j == rel) zt = v[j];
-                        if (row_ok) p.tlogit[row] = zt;
+                                for (int j = 0; j < 32; ++j) s4[j & 3] += exp2_approx(fmaf(v[j], kLog2e, -off));
+                            } else {
+                                for (int j = 0; j < 32; ++j)
+                                    if (n + j < p.N) s4[0] += exp2_approx(fmaf(v[j], kLog2e, -off));
+                            }
+                            run_sum = run_sum * exp2_approx((run_max - new_max) * kLog2e) +
+                                      ((s4[0] + s4[1]) + (s4[2] + s4[3]));
+                            run_max = new_max;
+                            const long long rel = tgt - n;
+                            if (rel >= 0 && rel < 32) {
+                                float zt = 0.f;
+#pragma unroll
+                                for (int j = 0; j < 32; ++j)
+                                    if (j == rel) zt = v[j];
+                                if (row_ok) p.tlogit[row] = zt;
+                            }
+                        }
+                        if (!band_ok) continue;  // warp-uniform: no row of this band exists
+                        if (lane == 0) bulk_wait_read_all();  // the buffer's previous tile was read
+                        __syncwarp();
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            srow[q ^ swz] = make_uint4(pack_bf16x2(v[8 * q + 0], v[8 * q + 1]),
+                                                       pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                                                       pack_bf16x2(v[8 * q + 4], v[8 * q + 5]),
+                                                       pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+                        fence_proxy_async_shared();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_2d(&tmC, stg, n, row0);
+                            bulk_commit();
+                        }
                     }
                 }
             }
@@ -340,6 +392,7 @@ __global__ void __launch_bounds__(Cfg<BN, NEPI>::THREADS, 1)
             acc ^= 1;
             if (acc == 0) acc_ph ^= 1u;
         }
+        if (lane == 0) bulk_wait_all();  // this warp's stores and reduce-adds have completed
     }
 
     __syncthreads();

@@ -12,7 +12,15 @@
 
 namespace gpt {
 
-int cuda_status(cudaError_t e) { return e == cudaSuccess ? GPT_OK : GPT_ERR_CUDA; }
+namespace {
+thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+}
+
+int cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return GPT_OK;
+    g_last_cuda_error = e;
+    return GPT_ERR_CUDA;
+}
 
 int num_sms() {
     int dev = 0;
@@ -47,16 +55,16 @@ EncodeTiledFn encode_fn() {
 }
 
 int encode(CUtensorMap* m, const void* base, cuuint32_t rank, const cuuint64_t* dims, const cuuint64_t* strides,
-           const cuuint32_t* box) {
+           const cuuint32_t* box, CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+           CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B) {
     if (reinterpret_cast<uintptr_t>(base) & 15) return GPT_ERR_BAD_ALIGN;
     for (cuuint32_t i = 0; i + 1 < rank; ++i)
         if (strides[i] & 15) return GPT_ERR_BAD_ALIGN;
     EncodeTiledFn fn = encode_fn();
     if (!fn) return GPT_ERR_CUDA;
     const cuuint32_t estr[4] = {1, 1, 1, 1};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    CUresult r = fn(m, dt, rank, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? GPT_OK : GPT_ERR_CUDA;
 }
 }  // namespace
@@ -67,6 +75,15 @@ int make_tmap_bf16_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t
     const cuuint64_t strides[1] = {row_stride_bytes};
     const cuuint32_t box[2] = {box_inner, box_outer};
     return encode(m, base, 2, dims, strides, box);
+}
+
+int make_tmap_2d_sw64(CUtensorMap* m, const void* base, bool fp32, uint64_t inner, uint64_t outer,
+                      uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer) {
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {row_stride_bytes};
+    const cuuint32_t box[2] = {box_inner, box_outer};
+    return encode(m, base, 2, dims, strides, box,
+                  fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
 int make_tmap_bf16_4d(CUtensorMap* m, const void* base, const uint64_t dims[4], const uint64_t strides_bytes[3],
@@ -192,10 +209,13 @@ Plan plan_ws(const gpt_config_t* c, long long B, long long T) {
 int32_t* status_word(void* ws) { return static_cast<int32_t*>(ws); }
 
 int sync_and_read_status(void* ws, cudaStream_t s) {
-    if (cudaStreamSynchronize(s) != cudaSuccess) return GPT_ERR_CUDA;
+    int rc = cuda_status(cudaStreamSynchronize(s));
+    if (rc) return rc;
     int32_t st = 0;
-    if (cudaMemcpy(&st, ws, sizeof(st), cudaMemcpyDeviceToHost) != cudaSuccess) return GPT_ERR_CUDA;
-    if (cudaMemset(ws, 0, sizeof(st)) != cudaSuccess) return GPT_ERR_CUDA;
+    rc = cuda_status(cudaMemcpy(&st, ws, sizeof(st), cudaMemcpyDeviceToHost));
+    if (rc) return rc;
+    rc = cuda_status(cudaMemset(ws, 0, sizeof(st)));
+    if (rc) return rc;
     return st;
 }
 
@@ -320,6 +340,10 @@ GPT_API const char* gpt_status_string(int status) {
 }
 
 GPT_API int gpt_abi_version(void) { return GPT_ABI_VERSION; }
+
+GPT_API const char* gpt_last_cuda_error(void) {
+    return g_last_cuda_error == cudaSuccess ? "no error" : cudaGetErrorString(g_last_cuda_error);
+}
 
 GPT_API int gpt_validate_config(const gpt_config_t* cfg) { return validate(cfg); }
 

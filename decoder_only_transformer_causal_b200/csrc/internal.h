@@ -20,6 +20,9 @@ int cuda_status(cudaError_t e);
 // ---- TMA descriptors (cuTensorMapEncodeTiled through the runtime's driver entry point)
 int make_tmap_bf16_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
                       uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer);
+// 2-D map with 64-byte swizzle for epilogue staging tiles (box rows of 64 bytes); fp32 or bf16.
+int make_tmap_2d_sw64(CUtensorMap* m, const void* base, bool fp32, uint64_t inner, uint64_t outer,
+                      uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer);
 int make_tmap_bf16_4d(CUtensorMap* m, const void* base, const uint64_t dims[4],
                       const uint64_t strides_bytes[3], const uint32_t box[4]);
 

@@ -41,7 +41,10 @@ GELUS = {"erf": GPT_GELU_ERF, "tanh": GPT_GELU_TANH}
 class GPTError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__(f"{where}: {status_string(status)} (status {status})")
+        msg = f"{where}: {status_string(status)} (status {status})"
+        if status == GPT_ERR_CUDA:
+            msg += f": {LIB.gpt_last_cuda_error().decode()}"
+        super().__init__(msg)
 
 
 class gpt_config_t(ctypes.Structure):
@@ -59,6 +62,7 @@ def _load() -> ctypes.CDLL:
     sig = {
         "gpt_status_string": (ctypes.c_char_p, [I]),
         "gpt_abi_version": (I, []),
+        "gpt_last_cuda_error": (ctypes.c_char_p, []),
         "gpt_validate_config": (I, [CFG]),
         "gpt_weights_bytes": (Z, [CFG]),
         "gpt_weights_count": (I, [CFG]),
@@ -84,7 +88,7 @@ def _load() -> ctypes.CDLL:
 
 LIB = _load()
 
-EXPORTED = ("gpt_status_string", "gpt_abi_version", "gpt_validate_config", "gpt_weights_bytes",
+EXPORTED = ("gpt_status_string", "gpt_abi_version", "gpt_last_cuda_error", "gpt_validate_config", "gpt_weights_bytes",
             "gpt_weights_count", "gpt_weights_layout", "gpt_workspace_bytes", "gpt_check_status",
             "gpt_forward", "gpt_block", "gpt_attention", "gpt_embed", "gpt_layernorm", "gpt_linear",
             "gpt_lm_head_workspace_bytes", "gpt_lm_head_loss", "gpt_lm_head_loss_noalloc")

@@ -80,6 +80,10 @@ const char* gpt_status_string(int status);
 /* GPT_ABI_VERSION of the loaded library. */
 int gpt_abi_version(void);
 
+/* The CUDA runtime's message for the last failed CUDA call made by this library on the calling
+ * thread (the cause behind a GPT_ERR_CUDA), or "no error".  Static string, never NULL. */
+const char* gpt_last_cuda_error(void);
+
 /* Checks a configuration: positive sizes, C % n_head == 0, dtype and gelu in range,
  * and, for GPT_DTYPE_BF16, hs == 64 and C % 8 == 0 (the tensor-core kernels' layout).
  * Returns GPT_OK, GPT_ERR_NULL, GPT_ERR_BAD_SHAPE or GPT_ERR_UNSUPPORTED. */
