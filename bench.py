@@ -314,6 +314,7 @@ def main():
     dev = torch.device("cuda", local)
 
     from decoder_only_transformer_causal_b200 import GPT, GPTConfig, native
+    from decoder_only_transformer_causal_b200.data_parallel import allreduce_loss_terms
 
     w = seeded.WORKLOADS[WORKLOAD]
     cfg = GPTConfig.from_dict(w.model_dict())
@@ -330,7 +331,7 @@ def main():
         native.forward(cfg, model.weights, idx, tgt, ws, logits=logits, loss=loss, loss_sum_count=sc,
                        stream=stream)
         if dist is not None:
-            dist.all_reduce(sc)          # global {sum of row losses, count}
+            allreduce_loss_terms(sc)     # global {sum of row losses, counted rows}
 
     # correctness guard before timing: the status word must be clean
     native.forward(cfg, model.weights, idx, tgt, ws, logits=logits, loss=loss, sync_check=True)

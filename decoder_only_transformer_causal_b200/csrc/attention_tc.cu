@@ -52,8 +52,8 @@ int launch_attention_bf16(const AttnLayout& L, int B, int nh, int T, int32_t* st
     const long long n_qt = (T + attn::BQ - 1) / attn::BQ;
     const long long blocks = n_qt * B * nh;
     if (blocks > 0x7fffffffLL) return GPT_ERR_UNSUPPORTED;
-    attn::attention_fwd_tc<<<static_cast<unsigned>(blocks), attn::THREADS, attn::SMEM_BYTES, s>>>(tq, tk, tv, p);
-    return cuda_status(cudaGetLastError());
+    return launch_overlapped(attn::attention_fwd_tc, dim3(static_cast<unsigned>(blocks)), dim3(attn::THREADS),
+                             attn::SMEM_BYTES, s, tq, tk, tv, p);
 }
 
 }  // namespace gpt

@@ -15,7 +15,10 @@
 //   warps 2-5   softmax, one query row per thread: load the S row from TMEM, mask the
 //               diagonal tile, update the running maximum / sum, write P (bf16) to TMEM,
 //               rescale O in TMEM when the maximum moved by more than 2^8, and finally
-//               write y = O / l.
+//               write y = O / l.  Packed f32x2 arithmetic and 3-input maxima cut the issue
+//               count; on the diagonal tile the 32-column chunks right of a warp's last row are
+//               fully masked and skip the exponential.  The exponential (MUFU ex2, 16 per clock
+//               per SM) is the unit this kernel is bound by at head size 64.
 // TMEM columns: S [0,128), P [128,192) (bf16 pairs), O [192,256).  256 columns and 80 KB of
 // shared memory let two CTAs share an SM, so one CTA's softmax overlaps the other's MMAs.
 //
@@ -40,6 +43,13 @@ constexpr uint32_t COL_S = 0, COL_P = 128, COL_O = 192;
 // The running maximum is only moved (forcing an O rescale) when it grows by more than this
 // many powers of two; P values then stay below 2^8, harmless in fp32 and bf16.
 constexpr float kRescaleThreshold = 8.0f;
+
+
+GPT_DEVINL uint64_t f2_pack(float lo, float hi) { uint64_t r; asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi)); return r; }
+GPT_DEVINL void f2_unpack(uint64_t v, float& lo, float& hi) { asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v)); }
+GPT_DEVINL uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) { uint64_t d; asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c)); return d; }
+GPT_DEVINL uint64_t f2_add(uint64_t a, uint64_t b) { uint64_t d; asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b)); return d; }
+GPT_DEVINL float max3(float a, float b, float c) { float d; asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c)); return d; }
 
 struct Params {
     int B, nh, T;
@@ -103,6 +113,9 @@ __global__ void __launch_bounds__(THREADS, 2)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // The set-up above overlapped the previous kernel; its outputs are read from here on.
+    griddep_launch_dependents();
+    griddep_wait();
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
@@ -198,7 +211,7 @@ __global__ void __launch_bounds__(THREADS, 2)
             }
             tc_fence_after();
             // S row -> registers (raw scores; the 1/sqrt(hs) * log2(e) scale is folded into the
-            // exponent below).  8 independent partial maxima / sums keep the dependency chains short.
+            // exponent below).  Independent partial maxima / sums keep the dependency chains short.
             float s[BKV];
 #pragma unroll
             for (int c = 0; c < BKV; c += 64) {
@@ -215,30 +228,45 @@ __global__ void __launch_bounds__(THREADS, 2)
                 for (int c = 0; c < BKV; ++c)
                     if (c > r) s[c] = -INFINITY;
             }
-            float m8[8];
+            float m4[4] = {s[0], s[1], s[2], s[3]};
 #pragma unroll
-            for (int e = 0; e < 8; ++e) m8[e] = s[e];
-#pragma unroll
-            for (int c = 8; c < BKV; ++c) m8[c & 7] = fmaxf(m8[c & 7], s[c]);
-            const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                                   fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * p.scale_log2;
+            for (int cc = 4; cc < BKV; cc += 8) {
+                m4[0] = max3(m4[0], s[cc], s[cc + 1]);
+                m4[1] = max3(m4[1], s[cc + 2], s[cc + 3]);
+                if (cc + 4 < BKV) {
+                    m4[2] = max3(m4[2], s[cc + 4], s[cc + 5]);
+                    m4[3] = max3(m4[3], s[cc + 6], s[cc + 7]);
+                }
+            }
+            const float mx = max3(m4[0], m4[1], fmaxf(m4[2], m4[3])) * p.scale_log2;
             float alpha = 1.f;
             if (mx > m_used + kRescaleThreshold || m_used == -INFINITY) {
-                alpha = exp2_approx(m_used - mx);  // 0 on the first tile
+                alpha = exp2_approx(m_used - mx);
                 m_used = mx;
             }
-            const float neg_m = -m_used;
-            float r8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            const bool diag = (j == n_kv - 1);
+            const uint64_t SC = f2_pack(p.scale_log2, p.scale_log2), NM = f2_pack(-m_used, -m_used);
+            uint64_t acc4[4] = {0, 0, 0, 0};
             uint32_t pk0[32], pk1[32];
+            // On the diagonal tile, 32-column chunks to the right of this warp's last row are
+            // masked for every lane: P is 0 there and no exponential is evaluated.
+            const int live_cols = diag ? (quarter + 1) * 32 : BKV;  // warp-uniform
 #pragma unroll
             for (int c = 0; c < BKV; c += 2) {
-                const float p0 = exp2_approx(fmaf(s[c], p.scale_log2, neg_m));
-                const float p1 = exp2_approx(fmaf(s[c + 1], p.scale_log2, neg_m));
-                r8[(c >> 1) & 7] += p0 + p1;
+                float p0 = 0.f, p1 = 0.f;
+                if (c < live_cols) {
+                    float x0, x1;
+                    f2_unpack(f2_fma(f2_pack(s[c], s[c + 1]), SC, NM), x0, x1);
+                    p0 = exp2_approx(x0);
+                    p1 = exp2_approx(x1);
+                    acc4[(c >> 1) & 3] = f2_add(acc4[(c >> 1) & 3], f2_pack(p0, p1));
+                }
                 if (c < 64) pk0[c / 2] = pack_bf16x2(p0, p1);
                 else pk1[(c - 64) / 2] = pack_bf16x2(p0, p1);
             }
-            const float rs = ((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7]));
+            float a0, a1, b0, b1, c0, c1, d0, d1;
+            f2_unpack(acc4[0], a0, a1); f2_unpack(acc4[1], b0, b1); f2_unpack(acc4[2], c0, c1); f2_unpack(acc4[3], d0, d1);
+            const float rs = ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
             l = l * alpha + rs;
             // P_j may overwrite P_{j-1} and O may be rescaled only after O += P_{j-1} V_{j-1}.
             if (j > 0) {

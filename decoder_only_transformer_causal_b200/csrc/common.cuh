@@ -267,6 +267,17 @@ GPT_DEVINL void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
         : "memory");
 }
 
+// 16 columns of this thread's lane; waits for completion.
+GPT_DEVINL void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};\n\t"
+        "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+
 GPT_DEVINL float exp2_approx(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -277,6 +288,14 @@ GPT_DEVINL uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
 }
+
+// Programmatic dependent launch.  A kernel launched with programmatic stream serialisation may
+// start before its predecessor in the stream has finished: it must call griddep_wait() before
+// it reads or writes memory the predecessor touches (the wait returns once the predecessor has
+// completed and its writes are visible).  griddep_launch_dependents() lets the successor start
+// as soon as every CTA of this grid has started or finished.
+GPT_DEVINL void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+GPT_DEVINL void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 // Records a device-side status (first writer wins).
 GPT_DEVINL void set_status(int32_t* status, int32_t code) {

@@ -21,8 +21,7 @@ int launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& 
     }
     const int tiles = ((p.M + gemm::BM - 1) / gemm::BM) * ((p.N + kBN - 1) / kBN);
     const int grid = tiles < num_sms() ? tiles : num_sms();
-    kern<<<grid, L::THREADS, L::SMEM_BYTES, s>>>(ta, tb, tc, p);
-    return cuda_status(cudaGetLastError());
+    return launch_overlapped(kern, dim3(grid), dim3(L::THREADS), L::SMEM_BYTES, s, ta, tb, tc, p);
 }
 
 }  // namespace

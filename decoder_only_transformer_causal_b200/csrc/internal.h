@@ -17,6 +17,25 @@ typedef __nv_bfloat16 bf16;
 int num_sms();
 int cuda_status(cudaError_t e);
 
+// Launches `kern` so that it may overlap the tail of the previous kernel in the stream
+// (programmatic stream serialisation); every kernel launched this way calls griddep_wait()
+// before touching memory its predecessor uses.
+template <typename... KArgs, typename... Args>
+int launch_overlapped(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                      Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cuda_status(cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...));
+}
+
 // ---- TMA descriptors (cuTensorMapEncodeTiled through the runtime's driver entry point)
 int make_tmap_bf16_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
                       uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer);

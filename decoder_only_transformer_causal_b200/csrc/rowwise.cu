@@ -42,6 +42,8 @@ template <typename Tw>
 __global__ void embed_kernel(const Tw* __restrict__ wte, const Tw* __restrict__ wpe,
                              const int64_t* __restrict__ idx, float* __restrict__ x, int T, int C,
                              int V, long long total4, int32_t* status) {
+    griddep_launch_dependents();
+    griddep_wait();
     const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (i >= total4) return;
     const int c4 = C >> 2;
@@ -65,6 +67,8 @@ constexpr int kLnMaxVec = 16;  // float4 per lane -> C <= 2048
 template <typename To>
 __global__ void layernorm_kernel(const float* __restrict__ x, const To* __restrict__ w,
                                  const To* __restrict__ bias, To* __restrict__ out, int rows, int C) {
+    griddep_launch_dependents();
+    griddep_wait();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int row = blockIdx.x * kWarpsPerBlock + warp;
     if (row >= rows) return;
@@ -115,6 +119,8 @@ __global__ void ce_rows_from_parts_kernel(const float2* __restrict__ part, int n
                                           const float* __restrict__ tlogit,
                                           const int64_t* __restrict__ targets, int rows, int V,
                                           float* __restrict__ row_loss, int32_t* status) {
+    griddep_launch_dependents();
+    griddep_wait();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int row = blockIdx.x * kWarpsPerBlock + warp;
     if (row >= rows) return;
@@ -143,6 +149,8 @@ __global__ void ce_rows_from_parts_kernel(const float2* __restrict__ part, int n
 __global__ void ce_rows_from_logits_kernel(const float* __restrict__ logits,
                                            const int64_t* __restrict__ targets, int rows, int V,
                                            float* __restrict__ row_loss, int32_t* status) {
+    griddep_launch_dependents();
+    griddep_wait();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int row = blockIdx.x * kWarpsPerBlock + warp;
     if (row >= rows) return;
@@ -168,6 +176,8 @@ constexpr int kFinThreads = 1024;
 __global__ void __launch_bounds__(kFinThreads)
     loss_finalize_kernel(const float* __restrict__ row_loss, const int64_t* __restrict__ targets,
                          int rows, int V, float* loss, double* sum_count) {
+    griddep_launch_dependents();
+    griddep_wait();
     __shared__ double s_sum[kFinThreads];
     __shared__ double s_cnt[kFinThreads];
     double a = 0.0, n = 0.0;
@@ -207,14 +217,10 @@ int launch_embed(const void* wte, const void* wpe, const int64_t* idx, float* x,
     const int threads = 256;
     const unsigned blocks = static_cast<unsigned>((total4 + threads - 1) / threads);
     if (dtype == GPT_DTYPE_BF16)
-        embed_kernel<bf16><<<blocks, threads, 0, s>>>(static_cast<const bf16*>(wte),
-                                                      static_cast<const bf16*>(wpe), idx, x, T, C, V,
-                                                      total4, status);
-    else
-        embed_kernel<float><<<blocks, threads, 0, s>>>(static_cast<const float*>(wte),
-                                                       static_cast<const float*>(wpe), idx, x, T, C,
-                                                       V, total4, status);
-    return cuda_status(cudaGetLastError());
+        return launch_overlapped(embed_kernel<bf16>, dim3(blocks), dim3(threads), 0, s, static_cast<const bf16*>(wte),
+                                 static_cast<const bf16*>(wpe), idx, x, T, C, V, total4, status);
+    return launch_overlapped(embed_kernel<float>, dim3(blocks), dim3(threads), 0, s, static_cast<const float*>(wte),
+                             static_cast<const float*>(wpe), idx, x, T, C, V, total4, status);
 }
 
 int launch_layernorm(const float* x, const void* w, const void* b, void* out, int rows, int C,
@@ -223,12 +229,12 @@ int launch_layernorm(const float* x, const void* w, const void* b, void* out, in
     if (rows == 0) return GPT_OK;
     const unsigned blocks = (rows + kWarpsPerBlock - 1) / kWarpsPerBlock;
     if (dtype == GPT_DTYPE_BF16)
-        layernorm_kernel<bf16><<<blocks, 32 * kWarpsPerBlock, 0, s>>>(
-            x, static_cast<const bf16*>(w), static_cast<const bf16*>(b), static_cast<bf16*>(out), rows, C);
-    else
-        layernorm_kernel<float><<<blocks, 32 * kWarpsPerBlock, 0, s>>>(
-            x, static_cast<const float*>(w), static_cast<const float*>(b), static_cast<float*>(out), rows, C);
-    return cuda_status(cudaGetLastError());
+        return launch_overlapped(layernorm_kernel<bf16>, dim3(blocks), dim3(32 * kWarpsPerBlock), 0, s, x,
+                                 static_cast<const bf16*>(w), static_cast<const bf16*>(b), static_cast<bf16*>(out),
+                                 rows, C);
+    return launch_overlapped(layernorm_kernel<float>, dim3(blocks), dim3(32 * kWarpsPerBlock), 0, s, x,
+                             static_cast<const float*>(w), static_cast<const float*>(b), static_cast<float*>(out),
+                             rows, C);
 }
 
 int launch_ce_rows_from_parts(const float2* part, int n_part, const float* tlogit,
@@ -236,24 +242,22 @@ int launch_ce_rows_from_parts(const float2* part, int n_part, const float* tlogi
                               int32_t* status, cudaStream_t s) {
     if (rows == 0) return GPT_OK;
     const unsigned blocks = (rows + kWarpsPerBlock - 1) / kWarpsPerBlock;
-    ce_rows_from_parts_kernel<<<blocks, 32 * kWarpsPerBlock, 0, s>>>(part, n_part, tlogit, targets,
-                                                                     rows, V, row_loss, status);
-    return cuda_status(cudaGetLastError());
+    return launch_overlapped(ce_rows_from_parts_kernel, dim3(blocks), dim3(32 * kWarpsPerBlock), 0, s, part, n_part,
+                             tlogit, targets, rows, V, row_loss, status);
 }
 
 int launch_ce_rows_from_logits(const float* logits, const int64_t* targets, int rows, int V,
                                float* row_loss, int32_t* status, cudaStream_t s) {
     if (rows == 0) return GPT_OK;
     const unsigned blocks = (rows + kWarpsPerBlock - 1) / kWarpsPerBlock;
-    ce_rows_from_logits_kernel<<<blocks, 32 * kWarpsPerBlock, 0, s>>>(logits, targets, rows, V,
-                                                                      row_loss, status);
-    return cuda_status(cudaGetLastError());
+    return launch_overlapped(ce_rows_from_logits_kernel, dim3(blocks), dim3(32 * kWarpsPerBlock), 0, s, logits,
+                             targets, rows, V, row_loss, status);
 }
 
 int launch_loss_finalize(const float* row_loss, const int64_t* targets, int rows, int V, float* loss,
                          double* sum_count, cudaStream_t s) {
-    loss_finalize_kernel<<<1, kFinThreads, 0, s>>>(row_loss, targets, rows, V, loss, sum_count);
-    return cuda_status(cudaGetLastError());
+    return launch_overlapped(loss_finalize_kernel, dim3(1), dim3(kFinThreads), 0, s, row_loss, targets, rows, V, loss,
+                             sum_count);
 }
 
 }  // namespace gpt

@@ -1,0 +1,56 @@
+"""Batch-sharded forward over several GPUs (one process per GPU).
+
+Sequences of a batch are independent through the whole forward pass ("nanoGPT 全局流程图", §3.2:
+every sequence goes through the same Blocks on its own), so each rank runs gpt_forward on its
+own contiguous slice of the batch with replicated weights; no activation crosses a device.  The
+only exchange is the loss: F.cross_entropy averages over every counted position of the batch
+(targets != -1), so the ranks add their {sum of row losses, number of counted rows} and divide
+the totals — not the mean of per-rank means, which would weight ranks with many ignored targets
+wrongly.  With NCCL over NVLink that is one 16-byte all-reduce per step.
+"""
+from __future__ import annotations
+
+import math
+
+import torch
+import torch.distributed as dist
+
+
+def shard_range(batch: int, world: int, rank: int) -> tuple[int, int]:
+    """[start, stop) of the sequences rank `rank` owns: contiguous, sizes differing by at most
+    one (the first batch % world ranks take one more)."""
+    if world < 1 or not 0 <= rank < world or batch < 0:
+        raise ValueError((batch, world, rank))
+    base, extra = divmod(batch, world)
+    start = rank * base + min(rank, extra)
+    return start, start + base + (1 if rank < extra else 0)
+
+
+def allreduce_loss_terms(loss_sum_count: torch.Tensor, group=None) -> torch.Tensor:
+    """Sums the fp64 {sum of row losses, counted rows} pair over the ranks, in place."""
+    if loss_sum_count.dtype != torch.float64 or loss_sum_count.numel() != 2:
+        raise ValueError("loss_sum_count must be a float64 tensor of 2 elements")
+    dist.all_reduce(loss_sum_count, op=dist.ReduceOp.SUM, group=group)
+    return loss_sum_count
+
+
+def global_loss(loss_sum_count: torch.Tensor) -> float:
+    """Mean row loss of the whole batch from the reduced pair (NaN when nothing is counted)."""
+    s, n = (float(v) for v in loss_sum_count.detach().cpu())
+    return s / n if n > 0 else math.nan
+
+
+def forward_sharded(model, idx: torch.Tensor, targets: torch.Tensor, group=None):
+    """Runs this rank's slice of (idx, targets) [B, T] through `model` (a GPT instance on this
+    rank's device) and returns (local logits, global loss).  idx / targets may be the full
+    batch on any device; only this rank's rows are copied to the model's device."""
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    a, b = shard_range(idx.shape[0], world, rank)
+    dev = model.device
+    sc = torch.zeros(2, dtype=torch.float64, device=dev)
+    logits = None
+    if b > a:
+        logits, _ = model(idx[a:b].to(dev), targets[a:b].to(dev), loss_sum_count=sc)
+    allreduce_loss_terms(sc, group)
+    return logits, global_loss(sc)

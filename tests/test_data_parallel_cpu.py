@@ -1,0 +1,77 @@
+"""Host logic of the batch-sharded forward on CPU ranks (gloo, world size 2 and 3).
+
+Each rank computes its shard's row losses with the fp64 oracle (the GPU kernels are not needed
+to check the sharding and the loss combination) and the ranks combine them with the same
+all-reduce the GPU path uses.  The combined loss must equal the oracle's loss of the whole
+batch, including when ignored targets (-1) are spread unevenly over the ranks."""
+import math
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import oracle
+import seeded
+from decoder_only_transformer_causal_b200.data_parallel import (
+    allreduce_loss_terms, global_loss, shard_range)
+
+TINY = seeded.WORKLOADS["tiny"].model_dict()
+
+
+def test_shard_range_partitions():
+    for batch in range(0, 13):
+        for world in range(1, 6):
+            spans = [shard_range(batch, world, r) for r in range(world)]
+            assert spans[0][0] == 0 and spans[-1][1] == batch
+            assert all(spans[i][1] == spans[i + 1][0] for i in range(world - 1))
+            sizes = [b - a for a, b in spans]
+            assert max(sizes) - min(sizes) <= 1
+    with pytest.raises(ValueError):
+        shard_range(4, 2, 2)
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _rank_main(rank, world, port, batch, ignore_frac, out_path):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        W = seeded.to_f64(seeded.make_weights(TINY, stress=True))
+        idx, tgt = seeded.make_tokens(batch, 32, TINY["vocab_size"], ignore_frac=ignore_frac)
+        # uneven ignores: rank 0's slice loses every target of its first sequence
+        tgt[0] = -1
+        a, b = shard_range(batch, world, rank)
+        sc = torch.zeros(2, dtype=torch.float64)
+        if b > a:
+            out = oracle.forward(W, TINY, idx[a:b].numpy(), tgt[a:b].numpy(), keep_logits=False)
+            sc[0] = float(out["row_loss"].sum())
+            sc[1] = float(out["count"])
+        allreduce_loss_terms(sc)
+        if rank == 0:
+            full = oracle.forward(W, TINY, idx.numpy(), tgt.numpy(), keep_logits=False)
+            np.save(out_path, np.array([global_loss(sc), full["loss"], sc[1].item(), full["count"]]))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,batch", [(2, 5), (3, 4), (2, 1)])
+def test_sharded_loss_matches_full_batch(tmp_path, world, batch):
+    out = tmp_path / "res.npy"
+    mp.spawn(_rank_main, args=(world, _free_port(), batch, 0.2, str(out)), nprocs=world, join=True)
+    got, want, n_got, n_want = np.load(out)
+    assert n_got == n_want
+    if math.isnan(want):
+        assert math.isnan(got)
+    else:
+        assert abs(got - want) <= 1e-12 * abs(want)
