@@ -66,3 +66,22 @@ class GPT:
         h_loss.copy_(loss, non_blocking=True)
         torch.cuda.current_stream(self.device).synchronize()
         return float(h_loss)
+
+    def generate(self, idx: torch.Tensor, max_new_tokens: int, temperature: float = 1.0,
+                 top_k: int | None = None, uniforms: torch.Tensor | None = None,
+                 generator: torch.Generator | None = None, step_logits: torch.Tensor | None = None):
+        """GPT.generate of the pages ("nanoGPT 全局流程图", 第五阶段) on device tensors: returns
+        int64 [B, T0 + max_new_tokens].  The draw of each step uses one uniform per sequence:
+        ``uniforms`` fp32 [max_new_tokens, B] in [0, 1) if given, else drawn here with torch
+        (from ``generator`` if given); the library itself generates no random numbers."""
+        B, T0 = idx.shape
+        if uniforms is None:
+            uniforms = torch.rand((max_new_tokens, B), generator=generator, device=self.device,
+                                  dtype=torch.float32)
+        key = ("gen", B)
+        if key not in self._host:
+            self._host[key] = native.alloc_kv_cache(self.cfg, B, self.device)
+        ws = native.alloc_workspace(native.generate_workspace_bytes(self.cfg, B, T0, max_new_tokens), self.device)
+        return native.generate(self.cfg, self.weights, idx, max_new_tokens, uniforms, temperature, top_k,
+                               kv_cache=self._host[key], workspace=ws, step_logits=step_logits)
+

@@ -226,8 +226,10 @@ int sync_and_read_status(void* ws, cudaStream_t s) {
     } while (0)
 
 // One pre-LN Block ("nanoGPT 全局流程图", §2.5): x += attn(ln_1(x)); x += mlp(ln_2(x)).
+// With kv_layer set, the layer's k and v of positions [0, T) are also copied into that cache
+// ([B, block_size, 2C]) for incremental decoding.
 int run_block(const gpt_config_t* c, const Weights& W, int l, float* x, int B, int T, uint8_t* ws,
-              const Plan& P, cudaStream_t s) {
+              const Plan& P, cudaStream_t s, void* kv_layer = nullptr) {
     const int C = c->n_embd, nh = c->n_head, hs = C / nh;
     const int N = B * T;
     int32_t* status = status_word(ws);
@@ -242,6 +244,7 @@ int run_block(const gpt_config_t* c, const Weights& W, int l, float* x, int B, i
         GPT_TRY(launch_gemm_bf16(ub, C, static_cast<const bf16*>(W.layer(l, W_ATTN_W)), C,
                                  static_cast<const bf16*>(W.bias(l, W_ATTN_B)), qkv, 3LL * C, N, 3 * C, C,
                                  GPT_EPI_STORE, c->gelu, nullptr, status, s));
+        if (kv_layer) GPT_TRY(launch_kv_store(qkv, kv_layer, B, T, C, 2, c->block_size, s));
         AttnLayout L{};
         L.q = qkvb;
         L.k = qkvb + C;
@@ -270,6 +273,7 @@ int run_block(const gpt_config_t* c, const Weights& W, int l, float* x, int B, i
         GPT_TRY(launch_linear_f32(uf, C, static_cast<const float*>(W.layer(l, W_ATTN_W)),
                                   static_cast<const float*>(W.bias(l, W_ATTN_B)), qkvf, 3LL * C, N, 3 * C, C,
                                   GPT_EPI_STORE, c->gelu, s));
+        if (kv_layer) GPT_TRY(launch_kv_store(qkv, kv_layer, B, T, C, 4, c->block_size, s));
         AttnLayoutF32 L{};
         L.q = qkvf;
         L.k = qkvf + C;
@@ -318,6 +322,122 @@ int check_common(const gpt_config_t* c, const void* weights, int B, int T, void*
     if (!aligned(weights, 256) || !aligned(ws, 256)) return GPT_ERR_BAD_ALIGN;
     *P = plan_ws(c, B, T);
     if (ws_bytes < P->total) return GPT_ERR_WS_TOO_SMALL;
+    return GPT_OK;
+}
+
+// ------------------------------------------------------------------ incremental decoding
+// Workspace of the decoding entry points: the forward plan for a prefill of up to T_pref
+// positions (its buffers also hold the one-row-per-sequence activations of a decode step),
+// then the split-attention partials, fp32 logits [B, V] and a token window [B, block_size].
+// The control block keeps the status word at byte 0 and the decode position at byte 4.
+struct DecodePlan {
+    Plan P;
+    size_t part, logits, window, total;
+};
+
+DecodePlan plan_decode(const gpt_config_t* c, int B, int T_pref) {
+    DecodePlan D;
+    D.P = plan_ws(c, B, T_pref);
+    size_t off = D.P.total;
+    const int hs = c->n_embd / c->n_head;
+    D.part = off; off += a256(decode_attn_part_floats(B, c->n_head, hs, c->block_size) * 4);
+    D.logits = off; off += a256(static_cast<size_t>(B) * c->vocab_size * 4);
+    D.window = off; off += a256(static_cast<size_t>(B) * c->block_size * 8);
+    D.total = off;
+    return D;
+}
+
+int* pos_word(void* ws) { return reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + 4); }
+
+size_t kv_layer_bytes(const gpt_config_t* c, int B) {
+    return static_cast<size_t>(B) * c->block_size * 2 * c->n_embd * elem_size(c);
+}
+
+int validate_decode(const gpt_config_t* c) {
+    GPT_TRY(validate(c));
+    const int hs = c->n_embd / c->n_head;
+    if ((c->n_embd % 8) || (hs % 8) || hs > 128) return GPT_ERR_UNSUPPORTED;
+    return GPT_OK;
+}
+
+int check_decode(const gpt_config_t* c, const void* weights, int B, const void* kv, void* ws, size_t ws_bytes,
+                 int T_pref, DecodePlan* D) {
+    GPT_TRY(validate_decode(c));
+    if (!weights || !kv || !ws) return GPT_ERR_NULL;
+    if (B < 1 || T_pref < 1 || T_pref > c->block_size) return GPT_ERR_BAD_SHAPE;
+    if (static_cast<long long>(B) * c->block_size > 0x7fffffffLL / 4 / c->n_embd) return GPT_ERR_UNSUPPORTED;
+    if (B > 65535 / c->n_head) return GPT_ERR_UNSUPPORTED;
+    if (!aligned(weights, 256) || !aligned(ws, 256) || !aligned(kv, 16)) return GPT_ERR_BAD_ALIGN;
+    *D = plan_decode(c, B, T_pref);
+    if (ws_bytes < D->total) return GPT_ERR_WS_TOO_SMALL;
+    return GPT_OK;
+}
+
+// Forward over idx [B, T] (contiguous) that fills every layer's cache at positions [0, T),
+// then logits fp32 [B, V] of position T-1 at row stride ldl, and sets the decode position to T.
+int prefill_impl(const gpt_config_t* c, const Weights& W, const int64_t* idx, int B, int T, uint8_t* kv,
+                 float* logits, long long ldl, uint8_t* ws, const DecodePlan& D, cudaStream_t s) {
+    const int C = c->n_embd, V = c->vocab_size, N = B * T;
+    const Plan& P = D.P;
+    int32_t* status = status_word(ws);
+    float* x = reinterpret_cast<float*>(ws + P.x);
+    void* u = ws + P.u;
+    GPT_TRY(launch_embed(W.wte(), W.wpe(), idx, x, B, T, C, V, c->dtype, status, s));
+    for (int l = 0; l < c->n_layer; ++l)
+        GPT_TRY(run_block(c, W, l, x, B, T, ws, P, s, kv + kv_layer_bytes(c, B) * l));
+    GPT_TRY(launch_layernorm(x, W.lnf_w(), W.lnf_b(), u, N, C, c->dtype, s));
+    const uint8_t* ulast = static_cast<const uint8_t*>(u) + static_cast<size_t>(T - 1) * C * elem_size(c);
+    GPT_TRY(launch_gemv(3, c->dtype, ulast, static_cast<long long>(T) * C, W.wte(), nullptr, logits, ldl, B, V, C,
+                        c->gelu == GPT_GELU_TANH, nullptr, nullptr, C, c->block_size, s));
+    return launch_set_pos(pos_word(ws), T, 0, s);
+}
+
+// One token per sequence (tok[b * ld_tok]) at the decode position p: every layer appends its
+// k, v at p and attends over positions [0, p]; logits fp32 [B, V] at row stride ldl; p += 1.
+int decode_step_impl(const gpt_config_t* c, const Weights& W, const int64_t* tok, long long ld_tok, int B,
+                     uint8_t* kv, float* logits, long long ldl, uint8_t* ws, const DecodePlan& D, cudaStream_t s) {
+    const int C = c->n_embd, V = c->vocab_size, nh = c->n_head, hs = C / nh, bs = c->block_size;
+    const int dt = c->dtype, gt = c->gelu == GPT_GELU_TANH;
+    const Plan& P = D.P;
+    int32_t* status = status_word(ws);
+    const int* pos = pos_word(ws);
+    float* x = reinterpret_cast<float*>(ws + P.x);
+    void* u = ws + P.u;
+    void* q = ws + P.qkv;
+    void* y = ws + P.y;
+    void* h = ws + P.h;
+    float* part = reinterpret_cast<float*>(ws + D.part);
+    GPT_TRY(launch_embed_pos(W.wte(), W.wpe(), tok, ld_tok, pos, x, B, C, V, bs, dt, status, s));
+    for (int l = 0; l < c->n_layer; ++l) {
+        uint8_t* kvl = kv + kv_layer_bytes(c, B) * l;
+        GPT_TRY(launch_layernorm(x, W.layer(l, W_LN1_W), W.bias(l, W_LN1_B), u, B, C, dt, s));
+        GPT_TRY(launch_gemv(4, dt, u, C, W.layer(l, W_ATTN_W), W.bias(l, W_ATTN_B), q, C, B, 3 * C, C, gt, kvl, pos,
+                            C, bs, s));
+        GPT_TRY(launch_decode_attention(dt, q, kvl, pos, part, y, B, nh, hs, bs, s));
+        GPT_TRY(launch_gemv(2, dt, y, C, W.layer(l, W_PROJ_W), W.bias(l, W_PROJ_B), x, C, B, C, C, gt, nullptr,
+                            nullptr, C, bs, s));
+        GPT_TRY(launch_layernorm(x, W.layer(l, W_LN2_W), W.bias(l, W_LN2_B), u, B, C, dt, s));
+        GPT_TRY(launch_gemv(1, dt, u, C, W.layer(l, W_FC_W), W.bias(l, W_FC_B), h, 4LL * C, B, 4 * C, C, gt,
+                            nullptr, nullptr, C, bs, s));
+        GPT_TRY(launch_gemv(2, dt, h, 4LL * C, W.layer(l, W_FC2_W), W.bias(l, W_FC2_B), x, C, B, C, 4 * C, gt,
+                            nullptr, nullptr, C, bs, s));
+    }
+    GPT_TRY(launch_layernorm(x, W.lnf_w(), W.lnf_b(), u, B, C, dt, s));
+    GPT_TRY(launch_gemv(3, dt, u, C, W.wte(), nullptr, logits, ldl, B, V, C, gt, nullptr, nullptr, C, bs, s));
+    return launch_set_pos(pos_word(ws), 1, 1, s);
+}
+
+// The widest prefill gpt_generate runs: the prompt (cropped to the window), or a full window
+// once the sequence outgrows it.
+int generate_prefill_len(const gpt_config_t* c, int T0, int max_new_tokens) {
+    const long long longest = static_cast<long long>(T0) + (max_new_tokens > 0 ? max_new_tokens - 1 : 0);
+    return longest > c->block_size ? c->block_size : T0;
+}
+
+int check_sample_args(int B, int V, float temperature, const float* logits, const float* u, const int64_t* out) {
+    if (!logits || !u || !out) return GPT_ERR_NULL;
+    if (B < 1 || V < 1) return GPT_ERR_BAD_SHAPE;
+    if (!(temperature > 0.f) || !isfinite(temperature)) return GPT_ERR_BAD_SHAPE;
     return GPT_OK;
 }
 
@@ -537,6 +657,103 @@ GPT_API int gpt_lm_head_loss(const void* u, const void* wte, const int64_t* targ
         return GPT_ERR_BAD_SHAPE;
     }
     GPT_TRY(launch_loss_finalize(rl, targets, rows, V, loss, loss_sum_count, s));
+    if (flags & GPT_FLAG_SYNC_CHECK) return sync_and_read_status(ws, s);
+    return GPT_OK;
+}
+
+// ------------------------------------------------------------------ generation (decode.cu)
+GPT_API size_t gpt_kv_cache_bytes(const gpt_config_t* cfg, int B) {
+    if (validate_decode(cfg) != GPT_OK || B < 1) return 0;
+    return kv_layer_bytes(cfg, B) * cfg->n_layer;
+}
+
+GPT_API size_t gpt_decode_workspace_bytes(const gpt_config_t* cfg, int B, int T_prefill) {
+    if (validate_decode(cfg) != GPT_OK || B < 1 || T_prefill < 1 || T_prefill > cfg->block_size) return 0;
+    return plan_decode(cfg, B, T_prefill).total;
+}
+
+GPT_API size_t gpt_generate_workspace_bytes(const gpt_config_t* cfg, int B, int T0, int max_new_tokens) {
+    if (validate_decode(cfg) != GPT_OK || B < 1 || T0 < 1 || max_new_tokens < 0) return 0;
+    return plan_decode(cfg, B, generate_prefill_len(cfg, T0, max_new_tokens)).total;
+}
+
+GPT_API int gpt_prefill(const gpt_config_t* cfg, const void* weights, const int64_t* idx, int B, int T,
+                        void* kv_cache, float* logits, void* workspace, size_t workspace_bytes, void* stream,
+                        int flags) {
+    DecodePlan D;
+    GPT_TRY(check_decode(cfg, weights, B, kv_cache, workspace, workspace_bytes, T, &D));
+    if (!idx || !logits) return GPT_ERR_NULL;
+    if (!aligned(logits, 16)) return GPT_ERR_BAD_ALIGN;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    Weights W;
+    fill_weights(W, cfg, weights);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    GPT_TRY(cuda_status(cudaMemsetAsync(status_word(ws), 0, sizeof(int32_t), s)));
+    GPT_TRY(prefill_impl(cfg, W, idx, B, T, static_cast<uint8_t*>(kv_cache), logits, cfg->vocab_size, ws, D, s));
+    if (flags & GPT_FLAG_SYNC_CHECK) return sync_and_read_status(ws, s);
+    return GPT_OK;
+}
+
+GPT_API int gpt_decode_step(const gpt_config_t* cfg, const void* weights, const int64_t* tok, long long ld_tok, int B,
+                            void* kv_cache, float* logits, void* workspace, size_t workspace_bytes, void* stream,
+                            int flags) {
+    DecodePlan D;
+    GPT_TRY(check_decode(cfg, weights, B, kv_cache, workspace, workspace_bytes, 1, &D));
+    if (!tok || !logits) return GPT_ERR_NULL;
+    if (!aligned(logits, 16)) return GPT_ERR_BAD_ALIGN;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    Weights W;
+    fill_weights(W, cfg, weights);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    GPT_TRY(decode_step_impl(cfg, W, tok, ld_tok, B, static_cast<uint8_t*>(kv_cache), logits, cfg->vocab_size, ws,
+                             D, s));
+    if (flags & GPT_FLAG_SYNC_CHECK) return sync_and_read_status(ws, s);
+    return GPT_OK;
+}
+
+GPT_API int gpt_sample(const float* logits, int B, int V, float temperature, int top_k, const float* u, int64_t* out,
+                       long long ld_out, void* stream) {
+    GPT_TRY(check_sample_args(B, V, temperature, logits, u, out));
+    return launch_sample(logits, V, B, V, temperature, top_k, u, out, ld_out, static_cast<cudaStream_t>(stream));
+}
+
+GPT_API int gpt_generate(const gpt_config_t* cfg, const void* weights, const int64_t* idx, int B, int T0,
+                         int max_new_tokens, float temperature, int top_k, const float* uniforms, int64_t* out,
+                         float* step_logits, void* kv_cache, void* workspace, size_t workspace_bytes, void* stream,
+                         int flags) {
+    GPT_TRY(validate_decode(cfg));
+    if (!idx || !out || (max_new_tokens > 0 && !uniforms)) return GPT_ERR_NULL;
+    if (B < 1 || T0 < 1 || max_new_tokens < 0) return GPT_ERR_BAD_SHAPE;
+    if (static_cast<long long>(T0) + max_new_tokens > 0x7fffffffLL) return GPT_ERR_BAD_SHAPE;
+    if (max_new_tokens > 0 && (!(temperature > 0.f) || !isfinite(temperature))) return GPT_ERR_BAD_SHAPE;
+    DecodePlan D;
+    GPT_TRY(check_decode(cfg, weights, B, kv_cache, workspace, workspace_bytes,
+                         generate_prefill_len(cfg, T0, max_new_tokens), &D));
+    if (step_logits && !aligned(step_logits, 16)) return GPT_ERR_BAD_ALIGN;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    Weights W;
+    fill_weights(W, cfg, weights);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    uint8_t* kv = static_cast<uint8_t*>(kv_cache);
+    int64_t* window = reinterpret_cast<int64_t*>(ws + D.window);
+    const int V = cfg->vocab_size, bs = cfg->block_size;
+    const long long ld = static_cast<long long>(T0) + max_new_tokens;
+    GPT_TRY(cuda_status(cudaMemsetAsync(status_word(ws), 0, sizeof(int32_t), s)));
+    GPT_TRY(launch_copy_tokens(idx, T0, out, ld, B, T0, s));
+    for (int st = 0; st < max_new_tokens; ++st) {
+        const long long n = static_cast<long long>(T0) + st;  // current length
+        float* lg = step_logits ? step_logits + static_cast<size_t>(st) * B * V : reinterpret_cast<float*>(ws + D.logits);
+        if (st == 0 || n > bs) {
+            // the model sees the last min(n, block_size) tokens; once the sequence is longer than
+            // the window every position shifts, so the cache is rebuilt from the window
+            const int Tw = static_cast<int>(n < bs ? n : bs);
+            GPT_TRY(launch_copy_tokens(out + (n - Tw), ld, window, Tw, B, Tw, s));
+            GPT_TRY(prefill_impl(cfg, W, window, B, Tw, kv, lg, V, ws, D, s));
+        } else {
+            GPT_TRY(decode_step_impl(cfg, W, out + (n - 1), ld, B, kv, lg, V, ws, D, s));
+        }
+        GPT_TRY(launch_sample(lg, V, B, V, temperature, top_k, uniforms + static_cast<size_t>(st) * B, out + n, ld, s));
+    }
     if (flags & GPT_FLAG_SYNC_CHECK) return sync_and_read_status(ws, s);
     return GPT_OK;
 }

@@ -58,6 +58,7 @@ def _load() -> ctypes.CDLL:
                           "`python decoder_only_transformer_causal_b200/build.py`")
     lib = ctypes.CDLL(LIB_PATH)
     P, I, Z, D = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_int
+    L, F = ctypes.c_longlong, ctypes.c_float
     CFG = ctypes.POINTER(gpt_config_t)
     sig = {
         "gpt_status_string": (ctypes.c_char_p, [I]),
@@ -78,6 +79,13 @@ def _load() -> ctypes.CDLL:
         "gpt_lm_head_workspace_bytes": (Z, [I, I]),
         "gpt_lm_head_loss": (I, [P, P, P, I, I, I, D, P, P, P, P, P, Z, P, I]),
         "gpt_lm_head_loss_noalloc": (I, [P, P, P, I, I, I, D, P, P, P, P, P, I]),
+        "gpt_kv_cache_bytes": (Z, [CFG, I]),
+        "gpt_decode_workspace_bytes": (Z, [CFG, I, I]),
+        "gpt_generate_workspace_bytes": (Z, [CFG, I, I, I]),
+        "gpt_prefill": (I, [CFG, P, P, I, I, P, P, P, Z, P, I]),
+        "gpt_decode_step": (I, [CFG, P, P, L, I, P, P, P, Z, P, I]),
+        "gpt_sample": (I, [P, I, I, F, I, P, P, L, P]),
+        "gpt_generate": (I, [CFG, P, P, I, I, I, F, I, P, P, P, P, P, Z, P, I]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -91,7 +99,9 @@ LIB = _load()
 EXPORTED = ("gpt_status_string", "gpt_abi_version", "gpt_last_cuda_error", "gpt_validate_config", "gpt_weights_bytes",
             "gpt_weights_count", "gpt_weights_layout", "gpt_workspace_bytes", "gpt_check_status",
             "gpt_forward", "gpt_block", "gpt_attention", "gpt_embed", "gpt_layernorm", "gpt_linear",
-            "gpt_lm_head_workspace_bytes", "gpt_lm_head_loss", "gpt_lm_head_loss_noalloc")
+            "gpt_lm_head_workspace_bytes", "gpt_lm_head_loss", "gpt_lm_head_loss_noalloc",
+            "gpt_kv_cache_bytes", "gpt_decode_workspace_bytes", "gpt_generate_workspace_bytes", "gpt_prefill",
+            "gpt_decode_step", "gpt_sample", "gpt_generate")
 
 
 def status_string(status: int) -> str:
@@ -322,3 +332,84 @@ def lm_head_loss(u, wte, targets, workspace=None, logits=None, loss=None, row_lo
                                 workspace.numel(), _stream(stream),
                                 GPT_FLAG_SYNC_CHECK if sync_check else 0), "gpt_lm_head_loss")
     return logits, loss
+
+
+# ---------------------------------------------------------------- generation
+def kv_cache_bytes(cfg: GPTConfig, B: int) -> int:
+    return LIB.gpt_kv_cache_bytes(ctypes.byref(cfg.c()), B)
+
+
+def decode_workspace_bytes(cfg: GPTConfig, B: int, T_prefill: int) -> int:
+    return LIB.gpt_decode_workspace_bytes(ctypes.byref(cfg.c()), B, T_prefill)
+
+
+def generate_workspace_bytes(cfg: GPTConfig, B: int, T0: int, max_new_tokens: int) -> int:
+    return LIB.gpt_generate_workspace_bytes(ctypes.byref(cfg.c()), B, T0, max_new_tokens)
+
+
+def alloc_kv_cache(cfg: GPTConfig, B: int, device="cuda") -> torch.Tensor:
+    n = kv_cache_bytes(cfg, B)
+    if n == 0:
+        raise GPTError(GPT_ERR_UNSUPPORTED, "gpt_kv_cache_bytes")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def prefill(cfg: GPTConfig, weights: torch.Tensor, idx: torch.Tensor, kv_cache: torch.Tensor,
+            workspace: torch.Tensor, logits: torch.Tensor | None = None, stream=None, sync_check=False):
+    """gpt_prefill: fills the cache for idx [B, T]; returns the last position's logits fp32 [B, V]."""
+    B, T = idx.shape
+    if logits is None:
+        logits = torch.empty((B, cfg.vocab_size), dtype=torch.float32, device=idx.device)
+    _check(LIB.gpt_prefill(ctypes.byref(cfg.c()), _ptr(weights), _ptr(idx), B, T, _ptr(kv_cache), _ptr(logits),
+                           _ptr(workspace), workspace.numel(), _stream(stream),
+                           GPT_FLAG_SYNC_CHECK if sync_check else 0), "gpt_prefill")
+    return logits
+
+
+def decode_step(cfg: GPTConfig, weights: torch.Tensor, tok: torch.Tensor, kv_cache: torch.Tensor,
+                workspace: torch.Tensor, logits: torch.Tensor | None = None, stream=None, sync_check=False):
+    """gpt_decode_step: tok int64 [B] (a strided column view is allowed); returns logits fp32 [B, V]."""
+    if tok.dim() != 1:
+        raise ValueError("tok must be 1-D [B]")
+    B = tok.shape[0]
+    if logits is None:
+        logits = torch.empty((B, cfg.vocab_size), dtype=torch.float32, device=tok.device)
+    _check(LIB.gpt_decode_step(ctypes.byref(cfg.c()), _ptr(weights), tok.data_ptr(), tok.stride(0), B,
+                               _ptr(kv_cache), _ptr(logits), _ptr(workspace), workspace.numel(), _stream(stream),
+                               GPT_FLAG_SYNC_CHECK if sync_check else 0), "gpt_decode_step")
+    return logits
+
+
+def sample(logits: torch.Tensor, u: torch.Tensor, temperature: float = 1.0, top_k: int | None = None,
+           out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """gpt_sample: logits fp32 [B, V], u fp32 [B] in [0, 1); returns int64 [B] (or writes the
+    strided 1-D view `out`)."""
+    B, V = logits.shape
+    if out is None:
+        out = torch.empty(B, dtype=torch.int64, device=logits.device)
+    _check(LIB.gpt_sample(_ptr(logits), B, V, float(temperature), int(top_k or 0), _ptr(u), out.data_ptr(),
+                          out.stride(0), _stream(stream)), "gpt_sample")
+    return out
+
+
+def generate(cfg: GPTConfig, weights: torch.Tensor, idx: torch.Tensor, max_new_tokens: int, uniforms: torch.Tensor,
+             temperature: float = 1.0, top_k: int | None = None, kv_cache: torch.Tensor | None = None,
+             workspace: torch.Tensor | None = None, step_logits: torch.Tensor | None = None, out=None,
+             stream=None, sync_check=False) -> torch.Tensor:
+    """gpt_generate: idx int64 [B, T0]; uniforms fp32 [max_new_tokens, B]; returns
+    int64 [B, T0 + max_new_tokens]."""
+    B, T0 = idx.shape
+    if uniforms.shape != (max_new_tokens, B) or uniforms.dtype != torch.float32:
+        raise ValueError("uniforms must be float32 [max_new_tokens, B]")
+    if kv_cache is None:
+        kv_cache = alloc_kv_cache(cfg, B, idx.device)
+    if workspace is None:
+        workspace = alloc_workspace(generate_workspace_bytes(cfg, B, T0, max_new_tokens), idx.device)
+    if out is None:
+        out = torch.empty((B, T0 + max_new_tokens), dtype=torch.int64, device=idx.device)
+    _check(LIB.gpt_generate(ctypes.byref(cfg.c()), _ptr(weights), _ptr(idx), B, T0, max_new_tokens,
+                            float(temperature), int(top_k or 0), _ptr(uniforms), _ptr(out), _ptr(step_logits),
+                            _ptr(kv_cache), _ptr(workspace), workspace.numel(), _stream(stream),
+                            GPT_FLAG_SYNC_CHECK if sync_check else 0), "gpt_generate")
+    return out
+

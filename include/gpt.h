@@ -218,6 +218,67 @@ int gpt_lm_head_loss_noalloc(const void* u, const void* wte, const int64_t* targ
                              int C, int V, int dtype, void* logits, float* loss, float* row_loss,
                              double* loss_sum_count, void* stream, int flags);
 
+/* ---- generation with a key/value cache ------------------------------------------------
+ * "nanoGPT 全局流程图", 第五阶段 生成文本 (GPT.generate); "nanoGPT 核心代码速查表", 七、关键函数签名
+ * (generate(idx, max_new_tokens, temperature, top_k) -> tokens).  Each step feeds the last
+ * block_size tokens of the sequence to the model, takes the last position's logits, divides
+ * them by the temperature, keeps the logits not below the top_k-th largest (every logit at
+ * that value is kept), turns them into probabilities with softmax and draws the next token
+ * from them.  The cache is this library's incremental form of the same forward ("DummyGPTModel",
+ * 扩展方向 names the KV cache as an inference optimisation): while the sequence fits in
+ * block_size, a step runs only the newest position against the cached keys and values of the
+ * earlier ones, which gives the logits of the full forward up to rounding.
+ *
+ * KV cache: n_layer x [B, block_size, 2, n_embd] in the configuration's dtype (k of position
+ * t in [.., t, 0, :], v in [.., t, 1, :]), gpt_kv_cache_bytes(cfg, B) bytes, 16-byte aligned,
+ * owned by the caller.  The draw: with u in [0, 1) supplied by the caller (one per sequence and
+ * step), the token is the smallest index i with p_0 + ... + p_i > u * (p_0 + ... + p_{V-1}),
+ * p the kept exponentials; random numbers are inputs, never generated here.
+ * Decoding entry points require n_embd % 8 == 0 and head size % 8 == 0, <= 128. */
+size_t gpt_kv_cache_bytes(const gpt_config_t* cfg, int B);
+
+/* Workspace of gpt_prefill (T <= T_prefill) and gpt_decode_step (any T_prefill >= 1), 256-byte
+ * aligned.  The same workspace carries the decode position between calls (device-side, so a
+ * captured step can be replayed); do not share it between sequences decoded concurrently. */
+size_t gpt_decode_workspace_bytes(const gpt_config_t* cfg, int B, int T_prefill);
+
+/* Forward over idx int64 [B, T] (1 <= T <= block_size) that writes every layer's k and v of
+ * positions [0, T) into kv_cache and the logits of position T-1 to logits fp32 [B, V]; sets the
+ * decode position to T.  flags: GPT_FLAG_SYNC_CHECK as in gpt_forward. */
+int gpt_prefill(const gpt_config_t* cfg, const void* weights, const int64_t* idx, int B, int T,
+                void* kv_cache, float* logits, void* workspace, size_t workspace_bytes,
+                void* stream, int flags);
+
+/* One new token per sequence, tok[b * ld_tok] (int64), at the decode position p held in the
+ * workspace: each layer appends its k, v at p and attends over positions [0, p]; writes the
+ * logits fp32 [B, V] of that position and advances p by one.  The cache must hold positions
+ * [0, p) from gpt_prefill and earlier steps with the same B.  p must be < block_size: beyond
+ * it the step writes nothing to the cache, records GPT_ERR_BAD_SHAPE in the status word and
+ * its logits are meaningless (gpt_generate re-runs gpt_prefill on the window instead). */
+int gpt_decode_step(const gpt_config_t* cfg, const void* weights, const int64_t* tok,
+                    long long ld_tok, int B, void* kv_cache, float* logits, void* workspace,
+                    size_t workspace_bytes, void* stream, int flags);
+
+/* The sampling step on logits fp32 [B, V]: temperature > 0 (GPT_ERR_BAD_SHAPE otherwise),
+ * top_k <= 0 for no top-k filter, u fp32 [B] in [0, 1); writes out[b * ld_out] (int64).  The
+ * top-k threshold is taken on the logits before the division (the same order for any
+ * positive temperature).  Sums run in a fixed order; the result is deterministic. */
+int gpt_sample(const float* logits, int B, int V, float temperature, int top_k, const float* u,
+               int64_t* out, long long ld_out, void* stream);
+
+/* GPT.generate: out int64 [B, T0 + max_new_tokens] = idx [B, T0] followed by max_new_tokens
+ * drawn tokens; uniforms fp32 [max_new_tokens, B] (step-major).  step_logits: optional fp32
+ * [max_new_tokens, B, V] that receives each step's logits before the temperature (NULL to
+ * skip).  Step s sees the last min(T0 + s, block_size) tokens: the first step and every step
+ * whose sequence is longer than block_size run gpt_prefill on that window (the positions of
+ * a cropped window shift, so the cache is rebuilt); the others run gpt_decode_step.
+ * workspace: gpt_generate_workspace_bytes(cfg, B, T0, max_new_tokens) bytes. */
+size_t gpt_generate_workspace_bytes(const gpt_config_t* cfg, int B, int T0, int max_new_tokens);
+int gpt_generate(const gpt_config_t* cfg, const void* weights, const int64_t* idx, int B, int T0,
+                 int max_new_tokens, float temperature, int top_k, const float* uniforms,
+                 int64_t* out, float* step_logits, void* kv_cache, void* workspace,
+                 size_t workspace_bytes, void* stream, int flags);
+
 #ifdef __cplusplus
 }
 #endif

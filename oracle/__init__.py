@@ -5,10 +5,12 @@ and the CPU-baseline leg of ``bench.py`` may import it.  It shares nothing with 
 CUDA path (no kernels, headers, helpers, tables or constants); the two meet only in
 the seeded inputs of the ``seeded`` module.
 
-See ``oracle/gpt.py`` for the definitions and their citations.
+See ``oracle/gpt.py`` (the forward pass) and ``oracle/generate.py`` (GPT.generate) for the
+definitions and their citations.
 """
 from .gpt import (  # noqa: F401
     PAGES, embed, layer_norm, linear, split_heads, merge_heads, attention_probs,
     causal_attention, gelu, causal_self_attention, mlp, block, final_hidden,
     lm_head, cross_entropy, forward, num_params,
 )
+from . import generate as gen  # noqa: F401,E402

@@ -188,6 +188,26 @@ def make_residual(batch: int, seq_len: int, n_embd: int, seed: int = BASE_SEED +
     return std * torch.randn((batch, seq_len, n_embd), generator=g, device=device)
 
 
+def make_uniforms(steps: int, batch: int, seed: int = BASE_SEED + 400_000) -> torch.Tensor:
+    """fp32 [steps, B] uniforms in [0, 1): the random numbers of the sampling draws, supplied
+    to both implementations."""
+    return torch.rand((steps, batch), generator=_gen(seed), dtype=torch.float32)
+
+
+def make_logits(batch: int, vocab: int, seed: int = BASE_SEED + 500_000, std: float = 2.0,
+                ties: int = 0) -> torch.Tensor:
+    """fp32 [B, V] logits N(0, std^2) for the sampling step.  ``ties`` > 0 copies the largest
+    value of each row onto that many other (seeded) positions, so the top-k threshold has
+    ties."""
+    g = _gen(seed)
+    z = std * torch.randn((batch, vocab), generator=g)
+    if ties:
+        for b in range(batch):
+            pos = torch.randperm(vocab, generator=g)[:ties]
+            z[b, pos] = z[b].max()
+    return z
+
+
 def to_f64(weights: dict[str, torch.Tensor]):
     """Widen stored weights to fp64 numpy arrays (what the oracle consumes)."""
     return {k: v.to(torch.float64).numpy() for k, v in weights.items()}

@@ -125,3 +125,53 @@ def test_kernel_entry_validation():
     assert L.gpt_lm_head_loss(FAKE, FAKE, FAKE, 4, 64, 128, native.GPT_DTYPE_BF16, FAKE, None, None, None,
                               FAKE, 16, None, 0) == native.GPT_ERR_WS_TOO_SMALL
     assert L.gpt_check_status(None, None) == native.GPT_ERR_NULL
+
+
+def test_generation_sizes():
+    cfg = _cfg("gpt2")
+    L, B, bs, C = 12, 4, 1024, 768
+    assert native.kv_cache_bytes(cfg, B) == L * B * bs * 2 * C * 2
+    assert native.kv_cache_bytes(_cfg("tiny"), 2) == 4 * 2 * 64 * 2 * 128 * 4
+    assert native.kv_cache_bytes(cfg, 0) == 0
+    d1 = native.decode_workspace_bytes(cfg, B, 1)
+    assert d1 >= native.workspace_bytes(cfg, B, 1) + B * 50304 * 4
+    assert native.decode_workspace_bytes(cfg, B, 1025) == 0
+    # generate: a sequence that outgrows the window needs a full-window prefill
+    assert native.generate_workspace_bytes(cfg, B, 8, 100) == native.decode_workspace_bytes(cfg, B, 8)
+    assert native.generate_workspace_bytes(cfg, B, 1000, 100) == native.decode_workspace_bytes(cfg, B, 1024)
+    assert native.generate_workspace_bytes(cfg, B, 2000, 0) == native.decode_workspace_bytes(cfg, B, 1024)
+    assert native.generate_workspace_bytes(_cfg("gpt2", n_embd=772, n_head=4), B, 8, 1) == 0   # hs 193
+
+
+def test_generation_host_validation():
+    Lb = native.LIB
+    cfg = _cfg("gpt2")
+    c = ctypes.byref(cfg.c())
+    big = 1 << 40
+    # gpt_sample: temperature must be positive and finite; pointers non-null
+    assert Lb.gpt_sample(FAKE, 2, 100, 0.0, 0, FAKE, FAKE, 1, None) == native.GPT_ERR_BAD_SHAPE
+    assert Lb.gpt_sample(FAKE, 2, 100, -1.0, 0, FAKE, FAKE, 1, None) == native.GPT_ERR_BAD_SHAPE
+    assert Lb.gpt_sample(FAKE, 2, 100, float("inf"), 0, FAKE, FAKE, 1, None) == native.GPT_ERR_BAD_SHAPE
+    assert Lb.gpt_sample(FAKE, 2, 100, 1.0, 0, None, FAKE, 1, None) == native.GPT_ERR_NULL
+    assert Lb.gpt_sample(FAKE, 0, 100, 1.0, 0, FAKE, FAKE, 1, None) == native.GPT_ERR_BAD_SHAPE
+    # gpt_prefill / gpt_decode_step
+    assert Lb.gpt_prefill(c, FAKE, FAKE, 2, 1025, FAKE, FAKE, FAKE, big, None, 0) == native.GPT_ERR_BAD_SHAPE
+    assert Lb.gpt_prefill(c, FAKE, FAKE, 2, 16, None, FAKE, FAKE, big, None, 0) == native.GPT_ERR_NULL
+    assert Lb.gpt_prefill(c, FAKE, FAKE, 2, 16, FAKE, FAKE, FAKE, 4096, None, 0) == native.GPT_ERR_WS_TOO_SMALL
+    assert Lb.gpt_prefill(c, FAKE, FAKE, 2, 16, FAKE + 8, FAKE, FAKE, big, None, 0) == native.GPT_ERR_BAD_ALIGN
+    assert Lb.gpt_decode_step(c, FAKE, None, 1, 2, FAKE, FAKE, FAKE, big, None, 0) == native.GPT_ERR_NULL
+    assert Lb.gpt_decode_step(c, FAKE, FAKE, 1, 0, FAKE, FAKE, FAKE, big, None, 0) == native.GPT_ERR_BAD_SHAPE
+    assert Lb.gpt_decode_step(c, FAKE, FAKE, 1, 2, FAKE, FAKE + 4, FAKE, big, None, 0) == native.GPT_ERR_BAD_ALIGN
+    # gpt_generate
+    gen = lambda **k: Lb.gpt_generate(c, k.get("w", FAKE), k.get("idx", FAKE), k.get("B", 2), k.get("T0", 8),
+                                      k.get("n", 4), k.get("temp", 1.0), 0, k.get("u", FAKE), FAKE, None,
+                                      FAKE, FAKE, k.get("ws", big), None, 0)
+    assert gen(u=None) == native.GPT_ERR_NULL
+    assert gen(temp=0.0) == native.GPT_ERR_BAD_SHAPE
+    assert gen(n=-1) == native.GPT_ERR_BAD_SHAPE
+    assert gen(T0=0) == native.GPT_ERR_BAD_SHAPE
+    assert gen(ws=4096) == native.GPT_ERR_WS_TOO_SMALL
+    assert gen(w=FAKE + 16) == native.GPT_ERR_BAD_ALIGN
+    # an unsupported head size for the decode kernels
+    c2 = ctypes.byref(_cfg("tiny", n_head=32).c())                                   # hs 4
+    assert Lb.gpt_prefill(c2, FAKE, FAKE, 1, 4, FAKE, FAKE, FAKE, big, None, 0) == native.GPT_ERR_UNSUPPORTED
