@@ -3,13 +3,13 @@
 // multinomial draw).
 //
 // A decode step reads every weight once for a handful of rows, so its matrix products are
-// matrix-vector products bound by HBM bandwidth, not tensor-core work: one warp per output
-// column streams the weight row with 16-byte loads against up to kGemvRows input rows staged
-// in shared memory as fp32, and the epilogue (bias, GELU, residual add, k/v append) is fused.
-// The attention of the new position against the cached keys is split over key ranges (so a
-// long cache is read by many CTAs at once) and merged by a combine kernel.  The position being
-// written lives in device memory, so a recorded graph of a step can be replayed as the
-// sequence grows.
+// matrix-vector products bound by HBM bandwidth, not tensor-core work: CTAs of 8 warps stage
+// the input rows in shared memory (fusing the LayerNorm that precedes ln_1 / ln_2 / ln_f
+// products) and stream weight rows with 16-byte loads; the epilogue (bias, GELU, residual
+// add, k/v append) is fused.  The attention of the new position against the cached keys is
+// split over 64-key ranges (so a long cache is read by many CTAs at once) and merged by the
+// last CTA of each head.  The position being written lives in device memory, so a recorded
+// graph of a step can be replayed as the sequence grows.
 //
 // Element type E is the configuration's storage type (bf16 or fp32) for weights, activations
 // and the cache; accumulation is fp32 throughout and the residual stream is fp32.
@@ -29,12 +29,6 @@
 namespace gpt {
 
 namespace {
-
-constexpr int kGemvWarps = 4;     // warps (= output columns in flight) per CTA
-constexpr int kGemvRows = 8;      // input rows per launch (larger batches are split)
-constexpr int kChunkK = 1024;     // K elements of each input row staged per pass
-constexpr int kSplitKeys = 128;   // keys per CTA in the decode attention
-constexpr int kMaxHs = 128;
 
 GPT_DEVINL float to_f(bf16 v) { return __bfloat162float(v); }
 GPT_DEVINL float to_f(float v) { return v; }
@@ -79,6 +73,27 @@ GPT_DEVINL float warp_sum(float v) {
     return v;
 }
 
+// Asks L2 to fetch [p, p + bytes) (both multiples of 16) from HBM; no completion to wait on.
+GPT_DEVINL void prefetch_l2(const void* p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+// This CTA's share of an L2 prefetch of [base, base + bytes): the whole range is split over the
+// grid in 16-byte-aligned pieces, so the first CTAs to start fetch all of it.
+GPT_DEVINL void prefetch_l2_share(const void* base, size_t bytes) {
+    const size_t per = ((bytes + gridDim.x - 1) / gridDim.x + 15) & ~static_cast<size_t>(15);
+    const size_t off = per * blockIdx.x;
+    if (off >= bytes) return;
+    size_t n = bytes - off < per ? bytes - off : per;
+    const uint8_t* p = static_cast<const uint8_t*>(base) + off;
+    while (n >= 16) {
+        const uint32_t chunk = n > (1u << 20) ? (1u << 20) : static_cast<uint32_t>(n & ~static_cast<size_t>(15));
+        prefetch_l2(p, chunk);
+        p += chunk;
+        n -= chunk;
+    }
+}
+
 GPT_DEVINL float gelu_erf(float v) { return 0.5f * v * (1.0f + erff(v * 0.70710678118654752f)); }
 GPT_DEVINL float gelu_tanh(float v) {
     return 0.5f * v * (1.0f + tanhf(0.79788456080286536f * (v + 0.044715f * v * v * v)));
@@ -107,184 +122,364 @@ __global__ void embed_pos_kernel(const E* __restrict__ wte, const E* __restrict_
     x[i] = to_f(wte[t * C + c]) + to_f(wpe[static_cast<long long>(p) * C + c]);
 }
 
+// ---------------------------------------------------------------- matrix-vector products
+// out[r, n] = epilogue(sum_k xin[r, k] W[n, k] + bias[n]) for up to kGemvRows rows r.
+//
+// A CTA of 8 warps stages its input rows in shared memory once (in E, as stored between
+// kernels), optionally as LayerNorm of the fp32 residual stream (the ln_1 / ln_2 / ln_f that
+// precedes the product, fused).  Warps then stream weight rows with 16-byte loads: KSPLIT
+// warps share one column, each over a contiguous K slice (narrow outputs need the extra
+// loads in flight), and each warp carries CPW columns (the vocabulary head).  Partial sums
+// are reduced over lanes by a butterfly and over the KSPLIT warps in slice order.
+constexpr int kGemvThreads = 256;
+constexpr int kGemvWarps = kGemvThreads / 32;
+constexpr int kGemvRows = 8;
+
 template <typename E>
 struct GemvArgs {
-    const E* x;         // [rows, K] at row stride ldx
+    const void* x;      // LN: fp32 residual rows [rows, K]; otherwise E rows [rows, K]; row stride ldx
     long long ldx;
+    const E* ln_w;      // LN prologue weight / bias (bias may be null)
+    const E* ln_b;
     const E* W;         // [N, K]
     const E* bias;      // [N] or null
-    void* out;          // see GemvEpi
+    void* out;          // see DecodeEpi
     long long ldo;
     int rows, N, K, gelu_tanh;
     E* kv;              // DV_QKV: this layer's cache [rows, block_size, 2C]
-    const int* pos;
-    int C, block_size;
+    int* pos;           // DV_QKV reads it; bump_pos: CTA 0 advances it by one
+    int C, block_size, bump_pos;
 };
 
-enum GemvEpi {
-    DV_STORE = 0,   // out E [rows, N]
+enum DecodeEpi {
     DV_GELU = 1,    // out E [rows, N] = gelu(.)
     DV_RESID = 2,   // out fp32 [rows, N] += .
     DV_F32 = 3,     // out fp32 [rows, N]
     DV_QKV = 4,     // columns [0, C) -> out E (q); [C, 3C) -> kv[row, *pos, :] (k then v)
 };
 
-// out[r, n] = epilogue(sum_k x[r, k] W[n, k] + bias[n]); one warp per column n, fixed
-// summation order (lane-strided partial sums, then a butterfly).
-template <typename E, int EPI>
-__global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const GemvArgs<E> a) {
+GPT_DEVINL void store4(bf16* p, float a, float b, float c, float d) {
+    __nv_bfloat162 lo = __floats2bfloat162_rn(a, b), hi = __floats2bfloat162_rn(c, d);
+    uint2 v;
+    v.x = *reinterpret_cast<uint32_t*>(&lo);
+    v.y = *reinterpret_cast<uint32_t*>(&hi);
+    *reinterpret_cast<uint2*>(p) = v;
+}
+GPT_DEVINL void store4(float* p, float a, float b, float c, float d) {
+    *reinterpret_cast<float4*>(p) = make_float4(a, b, c, d);
+}
+GPT_DEVINL float4 load4w(const bf16* p) {
+    const uint2 v = *reinterpret_cast<const uint2*>(p);
+    const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162*>(&v.x);
+    const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162*>(&v.y);
+    return make_float4(__low2float(lo), __high2float(lo), __low2float(hi), __high2float(hi));
+}
+GPT_DEVINL float4 load4w(const float* p) { return *reinterpret_cast<const float4*>(p); }
+
+template <typename E, int EPI, int KSPLIT, int CPW, bool LN>
+__global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const GemvArgs<E> a) {
     griddep_launch_dependents();
+    // the weights never change: start bringing them into L2 while the previous kernel finishes
+    if (threadIdx.x == 0) prefetch_l2_share(a.W, static_cast<size_t>(a.N) * a.K * sizeof(E));
     griddep_wait();
-    __shared__ __align__(16) float xs[kGemvRows * kChunkK];
+    extern __shared__ __align__(16) uint8_t gemv_smem[];
+    E* xs = reinterpret_cast<E*>(gemv_smem);  // [rows][K]
+    float* xf = reinterpret_cast<float*>(gemv_smem + static_cast<size_t>(a.rows) * a.K * sizeof(E));  // LN input
+    __shared__ float red[kGemvWarps][CPW][kGemvRows];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n = blockIdx.x * kGemvWarps + warp;
-    float acc[kGemvRows];
-#pragma unroll
-    for (int r = 0; r < kGemvRows; ++r) acc[r] = 0.f;
-    const E* wrow = a.W + static_cast<long long>(n < a.N ? n : 0) * a.K;
-    for (int k0 = 0; k0 < a.K; k0 += kChunkK) {
-        const int kc = min(kChunkK, a.K - k0);
-        __syncthreads();
-        for (int i = threadIdx.x; i < a.rows * kc; i += blockDim.x) {
-            const int r = i / kc, k = i % kc;
-            xs[r * kChunkK + k] = ld_act(a.x + r * a.ldx + k0 + k);
+    const int K = a.K;
+
+    if (LN) {
+        // LayerNorm of each fp32 row (population variance, eps 1e-5): the rows are copied to
+        // shared memory, then one warp per row takes the mean, the squared deviations and the
+        // normalised values from there
+        const float* x = static_cast<const float*>(a.x);
+        const int per_row = K / 4;
+        for (int i = threadIdx.x; i < a.rows * per_row; i += kGemvThreads) {
+            const int r = i / per_row, c = i % per_row;
+            reinterpret_cast<float4*>(xf + r * K)[c] = __ldcg(reinterpret_cast<const float4*>(x + r * a.ldx) + c);
         }
         __syncthreads();
-        if (n < a.N) {
-#pragma unroll 2
-            for (int k = lane * 8; k < kc; k += 256) {
-                float wf[8];
-                load8(wrow + k0 + k, wf);
+        for (int r = warp; r < a.rows; r += kGemvWarps) {
+            const float* xr = xf + r * K;
+            float sum = 0.f;
+            for (int k = lane * 4; k < K; k += 128) {
+                const float4 v = *reinterpret_cast<const float4*>(xr + k);
+                sum += (v.x + v.y) + (v.z + v.w);
+            }
+            const float mean = warp_sum(sum) / K;
+            float ss = 0.f;
+            for (int k = lane * 4; k < K; k += 128) {
+                const float4 v = *reinterpret_cast<const float4*>(xr + k);
+                const float p = v.x - mean, q = v.y - mean, t = v.z - mean, w = v.w - mean;
+                ss += (p * p + q * q) + (t * t + w * w);
+            }
+            const float rstd = rsqrtf(warp_sum(ss) / K + 1e-5f);
+            for (int k = lane * 4; k < K; k += 128) {
+                const float4 v = *reinterpret_cast<const float4*>(xr + k);
+                const float4 g = load4w(a.ln_w + k);
+                const float4 bb = a.ln_b ? load4w(a.ln_b + k) : make_float4(0.f, 0.f, 0.f, 0.f);
+                store4(xs + r * K + k, (v.x - mean) * rstd * g.x + bb.x, (v.y - mean) * rstd * g.y + bb.y,
+                       (v.z - mean) * rstd * g.z + bb.z, (v.w - mean) * rstd * g.w + bb.w);
+            }
+        }
+    } else {
+        const E* x = static_cast<const E*>(a.x);
+        const int per_row = K * static_cast<int>(sizeof(E)) / 16;
+        for (int i = threadIdx.x; i < a.rows * per_row; i += kGemvThreads) {
+            const int r = i / per_row, c = i % per_row;
+            reinterpret_cast<uint4*>(xs + r * K)[c] = __ldcg(reinterpret_cast<const uint4*>(x + r * a.ldx) + c);
+        }
+    }
+    __syncthreads();
+    if (a.bump_pos && blockIdx.x == 0 && threadIdx.x == 0) *a.pos = __ldcg(a.pos) + 1;
+
+    constexpr int kCols = (kGemvWarps / KSPLIT) * CPW;
+    const int ks = warp % KSPLIT;
+    const int slice = K / KSPLIT;
+    const int k_lo = ks * slice, k_hi = k_lo + slice;
+    const int n_groups = (a.N + kCols - 1) / kCols;
+    // column groups g = blockIdx.x, blockIdx.x + gridDim.x, ...: the staged rows serve them all
+    for (int g = blockIdx.x; g < n_groups; g += gridDim.x) {
+        const int n0 = g * kCols + (warp / KSPLIT) * CPW;
+        float acc[CPW][kGemvRows];
 #pragma unroll
-                for (int r = 0; r < kGemvRows; ++r) {
-                    if (r < a.rows) {
-                        const float4 x0 = *reinterpret_cast<const float4*>(&xs[r * kChunkK + k]);
-                        const float4 x1 = *reinterpret_cast<const float4*>(&xs[r * kChunkK + k + 4]);
-                        float s = acc[r];
-                        s = fmaf(wf[0], x0.x, s);
-                        s = fmaf(wf[1], x0.y, s);
-                        s = fmaf(wf[2], x0.z, s);
-                        s = fmaf(wf[3], x0.w, s);
-                        s = fmaf(wf[4], x1.x, s);
-                        s = fmaf(wf[5], x1.y, s);
-                        s = fmaf(wf[6], x1.z, s);
-                        s = fmaf(wf[7], x1.w, s);
-                        acc[r] = s;
+        for (int c = 0; c < CPW; ++c)
+#pragma unroll
+            for (int r = 0; r < kGemvRows; ++r) acc[c][r] = 0.f;
+        const E* wrow[CPW];
+#pragma unroll
+        for (int c = 0; c < CPW; ++c) wrow[c] = a.W + static_cast<long long>(min(n0 + c, a.N - 1)) * K;
+#pragma unroll 4
+        for (int k = k_lo + lane * 8; k < k_hi; k += 256) {
+            float wf[CPW][8];
+#pragma unroll
+            for (int c = 0; c < CPW; ++c) load8(wrow[c] + k, wf[c]);
+#pragma unroll
+            for (int r = 0; r < kGemvRows; ++r) {
+                if (r < a.rows) {
+                    float xf[8];
+                    load8(xs + r * K + k, xf);
+#pragma unroll
+                    for (int c = 0; c < CPW; ++c) {
+                        float sacc = acc[c][r];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) sacc = fmaf(wf[c][e], xf[e], sacc);
+                        acc[c][r] = sacc;
                     }
                 }
             }
         }
-    }
-    if (n >= a.N) return;
-    const float bias = a.bias ? to_f(a.bias[n]) : 0.f;
 #pragma unroll
-    for (int r = 0; r < kGemvRows; ++r) {
-        if (r >= a.rows) break;
-        float v = warp_sum(acc[r]) + bias;
-        if (lane != 0) continue;
-        if (EPI == DV_STORE) {
-            static_cast<E*>(a.out)[r * a.ldo + n] = from_f<E>(v);
-        } else if (EPI == DV_GELU) {
-            v = a.gelu_tanh ? gelu_tanh(v) : gelu_erf(v);
-            static_cast<E*>(a.out)[r * a.ldo + n] = from_f<E>(v);
-        } else if (EPI == DV_RESID) {
-            float* o = static_cast<float*>(a.out) + r * a.ldo + n;
-            *o = __ldcg(o) + v;
-        } else if (EPI == DV_F32) {
-            static_cast<float*>(a.out)[r * a.ldo + n] = v;
-        } else {  // DV_QKV
-            if (n < a.C) {
+        for (int c = 0; c < CPW; ++c)
+#pragma unroll
+            for (int r = 0; r < kGemvRows; ++r) {
+                if (r < a.rows) {
+                    const float v = warp_sum(acc[c][r]);
+                    if (lane == 0) red[warp][c][r] = v;
+                }
+            }
+        if (KSPLIT > 1) __syncthreads();
+        else __syncwarp();
+        const int c = lane / kGemvRows, r = lane % kGemvRows;
+        const int n = n0 + c;
+        if (ks == 0 && c < CPW && r < a.rows && n < a.N) {
+            float v = 0.f;
+#pragma unroll
+            for (int j = 0; j < KSPLIT; ++j) v += red[warp + j][c][r];
+            if (a.bias) v += to_f(a.bias[n]);
+            if (EPI == DV_GELU) {
+                v = a.gelu_tanh ? gelu_tanh(v) : gelu_erf(v);
                 static_cast<E*>(a.out)[r * a.ldo + n] = from_f<E>(v);
-            } else {
-                const int p = __ldcg(a.pos);
-                if (p >= 0 && p < a.block_size)
-                    a.kv[(static_cast<long long>(r) * a.block_size + p) * 2 * a.C + (n - a.C)] = from_f<E>(v);
+            } else if (EPI == DV_RESID) {
+                float* o = static_cast<float*>(a.out) + r * a.ldo + n;
+                *o = __ldcg(o) + v;
+            } else if (EPI == DV_F32) {
+                static_cast<float*>(a.out)[r * a.ldo + n] = v;
+            } else {  // DV_QKV
+                if (n < a.C) {
+                    static_cast<E*>(a.out)[r * a.ldo + n] = from_f<E>(v);
+                } else {
+                    const int p = __ldcg(a.pos);
+                    if (p >= 0 && p < a.block_size)
+                        a.kv[(static_cast<long long>(r) * a.block_size + p) * 2 * a.C + (n - a.C)] = from_f<E>(v);
+                }
             }
         }
+        if (KSPLIT > 1) __syncthreads();  // red is rewritten by the next group
+        else __syncwarp();
     }
 }
 
-// Attention of the newest position against cached keys 0..pos (the causal mask is implicit:
-// no later key exists yet).  CTA (split, b*nh + h) scores keys [split*kSplitKeys, ...) with one
-// key per thread and writes its partial {max m (log2 units), sum l, O[hs]} to part.
+// ---------------------------------------------------------------- decode attention
+// The newest position of sequence b, head h attends over cached positions 0..pos (the causal
+// mask is implicit: no later key exists yet).  CTA (split, b*nh + h) takes kSplitKeys keys,
+// one per thread for the scores; for p.v each warp takes half of the keys with a lane per
+// pair of dimensions (coalesced rows).  With more than one split, each CTA leaves
+// {m (log2 units), l, O[hs]} in part and the last CTA of the head to finish (a counter per
+// head, reset by that CTA) merges them: y = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s.
+constexpr int kSplitKeys = 64;
+constexpr int kMaxHs = 128;
+
+template <typename E> struct Pair;
+template <> struct Pair<bf16> {
+    static GPT_DEVINL float2 ld(const bf16* p) {
+        const uint32_t v = __ldcg(reinterpret_cast<const unsigned int*>(p));
+        const __nv_bfloat162 h = *reinterpret_cast<const __nv_bfloat162*>(&v);
+        return make_float2(__low2float(h), __high2float(h));
+    }
+    static GPT_DEVINL void st(bf16* p, float a, float b) {
+        *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(a, b);
+    }
+};
+template <> struct Pair<float> {
+    static GPT_DEVINL float2 ld(const float* p) { return __ldcg(reinterpret_cast<const float2*>(p)); }
+    static GPT_DEVINL void st(float* p, float a, float b) { *reinterpret_cast<float2*>(p) = make_float2(a, b); }
+};
+
 template <typename E>
 __global__ void __launch_bounds__(kSplitKeys)
-    decode_attn_partial(const E* __restrict__ q, const E* __restrict__ kv, const int* __restrict__ pos,
-                        float* __restrict__ part, int nh, int hs, int block_size, int n_split_max, float scale_log2) {
+    decode_attention_kernel(const E* __restrict__ q, const E* __restrict__ kv, const int* __restrict__ pos,
+                            float* __restrict__ part, int* __restrict__ counter, E* __restrict__ y, int nh, int hs,
+                            int block_size, int n_split_max, float scale_log2) {
     griddep_launch_dependents();
+    {
+        // cached keys and values before the newest position do not change during this step:
+        // prefetch this split's rows into L2 while the previous kernel finishes (a range read
+        // from a position that is about to move is harmless for a prefetch)
+        const int t = blockIdx.x * kSplitKeys + threadIdx.x;
+        const int b = blockIdx.y / nh, h = blockIdx.y % nh, C = nh * hs;
+        if (t < min(__ldcg(pos) + 1, block_size)) {
+            const E* row = kv + (static_cast<long long>(b) * block_size + t) * 2 * C + h * hs;
+            prefetch_l2(row, hs * sizeof(E));
+            prefetch_l2(row + C, hs * sizeof(E));
+        }
+    }
     griddep_wait();
     __shared__ __align__(16) float qs[kMaxHs];
     __shared__ float ps[kSplitKeys];
-    __shared__ float red[kSplitKeys / 32];
+    __shared__ float wmax[2], wsum[2];
+    __shared__ float o1[kMaxHs];
     const int split = blockIdx.x, bh = blockIdx.y;
     const int b = bh / nh, h = bh % nh;
     const int C = nh * hs;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n_keys = min(__ldcg(pos) + 1, block_size);
+    const int n_split = (n_keys + kSplitKeys - 1) / kSplitKeys;
+    if (split >= n_split) return;
     const int k0 = split * kSplitKeys;
-    float* out = part + (static_cast<long long>(bh) * n_split_max + split) * (hs + 2);
-    if (k0 >= n_keys) return;  // the combine reads only splits that hold keys
-    for (int d = threadIdx.x; d < hs; d += blockDim.x) qs[d] = ld_act(q + static_cast<long long>(b) * C + h * hs + d);
+    for (int d = threadIdx.x; d < hs; d += kSplitKeys) qs[d] = ld_act(q + static_cast<long long>(b) * C + h * hs + d);
     __syncthreads();
-    const E* base = kv + static_cast<long long>(b) * block_size * 2 * C;
+    const E* base = kv + static_cast<long long>(b) * block_size * 2 * C + h * hs;
     const int t = k0 + threadIdx.x;
     float s = -INFINITY;
     if (t < n_keys) {
-        const E* kr = base + static_cast<long long>(t) * 2 * C + h * hs;
-        float acc = 0.f;
-        for (int d = 0; d < hs; d += 8) {
-            float kf[8];
-            load8_act(kr + d, kf);
+        const E* kr = base + static_cast<long long>(t) * 2 * C;
+        float kf[kMaxHs / 8][8];  // the whole key row in flight at once
 #pragma unroll
-            for (int e = 0; e < 8; ++e) acc = fmaf(qs[d + e], kf[e], acc);
-        }
+        for (int j = 0; j < kMaxHs / 8; ++j)
+            if (8 * j < hs) load8_act(kr + 8 * j, kf[j]);
+        float acc = 0.f;
+#pragma unroll
+        for (int j = 0; j < kMaxHs / 8; ++j)
+            if (8 * j < hs) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc = fmaf(qs[8 * j + e], kf[j][e], acc);
+            }
         s = acc * scale_log2;
     }
     float m = s;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+    if (lane == 0) wmax[warp] = m;
     __syncthreads();
-    m = red[0];
-#pragma unroll
-    for (int w = 1; w < kSplitKeys / 32; ++w) m = fmaxf(m, red[w]);
-    ps[threadIdx.x] = (t < n_keys) ? exp2f(s - m) : 0.f;
+    m = fmaxf(wmax[0], wmax[1]);
+    const float p = (t < n_keys) ? exp2f(s - m) : 0.f;
+    ps[threadIdx.x] = p;
+    const float lw = warp_sum(p);
+    if (lane == 0) wsum[warp] = lw;
     __syncthreads();
-    // O[d] = sum_i p_i v_i[d] over this split's keys, in key order
+    // p.v: warp w over keys [32w, 32w + 32) of the split, lane over dimension pairs
     const int n_here = min(kSplitKeys, n_keys - k0);
-    for (int d = threadIdx.x; d < hs; d += blockDim.x) {
-        const E* vc = base + static_cast<long long>(k0) * 2 * C + C + h * hs + d;
-        float o = 0.f;
-        for (int i = 0; i < n_here; ++i) o = fmaf(ps[i], ld_act(vc + static_cast<long long>(i) * 2 * C), o);
-        out[2 + d] = o;
+    const int i_lo = warp * 32, i_hi = min(i_lo + 32, n_here);
+    float o[kMaxHs / 32];
+#pragma unroll
+    for (int j = 0; j < kMaxHs / 32; ++j) o[j] = 0.f;
+    const E* vbase = base + C + static_cast<long long>(k0) * 2 * C;
+#pragma unroll 16
+    for (int i = i_lo; i < i_hi; ++i) {
+        const float pi = ps[i];
+        const E* vr = vbase + static_cast<long long>(i) * 2 * C;
+#pragma unroll
+        for (int j = 0; j < kMaxHs / 64; ++j) {
+            const int d = 2 * lane + 64 * j;
+            if (d < hs) {
+                const float2 v = Pair<E>::ld(vr + d);
+                o[2 * j] = fmaf(pi, v.x, o[2 * j]);
+                o[2 * j + 1] = fmaf(pi, v.y, o[2 * j + 1]);
+            }
+        }
     }
-    if (threadIdx.x == 0) {
-        float l = 0.f;
-        for (int i = 0; i < n_here; ++i) l += ps[i];
-        out[0] = m;
-        out[1] = l;
+    if (warp == 1) {
+#pragma unroll
+        for (int j = 0; j < kMaxHs / 64; ++j) {
+            const int d = 2 * lane + 64 * j;
+            if (d < hs) o1[d] = o[2 * j], o1[d + 1] = o[2 * j + 1];
+        }
     }
-}
-
-// y = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s over the splits that hold keys.
-template <typename E>
-__global__ void decode_attn_combine(const float* __restrict__ part, const int* __restrict__ pos, E* __restrict__ y,
-                                    int nh, int hs, int block_size, int n_split_max) {
-    griddep_launch_dependents();
-    griddep_wait();
-    const int bh = blockIdx.x;
-    const int b = bh / nh, h = bh % nh;
-    const int n_keys = min(__ldcg(pos) + 1, block_size);
-    const int n_split = (n_keys + kSplitKeys - 1) / kSplitKeys;
+    __syncthreads();
+    if (warp != 0) return;
+#pragma unroll
+    for (int j = 0; j < kMaxHs / 64; ++j) {
+        const int d = 2 * lane + 64 * j;
+        if (d < hs) o[2 * j] += o1[d], o[2 * j + 1] += o1[d + 1];
+    }
+    const float l = wsum[0] + wsum[1];
+    E* yr = y + static_cast<long long>(b) * C + h * hs;
+    if (n_split == 1) {
+#pragma unroll
+        for (int j = 0; j < kMaxHs / 64; ++j) {
+            const int d = 2 * lane + 64 * j;
+            if (d < hs) Pair<E>::st(yr + d, o[2 * j] / l, o[2 * j + 1] / l);
+        }
+        return;
+    }
+    float* mine = part + (static_cast<long long>(bh) * n_split_max + split) * (hs + 2);
+#pragma unroll
+    for (int j = 0; j < kMaxHs / 64; ++j) {
+        const int d = 2 * lane + 64 * j;
+        if (d < hs) mine[2 + d] = o[2 * j], mine[3 + d] = o[2 * j + 1];
+    }
+    if (lane == 0) mine[0] = m, mine[1] = l;
+    __threadfence();
+    __syncwarp();
+    int ticket = 0;
+    if (lane == 0) ticket = atomicAdd(counter + bh, 1);
+    ticket = __shfl_sync(0xffffffffu, ticket, 0);
+    if (ticket != n_split - 1) return;
+    __threadfence();
     const float* pp = part + static_cast<long long>(bh) * n_split_max * (hs + 2);
     float M = -INFINITY;
-    for (int s = 0; s < n_split; ++s) M = fmaxf(M, __ldcg(pp + s * (hs + 2)));
+#pragma unroll 8
+    for (int sp = 0; sp < n_split; ++sp) M = fmaxf(M, __ldcg(pp + sp * (hs + 2)));
     float L = 0.f;
-    for (int s = 0; s < n_split; ++s) L += exp2f(__ldcg(pp + s * (hs + 2)) - M) * __ldcg(pp + s * (hs + 2) + 1);
-    for (int d = threadIdx.x; d < hs; d += blockDim.x) {
-        float o = 0.f;
-        for (int s = 0; s < n_split; ++s) o += exp2f(__ldcg(pp + s * (hs + 2)) - M) * __ldcg(pp + s * (hs + 2) + 2 + d);
-        y[static_cast<long long>(b) * nh * hs + h * hs + d] = from_f<E>(o / L);
+#pragma unroll 8
+    for (int sp = 0; sp < n_split; ++sp) L += exp2f(__ldcg(pp + sp * (hs + 2)) - M) * __ldcg(pp + sp * (hs + 2) + 1);
+#pragma unroll
+    for (int j = 0; j < kMaxHs / 64; ++j) {
+        const int d = 2 * lane + 64 * j;
+        if (d < hs) {
+            float a0 = 0.f, a1 = 0.f;
+#pragma unroll 8
+            for (int sp = 0; sp < n_split; ++sp) {
+                const float wgt = exp2f(__ldcg(pp + sp * (hs + 2)) - M);
+                a0 = fmaf(wgt, __ldcg(pp + sp * (hs + 2) + 2 + d), a0);
+                a1 = fmaf(wgt, __ldcg(pp + sp * (hs + 2) + 3 + d), a1);
+            }
+            Pair<E>::st(yr + d, a0 / L, a1 / L);
+        }
     }
+    if (lane == 0) counter[bh] = 0;
 }
 
 // k and v of positions [0, T) from the c_attn output qkv [B, T, 3C] into a layer's cache
@@ -314,10 +509,13 @@ __global__ void copy_tokens_kernel(const int64_t* __restrict__ src, long long ld
     dst[b * ld_dst + t] = __ldcg(src + b * ld_src + t);
 }
 
-__global__ void set_pos_kernel(int* pos, int value, int add) {
+// Sets the decode position and clears the attention merge counters (after a prefill).
+__global__ void decode_reset_kernel(int* pos, int value, int* counter, int n_counter) {
     griddep_launch_dependents();
     griddep_wait();
-    *pos = add ? __ldcg(pos) + value : value;
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i == 0) *pos = value;
+    if (i < n_counter) counter[i] = 0;
 }
 
 // ---------------------------------------------------------------- sampling
@@ -329,104 +527,180 @@ GPT_DEVINL uint32_t fkey(float f) {
 }
 
 constexpr int kSampleThreads = 1024;
+constexpr int kSampleWarps = kSampleThreads / 32;
+constexpr int kSampleMaxV = 52 * 1024;  // the row in shared memory: 208 KB (plus 16 KB of tables)
 
 // Per row b: z = logits / temperature; keep z >= the top_k-th largest z (every z when
 // top_k <= 0 or >= V; ties at the threshold are all kept); p = exp(z - max z) over the kept;
 // choose the smallest index i with p_0 + ... + p_i > u[b] * sum(p).  The selection is made on
-// the raw logits (dividing by a positive temperature keeps their order).  The exponentials
-// are fp32; their sums are fp64, because with a flat distribution over tens of thousands of
-// entries one entry's share (~1/V) is not far above fp32 accumulation error.  Fixed-order
-// sums: thread j owns the contiguous range [j*chunk, (j+1)*chunk), and the per-thread sums
-// are scanned in thread order.
+// the raw logits (dividing by a positive temperature keeps their order).
+//
+// One CTA per row stages the row in shared memory (V <= kSampleMaxV) and, in the same pass,
+// counts the order-preserving 32-bit keys by their top 11 bits.  A scan from the top bin finds
+// the bin holding the top_k-th largest key; its members (few, for a top-k of a spread-out
+// row) are gathered and the remaining 21 bits found by bisection over them: the largest t with
+// count(key >= t) >= top_k is the k-th largest key itself.  (A bin with more than
+// kSampleCand members is bisected over the whole row instead.)  For the draw, warp w owns the
+// contiguous segment [w*seg, (w+1)*seg): the exponentials are fp32 and their sums fp64 (one
+// entry's share of a flat distribution over tens of thousands of entries is not far above
+// fp32 accumulation error).  Every thread adds the 32 segment sums in the same order, so
+// exactly one warp's [prefix, prefix + sum) holds u * total; that warp walks its segment 32
+// entries at a time with a warp scan.
+constexpr int kSampleBins = 2048;
+constexpr int kSampleCand = 2048;
+
+// Block-wide sum of per-thread counts with one barrier.  Three accumulators rotate: call n adds
+// into acc[n % 3] and clears acc[(n + 1) % 3], which no thread can still be reading (a thread
+// reads acc[(n - 1) % 3] before it reaches call n's barrier).  acc[0] and acc[1] start at 0.
+GPT_DEVINL uint32_t block_count(uint32_t c, uint32_t* acc, int& phase) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+    uint32_t* cur = acc + phase % 3;
+    if ((threadIdx.x & 31) == 0) atomicAdd(cur, c);
+    if (threadIdx.x == 0) acc[(phase + 1) % 3] = 0;
+    __syncthreads();
+    ++phase;
+    return *cur;
+}
+
 __global__ void __launch_bounds__(kSampleThreads)
     sample_kernel(const float* __restrict__ logits, long long ld_logits, int V, float temperature, int top_k,
                   const float* __restrict__ u, int64_t* __restrict__ out, long long ld_out) {
     griddep_launch_dependents();
     griddep_wait();
-    __shared__ uint32_t hist[256];
-    __shared__ uint32_t s_prefix, s_need;
-    __shared__ float s_f[kSampleThreads];
-    __shared__ double s_d[kSampleThreads];
-    __shared__ float s_max;
+    extern __shared__ __align__(16) float zs[];  // the row, V floats
+    __shared__ uint32_t hist[kSampleBins];
+    __shared__ uint32_t cand[kSampleCand];
+    __shared__ uint32_t s_acc[3], s_ncand, s_bin, s_need;
+    __shared__ uint32_t s_wtot[kSampleWarps];
+    __shared__ float s_wmax[kSampleWarps];
+    __shared__ double s_wsum[kSampleWarps];
     const int b = blockIdx.x;
     const float* lg = logits + b * ld_logits;
-    const int tid = threadIdx.x;
-    const int chunk = (V + kSampleThreads - 1) / kSampleThreads;
-    const int lo = min(V, tid * chunk), hi = min(V, lo + chunk);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const bool filter = top_k > 0 && top_k < V;
 
-    uint32_t thr_key = 0;  // key of the top_k-th largest logit (radix select, 8 bits a pass)
-    if (top_k > 0 && top_k < V) {
-        uint32_t prefix = 0, mask = 0, need = static_cast<uint32_t>(top_k);
-        for (int shift = 24; shift >= 0; shift -= 8) {
-            for (int i = tid; i < 256; i += kSampleThreads) hist[i] = 0;
-            __syncthreads();
-            for (int i = lo; i < hi; ++i) {
-                const uint32_t key = fkey(__ldcg(lg + i));
-                if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
-            }
-            __syncthreads();
-            if (tid == 0) {
-                uint32_t cum = 0;
-                int d = 255;
-                for (; d > 0; --d) {
-                    if (cum + hist[d] >= need) break;
-                    cum += hist[d];
-                }
-                s_prefix = prefix | (static_cast<uint32_t>(d) << shift);
-                s_need = need - cum;
-            }
-            __syncthreads();
-            prefix = s_prefix;
-            need = s_need;
-            mask |= 255u << shift;
-        }
-        thr_key = prefix;
-    }
+    for (int i = tid; i < kSampleBins; i += kSampleThreads) hist[i] = 0;
+    if (tid < 2) s_acc[tid] = 0;
+    if (tid == 0) s_ncand = 0;
+    __syncthreads();
     float mx = -INFINITY;
-    for (int i = lo; i < hi; ++i) mx = fmaxf(mx, __ldcg(lg + i) / temperature);
-    s_f[tid] = mx;
-    __syncthreads();
-    for (int w = kSampleThreads / 2; w > 0; w >>= 1) {
-        if (tid < w) s_f[tid] = fmaxf(s_f[tid], s_f[tid + w]);
-        __syncthreads();
+    for (int i = tid; i < V; i += kSampleThreads) {
+        const float v = __ldcg(lg + i);
+        zs[i] = v;
+        mx = fmaxf(mx, v);
+        if (filter) atomicAdd(&hist[fkey(v) >> 21], 1u);
     }
-    if (tid == 0) s_max = s_f[0];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if (lane == 0) s_wmax[warp] = mx;
     __syncthreads();
-    const float m = s_max;
-    double part = 0.0;
-    for (int i = lo; i < hi; ++i)
-        if (fkey(__ldcg(lg + i)) >= thr_key) part += static_cast<double>(expf(__ldcg(lg + i) / temperature - m));
-    s_d[tid] = part;
-    __syncthreads();
-    if (tid != 0) return;
-    double total = 0.0;
-    for (int j = 0; j < kSampleThreads; ++j) total += s_d[j];
-    const double target = static_cast<double>(__ldcg(u + b)) * total;
-    double cum = 0.0;
-    int j = 0;
-    for (; j < kSampleThreads - 1; ++j) {
-        if (cum + s_d[j] > target) break;
-        cum += s_d[j];
-    }
-    long long pick = -1, last_kept = -1;
-    for (int i = min(V, j * chunk), e = min(V, j * chunk + chunk); i < e; ++i) {
-        if (fkey(__ldcg(lg + i)) < thr_key) continue;
-        const float p = expf(__ldcg(lg + i) / temperature - m);
-        if (p > 0.f) last_kept = i;
-        cum += static_cast<double>(p);
-        if (cum > target && p > 0.f) {
-            pick = i;
-            break;
+    float lmax = s_wmax[0];
+    for (int w = 1; w < kSampleWarps; ++w) lmax = fmaxf(lmax, s_wmax[w]);
+    const float m = lmax / temperature;  // the largest z (division is monotone)
+
+    uint32_t thr_key = 0;  // key of the top_k-th largest logit
+    if (filter) {
+        // bins from the top: thread t holds bins 2047-2t and 2046-2t
+        const uint32_t h0 = hist[kSampleBins - 1 - 2 * tid], h1 = hist[kSampleBins - 2 - 2 * tid];
+        uint32_t incl = h0 + h1;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t n = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += n;
         }
+        if (lane == 31) s_wtot[warp] = incl;
+        __syncthreads();
+        uint32_t before = 0;
+        for (int w = 0; w < warp; ++w) before += s_wtot[w];
+        incl += before;
+        const uint32_t excl = incl - h0 - h1, need = static_cast<uint32_t>(top_k);
+        if (excl < need && incl >= need) {
+            const bool first = excl + h0 >= need;
+            s_bin = first ? kSampleBins - 1 - 2 * tid : kSampleBins - 2 - 2 * tid;
+            s_need = first ? need - excl : need - excl - h0;
+        }
+        __syncthreads();
+        const uint32_t bin = s_bin, need2 = s_need;
+        const uint32_t nbin = hist[bin];
+        int phase = 0;
+        uint32_t lo = bin << 21, hi = lo | ((1u << 21) - 1);  // invariant: count(key >= lo) >= need
+        if (nbin <= kSampleCand) {
+            for (int i = tid; i < V; i += kSampleThreads) {
+                const uint32_t key = fkey(zs[i]);
+                if ((key >> 21) == bin) cand[atomicAdd(&s_ncand, 1u)] = key;
+            }
+            __syncthreads();
+            for (int it = 0; it < 22 && lo < hi; ++it) {  // the range halves: 21 steps suffice
+                const uint32_t mid = lo + (hi - lo + 1) / 2;
+                uint32_t c = 0;
+                for (uint32_t i = tid; i < nbin; i += kSampleThreads) c += cand[i] >= mid;
+                if (block_count(c, s_acc, phase) >= need2) lo = mid;
+                else hi = mid - 1;
+            }
+        } else {
+            for (int it = 0; it < 22 && lo < hi; ++it) {
+                const uint32_t mid = lo + (hi - lo + 1) / 2;
+                uint32_t c = 0;
+                for (int i = tid; i < V; i += kSampleThreads) {
+                    const uint32_t key = fkey(zs[i]);
+                    c += (key >> 21) == bin && key >= mid;
+                }
+                if (block_count(c, s_acc, phase) >= need2) lo = mid;
+                else hi = mid - 1;
+            }
+        }
+        thr_key = lo;
     }
-    if (pick < 0) {
-        // rounding left the target at or past the end of range j: take the last kept index
-        // with nonzero probability at or before the end of that range
-        for (int i = min(V, j * chunk + chunk) - 1; i >= 0 && last_kept < 0; --i)
-            if (fkey(__ldcg(lg + i)) >= thr_key && expf(__ldcg(lg + i) / temperature - m) > 0.f) last_kept = i;
-        pick = last_kept < 0 ? 0 : last_kept;
+
+    // segment sums: lane-strided fp64 partials, then a butterfly
+    const int seg = ((V + kSampleWarps * 32 - 1) / (kSampleWarps * 32)) * 32;
+    const int s0 = min(V, warp * seg), s1 = min(V, s0 + seg);
+    double part = 0.0;
+    for (int i = s0 + lane; i < s1; i += 32) {
+        const float li = zs[i];
+        if (fkey(li) >= thr_key) part += static_cast<double>(expf(li / temperature - m));
     }
-    out[b * ld_out] = pick;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+    if (lane == 0) s_wsum[warp] = part;
+    __syncthreads();
+    double excl = 0.0, total = 0.0;
+    for (int w = 0; w < kSampleWarps; ++w) {
+        if (w == warp) excl = total;
+        total += s_wsum[w];
+    }
+    const double seg_sum = s_wsum[warp];
+    const double target = static_cast<double>(__ldcg(u + b)) * total;
+    if (!(seg_sum > 0.0 && excl <= target && target < excl + seg_sum)) return;
+    // this warp's segment holds the target: the first entry whose running sum passes it
+    double cum = excl;
+    long long last = -1;
+    for (int i0 = s0; i0 < s1; i0 += 32) {
+        const int i = i0 + lane;
+        double p = 0.0;
+        if (i < s1) {
+            const float li = zs[i];
+            if (fkey(li) >= thr_key) p = static_cast<double>(expf(li / temperature - m));
+        }
+        double c = p;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const double n = __shfl_up_sync(0xffffffffu, c, o);
+            if (lane >= o) c += n;
+        }
+        c += cum;
+        const uint32_t hit = __ballot_sync(0xffffffffu, p > 0.0 && c > target);
+        if (hit) {
+            if (lane == __ffs(hit) - 1) out[b * ld_out] = i;
+            return;
+        }
+        const uint32_t nz = __ballot_sync(0xffffffffu, p > 0.0);
+        if (nz) last = i0 + 31 - __clz(nz);
+        cum = __shfl_sync(0xffffffffu, c, 31);
+    }
+    // rounding left the target past the segment's running sum: its last entry with p > 0
+    if (lane == 0) out[b * ld_out] = last;
 }
 
 }  // namespace
@@ -443,34 +717,71 @@ int launch_embed_pos(const void* wte, const void* wpe, const int64_t* tok, long 
 }
 
 namespace {
+template <typename E, int EPI, int KSPLIT, int CPW, bool LN>
+int launch_gemv_inst(const GemvArgs<E>& a, cudaStream_t s) {
+    constexpr int kCols = (kGemvWarps / KSPLIT) * CPW;
+    const size_t smem = static_cast<size_t>(a.rows) * a.K * (sizeof(E) + (LN ? sizeof(float) : 0));
+    auto kern = gemv_kernel<E, EPI, KSPLIT, CPW, LN>;
+    static size_t configured = 0;  // dynamic shared memory this kernel is opted in for
+    if (smem > configured) {
+        const int rc = cuda_status(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                        static_cast<int>(smem)));
+        if (rc) return rc;
+        configured = smem;
+    }
+    return launch_overlapped(kern, dim3((a.N + kCols - 1) / kCols), dim3(kGemvThreads), smem, s, a);
+}
+
+// Warps per column: enough CTAs for narrow outputs, one with four columns a warp for the head.
+template <typename E, int EPI, bool LN>
+int launch_gemv_mode(const GemvArgs<E>& a, cudaStream_t s) {
+    if (a.N >= 16384) return launch_gemv_inst<E, EPI, 1, 4, LN>(a, s);
+    int ksplit = a.N <= 2048 ? 4 : 2;
+    while (ksplit > 1 && (a.K % (8 * ksplit))) ksplit >>= 1;
+    if (ksplit == 4) return launch_gemv_inst<E, EPI, 4, 1, LN>(a, s);
+    if (ksplit == 2) return launch_gemv_inst<E, EPI, 2, 1, LN>(a, s);
+    return launch_gemv_inst<E, EPI, 1, 1, LN>(a, s);
+}
+
 template <typename E>
-int gemv_typed(int epi, const E* x, long long ldx, const E* W, const E* bias, void* out, long long ldo, int B, int N,
-               int K, int gelu_tanh, E* kv, const int* pos, int C, int block_size, cudaStream_t s) {
-    const dim3 grid((N + kGemvWarps - 1) / kGemvWarps), block(kGemvWarps * 32);
+int gemv_typed(int epi, bool ln, const void* x, long long ldx, const E* ln_w, const E* ln_b, const E* W, const E* bias,
+               void* out, long long ldo, int B, int N, int K, int gelu_tanh, E* kv, int* pos, int C, int block_size,
+               int bump_pos, cudaStream_t s) {
+    const size_t in_es = ln ? 4 : sizeof(E);
     const size_t out_es = (epi == DV_RESID || epi == DV_F32) ? 4 : sizeof(E);
     for (int r0 = 0; r0 < B; r0 += kGemvRows) {
-        GemvArgs<E> a{x + r0 * ldx,
+        const int rows = min(kGemvRows, B - r0);
+        GemvArgs<E> a{static_cast<const uint8_t*>(x) + static_cast<size_t>(r0) * ldx * in_es,
                       ldx,
+                      ln_w,
+                      ln_b,
                       W,
                       bias,
                       static_cast<uint8_t*>(out) + static_cast<size_t>(r0) * ldo * out_es,
                       ldo,
-                      min(kGemvRows, B - r0),
+                      rows,
                       N,
                       K,
                       gelu_tanh,
                       kv ? kv + static_cast<long long>(r0) * block_size * 2 * C : nullptr,
                       pos,
                       C,
-                      block_size};
+                      block_size,
+                      (bump_pos && r0 + rows >= B) ? 1 : 0};
         int rc;
-        switch (epi) {
-            case DV_STORE: rc = launch_overlapped(gemv_kernel<E, DV_STORE>, grid, block, 0, s, a); break;
-            case DV_GELU: rc = launch_overlapped(gemv_kernel<E, DV_GELU>, grid, block, 0, s, a); break;
-            case DV_RESID: rc = launch_overlapped(gemv_kernel<E, DV_RESID>, grid, block, 0, s, a); break;
-            case DV_F32: rc = launch_overlapped(gemv_kernel<E, DV_F32>, grid, block, 0, s, a); break;
-            case DV_QKV: rc = launch_overlapped(gemv_kernel<E, DV_QKV>, grid, block, 0, s, a); break;
-            default: return GPT_ERR_UNSUPPORTED;
+        if (ln) {
+            switch (epi) {
+                case DV_GELU: rc = launch_gemv_mode<E, DV_GELU, true>(a, s); break;
+                case DV_F32: rc = launch_gemv_mode<E, DV_F32, true>(a, s); break;
+                case DV_QKV: rc = launch_gemv_mode<E, DV_QKV, true>(a, s); break;
+                default: return GPT_ERR_UNSUPPORTED;
+            }
+        } else {
+            switch (epi) {
+                case DV_RESID: rc = launch_gemv_mode<E, DV_RESID, false>(a, s); break;
+                case DV_F32: rc = launch_gemv_mode<E, DV_F32, false>(a, s); break;
+                default: return GPT_ERR_UNSUPPORTED;
+            }
         }
         if (rc) return rc;
     }
@@ -478,17 +789,17 @@ int gemv_typed(int epi, const E* x, long long ldx, const E* W, const E* bias, vo
 }
 }  // namespace
 
-int launch_gemv(int epi, int dtype, const void* x, long long ldx, const void* W, const void* bias, void* out,
-                long long ldo, int B, int N, int K, int gelu_tanh, void* kv, const int* pos, int C, int block_size,
-                cudaStream_t s) {
-    if (B < 1 || (K % 8)) return GPT_ERR_UNSUPPORTED;
+int launch_gemv(int epi, bool ln, int dtype, const void* x, long long ldx, const void* ln_w, const void* ln_b,
+                const void* W, const void* bias, void* out, long long ldo, int B, int N, int K, int gelu_tanh,
+                void* kv, int* pos, int C, int block_size, int bump_pos, cudaStream_t s) {
+    if (B < 1 || (K % 8) || (ln && (K % 4))) return GPT_ERR_UNSUPPORTED;
     if (dtype == GPT_DTYPE_BF16)
-        return gemv_typed<bf16>(epi, static_cast<const bf16*>(x), ldx, static_cast<const bf16*>(W),
-                                static_cast<const bf16*>(bias), out, ldo, B, N, K, gelu_tanh, static_cast<bf16*>(kv),
-                                pos, C, block_size, s);
-    return gemv_typed<float>(epi, static_cast<const float*>(x), ldx, static_cast<const float*>(W),
-                             static_cast<const float*>(bias), out, ldo, B, N, K, gelu_tanh, static_cast<float*>(kv),
-                             pos, C, block_size, s);
+        return gemv_typed<bf16>(epi, ln, x, ldx, static_cast<const bf16*>(ln_w), static_cast<const bf16*>(ln_b),
+                                static_cast<const bf16*>(W), static_cast<const bf16*>(bias), out, ldo, B, N, K,
+                                gelu_tanh, static_cast<bf16*>(kv), pos, C, block_size, bump_pos, s);
+    return gemv_typed<float>(epi, ln, x, ldx, static_cast<const float*>(ln_w), static_cast<const float*>(ln_b),
+                             static_cast<const float*>(W), static_cast<const float*>(bias), out, ldo, B, N, K,
+                             gelu_tanh, static_cast<float*>(kv), pos, C, block_size, bump_pos, s);
 }
 
 size_t decode_attn_part_floats(int B, int nh, int hs, int block_size) {
@@ -496,25 +807,19 @@ size_t decode_attn_part_floats(int B, int nh, int hs, int block_size) {
     return static_cast<size_t>(B) * nh * n_split_max * (hs + 2);
 }
 
-int launch_decode_attention(int dtype, const void* q, const void* kv, const int* pos, float* part, void* y, int B,
-                            int nh, int hs, int block_size, cudaStream_t s) {
+int launch_decode_attention(int dtype, const void* q, const void* kv, const int* pos, float* part, int* counter,
+                            void* y, int B, int nh, int hs, int block_size, cudaStream_t s) {
     if (hs > kMaxHs || (hs % 8)) return GPT_ERR_UNSUPPORTED;
     const int n_split_max = (block_size + kSplitKeys - 1) / kSplitKeys;
     const float scale_log2 = static_cast<float>(1.4426950408889634 / sqrt(static_cast<double>(hs)));
-    const dim3 g1(n_split_max, B * nh), b1(kSplitKeys), g2(B * nh), b2(64);
-    int rc;
-    if (dtype == GPT_DTYPE_BF16) {
-        rc = launch_overlapped(decode_attn_partial<bf16>, g1, b1, 0, s, static_cast<const bf16*>(q),
-                               static_cast<const bf16*>(kv), pos, part, nh, hs, block_size, n_split_max, scale_log2);
-        if (rc) return rc;
-        return launch_overlapped(decode_attn_combine<bf16>, g2, b2, 0, s, static_cast<const float*>(part), pos,
-                                 static_cast<bf16*>(y), nh, hs, block_size, n_split_max);
-    }
-    rc = launch_overlapped(decode_attn_partial<float>, g1, b1, 0, s, static_cast<const float*>(q),
-                           static_cast<const float*>(kv), pos, part, nh, hs, block_size, n_split_max, scale_log2);
-    if (rc) return rc;
-    return launch_overlapped(decode_attn_combine<float>, g2, b2, 0, s, static_cast<const float*>(part), pos,
-                             static_cast<float*>(y), nh, hs, block_size, n_split_max);
+    const dim3 grid(n_split_max, B * nh), block(kSplitKeys);
+    if (dtype == GPT_DTYPE_BF16)
+        return launch_overlapped(decode_attention_kernel<bf16>, grid, block, 0, s, static_cast<const bf16*>(q),
+                                 static_cast<const bf16*>(kv), pos, part, counter, static_cast<bf16*>(y), nh, hs,
+                                 block_size, n_split_max, scale_log2);
+    return launch_overlapped(decode_attention_kernel<float>, grid, block, 0, s, static_cast<const float*>(q),
+                             static_cast<const float*>(kv), pos, part, counter, static_cast<float*>(y), nh, hs,
+                             block_size, n_split_max, scale_log2);
 }
 
 int launch_kv_store(const void* qkv, void* kv, int B, int T, int C, int elem_bytes, int block_size, cudaStream_t s) {
@@ -535,14 +840,27 @@ int launch_copy_tokens(const int64_t* src, long long ld_src, int64_t* dst, long 
                              ld_src, dst, ld_dst, B, T);
 }
 
-int launch_set_pos(int* pos, int value, int add, cudaStream_t s) {
-    return launch_overlapped(set_pos_kernel, dim3(1), dim3(1), 0, s, pos, value, add);
+int launch_decode_reset(int* pos, int value, int* counter, int n_counter, cudaStream_t s) {
+    const int n = n_counter > 1 ? n_counter : 1;
+    return launch_overlapped(decode_reset_kernel, dim3((n + 255) / 256), dim3(256), 0, s, pos, value, counter,
+                             n_counter);
 }
+
+int sample_max_vocab() { return kSampleMaxV; }
 
 int launch_sample(const float* logits, long long ld_logits, int B, int V, float temperature, int top_k,
                   const float* u, int64_t* out, long long ld_out, cudaStream_t s) {
-    return launch_overlapped(sample_kernel, dim3(B), dim3(kSampleThreads), 0, s, logits, ld_logits, V, temperature,
-                             top_k, u, out, ld_out);
+    if (V > kSampleMaxV) return GPT_ERR_UNSUPPORTED;
+    static int configured = 0;  // dynamic shared memory the kernel is opted in for
+    const int smem = V * static_cast<int>(sizeof(float));
+    if (smem > configured) {
+        const int rc = cuda_status(cudaFuncSetAttribute(sample_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                        kSampleMaxV * static_cast<int>(sizeof(float))));
+        if (rc) return rc;
+        configured = kSampleMaxV * static_cast<int>(sizeof(float));
+    }
+    return launch_overlapped(sample_kernel, dim3(B), dim3(kSampleThreads), static_cast<size_t>(smem), s, logits,
+                             ld_logits, V, temperature, top_k, u, out, ld_out);
 }
 
 }  // namespace gpt

@@ -326,24 +326,32 @@ int check_common(const gpt_config_t* c, const void* weights, int B, int T, void*
 }
 
 // ------------------------------------------------------------------ incremental decoding
-// Workspace of the decoding entry points: the forward plan for a prefill of up to T_pref
-// positions (its buffers also hold the one-row-per-sequence activations of a decode step),
-// then the split-attention partials, fp32 logits [B, V] and a token window [B, block_size].
-// The control block keeps the status word at byte 0 and the decode position at byte 4.
+// Workspace of the decoding entry points.  The state that lives across calls, and the buffers
+// whose size does not depend on the prefill length, come first at fixed offsets (the control
+// block with the status word at byte 0 and the decode position at byte 4, the attention merge
+// counters, the split-attention partials, fp32 logits [B, V], a token window [B, block_size]);
+// then the forward plan for a prefill of up to T_pref positions, whose buffers also hold the
+// one-row-per-sequence activations of a decode step.  A prefill and the decode steps after it
+// may therefore size the workspace for different T_pref.
 struct DecodePlan {
     Plan P;
-    size_t part, logits, window, total;
+    size_t counter, part, logits, window, total;
 };
 
 DecodePlan plan_decode(const gpt_config_t* c, int B, int T_pref) {
     DecodePlan D;
-    D.P = plan_ws(c, B, T_pref);
-    size_t off = D.P.total;
     const int hs = c->n_embd / c->n_head;
+    size_t off = 256;
+    D.counter = off; off += a256(static_cast<size_t>(B) * c->n_head * 4);
     D.part = off; off += a256(decode_attn_part_floats(B, c->n_head, hs, c->block_size) * 4);
     D.logits = off; off += a256(static_cast<size_t>(B) * c->vocab_size * 4);
     D.window = off; off += a256(static_cast<size_t>(B) * c->block_size * 8);
-    D.total = off;
+    // the forward plan shares the control block at 0; its buffers move past the fixed region
+    Plan P = plan_ws(c, B, T_pref);
+    const size_t shift = off - 256;
+    for (size_t* f : {&P.x, &P.u, &P.qkv, &P.y, &P.h, &P.part, &P.tlogit, &P.rowloss, &P.total}) *f += shift;
+    D.P = P;
+    D.total = P.total;
     return D;
 }
 
@@ -387,9 +395,9 @@ int prefill_impl(const gpt_config_t* c, const Weights& W, const int64_t* idx, in
         GPT_TRY(run_block(c, W, l, x, B, T, ws, P, s, kv + kv_layer_bytes(c, B) * l));
     GPT_TRY(launch_layernorm(x, W.lnf_w(), W.lnf_b(), u, N, C, c->dtype, s));
     const uint8_t* ulast = static_cast<const uint8_t*>(u) + static_cast<size_t>(T - 1) * C * elem_size(c);
-    GPT_TRY(launch_gemv(3, c->dtype, ulast, static_cast<long long>(T) * C, W.wte(), nullptr, logits, ldl, B, V, C,
-                        c->gelu == GPT_GELU_TANH, nullptr, nullptr, C, c->block_size, s));
-    return launch_set_pos(pos_word(ws), T, 0, s);
+    GPT_TRY(launch_gemv(3, false, c->dtype, ulast, static_cast<long long>(T) * C, nullptr, nullptr, W.wte(), nullptr,
+                        logits, ldl, B, V, C, c->gelu == GPT_GELU_TANH, nullptr, nullptr, C, c->block_size, 0, s));
+    return launch_decode_reset(pos_word(ws), T, reinterpret_cast<int*>(ws + D.counter), B * c->n_head, s);
 }
 
 // One token per sequence (tok[b * ld_tok]) at the decode position p: every layer appends its
@@ -400,31 +408,30 @@ int decode_step_impl(const gpt_config_t* c, const Weights& W, const int64_t* tok
     const int dt = c->dtype, gt = c->gelu == GPT_GELU_TANH;
     const Plan& P = D.P;
     int32_t* status = status_word(ws);
-    const int* pos = pos_word(ws);
+    int* pos = pos_word(ws);
     float* x = reinterpret_cast<float*>(ws + P.x);
-    void* u = ws + P.u;
     void* q = ws + P.qkv;
     void* y = ws + P.y;
     void* h = ws + P.h;
     float* part = reinterpret_cast<float*>(ws + D.part);
+    int* counter = reinterpret_cast<int*>(ws + D.counter);
     GPT_TRY(launch_embed_pos(W.wte(), W.wpe(), tok, ld_tok, pos, x, B, C, V, bs, dt, status, s));
     for (int l = 0; l < c->n_layer; ++l) {
         uint8_t* kvl = kv + kv_layer_bytes(c, B) * l;
-        GPT_TRY(launch_layernorm(x, W.layer(l, W_LN1_W), W.bias(l, W_LN1_B), u, B, C, dt, s));
-        GPT_TRY(launch_gemv(4, dt, u, C, W.layer(l, W_ATTN_W), W.bias(l, W_ATTN_B), q, C, B, 3 * C, C, gt, kvl, pos,
-                            C, bs, s));
-        GPT_TRY(launch_decode_attention(dt, q, kvl, pos, part, y, B, nh, hs, bs, s));
-        GPT_TRY(launch_gemv(2, dt, y, C, W.layer(l, W_PROJ_W), W.bias(l, W_PROJ_B), x, C, B, C, C, gt, nullptr,
-                            nullptr, C, bs, s));
-        GPT_TRY(launch_layernorm(x, W.layer(l, W_LN2_W), W.bias(l, W_LN2_B), u, B, C, dt, s));
-        GPT_TRY(launch_gemv(1, dt, u, C, W.layer(l, W_FC_W), W.bias(l, W_FC_B), h, 4LL * C, B, 4 * C, C, gt,
-                            nullptr, nullptr, C, bs, s));
-        GPT_TRY(launch_gemv(2, dt, h, 4LL * C, W.layer(l, W_FC2_W), W.bias(l, W_FC2_B), x, C, B, C, 4 * C, gt,
-                            nullptr, nullptr, C, bs, s));
+        // q, k, v = c_attn(ln_1(x)); k, v appended to the cache at the position
+        GPT_TRY(launch_gemv(4, true, dt, x, C, W.layer(l, W_LN1_W), W.bias(l, W_LN1_B), W.layer(l, W_ATTN_W),
+                            W.bias(l, W_ATTN_B), q, C, B, 3 * C, C, gt, kvl, pos, C, bs, 0, s));
+        GPT_TRY(launch_decode_attention(dt, q, kvl, pos, part, counter, y, B, nh, hs, bs, s));
+        GPT_TRY(launch_gemv(2, false, dt, y, C, nullptr, nullptr, W.layer(l, W_PROJ_W), W.bias(l, W_PROJ_B), x, C,
+                            B, C, C, gt, nullptr, nullptr, C, bs, 0, s));
+        GPT_TRY(launch_gemv(1, true, dt, x, C, W.layer(l, W_LN2_W), W.bias(l, W_LN2_B), W.layer(l, W_FC_W),
+                            W.bias(l, W_FC_B), h, 4LL * C, B, 4 * C, C, gt, nullptr, nullptr, C, bs, 0, s));
+        GPT_TRY(launch_gemv(2, false, dt, h, 4LL * C, nullptr, nullptr, W.layer(l, W_FC2_W), W.bias(l, W_FC2_B), x,
+                            C, B, C, 4 * C, gt, nullptr, nullptr, C, bs, 0, s));
     }
-    GPT_TRY(launch_layernorm(x, W.lnf_w(), W.lnf_b(), u, B, C, dt, s));
-    GPT_TRY(launch_gemv(3, dt, u, C, W.wte(), nullptr, logits, ldl, B, V, C, gt, nullptr, nullptr, C, bs, s));
-    return launch_set_pos(pos_word(ws), 1, 1, s);
+    // logits = ln_f(x) wte^T; the same kernel advances the position
+    return launch_gemv(3, true, dt, x, C, W.lnf_w(), W.lnf_b(), W.wte(), nullptr, logits, ldl, B, V, C, gt, nullptr,
+                       pos, C, bs, 1, s);
 }
 
 // The widest prefill gpt_generate runs: the prompt (cropped to the window), or a full window
@@ -438,6 +445,7 @@ int check_sample_args(int B, int V, float temperature, const float* logits, cons
     if (!logits || !u || !out) return GPT_ERR_NULL;
     if (B < 1 || V < 1) return GPT_ERR_BAD_SHAPE;
     if (!(temperature > 0.f) || !isfinite(temperature)) return GPT_ERR_BAD_SHAPE;
+    if (V > sample_max_vocab()) return GPT_ERR_UNSUPPORTED;
     return GPT_OK;
 }
 
@@ -726,6 +734,7 @@ GPT_API int gpt_generate(const gpt_config_t* cfg, const void* weights, const int
     if (B < 1 || T0 < 1 || max_new_tokens < 0) return GPT_ERR_BAD_SHAPE;
     if (static_cast<long long>(T0) + max_new_tokens > 0x7fffffffLL) return GPT_ERR_BAD_SHAPE;
     if (max_new_tokens > 0 && (!(temperature > 0.f) || !isfinite(temperature))) return GPT_ERR_BAD_SHAPE;
+    if (max_new_tokens > 0 && cfg->vocab_size > sample_max_vocab()) return GPT_ERR_UNSUPPORTED;
     DecodePlan D;
     GPT_TRY(check_decode(cfg, weights, B, kv_cache, workspace, workspace_bytes,
                          generate_prefill_len(cfg, T0, max_new_tokens), &D));

@@ -97,18 +97,22 @@ int launch_attention_f32(const AttnLayoutF32& L, int B, int nh, int T, int hs, c
 // x[b, :] = wte[tok[b * ld_tok]] + wpe[*pos] (fp32 x [B, C]).
 int launch_embed_pos(const void* wte, const void* wpe, const int64_t* tok, long long ld_tok, const int* pos, float* x,
                      int B, int C, int V, int block_size, int dtype, int32_t* status, cudaStream_t s);
-// Matrix-vector products of B rows against W [N, K]; epi 0 store E, 1 gelu -> E, 2 fp32 +=,
-// 3 fp32 store, 4 qkv split (q -> out, k/v -> kv[b, *pos]).
-int launch_gemv(int epi, int dtype, const void* x, long long ldx, const void* W, const void* bias, void* out,
-                long long ldo, int B, int N, int K, int gelu_tanh, void* kv, const int* pos, int C, int block_size,
-                cudaStream_t s);
+// Matrix-vector products of B rows against W [N, K]; epi 1 gelu -> E, 2 fp32 +=, 3 fp32
+// store, 4 qkv split (q -> out, k/v -> kv[b, *pos]).  ln: the input is the fp32 residual
+// stream and LayerNorm(ln_w, ln_b) is applied to it first.  bump_pos: advance *pos by one.
+int launch_gemv(int epi, bool ln, int dtype, const void* x, long long ldx, const void* ln_w, const void* ln_b,
+                const void* W, const void* bias, void* out, long long ldo, int B, int N, int K, int gelu_tanh,
+                void* kv, int* pos, int C, int block_size, int bump_pos, cudaStream_t s);
 size_t decode_attn_part_floats(int B, int nh, int hs, int block_size);
-int launch_decode_attention(int dtype, const void* q, const void* kv, const int* pos, float* part, void* y, int B,
-                            int nh, int hs, int block_size, cudaStream_t s);
+// counter: B * nh ints, zero on entry and on return.
+int launch_decode_attention(int dtype, const void* q, const void* kv, const int* pos, float* part, int* counter,
+                            void* y, int B, int nh, int hs, int block_size, cudaStream_t s);
 int launch_kv_store(const void* qkv, void* kv, int B, int T, int C, int elem_bytes, int block_size, cudaStream_t s);
 int launch_copy_tokens(const int64_t* src, long long ld_src, int64_t* dst, long long ld_dst, int B, int T,
                        cudaStream_t s);
-int launch_set_pos(int* pos, int value, int add, cudaStream_t s);
+// *pos = value and counter[0, n_counter) = 0.
+int launch_decode_reset(int* pos, int value, int* counter, int n_counter, cudaStream_t s);
+int sample_max_vocab();  // largest V the sampling kernel takes (the row sits in shared memory)
 int launch_sample(const float* logits, long long ld_logits, int B, int V, float temperature, int top_k,
                   const float* u, int64_t* out, long long ld_out, cudaStream_t s);
 

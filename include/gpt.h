@@ -259,7 +259,8 @@ int gpt_decode_step(const gpt_config_t* cfg, const void* weights, const int64_t*
                     long long ld_tok, int B, void* kv_cache, float* logits, void* workspace,
                     size_t workspace_bytes, void* stream, int flags);
 
-/* The sampling step on logits fp32 [B, V]: temperature > 0 (GPT_ERR_BAD_SHAPE otherwise),
+/* The sampling step on logits fp32 [B, V] (V <= 53248: one row is staged in shared memory;
+ * GPT_ERR_UNSUPPORTED above that), temperature > 0 (GPT_ERR_BAD_SHAPE otherwise),
  * top_k <= 0 for no top-k filter, u fp32 [B] in [0, 1); writes out[b * ld_out] (int64).  The
  * top-k threshold is taken on the logits before the division (the same order for any
  * positive temperature).  Sums run in a fixed order; the result is deterministic. */

@@ -175,3 +175,11 @@ def test_generation_host_validation():
     # an unsupported head size for the decode kernels
     c2 = ctypes.byref(_cfg("tiny", n_head=32).c())                                   # hs 4
     assert Lb.gpt_prefill(c2, FAKE, FAKE, 1, 4, FAKE, FAKE, FAKE, big, None, 0) == native.GPT_ERR_UNSUPPORTED
+
+
+def test_sample_vocab_limit():
+    Lb = native.LIB
+    assert Lb.gpt_sample(FAKE, 2, 53248 + 1, 1.0, 0, FAKE, FAKE, 1, None) == native.GPT_ERR_UNSUPPORTED
+    c = ctypes.byref(_cfg("gpt2", vocab_size=60000).c())
+    assert Lb.gpt_generate(c, FAKE, FAKE, 1, 4, 2, 1.0, 0, FAKE, FAKE, None, FAKE, FAKE, 1 << 40, None, 0) \
+        == native.GPT_ERR_UNSUPPORTED
