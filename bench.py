@@ -45,6 +45,10 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-kernels", action="store_true", help="skip the per-kernel timings")
+    ap.add_argument("--decode-only", action="store_true",
+                    help="run only the decode measurement (--steps graph replays after --warmup) and print it; "
+                         "with --no-e2e the generate call is skipped (for profiler captures)")
+    ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--profile-kernel", default=None,
                     help="launch only this kernel of the forward (names as in kernels_ms_per_forward): "
                          "--warmup untimed then --steps timed launches; for profiler captures")
@@ -295,12 +299,113 @@ def kernel_timings(w, native, dev, stream):
     return out
 
 
+def decode_bench(model, native, dev, stream, peaks, peak_src, steps: int = 64, warmup: int = 8, e2e: bool = True):
+    """Incremental decoding of the same model ("nanoGPT 全局流程图", 第五阶段 generate with a key/value
+    cache): one step = gpt_decode_step + gpt_sample (temperature 0.8, top_k 200, the pages'
+    sample settings) for every sequence of the batch, replayed from a captured CUDA graph after a
+    512-token prefill.  Each step streams the 0.25 GB of weights, more than the 126 MB L2, so no
+    flush is needed.  The HBM roofline counts the bytes a step must move: every weight once
+    (wte once for the head, one wpe row), the cache rows read and the new k/v rows written, and
+    the fp32 logits written and read by the sampler."""
+    cfg = model.cfg
+    C, L, V, bs = cfg.n_embd, cfg.n_layer, cfg.vocab_size, cfg.block_size
+    T0 = 512
+    out = {"workload": f"GPT-2 124M bf16 decode after a {T0}-token prompt, temperature 0.8, top_k 200, "
+                       f"{steps} steps replayed from a CUDA graph (decode step + sampling)"}
+    entries, total = native.weights_layout(cfg)
+    wpe_bytes = dict((n, k) for n, _, k in entries)["wpe"] * 2
+    for B in (1, 16):
+        prompt, _ = seeded.make_tokens(B, T0, 50257, seed=seeded.BASE_SEED + 600_000)
+        kv = native.alloc_kv_cache(cfg, B, dev)
+        ws = native.alloc_workspace(native.decode_workspace_bytes(cfg, B, T0), dev)
+        logits = torch.empty((B, V), device=dev)
+        tok = torch.zeros(B, dtype=torch.int64, device=dev)
+        u = torch.rand(B, device=dev, generator=torch.Generator(device=dev).manual_seed(5))
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        native.prefill(cfg, model.weights, prompt.to(dev), kv, ws, sync_check=True)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(g, stream=side):
+                native.decode_step(cfg, model.weights, tok, kv, ws, logits=logits, stream=side)
+                native.sample(logits, u, 0.8, 200, out=tok, stream=side)
+        torch.cuda.synchronize()
+        native.prefill(cfg, model.weights, prompt.to(dev), kv, ws, sync_check=True)
+        for _ in range(warmup):
+            g.replay()
+        torch.cuda.synchronize()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for _ in range(steps):
+            g.replay()
+        s1.record(stream)
+        torch.cuda.synchronize()
+        ms = s0.elapsed_time(s1) / steps
+        status = native.check_status(ws)
+        del g
+        # positions T0 + warmup .. T0 + warmup + steps - 1: the mean cache length read per step
+        mean_keys = T0 + warmup + (steps - 1) / 2 + 1
+        bytes_step = (total - wpe_bytes + C * 2) + B * L * (mean_keys * 2 * C * 2 + 2 * C * 2) + B * V * 4 * 2
+        gbs = bytes_step / (ms / 1000.0) / 1e9
+        out[f"B{B}"] = {"tokens_per_s": B / (ms / 1000.0), "ms_per_token_step": ms,
+                        "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                     "frac": gbs / peaks["hbm_gbs"], "bytes_per_step": bytes_step,
+                                     "peak_source": peak_src},
+                        "status": native.status_string(status)}
+    if not e2e:
+        return out
+    # end to end: the public generate call from host buffers, 500 new tokens ("nanoGPT 核心代码速查表",
+    # sample.py settings), one sequence
+    B, n_new = 1, 500
+    prompt_h = torch.zeros((B, 1), dtype=torch.int64).pin_memory()
+    u_h = torch.rand((n_new, B), generator=torch.Generator().manual_seed(7)).pin_memory()
+    toks_h = torch.empty((B, 1 + n_new), dtype=torch.int64).pin_memory()
+    kv = native.alloc_kv_cache(cfg, B, dev)
+    ws = native.alloc_workspace(native.generate_workspace_bytes(cfg, B, 1, n_new), dev)
+    p_d = torch.empty((B, 1), dtype=torch.int64, device=dev)
+    u_d = torch.empty((n_new, B), device=dev)
+    o_d = torch.empty((B, 1 + n_new), dtype=torch.int64, device=dev)
+
+    def gen():
+        p_d.copy_(prompt_h, non_blocking=True)
+        u_d.copy_(u_h, non_blocking=True)
+        native.generate(cfg, model.weights, p_d, n_new, u_d, 0.8, 200, kv_cache=kv, workspace=ws, out=o_d)
+        toks_h.copy_(o_d, non_blocking=True)
+        stream.synchronize()
+
+    gen()
+    t0 = time.perf_counter()
+    reps = 3
+    for _ in range(reps):
+        gen()
+    dt = (time.perf_counter() - t0) / reps
+    out["generate_e2e"] = {"tokens_per_s": B * n_new / dt, "ms_per_call": dt * 1000.0, "new_tokens": n_new,
+                           "batch": B, "prompt": 1,
+                           "note": "host wall clock around gpt_generate with pinned host copies in and out; "
+                                   "launched eagerly (no graph), one launch sequence per token"}
+    return out
+
+
+def decode_only(args):
+    from decoder_only_transformer_causal_b200 import GPT, GPTConfig, native
+    dev = torch.device("cuda", 0)
+    w = seeded.WORKLOADS[WORKLOAD]
+    model = GPT(GPTConfig.from_dict(w.model_dict()), seeded.make_weights(w.model_dict(), device=str(dev)), dev)
+    peaks, peak_src = load_peaks()
+    d = decode_bench(model, native, dev, torch.cuda.current_stream(dev), peaks, peak_src, steps=args.steps,
+                     warmup=max(3, args.warmup), e2e=not args.no_e2e)
+    print(json.dumps({"decode": d}), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
     if args.profile_kernel:
         return profile_kernel(args)
+    if args.decode_only:
+        return decode_only(args)
     assert args.warmup >= 3, "at least 3 warm-up steps"
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -436,6 +541,8 @@ def main():
                              "tflops": a_tf, "ms": a["ms"], "frac_of_bf16_peak": a_tf / peaks["bf16_tflops"],
                              "flops": a["work"], "peak_source": peak_src}
         line["kernels_ms_per_forward"] = {k: round(v, 4) for k, v in share.items()}
+    if rank == 0 and not args.no_kernels:
+        line["decode"] = decode_bench(model, native, dev, stream, peaks, peak_src)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         times, threads = oracle_sample(w, 256, budget_s=12.0)
         tok_s = 256 * len(times) / sum(times)
