@@ -49,6 +49,8 @@ def parse():
                     help="run only the decode measurement (--steps graph replays after --warmup) and print it; "
                          "with --no-e2e the generate call is skipped (for profiler captures)")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--adamw-only", action="store_true",
+                    help="run only the optimizer-step measurement (--steps timed after --warmup) and print it")
     ap.add_argument("--profile-kernel", default=None,
                     help="launch only this kernel of the forward (names as in kernels_ms_per_forward): "
                          "--warmup untimed then --steps timed launches; for profiler captures")
@@ -386,6 +388,62 @@ def decode_bench(model, native, dev, stream, peaks, peak_src, steps: int = 64, w
     return out
 
 
+def adamw_bench(model, native, dev, stream, peaks, peak_src, steps: int = 20, warmup: int = 3):
+    """One optimizer step over GPT-2 124M ("nanoGPT 全局流程图" 3.6 and 优化器配置): the global
+    gradient norm, clipping to 1.0, AdamW (betas 0.9/0.95, weight decay 0.1 on matrices) on fp32
+    master parameters and moments, and the bf16 copy into the packed weights the forward reads.
+    Gradients are seeded N(0, 0.05^2) (norm ~560: clipping active).  Algorithmic traffic per
+    parameter: 4 B (norm: read g) + 16 B (read p, g, m, v) + 12 B (write p, m, v) + 2 B (bf16
+    copy) = 34 B; the 2 GB of fp32 arrays exceed the 126 MB L2, so no flush is needed."""
+    cfg = model.cfg
+    g = torch.randn(native.param_elems(cfg), device=dev, generator=torch.Generator(device=dev).manual_seed(11))
+    g.mul_(0.05)
+    entries, _ = native.weights_layout(cfg)
+    n_params = sum(k for _, _, k in entries)
+    p = torch.zeros_like(g)
+    es = 2
+    for name, off, numel in entries:       # master copy of the current weights
+        p[off // es: off // es + numel] = model.weights[off: off + numel * es].view(torch.bfloat16).float()
+    m = torch.zeros_like(g)
+    v = torch.zeros_like(g)
+    ws = native.alloc_workspace(native.LIB.gpt_adamw_workspace_bytes(), dev)
+    norm = torch.empty((), device=dev)
+    native.adamw_step(cfg, p, g, m, v, 1, 6e-4, weights=model.weights, grad_norm=norm, workspace=ws,
+                      sync_check=True)
+    for i in range(warmup):
+        native.adamw_step(cfg, p, g, m, v, 2 + i, 6e-4, weights=model.weights, grad_norm=norm, workspace=ws)
+    torch.cuda.synchronize()
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s0.record(stream)
+    for i in range(steps):
+        native.adamw_step(cfg, p, g, m, v, 2 + warmup + i, 6e-4, weights=model.weights, grad_norm=norm,
+                          workspace=ws)
+    s1.record(stream)
+    torch.cuda.synchronize()
+    ms = s0.elapsed_time(s1) / steps
+    bytes_step = 34 * n_params
+    gbs = bytes_step / (ms / 1000.0) / 1e9
+    return {"workload": "AdamW step over GPT-2 124M (124,475,904 fp32 parameters): grad norm + clip 1.0 + "
+                        "update + bf16 copy into the packed weights",
+            "ms_per_step": ms, "params_per_s": n_params / (ms / 1000.0),
+            "grad_norm": float(norm),
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / peaks["hbm_gbs"], "bytes_per_step": bytes_step, "peak_source": peak_src},
+            "gpu_launches_per_step": 2}
+
+
+def adamw_only(args):
+    from decoder_only_transformer_causal_b200 import GPT, GPTConfig, native
+    dev = torch.device("cuda", 0)
+    w = seeded.WORKLOADS[WORKLOAD]
+    model = GPT(GPTConfig.from_dict(w.model_dict()), seeded.make_weights(w.model_dict(), device=str(dev)), dev)
+    peaks, peak_src = load_peaks()
+    d = adamw_bench(model, native, dev, torch.cuda.current_stream(dev), peaks, peak_src, steps=args.steps,
+                    warmup=max(3, args.warmup))
+    print(json.dumps({"adamw": d}), flush=True)
+    return 0
+
+
 def decode_only(args):
     from decoder_only_transformer_causal_b200 import GPT, GPTConfig, native
     dev = torch.device("cuda", 0)
@@ -406,6 +464,8 @@ def main():
         return profile_kernel(args)
     if args.decode_only:
         return decode_only(args)
+    if args.adamw_only:
+        return adamw_only(args)
     assert args.warmup >= 3, "at least 3 warm-up steps"
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -543,6 +603,7 @@ def main():
         line["kernels_ms_per_forward"] = {k: round(v, 4) for k, v in share.items()}
     if rank == 0 and not args.no_kernels:
         line["decode"] = decode_bench(model, native, dev, stream, peaks, peak_src)
+        line["adamw"] = adamw_bench(model, native, dev, stream, peaks, peak_src)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         times, threads = oracle_sample(w, 256, budget_s=12.0)
         tok_s = 256 * len(times) / sum(times)

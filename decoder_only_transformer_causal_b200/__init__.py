@@ -12,7 +12,7 @@ import torch
 from . import native
 from .native import GPTConfig, GPTError  # noqa: F401
 
-__all__ = ["GPT", "GPTConfig", "GPTError", "native"]
+__all__ = ["GPT", "GPTConfig", "GPTError", "AdamW", "native"]
 
 
 class GPT:
@@ -84,4 +84,32 @@ class GPT:
         ws = native.alloc_workspace(native.generate_workspace_bytes(self.cfg, B, T0, max_new_tokens), self.device)
         return native.generate(self.cfg, self.weights, idx, max_new_tokens, uniforms, temperature, top_k,
                                kv_cache=self._host[key], workspace=ws, step_logits=step_logits)
+
+
+class AdamW:
+    """Optimizer state for a GPT's packed parameters ("nanoGPT 全局流程图", 3.5 and 3.6,
+    优化器配置): fp32 master parameters and both Adam moments as flat device arrays in the packed
+    element layout, the schedule of get_lr, clipping to max_grad_norm, weight decay on the
+    two-dimensional tensors.  ``step(grads)`` takes a flat fp32 gradient array in the same layout
+    and writes the updated parameters into the model's packed weights."""
+
+    def __init__(self, model: GPT, tensors: dict, learning_rate=6e-4, min_lr=6e-5, warmup_iters=2000,
+                 lr_decay_iters=600000, betas=(0.9, 0.95), eps=1e-8, weight_decay=0.1, max_grad_norm=1.0):
+        self.model = model
+        self.params = native.flat_params(model.cfg, tensors, model.device)
+        self.exp_avg = torch.zeros_like(self.params)
+        self.exp_avg_sq = torch.zeros_like(self.params)
+        self.workspace = native.alloc_workspace(native.LIB.gpt_adamw_workspace_bytes(), model.device)
+        self.grad_norm = torch.empty((), dtype=torch.float32, device=model.device)
+        self.schedule = (learning_rate, min_lr, warmup_iters, lr_decay_iters)
+        self.betas, self.eps, self.weight_decay, self.max_grad_norm = betas, eps, weight_decay, max_grad_norm
+        self.it = 0
+
+    def step(self, grads: torch.Tensor) -> torch.Tensor:
+        lr = native.lr_schedule(self.it, *self.schedule)
+        self.it += 1
+        return native.adamw_step(self.model.cfg, self.params, grads, self.exp_avg, self.exp_avg_sq, self.it, lr,
+                                 weights=self.model.weights, betas=self.betas, eps=self.eps,
+                                 weight_decay=self.weight_decay, max_grad_norm=self.max_grad_norm,
+                                 grad_norm=self.grad_norm, workspace=self.workspace)
 

@@ -766,3 +766,71 @@ GPT_API int gpt_generate(const gpt_config_t* cfg, const void* weights, const int
     if (flags & GPT_FLAG_SYNC_CHECK) return sync_and_read_status(ws, s);
     return GPT_OK;
 }
+
+// ------------------------------------------------------------------ optimizer step (optim.cu)
+GPT_API double gpt_lr_schedule(long long it, double learning_rate, double min_lr, long long warmup_iters,
+                               long long lr_decay_iters) {
+    if (it < warmup_iters) return learning_rate * static_cast<double>(it + 1) / static_cast<double>(warmup_iters + 1);
+    if (it > lr_decay_iters) return min_lr;
+    const double decay_ratio =
+        static_cast<double>(it - warmup_iters) / static_cast<double>(lr_decay_iters - warmup_iters);
+    const double coeff = 0.5 * (1.0 + cos(3.14159265358979323846 * decay_ratio));
+    return min_lr + coeff * (learning_rate - min_lr);
+}
+
+GPT_API size_t gpt_param_elems(const gpt_config_t* cfg) {
+    if (validate(cfg) != GPT_OK) return 0;
+    return weights_total(cfg) / elem_size(cfg);
+}
+
+GPT_API size_t gpt_adamw_workspace_bytes(void) { return adamw_workspace_bytes(); }
+
+GPT_API int gpt_adamw_step(const gpt_config_t* cfg, float* params, const float* grads, float* exp_avg,
+                           float* exp_avg_sq, void* weights, const gpt_adamw_t* hp, float* grad_norm,
+                           void* workspace, size_t workspace_bytes, void* stream, int flags) {
+    GPT_TRY(validate(cfg));
+    if (!params || !grads || !exp_avg || !exp_avg_sq || !hp || !workspace) return GPT_ERR_NULL;
+    if (hp->step < 1 || !(hp->lr >= 0.f) || !isfinite(hp->lr) || !(hp->beta1 >= 0.f && hp->beta1 < 1.f) ||
+        !(hp->beta2 >= 0.f && hp->beta2 < 1.f) || !(hp->eps > 0.f) || !(hp->weight_decay >= 0.f) ||
+        !isfinite(hp->max_grad_norm))
+        return GPT_ERR_BAD_SHAPE;
+    if (workspace_bytes < adamw_workspace_bytes()) return GPT_ERR_WS_TOO_SMALL;
+    if (!aligned(params, 16) || !aligned(grads, 16) || !aligned(exp_avg, 16) || !aligned(exp_avg_sq, 16) ||
+        !aligned(workspace, 256) || (weights && !aligned(weights, 256)) || (grad_norm && !aligned(grad_norm, 4)))
+        return GPT_ERR_BAD_ALIGN;
+    const int count = 2 + kTensorsPerLayer * cfg->n_layer + 2;
+    if (count > kOptMaxTensors) return GPT_ERR_UNSUPPORTED;
+    static thread_local OptTable tab;  // ~25 KB: not on the stack
+    size_t offs[kOptMaxTensors], numels[kOptMaxTensors];
+    layout(cfg, offs, numels, count);
+    const long long ch = opt_chunk_elems();
+    long long chunks = 0;
+    int n = 0;
+    for (int i = 0; i < count; ++i) {
+        // configure_optimizers: decay iff the tensor has two dimensions (wte, wpe, the four
+        // Linear weights of a layer).  Without biases (cfg->bias == 0) the bias slots are not
+        // parameters: they are skipped like padding.
+        bool two_d = i < 2, is_bias = i == count - 1;
+        if (i >= 2 && i < 2 + kTensorsPerLayer * cfg->n_layer) {
+            const int j = (i - 2) % kTensorsPerLayer;
+            two_d = j == W_ATTN_W || j == W_PROJ_W || j == W_FC_W || j == W_FC2_W;
+            is_bias = j == W_LN1_B || j == W_ATTN_B || j == W_PROJ_B || j == W_LN2_B || j == W_FC_B || j == W_FC2_B;
+        }
+        if (is_bias && !cfg->bias) continue;
+        tab.off[n] = static_cast<long long>(offs[i] / elem_size(cfg));
+        tab.numel[n] = static_cast<long long>(numels[i]);
+        if (tab.numel[n] % 4) return GPT_ERR_UNSUPPORTED;  // float4 rows
+        tab.decay[n] = two_d ? 1 : 0;
+        tab.chunk0[n] = chunks;
+        chunks += (tab.numel[n] + ch - 1) / ch;
+        ++n;
+    }
+    tab.n = n;
+    tab.chunk0[n] = chunks;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    GPT_TRY(launch_adamw(tab, cfg->dtype, params, grads, exp_avg, exp_avg_sq, weights, hp->lr, hp->beta1, hp->beta2,
+                         hp->eps, hp->weight_decay, hp->step, hp->max_grad_norm, grad_norm, workspace, s));
+    if (flags & GPT_FLAG_SYNC_CHECK) return cuda_status(cudaStreamSynchronize(s));
+    return GPT_OK;
+}
+

@@ -116,4 +116,22 @@ int sample_max_vocab();  // largest V the sampling kernel takes (the row sits in
 int launch_sample(const float* logits, long long ld_logits, int B, int V, float temperature, int top_k,
                   const float* u, int64_t* out, long long ld_out, cudaStream_t s);
 
+// ---- optimizer step (optim.cu)
+constexpr int kOptMaxTensors = 1024;
+// The packed tensors in element units: tensor i spans [off[i], off[i] + numel[i]) of the flat
+// fp32 arrays, is cut into chunks starting at chunk index chunk0[i] (chunk0[n] = total), and
+// takes weight decay iff decay[i].
+struct OptTable {
+    int n;
+    long long off[kOptMaxTensors];
+    long long numel[kOptMaxTensors];
+    long long chunk0[kOptMaxTensors + 1];
+    unsigned char decay[kOptMaxTensors];
+};
+long long opt_chunk_elems();
+size_t adamw_workspace_bytes();
+int launch_adamw(const OptTable& tab, int dtype, float* params, const float* grads, float* m, float* v, void* copy,
+                 float lr, float beta1, float beta2, float eps, float weight_decay, int step, float max_norm,
+                 float* norm_out, void* ws, cudaStream_t s);
+
 }  // namespace gpt

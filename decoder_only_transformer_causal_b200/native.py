@@ -52,6 +52,12 @@ class gpt_config_t(ctypes.Structure):
                 ("n_layer", "n_head", "n_embd", "block_size", "vocab_size", "bias", "dtype", "gelu")]
 
 
+class gpt_adamw_t(ctypes.Structure):
+    _fields_ = [("lr", ctypes.c_float), ("beta1", ctypes.c_float), ("beta2", ctypes.c_float),
+                ("eps", ctypes.c_float), ("weight_decay", ctypes.c_float), ("max_grad_norm", ctypes.c_float),
+                ("step", ctypes.c_int32)]
+
+
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"{LIB_PATH} is missing: build it with "
@@ -86,6 +92,10 @@ def _load() -> ctypes.CDLL:
         "gpt_decode_step": (I, [CFG, P, P, L, I, P, P, P, Z, P, I]),
         "gpt_sample": (I, [P, I, I, F, I, P, P, L, P]),
         "gpt_generate": (I, [CFG, P, P, I, I, I, F, I, P, P, P, P, P, Z, P, I]),
+        "gpt_lr_schedule": (ctypes.c_double, [L, ctypes.c_double, ctypes.c_double, L, L]),
+        "gpt_param_elems": (Z, [CFG]),
+        "gpt_adamw_workspace_bytes": (Z, []),
+        "gpt_adamw_step": (I, [CFG, P, P, P, P, P, ctypes.POINTER(gpt_adamw_t), P, P, Z, P, I]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -101,7 +111,8 @@ EXPORTED = ("gpt_status_string", "gpt_abi_version", "gpt_last_cuda_error", "gpt_
             "gpt_forward", "gpt_block", "gpt_attention", "gpt_embed", "gpt_layernorm", "gpt_linear",
             "gpt_lm_head_workspace_bytes", "gpt_lm_head_loss", "gpt_lm_head_loss_noalloc",
             "gpt_kv_cache_bytes", "gpt_decode_workspace_bytes", "gpt_generate_workspace_bytes", "gpt_prefill",
-            "gpt_decode_step", "gpt_sample", "gpt_generate")
+            "gpt_decode_step", "gpt_sample", "gpt_generate", "gpt_lr_schedule", "gpt_param_elems",
+            "gpt_adamw_workspace_bytes", "gpt_adamw_step")
 
 
 def status_string(status: int) -> str:
@@ -412,4 +423,55 @@ def generate(cfg: GPTConfig, weights: torch.Tensor, idx: torch.Tensor, max_new_t
                             _ptr(kv_cache), _ptr(workspace), workspace.numel(), _stream(stream),
                             GPT_FLAG_SYNC_CHECK if sync_check else 0), "gpt_generate")
     return out
+
+
+# ---------------------------------------------------------------- optimizer step
+def lr_schedule(it: int, learning_rate: float = 6e-4, min_lr: float = 6e-5, warmup_iters: int = 2000,
+                lr_decay_iters: int = 600000) -> float:
+    """gpt_lr_schedule: get_lr(it) of the pages (host function)."""
+    return LIB.gpt_lr_schedule(int(it), float(learning_rate), float(min_lr), int(warmup_iters), int(lr_decay_iters))
+
+
+def param_elems(cfg: GPTConfig) -> int:
+    return LIB.gpt_param_elems(ctypes.byref(cfg.c()))
+
+
+def flat_params(cfg: GPTConfig, tensors: dict, device="cuda") -> torch.Tensor:
+    """fp32 [param_elems] in the packed element layout (tensor i at byte offset / element size);
+    absent tensors (biases when cfg.bias is False) and the padding stay zero."""
+    entries, _ = weights_layout(cfg)
+    es = 2 if cfg.dtype == "bf16" else 4
+    buf = torch.zeros(param_elems(cfg), dtype=torch.float32, device=device)
+    for name, off, numel in entries:
+        t = tensors.get(name)
+        if t is None:
+            continue
+        buf[off // es: off // es + numel].copy_(t.reshape(-1).to(torch.float32))
+    return buf
+
+
+def unflatten(cfg: GPTConfig, flat: torch.Tensor, shapes: dict) -> dict:
+    """Views of a flat fp32 array per tensor name (names in `shapes` only)."""
+    entries, _ = weights_layout(cfg)
+    es = 2 if cfg.dtype == "bf16" else 4
+    return {name: flat[off // es: off // es + numel].view(shapes[name])
+            for name, off, numel in entries if name in shapes}
+
+
+def adamw_step(cfg: GPTConfig, params: torch.Tensor, grads: torch.Tensor, exp_avg: torch.Tensor,
+               exp_avg_sq: torch.Tensor, step: int, lr: float, weights: torch.Tensor | None = None,
+               betas=(0.9, 0.95), eps: float = 1e-8, weight_decay: float = 0.1, max_grad_norm: float = 1.0,
+               grad_norm: torch.Tensor | None = None, workspace: torch.Tensor | None = None, stream=None,
+               sync_check=False):
+    """gpt_adamw_step on flat fp32 arrays; returns the device grad-norm tensor."""
+    if workspace is None:
+        workspace = alloc_workspace(LIB.gpt_adamw_workspace_bytes(), params.device)
+    if grad_norm is None:
+        grad_norm = torch.empty((), dtype=torch.float32, device=params.device)
+    hp = gpt_adamw_t(float(lr), float(betas[0]), float(betas[1]), float(eps), float(weight_decay),
+                     float(max_grad_norm), int(step))
+    _check(LIB.gpt_adamw_step(ctypes.byref(cfg.c()), _ptr(params), _ptr(grads), _ptr(exp_avg), _ptr(exp_avg_sq),
+                              _ptr(weights), ctypes.byref(hp), _ptr(grad_norm), _ptr(workspace), workspace.numel(),
+                              _stream(stream), GPT_FLAG_SYNC_CHECK if sync_check else 0), "gpt_adamw_step")
+    return grad_norm
 

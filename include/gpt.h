@@ -280,6 +280,47 @@ int gpt_generate(const gpt_config_t* cfg, const void* weights, const int64_t* id
                  int64_t* out, float* step_logits, void* kv_cache, void* workspace,
                  size_t workspace_bytes, void* stream, int flags);
 
+/* ---- optimizer step -------------------------------------------------------------------
+ * "nanoGPT 全局流程图", 3.5 学习率调度, 3.6 梯度裁剪 + 参数更新 and 优化器配置; "nanoGPT 代码解析",
+ * configure_optimizers.  One training step's update of every parameter: the gradients are
+ * scaled by min(1, max_grad_norm / (||g||_2 + 1e-6)) with ||g||_2 the norm over ALL gradient
+ * entries (torch.nn.utils.clip_grad_norm_), then torch.optim.AdamW's update with decoupled weight
+ * decay, applied with weight_decay to the tensors of two dimensions (wte, wpe and each layer's
+ * four Linear weights) and with none to the rest (biases, LayerNorm weights and biases). */
+
+/* get_lr(it): linear warm-up to learning_rate over warmup_iters, cosine decay to min_lr at
+ * lr_decay_iters, min_lr afterwards (the page's curve; its listing stops at the cosine).  The
+ * page's values: 6e-4, 6e-5, 2000, 600000.  Host function. */
+double gpt_lr_schedule(long long it, double learning_rate, double min_lr, long long warmup_iters,
+                       long long lr_decay_iters);
+
+typedef struct gpt_adamw {
+    float lr;             /* this step's learning rate (gpt_lr_schedule) */
+    float beta1, beta2;   /* 0.9, 0.95 on the page */
+    float eps;            /* 1e-8 (torch's default; the page does not set it) */
+    float weight_decay;   /* 0.1 on the page; applied to two-dimensional tensors only */
+    float max_grad_norm;  /* 1.0 on the page; <= 0 disables clipping */
+    int32_t step;         /* optimizer steps taken including this one, >= 1 (bias corrections) */
+} gpt_adamw_t;
+
+/* Elements of each flat fp32 optimizer array: gpt_weights_bytes(cfg) / element size of
+ * cfg->dtype.  Tensor i of gpt_weights_layout sits at element offset offsets[i] / element size;
+ * the padding between tensors, and the bias slots when cfg->bias == 0, are never read or
+ * written. */
+size_t gpt_param_elems(const gpt_config_t* cfg);
+size_t gpt_adamw_workspace_bytes(void);   /* scratch of gpt_adamw_step, 256-byte aligned */
+
+/* params, grads, exp_avg, exp_avg_sq: fp32 [gpt_param_elems(cfg)], 16-byte aligned; params and
+ * both moments are updated in place (moments start at zero before step 1).  weights: the packed
+ * buffer in cfg->dtype that the forward reads, or NULL; when given, each updated parameter is
+ * also written there (rounded to bf16 for GPT_DTYPE_BF16).  grad_norm: optional device float
+ * that receives ||g||_2 before clipping.  Sums run in a fixed order: results are deterministic.
+ * GPT_ERR_BAD_SHAPE for step < 1, negative or non-finite lr, betas outside [0, 1), eps <= 0,
+ * negative weight_decay.  flags: GPT_FLAG_SYNC_CHECK synchronises the stream before returning. */
+int gpt_adamw_step(const gpt_config_t* cfg, float* params, const float* grads, float* exp_avg,
+                   float* exp_avg_sq, void* weights, const gpt_adamw_t* hp, float* grad_norm,
+                   void* workspace, size_t workspace_bytes, void* stream, int flags);
+
 #ifdef __cplusplus
 }
 #endif

@@ -208,6 +208,14 @@ def make_logits(batch: int, vocab: int, seed: int = BASE_SEED + 500_000, std: fl
     return z
 
 
+def make_grads(m: dict, seed: int = BASE_SEED + 700_000, scale: float = 1e-3) -> dict[str, torch.Tensor]:
+    """fp32 gradients N(0, scale^2), one per parameter tensor of ``make_weights(m)`` (biases
+    only when m["bias"]), for the optimizer step."""
+    shapes = weight_shapes(m)
+    names = [n for n in weight_names(m["n_layer"]) if m.get("bias", True) or not n.endswith(".bias")]
+    return {n: scale * torch.randn(shapes[n], generator=_gen(seed + k)) for k, n in enumerate(names)}
+
+
 def to_f64(weights: dict[str, torch.Tensor]):
     """Widen stored weights to fp64 numpy arrays (what the oracle consumes)."""
     return {k: v.to(torch.float64).numpy() for k, v in weights.items()}

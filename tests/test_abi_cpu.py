@@ -183,3 +183,38 @@ def test_sample_vocab_limit():
     c = ctypes.byref(_cfg("gpt2", vocab_size=60000).c())
     assert Lb.gpt_generate(c, FAKE, FAKE, 1, 4, 2, 1.0, 0, FAKE, FAKE, None, FAKE, FAKE, 1 << 40, None, 0) \
         == native.GPT_ERR_UNSUPPORTED
+
+
+def test_lr_schedule_matches_oracle():
+    import oracle.optim as oo
+    for it in (0, 1, 999, 1999, 2000, 2001, 123456, 301000, 599999, 600000, 600001, 10 ** 7):
+        assert native.lr_schedule(it) == pytest.approx(oo.lr_at(it), rel=1e-14, abs=0)
+    assert native.lr_schedule(5, 1.0, 0.1, 10, 100) == pytest.approx(oo.lr_at(5, 1.0, 0.1, 10, 100), rel=1e-14)
+
+
+def test_adamw_host_validation():
+    Lb = native.LIB
+    cfg = _cfg("gpt2")
+    c = ctypes.byref(cfg.c())
+    assert native.param_elems(cfg) == native.LIB.gpt_weights_bytes(c) // 2
+    ws = Lb.gpt_adamw_workspace_bytes()
+    ok = dict(lr=6e-4, beta1=0.9, beta2=0.95, eps=1e-8, weight_decay=0.1, max_grad_norm=1.0, step=1)
+
+    def call(ws_bytes=ws, params=FAKE, weights=None, **kw):
+        hp = native.gpt_adamw_t(**dict(ok, **kw))
+        return Lb.gpt_adamw_step(c, params, FAKE, FAKE, FAKE, weights, ctypes.byref(hp), None, FAKE, ws_bytes,
+                                 None, 0)
+    assert call(step=0) == native.GPT_ERR_BAD_SHAPE
+    assert call(lr=-1.0) == native.GPT_ERR_BAD_SHAPE
+    assert call(lr=float("nan")) == native.GPT_ERR_BAD_SHAPE
+    assert call(beta1=1.0) == native.GPT_ERR_BAD_SHAPE
+    assert call(eps=0.0) == native.GPT_ERR_BAD_SHAPE
+    assert call(weight_decay=-0.1) == native.GPT_ERR_BAD_SHAPE
+    assert call(ws_bytes=16) == native.GPT_ERR_WS_TOO_SMALL
+    assert call(params=None) == native.GPT_ERR_NULL
+    assert call(params=FAKE + 4) == native.GPT_ERR_BAD_ALIGN
+    assert call(weights=FAKE + 16) == native.GPT_ERR_BAD_ALIGN
+    hp = native.gpt_adamw_t(**ok)
+    big = ctypes.byref(_cfg("tiny", n_layer=90).c())                                  # > 1024 tensors
+    assert Lb.gpt_adamw_step(big, FAKE, FAKE, FAKE, FAKE, None, ctypes.byref(hp), None, FAKE, ws, None, 0) \
+        == native.GPT_ERR_UNSUPPORTED
