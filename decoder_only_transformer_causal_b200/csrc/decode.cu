@@ -123,7 +123,8 @@ __global__ void embed_pos_kernel(const E* __restrict__ wte, const E* __restrict_
 }
 
 // ---------------------------------------------------------------- matrix-vector products
-// out[r, n] = epilogue(sum_k xin[r, k] W[n, k] + bias[n]) for up to kGemvRows rows r.
+// out[r, n] = epilogue(sum_k xin[r, k] W[n, k] + bias[n]) for up to kGemvRows rows r (launches of
+// more rows are split).
 //
 // A CTA of 8 warps stages its input rows in shared memory once (in E, as stored between
 // kernels), optionally as LayerNorm of the fp32 residual stream (the ln_1 / ln_2 / ln_f that
@@ -133,7 +134,7 @@ __global__ void embed_pos_kernel(const E* __restrict__ wte, const E* __restrict_
 // are reduced over lanes by a butterfly and over the KSPLIT warps in slice order.
 constexpr int kGemvThreads = 256;
 constexpr int kGemvWarps = kGemvThreads / 32;
-constexpr int kGemvRows = 8;
+constexpr int kGemvRows = 16;
 
 template <typename E>
 struct GemvArgs {
@@ -176,7 +177,7 @@ GPT_DEVINL float4 load4w(const bf16* p) {
 }
 GPT_DEVINL float4 load4w(const float* p) { return *reinterpret_cast<const float4*>(p); }
 
-template <typename E, int EPI, int KSPLIT, int CPW, bool LN>
+template <typename E, int EPI, int KSPLIT, int CPW, bool LN, int ROWS>
 __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const GemvArgs<E> a) {
     griddep_launch_dependents();
     // the weights never change: start bringing them into L2 while the previous kernel finishes
@@ -185,7 +186,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const GemvArgs<E> a)
     extern __shared__ __align__(16) uint8_t gemv_smem[];
     E* xs = reinterpret_cast<E*>(gemv_smem);  // [rows][K]
     float* xf = reinterpret_cast<float*>(gemv_smem + static_cast<size_t>(a.rows) * a.K * sizeof(E));  // LN input
-    __shared__ float red[kGemvWarps][CPW][kGemvRows];
+    __shared__ float red[kGemvWarps][CPW][ROWS];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int K = a.K;
 
@@ -242,11 +243,11 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const GemvArgs<E> a)
     // column groups g = blockIdx.x, blockIdx.x + gridDim.x, ...: the staged rows serve them all
     for (int g = blockIdx.x; g < n_groups; g += gridDim.x) {
         const int n0 = g * kCols + (warp / KSPLIT) * CPW;
-        float acc[CPW][kGemvRows];
+        float acc[CPW][ROWS];
 #pragma unroll
         for (int c = 0; c < CPW; ++c)
 #pragma unroll
-            for (int r = 0; r < kGemvRows; ++r) acc[c][r] = 0.f;
+            for (int r = 0; r < ROWS; ++r) acc[c][r] = 0.f;
         const E* wrow[CPW];
 #pragma unroll
         for (int c = 0; c < CPW; ++c) wrow[c] = a.W + static_cast<long long>(min(n0 + c, a.N - 1)) * K;
@@ -256,7 +257,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const GemvArgs<E> a)
 #pragma unroll
             for (int c = 0; c < CPW; ++c) load8(wrow[c] + k, wf[c]);
 #pragma unroll
-            for (int r = 0; r < kGemvRows; ++r) {
+            for (int r = 0; r < ROWS; ++r) {
                 if (r < a.rows) {
                     float xf[8];
                     load8(xs + r * K + k, xf);
@@ -273,7 +274,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const GemvArgs<E> a)
 #pragma unroll
         for (int c = 0; c < CPW; ++c)
 #pragma unroll
-            for (int r = 0; r < kGemvRows; ++r) {
+            for (int r = 0; r < ROWS; ++r) {
                 if (r < a.rows) {
                     const float v = warp_sum(acc[c][r]);
                     if (lane == 0) red[warp][c][r] = v;
@@ -281,28 +282,30 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const GemvArgs<E> a)
             }
         if (KSPLIT > 1) __syncthreads();
         else __syncwarp();
-        const int c = lane / kGemvRows, r = lane % kGemvRows;
-        const int n = n0 + c;
-        if (ks == 0 && c < CPW && r < a.rows && n < a.N) {
-            float v = 0.f;
+        for (int cr = lane; cr < CPW * ROWS; cr += 32) {
+            const int c = cr / ROWS, r = cr % ROWS;
+            const int n = n0 + c;
+            if (ks == 0 && r < a.rows && n < a.N) {
+                float v = 0.f;
 #pragma unroll
-            for (int j = 0; j < KSPLIT; ++j) v += red[warp + j][c][r];
-            if (a.bias) v += to_f(a.bias[n]);
-            if (EPI == DV_GELU) {
-                v = a.gelu_tanh ? gelu_tanh(v) : gelu_erf(v);
-                static_cast<E*>(a.out)[r * a.ldo + n] = from_f<E>(v);
-            } else if (EPI == DV_RESID) {
-                float* o = static_cast<float*>(a.out) + r * a.ldo + n;
-                *o = __ldcg(o) + v;
-            } else if (EPI == DV_F32) {
-                static_cast<float*>(a.out)[r * a.ldo + n] = v;
-            } else {  // DV_QKV
-                if (n < a.C) {
+                for (int j = 0; j < KSPLIT; ++j) v += red[warp + j][c][r];
+                if (a.bias) v += to_f(a.bias[n]);
+                if (EPI == DV_GELU) {
+                    v = a.gelu_tanh ? gelu_tanh(v) : gelu_erf(v);
                     static_cast<E*>(a.out)[r * a.ldo + n] = from_f<E>(v);
-                } else {
-                    const int p = __ldcg(a.pos);
-                    if (p >= 0 && p < a.block_size)
-                        a.kv[(static_cast<long long>(r) * a.block_size + p) * 2 * a.C + (n - a.C)] = from_f<E>(v);
+                } else if (EPI == DV_RESID) {
+                    float* o = static_cast<float*>(a.out) + r * a.ldo + n;
+                    *o = __ldcg(o) + v;
+                } else if (EPI == DV_F32) {
+                    static_cast<float*>(a.out)[r * a.ldo + n] = v;
+                } else {  // DV_QKV
+                    if (n < a.C) {
+                        static_cast<E*>(a.out)[r * a.ldo + n] = from_f<E>(v);
+                    } else {
+                        const int p = __ldcg(a.pos);
+                        if (p >= 0 && p < a.block_size)
+                            a.kv[(static_cast<long long>(r) * a.block_size + p) * 2 * a.C + (n - a.C)] = from_f<E>(v);
+                    }
                 }
             }
         }
@@ -717,11 +720,11 @@ int launch_embed_pos(const void* wte, const void* wpe, const int64_t* tok, long 
 }
 
 namespace {
-template <typename E, int EPI, int KSPLIT, int CPW, bool LN>
+template <typename E, int EPI, int KSPLIT, int CPW, bool LN, int ROWS>
 int launch_gemv_inst(const GemvArgs<E>& a, cudaStream_t s) {
     constexpr int kCols = (kGemvWarps / KSPLIT) * CPW;
     const size_t smem = static_cast<size_t>(a.rows) * a.K * (sizeof(E) + (LN ? sizeof(float) : 0));
-    auto kern = gemv_kernel<E, EPI, KSPLIT, CPW, LN>;
+    auto kern = gemv_kernel<E, EPI, KSPLIT, CPW, LN, ROWS>;
     static size_t configured = 0;  // dynamic shared memory this kernel is opted in for
     if (smem > configured) {
         const int rc = cuda_status(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -732,15 +735,25 @@ int launch_gemv_inst(const GemvArgs<E>& a, cudaStream_t s) {
     return launch_overlapped(kern, dim3((a.N + kCols - 1) / kCols), dim3(kGemvThreads), smem, s, a);
 }
 
-// Warps per column: enough CTAs for narrow outputs, one with four columns a warp for the head.
-template <typename E, int EPI, bool LN>
+// Warps per column: enough CTAs for narrow outputs, four columns a warp for the head (two with
+// more than 8 rows, to keep the accumulators in registers).  ROWS: accumulator rows (8 or 16).
+template <typename E, int EPI, bool LN, int ROWS>
 int launch_gemv_mode(const GemvArgs<E>& a, cudaStream_t s) {
-    if (a.N >= 16384) return launch_gemv_inst<E, EPI, 1, 4, LN>(a, s);
+    if (a.N >= 16384) {
+        if (ROWS > 8) return launch_gemv_inst<E, EPI, 1, 2, LN, ROWS>(a, s);
+        return launch_gemv_inst<E, EPI, 1, 4, LN, ROWS>(a, s);
+    }
     int ksplit = a.N <= 2048 ? 4 : 2;
     while (ksplit > 1 && (a.K % (8 * ksplit))) ksplit >>= 1;
-    if (ksplit == 4) return launch_gemv_inst<E, EPI, 4, 1, LN>(a, s);
-    if (ksplit == 2) return launch_gemv_inst<E, EPI, 2, 1, LN>(a, s);
-    return launch_gemv_inst<E, EPI, 1, 1, LN>(a, s);
+    if (ksplit == 4) return launch_gemv_inst<E, EPI, 4, 1, LN, ROWS>(a, s);
+    if (ksplit == 2) return launch_gemv_inst<E, EPI, 2, 1, LN, ROWS>(a, s);
+    return launch_gemv_inst<E, EPI, 1, 1, LN, ROWS>(a, s);
+}
+
+template <typename E, int EPI, bool LN>
+int launch_gemv_rows(const GemvArgs<E>& a, cudaStream_t s) {
+    if (a.rows > 8) return launch_gemv_mode<E, EPI, LN, 16>(a, s);
+    return launch_gemv_mode<E, EPI, LN, 8>(a, s);
 }
 
 template <typename E>
@@ -771,15 +784,15 @@ int gemv_typed(int epi, bool ln, const void* x, long long ldx, const E* ln_w, co
         int rc;
         if (ln) {
             switch (epi) {
-                case DV_GELU: rc = launch_gemv_mode<E, DV_GELU, true>(a, s); break;
-                case DV_F32: rc = launch_gemv_mode<E, DV_F32, true>(a, s); break;
-                case DV_QKV: rc = launch_gemv_mode<E, DV_QKV, true>(a, s); break;
+                case DV_GELU: rc = launch_gemv_rows<E, DV_GELU, true>(a, s); break;
+                case DV_F32: rc = launch_gemv_rows<E, DV_F32, true>(a, s); break;
+                case DV_QKV: rc = launch_gemv_rows<E, DV_QKV, true>(a, s); break;
                 default: return GPT_ERR_UNSUPPORTED;
             }
         } else {
             switch (epi) {
-                case DV_RESID: rc = launch_gemv_mode<E, DV_RESID, false>(a, s); break;
-                case DV_F32: rc = launch_gemv_mode<E, DV_F32, false>(a, s); break;
+                case DV_RESID: rc = launch_gemv_rows<E, DV_RESID, false>(a, s); break;
+                case DV_F32: rc = launch_gemv_rows<E, DV_F32, false>(a, s); break;
                 default: return GPT_ERR_UNSUPPORTED;
             }
         }

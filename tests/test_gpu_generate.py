@@ -121,7 +121,8 @@ def decode_logits_oracle(cfg, W64, prompt, forced, steps, gelu="erf"):
 DECODE_CASES = [
     # workload, stress, layers, B, T0, n_forced, steps checked by the oracle, gelu
     ("tiny", True, None, 3, 5, 59, "all", "erf"),          # up to the last position (63)
-    ("tiny", True, None, 9, 3, 6, "all", "tanh"),           # B > 8: the row-chunked products
+    ("tiny", True, None, 9, 3, 6, "all", "tanh"),           # rows 9..16 of one product launch
+    ("tiny", True, None, 17, 3, 4, "all", "erf"),           # B > 16: the row-chunked products
     ("gpt2", True, 2, 2, 120, 12, "all", "erf"),            # crosses the 128-key split
     ("gpt2", False, None, 4, 1, 8, "all", "erf"),           # the 124M model from one token
     ("gpt2", True, 2, 9, 40, 3, "all", "erf"),
