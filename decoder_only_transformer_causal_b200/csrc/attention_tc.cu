@@ -42,13 +42,9 @@ int launch_attention_bf16(const AttnLayout& L, int B, int nh, int T, int32_t* st
     p.scale_log2 = static_cast<float>(1.4426950408889634 / sqrt(static_cast<double>(attn::HS)));
     p.status = status;
 
-    static bool configured = false;
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(attn::attention_fwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             attn::SMEM_BYTES);
-        if (e != cudaSuccess) return cuda_status(e);
-        configured = true;
-    }
+    static size_t opted[kMaxDevices] = {};
+    rc = opt_in_smem(reinterpret_cast<const void*>(attn::attention_fwd_tc), attn::SMEM_BYTES, opted);
+    if (rc) return rc;
     const long long n_qt = (T + attn::BQ - 1) / attn::BQ;
     const long long blocks = n_qt * B * nh;
     if (blocks > 0x7fffffffLL) return GPT_ERR_UNSUPPORTED;

@@ -725,13 +725,9 @@ int launch_gemv_inst(const GemvArgs<E>& a, cudaStream_t s) {
     constexpr int kCols = (kGemvWarps / KSPLIT) * CPW;
     const size_t smem = static_cast<size_t>(a.rows) * a.K * (sizeof(E) + (LN ? sizeof(float) : 0));
     auto kern = gemv_kernel<E, EPI, KSPLIT, CPW, LN, ROWS>;
-    static size_t configured = 0;  // dynamic shared memory this kernel is opted in for
-    if (smem > configured) {
-        const int rc = cuda_status(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                        static_cast<int>(smem)));
-        if (rc) return rc;
-        configured = smem;
-    }
+    static size_t opted[kMaxDevices] = {};
+    const int rc = opt_in_smem(reinterpret_cast<const void*>(kern), smem, opted);
+    if (rc) return rc;
     return launch_overlapped(kern, dim3((a.N + kCols - 1) / kCols), dim3(kGemvThreads), smem, s, a);
 }
 
@@ -864,14 +860,10 @@ int sample_max_vocab() { return kSampleMaxV; }
 int launch_sample(const float* logits, long long ld_logits, int B, int V, float temperature, int top_k,
                   const float* u, int64_t* out, long long ld_out, cudaStream_t s) {
     if (V > kSampleMaxV) return GPT_ERR_UNSUPPORTED;
-    static int configured = 0;  // dynamic shared memory the kernel is opted in for
+    static size_t opted[kMaxDevices] = {};
     const int smem = V * static_cast<int>(sizeof(float));
-    if (smem > configured) {
-        const int rc = cuda_status(cudaFuncSetAttribute(sample_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                        kSampleMaxV * static_cast<int>(sizeof(float))));
-        if (rc) return rc;
-        configured = kSampleMaxV * static_cast<int>(sizeof(float));
-    }
+    const int rc = opt_in_smem(reinterpret_cast<const void*>(sample_kernel), kSampleMaxV * sizeof(float), opted);
+    if (rc) return rc;
     return launch_overlapped(sample_kernel, dim3(B), dim3(kSampleThreads), static_cast<size_t>(smem), s, logits,
                              ld_logits, V, temperature, top_k, u, out, ld_out);
 }

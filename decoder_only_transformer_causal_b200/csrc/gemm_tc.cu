@@ -13,12 +13,9 @@ int launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& 
                cudaStream_t s) {
     using L = gemm::Cfg<kBN>;
     auto kern = gemm::gemm_bf16_tc<kBN, EPI, GELU_TANH>;
-    static bool configured = false;
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_BYTES);
-        if (e != cudaSuccess) return cuda_status(e);
-        configured = true;
-    }
+    static size_t opted[kMaxDevices] = {};
+    const int rc = opt_in_smem(reinterpret_cast<const void*>(kern), L::SMEM_BYTES, opted);
+    if (rc) return rc;
     const int tiles = ((p.M + gemm::BM - 1) / gemm::BM) * ((p.N + kBN - 1) / kBN);
     const int grid = tiles < num_sms() ? tiles : num_sms();
     return launch_overlapped(kern, dim3(grid), dim3(L::THREADS), L::SMEM_BYTES, s, ta, tb, tc, p);

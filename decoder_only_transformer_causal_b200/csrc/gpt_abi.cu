@@ -35,6 +35,17 @@ int num_sms() {
     return cached[dev];
 }
 
+int opt_in_smem(const void* kern, size_t bytes, size_t (&opted)[kMaxDevices]) {
+    int dev = 0;
+    int rc = cuda_status(cudaGetDevice(&dev));
+    if (rc) return rc;
+    if (dev >= 0 && dev < kMaxDevices && bytes <= opted[dev]) return GPT_OK;
+    rc = cuda_status(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes)));
+    if (rc) return rc;
+    if (dev >= 0 && dev < kMaxDevices) opted[dev] = bytes;
+    return GPT_OK;
+}
+
 // ------------------------------------------------------------------ TMA descriptors
 namespace {
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,

@@ -17,6 +17,12 @@ typedef __nv_bfloat16 bf16;
 int num_sms();
 int cuda_status(cudaError_t e);
 
+// Opts a kernel in for `bytes` of dynamic shared memory on the current device.  `opted` is a
+// per-kernel table (a function-local static of the caller) of the size each device is opted in
+// for; the attribute is set the first time a device needs a size, or a larger one.
+constexpr int kMaxDevices = 64;
+int opt_in_smem(const void* kern, size_t bytes, size_t (&opted)[kMaxDevices]);
+
 // Launches `kern` so that it may overlap the tail of the previous kernel in the stream
 // (programmatic stream serialisation); every kernel launched this way calls griddep_wait()
 // before touching memory its predecessor uses.

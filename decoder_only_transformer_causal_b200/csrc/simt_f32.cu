@@ -152,9 +152,9 @@ int launch_attention_f32(const AttnLayoutF32& L, int B, int nh, int T, int hs, c
     if (rows == 0) return GPT_OK;
     const size_t smem = static_cast<size_t>(kAttWarps) * (kMaxHs + T) * sizeof(float);
     if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(attention_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(smem));
-        if (e != cudaSuccess) return cuda_status(e);
+        static size_t opted[kMaxDevices] = {};
+        const int rc = opt_in_smem(reinterpret_cast<const void*>(attention_f32_kernel), smem, opted);
+        if (rc) return rc;
     }
     const unsigned blocks = static_cast<unsigned>((rows + kAttWarps - 1) / kAttWarps);
     attention_f32_kernel<<<blocks, kAttWarps * 32, smem, s>>>(L, B, nh, T, hs, 1.0f / sqrtf(static_cast<float>(hs)));
