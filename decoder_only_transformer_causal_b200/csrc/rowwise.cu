@@ -64,7 +64,7 @@ __global__ void embed_kernel(const Tw* __restrict__ wte, const Tw* __restrict__ 
 // §2.5 (A)).  The row stays in registers: mean, then sum of squared deviations.
 constexpr int kLnMaxVec = 16;  // float4 per lane -> C <= 2048
 
-template <typename To>
+template <typename To, int VEC>  // VEC = float4 per lane, ceil(C / 128): registers sized to the row
 __global__ void layernorm_kernel(const float* __restrict__ x, const To* __restrict__ w,
                                  const To* __restrict__ bias, To* __restrict__ out, int rows, int C) {
     griddep_launch_dependents();
@@ -74,10 +74,10 @@ __global__ void layernorm_kernel(const float* __restrict__ x, const To* __restri
     if (row >= rows) return;
     const float* xr = x + static_cast<long long>(row) * C;
     const int nv = C >> 2;
-    float4 v[kLnMaxVec];
+    float4 v[VEC];
     float s = 0.f;
 #pragma unroll
-    for (int k = 0; k < kLnMaxVec; ++k) {
+    for (int k = 0; k < VEC; ++k) {
         const int j = lane + 32 * k;
         if (j < nv) {
             v[k] = load4(xr + 4 * j);
@@ -87,7 +87,7 @@ __global__ void layernorm_kernel(const float* __restrict__ x, const To* __restri
     const float mean = warp_sum(s) / C;
     float ss = 0.f;
 #pragma unroll
-    for (int k = 0; k < kLnMaxVec; ++k) {
+    for (int k = 0; k < VEC; ++k) {
         const int j = lane + 32 * k;
         if (j < nv) {
             const float a = v[k].x - mean, b = v[k].y - mean, c = v[k].z - mean, d = v[k].w - mean;
@@ -97,7 +97,7 @@ __global__ void layernorm_kernel(const float* __restrict__ x, const To* __restri
     const float rstd = rsqrtf(warp_sum(ss) / C + 1e-5f);
     To* orow = out + static_cast<long long>(row) * C;
 #pragma unroll
-    for (int k = 0; k < kLnMaxVec; ++k) {
+    for (int k = 0; k < VEC; ++k) {
         const int j = lane + 32 * k;
         if (j < nv) {
             const float4 g = load4(w + 4 * j);
@@ -223,18 +223,29 @@ int launch_embed(const void* wte, const void* wpe, const int64_t* idx, float* x,
                              static_cast<const float*>(wpe), idx, x, T, C, V, total4, status);
 }
 
+namespace {
+template <typename To, int VEC>
+int launch_ln_vec(const float* x, const void* w, const void* b, void* out, int rows, int C, cudaStream_t s) {
+    const unsigned blocks = (rows + kWarpsPerBlock - 1) / kWarpsPerBlock;
+    return launch_overlapped(layernorm_kernel<To, VEC>, dim3(blocks), dim3(32 * kWarpsPerBlock), 0, s, x,
+                             static_cast<const To*>(w), static_cast<const To*>(b), static_cast<To*>(out), rows, C);
+}
+
+template <typename To, int VEC = 1>
+int launch_ln(const float* x, const void* w, const void* b, void* out, int rows, int C, cudaStream_t s) {
+    if constexpr (VEC < kLnMaxVec) {
+        if (C > 128 * VEC) return launch_ln<To, VEC + 1>(x, w, b, out, rows, C, s);
+    }
+    return launch_ln_vec<To, VEC>(x, w, b, out, rows, C, s);
+}
+}  // namespace
+
 int launch_layernorm(const float* x, const void* w, const void* b, void* out, int rows, int C,
                      int dtype, cudaStream_t s) {
     if (C > 4 * 32 * kLnMaxVec || (C & 3)) return GPT_ERR_UNSUPPORTED;
     if (rows == 0) return GPT_OK;
-    const unsigned blocks = (rows + kWarpsPerBlock - 1) / kWarpsPerBlock;
-    if (dtype == GPT_DTYPE_BF16)
-        return launch_overlapped(layernorm_kernel<bf16>, dim3(blocks), dim3(32 * kWarpsPerBlock), 0, s, x,
-                                 static_cast<const bf16*>(w), static_cast<const bf16*>(b), static_cast<bf16*>(out),
-                                 rows, C);
-    return launch_overlapped(layernorm_kernel<float>, dim3(blocks), dim3(32 * kWarpsPerBlock), 0, s, x,
-                             static_cast<const float*>(w), static_cast<const float*>(b), static_cast<float*>(out),
-                             rows, C);
+    if (dtype == GPT_DTYPE_BF16) return launch_ln<bf16>(x, w, b, out, rows, C, s);
+    return launch_ln<float>(x, w, b, out, rows, C, s);
 }
 
 int launch_ce_rows_from_parts(const float2* part, int n_part, const float* tlogit,
