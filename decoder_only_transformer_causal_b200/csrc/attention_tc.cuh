@@ -248,21 +248,34 @@ __global__ void __launch_bounds__(THREADS, 2)
             const uint64_t SC = f2_pack(p.scale_log2, p.scale_log2), NM = f2_pack(-m_used, -m_used);
             uint64_t acc4[4] = {0, 0, 0, 0};
             uint32_t pk0[32], pk1[32];
-            // On the diagonal tile, 32-column chunks to the right of this warp's last row are
-            // masked for every lane: P is 0 there and no exponential is evaluated.
+            // Off the diagonal every column is live (a loop with no per-column test).  On the
+            // diagonal tile, 32-column chunks to the right of this warp's last row are masked for
+            // every lane: P is 0 there and no exponential is evaluated.
             const int live_cols = diag ? (quarter + 1) * 32 : BKV;  // warp-uniform
+            if (!diag) {
 #pragma unroll
-            for (int c = 0; c < BKV; c += 2) {
-                float p0 = 0.f, p1 = 0.f;
-                if (c < live_cols) {
+                for (int c = 0; c < BKV; c += 2) {
                     float x0, x1;
                     f2_unpack(f2_fma(f2_pack(s[c], s[c + 1]), SC, NM), x0, x1);
-                    p0 = exp2_approx(x0);
-                    p1 = exp2_approx(x1);
+                    const float p0 = exp2_approx(x0), p1 = exp2_approx(x1);
                     acc4[(c >> 1) & 3] = f2_add(acc4[(c >> 1) & 3], f2_pack(p0, p1));
+                    if (c < 64) pk0[c / 2] = pack_bf16x2(p0, p1);
+                    else pk1[(c - 64) / 2] = pack_bf16x2(p0, p1);
                 }
-                if (c < 64) pk0[c / 2] = pack_bf16x2(p0, p1);
-                else pk1[(c - 64) / 2] = pack_bf16x2(p0, p1);
+            } else {
+#pragma unroll
+                for (int c = 0; c < BKV; c += 2) {
+                    float p0 = 0.f, p1 = 0.f;
+                    if (c < live_cols) {
+                        float x0, x1;
+                        f2_unpack(f2_fma(f2_pack(s[c], s[c + 1]), SC, NM), x0, x1);
+                        p0 = exp2_approx(x0);
+                        p1 = exp2_approx(x1);
+                        acc4[(c >> 1) & 3] = f2_add(acc4[(c >> 1) & 3], f2_pack(p0, p1));
+                    }
+                    if (c < 64) pk0[c / 2] = pack_bf16x2(p0, p1);
+                    else pk1[(c - 64) / 2] = pack_bf16x2(p0, p1);
+                }
             }
             float a0, a1, b0, b1, c0, c1, d0, d1;
             f2_unpack(acc4[0], a0, a1); f2_unpack(acc4[1], b0, b1); f2_unpack(acc4[2], c0, c1); f2_unpack(acc4[3], d0, d1);
