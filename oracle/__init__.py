@@ -5,7 +5,8 @@ and the CPU-baseline leg of ``bench.py`` may import it.  It shares nothing with 
 CUDA path (no kernels, headers, helpers, tables or constants); the two meet only in
 the seeded inputs of the ``seeded`` module.
 
-See ``oracle/gpt.py`` (the forward pass) and ``oracle/generate.py`` (GPT.generate) for the
+See ``oracle/gpt.py`` (the forward pass), ``oracle/generate.py`` (GPT.generate),
+``oracle/optim.py`` (the optimizer step) and ``oracle/backward.py`` (the gradients) for the
 definitions and their citations.
 """
 from .gpt import (  # noqa: F401
