@@ -432,6 +432,44 @@ def adamw_bench(model, native, dev, stream, peaks, peak_src, steps: int = 20, wa
             "gpu_launches_per_step": 2}
 
 
+def backward_pieces_bench(native, dev, stream, peaks, peak_src, reps: int = 10):
+    """The largest backward steps that are not matrix products, at the GPT-2 124M shapes
+    ("nanoGPT 全局流程图" 3.4): the cross-entropy gradient over the full logits [12288, 50304] bf16
+    (reads the logits twice, writes the gradient: 3 x 1.24 GB) and one LayerNorm backward
+    [12288, 768] (reads dy and x, reads and writes dx: 4 x 37.7 MB).  Inputs exceed the L2."""
+    rows, V, C = 12 * 1024, 50304, 768
+    g = torch.Generator(device=dev).manual_seed(3)
+    z = (torch.randn((rows, V), device=dev, generator=g) * 1.5).to(torch.bfloat16)
+    tgt = torch.randint(0, 50257, (rows,), device=dev, generator=g)
+    sc = torch.tensor([0.0, float(rows)], dtype=torch.float64, device=dev)
+    dz = torch.empty_like(z)
+    x = torch.randn((rows, C), device=dev, generator=g)
+    dy = torch.randn((rows, C), device=dev, generator=g) * 0.01
+    w = torch.ones(C, device=dev, dtype=torch.bfloat16)
+    dx = torch.zeros_like(x)
+    dw = torch.empty(C, device=dev)
+    db = torch.empty(C, device=dev)
+    out = {}
+    for name, fn, nbytes in (
+            ("cross_entropy_backward", lambda: native.cross_entropy_backward(z, tgt, sc, dlogits=dz), 3 * rows * V * 2),
+            ("layernorm_backward", lambda: native.layernorm_backward(dy, x, w, dx=dx, accumulate=True, dw=dw, db=db),
+             4 * rows * C * 4)):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / reps
+        gbs = nbytes / (ms / 1000.0) / 1e9
+        out[name] = {"ms": ms, "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                            "frac": gbs / peaks["hbm_gbs"], "bytes": nbytes, "peak_source": peak_src}}
+    return out
+
+
 def adamw_only(args):
     from decoder_only_transformer_causal_b200 import GPT, GPTConfig, native
     dev = torch.device("cuda", 0)
@@ -604,6 +642,7 @@ def main():
     if rank == 0 and not args.no_kernels:
         line["decode"] = decode_bench(model, native, dev, stream, peaks, peak_src)
         line["adamw"] = adamw_bench(model, native, dev, stream, peaks, peak_src)
+        line["backward_pieces"] = backward_pieces_bench(native, dev, stream, peaks, peak_src)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         times, threads = oracle_sample(w, 256, budget_s=12.0)
         tok_s = 256 * len(times) / sum(times)

@@ -1,0 +1,366 @@
+// Backward kernels of the pieces of the forward that are not matrix products ("nanoGPT 全局流程图",
+// 3.4 反向传播: loss.backward() applies the chain rule from the loss back to every parameter):
+// the cross-entropy's gradient with respect to the logits, LayerNorm's backward, GELU's
+// derivative, column sums for bias (and LayerNorm weight) gradients, and the embedding's
+// backward.  Every reduction runs in a fixed order, so results are deterministic.
+//
+// All are HBM-bound row or column sweeps: the logits gradient reads the logits twice (an online
+// max/sum pass, then the write pass) and writes one gradient per logit; LayerNorm's backward
+// reads dy and x once and writes dx; the column sums read their input once.
+#include <math.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace gpt {
+
+namespace {
+
+constexpr int kBwdWarps = 8;
+
+// Every load is an L2 load (ld.global.cg): these kernels run under programmatic dependent launch
+// and read data written several kernels earlier (the logits, the saved activations), which only
+// the immediately preceding kernel's writes are guaranteed visible past griddepcontrol.wait.
+GPT_DEVINL float ld1(const bf16* p) {
+    return __bfloat162float(__ushort_as_bfloat16(__ldcg(reinterpret_cast<const unsigned short*>(p))));
+}
+GPT_DEVINL float ld1(const float* p) { return __ldcg(p); }
+template <typename E> GPT_DEVINL E st1(float v);
+template <> GPT_DEVINL bf16 st1<bf16>(float v) { return __float2bfloat16_rn(v); }
+template <> GPT_DEVINL float st1<float>(float v) { return v; }
+
+GPT_DEVINL float wsum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// dlogits[r, v] = (exp(z_rv - lse_r) - [v == t_r]) / n for rows whose target is not -1, and 0
+// for the rest; n = the number of counted rows, read from sum_count[1] (the forward's {sum of row
+// losses, counted rows}).  One warp per row: an online (max, sum) pass over the row, then the
+// write pass.
+template <typename E>
+__global__ void __launch_bounds__(kBwdWarps * 32)
+    ce_backward_kernel(const E* __restrict__ z, const int64_t* __restrict__ targets, const double* __restrict__ sum_count,
+                       E* __restrict__ dz, int rows, int V, int32_t* status) {
+    griddep_launch_dependents();
+    griddep_wait();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int r = blockIdx.x * kBwdWarps + warp;
+    if (r >= rows) return;
+    const E* zr = z + static_cast<long long>(r) * V;
+    E* dr = dz + static_cast<long long>(r) * V;
+    const long long t = __ldcg(targets + r);
+    const double n = __ldcg(sum_count + 1);
+    if (t == -1 || n <= 0.0) {
+        for (int v = lane; v < V; v += 32) dr[v] = st1<E>(0.f);
+        return;
+    }
+    if (t < 0 || t >= V) {
+        if (lane == 0) set_status(status, GPT_ERR_INDEX);
+        for (int v = lane; v < V; v += 32) dr[v] = st1<E>(0.f);
+        return;
+    }
+    float m = -INFINITY, s = 0.f;
+    for (int v = lane; v < V; v += 32) {
+        const float x = ld1(zr + v);
+        if (x > m) {
+            s = s * __expf(m - x) + 1.f;
+            m = x;
+        } else {
+            s += __expf(x - m);
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const float m2 = __shfl_xor_sync(0xffffffffu, m, o), s2 = __shfl_xor_sync(0xffffffffu, s, o);
+        const float mm = fmaxf(m, m2);
+        s = (m == -INFINITY ? 0.f : s * __expf(m - mm)) + (m2 == -INFINITY ? 0.f : s2 * __expf(m2 - mm));
+        m = mm;
+    }
+    const float lse = m + __logf(s);
+    const float inv_n = static_cast<float>(1.0 / n);
+    for (int v = lane; v < V; v += 32) {
+        const float p = __expf(ld1(zr + v) - lse);
+        dr[v] = st1<E>((p - (v == t ? 1.f : 0.f)) * inv_n);
+    }
+}
+
+// LayerNorm backward, one warp per row: y = xhat w + b, xhat = (x - mean) * rstd;
+// dx (+)= rstd (dxhat - mean(dxhat) - xhat mean(dxhat xhat)), dxhat = dy w.  Each CTA also
+// leaves its rows' sums of dy * xhat and dy per column in part[blockIdx.x] (the weight and bias
+// gradients after the column reduction).
+template <typename Tw>
+__global__ void __launch_bounds__(kBwdWarps * 32)
+    layernorm_backward_kernel(const float* __restrict__ dy, const float* __restrict__ x, const Tw* __restrict__ w,
+                              float* __restrict__ dx, int accumulate, float* __restrict__ part, int rows, int C) {
+    griddep_launch_dependents();
+    griddep_wait();
+    extern __shared__ float sm[];  // [kBwdWarps][2][C] per-warp column sums
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    float* my = sm + static_cast<size_t>(warp) * 2 * C;
+    for (int c = lane; c < 2 * C; c += 32) my[c] = 0.f;
+    __syncwarp();
+    const int r = blockIdx.x * kBwdWarps + warp;
+    if (r < rows) {
+        const float* xr = x + static_cast<long long>(r) * C;
+        const float* dyr = dy + static_cast<long long>(r) * C;
+        float s = 0.f;
+        for (int c = lane; c < C; c += 32) s += __ldcg(xr + c);
+        const float mean = wsum(s) / C;
+        float ss = 0.f;
+        for (int c = lane; c < C; c += 32) {
+            const float d = __ldcg(xr + c) - mean;
+            ss += d * d;
+        }
+        const float rstd = rsqrtf(wsum(ss) / C + 1e-5f);
+        float a = 0.f, bsum = 0.f;  // sum of dxhat, sum of dxhat * xhat
+        for (int c = lane; c < C; c += 32) {
+            const float xh = (__ldcg(xr + c) - mean) * rstd;
+            const float g = __ldcg(dyr + c);
+            const float dxh = g * ld1(w + c);
+            a += dxh;
+            bsum += dxh * xh;
+            my[c] += g * xh;
+            my[C + c] += g;
+        }
+        const float ma = wsum(a) / C, mb = wsum(bsum) / C;
+        float* dxr = dx + static_cast<long long>(r) * C;
+        for (int c = lane; c < C; c += 32) {
+            const float xh = (__ldcg(xr + c) - mean) * rstd;
+            const float v = rstd * (__ldcg(dyr + c) * ld1(w + c) - ma - xh * mb);
+            dxr[c] = accumulate ? __ldcg(dxr + c) + v : v;
+        }
+    }
+    __syncthreads();
+    // this CTA's column sums, warps added in order
+    for (int c = threadIdx.x; c < 2 * C; c += kBwdWarps * 32) {
+        float v = 0.f;
+        for (int wp = 0; wp < kBwdWarps; ++wp) v += sm[static_cast<size_t>(wp) * 2 * C + c];
+        part[static_cast<long long>(blockIdx.x) * 2 * C + c] = v;
+    }
+}
+
+// out[c] (+)= sum over i < n_part of part[i * ld + c], in order of i (the second stage of a
+// column reduction).
+__global__ void colsum_parts_kernel(const float* __restrict__ part, long long ld, int n_part, int C,
+                                    float* __restrict__ out, int accumulate) {
+    griddep_launch_dependents();
+    griddep_wait();
+    const int c = blockIdx.x * blockDim.x + threadIdx.x;
+    if (c >= C) return;
+    float v = 0.f;
+    for (int i = 0; i < n_part; ++i) v += __ldcg(part + i * ld + c);
+    out[c] = accumulate ? __ldcg(out + c) + v : v;
+}
+
+// part[blockIdx.y][c] = sum of y[r, c] over this CTA's row block (rows in order); first stage of
+// the bias gradient (column sums of the output gradient).
+constexpr int kColRows = 128;
+template <typename E>
+__global__ void colsum_rows_kernel(const E* __restrict__ y, int rows, int C, float* __restrict__ part) {
+    griddep_launch_dependents();
+    griddep_wait();
+    const int c = blockIdx.x * blockDim.x + threadIdx.x;
+    if (c >= C) return;
+    const int r0 = blockIdx.y * kColRows, r1 = min(rows, r0 + kColRows);
+    float v = 0.f;
+    for (int r = r0; r < r1; ++r) v += ld1(y + static_cast<long long>(r) * C + c);
+    part[static_cast<long long>(blockIdx.y) * C + c] = v;
+}
+
+// dpre = dh * gelu'(pre): erf form Phi(z) + z phi(z); tanh form 0.5 (1 + tanh a) +
+// 0.5 z (1 - tanh^2 a) sqrt(2/pi) (1 + 3 * 0.044715 z^2), a = sqrt(2/pi) (z + 0.044715 z^3).
+template <typename E>
+__global__ void gelu_backward_kernel(const float* __restrict__ dh, const E* __restrict__ pre, E* __restrict__ dpre,
+                                     long long n, int tanh_form) {
+    griddep_launch_dependents();
+    griddep_wait();
+    const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (i >= n) return;
+    const float z = ld1(pre + i);
+    float d;
+    if (tanh_form) {
+        const float c = 0.7978845608028654f;
+        const float th = tanhf(c * (z + 0.044715f * z * z * z));
+        d = 0.5f * (1.f + th) + 0.5f * z * (1.f - th * th) * c * (1.f + 3.f * 0.044715f * z * z);
+    } else {
+        d = 0.5f * (1.f + erff(z * 0.7071067811865476f)) + z * 0.3989422804014327f * __expf(-0.5f * z * z);
+    }
+    dpre[i] = st1<E>(__ldcg(dh + i) * d);
+}
+
+// ------------------------------------------------------------------ embedding backward
+// dwte[v] += sum of dx[r] over rows r with idx[r] = v, in row order; dwpe[t] += sum over the
+// batch of dx[b, t].  The rows are ordered by (token, row) with a bitonic sort of 64-bit keys in
+// one CTA's shared memory (N <= kEmbSortMax rows), then each run of equal tokens is summed by one
+// warp in row order.
+constexpr int kEmbSortMax = 16384;
+constexpr int kEmbSortThreads = 1024;
+
+__global__ void __launch_bounds__(kEmbSortThreads)
+    embed_sort_kernel(const int64_t* __restrict__ idx, int N, int V, unsigned long long* __restrict__ sorted,
+                      int32_t* status) {
+    griddep_launch_dependents();
+    griddep_wait();
+    extern __shared__ unsigned long long keys[];  // next power of two >= N
+    int n2 = 1;
+    while (n2 < N) n2 <<= 1;
+    for (int i = threadIdx.x; i < n2; i += kEmbSortThreads) {
+        unsigned long long k = ~0ull;
+        if (i < N) {
+            long long t = __ldcg(idx + i);
+            if (t < 0 || t >= V) {
+                set_status(status, GPT_ERR_INDEX);
+                t = V;  // sorts after every valid token; skipped below
+            }
+            k = (static_cast<unsigned long long>(t) << 32) | static_cast<unsigned>(i);
+        }
+        keys[i] = k;
+    }
+    __syncthreads();
+    for (int size = 2; size <= n2; size <<= 1) {
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            for (int i = threadIdx.x; i < n2; i += kEmbSortThreads) {
+                const int j = i ^ stride;
+                if (j > i) {
+                    const bool up = (i & size) == 0;
+                    const unsigned long long a = keys[i], b = keys[j];
+                    if ((a > b) == up) {
+                        keys[i] = b;
+                        keys[j] = a;
+                    }
+                }
+            }
+            __syncthreads();
+        }
+    }
+    for (int i = threadIdx.x; i < N; i += kEmbSortThreads) sorted[i] = keys[i];
+}
+
+// One warp per sorted position that starts a run of equal tokens: adds the run's dx rows (in
+// row order) into dwte[token].
+__global__ void embed_runs_kernel(const unsigned long long* __restrict__ sorted, int N, int V,
+                                  const float* __restrict__ dx, int C, float* __restrict__ dwte) {
+    griddep_launch_dependents();
+    griddep_wait();
+    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+    if (warp >= N) return;
+    const unsigned long long k = __ldcg(sorted + warp);
+    const unsigned tok = static_cast<unsigned>(k >> 32);
+    if (tok >= static_cast<unsigned>(V)) return;
+    if (warp > 0 && static_cast<unsigned>(__ldcg(sorted + warp - 1) >> 32) == tok) return;  // not a run start
+    int end = warp + 1;
+    while (end < N && static_cast<unsigned>(__ldcg(sorted + end) >> 32) == tok) ++end;
+    float* out = dwte + static_cast<long long>(tok) * C;
+    for (int c = lane; c < C; c += 32) {
+        float v = 0.f;
+        for (int s = warp; s < end; ++s) {
+            const unsigned r = static_cast<unsigned>(__ldcg(sorted + s) & 0xffffffffull);
+            v += __ldcg(dx + static_cast<long long>(r) * C + c);
+        }
+        out[c] = __ldcg(out + c) + v;
+    }
+}
+
+__global__ void embed_wpe_kernel(const float* __restrict__ dx, int B, int T, int C, float* __restrict__ dwpe) {
+    griddep_launch_dependents();
+    griddep_wait();
+    const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (i >= static_cast<long long>(T) * C) return;
+    float v = 0.f;
+    for (int b = 0; b < B; ++b) v += __ldcg(dx + static_cast<long long>(b) * T * C + i);
+    dwpe[i] = __ldcg(dwpe + i) + v;
+}
+
+}  // namespace
+
+int launch_ce_backward(const void* logits, int dtype, const int64_t* targets, const double* sum_count, void* dlogits,
+                       int rows, int V, int32_t* status, cudaStream_t s) {
+    const dim3 grid((rows + kBwdWarps - 1) / kBwdWarps), block(kBwdWarps * 32);
+    if (dtype == GPT_DTYPE_BF16)
+        return launch_overlapped(ce_backward_kernel<bf16>, grid, block, 0, s, static_cast<const bf16*>(logits),
+                                 targets, sum_count, static_cast<bf16*>(dlogits), rows, V, status);
+    return launch_overlapped(ce_backward_kernel<float>, grid, block, 0, s, static_cast<const float*>(logits), targets,
+                             sum_count, static_cast<float*>(dlogits), rows, V, status);
+}
+
+int layernorm_backward_parts(int rows) { return (rows + kBwdWarps - 1) / kBwdWarps; }
+
+int launch_layernorm_backward(const float* dy, const float* x, const void* w, int dtype, float* dx, int accumulate,
+                              float* dw, float* db, int accumulate_wb, float* part, int rows, int C,
+                              cudaStream_t s) {
+    const int n_part = layernorm_backward_parts(rows);
+    const size_t smem = static_cast<size_t>(kBwdWarps) * 2 * C * sizeof(float);
+    int rc;
+    if (dtype == GPT_DTYPE_BF16) {
+        static size_t opted[kMaxDevices] = {};
+        rc = opt_in_smem(reinterpret_cast<const void*>(layernorm_backward_kernel<bf16>), smem, opted);
+        if (!rc)
+            rc = launch_overlapped(layernorm_backward_kernel<bf16>, dim3(n_part), dim3(kBwdWarps * 32), smem, s, dy,
+                                   x, static_cast<const bf16*>(w), dx, accumulate, part, rows, C);
+    } else {
+        static size_t opted[kMaxDevices] = {};
+        rc = opt_in_smem(reinterpret_cast<const void*>(layernorm_backward_kernel<float>), smem, opted);
+        if (!rc)
+            rc = launch_overlapped(layernorm_backward_kernel<float>, dim3(n_part), dim3(kBwdWarps * 32), smem, s, dy,
+                                   x, static_cast<const float*>(w), dx, accumulate, part, rows, C);
+    }
+    if (rc) return rc;
+    const dim3 g((C + 255) / 256), b(256);
+    rc = launch_overlapped(colsum_parts_kernel, g, b, 0, s, static_cast<const float*>(part), 2LL * C, n_part, C, dw,
+                           accumulate_wb);
+    if (rc) return rc;
+    if (!db) return GPT_OK;
+    return launch_overlapped(colsum_parts_kernel, g, b, 0, s, static_cast<const float*>(part + C), 2LL * C, n_part, C,
+                             db, accumulate_wb);
+}
+
+int colsum_parts(int rows) { return (rows + kColRows - 1) / kColRows; }
+
+int launch_colsum(const void* y, int dtype, int rows, int C, float* out, int accumulate, float* part,
+                  cudaStream_t s) {
+    const int n_part = colsum_parts(rows);
+    const dim3 g1((C + 255) / 256, n_part), b(256);
+    int rc = dtype == GPT_DTYPE_BF16
+                 ? launch_overlapped(colsum_rows_kernel<bf16>, g1, b, 0, s, static_cast<const bf16*>(y), rows, C, part)
+                 : launch_overlapped(colsum_rows_kernel<float>, g1, b, 0, s, static_cast<const float*>(y), rows, C,
+                                     part);
+    if (rc) return rc;
+    return launch_overlapped(colsum_parts_kernel, dim3((C + 255) / 256), b, 0, s, static_cast<const float*>(part),
+                             static_cast<long long>(C), n_part, C, out, accumulate);
+}
+
+int launch_gelu_backward(const float* dh, const void* pre, int dtype, void* dpre, long long n, int tanh_form,
+                         cudaStream_t s) {
+    const dim3 g(static_cast<unsigned>((n + 255) / 256)), b(256);
+    if (dtype == GPT_DTYPE_BF16)
+        return launch_overlapped(gelu_backward_kernel<bf16>, g, b, 0, s, dh, static_cast<const bf16*>(pre),
+                                 static_cast<bf16*>(dpre), n, tanh_form);
+    return launch_overlapped(gelu_backward_kernel<float>, g, b, 0, s, dh, static_cast<const float*>(pre),
+                             static_cast<float*>(dpre), n, tanh_form);
+}
+
+int embed_backward_max_rows() { return kEmbSortMax; }
+
+int launch_embed_backward(const int64_t* idx, const float* dx, int B, int T, int C, int V, float* dwte, float* dwpe,
+                          unsigned long long* sorted, int32_t* status, cudaStream_t s) {
+    const int N = B * T;
+    if (N > kEmbSortMax) return GPT_ERR_UNSUPPORTED;
+    int n2 = 1;
+    while (n2 < N) n2 <<= 1;
+    const size_t smem = static_cast<size_t>(n2) * sizeof(unsigned long long);
+    static size_t opted[kMaxDevices] = {};
+    int rc = opt_in_smem(reinterpret_cast<const void*>(embed_sort_kernel), smem, opted);
+    if (rc) return rc;
+    rc = launch_overlapped(embed_sort_kernel, dim3(1), dim3(kEmbSortThreads), smem, s, idx, N, V, sorted, status);
+    if (rc) return rc;
+    rc = launch_overlapped(embed_runs_kernel, dim3((N * 32 + 255) / 256), dim3(256), 0, s,
+                           static_cast<const unsigned long long*>(sorted), N, V, dx, C, dwte);
+    if (rc) return rc;
+    const long long n = static_cast<long long>(T) * C;
+    return launch_overlapped(embed_wpe_kernel, dim3(static_cast<unsigned>((n + 255) / 256)), dim3(256), 0, s, dx, B,
+                             T, C, dwpe);
+}
+
+}  // namespace gpt

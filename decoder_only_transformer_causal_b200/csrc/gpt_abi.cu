@@ -845,3 +845,74 @@ GPT_API int gpt_adamw_step(const gpt_config_t* cfg, float* params, const float* 
     return GPT_OK;
 }
 
+// ------------------------------------------------------------------ backward pieces (backward.cu)
+GPT_API int gpt_cross_entropy_backward(const void* logits, const int64_t* targets, const double* loss_sum_count,
+                                       int rows, int V, int dtype, void* dlogits, int32_t* status, void* stream) {
+    if (!logits || !targets || !loss_sum_count || !dlogits) return GPT_ERR_NULL;
+    if (rows < 0 || V <= 0) return GPT_ERR_BAD_SHAPE;
+    if (dtype != GPT_DTYPE_BF16 && dtype != GPT_DTYPE_F32) return GPT_ERR_BAD_SHAPE;
+    if (rows == 0) return GPT_OK;
+    return launch_ce_backward(logits, dtype, targets, loss_sum_count, dlogits, rows, V, status,
+                              static_cast<cudaStream_t>(stream));
+}
+
+GPT_API size_t gpt_layernorm_backward_workspace_bytes(int rows, int C) {
+    if (rows < 1 || C < 1) return 0;
+    return a256(static_cast<size_t>(layernorm_backward_parts(rows)) * 2 * C * 4);
+}
+
+GPT_API int gpt_layernorm_backward(const float* dy, const float* x, const void* w, int rows, int C, int dtype,
+                                   float* dx, int accumulate, float* dw, float* db, int accumulate_wb, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
+    if (!dy || !x || !w || !dx || !dw || !workspace) return GPT_ERR_NULL;
+    if (rows < 1 || C < 1 || C > 4096) return GPT_ERR_BAD_SHAPE;
+    if (dtype != GPT_DTYPE_BF16 && dtype != GPT_DTYPE_F32) return GPT_ERR_BAD_SHAPE;
+    if (workspace_bytes < gpt_layernorm_backward_workspace_bytes(rows, C)) return GPT_ERR_WS_TOO_SMALL;
+    if (!aligned(workspace, 256)) return GPT_ERR_BAD_ALIGN;
+    return launch_layernorm_backward(dy, x, w, dtype, dx, accumulate, dw, db, accumulate_wb,
+                                     static_cast<float*>(workspace), rows, C, static_cast<cudaStream_t>(stream));
+}
+
+GPT_API size_t gpt_bias_grad_workspace_bytes(int rows, int C) {
+    if (rows < 1 || C < 1) return 0;
+    return a256(static_cast<size_t>(colsum_parts(rows)) * C * 4);
+}
+
+GPT_API int gpt_bias_grad(const void* dy, int rows, int C, int dtype, float* db, int accumulate, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+    if (!dy || !db || !workspace) return GPT_ERR_NULL;
+    if (rows < 1 || C < 1 || rows > 65535 * 128) return GPT_ERR_BAD_SHAPE;
+    if (dtype != GPT_DTYPE_BF16 && dtype != GPT_DTYPE_F32) return GPT_ERR_BAD_SHAPE;
+    if (workspace_bytes < gpt_bias_grad_workspace_bytes(rows, C)) return GPT_ERR_WS_TOO_SMALL;
+    if (!aligned(workspace, 256)) return GPT_ERR_BAD_ALIGN;
+    return launch_colsum(dy, dtype, rows, C, db, accumulate, static_cast<float*>(workspace),
+                         static_cast<cudaStream_t>(stream));
+}
+
+GPT_API int gpt_gelu_backward(const float* dh, const void* pre, long long n, int dtype, int gelu, void* dpre,
+                              void* stream) {
+    if (!dh || !pre || !dpre) return GPT_ERR_NULL;
+    if (n < 0) return GPT_ERR_BAD_SHAPE;
+    if (dtype != GPT_DTYPE_BF16 && dtype != GPT_DTYPE_F32) return GPT_ERR_BAD_SHAPE;
+    if (gelu != GPT_GELU_ERF && gelu != GPT_GELU_TANH) return GPT_ERR_BAD_SHAPE;
+    if (n == 0) return GPT_OK;
+    return launch_gelu_backward(dh, pre, dtype, dpre, n, gelu == GPT_GELU_TANH, static_cast<cudaStream_t>(stream));
+}
+
+GPT_API size_t gpt_embedding_backward_workspace_bytes(int B, int T) {
+    if (B < 1 || T < 1 || static_cast<long long>(B) * T > embed_backward_max_rows()) return 0;
+    return a256(static_cast<size_t>(B) * T * 8);
+}
+
+GPT_API int gpt_embedding_backward(const int64_t* idx, const float* dx, int B, int T, int C, int V, float* dwte,
+                                   float* dwpe, void* workspace, size_t workspace_bytes, int32_t* status,
+                                   void* stream) {
+    if (!idx || !dx || !dwte || !dwpe || !workspace) return GPT_ERR_NULL;
+    if (B < 1 || T < 1 || C < 1 || V < 1) return GPT_ERR_BAD_SHAPE;
+    if (static_cast<long long>(B) * T > embed_backward_max_rows()) return GPT_ERR_UNSUPPORTED;
+    if (workspace_bytes < gpt_embedding_backward_workspace_bytes(B, T)) return GPT_ERR_WS_TOO_SMALL;
+    if (!aligned(workspace, 256)) return GPT_ERR_BAD_ALIGN;
+    return launch_embed_backward(idx, dx, B, T, C, V, dwte, dwpe, static_cast<unsigned long long*>(workspace), status,
+                                 static_cast<cudaStream_t>(stream));
+}
+

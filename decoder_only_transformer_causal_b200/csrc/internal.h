@@ -140,4 +140,19 @@ int launch_adamw(const OptTable& tab, int dtype, float* params, const float* gra
                  float lr, float beta1, float beta2, float eps, float weight_decay, int step, float max_norm,
                  float* norm_out, void* ws, cudaStream_t s);
 
+// ---- backward kernels of the non-matmul pieces (backward.cu)
+int launch_ce_backward(const void* logits, int dtype, const int64_t* targets, const double* sum_count, void* dlogits,
+                       int rows, int V, int32_t* status, cudaStream_t s);
+int layernorm_backward_parts(int rows);  // part: [parts, 2C] floats
+int launch_layernorm_backward(const float* dy, const float* x, const void* w, int dtype, float* dx, int accumulate,
+                              float* dw, float* db, int accumulate_wb, float* part, int rows, int C, cudaStream_t s);
+int colsum_parts(int rows);              // part: [parts, C] floats
+int launch_colsum(const void* y, int dtype, int rows, int C, float* out, int accumulate, float* part,
+                  cudaStream_t s);
+int launch_gelu_backward(const float* dh, const void* pre, int dtype, void* dpre, long long n, int tanh_form,
+                         cudaStream_t s);
+int embed_backward_max_rows();
+int launch_embed_backward(const int64_t* idx, const float* dx, int B, int T, int C, int V, float* dwte, float* dwpe,
+                          unsigned long long* sorted, int32_t* status, cudaStream_t s);
+
 }  // namespace gpt

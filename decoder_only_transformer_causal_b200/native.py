@@ -96,6 +96,14 @@ def _load() -> ctypes.CDLL:
         "gpt_param_elems": (Z, [CFG]),
         "gpt_adamw_workspace_bytes": (Z, []),
         "gpt_adamw_step": (I, [CFG, P, P, P, P, P, ctypes.POINTER(gpt_adamw_t), P, P, Z, P, I]),
+        "gpt_cross_entropy_backward": (I, [P, P, P, I, I, D, P, P, P]),
+        "gpt_layernorm_backward_workspace_bytes": (Z, [I, I]),
+        "gpt_layernorm_backward": (I, [P, P, P, I, I, D, P, I, P, P, I, P, Z, P]),
+        "gpt_bias_grad_workspace_bytes": (Z, [I, I]),
+        "gpt_bias_grad": (I, [P, I, I, D, P, I, P, Z, P]),
+        "gpt_gelu_backward": (I, [P, P, L, D, I, P, P]),
+        "gpt_embedding_backward_workspace_bytes": (Z, [I, I]),
+        "gpt_embedding_backward": (I, [P, P, I, I, I, I, P, P, P, Z, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -112,7 +120,9 @@ EXPORTED = ("gpt_status_string", "gpt_abi_version", "gpt_last_cuda_error", "gpt_
             "gpt_lm_head_workspace_bytes", "gpt_lm_head_loss", "gpt_lm_head_loss_noalloc",
             "gpt_kv_cache_bytes", "gpt_decode_workspace_bytes", "gpt_generate_workspace_bytes", "gpt_prefill",
             "gpt_decode_step", "gpt_sample", "gpt_generate", "gpt_lr_schedule", "gpt_param_elems",
-            "gpt_adamw_workspace_bytes", "gpt_adamw_step")
+            "gpt_adamw_workspace_bytes", "gpt_adamw_step", "gpt_cross_entropy_backward",
+            "gpt_layernorm_backward_workspace_bytes", "gpt_layernorm_backward", "gpt_bias_grad_workspace_bytes",
+            "gpt_bias_grad", "gpt_gelu_backward", "gpt_embedding_backward_workspace_bytes", "gpt_embedding_backward")
 
 
 def status_string(status: int) -> str:
@@ -474,4 +484,68 @@ def adamw_step(cfg: GPTConfig, params: torch.Tensor, grads: torch.Tensor, exp_av
                               _ptr(weights), ctypes.byref(hp), _ptr(grad_norm), _ptr(workspace), workspace.numel(),
                               _stream(stream), GPT_FLAG_SYNC_CHECK if sync_check else 0), "gpt_adamw_step")
     return grad_norm
+
+
+# ---------------------------------------------------------------- backward pieces
+def _dt(t: torch.Tensor) -> int:
+    return {torch.bfloat16: GPT_DTYPE_BF16, torch.float32: GPT_DTYPE_F32}[t.dtype]
+
+
+def cross_entropy_backward(logits: torch.Tensor, targets: torch.Tensor, loss_sum_count: torch.Tensor,
+                           dlogits: torch.Tensor | None = None, status=None, stream=None) -> torch.Tensor:
+    """gpt_cross_entropy_backward: logits [rows, V] (bf16 or fp32), targets int64 [rows],
+    loss_sum_count fp64 [2] from the forward."""
+    V = logits.shape[-1]
+    rows = logits.numel() // V
+    if dlogits is None:
+        dlogits = torch.empty_like(logits)
+    _check(LIB.gpt_cross_entropy_backward(_ptr(logits), _ptr(targets), _ptr(loss_sum_count), rows, V, _dt(logits),
+                                          _ptr(dlogits), _ptr(status), _stream(stream)), "gpt_cross_entropy_backward")
+    return dlogits
+
+
+def layernorm_backward(dy: torch.Tensor, x: torch.Tensor, w: torch.Tensor, dx: torch.Tensor | None = None,
+                       accumulate=False, dw=None, db=None, accumulate_wb=False, stream=None):
+    """gpt_layernorm_backward: dy, x fp32 [rows, C]; w [C] bf16/fp32; returns (dx, dw, db)."""
+    C = x.shape[-1]
+    rows = x.numel() // C
+    if dx is None:
+        dx = torch.empty_like(x)
+    if dw is None:
+        dw = torch.empty(C, dtype=torch.float32, device=x.device)
+    ws = alloc_workspace(LIB.gpt_layernorm_backward_workspace_bytes(rows, C), x.device)
+    _check(LIB.gpt_layernorm_backward(_ptr(dy), _ptr(x), _ptr(w), rows, C, _dt(w), _ptr(dx), int(accumulate),
+                                      _ptr(dw), _ptr(db), int(accumulate_wb), _ptr(ws), ws.numel(), _stream(stream)),
+           "gpt_layernorm_backward")
+    return dx, dw, db
+
+
+def bias_grad(dy: torch.Tensor, db: torch.Tensor | None = None, accumulate=False, stream=None) -> torch.Tensor:
+    C = dy.shape[-1]
+    rows = dy.numel() // C
+    if db is None:
+        db = torch.empty(C, dtype=torch.float32, device=dy.device)
+    ws = alloc_workspace(LIB.gpt_bias_grad_workspace_bytes(rows, C), dy.device)
+    _check(LIB.gpt_bias_grad(_ptr(dy), rows, C, _dt(dy), _ptr(db), int(accumulate), _ptr(ws), ws.numel(),
+                             _stream(stream)), "gpt_bias_grad")
+    return db
+
+
+def gelu_backward(dh: torch.Tensor, pre: torch.Tensor, gelu=GPT_GELU_ERF, dpre=None, stream=None) -> torch.Tensor:
+    if dpre is None:
+        dpre = torch.empty_like(pre)
+    _check(LIB.gpt_gelu_backward(_ptr(dh), _ptr(pre), pre.numel(), _dt(pre), gelu, _ptr(dpre), _stream(stream)),
+           "gpt_gelu_backward")
+    return dpre
+
+
+def embedding_backward(idx: torch.Tensor, dx: torch.Tensor, dwte: torch.Tensor, dwpe: torch.Tensor, status=None,
+                       stream=None):
+    """gpt_embedding_backward: adds into dwte [V, C] and dwpe [>= T, C] (fp32)."""
+    B, T = idx.shape
+    C = dx.shape[-1]
+    ws = alloc_workspace(LIB.gpt_embedding_backward_workspace_bytes(B, T), dx.device)
+    _check(LIB.gpt_embedding_backward(_ptr(idx), _ptr(dx), B, T, C, dwte.shape[0], _ptr(dwte), _ptr(dwpe), _ptr(ws),
+                                      ws.numel(), _ptr(status), _stream(stream)), "gpt_embedding_backward")
+    return dwte, dwpe
 

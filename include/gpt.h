@@ -321,6 +321,51 @@ int gpt_adamw_step(const gpt_config_t* cfg, float* params, const float* grads, f
                    float* exp_avg_sq, void* weights, const gpt_adamw_t* hp, float* grad_norm,
                    void* workspace, size_t workspace_bytes, void* stream, int flags);
 
+/* ---- backward pieces ------------------------------------------------------------------
+ * "nanoGPT 全局流程图", 3.4 反向传播 (loss.backward(): the chain rule from the mean cross-entropy
+ * back to every parameter).  These are the steps of the backward pass that are not matrix
+ * products; each is the derivative of the forward operation named, in fp32 unless stated, with
+ * every reduction in a fixed order (deterministic). */
+
+/* d(loss)/d(logits) for the mean cross-entropy over rows whose target is not -1:
+ * dlogits[r, v] = (softmax(logits[r])[v] - [v == targets[r]]) / n, 0 for ignored rows, n the
+ * counted rows read from loss_sum_count[1] (the {sum, count} pair gpt_forward writes; device
+ * fp64).  logits / dlogits [rows, V] in `dtype`; the softmax is taken over all V columns.  A target
+ * outside [0, V) and != -1 gives a zero row and GPT_ERR_INDEX in *status (optional). */
+int gpt_cross_entropy_backward(const void* logits, const int64_t* targets, const double* loss_sum_count,
+                               int rows, int V, int dtype, void* dlogits, int32_t* status, void* stream);
+
+/* LayerNorm backward (eps 1e-5, population variance): y = xhat w + b.  dy, x, dx fp32 [rows, C]
+ * (C <= 4096); w [C] in `dtype`.  dx = rstd (dxhat - mean(dxhat) - xhat mean(dxhat xhat)) with
+ * dxhat = dy w, added to dx when accumulate != 0.  dw = sum over rows of dy xhat and db = sum of
+ * dy (fp32 [C]; db may be NULL), added when accumulate_wb != 0.  workspace: the column partials,
+ * gpt_layernorm_backward_workspace_bytes(rows, C) bytes, 256-byte aligned. */
+size_t gpt_layernorm_backward_workspace_bytes(int rows, int C);
+int gpt_layernorm_backward(const float* dy, const float* x, const void* w, int rows, int C, int dtype,
+                           float* dx, int accumulate, float* dw, float* db, int accumulate_wb,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bias gradient of a Linear layer: db[c] (+)= sum over rows of dy[r, c]; dy [rows, C] in
+ * `dtype`, db fp32 [C].  workspace: gpt_bias_grad_workspace_bytes(rows, C) bytes. */
+size_t gpt_bias_grad_workspace_bytes(int rows, int C);
+int gpt_bias_grad(const void* dy, int rows, int C, int dtype, float* db, int accumulate,
+                  void* workspace, size_t workspace_bytes, void* stream);
+
+/* GELU backward: dpre = dh * gelu'(pre) elementwise (n elements); dh fp32, pre and dpre in
+ * `dtype`; gelu = GPT_GELU_ERF (Phi(z) + z phi(z)) or GPT_GELU_TANH (the tanh form's derivative). */
+int gpt_gelu_backward(const float* dh, const void* pre, long long n, int dtype, int gelu, void* dpre,
+                      void* stream);
+
+/* Embedding backward ("全局流程图" §3.2 ①: x = wte[idx] + wpe[t]): dwte[v] += sum of dx[b, t] over
+ * the positions with idx[b, t] = v, in position order; dwpe[t] += sum over the batch of dx[b, t].
+ * idx int64 [B, T], dx fp32 [B, T, C], dwte fp32 [V, C], dwpe fp32 [>= T, C].  B * T <= 16384 (the
+ * positions are ordered by token inside one CTA).  workspace: gpt_embedding_backward_workspace_bytes
+ * bytes.  An id outside [0, V) is skipped and GPT_ERR_INDEX written to *status (optional). */
+size_t gpt_embedding_backward_workspace_bytes(int B, int T);
+int gpt_embedding_backward(const int64_t* idx, const float* dx, int B, int T, int C, int V, float* dwte,
+                           float* dwpe, void* workspace, size_t workspace_bytes, int32_t* status,
+                           void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -218,3 +218,22 @@ def test_adamw_host_validation():
     big = ctypes.byref(_cfg("tiny", n_layer=90).c())                                  # > 1024 tensors
     assert Lb.gpt_adamw_step(big, FAKE, FAKE, FAKE, FAKE, None, ctypes.byref(hp), None, FAKE, ws, None, 0) \
         == native.GPT_ERR_UNSUPPORTED
+
+
+def test_backward_pieces_host_validation():
+    Lb = native.LIB
+    bf, f32 = native.GPT_DTYPE_BF16, native.GPT_DTYPE_F32
+    assert Lb.gpt_cross_entropy_backward(None, FAKE, FAKE, 4, 10, bf, FAKE, None, None) == native.GPT_ERR_NULL
+    assert Lb.gpt_cross_entropy_backward(FAKE, FAKE, FAKE, 4, 0, bf, FAKE, None, None) == native.GPT_ERR_BAD_SHAPE
+    assert Lb.gpt_cross_entropy_backward(FAKE, FAKE, FAKE, 4, 10, 7, FAKE, None, None) == native.GPT_ERR_BAD_SHAPE
+    ws = Lb.gpt_layernorm_backward_workspace_bytes(100, 768)
+    assert ws >= ((100 + 7) // 8) * 2 * 768 * 4
+    assert Lb.gpt_layernorm_backward(FAKE, FAKE, FAKE, 100, 768, bf, FAKE, 0, FAKE, None, 0, FAKE, ws - 1, None) \
+        == native.GPT_ERR_WS_TOO_SMALL
+    assert Lb.gpt_layernorm_backward(FAKE, FAKE, FAKE, 100, 5000, bf, FAKE, 0, FAKE, None, 0, FAKE, 1 << 40, None) \
+        == native.GPT_ERR_BAD_SHAPE
+    assert Lb.gpt_bias_grad(FAKE, 10, 8, f32, None, 0, FAKE, 1 << 20, None) == native.GPT_ERR_NULL
+    assert Lb.gpt_gelu_backward(FAKE, FAKE, 10, bf, 5, FAKE, None) == native.GPT_ERR_BAD_SHAPE
+    assert Lb.gpt_embedding_backward_workspace_bytes(16, 1025) == 0                   # > 16384 positions
+    assert Lb.gpt_embedding_backward(FAKE, FAKE, 16, 1025, 8, 10, FAKE, FAKE, FAKE, 1 << 30, None, None) \
+        == native.GPT_ERR_UNSUPPORTED
