@@ -29,6 +29,28 @@ template <typename E> GPT_DEVINL E st1(float v);
 template <> GPT_DEVINL bf16 st1<bf16>(float v) { return __float2bfloat16_rn(v); }
 template <> GPT_DEVINL float st1<float>(float v) { return v; }
 
+// 16-byte L2 loads / stores of 8 bf16 or 4 fp32 values.
+GPT_DEVINL void ld_vec(const bf16* p, float (&f)[8]) {
+    const uint4 w = __ldcg(reinterpret_cast<const uint4*>(p));
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) f[2 * i] = __low2float(h[i]), f[2 * i + 1] = __high2float(h[i]);
+}
+GPT_DEVINL void ld_vec(const float* p, float (&f)[4]) {
+    const float4 w = __ldcg(reinterpret_cast<const float4*>(p));
+    f[0] = w.x, f[1] = w.y, f[2] = w.z, f[3] = w.w;
+}
+GPT_DEVINL void st_vec(bf16* p, const float (&f)[8]) {
+    uint4 w;
+    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&w);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+    *reinterpret_cast<uint4*>(p) = w;
+}
+GPT_DEVINL void st_vec(float* p, const float (&f)[4]) {
+    *reinterpret_cast<float4*>(p) = make_float4(f[0], f[1], f[2], f[3]);
+}
+
 GPT_DEVINL float wsum(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -62,13 +84,31 @@ __global__ void __launch_bounds__(kBwdWarps * 32)
         return;
     }
     float m = -INFINITY, s = 0.f;
-    for (int v = lane; v < V; v += 32) {
-        const float x = ld1(zr + v);
-        if (x > m) {
-            s = s * __expf(m - x) + 1.f;
-            m = x;
-        } else {
-            s += __expf(x - m);
+    constexpr int VW = 16 / sizeof(E);  // elements per 16-byte access
+    const bool vec = (V % VW) == 0;     // rows are then 16-byte aligned
+    if (vec) {
+        for (int v = lane * VW; v < V; v += 32 * VW) {
+            float f[VW];
+            ld_vec(zr + v, f);
+            float mx = f[0];
+#pragma unroll
+            for (int e = 1; e < VW; ++e) mx = fmaxf(mx, f[e]);
+            const float mn = fmaxf(m, mx);
+            float add = 0.f;
+#pragma unroll
+            for (int e = 0; e < VW; ++e) add += __expf(f[e] - mn);
+            s = (m == -INFINITY ? 0.f : s * __expf(m - mn)) + add;
+            m = mn;
+        }
+    } else {
+        for (int v = lane; v < V; v += 32) {
+            const float x = ld1(zr + v);
+            if (x > m) {
+                s = s * __expf(m - x) + 1.f;
+                m = x;
+            } else {
+                s += __expf(x - m);
+            }
         }
     }
 #pragma unroll
@@ -80,9 +120,19 @@ __global__ void __launch_bounds__(kBwdWarps * 32)
     }
     const float lse = m + __logf(s);
     const float inv_n = static_cast<float>(1.0 / n);
-    for (int v = lane; v < V; v += 32) {
-        const float p = __expf(ld1(zr + v) - lse);
-        dr[v] = st1<E>((p - (v == t ? 1.f : 0.f)) * inv_n);
+    if (vec) {
+        for (int v = lane * VW; v < V; v += 32 * VW) {
+            float f[VW];
+            ld_vec(zr + v, f);
+#pragma unroll
+            for (int e = 0; e < VW; ++e) f[e] = (__expf(f[e] - lse) - (v + e == t ? 1.f : 0.f)) * inv_n;
+            st_vec(dr + v, f);
+        }
+    } else {
+        for (int v = lane; v < V; v += 32) {
+            const float p = __expf(ld1(zr + v) - lse);
+            dr[v] = st1<E>((p - (v == t ? 1.f : 0.f)) * inv_n);
+        }
     }
 }
 
@@ -141,6 +191,94 @@ __global__ void __launch_bounds__(kBwdWarps * 32)
     }
 }
 
+// The same with each row held in registers (VEC float4 of x and of dy per lane, C <= 128 VEC):
+// x and dy are read once, and each warp takes kLnRowsPerWarp consecutive rows into its column
+// sums, so a CTA leaves one partial per 64 rows.
+constexpr int kLnRowsPerWarp = 8;  // rows per warp in the register kernel: 64 per CTA
+
+template <typename Tw, int VEC>
+__global__ void __launch_bounds__(kBwdWarps * 32)
+    layernorm_backward_reg_kernel(const float* __restrict__ dy, const float* __restrict__ x, const Tw* __restrict__ w,
+                                  float* __restrict__ dx, int accumulate, float* __restrict__ part, int rows, int C) {
+    griddep_launch_dependents();
+    griddep_wait();
+    extern __shared__ float sm[];  // [kBwdWarps][2][C] per-warp column sums
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    float* my = sm + static_cast<size_t>(warp) * 2 * C;
+    for (int c = lane; c < 2 * C; c += 32) my[c] = 0.f;
+    __syncwarp();
+    float4 wv[VEC];
+#pragma unroll
+    for (int j = 0; j < VEC; ++j) {
+        const int c = (lane + 32 * j) * 4;
+        if (c < C) wv[j] = make_float4(ld1(w + c), ld1(w + c + 1), ld1(w + c + 2), ld1(w + c + 3));
+    }
+    const int r0 = (blockIdx.x * kBwdWarps + warp) * kLnRowsPerWarp;
+    for (int r = r0; r < min(rows, r0 + kLnRowsPerWarp); ++r) {
+        const float* xr = x + static_cast<long long>(r) * C;
+        const float* dyr = dy + static_cast<long long>(r) * C;
+        float4 xv[VEC], gv[VEC];
+        float s = 0.f;
+#pragma unroll
+        for (int j = 0; j < VEC; ++j) {
+            const int c = (lane + 32 * j) * 4;
+            if (c < C) {
+                xv[j] = __ldcg(reinterpret_cast<const float4*>(xr + c));
+                gv[j] = __ldcg(reinterpret_cast<const float4*>(dyr + c));
+                s += (xv[j].x + xv[j].y) + (xv[j].z + xv[j].w);
+            }
+        }
+        const float mean = wsum(s) / C;
+        float ss = 0.f;
+#pragma unroll
+        for (int j = 0; j < VEC; ++j) {
+            const int c = (lane + 32 * j) * 4;
+            if (c < C) {
+                xv[j].x -= mean, xv[j].y -= mean, xv[j].z -= mean, xv[j].w -= mean;
+                ss += (xv[j].x * xv[j].x + xv[j].y * xv[j].y) + (xv[j].z * xv[j].z + xv[j].w * xv[j].w);
+            }
+        }
+        const float rstd = rsqrtf(wsum(ss) / C + 1e-5f);
+        float a = 0.f, bsum = 0.f;  // sums of dxhat and dxhat * xhat
+#pragma unroll
+        for (int j = 0; j < VEC; ++j) {
+            const int c = (lane + 32 * j) * 4;
+            if (c < C) {
+                xv[j].x *= rstd, xv[j].y *= rstd, xv[j].z *= rstd, xv[j].w *= rstd;  // xhat
+                a += (gv[j].x * wv[j].x + gv[j].y * wv[j].y) + (gv[j].z * wv[j].z + gv[j].w * wv[j].w);
+                bsum += (gv[j].x * wv[j].x * xv[j].x + gv[j].y * wv[j].y * xv[j].y) +
+                        (gv[j].z * wv[j].z * xv[j].z + gv[j].w * wv[j].w * xv[j].w);
+                my[c] += gv[j].x * xv[j].x, my[c + 1] += gv[j].y * xv[j].y;
+                my[c + 2] += gv[j].z * xv[j].z, my[c + 3] += gv[j].w * xv[j].w;
+                my[C + c] += gv[j].x, my[C + c + 1] += gv[j].y, my[C + c + 2] += gv[j].z, my[C + c + 3] += gv[j].w;
+            }
+        }
+        const float ma = wsum(a) / C, mb = wsum(bsum) / C;
+        float* dxr = dx + static_cast<long long>(r) * C;
+#pragma unroll
+        for (int j = 0; j < VEC; ++j) {
+            const int c = (lane + 32 * j) * 4;
+            if (c < C) {
+                float4 o = make_float4(rstd * (gv[j].x * wv[j].x - ma - xv[j].x * mb),
+                                       rstd * (gv[j].y * wv[j].y - ma - xv[j].y * mb),
+                                       rstd * (gv[j].z * wv[j].z - ma - xv[j].z * mb),
+                                       rstd * (gv[j].w * wv[j].w - ma - xv[j].w * mb));
+                if (accumulate) {
+                    const float4 old = __ldcg(reinterpret_cast<const float4*>(dxr + c));
+                    o.x += old.x, o.y += old.y, o.z += old.z, o.w += old.w;
+                }
+                *reinterpret_cast<float4*>(dxr + c) = o;
+            }
+        }
+    }
+    __syncthreads();
+    for (int c = threadIdx.x; c < 2 * C; c += kBwdWarps * 32) {
+        float v = 0.f;
+        for (int wp = 0; wp < kBwdWarps; ++wp) v += sm[static_cast<size_t>(wp) * 2 * C + c];
+        part[static_cast<long long>(blockIdx.x) * 2 * C + c] = v;
+    }
+}
+
 // out[c] (+)= sum over i < n_part of part[i * ld + c], in order of i (the second stage of a
 // column reduction).
 __global__ void colsum_parts_kernel(const float* __restrict__ part, long long ld, int n_part, int C,
@@ -150,6 +288,7 @@ __global__ void colsum_parts_kernel(const float* __restrict__ part, long long ld
     const int c = blockIdx.x * blockDim.x + threadIdx.x;
     if (c >= C) return;
     float v = 0.f;
+#pragma unroll 8
     for (int i = 0; i < n_part; ++i) v += __ldcg(part + i * ld + c);
     out[c] = accumulate ? __ldcg(out + c) + v : v;
 }
@@ -285,15 +424,37 @@ int launch_ce_backward(const void* logits, int dtype, const int64_t* targets, co
                              sum_count, static_cast<float*>(dlogits), rows, V, status);
 }
 
-int layernorm_backward_parts(int rows) { return (rows + kBwdWarps - 1) / kBwdWarps; }
+int layernorm_backward_parts(int rows, int C) {
+    const int per = (C <= 2048 && C % 4 == 0) ? kBwdWarps * kLnRowsPerWarp : kBwdWarps;
+    return (rows + per - 1) / per;
+}
+
+namespace {
+template <typename Tw, int VEC = 1>
+int launch_ln_bwd_reg(const float* dy, const float* x, const void* w, float* dx, int accumulate, float* part, int rows,
+                      int C, size_t smem, cudaStream_t s) {
+    if constexpr (VEC < 16) {
+        if (C > 128 * VEC) return launch_ln_bwd_reg<Tw, VEC + 1>(dy, x, w, dx, accumulate, part, rows, C, smem, s);
+    }
+    static size_t opted[kMaxDevices] = {};
+    const int rc = opt_in_smem(reinterpret_cast<const void*>(layernorm_backward_reg_kernel<Tw, VEC>), smem, opted);
+    if (rc) return rc;
+    return launch_overlapped(layernorm_backward_reg_kernel<Tw, VEC>, dim3(layernorm_backward_parts(rows, C)),
+                             dim3(kBwdWarps * 32), smem, s, dy, x, static_cast<const Tw*>(w), dx, accumulate, part,
+                             rows, C);
+}
+}  // namespace
 
 int launch_layernorm_backward(const float* dy, const float* x, const void* w, int dtype, float* dx, int accumulate,
                               float* dw, float* db, int accumulate_wb, float* part, int rows, int C,
                               cudaStream_t s) {
-    const int n_part = layernorm_backward_parts(rows);
+    const int n_part = layernorm_backward_parts(rows, C);
     const size_t smem = static_cast<size_t>(kBwdWarps) * 2 * C * sizeof(float);
     int rc;
-    if (dtype == GPT_DTYPE_BF16) {
+    if (C <= 2048 && C % 4 == 0) {
+        rc = dtype == GPT_DTYPE_BF16 ? launch_ln_bwd_reg<bf16>(dy, x, w, dx, accumulate, part, rows, C, smem, s)
+                                     : launch_ln_bwd_reg<float>(dy, x, w, dx, accumulate, part, rows, C, smem, s);
+    } else if (dtype == GPT_DTYPE_BF16) {
         static size_t opted[kMaxDevices] = {};
         rc = opt_in_smem(reinterpret_cast<const void*>(layernorm_backward_kernel<bf16>), smem, opted);
         if (!rc)

@@ -858,7 +858,7 @@ GPT_API int gpt_cross_entropy_backward(const void* logits, const int64_t* target
 
 GPT_API size_t gpt_layernorm_backward_workspace_bytes(int rows, int C) {
     if (rows < 1 || C < 1) return 0;
-    return a256(static_cast<size_t>(layernorm_backward_parts(rows)) * 2 * C * 4);
+    return a256(static_cast<size_t>(layernorm_backward_parts(rows, C)) * 2 * C * 4);
 }
 
 GPT_API int gpt_layernorm_backward(const float* dy, const float* x, const void* w, int rows, int C, int dtype,
