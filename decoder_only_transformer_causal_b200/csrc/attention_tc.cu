@@ -41,6 +41,7 @@ int launch_attention_bf16(const AttnLayout& L, int B, int nh, int T, int32_t* st
     p.y_st = L.y_st;
     p.scale_log2 = static_cast<float>(1.4426950408889634 / sqrt(static_cast<double>(attn::HS)));
     p.status = status;
+    p.lse = L.lse;
 
     static size_t opted[kMaxDevices] = {};
     rc = opt_in_smem(reinterpret_cast<const void*>(attn::attention_fwd_tc), attn::SMEM_BYTES, opted);

@@ -58,6 +58,7 @@ struct Params {
     long long y_sb, y_sh, y_st;  // element strides of y for b, h, t (hs is contiguous)
     float scale_log2;        // log2(e) / sqrt(hs)
     int32_t* status;
+    float* lse;              // optional [B, nh, T]: m + log2(l) per row (log2 units of the scaled score)
 };
 
 __global__ void __launch_bounds__(THREADS, 2)
@@ -312,6 +313,7 @@ __global__ void __launch_bounds__(THREADS, 2)
             tc_fence_after();
             const int t = q0 + r;
             const float inv_l = 1.f / l;
+            if (p.lse && t < p.T) p.lse[(static_cast<long long>(b) * p.nh + h) * p.T + t] = m_used + __log2f(l);
             uint32_t out[32];
 #pragma unroll
             for (int c = 0; c < HS; c += 32) {

@@ -916,3 +916,61 @@ GPT_API int gpt_embedding_backward(const int64_t* idx, const float* dx, int B, i
                                  static_cast<cudaStream_t>(stream));
 }
 
+// ------------------------------------------------------------------ attention for training (train.cu)
+GPT_API int gpt_attention_train(const void* q, const void* k, const void* v, void* y, float* lse, int B, int nh, int T,
+                                int hs, int dtype, int32_t* status, void* stream) {
+    if (!q || !k || !v || !y || !lse) return GPT_ERR_NULL;
+    if (B < 0 || nh < 0 || T < 0 || hs <= 0) return GPT_ERR_BAD_SHAPE;
+    if (dtype != GPT_DTYPE_BF16 && dtype != GPT_DTYPE_F32) return GPT_ERR_BAD_SHAPE;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(y, 16)) return GPT_ERR_BAD_ALIGN;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const long long sh = static_cast<long long>(T) * hs, sb = sh * nh;
+    if (dtype == GPT_DTYPE_BF16) {
+        if (hs != 64) return GPT_ERR_UNSUPPORTED;
+        AttnLayout L{static_cast<const bf16*>(q), static_cast<const bf16*>(k), static_cast<const bf16*>(v), sb, sh, hs,
+                     static_cast<bf16*>(y), sb, sh, hs, lse};
+        return launch_attention_bf16(L, B, nh, T, status, s);
+    }
+    if (hs > 128) return GPT_ERR_UNSUPPORTED;
+    AttnLayoutF32 L{static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v), sb, sh, hs,
+                    static_cast<float*>(y), sb, sh, hs, lse};
+    return launch_attention_f32(L, B, nh, T, hs, s);
+}
+
+GPT_API size_t gpt_attention_backward_workspace_bytes(int B, int nh, int T) {
+    if (B < 1 || nh < 1 || T < 1) return 0;
+    return a256(static_cast<size_t>(B) * nh * T * 4);
+}
+
+GPT_API int gpt_attention_backward(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                                   const float* lse, void* dq, void* dk, void* dv, int B, int nh, int T, int hs,
+                                   int dtype, void* workspace, size_t workspace_bytes, void* stream) {
+    if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !workspace) return GPT_ERR_NULL;
+    if (B < 0 || nh < 0 || T < 0 || hs <= 0) return GPT_ERR_BAD_SHAPE;
+    if (dtype != GPT_DTYPE_BF16 && dtype != GPT_DTYPE_F32) return GPT_ERR_BAD_SHAPE;
+    if (hs != 32 && hs != 64) return GPT_ERR_UNSUPPORTED;
+    if (workspace_bytes < gpt_attention_backward_workspace_bytes(B, nh, T)) return GPT_ERR_WS_TOO_SMALL;
+    const long long sh = static_cast<long long>(T) * hs, sb = sh * nh;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    float* D = static_cast<float*>(workspace);
+    if (dtype == GPT_DTYPE_BF16) {
+        AttnBwdLayout<bf16> L{static_cast<const bf16*>(q), static_cast<const bf16*>(k), static_cast<const bf16*>(v),
+                              sb, sh, hs, static_cast<const bf16*>(o), static_cast<const bf16*>(dout), sb, sh, hs,
+                              static_cast<bf16*>(dq), static_cast<bf16*>(dk), static_cast<bf16*>(dv), lse};
+        return launch_attention_backward(&L, nullptr, B, nh, T, hs, D, s);
+    }
+    AttnBwdLayout<float> L{static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v), sb,
+                           sh, hs, static_cast<const float*>(o), static_cast<const float*>(dout), sb, sh, hs,
+                           static_cast<float*>(dq), static_cast<float*>(dk), static_cast<float*>(dv), lse};
+    return launch_attention_backward(nullptr, &L, B, nh, T, hs, D, s);
+}
+
+GPT_API int gpt_transpose(const void* in, int in_dtype, long long ld_in, void* out, int out_dtype, long long ld_out,
+                          int rows, int cols, void* stream) {
+    if (!in || !out) return GPT_ERR_NULL;
+    if (rows < 0 || cols < 0 || ld_in < cols || ld_out < rows) return GPT_ERR_BAD_SHAPE;
+    for (int d : {in_dtype, out_dtype})
+        if (d != GPT_DTYPE_BF16 && d != GPT_DTYPE_F32) return GPT_ERR_BAD_SHAPE;
+    return launch_transpose(in, in_dtype, ld_in, out, out_dtype, ld_out, rows, cols, static_cast<cudaStream_t>(stream));
+}
+

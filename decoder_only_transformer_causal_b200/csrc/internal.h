@@ -85,6 +85,7 @@ struct AttnLayout {
     long long sb, sh, st;  // strides of q/k/v for batch, head, position (hs contiguous)
     bf16* y;
     long long y_sb, y_sh, y_st;
+    float* lse = nullptr;  // optional [B, nh, T]: log2 sum_j 2^(s_ij * scale_log2), for the backward
 };
 int launch_attention_bf16(const AttnLayout& L, int B, int nh, int T, int32_t* status, cudaStream_t s);
 
@@ -96,6 +97,7 @@ struct AttnLayoutF32 {
     long long sb, sh, st;
     float* y;
     long long y_sb, y_sh, y_st;
+    float* lse = nullptr;  // optional [B, nh, T], as in AttnLayout
 };
 int launch_attention_f32(const AttnLayoutF32& L, int B, int nh, int T, int hs, cudaStream_t s);
 
@@ -154,5 +156,23 @@ int launch_gelu_backward(const float* dh, const void* pre, int dtype, void* dpre
 int embed_backward_max_rows();
 int launch_embed_backward(const int64_t* idx, const float* dx, int B, int T, int C, int V, float* dwte, float* dwpe,
                           unsigned long long* sorted, int32_t* status, cudaStream_t s);
+
+// ---- training-step helpers and the attention backward (train.cu)
+template <typename E>
+struct AttnBwdLayout {
+    const E *q, *k, *v;             // forward inputs, strides sb, sh, st (hs contiguous)
+    long long sb, sh, st;
+    const E *o, *dout;              // forward output and its gradient, strides o_sb, o_sh, o_st
+    long long o_sb, o_sh, o_st;
+    E *dq, *dk, *dv;                // gradients, with the q / k / v strides
+    const float* lse;               // [B, nh, T] from the forward
+};
+int launch_transpose(const void* in, int in_dtype, long long ld_in, void* out, int out_dtype, long long ld_out, int R,
+                     int Cc, cudaStream_t s);
+int launch_convert(const void* in, int in_dtype, void* out, int out_dtype, long long n, cudaStream_t s);
+int launch_gelu_forward(const void* pre, void* h, long long n, int dtype, int tanh_form, cudaStream_t s);
+// D: [B, nh, T] fp32 scratch.  Exactly one of Lb / Lf is non-null; hs 32 or 64.
+int launch_attention_backward(const AttnBwdLayout<bf16>* Lb, const AttnBwdLayout<float>* Lf, int B, int nh, int T,
+                              int hs, float* D, cudaStream_t s);
 
 }  // namespace gpt

@@ -116,6 +116,7 @@ __global__ void __launch_bounds__(kAttWarps * 32)
     for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
     __syncwarp();
     const float inv = 1.f / sum;
+    if (L.lse && lane == 0) L.lse[static_cast<long long>(bh) * T + i] = (mx + logf(sum)) * 1.4426950408889634f;
     float* y = L.y + b * L.y_sb + h * L.y_sh + static_cast<long long>(i) * L.y_st;
     for (int d = lane; d < hs; d += 32) {
         float acc = 0.f;

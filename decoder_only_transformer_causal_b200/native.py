@@ -104,6 +104,10 @@ def _load() -> ctypes.CDLL:
         "gpt_gelu_backward": (I, [P, P, L, D, I, P, P]),
         "gpt_embedding_backward_workspace_bytes": (Z, [I, I]),
         "gpt_embedding_backward": (I, [P, P, I, I, I, I, P, P, P, Z, P, P]),
+        "gpt_attention_train": (I, [P, P, P, P, P, I, I, I, I, D, P, P]),
+        "gpt_attention_backward_workspace_bytes": (Z, [I, I, I]),
+        "gpt_attention_backward": (I, [P, P, P, P, P, P, P, P, P, I, I, I, I, D, P, Z, P]),
+        "gpt_transpose": (I, [P, D, L, P, D, L, I, I, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -122,7 +126,8 @@ EXPORTED = ("gpt_status_string", "gpt_abi_version", "gpt_last_cuda_error", "gpt_
             "gpt_decode_step", "gpt_sample", "gpt_generate", "gpt_lr_schedule", "gpt_param_elems",
             "gpt_adamw_workspace_bytes", "gpt_adamw_step", "gpt_cross_entropy_backward",
             "gpt_layernorm_backward_workspace_bytes", "gpt_layernorm_backward", "gpt_bias_grad_workspace_bytes",
-            "gpt_bias_grad", "gpt_gelu_backward", "gpt_embedding_backward_workspace_bytes", "gpt_embedding_backward")
+            "gpt_bias_grad", "gpt_gelu_backward", "gpt_embedding_backward_workspace_bytes", "gpt_embedding_backward",
+            "gpt_attention_train", "gpt_attention_backward_workspace_bytes", "gpt_attention_backward", "gpt_transpose")
 
 
 def status_string(status: int) -> str:
@@ -548,4 +553,33 @@ def embedding_backward(idx: torch.Tensor, dx: torch.Tensor, dwte: torch.Tensor, 
     _check(LIB.gpt_embedding_backward(_ptr(idx), _ptr(dx), B, T, C, dwte.shape[0], _ptr(dwte), _ptr(dwpe), _ptr(ws),
                                       ws.numel(), _ptr(status), _stream(stream)), "gpt_embedding_backward")
     return dwte, dwpe
+
+
+def attention_train(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, status=None, stream=None):
+    """gpt_attention_train: returns (y, lse) for q, k, v [B, nh, T, hs]."""
+    B, nh, T, hs = q.shape
+    y = torch.empty_like(q)
+    lse = torch.empty((B, nh, T), dtype=torch.float32, device=q.device)
+    _check(LIB.gpt_attention_train(_ptr(q), _ptr(k), _ptr(v), _ptr(y), _ptr(lse), B, nh, T, hs, _dt(q), _ptr(status),
+                                   _stream(stream)), "gpt_attention_train")
+    return y, lse
+
+
+def attention_backward(q, k, v, o, dout, lse, stream=None):
+    """gpt_attention_backward: returns (dq, dk, dv) for [B, nh, T, hs] tensors."""
+    B, nh, T, hs = q.shape
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = alloc_workspace(LIB.gpt_attention_backward_workspace_bytes(B, nh, T), q.device)
+    _check(LIB.gpt_attention_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
+                                      _ptr(dv), B, nh, T, hs, _dt(q), _ptr(ws), ws.numel(), _stream(stream)),
+           "gpt_attention_backward")
+    return dq, dk, dv
+
+
+def transpose(x: torch.Tensor, out_dtype=None, stream=None) -> torch.Tensor:
+    """gpt_transpose of a 2-D tensor (optionally converting bf16 <-> fp32)."""
+    R, Cc = x.shape
+    out = torch.empty((Cc, R), dtype=out_dtype or x.dtype, device=x.device)
+    _check(LIB.gpt_transpose(_ptr(x), _dt(x), Cc, _ptr(out), _dt(out), R, R, Cc, _stream(stream)), "gpt_transpose")
+    return out
 

@@ -366,6 +366,27 @@ int gpt_embedding_backward(const int64_t* idx, const float* dx, int B, int T, in
                            float* dwpe, void* workspace, size_t workspace_bytes, int32_t* status,
                            void* stream);
 
+/* Causal attention as gpt_attention, also writing lse [B, nh, T] fp32: for each query row,
+ * log2 of sum_j 2^(s_ij log2(e) / sqrt(hs)) with s_ij = q_i . k_j — the row's log-sum-exp in
+ * base-2 units of the scaled score, which lets the backward recompute the probabilities. */
+int gpt_attention_train(const void* q, const void* k, const void* v, void* y, float* lse, int B, int nh,
+                        int T, int hs, int dtype, int32_t* status, void* stream);
+
+/* Backward of causal attention ("全局流程图" 3.4 applied to §2.5 (B)): with p_ij recomputed from
+ * q, k and lse, D_i = dout_i . o_i and dS_ij = p_ij (dout_i . v_j - D_i) for j <= i,
+ *   dq_i = sum_j dS_ij k_j / sqrt(hs),  dk_j = sum_i dS_ij q_i / sqrt(hs),  dv_j = sum_i p_ij dout_i.
+ * All [B, nh, T, hs] in `dtype` (o = the forward's y, lse from gpt_attention_train); hs 32 or 64;
+ * fp32 accumulation.  workspace: gpt_attention_backward_workspace_bytes(B, nh, T) bytes (D). */
+size_t gpt_attention_backward_workspace_bytes(int B, int nh, int T);
+int gpt_attention_backward(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                           const float* lse, void* dq, void* dk, void* dv, int B, int nh, int T, int hs,
+                           int dtype, void* workspace, size_t workspace_bytes, void* stream);
+
+/* out[c * ld_out + r] = in[r * ld_in + c] for r < rows, c < cols, converting between bf16 and fp32
+ * (the operand layouts of the backward's products). */
+int gpt_transpose(const void* in, int in_dtype, long long ld_in, void* out, int out_dtype,
+                  long long ld_out, int rows, int cols, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
