@@ -12,7 +12,7 @@ import torch
 from . import native
 from .native import GPTConfig, GPTError  # noqa: F401
 
-__all__ = ["GPT", "GPTConfig", "GPTError", "AdamW", "native"]
+__all__ = ["GPT", "GPTConfig", "GPTError", "AdamW", "Trainer", "native"]
 
 
 class GPT:
@@ -112,4 +112,26 @@ class AdamW:
                                  weights=self.model.weights, betas=self.betas, eps=self.eps,
                                  weight_decay=self.weight_decay, max_grad_norm=self.max_grad_norm,
                                  grad_norm=self.grad_norm, workspace=self.workspace)
+
+
+class Trainer:
+    """One training step of the pages ("nanoGPT 全局流程图" 3.2-3.6) on a GPT: forward with targets
+    keeping activations, the backward into a flat fp32 gradient array, then the AdamW step
+    (clipping, schedule, decay on matrices), which also refreshes the model's packed weights.
+    ``step(idx, targets)`` returns the batch's loss as a device scalar."""
+
+    def __init__(self, model: GPT, tensors: dict, B: int, T: int, **adamw):
+        self.model = model
+        self.opt = AdamW(model, tensors, **adamw)
+        self.acts, self.fws, self.bws = native.train_buffers(model.cfg, B, T, model.device)
+        self.grads = torch.zeros_like(self.opt.params)
+        self.loss = torch.empty((), dtype=torch.float32, device=model.device)
+
+    def step(self, idx: torch.Tensor, targets: torch.Tensor) -> torch.Tensor:
+        cfg, w = self.model.cfg, self.model.weights
+        native.forward_train(cfg, w, idx, targets, self.acts, self.fws, loss=self.loss)
+        self.grads.zero_()
+        native.backward(cfg, w, idx, targets, self.acts, self.grads, self.bws)
+        self.opt.step(self.grads)
+        return self.loss
 

@@ -4,6 +4,7 @@
 #include <math.h>
 #include <string.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "internal.h"
@@ -972,5 +973,327 @@ GPT_API int gpt_transpose(const void* in, int in_dtype, long long ld_in, void* o
     for (int d : {in_dtype, out_dtype})
         if (d != GPT_DTYPE_BF16 && d != GPT_DTYPE_F32) return GPT_ERR_BAD_SHAPE;
     return launch_transpose(in, in_dtype, ld_in, out, out_dtype, ld_out, rows, cols, static_cast<cudaStream_t>(stream));
+}
+
+// ------------------------------------------------------------------ training step: forward + backward
+namespace {
+
+// Activations the backward needs, per layer and at the end (N = B * T rows, E = storage type).
+struct ActPlan {
+    size_t x_in, u1, qkv, y, lse, x_mid, u2, pre, h, layer;  // offsets within a layer's block
+    size_t final_off, x_f, u_f, logits, sum_count, total;
+};
+
+ActPlan plan_acts(const gpt_config_t* c, long long B, long long T) {
+    ActPlan A{};
+    const size_t N = static_cast<size_t>(B * T), C = c->n_embd, es = elem_size(c);
+    size_t off = 0;
+    A.x_in = off; off += a256(N * C * 4);
+    A.u1 = off; off += a256(N * C * es);
+    A.qkv = off; off += a256(N * 3 * C * es);
+    A.y = off; off += a256(N * C * es);
+    A.lse = off; off += a256(static_cast<size_t>(B) * c->n_head * T * 4);
+    A.x_mid = off; off += a256(N * C * 4);
+    A.u2 = off; off += a256(N * C * es);
+    A.pre = off; off += a256(N * 4 * C * es);
+    A.h = off; off += a256(N * 4 * C * es);
+    A.layer = off;
+    size_t f = A.layer * c->n_layer;
+    A.final_off = f;
+    A.x_f = f; f += a256(N * C * 4);
+    A.u_f = f; f += a256(N * C * es);
+    A.logits = f; f += a256(N * static_cast<size_t>(c->vocab_size) * es);
+    A.sum_count = f; f += 256;
+    A.total = f;
+    return A;
+}
+
+// Scratch of the backward pass.
+struct BwdPlan {
+    size_t ctrl, dz, dzT, wT, gE, gT, aT, d1, dx, dpre, dqkv, dy, D, parts, sort, total;
+};
+
+BwdPlan plan_bwd(const gpt_config_t* c, long long B, long long T) {
+    BwdPlan P{};
+    const size_t N = static_cast<size_t>(B * T), C = c->n_embd, V = c->vocab_size, es = elem_size(c);
+    size_t off = 0;
+    P.ctrl = off; off += 256;
+    P.dz = off; off += a256(N * V * es);
+    P.dzT = off; off += a256(N * V * es);
+    P.wT = off; off += a256(std::max(V * C, 4 * C * C) * es);
+    P.gE = off; off += a256(N * 4 * C * es);
+    P.gT = off; off += a256(N * 4 * C * es);
+    P.aT = off; off += a256(N * 4 * C * es);
+    P.d1 = off; off += a256(N * 4 * C * 4);
+    P.dx = off; off += a256(N * C * 4);
+    P.dpre = off; off += a256(N * 4 * C * es);
+    P.dqkv = off; off += a256(N * 3 * C * es);
+    P.dy = off; off += a256(N * C * es);
+    P.D = off; off += a256(static_cast<size_t>(B) * c->n_head * T * 4);
+    const size_t lnp = static_cast<size_t>(layernorm_backward_parts(static_cast<int>(N), static_cast<int>(C))) * 2 * C;
+    const size_t csp = static_cast<size_t>(colsum_parts(static_cast<int>(N))) * 4 * C;
+    P.parts = off; off += a256(std::max(lnp, csp) * 4);
+    P.sort = off; off += a256(N * 8);
+    P.total = off;
+    return P;
+}
+
+int check_train(const gpt_config_t* c, const void* weights, const int64_t* idx, const int64_t* targets, int B, int T,
+                const void* acts, size_t acts_bytes, ActPlan* A) {
+    GPT_TRY(validate(c));
+    if (!weights || !idx || !targets || !acts) return GPT_ERR_NULL;
+    if (B < 1 || T < 1 || T > c->block_size) return GPT_ERR_BAD_SHAPE;
+    const int hs = c->n_embd / c->n_head;
+    if (hs != 32 && hs != 64) return GPT_ERR_UNSUPPORTED;
+    const long long N = static_cast<long long>(B) * T;
+    if (c->dtype == GPT_DTYPE_BF16 && (N % 8)) return GPT_ERR_UNSUPPORTED;  // K of the weight-gradient products
+    if (N > embed_backward_max_rows()) return GPT_ERR_UNSUPPORTED;
+    if (N * std::max<long long>(c->vocab_size, 4LL * c->n_embd) > 0x7fffffffLL) return GPT_ERR_UNSUPPORTED;
+    if (!aligned(weights, 256) || !aligned(acts, 256)) return GPT_ERR_BAD_ALIGN;
+    *A = plan_acts(c, B, T);
+    if (acts_bytes < A->total) return GPT_ERR_WS_TOO_SMALL;
+    return GPT_OK;
+}
+
+// out[M, N] (fp32) += A[M, K] B[N, K]^T with A, B dense (row strides lda, ldb) in the config dtype.
+int gemm_acc(const gpt_config_t* c, const void* A, long long lda, const void* Bm, long long ldb, float* out,
+             long long ldo, int M, int N, int K, int32_t* status, cudaStream_t s) {
+    if (c->dtype == GPT_DTYPE_BF16)
+        return launch_gemm_bf16(static_cast<const bf16*>(A), lda, static_cast<const bf16*>(Bm), ldb, nullptr, out, ldo,
+                                M, N, K, GPT_EPI_RESID, c->gelu, nullptr, status, s);
+    if (ldb != K) return GPT_ERR_UNSUPPORTED;
+    return launch_linear_f32(static_cast<const float*>(A), lda, static_cast<const float*>(Bm), nullptr, out, ldo, M, N,
+                             K, GPT_EPI_RESID, c->gelu, s);
+}
+
+}  // namespace
+
+GPT_API size_t gpt_train_activation_bytes(const gpt_config_t* cfg, int B, int T) {
+    if (validate(cfg) != GPT_OK || B < 1 || T < 1 || T > cfg->block_size) return 0;
+    return plan_acts(cfg, B, T).total;
+}
+
+GPT_API size_t gpt_backward_workspace_bytes(const gpt_config_t* cfg, int B, int T) {
+    if (validate(cfg) != GPT_OK || B < 1 || T < 1 || T > cfg->block_size) return 0;
+    return plan_bwd(cfg, B, T).total;
+}
+
+GPT_API int gpt_forward_train(const gpt_config_t* cfg, const void* weights, const int64_t* idx, const int64_t* targets,
+                              int B, int T, void* acts, size_t acts_bytes, float* loss, void* workspace,
+                              size_t workspace_bytes, void* stream, int flags) {
+    ActPlan A;
+    GPT_TRY(check_train(cfg, weights, idx, targets, B, T, acts, acts_bytes, &A));
+    Plan P;
+    GPT_TRY(check_common(cfg, weights, B, T, workspace, workspace_bytes, &P));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    Weights W;
+    fill_weights(W, cfg, weights);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    uint8_t* ab = static_cast<uint8_t*>(acts);
+    int32_t* status = status_word(ws);
+    const int C = cfg->n_embd, V = cfg->vocab_size, nh = cfg->n_head, hs = C / nh, N = B * T, dt = cfg->dtype;
+    const size_t es = elem_size(cfg);
+    const bool bf = dt == GPT_DTYPE_BF16;
+    GPT_TRY(cuda_status(cudaMemsetAsync(status, 0, sizeof(int32_t), s)));
+    GPT_TRY(launch_embed(W.wte(), W.wpe(), idx, reinterpret_cast<float*>(ab + A.x_in), B, T, C, V, dt, status, s));
+    for (int l = 0; l < cfg->n_layer; ++l) {
+        uint8_t* L = ab + A.layer * l;
+        float* x_in = reinterpret_cast<float*>(L + A.x_in);
+        float* x_mid = reinterpret_cast<float*>(L + A.x_mid);
+        float* x_out = l + 1 < cfg->n_layer ? reinterpret_cast<float*>(ab + A.layer * (l + 1) + A.x_in)
+                                            : reinterpret_cast<float*>(ab + A.x_f);
+        void* u1 = L + A.u1;
+        void* qkv = L + A.qkv;
+        void* y = L + A.y;
+        float* lse = reinterpret_cast<float*>(L + A.lse);
+        void* u2 = L + A.u2;
+        void* pre = L + A.pre;
+        void* hh = L + A.h;
+        GPT_TRY(launch_layernorm(x_in, W.layer(l, W_LN1_W), W.bias(l, W_LN1_B), u1, N, C, dt, s));
+        if (bf) {
+            GPT_TRY(launch_gemm_bf16(static_cast<const bf16*>(u1), C, static_cast<const bf16*>(W.layer(l, W_ATTN_W)), C,
+                                     static_cast<const bf16*>(W.bias(l, W_ATTN_B)), qkv, 3LL * C, N, 3 * C, C,
+                                     GPT_EPI_STORE, cfg->gelu, nullptr, status, s));
+            const bf16* qb = static_cast<const bf16*>(qkv);
+            AttnLayout AL{qb, qb + C, qb + 2 * C, 3LL * C * T, hs, 3LL * C, static_cast<bf16*>(y),
+                          static_cast<long long>(C) * T, hs, C, lse};
+            GPT_TRY(launch_attention_bf16(AL, B, nh, T, status, s));
+        } else {
+            GPT_TRY(launch_linear_f32(static_cast<const float*>(u1), C, static_cast<const float*>(W.layer(l, W_ATTN_W)),
+                                      static_cast<const float*>(W.bias(l, W_ATTN_B)), static_cast<float*>(qkv), 3LL * C,
+                                      N, 3 * C, C, GPT_EPI_STORE, cfg->gelu, s));
+            const float* qf = static_cast<const float*>(qkv);
+            AttnLayoutF32 AL{qf, qf + C, qf + 2 * C, 3LL * C * T, hs, 3LL * C, static_cast<float*>(y),
+                             static_cast<long long>(C) * T, hs, C, lse};
+            GPT_TRY(launch_attention_f32(AL, B, nh, T, hs, s));
+        }
+        GPT_TRY(cuda_status(cudaMemcpyAsync(x_mid, x_in, static_cast<size_t>(N) * C * 4, cudaMemcpyDeviceToDevice, s)));
+        if (bf)
+            GPT_TRY(launch_gemm_bf16(static_cast<const bf16*>(y), C, static_cast<const bf16*>(W.layer(l, W_PROJ_W)), C,
+                                     static_cast<const bf16*>(W.bias(l, W_PROJ_B)), x_mid, C, N, C, C, GPT_EPI_RESID,
+                                     cfg->gelu, nullptr, status, s));
+        else
+            GPT_TRY(launch_linear_f32(static_cast<const float*>(y), C, static_cast<const float*>(W.layer(l, W_PROJ_W)),
+                                      static_cast<const float*>(W.bias(l, W_PROJ_B)), x_mid, C, N, C, C, GPT_EPI_RESID,
+                                      cfg->gelu, s));
+        GPT_TRY(launch_layernorm(x_mid, W.layer(l, W_LN2_W), W.bias(l, W_LN2_B), u2, N, C, dt, s));
+        if (bf)
+            GPT_TRY(launch_gemm_bf16(static_cast<const bf16*>(u2), C, static_cast<const bf16*>(W.layer(l, W_FC_W)), C,
+                                     static_cast<const bf16*>(W.bias(l, W_FC_B)), pre, 4LL * C, N, 4 * C, C,
+                                     GPT_EPI_STORE, cfg->gelu, nullptr, status, s));
+        else
+            GPT_TRY(launch_linear_f32(static_cast<const float*>(u2), C, static_cast<const float*>(W.layer(l, W_FC_W)),
+                                      static_cast<const float*>(W.bias(l, W_FC_B)), static_cast<float*>(pre), 4LL * C, N,
+                                      4 * C, C, GPT_EPI_STORE, cfg->gelu, s));
+        GPT_TRY(launch_gelu_forward(pre, hh, static_cast<long long>(N) * 4 * C, dt, cfg->gelu == GPT_GELU_TANH, s));
+        GPT_TRY(cuda_status(cudaMemcpyAsync(x_out, x_mid, static_cast<size_t>(N) * C * 4, cudaMemcpyDeviceToDevice, s)));
+        if (bf)
+            GPT_TRY(launch_gemm_bf16(static_cast<const bf16*>(hh), 4LL * C, static_cast<const bf16*>(W.layer(l, W_FC2_W)),
+                                     4LL * C, static_cast<const bf16*>(W.bias(l, W_FC2_B)), x_out, C, N, C, 4 * C,
+                                     GPT_EPI_RESID, cfg->gelu, nullptr, status, s));
+        else
+            GPT_TRY(launch_linear_f32(static_cast<const float*>(hh), 4LL * C, static_cast<const float*>(W.layer(l, W_FC2_W)),
+                                      static_cast<const float*>(W.bias(l, W_FC2_B)), x_out, C, N, C, 4 * C, GPT_EPI_RESID,
+                                      cfg->gelu, s));
+    }
+    void* u_f = ab + A.u_f;
+    void* logits = ab + A.logits;
+    double* sc = reinterpret_cast<double*>(ab + A.sum_count);
+    GPT_TRY(launch_layernorm(reinterpret_cast<float*>(ab + A.x_f), W.lnf_w(), W.lnf_b(), u_f, N, C, dt, s));
+    float* rl = reinterpret_cast<float*>(ws + P.rowloss);
+    if (bf) {
+        CeArgs ce{targets, reinterpret_cast<float2*>(ws + P.part), reinterpret_cast<float*>(ws + P.tlogit), P.n_part};
+        GPT_TRY(launch_gemm_bf16(static_cast<const bf16*>(u_f), C, static_cast<const bf16*>(W.wte()), C, nullptr, logits, V,
+                                 N, V, C, 3 /* EPI_CE */, cfg->gelu, &ce, status, s));
+        GPT_TRY(launch_ce_rows_from_parts(ce.part, P.n_part, ce.tlogit, targets, N, V, rl, status, s));
+    } else {
+        GPT_TRY(launch_linear_f32(static_cast<const float*>(u_f), C, static_cast<const float*>(W.wte()), nullptr,
+                                  static_cast<float*>(logits), V, N, V, C, GPT_EPI_STORE, cfg->gelu, s));
+        GPT_TRY(launch_ce_rows_from_logits(static_cast<const float*>(logits), targets, N, V, rl, status, s));
+    }
+    GPT_TRY(launch_loss_finalize(rl, targets, N, V, loss, sc, s));
+    (void)es;
+    if (flags & GPT_FLAG_SYNC_CHECK) return sync_and_read_status(ws, s);
+    return GPT_OK;
+}
+
+GPT_API int gpt_backward(const gpt_config_t* cfg, const void* weights, const int64_t* idx, const int64_t* targets, int B,
+                         int T, const void* acts, size_t acts_bytes, float* grads, void* workspace,
+                         size_t workspace_bytes, void* stream, int flags) {
+    ActPlan A;
+    GPT_TRY(check_train(cfg, weights, idx, targets, B, T, acts, acts_bytes, &A));
+    if (!grads || !workspace) return GPT_ERR_NULL;
+    if (!aligned(grads, 16) || !aligned(workspace, 256)) return GPT_ERR_BAD_ALIGN;
+    const BwdPlan P = plan_bwd(cfg, B, T);
+    if (workspace_bytes < P.total) return GPT_ERR_WS_TOO_SMALL;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    Weights W;
+    fill_weights(W, cfg, weights);
+    const uint8_t* ab = static_cast<const uint8_t*>(acts);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    int32_t* status = status_word(ws);
+    const int C = cfg->n_embd, V = cfg->vocab_size, nh = cfg->n_head, hs = C / nh, N = B * T, dt = cfg->dtype;
+    const bool bf = dt == GPT_DTYPE_BF16;
+    const size_t es = elem_size(cfg);
+    // gradient slots: the packed layout in fp32 elements
+    size_t offs[kOptMaxTensors];
+    const int count = 2 + kTensorsPerLayer * cfg->n_layer + 2;
+    if (count > kOptMaxTensors) return GPT_ERR_UNSUPPORTED;
+    layout(cfg, offs, nullptr, count);
+    auto G = [&](int i) { return grads + offs[i] / es; };
+    auto GL = [&](int l, int which) { return G(2 + kTensorsPerLayer * l + which); };
+    void* dz = ws + P.dz;
+    void* dzT = ws + P.dzT;
+    void* wT = ws + P.wT;
+    void* gE = ws + P.gE;
+    void* gT = ws + P.gT;
+    void* aT = ws + P.aT;
+    float* d1 = reinterpret_cast<float*>(ws + P.d1);
+    float* dx = reinterpret_cast<float*>(ws + P.dx);
+    void* dpre = ws + P.dpre;
+    void* dqkv = ws + P.dqkv;
+    void* dy = ws + P.dy;
+    float* D = reinterpret_cast<float*>(ws + P.D);
+    float* parts = reinterpret_cast<float*>(ws + P.parts);
+    const int F32 = GPT_DTYPE_F32;
+    const size_t nc = static_cast<size_t>(N) * C;
+
+    GPT_TRY(cuda_status(cudaMemsetAsync(status, 0, sizeof(int32_t), s)));
+    // d loss / d logits, then the tied head: du_f = dz wte, dwte += dz^T u_f
+    GPT_TRY(launch_ce_backward(ab + A.logits, dt, targets, reinterpret_cast<const double*>(ab + A.sum_count), dz, N, V,
+                               status, s));
+    GPT_TRY(launch_transpose(W.wte(), dt, C, wT, dt, V, V, C, s));
+    GPT_TRY(cuda_status(cudaMemsetAsync(d1, 0, nc * 4, s)));
+    GPT_TRY(gemm_acc(cfg, dz, V, wT, V, d1, C, N, C, V, status, s));
+    GPT_TRY(launch_transpose(dz, dt, V, dzT, dt, N, N, V, s));
+    GPT_TRY(launch_transpose(ab + A.u_f, dt, C, aT, dt, N, N, C, s));
+    GPT_TRY(gemm_acc(cfg, dzT, N, aT, N, G(0), C, V, C, N, status, s));
+    GPT_TRY(launch_layernorm_backward(d1, reinterpret_cast<const float*>(ab + A.x_f), W.lnf_w(), dt, dx, 0, G(count - 2),
+                                      cfg->bias ? G(count - 1) : nullptr, 1, parts, N, C, s));
+    for (int l = cfg->n_layer - 1; l >= 0; --l) {
+        const uint8_t* L = ab + A.layer * l;
+        // mlp c_proj: dh = dx W_fc2 (into d1 [N, 4C]); dW_fc2 += dx^T h; db_fc2 += sum dx
+        GPT_TRY(launch_convert(dx, F32, gE, dt, static_cast<long long>(nc), s));
+        GPT_TRY(launch_transpose(W.layer(l, W_FC2_W), dt, 4LL * C, wT, dt, C, C, 4 * C, s));
+        GPT_TRY(cuda_status(cudaMemsetAsync(d1, 0, nc * 4 * 4, s)));
+        GPT_TRY(gemm_acc(cfg, gE, C, wT, C, d1, 4LL * C, N, 4 * C, C, status, s));
+        GPT_TRY(launch_transpose(dx, F32, C, gT, dt, N, N, C, s));
+        GPT_TRY(launch_transpose(L + A.h, dt, 4LL * C, aT, dt, N, N, 4 * C, s));
+        GPT_TRY(gemm_acc(cfg, gT, N, aT, N, GL(l, W_FC2_W), 4LL * C, C, 4 * C, N, status, s));
+        if (cfg->bias) GPT_TRY(launch_colsum(dx, F32, N, C, GL(l, W_FC2_B), 1, parts, s));
+        // GELU, then c_fc: du2 = dpre W_fc (into d1 [N, C]); dW_fc += dpre^T u2; db_fc += sum dpre
+        GPT_TRY(launch_gelu_backward(d1, L + A.pre, dt, dpre, static_cast<long long>(nc) * 4, cfg->gelu == GPT_GELU_TANH, s));
+        GPT_TRY(launch_transpose(W.layer(l, W_FC_W), dt, C, wT, dt, 4LL * C, 4 * C, C, s));
+        GPT_TRY(cuda_status(cudaMemsetAsync(d1, 0, nc * 4, s)));
+        GPT_TRY(gemm_acc(cfg, dpre, 4LL * C, wT, 4LL * C, d1, C, N, C, 4 * C, status, s));
+        GPT_TRY(launch_transpose(dpre, dt, 4LL * C, gT, dt, N, N, 4 * C, s));
+        GPT_TRY(launch_transpose(L + A.u2, dt, C, aT, dt, N, N, C, s));
+        GPT_TRY(gemm_acc(cfg, gT, N, aT, N, GL(l, W_FC_W), C, 4 * C, C, N, status, s));
+        if (cfg->bias) GPT_TRY(launch_colsum(dpre, dt, N, 4 * C, GL(l, W_FC_B), 1, parts, s));
+        GPT_TRY(launch_layernorm_backward(d1, reinterpret_cast<const float*>(L + A.x_mid), W.layer(l, W_LN2_W), dt, dx, 1,
+                                          GL(l, W_LN2_W), cfg->bias ? GL(l, W_LN2_B) : nullptr, 1, parts, N, C, s));
+        // attn c_proj: dy = dx W_proj; dW_proj += dx^T y; db_proj += sum dx
+        GPT_TRY(launch_convert(dx, F32, gE, dt, static_cast<long long>(nc), s));
+        GPT_TRY(launch_transpose(W.layer(l, W_PROJ_W), dt, C, wT, dt, C, C, C, s));
+        GPT_TRY(cuda_status(cudaMemsetAsync(d1, 0, nc * 4, s)));
+        GPT_TRY(gemm_acc(cfg, gE, C, wT, C, d1, C, N, C, C, status, s));
+        GPT_TRY(launch_convert(d1, F32, dy, dt, static_cast<long long>(nc), s));
+        GPT_TRY(launch_transpose(dx, F32, C, gT, dt, N, N, C, s));
+        GPT_TRY(launch_transpose(L + A.y, dt, C, aT, dt, N, N, C, s));
+        GPT_TRY(gemm_acc(cfg, gT, N, aT, N, GL(l, W_PROJ_W), C, C, C, N, status, s));
+        if (cfg->bias) GPT_TRY(launch_colsum(dx, F32, N, C, GL(l, W_PROJ_B), 1, parts, s));
+        // attention backward into dqkv (the qkv layout)
+        const float* lse = reinterpret_cast<const float*>(L + A.lse);
+        const long long qsb = 3LL * C * T, ysb = static_cast<long long>(C) * T;
+        if (bf) {
+            const bf16* q = reinterpret_cast<const bf16*>(L + A.qkv);
+            bf16* dq = static_cast<bf16*>(dqkv);
+            AttnBwdLayout<bf16> AL{q, q + C, q + 2 * C, qsb, hs, 3LL * C,
+                                   reinterpret_cast<const bf16*>(L + A.y), static_cast<const bf16*>(dy), ysb, hs, C,
+                                   dq, dq + C, dq + 2 * C, lse};
+            GPT_TRY(launch_attention_backward(&AL, nullptr, B, nh, T, hs, D, s));
+        } else {
+            const float* q = reinterpret_cast<const float*>(L + A.qkv);
+            float* dq = static_cast<float*>(dqkv);
+            AttnBwdLayout<float> AL{q, q + C, q + 2 * C, qsb, hs, 3LL * C,
+                                    reinterpret_cast<const float*>(L + A.y), static_cast<const float*>(dy), ysb, hs, C,
+                                    dq, dq + C, dq + 2 * C, lse};
+            GPT_TRY(launch_attention_backward(nullptr, &AL, B, nh, T, hs, D, s));
+        }
+        // c_attn: du1 = dqkv W_attn (into d1 [N, C]); dW_attn += dqkv^T u1; db_attn += sum dqkv
+        GPT_TRY(launch_transpose(W.layer(l, W_ATTN_W), dt, C, wT, dt, 3LL * C, 3 * C, C, s));
+        GPT_TRY(cuda_status(cudaMemsetAsync(d1, 0, nc * 4, s)));
+        GPT_TRY(gemm_acc(cfg, dqkv, 3LL * C, wT, 3LL * C, d1, C, N, C, 3 * C, status, s));
+        GPT_TRY(launch_transpose(dqkv, dt, 3LL * C, gT, dt, N, N, 3 * C, s));
+        GPT_TRY(launch_transpose(L + A.u1, dt, C, aT, dt, N, N, C, s));
+        GPT_TRY(gemm_acc(cfg, gT, N, aT, N, GL(l, W_ATTN_W), C, 3 * C, C, N, status, s));
+        if (cfg->bias) GPT_TRY(launch_colsum(dqkv, dt, N, 3 * C, GL(l, W_ATTN_B), 1, parts, s));
+        GPT_TRY(launch_layernorm_backward(d1, reinterpret_cast<const float*>(L + A.x_in), W.layer(l, W_LN1_W), dt, dx, 1,
+                                          GL(l, W_LN1_W), cfg->bias ? GL(l, W_LN1_B) : nullptr, 1, parts, N, C, s));
+    }
+    GPT_TRY(launch_embed_backward(idx, dx, B, T, C, V, G(0), G(1), reinterpret_cast<unsigned long long*>(ws + P.sort),
+                                  status, s));
+    if (flags & GPT_FLAG_SYNC_CHECK) return sync_and_read_status(ws, s);
+    return GPT_OK;
 }
 

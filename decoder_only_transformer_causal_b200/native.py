@@ -108,6 +108,10 @@ def _load() -> ctypes.CDLL:
         "gpt_attention_backward_workspace_bytes": (Z, [I, I, I]),
         "gpt_attention_backward": (I, [P, P, P, P, P, P, P, P, P, I, I, I, I, D, P, Z, P]),
         "gpt_transpose": (I, [P, D, L, P, D, L, I, I, P]),
+        "gpt_train_activation_bytes": (Z, [CFG, I, I]),
+        "gpt_backward_workspace_bytes": (Z, [CFG, I, I]),
+        "gpt_forward_train": (I, [CFG, P, P, P, I, I, P, Z, P, P, Z, P, I]),
+        "gpt_backward": (I, [CFG, P, P, P, I, I, P, Z, P, P, Z, P, I]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -127,7 +131,8 @@ EXPORTED = ("gpt_status_string", "gpt_abi_version", "gpt_last_cuda_error", "gpt_
             "gpt_adamw_workspace_bytes", "gpt_adamw_step", "gpt_cross_entropy_backward",
             "gpt_layernorm_backward_workspace_bytes", "gpt_layernorm_backward", "gpt_bias_grad_workspace_bytes",
             "gpt_bias_grad", "gpt_gelu_backward", "gpt_embedding_backward_workspace_bytes", "gpt_embedding_backward",
-            "gpt_attention_train", "gpt_attention_backward_workspace_bytes", "gpt_attention_backward", "gpt_transpose")
+            "gpt_attention_train", "gpt_attention_backward_workspace_bytes", "gpt_attention_backward", "gpt_transpose",
+            "gpt_train_activation_bytes", "gpt_backward_workspace_bytes", "gpt_forward_train", "gpt_backward")
 
 
 def status_string(status: int) -> str:
@@ -582,4 +587,34 @@ def transpose(x: torch.Tensor, out_dtype=None, stream=None) -> torch.Tensor:
     out = torch.empty((Cc, R), dtype=out_dtype or x.dtype, device=x.device)
     _check(LIB.gpt_transpose(_ptr(x), _dt(x), Cc, _ptr(out), _dt(out), R, R, Cc, _stream(stream)), "gpt_transpose")
     return out
+
+
+# ---------------------------------------------------------------- training step
+def train_buffers(cfg: GPTConfig, B: int, T: int, device="cuda"):
+    """(acts, forward workspace, backward workspace) for gpt_forward_train / gpt_backward."""
+    c = ctypes.byref(cfg.c())
+    na, nb = LIB.gpt_train_activation_bytes(c, B, T), LIB.gpt_backward_workspace_bytes(c, B, T)
+    if na == 0 or nb == 0:
+        raise GPTError(GPT_ERR_BAD_SHAPE, "gpt_train_activation_bytes")
+    return (alloc_workspace(na, device), alloc_workspace(workspace_bytes(cfg, B, T), device),
+            alloc_workspace(nb, device))
+
+
+def forward_train(cfg, weights, idx, targets, acts, workspace, loss=None, stream=None, sync_check=False):
+    B, T = idx.shape
+    if loss is None:
+        loss = torch.empty((), dtype=torch.float32, device=idx.device)
+    _check(LIB.gpt_forward_train(ctypes.byref(cfg.c()), _ptr(weights), _ptr(idx), _ptr(targets), B, T, _ptr(acts),
+                                 acts.numel(), _ptr(loss), _ptr(workspace), workspace.numel(), _stream(stream),
+                                 GPT_FLAG_SYNC_CHECK if sync_check else 0), "gpt_forward_train")
+    return loss
+
+
+def backward(cfg, weights, idx, targets, acts, grads, workspace, stream=None, sync_check=False):
+    """gpt_backward: adds the gradients into grads (fp32 [param_elems])."""
+    B, T = idx.shape
+    _check(LIB.gpt_backward(ctypes.byref(cfg.c()), _ptr(weights), _ptr(idx), _ptr(targets), B, T, _ptr(acts),
+                            acts.numel(), _ptr(grads), _ptr(workspace), workspace.numel(), _stream(stream),
+                            GPT_FLAG_SYNC_CHECK if sync_check else 0), "gpt_backward")
+    return grads
 

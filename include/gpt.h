@@ -387,6 +387,28 @@ int gpt_attention_backward(const void* q, const void* k, const void* v, const vo
 int gpt_transpose(const void* in, int in_dtype, long long ld_in, void* out, int out_dtype,
                   long long ld_out, int rows, int cols, void* stream);
 
+/* ---- the training step ----------------------------------------------------------------
+ * "nanoGPT 全局流程图" 3.2-3.4: forward with targets, then loss.backward().  gpt_forward_train runs
+ * gpt_forward's computation and keeps what the backward needs in `acts`
+ * (gpt_train_activation_bytes(cfg, B, T) bytes, 256-byte aligned; per layer the residual input,
+ * both LayerNorm outputs, q/k/v, the attention output and its per-row log-sum-exp, the c_fc
+ * pre-activation and the GELU output; then the final residual, ln_f's output, the logits and the
+ * {sum of row losses, counted rows} pair).  loss: device fp32 scalar.  workspace: as gpt_forward.
+ * gpt_backward adds d(loss)/d(parameter) to grads (fp32, the flat element layout of
+ * gpt_param_elems; zero it before the first micro-batch), reading acts; the tied head's and the
+ * embedding's contributions to wte are both added.  workspace: gpt_backward_workspace_bytes.
+ * Head size 32 or 64; for bf16, B * T % 8 == 0; B * T <= 16384.  Linear layers' backward products
+ * run on the tensor-core GEMM (bf16) after explicit transposes; the attention backward is the
+ * SIMT kernel of gpt_attention_backward. */
+size_t gpt_train_activation_bytes(const gpt_config_t* cfg, int B, int T);
+size_t gpt_backward_workspace_bytes(const gpt_config_t* cfg, int B, int T);
+int gpt_forward_train(const gpt_config_t* cfg, const void* weights, const int64_t* idx,
+                      const int64_t* targets, int B, int T, void* acts, size_t acts_bytes, float* loss,
+                      void* workspace, size_t workspace_bytes, void* stream, int flags);
+int gpt_backward(const gpt_config_t* cfg, const void* weights, const int64_t* idx, const int64_t* targets,
+                 int B, int T, const void* acts, size_t acts_bytes, float* grads, void* workspace,
+                 size_t workspace_bytes, void* stream, int flags);
+
 #ifdef __cplusplus
 }
 #endif
