@@ -470,6 +470,58 @@ def backward_pieces_bench(native, dev, stream, peaks, peak_src, reps: int = 10):
     return out
 
 
+def train_bench(native, dev, stream, world, rank, dist, steps: int = 5, warmup: int = 2):
+    """One training step of GPT-2 124M per rank ("nanoGPT 全局流程图" 3.2-3.6), B 12, T 1024 per GPU
+    (weak scaling): training forward keeping activations, backward, AdamW (clip 1.0, decay on
+    matrices, get_lr); with N > 1 the loss terms and the gradients are all-reduced (NCCL) between
+    the backward's start and the optimizer.  Synthetic seeded data, GPT-2-init weights.  Time per
+    phase from CUDA events on one extra step."""
+    from decoder_only_transformer_causal_b200 import GPT, GPTConfig, Trainer
+    from decoder_only_transformer_causal_b200.data_parallel import train_step_sharded
+    w = seeded.WORKLOADS[WORKLOAD]
+    W = seeded.make_weights(w.model_dict(), seed=seeded.BASE_SEED + 31, device=str(dev))
+    model = GPT(GPTConfig.from_dict(w.model_dict()), W, dev)
+    tr = Trainer(model, W, w.batch, w.seq_len)
+    idx, tgt = seeded.make_tokens(w.batch, w.seq_len, w.token_high, seed=seeded.BASE_SEED + 700 + rank)
+    idx, tgt = idx.to(dev), tgt.to(dev)
+    step = (lambda: train_step_sharded(tr, idx, tgt)) if world > 1 else (lambda: tr.step(idx, tgt))
+    for _ in range(warmup):
+        step()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t = torch.tensor([e0.elapsed_time(e1) / steps], device=dev)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = float(t)
+    # phase split of one more (single-GPU) step
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    cfg = model.cfg
+    ev[0].record(stream)
+    native.forward_train(cfg, model.weights, idx, tgt, tr.acts, tr.fws, loss=tr.loss)
+    ev[1].record(stream)
+    tr.grads.zero_()
+    native.backward(cfg, model.weights, idx, tgt, tr.acts, tr.grads, tr.bws)
+    ev[2].record(stream)
+    tr.opt.step(tr.grads)
+    ev[3].record(stream)
+    torch.cuda.synchronize()
+    loss = float(tr.loss)
+    del tr, model
+    return {"workload": f"GPT-2 124M training step, B {w.batch} x T {w.seq_len} per GPU, bf16 weights/activations, "
+                        "fp32 master weights and Adam moments" + (f", data-parallel over {world} GPUs" if world > 1 else ""),
+            "tokens_per_s": world * w.batch * w.seq_len / (ms / 1000.0), "ms_per_step": ms,
+            "phase_ms": {"forward_train": ev[0].elapsed_time(ev[1]), "backward": ev[1].elapsed_time(ev[2]),
+                         "adamw": ev[2].elapsed_time(ev[3])},
+            "loss_after": loss}
+
+
 def adamw_only(args):
     from decoder_only_transformer_causal_b200 import GPT, GPTConfig, native
     dev = torch.device("cuda", 0)
@@ -643,6 +695,10 @@ def main():
         line["decode"] = decode_bench(model, native, dev, stream, peaks, peak_src)
         line["adamw"] = adamw_bench(model, native, dev, stream, peaks, peak_src)
         line["backward_pieces"] = backward_pieces_bench(native, dev, stream, peaks, peak_src)
+    if not args.no_kernels:
+        tr = train_bench(native, dev, stream, world, rank, dist)
+        if rank == 0:
+            line["train"] = tr
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         times, threads = oracle_sample(w, 256, budget_s=12.0)
         tok_s = 256 * len(times) / sum(times)

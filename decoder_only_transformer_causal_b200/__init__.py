@@ -135,3 +135,19 @@ class Trainer:
         self.opt.step(self.grads)
         return self.loss
 
+    def step_accumulated(self, micro_batches) -> list:
+        """Gradient accumulation ("nanoGPT 全局流程图" 3.7): the gradients of K micro-batches
+        [(idx, targets), ...] each scaled by 1/K (the page's loss / gradient_accumulation_steps),
+        summed, then one optimizer step.  Returns the micro-batches' losses (device scalars)."""
+        cfg, w = self.model.cfg, self.model.weights
+        K = len(micro_batches)
+        self.grads.zero_()
+        losses = []
+        for idx, targets in micro_batches:
+            loss = torch.empty((), dtype=torch.float32, device=self.model.device)
+            native.forward_train(cfg, w, idx, targets, self.acts, self.fws, loss=loss)
+            native.backward(cfg, w, idx, targets, self.acts, self.grads, self.bws, loss_scale=1.0 / K)
+            losses.append(loss)
+        self.opt.step(self.grads)
+        return losses
+

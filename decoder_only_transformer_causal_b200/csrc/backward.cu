@@ -57,14 +57,14 @@ GPT_DEVINL float wsum(float v) {
     return v;
 }
 
-// dlogits[r, v] = (exp(z_rv - lse_r) - [v == t_r]) / n for rows whose target is not -1, and 0
-// for the rest; n = the number of counted rows, read from sum_count[1] (the forward's {sum of row
-// losses, counted rows}).  One warp per row: an online (max, sum) pass over the row, then the
+// dlogits[r, v] = scale (exp(z_rv - lse_r) - [v == t_r]) / n for rows whose target is not -1,
+// and 0 for the rest; n = the number of counted rows, read from sum_count[1] (the forward's {sum
+// of row losses, counted rows}, or its sum over data-parallel ranks).  One warp per row: an online (max, sum) pass over the row, then the
 // write pass.
 template <typename E>
 __global__ void __launch_bounds__(kBwdWarps * 32)
     ce_backward_kernel(const E* __restrict__ z, const int64_t* __restrict__ targets, const double* __restrict__ sum_count,
-                       E* __restrict__ dz, int rows, int V, int32_t* status) {
+                       E* __restrict__ dz, int rows, int V, float scale, int32_t* status) {
     griddep_launch_dependents();
     griddep_wait();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -119,7 +119,7 @@ __global__ void __launch_bounds__(kBwdWarps * 32)
         m = mm;
     }
     const float lse = m + __logf(s);
-    const float inv_n = static_cast<float>(1.0 / n);
+    const float inv_n = static_cast<float>(static_cast<double>(scale) / n);
     if (vec) {
         for (int v = lane * VW; v < V; v += 32 * VW) {
             float f[VW];
@@ -415,13 +415,13 @@ __global__ void embed_wpe_kernel(const float* __restrict__ dx, int B, int T, int
 }  // namespace
 
 int launch_ce_backward(const void* logits, int dtype, const int64_t* targets, const double* sum_count, void* dlogits,
-                       int rows, int V, int32_t* status, cudaStream_t s) {
+                       int rows, int V, int32_t* status, cudaStream_t s, float scale) {
     const dim3 grid((rows + kBwdWarps - 1) / kBwdWarps), block(kBwdWarps * 32);
     if (dtype == GPT_DTYPE_BF16)
         return launch_overlapped(ce_backward_kernel<bf16>, grid, block, 0, s, static_cast<const bf16*>(logits),
-                                 targets, sum_count, static_cast<bf16*>(dlogits), rows, V, status);
+                                 targets, sum_count, static_cast<bf16*>(dlogits), rows, V, scale, status);
     return launch_overlapped(ce_backward_kernel<float>, grid, block, 0, s, static_cast<const float*>(logits), targets,
-                             sum_count, static_cast<float*>(dlogits), rows, V, status);
+                             sum_count, static_cast<float*>(dlogits), rows, V, scale, status);
 }
 
 int layernorm_backward_parts(int rows, int C) {

@@ -1177,8 +1177,13 @@ GPT_API int gpt_forward_train(const gpt_config_t* cfg, const void* weights, cons
     return GPT_OK;
 }
 
+GPT_API size_t gpt_train_loss_terms_offset(const gpt_config_t* cfg, int B, int T) {
+    if (validate(cfg) != GPT_OK || B < 1 || T < 1 || T > cfg->block_size) return 0;
+    return plan_acts(cfg, B, T).sum_count;
+}
+
 GPT_API int gpt_backward(const gpt_config_t* cfg, const void* weights, const int64_t* idx, const int64_t* targets, int B,
-                         int T, const void* acts, size_t acts_bytes, float* grads, void* workspace,
+                         int T, const void* acts, size_t acts_bytes, float* grads, float loss_scale, void* workspace,
                          size_t workspace_bytes, void* stream, int flags) {
     ActPlan A;
     GPT_TRY(check_train(cfg, weights, idx, targets, B, T, acts, acts_bytes, &A));
@@ -1220,8 +1225,9 @@ GPT_API int gpt_backward(const gpt_config_t* cfg, const void* weights, const int
 
     GPT_TRY(cuda_status(cudaMemsetAsync(status, 0, sizeof(int32_t), s)));
     // d loss / d logits, then the tied head: du_f = dz wte, dwte += dz^T u_f
+    if (!(loss_scale > 0.f) || !isfinite(loss_scale)) return GPT_ERR_BAD_SHAPE;
     GPT_TRY(launch_ce_backward(ab + A.logits, dt, targets, reinterpret_cast<const double*>(ab + A.sum_count), dz, N, V,
-                               status, s));
+                               status, s, loss_scale));
     GPT_TRY(launch_transpose(W.wte(), dt, C, wT, dt, V, V, C, s));
     GPT_TRY(cuda_status(cudaMemsetAsync(d1, 0, nc * 4, s)));
     GPT_TRY(gemm_acc(cfg, dz, V, wT, V, d1, C, N, C, V, status, s));

@@ -144,7 +144,7 @@ int launch_adamw(const OptTable& tab, int dtype, float* params, const float* gra
 
 // ---- backward kernels of the non-matmul pieces (backward.cu)
 int launch_ce_backward(const void* logits, int dtype, const int64_t* targets, const double* sum_count, void* dlogits,
-                       int rows, int V, int32_t* status, cudaStream_t s);
+                       int rows, int V, int32_t* status, cudaStream_t s, float scale = 1.f);
 int layernorm_backward_parts(int rows, int C);  // part: [parts, 2C] floats
 int launch_layernorm_backward(const float* dy, const float* x, const void* w, int dtype, float* dx, int accumulate,
                               float* dw, float* db, int accumulate_wb, float* part, int rows, int C, cudaStream_t s);

@@ -7,6 +7,12 @@ only exchange is the loss: F.cross_entropy averages over every counted position 
 (targets != -1), so the ranks add their {sum of row losses, number of counted rows} and divide
 the totals — not the mean of per-rank means, which would weight ranks with many ignored targets
 wrongly.  With NCCL over NVLink that is one 16-byte all-reduce per step.
+
+Data-parallel training ("nanoGPT 全局流程图" 3.4-3.7; "nanoGPT 核心代码速查表" 七 per-GPU batch):
+each rank runs the training forward on its shard, the {sum, count} pair is all-reduced *before*
+the backward so every rank's cross-entropy gradient divides by the global count, and a SUM
+all-reduce of the flat fp32 gradients then gives exactly the whole batch's gradient (also when
+ignored targets are spread unevenly); every rank applies the same AdamW step.
 """
 from __future__ import annotations
 
@@ -54,3 +60,30 @@ def forward_sharded(model, idx: torch.Tensor, targets: torch.Tensor, group=None)
         logits, _ = model(idx[a:b].to(dev), targets[a:b].to(dev), loss_sum_count=sc)
     allreduce_loss_terms(sc, group)
     return logits, global_loss(sc)
+
+
+def allreduce_grads(grads: torch.Tensor, group=None) -> torch.Tensor:
+    """SUM all-reduce of the flat fp32 gradient array, in place (each rank holds its share of the
+    global mean after a backward against the all-reduced count)."""
+    if grads.dtype != torch.float32:
+        raise ValueError("grads must be float32")
+    dist.all_reduce(grads, op=dist.ReduceOp.SUM, group=group)
+    return grads
+
+
+def train_step_sharded(trainer, idx: torch.Tensor, targets: torch.Tensor, group=None) -> float:
+    """One data-parallel training step of a Trainer on this rank's shard [B_r, T] (already on the
+    rank's device): training forward, all-reduce of the loss terms, backward against the global
+    count, SUM all-reduce of the gradients, AdamW.  Returns the global mean loss (host float)."""
+    from . import native
+    cfg, w = trainer.model.cfg, trainer.model.weights
+    B, T = idx.shape
+    native.forward_train(cfg, w, idx, targets, trainer.acts, trainer.fws, loss=trainer.loss)
+    lt = native.loss_terms(cfg, trainer.acts, B, T)
+    allreduce_loss_terms(lt, group)
+    trainer.grads.zero_()
+    native.backward(cfg, w, idx, targets, trainer.acts, trainer.grads, trainer.bws)
+    allreduce_grads(trainer.grads, group)
+    trainer.opt.step(trainer.grads)
+    return global_loss(lt)
+

@@ -111,7 +111,8 @@ def _load() -> ctypes.CDLL:
         "gpt_train_activation_bytes": (Z, [CFG, I, I]),
         "gpt_backward_workspace_bytes": (Z, [CFG, I, I]),
         "gpt_forward_train": (I, [CFG, P, P, P, I, I, P, Z, P, P, Z, P, I]),
-        "gpt_backward": (I, [CFG, P, P, P, I, I, P, Z, P, P, Z, P, I]),
+        "gpt_backward": (I, [CFG, P, P, P, I, I, P, Z, P, F, P, Z, P, I]),
+        "gpt_train_loss_terms_offset": (Z, [CFG, I, I]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -132,7 +133,8 @@ EXPORTED = ("gpt_status_string", "gpt_abi_version", "gpt_last_cuda_error", "gpt_
             "gpt_layernorm_backward_workspace_bytes", "gpt_layernorm_backward", "gpt_bias_grad_workspace_bytes",
             "gpt_bias_grad", "gpt_gelu_backward", "gpt_embedding_backward_workspace_bytes", "gpt_embedding_backward",
             "gpt_attention_train", "gpt_attention_backward_workspace_bytes", "gpt_attention_backward", "gpt_transpose",
-            "gpt_train_activation_bytes", "gpt_backward_workspace_bytes", "gpt_forward_train", "gpt_backward")
+            "gpt_train_activation_bytes", "gpt_backward_workspace_bytes", "gpt_forward_train", "gpt_backward",
+            "gpt_train_loss_terms_offset")
 
 
 def status_string(status: int) -> str:
@@ -610,11 +612,18 @@ def forward_train(cfg, weights, idx, targets, acts, workspace, loss=None, stream
     return loss
 
 
-def backward(cfg, weights, idx, targets, acts, grads, workspace, stream=None, sync_check=False):
-    """gpt_backward: adds the gradients into grads (fp32 [param_elems])."""
+def backward(cfg, weights, idx, targets, acts, grads, workspace, loss_scale=1.0, stream=None, sync_check=False):
+    """gpt_backward: adds loss_scale * the gradients into grads (fp32 [param_elems])."""
     B, T = idx.shape
     _check(LIB.gpt_backward(ctypes.byref(cfg.c()), _ptr(weights), _ptr(idx), _ptr(targets), B, T, _ptr(acts),
-                            acts.numel(), _ptr(grads), _ptr(workspace), workspace.numel(), _stream(stream),
-                            GPT_FLAG_SYNC_CHECK if sync_check else 0), "gpt_backward")
+                            acts.numel(), _ptr(grads), float(loss_scale), _ptr(workspace), workspace.numel(),
+                            _stream(stream), GPT_FLAG_SYNC_CHECK if sync_check else 0), "gpt_backward")
     return grads
+
+
+def loss_terms(cfg, acts: torch.Tensor, B: int, T: int) -> torch.Tensor:
+    """The fp64 {sum of row losses, counted rows} pair inside acts (a view: all-reduce it in place
+    before gpt_backward for a data-parallel step)."""
+    off = LIB.gpt_train_loss_terms_offset(ctypes.byref(cfg.c()), B, T)
+    return acts[off: off + 16].view(torch.float64)
 

@@ -394,9 +394,14 @@ int gpt_transpose(const void* in, int in_dtype, long long ld_in, void* out, int 
  * both LayerNorm outputs, q/k/v, the attention output and its per-row log-sum-exp, the c_fc
  * pre-activation and the GELU output; then the final residual, ln_f's output, the logits and the
  * {sum of row losses, counted rows} pair).  loss: device fp32 scalar.  workspace: as gpt_forward.
- * gpt_backward adds d(loss)/d(parameter) to grads (fp32, the flat element layout of
+ * gpt_backward adds loss_scale * d(loss)/d(parameter) to grads (fp32, the flat element layout of
  * gpt_param_elems; zero it before the first micro-batch), reading acts; the tied head's and the
- * embedding's contributions to wte are both added.  workspace: gpt_backward_workspace_bytes.
+ * embedding's contributions to wte are both added.  The mean is over the counted rows in acts'
+ * {sum, count} pair (at byte offset gpt_train_loss_terms_offset): a data-parallel caller sums the
+ * pair over its ranks before the backward, so each rank's gradient is its share of the global
+ * mean and a SUM all-reduce of grads gives the whole batch's gradient.  loss_scale: 1, or 1/K for
+ * K accumulated micro-batches (the page's loss / gradient_accumulation_steps); must be > 0.
+ * workspace: gpt_backward_workspace_bytes.
  * Head size 32 or 64; for bf16, B * T % 8 == 0; B * T <= 16384.  Linear layers' backward products
  * run on the tensor-core GEMM (bf16) after explicit transposes; the attention backward is the
  * SIMT kernel of gpt_attention_backward. */
@@ -405,9 +410,10 @@ size_t gpt_backward_workspace_bytes(const gpt_config_t* cfg, int B, int T);
 int gpt_forward_train(const gpt_config_t* cfg, const void* weights, const int64_t* idx,
                       const int64_t* targets, int B, int T, void* acts, size_t acts_bytes, float* loss,
                       void* workspace, size_t workspace_bytes, void* stream, int flags);
+size_t gpt_train_loss_terms_offset(const gpt_config_t* cfg, int B, int T);
 int gpt_backward(const gpt_config_t* cfg, const void* weights, const int64_t* idx, const int64_t* targets,
-                 int B, int T, const void* acts, size_t acts_bytes, float* grads, void* workspace,
-                 size_t workspace_bytes, void* stream, int flags);
+                 int B, int T, const void* acts, size_t acts_bytes, float* grads, float loss_scale,
+                 void* workspace, size_t workspace_bytes, void* stream, int flags);
 
 #ifdef __cplusplus
 }

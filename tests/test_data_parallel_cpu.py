@@ -75,3 +75,48 @@ def test_sharded_loss_matches_full_batch(tmp_path, world, batch):
         assert math.isnan(got)
     else:
         assert abs(got - want) <= 1e-12 * abs(want)
+
+
+def _grad_rank_main(rank, world, port, batch, out_path):
+    """Data-parallel gradient combination on gloo ranks: each rank's oracle gradient of its shard,
+    taken against the all-reduced global count (its own mean scaled by n_r / n_total, which is
+    what dividing by the global count gives), SUM-all-reduced with the product's helpers, must equal
+    the oracle gradient of the whole batch."""
+    import oracle.backward as ob
+    from decoder_only_transformer_causal_b200.data_parallel import allreduce_grads
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        cfg = dict(TINY, n_layer=1)
+        W = seeded.to_f64(seeded.make_weights(cfg, stress=True))
+        idx, tgt = seeded.make_tokens(batch, 16, cfg["vocab_size"], ignore_frac=0.3)
+        tgt[0, :12] = -1                                    # rank 0's shard has fewer counted rows
+        a, b = shard_range(batch, world, rank)
+        sc = torch.zeros(2, dtype=torch.float64)
+        names = sorted(W)
+        flat = torch.zeros(sum(W[n].size for n in names), dtype=torch.float32)
+        if b > a:
+            g, _ = ob.backward(W, cfg, idx[a:b].numpy(), tgt[a:b].numpy())
+            n_r = float((tgt[a:b] != -1).sum())
+            sc[1] = n_r
+            allreduce_loss_terms(sc)
+            scale = n_r / float(sc[1])
+            flat = torch.from_numpy(np.concatenate([(g[n] * scale).ravel() for n in names]).astype(np.float32))
+        else:
+            allreduce_loss_terms(sc)
+        allreduce_grads(flat)
+        if rank == 0:
+            g_full, _ = ob.backward(W, cfg, idx.numpy(), tgt.numpy())
+            ref = np.concatenate([g_full[n].ravel() for n in names])
+            np.save(out_path, np.array([np.abs(flat.numpy() - ref).max(), np.abs(ref).max()]))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,batch", [(2, 3), (3, 5)])
+def test_sharded_gradients_match_full_batch(tmp_path, world, batch):
+    out = tmp_path / "g.npy"
+    mp.spawn(_grad_rank_main, args=(world, _free_port(), batch, str(out)), nprocs=world, join=True)
+    err, scale = np.load(out)
+    assert err <= 1e-6 * scale                     # fp32 transport of fp64 gradients
