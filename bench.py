@@ -49,6 +49,8 @@ def parse():
                     help="run only the decode measurement (--steps graph replays after --warmup) and print it; "
                          "with --no-e2e the generate call is skipped (for profiler captures)")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--train-only", action="store_true",
+                    help="run only the training-step measurement (--steps timed after --warmup) and print it")
     ap.add_argument("--adamw-only", action="store_true",
                     help="run only the optimizer-step measurement (--steps timed after --warmup) and print it")
     ap.add_argument("--profile-kernel", default=None,
@@ -556,6 +558,12 @@ def main():
         return decode_only(args)
     if args.adamw_only:
         return adamw_only(args)
+    if args.train_only:
+        dev = torch.device("cuda", 0)
+        from decoder_only_transformer_causal_b200 import native
+        print(json.dumps({"train": train_bench(native, dev, torch.cuda.current_stream(dev), 1, 0, None,
+                                               steps=args.steps, warmup=max(1, args.warmup))}), flush=True)
+        return 0
     assert args.warmup >= 3, "at least 3 warm-up steps"
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -86,3 +86,29 @@ def test_training_steps_lower_the_loss():
     # the model's packed weights now give the trained loss in the plain forward
     logits, loss = model(idx.cuda(), tgt.cuda())
     assert float(loss) < losses[0]
+
+
+def test_accumulated_micro_batches_equal_the_full_batch():
+    """The page's accumulation (loss / K per micro-batch, gradients summed) equals the full batch's
+    mean gradient when the micro-batches count the same number of rows (no ignored targets)."""
+    from decoder_only_transformer_causal_b200 import GPT, native
+    from decoder_only_transformer_causal_b200.native import GPTConfig
+    cfgd = dict(seeded.WORKLOADS["tiny"].model_dict(), n_layer=2)
+    W = seeded.make_weights(cfgd, stress=True)
+    cfg = GPTConfig.from_dict(cfgd)
+    m = GPT(cfg, W)
+    idx, tgt = seeded.make_tokens(4, 32, cfgd["vocab_size"], seed=558)
+    idx, tgt = idx.cuda(), tgt.cuda()
+    full = torch.zeros(native.param_elems(cfg), device="cuda")
+    acts, fws, bws = native.train_buffers(cfg, 4, 32)
+    native.forward_train(cfg, m.weights, idx, tgt, acts, fws)
+    native.backward(cfg, m.weights, idx, tgt, acts, full, bws)
+    acc = torch.zeros_like(full)
+    acts2, fws2, bws2 = native.train_buffers(cfg, 2, 32)
+    for k in range(2):
+        sl = slice(2 * k, 2 * k + 2)
+        native.forward_train(cfg, m.weights, idx[sl].contiguous(), tgt[sl].contiguous(), acts2, fws2)
+        native.backward(cfg, m.weights, idx[sl].contiguous(), tgt[sl].contiguous(), acts2, acc, bws2, loss_scale=0.5)
+    torch.cuda.synchronize()
+    err = float((acc - full).abs().max()) / float(full.abs().max())
+    assert err <= 1e-5, err
