@@ -310,23 +310,34 @@ __global__ void colsum_rows_kernel(const E* __restrict__ y, int rows, int C, flo
 
 // dpre = dh * gelu'(pre): erf form Phi(z) + z phi(z); tanh form 0.5 (1 + tanh a) +
 // 0.5 z (1 - tanh^2 a) sqrt(2/pi) (1 + 3 * 0.044715 z^2), a = sqrt(2/pi) (z + 0.044715 z^3).
-template <typename E>
-__global__ void gelu_backward_kernel(const float* __restrict__ dh, const E* __restrict__ pre, E* __restrict__ dpre,
-                                     long long n, int tanh_form) {
-    griddep_launch_dependents();
-    griddep_wait();
-    const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-    if (i >= n) return;
-    const float z = ld1(pre + i);
-    float d;
+// d gelu(z) / dz for either form
+GPT_DEVINL float gelu_slope(float z, int tanh_form) {
     if (tanh_form) {
         const float c = 0.7978845608028654f;
         const float th = tanhf(c * (z + 0.044715f * z * z * z));
-        d = 0.5f * (1.f + th) + 0.5f * z * (1.f - th * th) * c * (1.f + 3.f * 0.044715f * z * z);
-    } else {
-        d = 0.5f * (1.f + erff(z * 0.7071067811865476f)) + z * 0.3989422804014327f * __expf(-0.5f * z * z);
+        return 0.5f * (1.f + th) + 0.5f * z * (1.f - th * th) * c * (1.f + 3.f * 0.044715f * z * z);
     }
-    dpre[i] = st1<E>(__ldcg(dh + i) * d);
+    return 0.5f * (1.f + erff(z * 0.7071067811865476f)) + z * 0.3989422804014327f * __expf(-0.5f * z * z);
+}
+
+template <typename E>
+__global__ void gelu_backward_kernel(const float* __restrict__ dh, const E* __restrict__ pre, E* __restrict__ dpre,
+                                     long long n, int tanh_form, int vec) {
+    griddep_launch_dependents();
+    griddep_wait();
+    // thread t: values [8t, 8t + 8), 16-byte accesses when `vec` and the group is whole
+    const long long i0 = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) * 8;
+    if (i0 >= n) return;
+    if (vec && i0 + 8 <= n) {
+        float z[8], g[8];
+        ld8(pre + i0, z);
+        ld8(dh + i0, g);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) g[e] *= gelu_slope(z[e], tanh_form);
+        st8(dpre + i0, g);
+        return;
+    }
+    for (long long i = i0; i < n && i < i0 + 8; ++i) dpre[i] = st1<E>(__ldcg(dh + i) * gelu_slope(ld1(pre + i), tanh_form));
 }
 
 // ------------------------------------------------------------------ embedding backward
@@ -494,12 +505,15 @@ int launch_colsum(const void* y, int dtype, int rows, int C, float* out, int acc
 
 int launch_gelu_backward(const float* dh, const void* pre, int dtype, void* dpre, long long n, int tanh_form,
                          cudaStream_t s) {
-    const dim3 g(static_cast<unsigned>((n + 255) / 256)), b(256);
+    if (n == 0) return GPT_OK;
+    const dim3 g(static_cast<unsigned>((n + 8LL * 256 - 1) / (8LL * 256))), b(256);
+    auto al = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
+    const int vec = al(dh) && al(pre) && al(dpre);
     if (dtype == GPT_DTYPE_BF16)
         return launch_overlapped(gelu_backward_kernel<bf16>, g, b, 0, s, dh, static_cast<const bf16*>(pre),
-                                 static_cast<bf16*>(dpre), n, tanh_form);
+                                 static_cast<bf16*>(dpre), n, tanh_form, vec);
     return launch_overlapped(gelu_backward_kernel<float>, g, b, 0, s, dh, static_cast<const float*>(pre),
-                             static_cast<float*>(dpre), n, tanh_form);
+                             static_cast<float*>(dpre), n, tanh_form, vec);
 }
 
 int embed_backward_max_rows() { return kEmbSortMax; }

@@ -113,6 +113,15 @@ GPT_DEVINL void tma_load_4d(void* dst, const CUtensorMap* map, uint64_t* bar, in
         : "memory");
 }
 
+// Contiguous global -> shared copy of `bytes` (a multiple of 16; both addresses 16-byte aligned),
+// counted on `bar` like a tensor load.
+GPT_DEVINL void bulk_load_1d(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_addr(dst)),
+                 "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_addr(bar))
+                 : "memory");
+}
+
 // Shared -> global tile store and tile reduce-add (fp32 add at the destination), tracked by the
 // issuing thread's bulk-async group.  The tile must have been written to shared memory by
 // threads that then executed fence_proxy_async_shared() and synchronised with the issuer.
@@ -185,12 +194,13 @@ GPT_DEVINL void umma_commit(uint64_t* bar) {
         : "memory");
 }
 
-// Instruction descriptor of kind::f16: bf16 x bf16 -> fp32, M x N, A K-major, B K-major
-// unless b_mn_major.
-__host__ __device__ constexpr uint32_t make_idesc_bf16(int M, int N, bool b_mn_major) {
+// Instruction descriptor of kind::f16: bf16 x bf16 -> fp32, M x N, A K-major unless a_mn_major,
+// B K-major unless b_mn_major.
+__host__ __device__ constexpr uint32_t make_idesc_bf16(int M, int N, bool b_mn_major, bool a_mn_major = false) {
     return (1u << 4)                         // D format fp32
            | (1u << 7)                       // A format bf16
            | (1u << 10)                      // B format bf16
+           | ((a_mn_major ? 1u : 0u) << 15)  // A major-ness
            | ((b_mn_major ? 1u : 0u) << 16)  // B major-ness
            | ((uint32_t)(N >> 3) << 17)      // N / 8
            | ((uint32_t)(M >> 4) << 24);     // M / 16
@@ -205,6 +215,17 @@ GPT_DEVINL uint64_t make_sdesc_sw128(uint32_t saddr) {
            | ((uint64_t)(1024 >> 4) << 32)      // stride byte offset: 8 rows x 128 B
            | ((uint64_t)1 << 46)                // descriptor version for sm_100
            | ((uint64_t)2 << 61);               // 128-byte swizzle
+}
+
+// MN-major operand wider than one 64-element swizzle atom: rows of 128 bytes along K (8-row groups
+// 1024 bytes apart), and the next 64 elements of M or N `mn_stride` bytes further on (the leading
+// byte offset of the canonical MN-major 128-byte-swizzle layout).
+GPT_DEVINL uint64_t make_sdesc_sw128_mn(uint32_t saddr, uint32_t mn_stride) {
+    return (uint64_t)((saddr & 0x3FFFFu) >> 4)
+           | ((uint64_t)((mn_stride >> 4) & 0x3FFFu) << 16)
+           | ((uint64_t)(1024 >> 4) << 32)
+           | ((uint64_t)1 << 46)
+           | ((uint64_t)2 << 61);
 }
 
 // 32 lanes x 32 bit, 32 consecutive columns per thread: thread i of the warp receives
@@ -296,6 +317,28 @@ GPT_DEVINL uint32_t pack_bf16x2(float lo, float hi) {
 // as soon as every CTA of this grid has started or finished.
 GPT_DEVINL void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 GPT_DEVINL void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Eight consecutive values through one 16-byte L2 load (bf16) or two (fp32), and the matching
+// plain stores; p must be 16-byte aligned.  The loads bypass L1 (data written by earlier kernels of
+// an overlapped launch chain may be stale there).
+GPT_DEVINL void ld8(const bf16* p, float (&f)[8]) {
+    const uint4 w = __ldcg(reinterpret_cast<const uint4*>(p));
+    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) f[2 * i] = __uint_as_float(u[i] << 16), f[2 * i + 1] = __uint_as_float(u[i] & 0xffff0000u);
+}
+GPT_DEVINL void ld8(const float* p, float (&f)[8]) {
+    const float4 a = __ldcg(reinterpret_cast<const float4*>(p)), b = __ldcg(reinterpret_cast<const float4*>(p) + 1);
+    f[0] = a.x, f[1] = a.y, f[2] = a.z, f[3] = a.w, f[4] = b.x, f[5] = b.y, f[6] = b.z, f[7] = b.w;
+}
+GPT_DEVINL void st8(bf16* p, const float (&f)[8]) {
+    *reinterpret_cast<uint4*>(p) = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
+                                              pack_bf16x2(f[6], f[7]));
+}
+GPT_DEVINL void st8(float* p, const float (&f)[8]) {
+    reinterpret_cast<float4*>(p)[0] = make_float4(f[0], f[1], f[2], f[3]);
+    reinterpret_cast<float4*>(p)[1] = make_float4(f[4], f[5], f[6], f[7]);
+}
 
 // Records a device-side status (first writer wins).
 GPT_DEVINL void set_status(int32_t* status, int32_t code) {

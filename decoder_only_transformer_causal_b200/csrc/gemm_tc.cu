@@ -8,11 +8,11 @@ namespace {
 
 constexpr int kBN = 256;
 
-template <int EPI, int GELU_TANH>
+template <int EPI, int GELU_TANH, int A_MN = 0, int B_MN = 0>
 int launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, const gemm::Params& p,
                cudaStream_t s) {
     using L = gemm::Cfg<kBN>;
-    auto kern = gemm::gemm_bf16_tc<kBN, EPI, GELU_TANH>;
+    auto kern = gemm::gemm_bf16_tc<kBN, EPI, GELU_TANH, A_MN, B_MN>;
     static size_t opted[kMaxDevices] = {};
     const int rc = opt_in_smem(reinterpret_cast<const void*>(kern), L::SMEM_BYTES, opted);
     if (rc) return rc;
@@ -67,6 +67,36 @@ int launch_gemm_bf16(const bf16* A, long long lda, const bf16* W, long long ldw,
             return launch_one<gemm::EPI_CE, 0>(ta, tb, tc, p, s);
         default: return GPT_ERR_UNSUPPORTED;
     }
+}
+
+int launch_gemm_bf16_acc(const bf16* A, long long lda, bool a_mn, const bf16* W, long long ldw, bool b_mn, float* out,
+                         long long ldo, int M, int N, int K, int32_t* status, cudaStream_t s) {
+    if (M == 0 || N == 0) return GPT_OK;
+    if (a_mn == false && b_mn == false)
+        return launch_gemm_bf16(A, lda, W, ldw, nullptr, out, ldo, M, N, K, GPT_EPI_RESID, 0, nullptr, status, s);
+    if (!b_mn) return GPT_ERR_UNSUPPORTED;  // MN-major A is only paired with MN-major B
+    CUtensorMap ta, tb, tc;
+    int rc = a_mn ? make_tmap_bf16_2d(&ta, A, static_cast<uint64_t>(M), static_cast<uint64_t>(K),
+                                      static_cast<uint64_t>(lda) * 2, 64, gemm::BK)
+                  : make_tmap_bf16_2d(&ta, A, static_cast<uint64_t>(K), static_cast<uint64_t>(M),
+                                      static_cast<uint64_t>(lda) * 2, gemm::BK, gemm::BM);
+    if (rc) return rc;
+    rc = make_tmap_bf16_2d(&tb, W, static_cast<uint64_t>(N), static_cast<uint64_t>(K), static_cast<uint64_t>(ldw) * 2,
+                           64, gemm::BK);
+    if (rc) return rc;
+    rc = make_tmap_2d_sw64(&tc, out, true, static_cast<uint64_t>(N), static_cast<uint64_t>(M),
+                           static_cast<uint64_t>(ldo) * 4, 16, 32);
+    if (rc) return rc;
+    gemm::Params p{};
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    p.out = out;
+    p.ldo = ldo;
+    p.n_fastest = static_cast<long long>(M) >= static_cast<long long>(N) ? 1 : 0;
+    p.status = status;
+    return a_mn ? launch_one<gemm::EPI_RESID, 0, 1, 1>(ta, tb, tc, p, s)
+                : launch_one<gemm::EPI_RESID, 0, 0, 1>(ta, tb, tc, p, s);
 }
 
 }  // namespace gpt

@@ -97,7 +97,11 @@ GPT_DEVINL float gelu_f(float x) {
     return 0.5f * x * (1.0f + copysignf(erf_abs, x));
 }
 
-template <int BN, int EPI, int GELU_TANH>
+// A_MN / B_MN: the operand is stored MN-major, i.e. as the [K, M] (or [K, N]) row-major matrix
+// whose transpose the product needs (the backward's dY^T X and dY W).  Its tile is then loaded
+// as 64-column TMA boxes (64 K rows x 128 bytes each, 8 KB apart) and described to the MMA with
+// the MN-major layout; no transposed copy is made.
+template <int BN, int EPI, int GELU_TANH, int A_MN = 0, int B_MN = 0>
 __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)  // 10 warps: <= 168 registers per thread
     gemm_bf16_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const __grid_constant__ CUtensorMap tmC, const Params p) {
@@ -178,8 +182,20 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)  // 10 warps: <= 168 regi
                     }
                     uint8_t* st = smem + stage * L::STAGE_BYTES;
                     mbar_arrive_expect_tx(&full[stage], L::STAGE_BYTES);
-                    tma_load_2d(st, &tmA, &full[stage], kb * BK, m0);
-                    tma_load_2d(st + L::A_BYTES, &tmB, &full[stage], kb * BK, n0);
+                    if (A_MN) {
+#pragma unroll
+                        for (int j = 0; j < BM / 64; ++j)
+                            tma_load_2d(st + j * 8192, &tmA, &full[stage], m0 + 64 * j, kb * BK);
+                    } else {
+                        tma_load_2d(st, &tmA, &full[stage], kb * BK, m0);
+                    }
+                    if (B_MN) {
+#pragma unroll
+                        for (int j = 0; j < BN / 64; ++j)
+                            tma_load_2d(st + L::A_BYTES + j * 8192, &tmB, &full[stage], n0 + 64 * j, kb * BK);
+                    } else {
+                        tma_load_2d(st + L::A_BYTES, &tmB, &full[stage], kb * BK, n0);
+                    }
                     ++issued;
                     if (++stage == kStages) {
                         stage = 0;
@@ -198,7 +214,7 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)  // 10 warps: <= 168 regi
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idesc = make_idesc_bf16(BM, BN, false);
+            constexpr uint32_t idesc = make_idesc_bf16(BM, BN, B_MN != 0, A_MN != 0);
             int stage = 0;
             uint32_t ph = 0;
             int acc = 0;
@@ -218,8 +234,13 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)  // 10 warps: <= 168 regi
                     const uint32_t b_addr = a_addr + L::A_BYTES;
 #pragma unroll
                     for (int k = 0; k < BK / 16; ++k) {
-                        umma_ss(d, make_sdesc_sw128(a_addr + k * 32), make_sdesc_sw128(b_addr + k * 32),
-                                idesc, (kb | k) != 0 ? 1u : 0u);
+                        // K step of 16: 32 bytes along a K-major row, 16 rows (2048 bytes) of an
+                        // MN-major tile.
+                        const uint64_t da = A_MN ? make_sdesc_sw128_mn(a_addr + k * 2048, 8192)
+                                                 : make_sdesc_sw128(a_addr + k * 32);
+                        const uint64_t db = B_MN ? make_sdesc_sw128_mn(b_addr + k * 2048, 8192)
+                                                 : make_sdesc_sw128(b_addr + k * 32);
+                        umma_ss(d, da, db, idesc, (kb | k) != 0 ? 1u : 0u);
                     }
                     umma_commit(&empty[stage]);
                     if (++stage == kStages) {

@@ -940,7 +940,7 @@ GPT_API int gpt_attention_train(const void* q, const void* k, const void* v, voi
 
 GPT_API size_t gpt_attention_backward_workspace_bytes(int B, int nh, int T) {
     if (B < 1 || nh < 1 || T < 1) return 0;
-    return a256(static_cast<size_t>(B) * nh * T * 4);
+    return a256(attn_bwd_scratch_bytes(B, nh, T));
 }
 
 GPT_API int gpt_attention_backward(const void* q, const void* k, const void* v, const void* o, const void* dout,
@@ -958,12 +958,55 @@ GPT_API int gpt_attention_backward(const void* q, const void* k, const void* v, 
         AttnBwdLayout<bf16> L{static_cast<const bf16*>(q), static_cast<const bf16*>(k), static_cast<const bf16*>(v),
                               sb, sh, hs, static_cast<const bf16*>(o), static_cast<const bf16*>(dout), sb, sh, hs,
                               static_cast<bf16*>(dq), static_cast<bf16*>(dk), static_cast<bf16*>(dv), lse};
-        return launch_attention_backward(&L, nullptr, B, nh, T, hs, D, s);
+        return launch_attention_backward(&L, nullptr, B, nh, T, hs, D, nullptr, s);
     }
     AttnBwdLayout<float> L{static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v), sb,
                            sh, hs, static_cast<const float*>(o), static_cast<const float*>(dout), sb, sh, hs,
                            static_cast<float*>(dq), static_cast<float*>(dk), static_cast<float*>(dv), lse};
-    return launch_attention_backward(nullptr, &L, B, nh, T, hs, D, s);
+    return launch_attention_backward(nullptr, &L, B, nh, T, hs, D, nullptr, s);
+}
+
+GPT_API size_t gpt_linear_backward_workspace_bytes(int rows, int n_out, int n_in, int dtype) {
+    if (rows < 1 || n_out < 1 || n_in < 1) return 0;
+    if (dtype == GPT_DTYPE_BF16) return 256;
+    if (dtype != GPT_DTYPE_F32) return 0;
+    const size_t r = rows, o = n_out, i = n_in;
+    return 256 + a256(i * o * 4) + a256(o * r * 4) + a256(i * r * 4);
+}
+
+GPT_API int gpt_linear_backward(const void* dy, const void* x, const void* W, int rows, int n_out, int n_in, int dtype,
+                                float* dx, float* dW, void* workspace, size_t workspace_bytes, int32_t* status,
+                                void* stream) {
+    if (!dy || !x || !W || !dx || !dW || !workspace) return GPT_ERR_NULL;
+    if (rows < 0 || n_out <= 0 || n_in <= 0) return GPT_ERR_BAD_SHAPE;
+    if (dtype != GPT_DTYPE_BF16 && dtype != GPT_DTYPE_F32) return GPT_ERR_BAD_SHAPE;
+    if (rows == 0) return GPT_OK;
+    if (workspace_bytes < gpt_linear_backward_workspace_bytes(rows, n_out, n_in, dtype)) return GPT_ERR_WS_TOO_SMALL;
+    if (!aligned(workspace, 256) || !aligned(dx, 16) || !aligned(dW, 16)) return GPT_ERR_BAD_ALIGN;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    GPT_TRY(cuda_status(cudaMemsetAsync(dx, 0, static_cast<size_t>(rows) * n_in * 4, s)));
+    if (dtype == GPT_DTYPE_BF16) {
+        if ((n_out % 8) || (n_in % 8)) return GPT_ERR_UNSUPPORTED;
+        if (!aligned(dy, 16) || !aligned(x, 16) || !aligned(W, 16)) return GPT_ERR_BAD_ALIGN;
+        const bf16* y = static_cast<const bf16*>(dy);
+        // dx = dy W: dy K-major, W stored [n_out = K, n_in = N] (MN-major B)
+        GPT_TRY(launch_gemm_bf16_acc(y, n_out, false, static_cast<const bf16*>(W), n_in, true, dx, n_in, rows, n_in,
+                                     n_out, status, s));
+        // dW += dy^T x: dy stored [rows = K, n_out = M], x stored [rows = K, n_in = N] (both MN-major)
+        return launch_gemm_bf16_acc(y, n_out, true, static_cast<const bf16*>(x), n_in, true, dW, n_in, n_out, n_in,
+                                    rows, status, s);
+    }
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    const size_t r = rows, o = n_out, i = n_in;
+    float* wT = reinterpret_cast<float*>(ws + 256);
+    float* yT = reinterpret_cast<float*>(ws + 256 + a256(i * o * 4));
+    float* xT = reinterpret_cast<float*>(ws + 256 + a256(i * o * 4) + a256(o * r * 4));
+    GPT_TRY(launch_transpose(W, GPT_DTYPE_F32, n_in, wT, GPT_DTYPE_F32, n_out, n_out, n_in, s));
+    GPT_TRY(launch_linear_f32(static_cast<const float*>(dy), n_out, wT, nullptr, dx, n_in, rows, n_in, n_out,
+                              GPT_EPI_RESID, GPT_GELU_ERF, s));
+    GPT_TRY(launch_transpose(dy, GPT_DTYPE_F32, n_out, yT, GPT_DTYPE_F32, rows, rows, n_out, s));
+    GPT_TRY(launch_transpose(x, GPT_DTYPE_F32, n_in, xT, GPT_DTYPE_F32, rows, rows, n_in, s));
+    return launch_linear_f32(yT, rows, xT, nullptr, dW, n_in, n_out, n_in, rows, GPT_EPI_RESID, GPT_GELU_ERF, s);
 }
 
 GPT_API int gpt_transpose(const void* in, int in_dtype, long long ld_in, void* out, int out_dtype, long long ld_out,
@@ -1018,18 +1061,21 @@ BwdPlan plan_bwd(const gpt_config_t* c, long long B, long long T) {
     const size_t N = static_cast<size_t>(B * T), C = c->n_embd, V = c->vocab_size, es = elem_size(c);
     size_t off = 0;
     P.ctrl = off; off += 256;
+    // Transposed copies of the Linear layers' operands: fp32 only (bf16 hands the GEMM the stored
+    // matrices as MN-major operands).
+    const size_t tr = c->dtype == GPT_DTYPE_BF16 ? 0 : 1;
     P.dz = off; off += a256(N * V * es);
-    P.dzT = off; off += a256(N * V * es);
-    P.wT = off; off += a256(std::max(V * C, 4 * C * C) * es);
+    P.dzT = off; off += a256(tr * N * V * es);
+    P.wT = off; off += a256(tr * std::max(V * C, 4 * C * C) * es);
     P.gE = off; off += a256(N * 4 * C * es);
-    P.gT = off; off += a256(N * 4 * C * es);
-    P.aT = off; off += a256(N * 4 * C * es);
+    P.gT = off; off += a256(tr * N * 4 * C * es);
+    P.aT = off; off += a256(tr * N * 4 * C * es);
     P.d1 = off; off += a256(N * 4 * C * 4);
     P.dx = off; off += a256(N * C * 4);
     P.dpre = off; off += a256(N * 4 * C * es);
     P.dqkv = off; off += a256(N * 3 * C * es);
     P.dy = off; off += a256(N * C * es);
-    P.D = off; off += a256(static_cast<size_t>(B) * c->n_head * T * 4);
+    P.D = off; off += a256(attn_bwd_scratch_bytes(B, c->n_head, T));
     const size_t lnp = static_cast<size_t>(layernorm_backward_parts(static_cast<int>(N), static_cast<int>(C))) * 2 * C;
     const size_t csp = static_cast<size_t>(colsum_parts(static_cast<int>(N))) * 4 * C;
     P.parts = off; off += a256(std::max(lnp, csp) * 4);
@@ -1223,50 +1269,51 @@ GPT_API int gpt_backward(const gpt_config_t* cfg, const void* weights, const int
     const int F32 = GPT_DTYPE_F32;
     const size_t nc = static_cast<size_t>(N) * C;
 
+    // Linear backward: dIn (fp32 [N, n_in], zeroed here) = dY W and dW (fp32) += dY^T X, for dY
+    // [N, n_out] (row stride ldy), X [N, n_in] (row stride ldx) and W [n_out, n_in] in the config
+    // dtype.  bf16 hands the GEMM the stored dY, X and W as MN-major operands where the product needs
+    // their transposes; fp32 forms the transposes in scratch first (yT: room for dY^T).
+    auto linear_bwd = [&](const void* dYp, long long ldy, const void* Xp, long long ldx, const void* Wp, int n_out,
+                          int n_in, float* dIn, float* dW, void* yT) -> int {
+        GPT_TRY(cuda_status(cudaMemsetAsync(dIn, 0, static_cast<size_t>(N) * n_in * 4, s)));
+        if (bf) {
+            const bf16* y = static_cast<const bf16*>(dYp);
+            GPT_TRY(launch_gemm_bf16_acc(y, ldy, false, static_cast<const bf16*>(Wp), n_in, true, dIn, n_in, N, n_in,
+                                         n_out, status, s));
+            return launch_gemm_bf16_acc(y, ldy, true, static_cast<const bf16*>(Xp), ldx, true, dW, n_in, n_out, n_in,
+                                        N, status, s);
+        }
+        GPT_TRY(launch_transpose(Wp, dt, n_in, wT, dt, n_out, n_out, n_in, s));
+        GPT_TRY(gemm_acc(cfg, dYp, ldy, wT, n_out, dIn, n_in, N, n_in, n_out, status, s));
+        GPT_TRY(launch_transpose(dYp, dt, ldy, yT, dt, N, N, n_out, s));
+        GPT_TRY(launch_transpose(Xp, dt, ldx, aT, dt, N, N, n_in, s));
+        return gemm_acc(cfg, yT, N, aT, N, dW, n_in, n_out, n_in, N, status, s);
+    };
+
     GPT_TRY(cuda_status(cudaMemsetAsync(status, 0, sizeof(int32_t), s)));
     // d loss / d logits, then the tied head: du_f = dz wte, dwte += dz^T u_f
     if (!(loss_scale > 0.f) || !isfinite(loss_scale)) return GPT_ERR_BAD_SHAPE;
     GPT_TRY(launch_ce_backward(ab + A.logits, dt, targets, reinterpret_cast<const double*>(ab + A.sum_count), dz, N, V,
                                status, s, loss_scale));
-    GPT_TRY(launch_transpose(W.wte(), dt, C, wT, dt, V, V, C, s));
-    GPT_TRY(cuda_status(cudaMemsetAsync(d1, 0, nc * 4, s)));
-    GPT_TRY(gemm_acc(cfg, dz, V, wT, V, d1, C, N, C, V, status, s));
-    GPT_TRY(launch_transpose(dz, dt, V, dzT, dt, N, N, V, s));
-    GPT_TRY(launch_transpose(ab + A.u_f, dt, C, aT, dt, N, N, C, s));
-    GPT_TRY(gemm_acc(cfg, dzT, N, aT, N, G(0), C, V, C, N, status, s));
+    GPT_TRY(linear_bwd(dz, V, ab + A.u_f, C, W.wte(), V, C, d1, G(0), dzT));
     GPT_TRY(launch_layernorm_backward(d1, reinterpret_cast<const float*>(ab + A.x_f), W.lnf_w(), dt, dx, 0, G(count - 2),
                                       cfg->bias ? G(count - 1) : nullptr, 1, parts, N, C, s));
     for (int l = cfg->n_layer - 1; l >= 0; --l) {
         const uint8_t* L = ab + A.layer * l;
         // mlp c_proj: dh = dx W_fc2 (into d1 [N, 4C]); dW_fc2 += dx^T h; db_fc2 += sum dx
         GPT_TRY(launch_convert(dx, F32, gE, dt, static_cast<long long>(nc), s));
-        GPT_TRY(launch_transpose(W.layer(l, W_FC2_W), dt, 4LL * C, wT, dt, C, C, 4 * C, s));
-        GPT_TRY(cuda_status(cudaMemsetAsync(d1, 0, nc * 4 * 4, s)));
-        GPT_TRY(gemm_acc(cfg, gE, C, wT, C, d1, 4LL * C, N, 4 * C, C, status, s));
-        GPT_TRY(launch_transpose(dx, F32, C, gT, dt, N, N, C, s));
-        GPT_TRY(launch_transpose(L + A.h, dt, 4LL * C, aT, dt, N, N, 4 * C, s));
-        GPT_TRY(gemm_acc(cfg, gT, N, aT, N, GL(l, W_FC2_W), 4LL * C, C, 4 * C, N, status, s));
+        GPT_TRY(linear_bwd(gE, C, L + A.h, 4LL * C, W.layer(l, W_FC2_W), C, 4 * C, d1, GL(l, W_FC2_W), gT));
         if (cfg->bias) GPT_TRY(launch_colsum(dx, F32, N, C, GL(l, W_FC2_B), 1, parts, s));
         // GELU, then c_fc: du2 = dpre W_fc (into d1 [N, C]); dW_fc += dpre^T u2; db_fc += sum dpre
         GPT_TRY(launch_gelu_backward(d1, L + A.pre, dt, dpre, static_cast<long long>(nc) * 4, cfg->gelu == GPT_GELU_TANH, s));
-        GPT_TRY(launch_transpose(W.layer(l, W_FC_W), dt, C, wT, dt, 4LL * C, 4 * C, C, s));
-        GPT_TRY(cuda_status(cudaMemsetAsync(d1, 0, nc * 4, s)));
-        GPT_TRY(gemm_acc(cfg, dpre, 4LL * C, wT, 4LL * C, d1, C, N, C, 4 * C, status, s));
-        GPT_TRY(launch_transpose(dpre, dt, 4LL * C, gT, dt, N, N, 4 * C, s));
-        GPT_TRY(launch_transpose(L + A.u2, dt, C, aT, dt, N, N, C, s));
-        GPT_TRY(gemm_acc(cfg, gT, N, aT, N, GL(l, W_FC_W), C, 4 * C, C, N, status, s));
+        GPT_TRY(linear_bwd(dpre, 4LL * C, L + A.u2, C, W.layer(l, W_FC_W), 4 * C, C, d1, GL(l, W_FC_W), gT));
         if (cfg->bias) GPT_TRY(launch_colsum(dpre, dt, N, 4 * C, GL(l, W_FC_B), 1, parts, s));
         GPT_TRY(launch_layernorm_backward(d1, reinterpret_cast<const float*>(L + A.x_mid), W.layer(l, W_LN2_W), dt, dx, 1,
                                           GL(l, W_LN2_W), cfg->bias ? GL(l, W_LN2_B) : nullptr, 1, parts, N, C, s));
         // attn c_proj: dy = dx W_proj; dW_proj += dx^T y; db_proj += sum dx
         GPT_TRY(launch_convert(dx, F32, gE, dt, static_cast<long long>(nc), s));
-        GPT_TRY(launch_transpose(W.layer(l, W_PROJ_W), dt, C, wT, dt, C, C, C, s));
-        GPT_TRY(cuda_status(cudaMemsetAsync(d1, 0, nc * 4, s)));
-        GPT_TRY(gemm_acc(cfg, gE, C, wT, C, d1, C, N, C, C, status, s));
+        GPT_TRY(linear_bwd(gE, C, L + A.y, C, W.layer(l, W_PROJ_W), C, C, d1, GL(l, W_PROJ_W), gT));
         GPT_TRY(launch_convert(d1, F32, dy, dt, static_cast<long long>(nc), s));
-        GPT_TRY(launch_transpose(dx, F32, C, gT, dt, N, N, C, s));
-        GPT_TRY(launch_transpose(L + A.y, dt, C, aT, dt, N, N, C, s));
-        GPT_TRY(gemm_acc(cfg, gT, N, aT, N, GL(l, W_PROJ_W), C, C, C, N, status, s));
         if (cfg->bias) GPT_TRY(launch_colsum(dx, F32, N, C, GL(l, W_PROJ_B), 1, parts, s));
         // attention backward into dqkv (the qkv layout)
         const float* lse = reinterpret_cast<const float*>(L + A.lse);
@@ -1277,22 +1324,17 @@ GPT_API int gpt_backward(const gpt_config_t* cfg, const void* weights, const int
             AttnBwdLayout<bf16> AL{q, q + C, q + 2 * C, qsb, hs, 3LL * C,
                                    reinterpret_cast<const bf16*>(L + A.y), static_cast<const bf16*>(dy), ysb, hs, C,
                                    dq, dq + C, dq + 2 * C, lse};
-            GPT_TRY(launch_attention_backward(&AL, nullptr, B, nh, T, hs, D, s));
+            GPT_TRY(launch_attention_backward(&AL, nullptr, B, nh, T, hs, D, status, s));
         } else {
             const float* q = reinterpret_cast<const float*>(L + A.qkv);
             float* dq = static_cast<float*>(dqkv);
             AttnBwdLayout<float> AL{q, q + C, q + 2 * C, qsb, hs, 3LL * C,
                                     reinterpret_cast<const float*>(L + A.y), static_cast<const float*>(dy), ysb, hs, C,
                                     dq, dq + C, dq + 2 * C, lse};
-            GPT_TRY(launch_attention_backward(nullptr, &AL, B, nh, T, hs, D, s));
+            GPT_TRY(launch_attention_backward(nullptr, &AL, B, nh, T, hs, D, status, s));
         }
         // c_attn: du1 = dqkv W_attn (into d1 [N, C]); dW_attn += dqkv^T u1; db_attn += sum dqkv
-        GPT_TRY(launch_transpose(W.layer(l, W_ATTN_W), dt, C, wT, dt, 3LL * C, 3 * C, C, s));
-        GPT_TRY(cuda_status(cudaMemsetAsync(d1, 0, nc * 4, s)));
-        GPT_TRY(gemm_acc(cfg, dqkv, 3LL * C, wT, 3LL * C, d1, C, N, C, 3 * C, status, s));
-        GPT_TRY(launch_transpose(dqkv, dt, 3LL * C, gT, dt, N, N, 3 * C, s));
-        GPT_TRY(launch_transpose(L + A.u1, dt, C, aT, dt, N, N, C, s));
-        GPT_TRY(gemm_acc(cfg, gT, N, aT, N, GL(l, W_ATTN_W), C, 3 * C, C, N, status, s));
+        GPT_TRY(linear_bwd(dqkv, 3LL * C, L + A.u1, C, W.layer(l, W_ATTN_W), 3 * C, C, d1, GL(l, W_ATTN_W), gT));
         if (cfg->bias) GPT_TRY(launch_colsum(dqkv, dt, N, 3 * C, GL(l, W_ATTN_B), 1, parts, s));
         GPT_TRY(launch_layernorm_backward(d1, reinterpret_cast<const float*>(L + A.x_in), W.layer(l, W_LN1_W), dt, dx, 1,
                                           GL(l, W_LN1_W), cfg->bias ? GL(l, W_LN1_B) : nullptr, 1, parts, N, C, s));

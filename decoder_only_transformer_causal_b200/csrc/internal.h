@@ -79,6 +79,12 @@ int launch_gemm_bf16(const bf16* A, long long lda, const bf16* W, long long ldw,
                      void* out, long long ldo, int M, int N, int K, int epilogue, int gelu,
                      const CeArgs* ce, int32_t* status, cudaStream_t s);
 
+// out[M, N] (fp32, row stride ldo) += A B^T.  A: [M, K] (a_mn false) or stored as [K, M] (a_mn);
+// W: [N, K] (b_mn false) or stored as [K, N] (b_mn); row strides lda / ldw in elements.  a_mn
+// requires b_mn.
+int launch_gemm_bf16_acc(const bf16* A, long long lda, bool a_mn, const bf16* W, long long ldw, bool b_mn, float* out,
+                         long long ldo, int M, int N, int K, int32_t* status, cudaStream_t s);
+
 // ---- tensor-core attention (attention_tc.cu); strides in elements
 struct AttnLayout {
     const bf16 *q, *k, *v;
@@ -171,8 +177,15 @@ int launch_transpose(const void* in, int in_dtype, long long ld_in, void* out, i
                      int Cc, cudaStream_t s);
 int launch_convert(const void* in, int in_dtype, void* out, int out_dtype, long long n, cudaStream_t s);
 int launch_gelu_forward(const void* pre, void* h, long long n, int dtype, int tanh_form, cudaStream_t s);
-// D: [B, nh, T] fp32 scratch.  Exactly one of Lb / Lf is non-null; hs 32 or 64.
+// scratch: attn_bwd_scratch_bytes(B, nh, T) bytes, 16-byte aligned (D and lse2 padded to a multiple
+// of 128 rows per head).  Exactly one of Lb / Lf is non-null; hs 32 or 64.  status: optional device
+// word that records GPT_ERR_TIMEOUT from the tensor-core kernels.
+size_t attn_bwd_scratch_bytes(long long B, long long nh, long long T);
 int launch_attention_backward(const AttnBwdLayout<bf16>* Lb, const AttnBwdLayout<float>* Lf, int B, int nh, int T,
-                              int hs, float* D, cudaStream_t s);
+                              int hs, float* scratch, int32_t* status, cudaStream_t s);
+// bf16, head size 64: returns GPT_ERR_BAD_ALIGN (nothing launched) when an operand cannot be
+// described by a TMA map.
+int launch_attention_backward_tc(const AttnBwdLayout<bf16>& L, int B, int nh, int T, const float* D,
+                                 const float* lse2, int32_t* status, cudaStream_t s);
 
 }  // namespace gpt

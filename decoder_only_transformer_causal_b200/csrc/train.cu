@@ -8,9 +8,10 @@
 //   D_i   = sum_d dO_i[d] O_i[d]
 //   dS_ij = p_ij (dO_i . v_j - D_i)               for j <= i, 0 above the diagonal
 //   dQ_i  = sum_j dS_ij k_j / sqrt(hs),  dK_j = sum_i dS_ij q_i / sqrt(hs),  dV_j = sum_i p_ij dO_i
-// This first version runs on the SIMT pipes: two threads per row, each holding half of the head
-// dimensions in registers, with the other side's 64-row tiles staged in shared memory and read by
-// broadcast; the two halves of a dot product meet in one shuffle.
+// bf16 with head size 64 runs on the tensor cores (attention_bwd_tc.cu); the kernels here cover fp32,
+// head size 32 and operands TMA cannot address: two threads per row, each holding half of the
+// head dimensions in registers, with the other side's 64-row tiles staged in shared memory and
+// read by broadcast; the two halves of a dot product meet in one shuffle.
 #include <math.h>
 
 #include "common.cuh"
@@ -48,44 +49,70 @@ __global__ void transpose_kernel(const Ti* __restrict__ in, long long ld_in, To*
     }
 }
 
+// Elementwise kernels: thread t takes values [8t, 8t + 8) with 16-byte accesses when `vec` (every
+// buffer 16-byte aligned) and the group is whole, one value at a time otherwise.
 template <typename Ti, typename To>
-__global__ void convert_kernel(const Ti* __restrict__ in, To* __restrict__ out, long long n) {
+__global__ void convert_kernel(const Ti* __restrict__ in, To* __restrict__ out, long long n, int vec) {
     griddep_launch_dependents();
     griddep_wait();
-    const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-    if (i < n) out[i] = stf<To>(ldf(in + i));
+    const long long i0 = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) * 8;
+    if (i0 >= n) return;
+    if (vec && i0 + 8 <= n) {
+        float v[8];
+        ld8(in + i0, v);
+        st8(out + i0, v);
+        return;
+    }
+    for (long long i = i0; i < n && i < i0 + 8; ++i) out[i] = stf<To>(ldf(in + i));
+}
+
+GPT_DEVINL float gelu_value(float z, int tanh_form) {
+    return tanh_form ? 0.5f * z * (1.f + tanhf(0.7978845608028654f * (z + 0.044715f * z * z * z)))
+                     : 0.5f * z * (1.f + erff(z * 0.7071067811865476f));
 }
 
 template <typename E>
-__global__ void gelu_forward_kernel(const E* __restrict__ pre, E* __restrict__ h, long long n, int tanh_form) {
+__global__ void gelu_forward_kernel(const E* __restrict__ pre, E* __restrict__ h, long long n, int tanh_form, int vec) {
     griddep_launch_dependents();
     griddep_wait();
-    const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-    if (i >= n) return;
-    const float z = ldf(pre + i);
-    const float g = tanh_form ? 0.5f * z * (1.f + tanhf(0.7978845608028654f * (z + 0.044715f * z * z * z)))
-                              : 0.5f * z * (1.f + erff(z * 0.7071067811865476f));
-    h[i] = stf<E>(g);
+    const long long i0 = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) * 8;
+    if (i0 >= n) return;
+    if (vec && i0 + 8 <= n) {
+        float v[8];
+        ld8(pre + i0, v);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[e] = gelu_value(v[e], tanh_form);
+        st8(h + i0, v);
+        return;
+    }
+    for (long long i = i0; i < n && i < i0 + 8; ++i) h[i] = stf<E>(gelu_value(ldf(pre + i), tanh_form));
 }
 
 // ------------------------------------------------------------------ attention backward
-// D[bh * T + i] = sum_d dO_i[d] O_i[d]; one warp per row.
+// Per (b, h) and query row i < Tp (Tp = T rounded up to 128): D[bh * Tp + i] = sum_d dO_i[d] O_i[d]
+// and L2[bh * Tp + i] = the forward's lse2_i; rows i >= T hold D = 0 and L2 = +inf (p = 0 there).
+// One warp per row.
 template <typename E>
-__global__ void attn_bwd_rowdot_kernel(const AttnBwdLayout<E> L, int B, int nh, int T, int hs, float* __restrict__ D) {
+__global__ void attn_bwd_rowdot_kernel(const AttnBwdLayout<E> L, int B, int nh, int T, int Tp, int hs,
+                                       float* __restrict__ D, float* __restrict__ L2) {
     griddep_launch_dependents();
     griddep_wait();
     const long long row = static_cast<long long>(blockIdx.x) * (blockDim.x / 32) + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
-    if (row >= static_cast<long long>(B) * nh * T) return;
-    const int i = static_cast<int>(row % T);
-    const int bh = static_cast<int>(row / T), b = bh / nh, h = bh % nh;
+    if (row >= static_cast<long long>(B) * nh * Tp) return;
+    const int i = static_cast<int>(row % Tp);
+    const int bh = static_cast<int>(row / Tp), b = bh / nh, h = bh % nh;
+    if (i >= T) {
+        if (lane == 0) D[row] = 0.f, L2[row] = INFINITY;
+        return;
+    }
     const E* o = L.o + b * L.o_sb + h * L.o_sh + static_cast<long long>(i) * L.o_st;
     const E* g = L.dout + b * L.o_sb + h * L.o_sh + static_cast<long long>(i) * L.o_st;
     float s = 0.f;
     for (int d = lane; d < hs; d += 32) s += ldf(o + d) * ldf(g + d);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-    if (lane == 0) D[row] = s;
+    if (lane == 0) D[row] = s, L2[row] = __ldcg(L.lse + static_cast<long long>(bh) * T + i);
 }
 
 constexpr int kBwdRows = 64;  // rows per CTA and per staged tile
@@ -93,15 +120,16 @@ constexpr int kBwdRows = 64;  // rows per CTA and per staged tile
 // dQ for 64 query rows of one (b, h): thread (row, half); key tiles of 64 in shared memory.
 template <typename E, int HS>
 __global__ void __launch_bounds__(2 * kBwdRows)
-    attn_bwd_dq_kernel(const AttnBwdLayout<E> L, int nh, int T, float scale_log2, float inv_sqrt_hs,
+    attn_bwd_dq_kernel(const AttnBwdLayout<E> L, int nh, int T, int Tp, float scale_log2, float inv_sqrt_hs,
                        const float* __restrict__ D) {
     griddep_launch_dependents();
     griddep_wait();
     constexpr int H2 = HS / 2;
-    __shared__ float ks[kBwdRows][HS + 1], vs[kBwdRows][HS + 1];
+    __shared__ __align__(16) float ks[kBwdRows][HS + 4], vs[kBwdRows][HS + 4];
     const int bh = blockIdx.y, b = bh / nh, h = bh % nh;
     const int half = threadIdx.x & 1;
-    const int i = blockIdx.x * kBwdRows + (threadIdx.x >> 1);
+    const int tile = gridDim.x - 1 - blockIdx.x;  // the last query tiles see the most keys: start them first
+    const int i = tile * kBwdRows + (threadIdx.x >> 1);
     const bool live = i < T;
     const int ic = live ? i : T - 1;
     const E* q = L.q + b * L.sb + h * L.sh + static_cast<long long>(ic) * L.st + half * H2;
@@ -110,8 +138,8 @@ __global__ void __launch_bounds__(2 * kBwdRows)
 #pragma unroll
     for (int d = 0; d < H2; ++d) qr[d] = ldf(q + d), gr[d] = ldf(g + d), acc[d] = 0.f;
     const float lse = __ldcg(L.lse + static_cast<long long>(bh) * T + ic);
-    const float Di = __ldcg(D + static_cast<long long>(bh) * T + ic);
-    const int last_row = min(T - 1, (blockIdx.x + 1) * kBwdRows - 1);
+    const float Di = __ldcg(D + static_cast<long long>(bh) * Tp + ic);
+    const int last_row = min(T - 1, (tile + 1) * kBwdRows - 1);
     for (int j0 = 0; j0 <= last_row; j0 += kBwdRows) {
         __syncthreads();
         for (int e = threadIdx.x; e < kBwdRows * HS; e += 2 * kBwdRows) {
@@ -123,18 +151,34 @@ __global__ void __launch_bounds__(2 * kBwdRows)
         const int jn = min(kBwdRows, last_row - j0 + 1);
         for (int jj = 0; jj < jn; ++jj) {
             const int j = j0 + jj;
-            float s = 0.f, dp = 0.f;
+            const float4* kr4 = reinterpret_cast<const float4*>(&ks[jj][half * H2]);
+            const float4* vr4 = reinterpret_cast<const float4*>(&vs[jj][half * H2]);
+            float s4[4] = {0.f, 0.f, 0.f, 0.f}, p4[4] = {0.f, 0.f, 0.f, 0.f};  // independent chains
 #pragma unroll
-            for (int d = 0; d < H2; ++d) {
-                s = fmaf(qr[d], ks[jj][half * H2 + d], s);
-                dp = fmaf(gr[d], vs[jj][half * H2 + d], dp);
+            for (int d = 0; d < H2 / 4; ++d) {
+                const float4 kk = kr4[d], vv = vr4[d];
+                s4[0] = fmaf(qr[4 * d], kk.x, s4[0]);
+                s4[1] = fmaf(qr[4 * d + 1], kk.y, s4[1]);
+                s4[2] = fmaf(qr[4 * d + 2], kk.z, s4[2]);
+                s4[3] = fmaf(qr[4 * d + 3], kk.w, s4[3]);
+                p4[0] = fmaf(gr[4 * d], vv.x, p4[0]);
+                p4[1] = fmaf(gr[4 * d + 1], vv.y, p4[1]);
+                p4[2] = fmaf(gr[4 * d + 2], vv.z, p4[2]);
+                p4[3] = fmaf(gr[4 * d + 3], vv.w, p4[3]);
             }
+            float s = (s4[0] + s4[1]) + (s4[2] + s4[3]), dp = (p4[0] + p4[1]) + (p4[2] + p4[3]);
             s += __shfl_xor_sync(0xffffffffu, s, 1);
             dp += __shfl_xor_sync(0xffffffffu, dp, 1);
             const float p = (live && j <= i) ? exp2f(s * scale_log2 - lse) : 0.f;
             const float ds = p * (dp - Di);
 #pragma unroll
-            for (int d = 0; d < H2; ++d) acc[d] = fmaf(ds, ks[jj][half * H2 + d], acc[d]);
+            for (int d = 0; d < H2 / 4; ++d) {
+                const float4 kk = kr4[d];
+                acc[4 * d] = fmaf(ds, kk.x, acc[4 * d]);
+                acc[4 * d + 1] = fmaf(ds, kk.y, acc[4 * d + 1]);
+                acc[4 * d + 2] = fmaf(ds, kk.z, acc[4 * d + 2]);
+                acc[4 * d + 3] = fmaf(ds, kk.w, acc[4 * d + 3]);
+            }
         }
     }
     if (!live) return;
@@ -147,12 +191,12 @@ __global__ void __launch_bounds__(2 * kBwdRows)
 // lse and D) in shared memory, from the diagonal tile down.
 template <typename E, int HS>
 __global__ void __launch_bounds__(2 * kBwdRows)
-    attn_bwd_dkdv_kernel(const AttnBwdLayout<E> L, int nh, int T, float scale_log2, float inv_sqrt_hs,
+    attn_bwd_dkdv_kernel(const AttnBwdLayout<E> L, int nh, int T, int Tp, float scale_log2, float inv_sqrt_hs,
                          const float* __restrict__ D) {
     griddep_launch_dependents();
     griddep_wait();
     constexpr int H2 = HS / 2;
-    __shared__ float qs[kBwdRows][HS + 1], gs[kBwdRows][HS + 1];
+    __shared__ __align__(16) float qs[kBwdRows][HS + 4], gs[kBwdRows][HS + 4];
     __shared__ float ls[kBwdRows], dsum[kBwdRows];
     const int bh = blockIdx.y, b = bh / nh, h = bh % nh;
     const int half = threadIdx.x & 1;
@@ -174,26 +218,43 @@ __global__ void __launch_bounds__(2 * kBwdRows)
         for (int ii = threadIdx.x; ii < kBwdRows; ii += 2 * kBwdRows) {
             const int i = min(i0 + ii, T - 1);
             ls[ii] = __ldcg(L.lse + static_cast<long long>(bh) * T + i);
-            dsum[ii] = __ldcg(D + static_cast<long long>(bh) * T + i);
+            dsum[ii] = __ldcg(D + static_cast<long long>(bh) * Tp + i);
         }
         __syncthreads();
         const int in = min(kBwdRows, T - i0);
         for (int ii = 0; ii < in; ++ii) {
             const int i = i0 + ii;
-            float s = 0.f, dp = 0.f;
+            const float4* qr4 = reinterpret_cast<const float4*>(&qs[ii][half * H2]);
+            const float4* gr4 = reinterpret_cast<const float4*>(&gs[ii][half * H2]);
+            float s4[4] = {0.f, 0.f, 0.f, 0.f}, p4[4] = {0.f, 0.f, 0.f, 0.f};  // independent chains
 #pragma unroll
-            for (int d = 0; d < H2; ++d) {
-                s = fmaf(kr[d], qs[ii][half * H2 + d], s);
-                dp = fmaf(vr[d], gs[ii][half * H2 + d], dp);
+            for (int d = 0; d < H2 / 4; ++d) {
+                const float4 qq = qr4[d], gg = gr4[d];
+                s4[0] = fmaf(kr[4 * d], qq.x, s4[0]);
+                s4[1] = fmaf(kr[4 * d + 1], qq.y, s4[1]);
+                s4[2] = fmaf(kr[4 * d + 2], qq.z, s4[2]);
+                s4[3] = fmaf(kr[4 * d + 3], qq.w, s4[3]);
+                p4[0] = fmaf(vr[4 * d], gg.x, p4[0]);
+                p4[1] = fmaf(vr[4 * d + 1], gg.y, p4[1]);
+                p4[2] = fmaf(vr[4 * d + 2], gg.z, p4[2]);
+                p4[3] = fmaf(vr[4 * d + 3], gg.w, p4[3]);
             }
+            float s = (s4[0] + s4[1]) + (s4[2] + s4[3]), dp = (p4[0] + p4[1]) + (p4[2] + p4[3]);
             s += __shfl_xor_sync(0xffffffffu, s, 1);
             dp += __shfl_xor_sync(0xffffffffu, dp, 1);
             const float p = (live && j <= i) ? exp2f(s * scale_log2 - ls[ii]) : 0.f;
             const float ds = p * (dp - dsum[ii]);
 #pragma unroll
-            for (int d = 0; d < H2; ++d) {
-                dv[d] = fmaf(p, gs[ii][half * H2 + d], dv[d]);
-                dk[d] = fmaf(ds, qs[ii][half * H2 + d], dk[d]);
+            for (int d = 0; d < H2 / 4; ++d) {
+                const float4 qq = qr4[d], gg = gr4[d];
+                dv[4 * d] = fmaf(p, gg.x, dv[4 * d]);
+                dv[4 * d + 1] = fmaf(p, gg.y, dv[4 * d + 1]);
+                dv[4 * d + 2] = fmaf(p, gg.z, dv[4 * d + 2]);
+                dv[4 * d + 3] = fmaf(p, gg.w, dv[4 * d + 3]);
+                dk[4 * d] = fmaf(ds, qq.x, dk[4 * d]);
+                dk[4 * d + 1] = fmaf(ds, qq.y, dk[4 * d + 1]);
+                dk[4 * d + 2] = fmaf(ds, qq.z, dk[4 * d + 2]);
+                dk[4 * d + 3] = fmaf(ds, qq.w, dk[4 * d + 3]);
             }
         }
     }
@@ -204,19 +265,28 @@ __global__ void __launch_bounds__(2 * kBwdRows)
     for (int d = 0; d < H2; ++d) odk[d] = stf<E>(dk[d] * inv_sqrt_hs), odv[d] = stf<E>(dv[d]);
 }
 
+// D / L2: the padded [B*nh, Tp] arrays of attn_bwd_rowdot_kernel.
 template <typename E, int HS>
-int attn_bwd_typed(const AttnBwdLayout<E>& L, int B, int nh, int T, float* D, cudaStream_t s) {
-    const long long rows = static_cast<long long>(B) * nh * T;
+int attn_bwd_typed(const AttnBwdLayout<E>& L, int B, int nh, int T, float* D, float* L2, int32_t* status,
+                   cudaStream_t s) {
+    const int Tp = (T + 127) / 128 * 128;
+    const long long rows = static_cast<long long>(B) * nh * Tp;
     int rc = launch_overlapped(attn_bwd_rowdot_kernel<E>, dim3(static_cast<unsigned>((rows + 7) / 8)), dim3(256), 0, s,
-                               L, B, nh, T, HS, D);
+                               L, B, nh, T, Tp, HS, D, L2);
     if (rc) return rc;
+    if constexpr (sizeof(E) == 2 && HS == 64) {
+        // Tensor-core kernels whenever the operands can be described by TMA maps (16-byte
+        // aligned bases and strides); the SIMT kernels below otherwise.
+        rc = launch_attention_backward_tc(L, B, nh, T, D, L2, status, s);
+        if (rc != GPT_ERR_BAD_ALIGN) return rc;
+    }
     const float scale_log2 = static_cast<float>(1.4426950408889634 / sqrt(static_cast<double>(HS)));
     const float inv = static_cast<float>(1.0 / sqrt(static_cast<double>(HS)));
     const dim3 grid((T + kBwdRows - 1) / kBwdRows, B * nh), block(2 * kBwdRows);
-    rc = launch_overlapped(attn_bwd_dq_kernel<E, HS>, grid, block, 0, s, L, nh, T, scale_log2, inv,
+    rc = launch_overlapped(attn_bwd_dq_kernel<E, HS>, grid, block, 0, s, L, nh, T, Tp, scale_log2, inv,
                            static_cast<const float*>(D));
     if (rc) return rc;
-    return launch_overlapped(attn_bwd_dkdv_kernel<E, HS>, grid, block, 0, s, L, nh, T, scale_log2, inv,
+    return launch_overlapped(attn_bwd_dkdv_kernel<E, HS>, grid, block, 0, s, L, nh, T, Tp, scale_log2, inv,
                              static_cast<const float*>(D));
 }
 
@@ -240,43 +310,52 @@ int launch_transpose(const void* in, int in_dtype, long long ld_in, void* out, i
                              static_cast<float*>(out), ld_out, R, Cc);
 }
 
+namespace {
+bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+dim3 grid8(long long n) { return dim3(static_cast<unsigned>((n + 8LL * 256 - 1) / (8LL * 256))); }
+}  // namespace
+
 int launch_convert(const void* in, int in_dtype, void* out, int out_dtype, long long n, cudaStream_t s) {
     if (n == 0) return GPT_OK;
-    const dim3 grid(static_cast<unsigned>((n + 255) / 256)), block(256);
+    const dim3 grid = grid8(n), block(256);
+    const int vec = al16(in) && al16(out);
     const bool ib = in_dtype == GPT_DTYPE_BF16, ob = out_dtype == GPT_DTYPE_BF16;
     if (!ib && ob)
         return launch_overlapped(convert_kernel<float, bf16>, grid, block, 0, s, static_cast<const float*>(in),
-                                 static_cast<bf16*>(out), n);
+                                 static_cast<bf16*>(out), n, vec);
     if (ib && !ob)
         return launch_overlapped(convert_kernel<bf16, float>, grid, block, 0, s, static_cast<const bf16*>(in),
-                                 static_cast<float*>(out), n);
+                                 static_cast<float*>(out), n, vec);
     if (ib)
         return launch_overlapped(convert_kernel<bf16, bf16>, grid, block, 0, s, static_cast<const bf16*>(in),
-                                 static_cast<bf16*>(out), n);
+                                 static_cast<bf16*>(out), n, vec);
     return launch_overlapped(convert_kernel<float, float>, grid, block, 0, s, static_cast<const float*>(in),
-                             static_cast<float*>(out), n);
+                             static_cast<float*>(out), n, vec);
 }
 
 int launch_gelu_forward(const void* pre, void* h, long long n, int dtype, int tanh_form, cudaStream_t s) {
     if (n == 0) return GPT_OK;
-    const dim3 grid(static_cast<unsigned>((n + 255) / 256)), block(256);
+    const dim3 grid = grid8(n), block(256);
+    const int vec = al16(pre) && al16(h);
     if (dtype == GPT_DTYPE_BF16)
         return launch_overlapped(gelu_forward_kernel<bf16>, grid, block, 0, s, static_cast<const bf16*>(pre),
-                                 static_cast<bf16*>(h), n, tanh_form);
+                                 static_cast<bf16*>(h), n, tanh_form, vec);
     return launch_overlapped(gelu_forward_kernel<float>, grid, block, 0, s, static_cast<const float*>(pre),
-                             static_cast<float*>(h), n, tanh_form);
+                             static_cast<float*>(h), n, tanh_form, vec);
 }
 
 int launch_attention_backward(const AttnBwdLayout<bf16>* Lb, const AttnBwdLayout<float>* Lf, int B, int nh, int T,
-                              int hs, float* D, cudaStream_t s) {
+                              int hs, float* scratch, int32_t* status, cudaStream_t s) {
     if (B == 0 || nh == 0 || T == 0) return GPT_OK;
+    float* D = scratch;
+    float* L2 = scratch + static_cast<long long>(B) * nh * ((T + 127) / 128 * 128);
     if (Lb) {
-        if (hs == 64) return attn_bwd_typed<bf16, 64>(*Lb, B, nh, T, D, s);
-        if (hs == 32) return attn_bwd_typed<bf16, 32>(*Lb, B, nh, T, D, s);
+        if (hs == 64) return attn_bwd_typed<bf16, 64>(*Lb, B, nh, T, D, L2, status, s);
+        if (hs == 32) return attn_bwd_typed<bf16, 32>(*Lb, B, nh, T, D, L2, status, s);
         return GPT_ERR_UNSUPPORTED;
     }
-    if (hs == 64) return attn_bwd_typed<float, 64>(*Lf, B, nh, T, D, s);
-    if (hs == 32) return attn_bwd_typed<float, 32>(*Lf, B, nh, T, D, s);
+    if (hs == 64) return attn_bwd_typed<float, 64>(*Lf, B, nh, T, D, L2, status, s);
+    if (hs == 32) return attn_bwd_typed<float, 32>(*Lf, B, nh, T, D, L2, status, s);
     return GPT_ERR_UNSUPPORTED;
 }
 

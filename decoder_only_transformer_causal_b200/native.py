@@ -106,6 +106,8 @@ def _load() -> ctypes.CDLL:
         "gpt_embedding_backward": (I, [P, P, I, I, I, I, P, P, P, Z, P, P]),
         "gpt_attention_train": (I, [P, P, P, P, P, I, I, I, I, D, P, P]),
         "gpt_attention_backward_workspace_bytes": (Z, [I, I, I]),
+        "gpt_linear_backward_workspace_bytes": (Z, [I, I, I, I]),
+        "gpt_linear_backward": (I, [P, P, P, I, I, I, I, P, P, P, Z, P, P]),
         "gpt_attention_backward": (I, [P, P, P, P, P, P, P, P, P, I, I, I, I, D, P, Z, P]),
         "gpt_transpose": (I, [P, D, L, P, D, L, I, I, P]),
         "gpt_train_activation_bytes": (Z, [CFG, I, I]),
@@ -133,6 +135,7 @@ EXPORTED = ("gpt_status_string", "gpt_abi_version", "gpt_last_cuda_error", "gpt_
             "gpt_layernorm_backward_workspace_bytes", "gpt_layernorm_backward", "gpt_bias_grad_workspace_bytes",
             "gpt_bias_grad", "gpt_gelu_backward", "gpt_embedding_backward_workspace_bytes", "gpt_embedding_backward",
             "gpt_attention_train", "gpt_attention_backward_workspace_bytes", "gpt_attention_backward", "gpt_transpose",
+            "gpt_linear_backward_workspace_bytes", "gpt_linear_backward",
             "gpt_train_activation_bytes", "gpt_backward_workspace_bytes", "gpt_forward_train", "gpt_backward",
             "gpt_train_loss_terms_offset")
 
@@ -581,6 +584,20 @@ def attention_backward(q, k, v, o, dout, lse, stream=None):
                                       _ptr(dv), B, nh, T, hs, _dt(q), _ptr(ws), ws.numel(), _stream(stream)),
            "gpt_attention_backward")
     return dq, dk, dv
+
+
+def linear_backward(dy, x, W, dW=None, status=None, stream=None):
+    """gpt_linear_backward: returns (dx fp32, dW fp32); dW is accumulated into when given."""
+    rows, n_out = dy.shape
+    n_in = x.shape[1]
+    dx = torch.empty((rows, n_in), dtype=torch.float32, device=dy.device)
+    if dW is None:
+        dW = torch.zeros((n_out, n_in), dtype=torch.float32, device=dy.device)
+    ws = alloc_workspace(LIB.gpt_linear_backward_workspace_bytes(max(rows, 1), n_out, n_in, _dt(dy)), dy.device)
+    _check(LIB.gpt_linear_backward(_ptr(dy), _ptr(x), _ptr(W), rows, n_out, n_in, _dt(dy), _ptr(dx), _ptr(dW), _ptr(ws),
+                                   ws.numel(), _ptr(status) if status is not None else None, _stream(stream)),
+           "gpt_linear_backward")
+    return dx, dW
 
 
 def transpose(x: torch.Tensor, out_dtype=None, stream=None) -> torch.Tensor:

@@ -376,11 +376,29 @@ int gpt_attention_train(const void* q, const void* k, const void* v, void* y, fl
  * q, k and lse, D_i = dout_i . o_i and dS_ij = p_ij (dout_i . v_j - D_i) for j <= i,
  *   dq_i = sum_j dS_ij k_j / sqrt(hs),  dk_j = sum_i dS_ij q_i / sqrt(hs),  dv_j = sum_i p_ij dout_i.
  * All [B, nh, T, hs] in `dtype` (o = the forward's y, lse from gpt_attention_train); hs 32 or 64;
- * fp32 accumulation.  workspace: gpt_attention_backward_workspace_bytes(B, nh, T) bytes (D). */
+ * fp32 accumulation.  bf16 with hs 64 and 16-byte aligned operands runs two tensor-core kernels
+ * (dK/dV per 128-key tile, dQ per 128-query tile; P and dS rounded to bf16 as MMA operands);
+ * everything else runs SIMT kernels.  Results are bit-reproducible (fixed summation order).
+ * workspace: gpt_attention_backward_workspace_bytes(B, nh, T) bytes, 256-byte aligned (D and a
+ * padded copy of lse). */
 size_t gpt_attention_backward_workspace_bytes(int B, int nh, int T);
 int gpt_attention_backward(const void* q, const void* k, const void* v, const void* o, const void* dout,
                            const float* lse, void* dq, void* dk, void* dv, int B, int nh, int T, int hs,
                            int dtype, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Backward of nn.Linear y = x W^T + b ("nanoGPT 全局流程图", 3.4 反向传播):
+ *   dx = dy W       fp32 [rows, n_in], overwritten
+ *   dW += dy^T x    fp32 [n_out, n_in], accumulated
+ * dy [rows, n_out], x [rows, n_in], W [n_out, n_in] (nn.Linear layout), dense, in `dtype`.  bf16: the
+ * tensor-core GEMM reads dy, x and W where they are, as MN-major operands wherever the product
+ * needs a transpose (no copies); n_out and n_in multiples of 8, pointers 16-byte aligned.  fp32:
+ * transposed copies in workspace feed the SIMT GEMM.  workspace:
+ * gpt_linear_backward_workspace_bytes(rows, n_out, n_in, dtype) bytes (256 for bf16), 256-byte
+ * aligned.  The bias gradient is gpt_bias_grad of dy.  status: as gpt_linear. */
+size_t gpt_linear_backward_workspace_bytes(int rows, int n_out, int n_in, int dtype);
+int gpt_linear_backward(const void* dy, const void* x, const void* W, int rows, int n_out, int n_in, int dtype,
+                        float* dx, float* dW, void* workspace, size_t workspace_bytes, int32_t* status,
+                        void* stream);
 
 /* out[c * ld_out + r] = in[r * ld_in + c] for r < rows, c < cols, converting between bf16 and fp32
  * (the operand layouts of the backward's products). */
@@ -403,8 +421,8 @@ int gpt_transpose(const void* in, int in_dtype, long long ld_in, void* out, int 
  * K accumulated micro-batches (the page's loss / gradient_accumulation_steps); must be > 0.
  * workspace: gpt_backward_workspace_bytes.
  * Head size 32 or 64; for bf16, B * T % 8 == 0; B * T <= 16384.  Linear layers' backward products
- * run on the tensor-core GEMM (bf16) after explicit transposes; the attention backward is the
- * SIMT kernel of gpt_attention_backward. */
+ * are gpt_linear_backward's (bf16: tensor-core GEMM on MN-major operands, no transposed copies);
+ * the attention backward is gpt_attention_backward's (bf16, head size 64: tensor cores). */
 size_t gpt_train_activation_bytes(const gpt_config_t* cfg, int B, int T);
 size_t gpt_backward_workspace_bytes(const gpt_config_t* cfg, int B, int T);
 int gpt_forward_train(const gpt_config_t* cfg, const void* weights, const int64_t* idx,
