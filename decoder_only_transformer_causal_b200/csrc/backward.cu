@@ -192,9 +192,31 @@ __global__ void __launch_bounds__(kBwdWarps * 32)
 }
 
 // The same with each row held in registers (VEC float4 of x and of dy per lane, C <= 128 VEC):
-// x and dy are read once, and each warp takes kLnRowsPerWarp consecutive rows into its column
-// sums, so a CTA leaves one partial per 64 rows.
-constexpr int kLnRowsPerWarp = 8;  // rows per warp in the register kernel: 64 per CTA
+// x and dy are read once; each warp takes kLnRowsPerWarp consecutive rows.  Up to C = 768 (VEC 6)
+// the next row's x, dy (and the dx it adds to) are loaded while the current one is reduced and
+// the lanes' dw / db column sums stay in registers; wider rows (whose registers would spill) load
+// row by row and add into per-warp sums in shared memory.  The warps' sums meet in warp order, so
+// a CTA leaves one partial per 32 rows.
+constexpr int kLnRowsPerWarp = 4;  // rows per warp in the register kernel: 32 per CTA
+
+template <int VEC>
+struct LnRow {
+    float4 x[VEC], g[VEC], old[VEC];
+};
+
+template <int VEC>
+GPT_DEVINL void ln_row_load(LnRow<VEC>& R, const float* x, const float* dy, const float* dx, int accumulate, int lane,
+                            int C) {
+#pragma unroll
+    for (int j = 0; j < VEC; ++j) {
+        const int c = (lane + 32 * j) * 4;
+        if (c < C) {
+            R.x[j] = __ldcg(reinterpret_cast<const float4*>(x + c));
+            R.g[j] = __ldcg(reinterpret_cast<const float4*>(dy + c));
+            R.old[j] = accumulate ? __ldcg(reinterpret_cast<const float4*>(dx + c)) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    }
+}
 
 template <typename Tw, int VEC>
 __global__ void __launch_bounds__(kBwdWarps * 32)
@@ -204,36 +226,49 @@ __global__ void __launch_bounds__(kBwdWarps * 32)
     griddep_wait();
     extern __shared__ float sm[];  // [kBwdWarps][2][C] per-warp column sums
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    float* my = sm + static_cast<size_t>(warp) * 2 * C;
-    for (int c = lane; c < 2 * C; c += 32) my[c] = 0.f;
-    __syncwarp();
-    float4 wv[VEC];
+    float4 wv[VEC], dwa[VEC], dba[VEC];
 #pragma unroll
     for (int j = 0; j < VEC; ++j) {
         const int c = (lane + 32 * j) * 4;
-        if (c < C) wv[j] = make_float4(ld1(w + c), ld1(w + c + 1), ld1(w + c + 2), ld1(w + c + 3));
+        wv[j] = c < C ? make_float4(ld1(w + c), ld1(w + c + 1), ld1(w + c + 2), ld1(w + c + 3))
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
+        dwa[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+        dba[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    constexpr bool kPipe = VEC <= 6;
+    float* my = sm + static_cast<size_t>(warp) * 2 * C;
+    if constexpr (!kPipe) {
+        for (int c = lane; c < 2 * C; c += 32) my[c] = 0.f;
+        __syncwarp();
     }
     const int r0 = (blockIdx.x * kBwdWarps + warp) * kLnRowsPerWarp;
-    for (int r = r0; r < min(rows, r0 + kLnRowsPerWarp); ++r) {
-        const float* xr = x + static_cast<long long>(r) * C;
-        const float* dyr = dy + static_cast<long long>(r) * C;
-        float4 xv[VEC], gv[VEC];
+    const int r1 = min(rows, r0 + kLnRowsPerWarp);
+    LnRow<VEC> cur, nxt;
+    if (kPipe && r0 < r1) {
+        const long long o = static_cast<long long>(r0) * C;
+        ln_row_load(cur, x + o, dy + o, dx + o, accumulate, lane, C);
+    }
+    for (int r = r0; r < r1; ++r) {
+        if constexpr (kPipe) {
+            if (r + 1 < r1) {
+                const long long o = static_cast<long long>(r + 1) * C;
+                ln_row_load(nxt, x + o, dy + o, dx + o, accumulate, lane, C);
+            }
+        } else {
+            const long long o = static_cast<long long>(r) * C;
+            ln_row_load(cur, x + o, dy + o, dx + o, accumulate, lane, C);
+        }
+        float4* xv = cur.x;
+        const float4* gv = cur.g;
         float s = 0.f;
 #pragma unroll
-        for (int j = 0; j < VEC; ++j) {
-            const int c = (lane + 32 * j) * 4;
-            if (c < C) {
-                xv[j] = __ldcg(reinterpret_cast<const float4*>(xr + c));
-                gv[j] = __ldcg(reinterpret_cast<const float4*>(dyr + c));
-                s += (xv[j].x + xv[j].y) + (xv[j].z + xv[j].w);
-            }
-        }
+        for (int j = 0; j < VEC; ++j)
+            if ((lane + 32 * j) * 4 < C) s += (xv[j].x + xv[j].y) + (xv[j].z + xv[j].w);
         const float mean = wsum(s) / C;
         float ss = 0.f;
 #pragma unroll
         for (int j = 0; j < VEC; ++j) {
-            const int c = (lane + 32 * j) * 4;
-            if (c < C) {
+            if ((lane + 32 * j) * 4 < C) {
                 xv[j].x -= mean, xv[j].y -= mean, xv[j].z -= mean, xv[j].w -= mean;
                 ss += (xv[j].x * xv[j].x + xv[j].y * xv[j].y) + (xv[j].z * xv[j].z + xv[j].w * xv[j].w);
             }
@@ -242,15 +277,21 @@ __global__ void __launch_bounds__(kBwdWarps * 32)
         float a = 0.f, bsum = 0.f;  // sums of dxhat and dxhat * xhat
 #pragma unroll
         for (int j = 0; j < VEC; ++j) {
-            const int c = (lane + 32 * j) * 4;
-            if (c < C) {
+            if ((lane + 32 * j) * 4 < C) {
                 xv[j].x *= rstd, xv[j].y *= rstd, xv[j].z *= rstd, xv[j].w *= rstd;  // xhat
                 a += (gv[j].x * wv[j].x + gv[j].y * wv[j].y) + (gv[j].z * wv[j].z + gv[j].w * wv[j].w);
                 bsum += (gv[j].x * wv[j].x * xv[j].x + gv[j].y * wv[j].y * xv[j].y) +
                         (gv[j].z * wv[j].z * xv[j].z + gv[j].w * wv[j].w * xv[j].w);
-                my[c] += gv[j].x * xv[j].x, my[c + 1] += gv[j].y * xv[j].y;
-                my[c + 2] += gv[j].z * xv[j].z, my[c + 3] += gv[j].w * xv[j].w;
-                my[C + c] += gv[j].x, my[C + c + 1] += gv[j].y, my[C + c + 2] += gv[j].z, my[C + c + 3] += gv[j].w;
+                if constexpr (kPipe) {
+                    dwa[j].x += gv[j].x * xv[j].x, dwa[j].y += gv[j].y * xv[j].y;
+                    dwa[j].z += gv[j].z * xv[j].z, dwa[j].w += gv[j].w * xv[j].w;
+                    dba[j].x += gv[j].x, dba[j].y += gv[j].y, dba[j].z += gv[j].z, dba[j].w += gv[j].w;
+                } else {
+                    const int c = (lane + 32 * j) * 4;
+                    my[c] += gv[j].x * xv[j].x, my[c + 1] += gv[j].y * xv[j].y;
+                    my[c + 2] += gv[j].z * xv[j].z, my[c + 3] += gv[j].w * xv[j].w;
+                    my[C + c] += gv[j].x, my[C + c + 1] += gv[j].y, my[C + c + 2] += gv[j].z, my[C + c + 3] += gv[j].w;
+                }
             }
         }
         const float ma = wsum(a) / C, mb = wsum(bsum) / C;
@@ -259,15 +300,22 @@ __global__ void __launch_bounds__(kBwdWarps * 32)
         for (int j = 0; j < VEC; ++j) {
             const int c = (lane + 32 * j) * 4;
             if (c < C) {
-                float4 o = make_float4(rstd * (gv[j].x * wv[j].x - ma - xv[j].x * mb),
-                                       rstd * (gv[j].y * wv[j].y - ma - xv[j].y * mb),
-                                       rstd * (gv[j].z * wv[j].z - ma - xv[j].z * mb),
-                                       rstd * (gv[j].w * wv[j].w - ma - xv[j].w * mb));
-                if (accumulate) {
-                    const float4 old = __ldcg(reinterpret_cast<const float4*>(dxr + c));
-                    o.x += old.x, o.y += old.y, o.z += old.z, o.w += old.w;
-                }
+                const float4 o = make_float4(cur.old[j].x + rstd * (gv[j].x * wv[j].x - ma - xv[j].x * mb),
+                                             cur.old[j].y + rstd * (gv[j].y * wv[j].y - ma - xv[j].y * mb),
+                                             cur.old[j].z + rstd * (gv[j].z * wv[j].z - ma - xv[j].z * mb),
+                                             cur.old[j].w + rstd * (gv[j].w * wv[j].w - ma - xv[j].w * mb));
                 *reinterpret_cast<float4*>(dxr + c) = o;
+            }
+        }
+        if constexpr (kPipe) cur = nxt;
+    }
+    if constexpr (kPipe) {
+#pragma unroll
+        for (int j = 0; j < VEC; ++j) {
+            const int c = (lane + 32 * j) * 4;
+            if (c < C) {
+                *reinterpret_cast<float4*>(my + c) = dwa[j];
+                *reinterpret_cast<float4*>(my + C + c) = dba[j];
             }
         }
     }
@@ -281,20 +329,33 @@ __global__ void __launch_bounds__(kBwdWarps * 32)
 
 // out[c] (+)= sum over i < n_part of part[i * ld + c], in order of i (the second stage of a
 // column reduction).
-__global__ void colsum_parts_kernel(const float* __restrict__ part, long long ld, int n_part, int C,
-                                    float* __restrict__ out, int accumulate) {
+__global__ void __launch_bounds__(256)
+    colsum_parts_kernel(const float* __restrict__ part, long long ld, int n_part, int C, float* __restrict__ out,
+                        int accumulate) {
     griddep_launch_dependents();
     griddep_wait();
-    const int c = blockIdx.x * blockDim.x + threadIdx.x;
-    if (c >= C) return;
+    // block (32, 8): column blockIdx.x * 32 + x; slice y sums parts y, y + 8, ... in order, then the
+    // eight slice sums are added in order (a fixed summation order for any launch).
+    __shared__ float red[8][33];
+    const int c = blockIdx.x * 32 + threadIdx.x;
     float v = 0.f;
-#pragma unroll 8
-    for (int i = 0; i < n_part; ++i) v += __ldcg(part + i * ld + c);
-    out[c] = accumulate ? __ldcg(out + c) + v : v;
+    if (c < C) {
+#pragma unroll 4
+        for (int i = threadIdx.y; i < n_part; i += 8) v += __ldcg(part + i * ld + c);
+    }
+    red[threadIdx.y][threadIdx.x] = v;
+    __syncthreads();
+    if (threadIdx.y == 0 && c < C) {
+        float t = red[0][threadIdx.x];
+#pragma unroll
+        for (int k = 1; k < 8; ++k) t += red[k][threadIdx.x];
+        out[c] = accumulate ? __ldcg(out + c) + t : t;
+    }
 }
 
-// part[blockIdx.y][c] = sum of y[r, c] over this CTA's row block (rows in order); first stage of
-// the bias gradient (column sums of the output gradient).
+// part[blockIdx.y][c] = sum of y[r, c] over this CTA's row block; first stage of the bias gradient
+// (column sums of the output gradient).  Rows are taken four at a time into four running sums
+// (more loads in flight), which are added in a fixed order at the end.
 constexpr int kColRows = 128;
 template <typename E>
 __global__ void colsum_rows_kernel(const E* __restrict__ y, int rows, int C, float* __restrict__ part) {
@@ -303,9 +364,17 @@ __global__ void colsum_rows_kernel(const E* __restrict__ y, int rows, int C, flo
     const int c = blockIdx.x * blockDim.x + threadIdx.x;
     if (c >= C) return;
     const int r0 = blockIdx.y * kColRows, r1 = min(rows, r0 + kColRows);
-    float v = 0.f;
-    for (int r = r0; r < r1; ++r) v += ld1(y + static_cast<long long>(r) * C + c);
-    part[static_cast<long long>(blockIdx.y) * C + c] = v;
+    float v0 = 0.f, v1 = 0.f, v2 = 0.f, v3 = 0.f;
+    int r = r0;
+    for (; r + 4 <= r1; r += 4) {
+        const E* q = y + static_cast<long long>(r) * C + c;
+        v0 += ld1(q);
+        v1 += ld1(q + C);
+        v2 += ld1(q + 2LL * C);
+        v3 += ld1(q + 3LL * C);
+    }
+    for (; r < r1; ++r) v0 += ld1(y + static_cast<long long>(r) * C + c);
+    part[static_cast<long long>(blockIdx.y) * C + c] = (v0 + v1) + (v2 + v3);
 }
 
 // dpre = dh * gelu'(pre): erf form Phi(z) + z phi(z); tanh form 0.5 (1 + tanh a) +
@@ -480,11 +549,12 @@ int launch_layernorm_backward(const float* dy, const float* x, const void* w, in
     }
     if (rc) return rc;
     const dim3 g((C + 255) / 256), b(256);
-    rc = launch_overlapped(colsum_parts_kernel, g, b, 0, s, static_cast<const float*>(part), 2LL * C, n_part, C, dw,
+    const dim3 gp((C + 31) / 32), bp(32, 8);
+    rc = launch_overlapped(colsum_parts_kernel, gp, bp, 0, s, static_cast<const float*>(part), 2LL * C, n_part, C, dw,
                            accumulate_wb);
     if (rc) return rc;
     if (!db) return GPT_OK;
-    return launch_overlapped(colsum_parts_kernel, g, b, 0, s, static_cast<const float*>(part + C), 2LL * C, n_part, C,
+    return launch_overlapped(colsum_parts_kernel, gp, bp, 0, s, static_cast<const float*>(part + C), 2LL * C, n_part, C,
                              db, accumulate_wb);
 }
 
@@ -499,8 +569,8 @@ int launch_colsum(const void* y, int dtype, int rows, int C, float* out, int acc
                  : launch_overlapped(colsum_rows_kernel<float>, g1, b, 0, s, static_cast<const float*>(y), rows, C,
                                      part);
     if (rc) return rc;
-    return launch_overlapped(colsum_parts_kernel, dim3((C + 255) / 256), b, 0, s, static_cast<const float*>(part),
-                             static_cast<long long>(C), n_part, C, out, accumulate);
+    return launch_overlapped(colsum_parts_kernel, dim3((C + 31) / 32), dim3(32, 8), 0, s,
+                             static_cast<const float*>(part), static_cast<long long>(C), n_part, C, out, accumulate);
 }
 
 int launch_gelu_backward(const float* dh, const void* pre, int dtype, void* dpre, long long n, int tanh_form,

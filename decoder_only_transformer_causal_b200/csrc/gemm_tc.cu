@@ -16,12 +16,57 @@ int launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& 
     static size_t opted[kMaxDevices] = {};
     const int rc = opt_in_smem(reinterpret_cast<const void*>(kern), L::SMEM_BYTES, opted);
     if (rc) return rc;
-    const int tiles = ((p.M + gemm::BM - 1) / gemm::BM) * ((p.N + kBN - 1) / kBN);
+    const int tiles = ((p.M + gemm::BM - 1) / gemm::BM) * ((p.N + kBN - 1) / kBN) * p.k_splits;
     const int grid = tiles < num_sms() ? tiles : num_sms();
     return launch_overlapped(kern, dim3(grid), dim3(L::THREADS), L::SMEM_BYTES, s, ta, tb, tc, p);
 }
 
+// out[m, n] += sum over s = 0..S-1, in order, of part[s * M + m][n]: the partial products of a
+// split-K launch (part rows of N fp32; N, ldo multiples of 4 and 16-byte aligned buffers).
+__global__ void splitk_reduce_kernel(const float* __restrict__ part, int S, int M, int N, float* __restrict__ out,
+                                     long long ldo) {
+    griddep_launch_dependents();
+    griddep_wait();
+    const long long n4 = N / 4;
+    const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (i >= static_cast<long long>(M) * n4) return;
+    const long long m = i / n4, c = (i % n4) * 4;
+    float4 t = __ldcg(reinterpret_cast<const float4*>(part + m * N + c));
+    for (int s = 1; s < S; ++s) {
+        const float4 v = __ldcg(reinterpret_cast<const float4*>(part + (static_cast<long long>(s) * M + m) * N + c));
+        t.x += v.x, t.y += v.y, t.z += v.z, t.w += v.w;
+    }
+    float4* o = reinterpret_cast<float4*>(out + m * ldo + c);
+    float4 d = __ldcg(o);
+    d.x += t.x, d.y += t.y, d.z += t.z, d.w += t.w;
+    *o = d;
+}
+
+// Split count for an accumulating product with MN-major A: enough K ranges that the tiles fill
+// about two waves of a 148-SM part when the M x N tiles alone would not, each range non-empty.
+// 1 = no split (also when M % 32 != 0 or N % 4 != 0).
+constexpr int kSplitTargetCtas = 296;
+void split_plan(int M, int N, int K, int* splits, int* kb_per) {
+    const int tiles = ((M + gemm::BM - 1) / gemm::BM) * ((N + kBN - 1) / kBN);
+    const int num_kb = (K + gemm::BK - 1) / gemm::BK;
+    *splits = 1;
+    *kb_per = num_kb;
+    if ((M % 32) || (N % 4) || tiles * 2 > kSplitTargetCtas || num_kb < 2) return;
+    int S = (kSplitTargetCtas + tiles - 1) / tiles;
+    S = S < num_kb ? S : num_kb;
+    S = S < 32 ? S : 32;
+    const int per = (num_kb + S - 1) / S;
+    *kb_per = per;
+    *splits = (num_kb + per - 1) / per;
+}
+
 }  // namespace
+
+size_t gemm_acc_split_bytes(int M, int N, int K) {
+    int S, per;
+    split_plan(M, N, K, &S, &per);
+    return S > 1 ? static_cast<size_t>(S) * M * N * 4 : 0;
+}
 
 int gemm_ce_parts(int N) { return ((N + kBN - 1) / kBN) * gemm::Cfg<kBN>::PARTS_PER_TILE; }
 
@@ -52,6 +97,8 @@ int launch_gemm_bf16(const bf16* A, long long lda, const bf16* W, long long ldw,
     // Visit tiles so that the larger operand streams from memory once (see gemm_tc.cuh).
     p.n_fastest = static_cast<long long>(M) >= static_cast<long long>(N) ? 1 : 0;
     p.status = status;
+    p.k_splits = 1;
+    p.kb_per_split = (K + gemm::BK - 1) / gemm::BK;
     switch (epilogue) {
         case GPT_EPI_STORE: return launch_one<gemm::EPI_STORE, 0>(ta, tb, tc, p, s);
         case GPT_EPI_GELU:
@@ -70,7 +117,7 @@ int launch_gemm_bf16(const bf16* A, long long lda, const bf16* W, long long ldw,
 }
 
 int launch_gemm_bf16_acc(const bf16* A, long long lda, bool a_mn, const bf16* W, long long ldw, bool b_mn, float* out,
-                         long long ldo, int M, int N, int K, int32_t* status, cudaStream_t s) {
+                         long long ldo, int M, int N, int K, int32_t* status, cudaStream_t s, float* split_ws) {
     if (M == 0 || N == 0) return GPT_OK;
     if (a_mn == false && b_mn == false)
         return launch_gemm_bf16(A, lda, W, ldw, nullptr, out, ldo, M, N, K, GPT_EPI_RESID, 0, nullptr, status, s);
@@ -84,17 +131,37 @@ int launch_gemm_bf16_acc(const bf16* A, long long lda, bool a_mn, const bf16* W,
     rc = make_tmap_bf16_2d(&tb, W, static_cast<uint64_t>(N), static_cast<uint64_t>(K), static_cast<uint64_t>(ldw) * 2,
                            64, gemm::BK);
     if (rc) return rc;
-    rc = make_tmap_2d_sw64(&tc, out, true, static_cast<uint64_t>(N), static_cast<uint64_t>(M),
-                           static_cast<uint64_t>(ldo) * 4, 16, 32);
-    if (rc) return rc;
     gemm::Params p{};
     p.M = M;
     p.N = N;
     p.K = K;
-    p.out = out;
-    p.ldo = ldo;
     p.n_fastest = static_cast<long long>(M) >= static_cast<long long>(N) ? 1 : 0;
     p.status = status;
+    int S = 1, per = (K + gemm::BK - 1) / gemm::BK;
+    if (a_mn && split_ws) split_plan(M, N, K, &S, &per);
+    p.k_splits = S;
+    p.kb_per_split = per;
+    if (S > 1) {
+        // Deterministic split-K: each K range stores its partial product into its own slice of
+        // split_ws, then one pass adds the slices to out in order.
+        if (((reinterpret_cast<uintptr_t>(out) | reinterpret_cast<uintptr_t>(split_ws)) & 15) || (ldo % 4))
+            return GPT_ERR_BAD_ALIGN;
+        rc = make_tmap_2d_sw64(&tc, split_ws, true, static_cast<uint64_t>(N), static_cast<uint64_t>(S) * M,
+                               static_cast<uint64_t>(N) * 4, 16, 32);
+        if (rc) return rc;
+        p.out = split_ws;
+        p.ldo = N;
+        rc = launch_one<gemm::EPI_F32, 0, 1, 1>(ta, tb, tc, p, s);
+        if (rc) return rc;
+        const long long n4 = static_cast<long long>(M) * (N / 4);
+        return launch_overlapped(splitk_reduce_kernel, dim3(static_cast<unsigned>((n4 + 255) / 256)), dim3(256), 0, s,
+                                 static_cast<const float*>(split_ws), S, M, N, out, ldo);
+    }
+    rc = make_tmap_2d_sw64(&tc, out, true, static_cast<uint64_t>(N), static_cast<uint64_t>(M),
+                           static_cast<uint64_t>(ldo) * 4, 16, 32);
+    if (rc) return rc;
+    p.out = out;
+    p.ldo = ldo;
     return a_mn ? launch_one<gemm::EPI_RESID, 0, 1, 1>(ta, tb, tc, p, s)
                 : launch_one<gemm::EPI_RESID, 0, 0, 1>(ta, tb, tc, p, s);
 }

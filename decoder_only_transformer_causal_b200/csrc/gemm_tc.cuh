@@ -35,7 +35,8 @@ constexpr int BK = 64;  // one 128-byte swizzle row of bf16
 constexpr int kStages = 4;
 constexpr int NEPI = 8;  // epilogue warps: two per TMEM lane quarter, each half of BN
 
-enum Epi { EPI_STORE = 0, EPI_GELU = 1, EPI_RESID = 2, EPI_CE = 3 };
+// EPI_F32: out_fp32 = acc, plain store (the partial products of a split-K launch).
+enum Epi { EPI_STORE = 0, EPI_GELU = 1, EPI_RESID = 2, EPI_CE = 3, EPI_F32 = 4 };
 
 struct Params {
     int M, N, K;
@@ -48,6 +49,10 @@ struct Params {
     float* tlogit;           // EPI_CE: [M], z[target] in fp32
     int n_part;
     int32_t* status;
+    // Split-K (EPI_F32 only): the K blocks are cut into k_splits ranges of kb_per_split blocks;
+    // split s stores its partial product at rows [s * M, s * M + M) of out (M % 32 == 0).
+    int k_splits;
+    int kb_per_split;
 };
 
 template <int BN>
@@ -123,9 +128,17 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)  // 10 warps: <= 168 regi
     const int lane = threadIdx.x & 31;
     const int num_m = (p.M + BM - 1) / BM;
     const int num_n = (p.N + BN - 1) / BN;
-    const int num_tiles = num_m * num_n;
+    const int num_mn = num_m * num_n;
+    const int num_tiles = num_mn * p.k_splits;
     const int num_kb = (p.K + BK - 1) / BK;
+    // K-block range of a tile: splits are the slowest tile index, so a wave works on one K range.
+    auto tile_kb = [&](int tile, int& kb0, int& kb1) {
+        const int ks = tile / num_mn;
+        kb0 = ks * p.kb_per_split;
+        kb1 = min(num_kb, kb0 + p.kb_per_split);
+    };
     auto tile_mn = [&](int tile, int& m_blk, int& n_blk) {
+        tile %= num_mn;
         if (p.n_fastest) {
             n_blk = tile % num_n;
             m_blk = tile / num_n;
@@ -175,7 +188,9 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)  // 10 warps: <= 168 regi
                 int m_blk, n_blk;
                 tile_mn(tile, m_blk, n_blk);
                 const int m0 = m_blk * BM, n0 = n_blk * BN;
-                for (int kb = 0; kb < num_kb; ++kb) {
+                int kb0, kb1;
+                tile_kb(tile, kb0, kb1);
+                for (int kb = kb0; kb < kb1; ++kb) {
                     if (!mbar_wait(&empty[stage], ph ^ 1u, abort_flag)) {
                         ok = false;
                         break;
@@ -224,7 +239,9 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)  // 10 warps: <= 168 regi
                 if (!mbar_wait(&tempty[acc], acc_ph ^ 1u, abort_flag)) break;
                 tc_fence_after();
                 const uint32_t d = tmem_base + static_cast<uint32_t>(acc * BN);
-                for (int kb = 0; kb < num_kb; ++kb) {
+                int kb0, kb1;
+                tile_kb(tile, kb0, kb1);
+                for (int kb = kb0; kb < kb1; ++kb) {
                     if (!mbar_wait(&full[stage], ph, abort_flag)) {
                         ok = false;
                         break;
@@ -240,7 +257,7 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)  // 10 warps: <= 168 regi
                                                  : make_sdesc_sw128(a_addr + k * 32);
                         const uint64_t db = B_MN ? make_sdesc_sw128_mn(b_addr + k * 2048, 8192)
                                                  : make_sdesc_sw128(b_addr + k * 32);
-                        umma_ss(d, da, db, idesc, (kb | k) != 0 ? 1u : 0u);
+                        umma_ss(d, da, db, idesc, (kb != kb0 || k != 0) ? 1u : 0u);
                     }
                     umma_commit(&empty[stage]);
                     if (++stage == kStages) {
@@ -302,7 +319,8 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)  // 10 warps: <= 168 regi
             float run_max = -INFINITY, run_sum = 0.f;
             constexpr float kLog2e = 1.4426950408889634f;
 
-            if (EPI == EPI_RESID) {
+            if (EPI == EPI_RESID || EPI == EPI_F32) {
+                const int out_row0 = row0 + (EPI == EPI_F32 ? (tile / num_mn) * p.M : 0);
 #pragma unroll 1
                 for (int c = 0; c < COLS; c += 32) {
                     uint32_t r[32];
@@ -323,7 +341,10 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)  // 10 warps: <= 168 regi
                         fence_proxy_async_shared();
                         __syncwarp();
                         if (lane == 0) {
-                            tma_reduce_add_2d(&tmC, stg, n, row0);
+                            if (EPI == EPI_RESID)
+                                tma_reduce_add_2d(&tmC, stg, n, out_row0);
+                            else
+                                tma_store_2d(&tmC, stg, n, out_row0);
                             bulk_commit();
                         }
                     }

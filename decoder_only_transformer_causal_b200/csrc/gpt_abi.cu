@@ -968,7 +968,7 @@ GPT_API int gpt_attention_backward(const void* q, const void* k, const void* v, 
 
 GPT_API size_t gpt_linear_backward_workspace_bytes(int rows, int n_out, int n_in, int dtype) {
     if (rows < 1 || n_out < 1 || n_in < 1) return 0;
-    if (dtype == GPT_DTYPE_BF16) return 256;
+    if (dtype == GPT_DTYPE_BF16) return 256 + a256(gemm_acc_split_bytes(n_out, n_in, rows));
     if (dtype != GPT_DTYPE_F32) return 0;
     const size_t r = rows, o = n_out, i = n_in;
     return 256 + a256(i * o * 4) + a256(o * r * 4) + a256(i * r * 4);
@@ -994,7 +994,7 @@ GPT_API int gpt_linear_backward(const void* dy, const void* x, const void* W, in
                                      n_out, status, s));
         // dW += dy^T x: dy stored [rows = K, n_out = M], x stored [rows = K, n_in = N] (both MN-major)
         return launch_gemm_bf16_acc(y, n_out, true, static_cast<const bf16*>(x), n_in, true, dW, n_in, n_out, n_in,
-                                    rows, status, s);
+                                    rows, status, s, reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + 256));
     }
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     const size_t r = rows, o = n_out, i = n_in;
@@ -1053,6 +1053,7 @@ ActPlan plan_acts(const gpt_config_t* c, long long B, long long T) {
 
 // Scratch of the backward pass.
 struct BwdPlan {
+    size_t splitk;
     size_t ctrl, dz, dzT, wT, gE, gT, aT, d1, dx, dpre, dqkv, dy, D, parts, sort, total;
 };
 
@@ -1080,6 +1081,14 @@ BwdPlan plan_bwd(const gpt_config_t* c, long long B, long long T) {
     const size_t csp = static_cast<size_t>(colsum_parts(static_cast<int>(N))) * 4 * C;
     P.parts = off; off += a256(std::max(lnp, csp) * 4);
     P.sort = off; off += a256(N * 8);
+    // split-K partial products of the weight-gradient GEMMs (bf16)
+    size_t sk = 0;
+    if (c->dtype == GPT_DTYPE_BF16) {
+        const int n = static_cast<int>(N), e = static_cast<int>(C);
+        sk = std::max({gemm_acc_split_bytes(3 * e, e, n), gemm_acc_split_bytes(e, e, n), gemm_acc_split_bytes(4 * e, e, n),
+                       gemm_acc_split_bytes(e, 4 * e, n), gemm_acc_split_bytes(static_cast<int>(V), e, n)});
+    }
+    P.splitk = off; off += a256(sk);
     P.total = off;
     return P;
 }
@@ -1281,7 +1290,7 @@ GPT_API int gpt_backward(const gpt_config_t* cfg, const void* weights, const int
             GPT_TRY(launch_gemm_bf16_acc(y, ldy, false, static_cast<const bf16*>(Wp), n_in, true, dIn, n_in, N, n_in,
                                          n_out, status, s));
             return launch_gemm_bf16_acc(y, ldy, true, static_cast<const bf16*>(Xp), ldx, true, dW, n_in, n_out, n_in,
-                                        N, status, s);
+                                        N, status, s, reinterpret_cast<float*>(ws + P.splitk));
         }
         GPT_TRY(launch_transpose(Wp, dt, n_in, wT, dt, n_out, n_out, n_in, s));
         GPT_TRY(gemm_acc(cfg, dYp, ldy, wT, n_out, dIn, n_in, N, n_in, n_out, status, s));

@@ -81,9 +81,13 @@ int launch_gemm_bf16(const bf16* A, long long lda, const bf16* W, long long ldw,
 
 // out[M, N] (fp32, row stride ldo) += A B^T.  A: [M, K] (a_mn false) or stored as [K, M] (a_mn);
 // W: [N, K] (b_mn false) or stored as [K, N] (b_mn); row strides lda / ldw in elements.  a_mn
-// requires b_mn.
+// requires b_mn.  split_ws (optional, 16-byte aligned, gemm_acc_split_bytes(M, N, K) bytes): with
+// a_mn, a product whose M x N tiles would leave SMs idle is split along K into partial products
+// that a second pass adds to out in a fixed order (results independent of scheduling).
 int launch_gemm_bf16_acc(const bf16* A, long long lda, bool a_mn, const bf16* W, long long ldw, bool b_mn, float* out,
-                         long long ldo, int M, int N, int K, int32_t* status, cudaStream_t s);
+                         long long ldo, int M, int N, int K, int32_t* status, cudaStream_t s,
+                         float* split_ws = nullptr);
+size_t gemm_acc_split_bytes(int M, int N, int K);
 
 // ---- tensor-core attention (attention_tc.cu); strides in elements
 struct AttnLayout {

@@ -91,28 +91,40 @@ __global__ void gelu_forward_kernel(const E* __restrict__ pre, E* __restrict__ h
 // ------------------------------------------------------------------ attention backward
 // Per (b, h) and query row i < Tp (Tp = T rounded up to 128): D[bh * Tp + i] = sum_d dO_i[d] O_i[d]
 // and L2[bh * Tp + i] = the forward's lse2_i; rows i >= T hold D = 0 and L2 = +inf (p = 0 there).
-// One warp per row.
+// hs / 8 threads per row, each with one 8-value slice of dO_i and O_i (16-byte loads when `vec`);
+// the slices meet in shuffles within the row's lane group.
 template <typename E>
 __global__ void attn_bwd_rowdot_kernel(const AttnBwdLayout<E> L, int B, int nh, int T, int Tp, int hs,
-                                       float* __restrict__ D, float* __restrict__ L2) {
+                                       float* __restrict__ D, float* __restrict__ L2, int vec) {
     griddep_launch_dependents();
     griddep_wait();
-    const long long row = static_cast<long long>(blockIdx.x) * (blockDim.x / 32) + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
-    if (row >= static_cast<long long>(B) * nh * Tp) return;
-    const int i = static_cast<int>(row % Tp);
-    const int bh = static_cast<int>(row / Tp), b = bh / nh, h = bh % nh;
-    if (i >= T) {
-        if (lane == 0) D[row] = 0.f, L2[row] = INFINITY;
-        return;
-    }
-    const E* o = L.o + b * L.o_sb + h * L.o_sh + static_cast<long long>(i) * L.o_st;
-    const E* g = L.dout + b * L.o_sb + h * L.o_sh + static_cast<long long>(i) * L.o_st;
+    const int G = hs / 8;  // 4 or 8: divides 32, so a row's lanes sit in one warp
+    const long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const long long row = t / G;
+    const int part = static_cast<int>(t % G);
+    const bool valid = row < static_cast<long long>(B) * nh * Tp;
+    const int i = valid ? static_cast<int>(row % Tp) : 0;
+    const int bh = valid ? static_cast<int>(row / Tp) : 0, b = bh / nh, h = bh % nh;
     float s = 0.f;
-    for (int d = lane; d < hs; d += 32) s += ldf(o + d) * ldf(g + d);
+    if (valid && i < T) {
+        const E* o = L.o + b * L.o_sb + h * L.o_sh + static_cast<long long>(i) * L.o_st + part * 8;
+        const E* g = L.dout + b * L.o_sb + h * L.o_sh + static_cast<long long>(i) * L.o_st + part * 8;
+        float ov[8], gv[8];
+        if (vec) {
+            ld8(o, ov);
+            ld8(g, gv);
+        } else {
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-    if (lane == 0) D[row] = s, L2[row] = __ldcg(L.lse + static_cast<long long>(bh) * T + i);
+            for (int e = 0; e < 8; ++e) ov[e] = ldf(o + e), gv[e] = ldf(g + e);
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) s = fmaf(ov[e], gv[e], s);
+    }
+    for (int off = G / 2; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+    if (valid && part == 0) {
+        D[row] = i < T ? s : 0.f;
+        L2[row] = i < T ? __ldcg(L.lse + static_cast<long long>(bh) * T + i) : INFINITY;
+    }
 }
 
 constexpr int kBwdRows = 64;  // rows per CTA and per staged tile
@@ -270,9 +282,11 @@ template <typename E, int HS>
 int attn_bwd_typed(const AttnBwdLayout<E>& L, int B, int nh, int T, float* D, float* L2, int32_t* status,
                    cudaStream_t s) {
     const int Tp = (T + 127) / 128 * 128;
-    const long long rows = static_cast<long long>(B) * nh * Tp;
-    int rc = launch_overlapped(attn_bwd_rowdot_kernel<E>, dim3(static_cast<unsigned>((rows + 7) / 8)), dim3(256), 0, s,
-                               L, B, nh, T, Tp, HS, D, L2);
+    const long long threads = static_cast<long long>(B) * nh * Tp * (HS / 8);
+    const int vec = ((reinterpret_cast<uintptr_t>(L.o) | reinterpret_cast<uintptr_t>(L.dout)) & 15) == 0 &&
+                    ((L.o_sb | L.o_sh | L.o_st) * static_cast<long long>(sizeof(E))) % 16 == 0;
+    int rc = launch_overlapped(attn_bwd_rowdot_kernel<E>, dim3(static_cast<unsigned>((threads + 255) / 256)), dim3(256),
+                               0, s, L, B, nh, T, Tp, HS, D, L2, vec);
     if (rc) return rc;
     if constexpr (sizeof(E) == 2 && HS == 64) {
         // Tensor-core kernels whenever the operands can be described by TMA maps (16-byte

@@ -227,7 +227,7 @@ def test_backward_pieces_host_validation():
     assert Lb.gpt_cross_entropy_backward(FAKE, FAKE, FAKE, 4, 0, bf, FAKE, None, None) == native.GPT_ERR_BAD_SHAPE
     assert Lb.gpt_cross_entropy_backward(FAKE, FAKE, FAKE, 4, 10, 7, FAKE, None, None) == native.GPT_ERR_BAD_SHAPE
     ws = Lb.gpt_layernorm_backward_workspace_bytes(100, 768)
-    assert ws >= ((100 + 63) // 64) * 2 * 768 * 4                                   # one partial per 64 rows
+    assert ws >= ((100 + 31) // 32) * 2 * 768 * 4                                   # one partial per 32 rows
     assert Lb.gpt_layernorm_backward(FAKE, FAKE, FAKE, 100, 768, bf, FAKE, 0, FAKE, None, 0, FAKE, ws - 1, None) \
         == native.GPT_ERR_WS_TOO_SMALL
     assert Lb.gpt_layernorm_backward(FAKE, FAKE, FAKE, 100, 5000, bf, FAKE, 0, FAKE, None, 0, FAKE, 1 << 40, None) \
