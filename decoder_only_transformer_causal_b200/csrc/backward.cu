@@ -143,7 +143,8 @@ __global__ void __launch_bounds__(kBwdWarps * 32)
 template <typename Tw>
 __global__ void __launch_bounds__(kBwdWarps * 32)
     layernorm_backward_kernel(const float* __restrict__ dy, const float* __restrict__ x, const Tw* __restrict__ w,
-                              float* __restrict__ dx, int accumulate, float* __restrict__ part, int rows, int C) {
+                              float* __restrict__ dx, int accumulate, float* __restrict__ part, int rows, int C,
+                              bf16* __restrict__ dx16) {
     griddep_launch_dependents();
     griddep_wait();
     extern __shared__ float sm[];  // [kBwdWarps][2][C] per-warp column sums
@@ -179,7 +180,9 @@ __global__ void __launch_bounds__(kBwdWarps * 32)
         for (int c = lane; c < C; c += 32) {
             const float xh = (__ldcg(xr + c) - mean) * rstd;
             const float v = rstd * (__ldcg(dyr + c) * ld1(w + c) - ma - xh * mb);
-            dxr[c] = accumulate ? __ldcg(dxr + c) + v : v;
+            const float o = accumulate ? __ldcg(dxr + c) + v : v;
+            dxr[c] = o;
+            if (dx16) dx16[static_cast<long long>(r) * C + c] = __float2bfloat16_rn(o);
         }
     }
     __syncthreads();
@@ -221,7 +224,8 @@ GPT_DEVINL void ln_row_load(LnRow<VEC>& R, const float* x, const float* dy, cons
 template <typename Tw, int VEC>
 __global__ void __launch_bounds__(kBwdWarps * 32)
     layernorm_backward_reg_kernel(const float* __restrict__ dy, const float* __restrict__ x, const Tw* __restrict__ w,
-                                  float* __restrict__ dx, int accumulate, float* __restrict__ part, int rows, int C) {
+                                  float* __restrict__ dx, int accumulate, float* __restrict__ part, int rows, int C,
+                                  bf16* __restrict__ dx16) {
     griddep_launch_dependents();
     griddep_wait();
     extern __shared__ float sm[];  // [kBwdWarps][2][C] per-warp column sums
@@ -305,6 +309,9 @@ __global__ void __launch_bounds__(kBwdWarps * 32)
                                              cur.old[j].z + rstd * (gv[j].z * wv[j].z - ma - xv[j].z * mb),
                                              cur.old[j].w + rstd * (gv[j].w * wv[j].w - ma - xv[j].w * mb));
                 *reinterpret_cast<float4*>(dxr + c) = o;
+                if (dx16)
+                    *reinterpret_cast<uint2*>(dx16 + static_cast<long long>(r) * C + c) =
+                        make_uint2(pack_bf16x2(o.x, o.y), pack_bf16x2(o.z, o.w));
             }
         }
         if constexpr (kPipe) cur = nxt;
@@ -511,44 +518,43 @@ int layernorm_backward_parts(int rows, int C) {
 
 namespace {
 template <typename Tw, int VEC = 1>
-int launch_ln_bwd_reg(const float* dy, const float* x, const void* w, float* dx, int accumulate, float* part, int rows,
+int launch_ln_bwd_reg(const float* dy, const float* x, const void* w, float* dx, bf16* dx16, int accumulate, float* part, int rows,
                       int C, size_t smem, cudaStream_t s) {
     if constexpr (VEC < 16) {
-        if (C > 128 * VEC) return launch_ln_bwd_reg<Tw, VEC + 1>(dy, x, w, dx, accumulate, part, rows, C, smem, s);
+        if (C > 128 * VEC) return launch_ln_bwd_reg<Tw, VEC + 1>(dy, x, w, dx, dx16, accumulate, part, rows, C, smem, s);
     }
     static size_t opted[kMaxDevices] = {};
     const int rc = opt_in_smem(reinterpret_cast<const void*>(layernorm_backward_reg_kernel<Tw, VEC>), smem, opted);
     if (rc) return rc;
     return launch_overlapped(layernorm_backward_reg_kernel<Tw, VEC>, dim3(layernorm_backward_parts(rows, C)),
                              dim3(kBwdWarps * 32), smem, s, dy, x, static_cast<const Tw*>(w), dx, accumulate, part,
-                             rows, C);
+                             rows, C, dx16);
 }
 }  // namespace
 
 int launch_layernorm_backward(const float* dy, const float* x, const void* w, int dtype, float* dx, int accumulate,
-                              float* dw, float* db, int accumulate_wb, float* part, int rows, int C,
-                              cudaStream_t s) {
+                              float* dw, float* db, int accumulate_wb, float* part, int rows, int C, cudaStream_t s,
+                              bf16* dx16) {
     const int n_part = layernorm_backward_parts(rows, C);
     const size_t smem = static_cast<size_t>(kBwdWarps) * 2 * C * sizeof(float);
     int rc;
     if (C <= 2048 && C % 4 == 0) {
-        rc = dtype == GPT_DTYPE_BF16 ? launch_ln_bwd_reg<bf16>(dy, x, w, dx, accumulate, part, rows, C, smem, s)
-                                     : launch_ln_bwd_reg<float>(dy, x, w, dx, accumulate, part, rows, C, smem, s);
+        rc = dtype == GPT_DTYPE_BF16 ? launch_ln_bwd_reg<bf16>(dy, x, w, dx, dx16, accumulate, part, rows, C, smem, s)
+                                     : launch_ln_bwd_reg<float>(dy, x, w, dx, dx16, accumulate, part, rows, C, smem, s);
     } else if (dtype == GPT_DTYPE_BF16) {
         static size_t opted[kMaxDevices] = {};
         rc = opt_in_smem(reinterpret_cast<const void*>(layernorm_backward_kernel<bf16>), smem, opted);
         if (!rc)
             rc = launch_overlapped(layernorm_backward_kernel<bf16>, dim3(n_part), dim3(kBwdWarps * 32), smem, s, dy,
-                                   x, static_cast<const bf16*>(w), dx, accumulate, part, rows, C);
+                                   x, static_cast<const bf16*>(w), dx, accumulate, part, rows, C, dx16);
     } else {
         static size_t opted[kMaxDevices] = {};
         rc = opt_in_smem(reinterpret_cast<const void*>(layernorm_backward_kernel<float>), smem, opted);
         if (!rc)
             rc = launch_overlapped(layernorm_backward_kernel<float>, dim3(n_part), dim3(kBwdWarps * 32), smem, s, dy,
-                                   x, static_cast<const float*>(w), dx, accumulate, part, rows, C);
+                                   x, static_cast<const float*>(w), dx, accumulate, part, rows, C, dx16);
     }
     if (rc) return rc;
-    const dim3 g((C + 255) / 256), b(256);
     const dim3 gp((C + 31) / 32), bp(32, 8);
     rc = launch_overlapped(colsum_parts_kernel, gp, bp, 0, s, static_cast<const float*>(part), 2LL * C, n_part, C, dw,
                            accumulate_wb);

@@ -116,12 +116,11 @@ int launch_gemm_bf16(const bf16* A, long long lda, const bf16* W, long long ldw,
     }
 }
 
-int launch_gemm_bf16_acc(const bf16* A, long long lda, bool a_mn, const bf16* W, long long ldw, bool b_mn, float* out,
-                         long long ldo, int M, int N, int K, int32_t* status, cudaStream_t s, float* split_ws) {
+int launch_gemm_bf16_bwd(const bf16* A, long long lda, bool a_mn, const bf16* W, long long ldw, bool b_mn, void* out,
+                         long long ldo, int M, int N, int K, int mode, const bf16* aux, long long ld_aux, int gelu,
+                         int32_t* status, cudaStream_t s, float* split_ws) {
     if (M == 0 || N == 0) return GPT_OK;
-    if (a_mn == false && b_mn == false)
-        return launch_gemm_bf16(A, lda, W, ldw, nullptr, out, ldo, M, N, K, GPT_EPI_RESID, 0, nullptr, status, s);
-    if (!b_mn) return GPT_ERR_UNSUPPORTED;  // MN-major A is only paired with MN-major B
+    if (!b_mn || (a_mn && mode != GEMM_BWD_ACC_F32)) return GPT_ERR_UNSUPPORTED;
     CUtensorMap ta, tb, tc;
     int rc = a_mn ? make_tmap_bf16_2d(&ta, A, static_cast<uint64_t>(M), static_cast<uint64_t>(K),
                                       static_cast<uint64_t>(lda) * 2, 64, gemm::BK)
@@ -137,33 +136,59 @@ int launch_gemm_bf16_acc(const bf16* A, long long lda, bool a_mn, const bf16* W,
     p.K = K;
     p.n_fastest = static_cast<long long>(M) >= static_cast<long long>(N) ? 1 : 0;
     p.status = status;
-    int S = 1, per = (K + gemm::BK - 1) / gemm::BK;
-    if (a_mn && split_ws) split_plan(M, N, K, &S, &per);
-    p.k_splits = S;
-    p.kb_per_split = per;
-    if (S > 1) {
-        // Deterministic split-K: each K range stores its partial product into its own slice of
-        // split_ws, then one pass adds the slices to out in order.
-        if (((reinterpret_cast<uintptr_t>(out) | reinterpret_cast<uintptr_t>(split_ws)) & 15) || (ldo % 4))
-            return GPT_ERR_BAD_ALIGN;
-        rc = make_tmap_2d_sw64(&tc, split_ws, true, static_cast<uint64_t>(N), static_cast<uint64_t>(S) * M,
-                               static_cast<uint64_t>(N) * 4, 16, 32);
-        if (rc) return rc;
-        p.out = split_ws;
-        p.ldo = N;
-        rc = launch_one<gemm::EPI_F32, 0, 1, 1>(ta, tb, tc, p, s);
-        if (rc) return rc;
-        const long long n4 = static_cast<long long>(M) * (N / 4);
-        return launch_overlapped(splitk_reduce_kernel, dim3(static_cast<unsigned>((n4 + 255) / 256)), dim3(256), 0, s,
-                                 static_cast<const float*>(split_ws), S, M, N, out, ldo);
-    }
-    rc = make_tmap_2d_sw64(&tc, out, true, static_cast<uint64_t>(N), static_cast<uint64_t>(M),
-                           static_cast<uint64_t>(ldo) * 4, 16, 32);
-    if (rc) return rc;
+    p.k_splits = 1;
+    p.kb_per_split = (K + gemm::BK - 1) / gemm::BK;
     p.out = out;
     p.ldo = ldo;
-    return a_mn ? launch_one<gemm::EPI_RESID, 0, 1, 1>(ta, tb, tc, p, s)
-                : launch_one<gemm::EPI_RESID, 0, 0, 1>(ta, tb, tc, p, s);
+    const bool f32 = mode == GEMM_BWD_ACC_F32 || mode == GEMM_BWD_STORE_F32;
+    if (mode == GEMM_BWD_ACC_F32 && a_mn && split_ws) {
+        int S, per;
+        split_plan(M, N, K, &S, &per);
+        if (S > 1) {
+            // Deterministic split-K: each K range stores its partial product into its own slice of
+            // split_ws, then one pass adds the slices to out in order.
+            if (((reinterpret_cast<uintptr_t>(out) | reinterpret_cast<uintptr_t>(split_ws)) & 15) || (ldo % 4))
+                return GPT_ERR_BAD_ALIGN;
+            rc = make_tmap_2d_sw64(&tc, split_ws, true, static_cast<uint64_t>(N), static_cast<uint64_t>(S) * M,
+                                   static_cast<uint64_t>(N) * 4, 16, 32);
+            if (rc) return rc;
+            p.out = split_ws;
+            p.ldo = N;
+            p.k_splits = S;
+            p.kb_per_split = per;
+            rc = launch_one<gemm::EPI_F32, 0, 1, 1>(ta, tb, tc, p, s);
+            if (rc) return rc;
+            const long long n4 = static_cast<long long>(M) * (N / 4);
+            return launch_overlapped(splitk_reduce_kernel, dim3(static_cast<unsigned>((n4 + 255) / 256)), dim3(256), 0,
+                                     s, static_cast<const float*>(split_ws), S, M, N, static_cast<float*>(out), ldo);
+        }
+    }
+    rc = make_tmap_2d_sw64(&tc, out, f32, static_cast<uint64_t>(N), static_cast<uint64_t>(M),
+                           static_cast<uint64_t>(ldo) * (f32 ? 4 : 2), f32 ? 16 : 32, 32);
+    if (rc) return rc;
+    switch (mode) {
+        case GEMM_BWD_ACC_F32:
+            return a_mn ? launch_one<gemm::EPI_RESID, 0, 1, 1>(ta, tb, tc, p, s)
+                        : launch_one<gemm::EPI_RESID, 0, 0, 1>(ta, tb, tc, p, s);
+        case GEMM_BWD_STORE_F32: return launch_one<gemm::EPI_F32, 0, 0, 1>(ta, tb, tc, p, s);
+        case GEMM_BWD_STORE_BF16: return launch_one<gemm::EPI_STORE, 0, 0, 1>(ta, tb, tc, p, s);
+        case GEMM_BWD_DGELU_BF16:
+            if (!aux) return GPT_ERR_NULL;
+            if ((reinterpret_cast<uintptr_t>(aux) & 15) || (ld_aux % 8)) return GPT_ERR_BAD_ALIGN;
+            p.aux = aux;
+            p.ld_aux = ld_aux;
+            return gelu == GPT_GELU_TANH ? launch_one<gemm::EPI_DGELU, 1, 0, 1>(ta, tb, tc, p, s)
+                                         : launch_one<gemm::EPI_DGELU, 0, 0, 1>(ta, tb, tc, p, s);
+        default: return GPT_ERR_UNSUPPORTED;
+    }
+}
+
+int launch_gemm_bf16_acc(const bf16* A, long long lda, bool a_mn, const bf16* W, long long ldw, bool b_mn, float* out,
+                         long long ldo, int M, int N, int K, int32_t* status, cudaStream_t s, float* split_ws) {
+    if (!a_mn && !b_mn)
+        return launch_gemm_bf16(A, lda, W, ldw, nullptr, out, ldo, M, N, K, GPT_EPI_RESID, 0, nullptr, status, s);
+    return launch_gemm_bf16_bwd(A, lda, a_mn, W, ldw, b_mn, out, ldo, M, N, K, GEMM_BWD_ACC_F32, nullptr, 0, 0, status,
+                                s, split_ws);
 }
 
 }  // namespace gpt

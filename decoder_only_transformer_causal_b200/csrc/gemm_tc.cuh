@@ -35,8 +35,11 @@ constexpr int BK = 64;  // one 128-byte swizzle row of bf16
 constexpr int kStages = 4;
 constexpr int NEPI = 8;  // epilogue warps: two per TMEM lane quarter, each half of BN
 
-// EPI_F32: out_fp32 = acc, plain store (the partial products of a split-K launch).
-enum Epi { EPI_STORE = 0, EPI_GELU = 1, EPI_RESID = 2, EPI_CE = 3, EPI_F32 = 4 };
+// EPI_F32: out_fp32 = acc, plain store (a backward product, or the partial products of a split-K
+//          launch).
+// EPI_DGELU: out_bf16 = acc * gelu'(aux), aux the bf16 pre-activation [M, ld_aux] (the MLP's
+//          backward through GELU, fused into the product that yields d loss / d gelu output).
+enum Epi { EPI_STORE = 0, EPI_GELU = 1, EPI_RESID = 2, EPI_CE = 3, EPI_F32 = 4, EPI_DGELU = 5 };
 
 struct Params {
     int M, N, K;
@@ -53,6 +56,8 @@ struct Params {
     // split s stores its partial product at rows [s * M, s * M + M) of out (M % 32 == 0).
     int k_splits;
     int kb_per_split;
+    const bf16* aux;  // EPI_DGELU: [M, ld_aux]
+    long long ld_aux;
 };
 
 template <int BN>
@@ -82,6 +87,32 @@ GPT_DEVINL float rcp_approx(float x) {
     float y;
     asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// d gelu(x) / dx with the same building blocks as gelu_f:
+//  erf form:  Phi(x) + x phi(x), phi(x) = exp(-x^2 / 2) / sqrt(2 pi) (the exponential the erf
+//             formula already takes);
+//  tanh form: 0.5 (1 + th) + 0.5 x (1 - th^2) sqrt(2/pi) (1 + 3 * 0.044715 x^2), th = tanh(u),
+//             tanh(u) = 1 - 2 / (1 + exp(2u)).
+template <int TANH>
+GPT_DEVINL float gelu_grad_f(float x) {
+    constexpr float kLog2e = 1.4426950408889634f;
+    if (TANH) {
+        const float c = 0.7978845608028654f;
+        const float u = c * x * fmaf(0.044715f * x, x, 1.0f);
+        const float th = 1.0f - 2.0f * rcp_approx(1.0f + exp2_approx(2.0f * u * kLog2e));
+        return 0.5f * (1.0f + th) + 0.5f * x * (1.0f - th * th) * c * fmaf(3.0f * 0.044715f * x, x, 1.0f);
+    }
+    const float z = fabsf(x) * 0.7071067811865476f;
+    const float t = rcp_approx(fmaf(0.3275911f, z, 1.0f));
+    float q = fmaf(t, 1.061405429f, -1.453152027f);
+    q = fmaf(t, q, 1.421413741f);
+    q = fmaf(t, q, -0.284496736f);
+    q = fmaf(t, q, 0.254829592f);
+    q *= t;
+    const float e = exp2_approx(-z * z * kLog2e);  // exp(-x^2 / 2)
+    const float erf_abs = fmaf(-q, e, 1.0f);
+    return 0.5f * (1.0f + copysignf(erf_abs, x)) + x * 0.3989422804014327f * e;
 }
 
 template <int TANH>
@@ -376,6 +407,26 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)  // 10 warps: <= 168 regi
                         if (EPI == EPI_GELU) {
 #pragma unroll
                             for (int j = 0; j < 32; ++j) v[j] = gelu_f<GELU_TANH>(v[j]);
+                        }
+                        if (EPI == EPI_DGELU && row_ok) {
+                            // this row's 32 pre-activations (64 bytes) of the chunk
+                            const bf16* ap = p.aux + static_cast<long long>(row) * p.ld_aux + n;
+                            float z[32];
+                            if (full_chunk) {
+#pragma unroll
+                                for (int q = 0; q < 4; ++q) {
+                                    float f[8];
+                                    ld8(ap + 8 * q, f);
+#pragma unroll
+                                    for (int e = 0; e < 8; ++e) z[8 * q + e] = f[e];
+                                }
+                            } else {
+#pragma unroll
+                                for (int j = 0; j < 32; ++j)
+                                    z[j] = n + j < p.N ? __bfloat162float(ap[j]) : 0.f;
+                            }
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) v[j] *= gelu_grad_f<GELU_TANH>(z[j]);
                         }
                         if (EPI == EPI_CE) {
                             float cmax = -INFINITY;

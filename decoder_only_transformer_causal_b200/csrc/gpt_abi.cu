@@ -984,18 +984,18 @@ GPT_API int gpt_linear_backward(const void* dy, const void* x, const void* W, in
     if (workspace_bytes < gpt_linear_backward_workspace_bytes(rows, n_out, n_in, dtype)) return GPT_ERR_WS_TOO_SMALL;
     if (!aligned(workspace, 256) || !aligned(dx, 16) || !aligned(dW, 16)) return GPT_ERR_BAD_ALIGN;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    GPT_TRY(cuda_status(cudaMemsetAsync(dx, 0, static_cast<size_t>(rows) * n_in * 4, s)));
     if (dtype == GPT_DTYPE_BF16) {
         if ((n_out % 8) || (n_in % 8)) return GPT_ERR_UNSUPPORTED;
         if (!aligned(dy, 16) || !aligned(x, 16) || !aligned(W, 16)) return GPT_ERR_BAD_ALIGN;
         const bf16* y = static_cast<const bf16*>(dy);
-        // dx = dy W: dy K-major, W stored [n_out = K, n_in = N] (MN-major B)
-        GPT_TRY(launch_gemm_bf16_acc(y, n_out, false, static_cast<const bf16*>(W), n_in, true, dx, n_in, rows, n_in,
-                                     n_out, status, s));
+        // dx = dy W: dy K-major, W stored [n_out = K, n_in = N] (MN-major B), stored (not added)
+        GPT_TRY(launch_gemm_bf16_bwd(y, n_out, false, static_cast<const bf16*>(W), n_in, true, dx, n_in, rows, n_in,
+                                     n_out, GEMM_BWD_STORE_F32, nullptr, 0, 0, status, s));
         // dW += dy^T x: dy stored [rows = K, n_out = M], x stored [rows = K, n_in = N] (both MN-major)
         return launch_gemm_bf16_acc(y, n_out, true, static_cast<const bf16*>(x), n_in, true, dW, n_in, n_out, n_in,
                                     rows, status, s, reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + 256));
     }
+    GPT_TRY(cuda_status(cudaMemsetAsync(dx, 0, static_cast<size_t>(rows) * n_in * 4, s)));
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     const size_t r = rows, o = n_out, i = n_in;
     float* wT = reinterpret_cast<float*>(ws + 256);
@@ -1278,51 +1278,69 @@ GPT_API int gpt_backward(const gpt_config_t* cfg, const void* weights, const int
     const int F32 = GPT_DTYPE_F32;
     const size_t nc = static_cast<size_t>(N) * C;
 
-    // Linear backward: dIn (fp32 [N, n_in], zeroed here) = dY W and dW (fp32) += dY^T X, for dY
-    // [N, n_out] (row stride ldy), X [N, n_in] (row stride ldx) and W [n_out, n_in] in the config
-    // dtype.  bf16 hands the GEMM the stored dY, X and W as MN-major operands where the product needs
-    // their transposes; fp32 forms the transposes in scratch first (yT: room for dY^T).
+    // Linear backward: the input gradient dIn = dY W and dW (fp32) += dY^T X, for dY [N, n_out] (row
+    // stride ldy), X [N, n_in] (row stride ldx) and W [n_out, n_in] in the config dtype.  dIn is
+    // written as `mode` says: GEMM_BWD_STORE_F32 (fp32 [N, n_in]), GEMM_BWD_STORE_BF16, or
+    // GEMM_BWD_DGELU_BF16 (bf16 (dY W) * gelu'(aux), aux the [N, n_in] pre-activation).  bf16 hands
+    // the GEMM the stored dY, X and W as MN-major operands where the product needs their transposes;
+    // fp32 (GEMM_BWD_STORE_F32 only) forms the transposes in scratch first (yT: room for dY^T).
     auto linear_bwd = [&](const void* dYp, long long ldy, const void* Xp, long long ldx, const void* Wp, int n_out,
-                          int n_in, float* dIn, float* dW, void* yT) -> int {
-        GPT_TRY(cuda_status(cudaMemsetAsync(dIn, 0, static_cast<size_t>(N) * n_in * 4, s)));
+                          int n_in, void* dIn, int mode, const void* aux, float* dW, void* yT) -> int {
         if (bf) {
             const bf16* y = static_cast<const bf16*>(dYp);
-            GPT_TRY(launch_gemm_bf16_acc(y, ldy, false, static_cast<const bf16*>(Wp), n_in, true, dIn, n_in, N, n_in,
-                                         n_out, status, s));
-            return launch_gemm_bf16_acc(y, ldy, true, static_cast<const bf16*>(Xp), ldx, true, dW, n_in, n_out, n_in,
-                                        N, status, s, reinterpret_cast<float*>(ws + P.splitk));
+            GPT_TRY(launch_gemm_bf16_bwd(y, ldy, false, static_cast<const bf16*>(Wp), n_in, true, dIn, n_in, N, n_in,
+                                         n_out, mode, static_cast<const bf16*>(aux), n_in, cfg->gelu, status, s));
+            return launch_gemm_bf16_bwd(y, ldy, true, static_cast<const bf16*>(Xp), ldx, true, dW, n_in, n_out, n_in, N,
+                                        GEMM_BWD_ACC_F32, nullptr, 0, 0, status, s,
+                                        reinterpret_cast<float*>(ws + P.splitk));
         }
+        if (mode != GEMM_BWD_STORE_F32) return GPT_ERR_UNSUPPORTED;
+        float* out = static_cast<float*>(dIn);
+        GPT_TRY(cuda_status(cudaMemsetAsync(out, 0, static_cast<size_t>(N) * n_in * 4, s)));
         GPT_TRY(launch_transpose(Wp, dt, n_in, wT, dt, n_out, n_out, n_in, s));
-        GPT_TRY(gemm_acc(cfg, dYp, ldy, wT, n_out, dIn, n_in, N, n_in, n_out, status, s));
+        GPT_TRY(gemm_acc(cfg, dYp, ldy, wT, n_out, out, n_in, N, n_in, n_out, status, s));
         GPT_TRY(launch_transpose(dYp, dt, ldy, yT, dt, N, N, n_out, s));
         GPT_TRY(launch_transpose(Xp, dt, ldx, aT, dt, N, N, n_in, s));
         return gemm_acc(cfg, yT, N, aT, N, dW, n_in, n_out, n_in, N, status, s);
     };
+    // The residual gradient dx stays fp32; the products read it as gx: the bf16 copy gE that each
+    // LayerNorm backward writes next to dx (bf16), or dx itself (fp32).
+    const void* gx = bf ? static_cast<const void*>(gE) : static_cast<const void*>(dx);
+    bf16* dx16 = bf ? static_cast<bf16*>(gE) : nullptr;
+    const int F32_OUT = GEMM_BWD_STORE_F32;
 
     GPT_TRY(cuda_status(cudaMemsetAsync(status, 0, sizeof(int32_t), s)));
     // d loss / d logits, then the tied head: du_f = dz wte, dwte += dz^T u_f
     if (!(loss_scale > 0.f) || !isfinite(loss_scale)) return GPT_ERR_BAD_SHAPE;
     GPT_TRY(launch_ce_backward(ab + A.logits, dt, targets, reinterpret_cast<const double*>(ab + A.sum_count), dz, N, V,
                                status, s, loss_scale));
-    GPT_TRY(linear_bwd(dz, V, ab + A.u_f, C, W.wte(), V, C, d1, G(0), dzT));
+    GPT_TRY(linear_bwd(dz, V, ab + A.u_f, C, W.wte(), V, C, d1, F32_OUT, nullptr, G(0), dzT));
     GPT_TRY(launch_layernorm_backward(d1, reinterpret_cast<const float*>(ab + A.x_f), W.lnf_w(), dt, dx, 0, G(count - 2),
-                                      cfg->bias ? G(count - 1) : nullptr, 1, parts, N, C, s));
+                                      cfg->bias ? G(count - 1) : nullptr, 1, parts, N, C, s, dx16));
     for (int l = cfg->n_layer - 1; l >= 0; --l) {
         const uint8_t* L = ab + A.layer * l;
-        // mlp c_proj: dh = dx W_fc2 (into d1 [N, 4C]); dW_fc2 += dx^T h; db_fc2 += sum dx
-        GPT_TRY(launch_convert(dx, F32, gE, dt, static_cast<long long>(nc), s));
-        GPT_TRY(linear_bwd(gE, C, L + A.h, 4LL * C, W.layer(l, W_FC2_W), C, 4 * C, d1, GL(l, W_FC2_W), gT));
+        // mlp c_proj, then GELU: dpre = (dx W_fc2) * gelu'(pre) (bf16: one fused product; fp32: dh
+        // into d1, then the GELU backward); dW_fc2 += dx^T h; db_fc2 += sum dx
+        if (bf) {
+            GPT_TRY(linear_bwd(gx, C, L + A.h, 4LL * C, W.layer(l, W_FC2_W), C, 4 * C, dpre, GEMM_BWD_DGELU_BF16,
+                               L + A.pre, GL(l, W_FC2_W), gT));
+        } else {
+            GPT_TRY(linear_bwd(gx, C, L + A.h, 4LL * C, W.layer(l, W_FC2_W), C, 4 * C, d1, F32_OUT, nullptr,
+                               GL(l, W_FC2_W), gT));
+            GPT_TRY(launch_gelu_backward(d1, L + A.pre, dt, dpre, static_cast<long long>(nc) * 4,
+                                         cfg->gelu == GPT_GELU_TANH, s));
+        }
         if (cfg->bias) GPT_TRY(launch_colsum(dx, F32, N, C, GL(l, W_FC2_B), 1, parts, s));
-        // GELU, then c_fc: du2 = dpre W_fc (into d1 [N, C]); dW_fc += dpre^T u2; db_fc += sum dpre
-        GPT_TRY(launch_gelu_backward(d1, L + A.pre, dt, dpre, static_cast<long long>(nc) * 4, cfg->gelu == GPT_GELU_TANH, s));
-        GPT_TRY(linear_bwd(dpre, 4LL * C, L + A.u2, C, W.layer(l, W_FC_W), 4 * C, C, d1, GL(l, W_FC_W), gT));
+        // c_fc: du2 = dpre W_fc (into d1 [N, C]); dW_fc += dpre^T u2; db_fc += sum dpre
+        GPT_TRY(linear_bwd(dpre, 4LL * C, L + A.u2, C, W.layer(l, W_FC_W), 4 * C, C, d1, F32_OUT, nullptr,
+                           GL(l, W_FC_W), gT));
         if (cfg->bias) GPT_TRY(launch_colsum(dpre, dt, N, 4 * C, GL(l, W_FC_B), 1, parts, s));
         GPT_TRY(launch_layernorm_backward(d1, reinterpret_cast<const float*>(L + A.x_mid), W.layer(l, W_LN2_W), dt, dx, 1,
-                                          GL(l, W_LN2_W), cfg->bias ? GL(l, W_LN2_B) : nullptr, 1, parts, N, C, s));
-        // attn c_proj: dy = dx W_proj; dW_proj += dx^T y; db_proj += sum dx
-        GPT_TRY(launch_convert(dx, F32, gE, dt, static_cast<long long>(nc), s));
-        GPT_TRY(linear_bwd(gE, C, L + A.y, C, W.layer(l, W_PROJ_W), C, C, d1, GL(l, W_PROJ_W), gT));
-        GPT_TRY(launch_convert(d1, F32, dy, dt, static_cast<long long>(nc), s));
+                                          GL(l, W_LN2_W), cfg->bias ? GL(l, W_LN2_B) : nullptr, 1, parts, N, C, s,
+                                          dx16));
+        // attn c_proj: dy = dx W_proj (straight into the config dtype); dW_proj += dx^T y; db_proj += sum dx
+        GPT_TRY(linear_bwd(gx, C, L + A.y, C, W.layer(l, W_PROJ_W), C, C, dy, bf ? GEMM_BWD_STORE_BF16 : F32_OUT,
+                           nullptr, GL(l, W_PROJ_W), gT));
         if (cfg->bias) GPT_TRY(launch_colsum(dx, F32, N, C, GL(l, W_PROJ_B), 1, parts, s));
         // attention backward into dqkv (the qkv layout)
         const float* lse = reinterpret_cast<const float*>(L + A.lse);
@@ -1343,10 +1361,12 @@ GPT_API int gpt_backward(const gpt_config_t* cfg, const void* weights, const int
             GPT_TRY(launch_attention_backward(nullptr, &AL, B, nh, T, hs, D, status, s));
         }
         // c_attn: du1 = dqkv W_attn (into d1 [N, C]); dW_attn += dqkv^T u1; db_attn += sum dqkv
-        GPT_TRY(linear_bwd(dqkv, 3LL * C, L + A.u1, C, W.layer(l, W_ATTN_W), 3 * C, C, d1, GL(l, W_ATTN_W), gT));
+        GPT_TRY(linear_bwd(dqkv, 3LL * C, L + A.u1, C, W.layer(l, W_ATTN_W), 3 * C, C, d1, F32_OUT, nullptr,
+                           GL(l, W_ATTN_W), gT));
         if (cfg->bias) GPT_TRY(launch_colsum(dqkv, dt, N, 3 * C, GL(l, W_ATTN_B), 1, parts, s));
         GPT_TRY(launch_layernorm_backward(d1, reinterpret_cast<const float*>(L + A.x_in), W.layer(l, W_LN1_W), dt, dx, 1,
-                                          GL(l, W_LN1_W), cfg->bias ? GL(l, W_LN1_B) : nullptr, 1, parts, N, C, s));
+                                          GL(l, W_LN1_W), cfg->bias ? GL(l, W_LN1_B) : nullptr, 1, parts, N, C, s,
+                                          dx16));
     }
     GPT_TRY(launch_embed_backward(idx, dx, B, T, C, V, G(0), G(1), reinterpret_cast<unsigned long long*>(ws + P.sort),
                                   status, s));

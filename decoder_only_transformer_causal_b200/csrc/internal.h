@@ -88,6 +88,15 @@ int launch_gemm_bf16_acc(const bf16* A, long long lda, bool a_mn, const bf16* W,
                          long long ldo, int M, int N, int K, int32_t* status, cudaStream_t s,
                          float* split_ws = nullptr);
 size_t gemm_acc_split_bytes(int M, int N, int K);
+// Products of the backward with W stored [K, N] (b_mn, required):
+//   GEMM_BWD_ACC_F32     out fp32 += A B^T (a_mn allowed; split-K as launch_gemm_bf16_acc)
+//   GEMM_BWD_STORE_F32   out fp32  = A B^T
+//   GEMM_BWD_STORE_BF16  out bf16  = A B^T
+//   GEMM_BWD_DGELU_BF16  out bf16  = (A B^T) * gelu'(aux), aux bf16 [M, ld_aux] (gelu = GPT_GELU_*)
+enum { GEMM_BWD_ACC_F32 = 0, GEMM_BWD_STORE_F32 = 1, GEMM_BWD_STORE_BF16 = 2, GEMM_BWD_DGELU_BF16 = 3 };
+int launch_gemm_bf16_bwd(const bf16* A, long long lda, bool a_mn, const bf16* W, long long ldw, bool b_mn, void* out,
+                         long long ldo, int M, int N, int K, int mode, const bf16* aux, long long ld_aux, int gelu,
+                         int32_t* status, cudaStream_t s, float* split_ws = nullptr);
 
 // ---- tensor-core attention (attention_tc.cu); strides in elements
 struct AttnLayout {
@@ -156,8 +165,10 @@ int launch_adamw(const OptTable& tab, int dtype, float* params, const float* gra
 int launch_ce_backward(const void* logits, int dtype, const int64_t* targets, const double* sum_count, void* dlogits,
                        int rows, int V, int32_t* status, cudaStream_t s, float scale = 1.f);
 int layernorm_backward_parts(int rows, int C);  // part: [parts, 2C] floats
+// dx16 (optional): a bf16 copy of the dx rows as written (the next products' operand).
 int launch_layernorm_backward(const float* dy, const float* x, const void* w, int dtype, float* dx, int accumulate,
-                              float* dw, float* db, int accumulate_wb, float* part, int rows, int C, cudaStream_t s);
+                              float* dw, float* db, int accumulate_wb, float* part, int rows, int C, cudaStream_t s,
+                              bf16* dx16 = nullptr);
 int colsum_parts(int rows);              // part: [parts, C] floats
 int launch_colsum(const void* y, int dtype, int rows, int C, float* out, int accumulate, float* part,
                   cudaStream_t s);

@@ -52,17 +52,19 @@ def test_tiny_fp32_gradients(gelu, bias):
         assert err <= 1e-4, (n, err)
 
 
-def test_gpt2_shape_bf16_gradients():
-    """2-layer stress model of the GPT-2 124M shape (C 768, 12 heads, V 50304), B 2, T 64.
+@pytest.mark.parametrize("gelu", ["erf", "tanh"])
+def test_gpt2_shape_bf16_gradients(gelu):
+    """2-layer stress model of the GPT-2 124M shape (C 768, 12 heads, V 50304), B 2, T 64, both GELU
+    forms (the bf16 backward folds GELU's derivative into the c_proj product's epilogue).
     Gradients pass through bf16 storage at about ten points (logits, dlogits, activations, the
     products' inputs, dq/dk/dv), each rounding 2^-9 relative; added in quadrature they leave
     ~1e-2 relative (Frobenius) per tensor.  Bound: 3e-2, and 0.9995 cosine similarity."""
     cfgd = dict(seeded.WORKLOADS["gpt2"].model_dict(), n_layer=2)
     W = seeded.make_weights(cfgd, stress=True)
     idx, tgt = seeded.make_tokens(2, 64, 50257, seed=556, ignore_frac=0.1)
-    loss, g = run_grads(cfgd, W, idx, tgt)
+    loss, g = run_grads(cfgd, W, idx, tgt, gelu)
     W64 = seeded.to_f64(W)
-    ref, rloss = ob.backward(W64, cfgd, idx.numpy(), tgt.numpy())
+    ref, rloss = ob.backward(W64, cfgd, idx.numpy(), tgt.numpy(), gelu)
     assert abs(loss - rloss) <= 1e-3 * abs(rloss)
     worst = {}
     for n in ref:
