@@ -80,6 +80,34 @@ GPT_DEVINL bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_fl
     }
 }
 
+// As mbar_wait, acquiring at cluster scope (the phase's arrivals include other CTAs' threads).
+GPT_DEVINL bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+    const uint32_t a = smem_addr(bar);
+    auto try_wait = [&]() {
+        uint32_t ok;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(a), "r"(parity)
+            : "memory");
+        return ok != 0;
+    };
+    if (try_wait()) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (try_wait()) return true;
+        if ((it & 63u) == 0u) {
+            if (*abort_flag) return false;
+            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                *abort_flag = 1;
+                return false;
+            }
+        }
+    }
+}
+
 // Waits for a phase with only a time bound and no abort check: used on the way out, to
 // let copies or MMAs already in flight finish before shared or tensor memory is released.
 GPT_DEVINL void mbar_drain(uint64_t* bar, uint32_t parity) {
@@ -88,6 +116,37 @@ GPT_DEVINL void mbar_drain(uint64_t* bar, uint32_t parity) {
     while (!mbar_try_wait(a, parity)) {
         if (globaltimer_ns() - t0 > kWaitLimitNs) return;
     }
+}
+
+// ------------------------------------------------------------------ CTA pairs (clusters of two)
+GPT_DEVINL uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+GPT_DEVINL uint32_t cluster_id_x() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+    return r;
+}
+GPT_DEVINL uint32_t num_clusters_x() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
+    return r;
+}
+// Every thread of both CTAs of the cluster (warp-aligned).
+GPT_DEVINL void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Cluster address of the same shared-memory object in CTA `rank` of this cluster.
+GPT_DEVINL uint32_t map_to_rank(const void* p, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr(p)), "r"(rank));
+    return r;
+}
+// Arrive on a barrier of another CTA of the cluster.
+GPT_DEVINL void mbar_arrive_remote(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 // ------------------------------------------------------------------ TMA
@@ -120,6 +179,16 @@ GPT_DEVINL void bulk_load_1d(void* dst, const void* src, uint32_t bytes, uint64_
                      smem_addr(dst)),
                  "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_addr(bar))
                  : "memory");
+}
+
+// 2-D tensor load by either CTA of a pair for a 2-SM MMA: data into this CTA's shared memory, the
+// bytes counted on the barrier at cluster address `bar` (the leader CTA's).  No multicast.
+GPT_DEVINL void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint32_t bar, int x, int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
+        : "memory");
 }
 
 // Shared -> global tile store and tile reduce-add (fp32 add at the destination), tracked by the
@@ -161,6 +230,20 @@ GPT_DEVINL void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
                  : "memory");
 }
 
+// The same for a CTA pair: one warp with the same warp index in each CTA executes these; the
+// columns are allocated in both CTAs' tensor memory at the same address.
+GPT_DEVINL void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(dst_smem)),
+                 "r"(ncols)
+                 : "memory");
+}
+GPT_DEVINL void tmem_relinquish_pair() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+GPT_DEVINL void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
 GPT_DEVINL void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 GPT_DEVINL void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
@@ -183,6 +266,27 @@ GPT_DEVINL void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint3
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
         "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// 2-SM MMA issued by the leader CTA of a pair: A rows [0, 128) from this CTA's shared memory and
+// [128, 256) from the peer's (same offsets), B's N columns split the same way, D in both CTAs'
+// tensor memory (each its 128 rows).
+GPT_DEVINL void umma_ss_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// Arrives on `bar` in each CTA of the pair named by `mask` (bit r = rank r) once the pair's MMAs
+// issued so far have completed.
+GPT_DEVINL void umma_commit_pair(uint64_t* bar, uint16_t mask) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            smem_addr(bar)),
+        "h"(mask)
         : "memory");
 }
 

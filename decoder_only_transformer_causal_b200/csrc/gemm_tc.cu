@@ -8,18 +8,56 @@ namespace {
 
 constexpr int kBN = 256;
 
-template <int EPI, int GELU_TANH, int A_MN = 0, int B_MN = 0>
+// Co-resident clusters of two for a kernel (cached per device; 0 if the query fails).
+int max_pairs(const void* kern, int threads, size_t smem, int* cache) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+    if (cache[dev] > 0) return cache[dev];
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * num_sms());
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    cache[dev] = n;
+    return n;
+}
+
+// PAIR: 256-row tiles on CTA pairs (the 2-SM MMA); the B map's box must then be 128 rows
+// (K-major B) — see b_box_rows().
+template <int EPI, int GELU_TANH, int A_MN = 0, int B_MN = 0, int PAIR = 0>
 int launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, const gemm::Params& p,
                cudaStream_t s) {
-    using L = gemm::Cfg<kBN>;
-    auto kern = gemm::gemm_bf16_tc<kBN, EPI, GELU_TANH, A_MN, B_MN>;
+    using L = gemm::Cfg<kBN, PAIR>;
+    auto kern = gemm::gemm_bf16_tc<kBN, EPI, GELU_TANH, A_MN, B_MN, PAIR>;
     static size_t opted[kMaxDevices] = {};
     const int rc = opt_in_smem(reinterpret_cast<const void*>(kern), L::SMEM_BYTES, opted);
     if (rc) return rc;
-    const int tiles = ((p.M + gemm::BM - 1) / gemm::BM) * ((p.N + kBN - 1) / kBN) * p.k_splits;
+    const int tm = PAIR ? 2 * gemm::BM : gemm::BM;
+    const int tiles = ((p.M + tm - 1) / tm) * ((p.N + kBN - 1) / kBN) * p.k_splits;
+    if (PAIR) {
+        static int cache[kMaxDevices] = {};
+        int units = max_pairs(reinterpret_cast<const void*>(kern), L::THREADS, L::SMEM_BYTES, cache);
+        if (units <= 0) units = num_sms() / 2;
+        units = tiles < units ? tiles : units;
+        return launch_overlapped_pairs(kern, dim3(2 * units), dim3(L::THREADS), L::SMEM_BYTES, s, ta, tb, tc, p);
+    }
     const int grid = tiles < num_sms() ? tiles : num_sms();
     return launch_overlapped(kern, dim3(grid), dim3(L::THREADS), L::SMEM_BYTES, s, ta, tb, tc, p);
 }
+
+// 2-SM pairs pay off once there are two 128-row blocks to pair.
+bool use_pairs(int M) { return M >= 2 * gemm::BM; }
 
 // out[m, n] += sum over s = 0..S-1, in order, of part[s * M + m][n]: the partial products of a
 // split-K launch (part rows of N fp32; N, ldo multiples of 4 and 16-byte aligned buffers).
@@ -78,8 +116,9 @@ int launch_gemm_bf16(const bf16* A, long long lda, const bf16* W, long long ldw,
     int rc = make_tmap_bf16_2d(&ta, A, static_cast<uint64_t>(K), static_cast<uint64_t>(M),
                                static_cast<uint64_t>(lda) * 2, gemm::BK, gemm::BM);
     if (rc) return rc;
+    const bool pair = use_pairs(M);
     rc = make_tmap_bf16_2d(&tb, W, static_cast<uint64_t>(K), static_cast<uint64_t>(N),
-                           static_cast<uint64_t>(ldw) * 2, gemm::BK, kBN);
+                           static_cast<uint64_t>(ldw) * 2, gemm::BK, pair ? kBN / 2 : kBN);
     if (rc) return rc;
     // Output map for the epilogue's TMA stores: 32-row boxes of 64 bytes (32 bf16 or 16 fp32).
     CUtensorMap tc;
@@ -99,19 +138,29 @@ int launch_gemm_bf16(const bf16* A, long long lda, const bf16* W, long long ldw,
     p.status = status;
     p.k_splits = 1;
     p.kb_per_split = (K + gemm::BK - 1) / gemm::BK;
+    if (epilogue == gemm::EPI_CE) {
+        if (!ce) return GPT_ERR_NULL;
+        p.targets = ce->targets;
+        p.part = ce->part;
+        p.tlogit = ce->tlogit;
+        p.n_part = ce->n_part;
+    }
     switch (epilogue) {
-        case GPT_EPI_STORE: return launch_one<gemm::EPI_STORE, 0>(ta, tb, tc, p, s);
+        case GPT_EPI_STORE:
+            return pair ? launch_one<gemm::EPI_STORE, 0, 0, 0, 1>(ta, tb, tc, p, s)
+                        : launch_one<gemm::EPI_STORE, 0>(ta, tb, tc, p, s);
         case GPT_EPI_GELU:
-            return gelu == GPT_GELU_TANH ? launch_one<gemm::EPI_GELU, 1>(ta, tb, tc, p, s)
-                                         : launch_one<gemm::EPI_GELU, 0>(ta, tb, tc, p, s);
-        case GPT_EPI_RESID: return launch_one<gemm::EPI_RESID, 0>(ta, tb, tc, p, s);
+            if (gelu == GPT_GELU_TANH)
+                return pair ? launch_one<gemm::EPI_GELU, 1, 0, 0, 1>(ta, tb, tc, p, s)
+                            : launch_one<gemm::EPI_GELU, 1>(ta, tb, tc, p, s);
+            return pair ? launch_one<gemm::EPI_GELU, 0, 0, 0, 1>(ta, tb, tc, p, s)
+                        : launch_one<gemm::EPI_GELU, 0>(ta, tb, tc, p, s);
+        case GPT_EPI_RESID:
+            return pair ? launch_one<gemm::EPI_RESID, 0, 0, 0, 1>(ta, tb, tc, p, s)
+                        : launch_one<gemm::EPI_RESID, 0>(ta, tb, tc, p, s);
         case gemm::EPI_CE:
-            if (!ce) return GPT_ERR_NULL;
-            p.targets = ce->targets;
-            p.part = ce->part;
-            p.tlogit = ce->tlogit;
-            p.n_part = ce->n_part;
-            return launch_one<gemm::EPI_CE, 0>(ta, tb, tc, p, s);
+            return pair ? launch_one<gemm::EPI_CE, 0, 0, 0, 1>(ta, tb, tc, p, s)
+                        : launch_one<gemm::EPI_CE, 0>(ta, tb, tc, p, s);
         default: return GPT_ERR_UNSUPPORTED;
     }
 }
@@ -166,19 +215,32 @@ int launch_gemm_bf16_bwd(const bf16* A, long long lda, bool a_mn, const bf16* W,
     rc = make_tmap_2d_sw64(&tc, out, f32, static_cast<uint64_t>(N), static_cast<uint64_t>(M),
                            static_cast<uint64_t>(ldo) * (f32 ? 4 : 2), f32 ? 16 : 32, 32);
     if (rc) return rc;
+    // The input-gradient products (K-major A, M = token rows) run on CTA pairs; MN-major B boxes are
+    // 64 columns wide either way.
+    const bool pair = !a_mn && use_pairs(M);
+    if (mode == GEMM_BWD_DGELU_BF16) {
+        if (!aux) return GPT_ERR_NULL;
+        if ((reinterpret_cast<uintptr_t>(aux) & 15) || (ld_aux % 8)) return GPT_ERR_BAD_ALIGN;
+        p.aux = aux;
+        p.ld_aux = ld_aux;
+    }
     switch (mode) {
         case GEMM_BWD_ACC_F32:
-            return a_mn ? launch_one<gemm::EPI_RESID, 0, 1, 1>(ta, tb, tc, p, s)
+            if (a_mn) return launch_one<gemm::EPI_RESID, 0, 1, 1>(ta, tb, tc, p, s);
+            return pair ? launch_one<gemm::EPI_RESID, 0, 0, 1, 1>(ta, tb, tc, p, s)
                         : launch_one<gemm::EPI_RESID, 0, 0, 1>(ta, tb, tc, p, s);
-        case GEMM_BWD_STORE_F32: return launch_one<gemm::EPI_F32, 0, 0, 1>(ta, tb, tc, p, s);
-        case GEMM_BWD_STORE_BF16: return launch_one<gemm::EPI_STORE, 0, 0, 1>(ta, tb, tc, p, s);
+        case GEMM_BWD_STORE_F32:
+            return pair ? launch_one<gemm::EPI_F32, 0, 0, 1, 1>(ta, tb, tc, p, s)
+                        : launch_one<gemm::EPI_F32, 0, 0, 1>(ta, tb, tc, p, s);
+        case GEMM_BWD_STORE_BF16:
+            return pair ? launch_one<gemm::EPI_STORE, 0, 0, 1, 1>(ta, tb, tc, p, s)
+                        : launch_one<gemm::EPI_STORE, 0, 0, 1>(ta, tb, tc, p, s);
         case GEMM_BWD_DGELU_BF16:
-            if (!aux) return GPT_ERR_NULL;
-            if ((reinterpret_cast<uintptr_t>(aux) & 15) || (ld_aux % 8)) return GPT_ERR_BAD_ALIGN;
-            p.aux = aux;
-            p.ld_aux = ld_aux;
-            return gelu == GPT_GELU_TANH ? launch_one<gemm::EPI_DGELU, 1, 0, 1>(ta, tb, tc, p, s)
-                                         : launch_one<gemm::EPI_DGELU, 0, 0, 1>(ta, tb, tc, p, s);
+            if (gelu == GPT_GELU_TANH)
+                return pair ? launch_one<gemm::EPI_DGELU, 1, 0, 1, 1>(ta, tb, tc, p, s)
+                            : launch_one<gemm::EPI_DGELU, 1, 0, 1>(ta, tb, tc, p, s);
+            return pair ? launch_one<gemm::EPI_DGELU, 0, 0, 1, 1>(ta, tb, tc, p, s)
+                        : launch_one<gemm::EPI_DGELU, 0, 0, 1>(ta, tb, tc, p, s);
         default: return GPT_ERR_UNSUPPORTED;
     }
 }

@@ -60,13 +60,17 @@ struct Params {
     long long ld_aux;
 };
 
-template <int BN>
+// PAIR: a cluster of two CTAs computes one 256 x BN tile with the 2-SM MMA; each CTA stages its
+// own 128 rows of A and half of B's BN rows, so a stage is 32 KB and six fit.
+template <int BN, int PAIR = 0>
 struct Cfg {
     static_assert(BN == 256, "BN");
+    static constexpr int STAGES = PAIR ? 6 : kStages;
+    static constexpr int B_ROWS = PAIR ? BN / 2 : BN;         // rows of B this CTA stages
     static constexpr int A_BYTES = BM * BK * 2;
-    static constexpr int B_BYTES = BN * BK * 2;
+    static constexpr int B_BYTES = B_ROWS * BK * 2;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-    static constexpr int BIAS_OFF = kStages * STAGE_BYTES;    // one bias slice per epilogue warp
+    static constexpr int BIAS_OFF = STAGES * STAGE_BYTES;     // one bias slice per epilogue warp
     static constexpr int STG_OFF = BIAS_OFF + NEPI * (BN / (NEPI / 4)) * 4;
     static constexpr int STG_BYTES = 32 * 64;                 // 32 rows x 64 bytes per warp
     static constexpr int BAR_OFF = STG_OFF + NEPI * STG_BYTES;
@@ -137,11 +141,18 @@ GPT_DEVINL float gelu_f(float x) {
 // whose transpose the product needs (the backward's dY^T X and dY W).  Its tile is then loaded
 // as 64-column TMA boxes (64 K rows x 128 bytes each, 8 KB apart) and described to the MMA with
 // the MN-major layout; no transposed copy is made.
-template <int BN, int EPI, int GELU_TANH, int A_MN = 0, int B_MN = 0>
+//
+// PAIR: launched in clusters of two.  Rank 0 (the leader) owns the barriers the pair shares: each
+// CTA's TMA loads count on the leader's `full`, the leader's one MMA thread issues the 2-SM MMAs
+// (M = 256) and its commits arrive on `empty` and `tfull` in both CTAs, and both CTAs' epilogue
+// threads arrive on the leader's `tempty`.  Each CTA's epilogue drains its own 128 rows.
+template <int BN, int EPI, int GELU_TANH, int A_MN = 0, int B_MN = 0, int PAIR = 0>
 __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)  // 10 warps: <= 168 registers per thread
     gemm_bf16_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const __grid_constant__ CUtensorMap tmC, const Params p) {
-    using L = Cfg<BN>;
+    using L = Cfg<BN, PAIR>;
+    constexpr int kStages = L::STAGES;
+    constexpr int TM = PAIR ? 2 * BM : BM;  // output rows per tile
     constexpr int COLS = L::COLS_PER_WARP;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -157,7 +168,10 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)  // 10 warps: <= 168 regi
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int num_m = (p.M + BM - 1) / BM;
+    const uint32_t rank = PAIR ? cluster_ctarank() : 0u;  // 0: leader
+    const int unit0 = PAIR ? static_cast<int>(cluster_id_x()) : static_cast<int>(blockIdx.x);
+    const int n_units = PAIR ? static_cast<int>(num_clusters_x()) : static_cast<int>(gridDim.x);
+    const int num_m = (p.M + TM - 1) / TM;
     const int num_n = (p.N + BN - 1) / BN;
     const int num_mn = num_m * num_n;
     const int num_tiles = num_mn * p.k_splits;
@@ -186,7 +200,7 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)  // 10 warps: <= 168 regi
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&tfull[a], 1);
-            mbar_init(&tempty[a], NEPI * 32);
+            mbar_init(&tempty[a], (PAIR ? 2 : 1) * NEPI * 32);
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -197,11 +211,17 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)  // 10 warps: <= 168 regi
         tma_prefetch_desc(&tmC);
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, L::TMEM_COLS);
-        tmem_relinquish();
+        if (PAIR) {
+            tmem_alloc_pair(tmem_slot, L::TMEM_COLS);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(tmem_slot, L::TMEM_COLS);
+            tmem_relinquish();
+        }
     }
     tc_fence_before();
     __syncthreads();
+    if (PAIR) cluster_sync();  // the leader's barriers are initialised before the peer's loads count on them
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     // The set-up above overlapped the previous kernel; its outputs are read from here on.
@@ -215,10 +235,18 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)  // 10 warps: <= 168 regi
             uint32_t ph = 0;
             long long issued = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+            const uint32_t full_leader = PAIR ? map_to_rank(full, 0) : 0u;  // cluster address of full[0]
+            auto load = [&](void* dst, const CUtensorMap* map, int x, int y) {
+                if (PAIR)
+                    tma_load_2d_pair(dst, map, full_leader + 8u * static_cast<uint32_t>(stage), x, y);
+                else
+                    tma_load_2d(dst, map, &full[stage], x, y);
+            };
+            for (int tile = unit0; tile < num_tiles && ok; tile += n_units) {
                 int m_blk, n_blk;
                 tile_mn(tile, m_blk, n_blk);
-                const int m0 = m_blk * BM, n0 = n_blk * BN;
+                const int m0 = m_blk * TM + static_cast<int>(rank) * BM;           // this CTA's A rows
+                const int n0 = n_blk * BN + static_cast<int>(rank) * L::B_ROWS;    // this CTA's B rows
                 int kb0, kb1;
                 tile_kb(tile, kb0, kb1);
                 for (int kb = kb0; kb < kb1; ++kb) {
@@ -227,20 +255,20 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)  // 10 warps: <= 168 regi
                         break;
                     }
                     uint8_t* st = smem + stage * L::STAGE_BYTES;
-                    mbar_arrive_expect_tx(&full[stage], L::STAGE_BYTES);
+                    // the leader expects both CTAs' bytes
+                    if (rank == 0) mbar_arrive_expect_tx(&full[stage], (PAIR ? 2 : 1) * L::STAGE_BYTES);
                     if (A_MN) {
 #pragma unroll
-                        for (int j = 0; j < BM / 64; ++j)
-                            tma_load_2d(st + j * 8192, &tmA, &full[stage], m0 + 64 * j, kb * BK);
+                        for (int j = 0; j < BM / 64; ++j) load(st + j * 8192, &tmA, m0 + 64 * j, kb * BK);
                     } else {
-                        tma_load_2d(st, &tmA, &full[stage], kb * BK, m0);
+                        load(st, &tmA, kb * BK, m0);
                     }
                     if (B_MN) {
 #pragma unroll
-                        for (int j = 0; j < BN / 64; ++j)
-                            tma_load_2d(st + L::A_BYTES + j * 8192, &tmB, &full[stage], n0 + 64 * j, kb * BK);
+                        for (int j = 0; j < L::B_ROWS / 64; ++j)
+                            load(st + L::A_BYTES + j * 8192, &tmB, n0 + 64 * j, kb * BK);
                     } else {
-                        tma_load_2d(st + L::A_BYTES, &tmB, &full[stage], kb * BK, n0);
+                        load(st + L::A_BYTES, &tmB, kb * BK, n0);
                     }
                     ++issued;
                     if (++stage == kStages) {
@@ -251,7 +279,8 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)  // 10 warps: <= 168 regi
             }
             // Make sure no bulk copy is still writing shared memory when the CTA exits: wait
             // for the latest load issued into each stage (already complete on the normal path).
-            const long long n_check = issued < kStages ? issued : kStages;
+            // The leader's `full` phases count the peer's bytes too.
+            const long long n_check = rank != 0 ? 0 : (issued < kStages ? issued : kStages);
             for (long long i = 1; i <= n_check; ++i) {
                 const long long idx = issued - i;
                 mbar_drain(&full[idx % kStages], static_cast<uint32_t>((idx / kStages) & 1));
@@ -259,15 +288,17 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)  // 10 warps: <= 168 regi
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t idesc = make_idesc_bf16(BM, BN, B_MN != 0, A_MN != 0);
+        if (lane == 0 && rank == 0) {
+            constexpr uint32_t idesc = make_idesc_bf16(TM, BN, B_MN != 0, A_MN != 0);
             int stage = 0;
             uint32_t ph = 0;
             int acc = 0;
             uint32_t acc_ph = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-                if (!mbar_wait(&tempty[acc], acc_ph ^ 1u, abort_flag)) break;
+            for (int tile = unit0; tile < num_tiles && ok; tile += n_units) {
+                if (!(PAIR ? mbar_wait_cluster(&tempty[acc], acc_ph ^ 1u, abort_flag)
+                           : mbar_wait(&tempty[acc], acc_ph ^ 1u, abort_flag)))
+                    break;
                 tc_fence_after();
                 const uint32_t d = tmem_base + static_cast<uint32_t>(acc * BN);
                 int kb0, kb1;
@@ -288,21 +319,33 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)  // 10 warps: <= 168 regi
                                                  : make_sdesc_sw128(a_addr + k * 32);
                         const uint64_t db = B_MN ? make_sdesc_sw128_mn(b_addr + k * 2048, 8192)
                                                  : make_sdesc_sw128(b_addr + k * 32);
-                        umma_ss(d, da, db, idesc, (kb != kb0 || k != 0) ? 1u : 0u);
+                        if (PAIR)
+                            umma_ss_pair(d, da, db, idesc, (kb != kb0 || k != 0) ? 1u : 0u);
+                        else
+                            umma_ss(d, da, db, idesc, (kb != kb0 || k != 0) ? 1u : 0u);
                     }
-                    umma_commit(&empty[stage]);
+                    if (PAIR)
+                        umma_commit_pair(&empty[stage], 0x3);
+                    else
+                        umma_commit(&empty[stage]);
                     if (++stage == kStages) {
                         stage = 0;
                         ph ^= 1u;
                     }
                 }
                 if (!ok) break;
-                umma_commit(&tfull[acc]);
+                if (PAIR)
+                    umma_commit_pair(&tfull[acc], 0x3);
+                else
+                    umma_commit(&tfull[acc]);
                 acc ^= 1;
                 if (acc == 0) acc_ph ^= 1u;
             }
             // All MMAs issued by this thread must be finished before TMEM is released.
-            umma_commit(drain);
+            if (PAIR)
+                umma_commit_pair(drain, 0x1);
+            else
+                umma_commit(drain);
             mbar_drain(drain, 0);
         }
     } else {
@@ -312,10 +355,10 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)  // 10 warps: <= 168 regi
         const int half = ew >> 2;            // which BN/2 columns of the tile
         int acc = 0;
         uint32_t acc_ph = 0;
-        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+        for (int tile = unit0; tile < num_tiles; tile += n_units) {
             int m_blk, n_blk;
             tile_mn(tile, m_blk, n_blk);
-            const int m0 = m_blk * BM, n0 = n_blk * BN;
+            const int m0 = m_blk * TM + static_cast<int>(rank) * BM, n0 = n_blk * BN;  // this CTA's rows
             const int row = m0 + quarter * 32 + lane;
             const bool row_ok = row < p.M;
             const int nw0 = n0 + half * COLS;  // first column of this warp's slice
@@ -484,7 +527,10 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)  // 10 warps: <= 168 regi
                     make_float2(run_max, run_sum);
             }
             tc_fence_before();
-            mbar_arrive(&tempty[acc]);
+            if (PAIR && rank != 0)
+                mbar_arrive_remote(map_to_rank(&tempty[acc], 0));
+            else
+                mbar_arrive(&tempty[acc]);
             acc ^= 1;
             if (acc == 0) acc_ph ^= 1u;
         }
@@ -492,10 +538,16 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)  // 10 warps: <= 168 regi
     }
 
     __syncthreads();
+    // A pair releases its tensor memory together, once neither CTA's MMAs, loads or arrivals can
+    // still reach the other.
+    if (PAIR) cluster_sync();
     if (warp == 1) {
         __syncwarp();
         tc_fence_after();
-        tmem_dealloc(tmem_base, L::TMEM_COLS);
+        if (PAIR)
+            tmem_dealloc_pair(tmem_base, L::TMEM_COLS);
+        else
+            tmem_dealloc(tmem_base, L::TMEM_COLS);
     }
     if (threadIdx.x == 0 && *abort_flag) set_status(p.status, GPT_ERR_TIMEOUT);
 }
