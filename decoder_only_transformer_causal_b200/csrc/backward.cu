@@ -555,6 +555,9 @@ int launch_layernorm_backward(const float* dy, const float* x, const void* w, in
                                    x, static_cast<const float*>(w), dx, accumulate, part, rows, C, dx16);
     }
     if (rc) return rc;
+    if (db == dw + C)  // adjacent gradients (the packed layout when C * 4 is a multiple of 256): one pass
+        return launch_overlapped(colsum_parts_kernel, dim3((2 * C + 31) / 32), dim3(32, 8), 0, s,
+                                 static_cast<const float*>(part), 2LL * C, n_part, 2 * C, dw, accumulate_wb);
     const dim3 gp((C + 31) / 32), bp(32, 8);
     rc = launch_overlapped(colsum_parts_kernel, gp, bp, 0, s, static_cast<const float*>(part), 2LL * C, n_part, C, dw,
                            accumulate_wb);

@@ -120,10 +120,13 @@ int launch_gemm_bf16(const bf16* A, long long lda, const bf16* W, long long ldw,
     rc = make_tmap_bf16_2d(&tb, W, static_cast<uint64_t>(K), static_cast<uint64_t>(N),
                            static_cast<uint64_t>(ldw) * 2, gemm::BK, pair ? kBN / 2 : kBN);
     if (rc) return rc;
-    // Output map for the epilogue's TMA stores: 32-row boxes of 64 bytes (32 bf16 or 16 fp32).
+    // Output map for the epilogue's TMA stores: 32-row boxes of 64 bytes (32 bf16 or 16 fp32);
+    // 2M rows for EPI_GELU2 (pre-activation, then GELU output).
     CUtensorMap tc;
     const bool out_f32 = epilogue == GPT_EPI_RESID;
-    rc = make_tmap_2d_sw64(&tc, out, out_f32, static_cast<uint64_t>(N), static_cast<uint64_t>(M),
+    if (epilogue == gemm::EPI_GELU2 && (M % 32)) return GPT_ERR_UNSUPPORTED;
+    const uint64_t out_rows = static_cast<uint64_t>(M) * (epilogue == gemm::EPI_GELU2 ? 2 : 1);
+    rc = make_tmap_2d_sw64(&tc, out, out_f32, static_cast<uint64_t>(N), out_rows,
                            static_cast<uint64_t>(ldo) * (out_f32 ? 4 : 2), out_f32 ? 16 : 32, 32);
     if (rc) return rc;
     gemm::Params p{};
@@ -161,6 +164,12 @@ int launch_gemm_bf16(const bf16* A, long long lda, const bf16* W, long long ldw,
         case gemm::EPI_CE:
             return pair ? launch_one<gemm::EPI_CE, 0, 0, 0, 1>(ta, tb, tc, p, s)
                         : launch_one<gemm::EPI_CE, 0>(ta, tb, tc, p, s);
+        case gemm::EPI_GELU2:
+            if (gelu == GPT_GELU_TANH)
+                return pair ? launch_one<gemm::EPI_GELU2, 1, 0, 0, 1>(ta, tb, tc, p, s)
+                            : launch_one<gemm::EPI_GELU2, 1>(ta, tb, tc, p, s);
+            return pair ? launch_one<gemm::EPI_GELU2, 0, 0, 0, 1>(ta, tb, tc, p, s)
+                        : launch_one<gemm::EPI_GELU2, 0>(ta, tb, tc, p, s);
         default: return GPT_ERR_UNSUPPORTED;
     }
 }

@@ -39,7 +39,9 @@ constexpr int NEPI = 8;  // epilogue warps: two per TMEM lane quarter, each half
 //          launch).
 // EPI_DGELU: out_bf16 = acc * gelu'(aux), aux the bf16 pre-activation [M, ld_aux] (the MLP's
 //          backward through GELU, fused into the product that yields d loss / d gelu output).
-enum Epi { EPI_STORE = 0, EPI_GELU = 1, EPI_RESID = 2, EPI_CE = 3, EPI_F32 = 4, EPI_DGELU = 5 };
+// EPI_GELU2: pre = acc + b at rows [0, M) of out and gelu(acc + b) at rows [M, 2M) (the training
+//          forward keeps both for the backward; M % 32 == 0).
+enum Epi { EPI_STORE = 0, EPI_GELU = 1, EPI_RESID = 2, EPI_CE = 3, EPI_F32 = 4, EPI_DGELU = 5, EPI_GELU2 = 6 };
 
 struct Params {
     int M, N, K;
@@ -376,6 +378,18 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)  // 10 warps: <= 168 regi
             }
             long long tgt = -1;
             if (EPI == EPI_CE && row_ok) tgt = p.targets[row];
+            // EPI_DGELU: the first chunk's pre-activations, loaded before the accumulator wait
+            uint32_t aux_next[EPI == EPI_DGELU ? 16 : 1];
+            bool aux_ok = false;
+            if (EPI == EPI_DGELU && row_ok && nw0 + 32 <= p.N) {
+                const uint4* an = reinterpret_cast<const uint4*>(p.aux + static_cast<long long>(row) * p.ld_aux + nw0);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const uint4 w = __ldcg(an + q);
+                    aux_next[4 * q] = w.x, aux_next[4 * q + 1] = w.y, aux_next[4 * q + 2] = w.z, aux_next[4 * q + 3] = w.w;
+                }
+                aux_ok = true;
+            }
 
             const bool got = mbar_wait(&tfull[acc], acc_ph, abort_flag);
             __syncwarp();  // tcgen05.ld below is warp-collective
@@ -437,7 +451,7 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)  // 10 warps: <= 168 regi
                         float v[32];
 #pragma unroll
                         for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[32 * h + j]);
-                        if (EPI == EPI_STORE || EPI == EPI_GELU) {
+                        if (EPI == EPI_STORE || EPI == EPI_GELU || EPI == EPI_GELU2) {
 #pragma unroll
                             for (int q = 0; q < 8; ++q) {
                                 const float4 b4 = *reinterpret_cast<const float4*>(sb + cc + 4 * q);
@@ -452,21 +466,33 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)  // 10 warps: <= 168 regi
                             for (int j = 0; j < 32; ++j) v[j] = gelu_f<GELU_TANH>(v[j]);
                         }
                         if (EPI == EPI_DGELU && row_ok) {
-                            // this row's 32 pre-activations (64 bytes) of the chunk
-                            const bf16* ap = p.aux + static_cast<long long>(row) * p.ld_aux + n;
+                            // this row's 32 pre-activations of the chunk: from the registers loaded
+                            // one chunk ahead (whole chunks), else element by element
                             float z[32];
-                            if (full_chunk) {
+                            if (full_chunk && aux_ok) {
 #pragma unroll
-                                for (int q = 0; q < 4; ++q) {
-                                    float f[8];
-                                    ld8(ap + 8 * q, f);
-#pragma unroll
-                                    for (int e = 0; e < 8; ++e) z[8 * q + e] = f[e];
+                                for (int q = 0; q < 16; ++q) {
+                                    z[2 * q] = __uint_as_float(aux_next[q] << 16);
+                                    z[2 * q + 1] = __uint_as_float(aux_next[q] & 0xffff0000u);
                                 }
                             } else {
+                                const bf16* ap = p.aux + static_cast<long long>(row) * p.ld_aux + n;
 #pragma unroll
                                 for (int j = 0; j < 32; ++j)
                                     z[j] = n + j < p.N ? __bfloat162float(ap[j]) : 0.f;
+                            }
+                            // the next chunk's pre-activations, loaded while this one is finished
+                            aux_ok = false;
+                            if (cc + 32 < COLS && nw0 + cc + 64 <= p.N) {
+                                const uint4* an = reinterpret_cast<const uint4*>(
+                                    p.aux + static_cast<long long>(row) * p.ld_aux + n + 32);
+#pragma unroll
+                                for (int q = 0; q < 4; ++q) {
+                                    const uint4 w = __ldcg(an + q);
+                                    aux_next[4 * q] = w.x, aux_next[4 * q + 1] = w.y;
+                                    aux_next[4 * q + 2] = w.z, aux_next[4 * q + 3] = w.w;
+                                }
+                                aux_ok = true;
                             }
 #pragma unroll
                             for (int j = 0; j < 32; ++j) v[j] *= gelu_grad_f<GELU_TANH>(z[j]);
@@ -505,19 +531,26 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)  // 10 warps: <= 168 regi
                             }
                         }
                         if (!band_ok) continue;  // warp-uniform: no row of this band exists
-                        if (lane == 0) bulk_wait_read_all();  // the buffer's previous tile was read
-                        __syncwarp();
 #pragma unroll
-                        for (int q = 0; q < 4; ++q)
-                            srow[q ^ swz] = make_uint4(pack_bf16x2(v[8 * q + 0], v[8 * q + 1]),
-                                                       pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
-                                                       pack_bf16x2(v[8 * q + 4], v[8 * q + 5]),
-                                                       pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
-                        fence_proxy_async_shared();
-                        __syncwarp();
-                        if (lane == 0) {
-                            tma_store_2d(&tmC, stg, n, row0);
-                            bulk_commit();
+                        for (int pass = 0; pass < (EPI == EPI_GELU2 ? 2 : 1); ++pass) {
+                            if (EPI == EPI_GELU2 && pass == 1) {
+#pragma unroll
+                                for (int j = 0; j < 32; ++j) v[j] = gelu_f<GELU_TANH>(v[j]);
+                            }
+                            if (lane == 0) bulk_wait_read_all();  // the buffer's previous tile was read
+                            __syncwarp();
+#pragma unroll
+                            for (int q = 0; q < 4; ++q)
+                                srow[q ^ swz] = make_uint4(pack_bf16x2(v[8 * q + 0], v[8 * q + 1]),
+                                                           pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                                                           pack_bf16x2(v[8 * q + 4], v[8 * q + 5]),
+                                                           pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+                            fence_proxy_async_shared();
+                            __syncwarp();
+                            if (lane == 0) {
+                                tma_store_2d(&tmC, stg, n, row0 + pass * p.M);
+                                bulk_commit();
+                            }
                         }
                     }
                 }

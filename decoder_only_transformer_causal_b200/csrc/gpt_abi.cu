@@ -1192,7 +1192,15 @@ GPT_API int gpt_forward_train(const gpt_config_t* cfg, const void* weights, cons
                                       static_cast<const float*>(W.bias(l, W_PROJ_B)), x_mid, C, N, C, C, GPT_EPI_RESID,
                                       cfg->gelu, s));
         GPT_TRY(launch_layernorm(x_mid, W.layer(l, W_LN2_W), W.bias(l, W_LN2_B), u2, N, C, dt, s));
-        if (bf)
+        // c_fc keeps both its pre-activation (for the GELU derivative) and the GELU output: one
+        // product writing both when h directly follows pre (bf16), else a store and a GELU pass.
+        const bool two_out = bf && (N % 32 == 0) &&
+                             static_cast<uint8_t*>(hh) == static_cast<uint8_t*>(pre) + static_cast<size_t>(N) * 4 * C * es;
+        if (two_out)
+            GPT_TRY(launch_gemm_bf16(static_cast<const bf16*>(u2), C, static_cast<const bf16*>(W.layer(l, W_FC_W)), C,
+                                     static_cast<const bf16*>(W.bias(l, W_FC_B)), pre, 4LL * C, N, 4 * C, C,
+                                     GEMM_EPI_GELU2, cfg->gelu, nullptr, status, s));
+        else if (bf)
             GPT_TRY(launch_gemm_bf16(static_cast<const bf16*>(u2), C, static_cast<const bf16*>(W.layer(l, W_FC_W)), C,
                                      static_cast<const bf16*>(W.bias(l, W_FC_B)), pre, 4LL * C, N, 4 * C, C,
                                      GPT_EPI_STORE, cfg->gelu, nullptr, status, s));
@@ -1200,7 +1208,8 @@ GPT_API int gpt_forward_train(const gpt_config_t* cfg, const void* weights, cons
             GPT_TRY(launch_linear_f32(static_cast<const float*>(u2), C, static_cast<const float*>(W.layer(l, W_FC_W)),
                                       static_cast<const float*>(W.bias(l, W_FC_B)), static_cast<float*>(pre), 4LL * C, N,
                                       4 * C, C, GPT_EPI_STORE, cfg->gelu, s));
-        GPT_TRY(launch_gelu_forward(pre, hh, static_cast<long long>(N) * 4 * C, dt, cfg->gelu == GPT_GELU_TANH, s));
+        if (!two_out)
+            GPT_TRY(launch_gelu_forward(pre, hh, static_cast<long long>(N) * 4 * C, dt, cfg->gelu == GPT_GELU_TANH, s));
         GPT_TRY(cuda_status(cudaMemcpyAsync(x_out, x_mid, static_cast<size_t>(N) * C * 4, cudaMemcpyDeviceToDevice, s)));
         if (bf)
             GPT_TRY(launch_gemm_bf16(static_cast<const bf16*>(hh), 4LL * C, static_cast<const bf16*>(W.layer(l, W_FC2_W)),

@@ -96,6 +96,8 @@ struct CeArgs {
     int n_part;
 };
 int gemm_ce_parts(int N);  // partial slots per row of the lm_head epilogue
+// launch_gemm_bf16 epilogue beyond GPT_EPI_*: out bf16 [2M, ldo] = {acc + b; gelu(acc + b)}, M % 32 == 0.
+constexpr int GEMM_EPI_GELU2 = 6;
 int launch_gemm_bf16(const bf16* A, long long lda, const bf16* W, long long ldw, const bf16* bias,
                      void* out, long long ldo, int M, int N, int K, int epilogue, int gelu,
                      const CeArgs* ce, int32_t* status, cudaStream_t s);
