@@ -278,13 +278,13 @@ def kernel_ops(w, native, dev, stream, only=None):
 # The kernel function (as ncu names it) behind each op of kernel_ops: ops sharing a function
 # are one kernel for the roofline, whose work and time add up.
 # Template arguments as ncu prints them: <BN, epilogue (0 store, 1 GELU, 2 residual add,
-# 3 cross-entropy partials), GELU tanh form>.
+# 3 cross-entropy partials), GELU tanh form, A MN-major, B MN-major, CTA pair>.
 KERNEL_OF = {
-    "gemm_c_attn": "gemm_bf16_tc<256, 0, 0>",
-    "gemm_attn_proj_resid": "gemm_bf16_tc<256, 2, 0>",
-    "gemm_mlp_proj_resid": "gemm_bf16_tc<256, 2, 0>",
-    "gemm_c_fc_gelu": "gemm_bf16_tc<256, 1, 0>",
-    "lm_head_ce": "gemm_bf16_tc<256, 3, 0> (+ ce_rows, loss_finalize)",
+    "gemm_c_attn": "gemm_bf16_tc<256, 0, 0, 0, 0, 1>",
+    "gemm_attn_proj_resid": "gemm_bf16_tc<256, 2, 0, 0, 0, 1>",
+    "gemm_mlp_proj_resid": "gemm_bf16_tc<256, 2, 0, 0, 0, 1>",
+    "gemm_c_fc_gelu": "gemm_bf16_tc<256, 1, 0, 0, 0, 1>",
+    "lm_head_ce": "gemm_bf16_tc<256, 3, 0, 0, 0, 1> (+ ce_rows, loss_finalize)",
     "attention": "attention_fwd_tc",
     "layernorm": "layernorm_kernel<bf16>",
 }
