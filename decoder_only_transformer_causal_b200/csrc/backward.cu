@@ -361,27 +361,51 @@ __global__ void __launch_bounds__(256)
 }
 
 // part[blockIdx.y][c] = sum of y[r, c] over this CTA's row block; first stage of the bias gradient
-// (column sums of the output gradient).  Rows are taken four at a time into four running sums
-// (more loads in flight), which are added in a fixed order at the end.
-constexpr int kColRows = 128;
+// (column sums of the output gradient).  Thread t takes columns [4t, 4t + 4) with one 16-byte
+// (fp32) or 8-byte (bf16) load per row when `vec`, eight rows at a time into eight running sums
+// (loads in flight), which are added in a fixed order at the end.
+constexpr int kColRows = 64;
+GPT_DEVINL float4 ld4(const float* p) { return __ldcg(reinterpret_cast<const float4*>(p)); }
+GPT_DEVINL float4 ld4(const bf16* p) {
+    const uint2 w = __ldcg(reinterpret_cast<const uint2*>(p));
+    return make_float4(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xffff0000u), __uint_as_float(w.y << 16),
+                       __uint_as_float(w.y & 0xffff0000u));
+}
 template <typename E>
-__global__ void colsum_rows_kernel(const E* __restrict__ y, int rows, int C, float* __restrict__ part) {
+__global__ void colsum_rows_kernel(const E* __restrict__ y, int rows, int C, float* __restrict__ part, int vec) {
     griddep_launch_dependents();
     griddep_wait();
-    const int c = blockIdx.x * blockDim.x + threadIdx.x;
-    if (c >= C) return;
+    const int c0 = (blockIdx.x * blockDim.x + threadIdx.x) * 4;
+    if (c0 >= C) return;
     const int r0 = blockIdx.y * kColRows, r1 = min(rows, r0 + kColRows);
-    float v0 = 0.f, v1 = 0.f, v2 = 0.f, v3 = 0.f;
-    int r = r0;
-    for (; r + 4 <= r1; r += 4) {
-        const E* q = y + static_cast<long long>(r) * C + c;
-        v0 += ld1(q);
-        v1 += ld1(q + C);
-        v2 += ld1(q + 2LL * C);
-        v3 += ld1(q + 3LL * C);
+    float* out = part + static_cast<long long>(blockIdx.y) * C;
+    if (vec && c0 + 4 <= C) {
+        float4 acc[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+        int r = r0;
+        for (; r + 8 <= r1; r += 8) {
+            float4 v[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) v[k] = ld4(y + static_cast<long long>(r + k) * C + c0);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) acc[k].x += v[k].x, acc[k].y += v[k].y, acc[k].z += v[k].z, acc[k].w += v[k].w;
+        }
+        for (; r < r1; ++r) {
+            const float4 v = ld4(y + static_cast<long long>(r) * C + c0);
+            acc[0].x += v.x, acc[0].y += v.y, acc[0].z += v.z, acc[0].w += v.w;
+        }
+#pragma unroll
+        for (int k = 1; k < 8; ++k)
+            acc[0].x += acc[k].x, acc[0].y += acc[k].y, acc[0].z += acc[k].z, acc[0].w += acc[k].w;
+        *reinterpret_cast<float4*>(out + c0) = acc[0];
+        return;
     }
-    for (; r < r1; ++r) v0 += ld1(y + static_cast<long long>(r) * C + c);
-    part[static_cast<long long>(blockIdx.y) * C + c] = (v0 + v1) + (v2 + v3);
+    for (int c = c0; c < C && c < c0 + 4; ++c) {
+        float v = 0.f;
+        for (int r = r0; r < r1; ++r) v += ld1(y + static_cast<long long>(r) * C + c);
+        out[c] = v;
+    }
 }
 
 // dpre = dh * gelu'(pre): erf form Phi(z) + z phi(z); tanh form 0.5 (1 + tanh a) +
@@ -572,11 +596,14 @@ int colsum_parts(int rows) { return (rows + kColRows - 1) / kColRows; }
 int launch_colsum(const void* y, int dtype, int rows, int C, float* out, int accumulate, float* part,
                   cudaStream_t s) {
     const int n_part = colsum_parts(rows);
-    const dim3 g1((C + 255) / 256, n_part), b(256);
+    const dim3 g1((C + 4 * 256 - 1) / (4 * 256), n_part), b(256);
+    // 16-byte rows of 4 values: C % 4 == 0 and aligned base and partial buffer
+    const int vec = (C % 4 == 0) && ((reinterpret_cast<uintptr_t>(y) | reinterpret_cast<uintptr_t>(part)) & 15) == 0;
     int rc = dtype == GPT_DTYPE_BF16
-                 ? launch_overlapped(colsum_rows_kernel<bf16>, g1, b, 0, s, static_cast<const bf16*>(y), rows, C, part)
+                 ? launch_overlapped(colsum_rows_kernel<bf16>, g1, b, 0, s, static_cast<const bf16*>(y), rows, C, part,
+                                     vec)
                  : launch_overlapped(colsum_rows_kernel<float>, g1, b, 0, s, static_cast<const float*>(y), rows, C,
-                                     part);
+                                     part, vec);
     if (rc) return rc;
     return launch_overlapped(colsum_parts_kernel, dim3((C + 31) / 32), dim3(32, 8), 0, s,
                              static_cast<const float*>(part), static_cast<long long>(C), n_part, C, out, accumulate);

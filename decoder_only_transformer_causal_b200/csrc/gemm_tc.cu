@@ -80,22 +80,36 @@ __global__ void splitk_reduce_kernel(const float* __restrict__ part, int S, int 
     *o = d;
 }
 
-// Split count for an accumulating product with MN-major A: enough K ranges that the tiles fill
-// about two waves of a 148-SM part when the M x N tiles alone would not, each range non-empty.
+// Split count for an accumulating product with MN-major A: the S that minimises the modelled
+// time  P * ceil(tiles * S / 148) / S  +  2 * S * M * N * 4 / B  — the product's time P at full
+// occupancy of a 148-SM part, stretched by the wave quantisation of tiles * S CTAs, plus writing
+// and re-reading the S partial products at HBM bandwidth B — with every K range non-empty.
 // 1 = no split (also when M % 32 != 0 or N % 4 != 0).
-constexpr int kSplitTargetCtas = 296;
+constexpr int kSplitSms = 148;
 void split_plan(int M, int N, int K, int* splits, int* kb_per) {
-    const int tiles = ((M + gemm::BM - 1) / gemm::BM) * ((N + kBN - 1) / kBN);
+    const long long tiles = static_cast<long long>((M + gemm::BM - 1) / gemm::BM) * ((N + kBN - 1) / kBN);
     const int num_kb = (K + gemm::BK - 1) / gemm::BK;
     *splits = 1;
     *kb_per = num_kb;
-    if ((M % 32) || (N % 4) || tiles * 2 > kSplitTargetCtas || num_kb < 2) return;
-    int S = (kSplitTargetCtas + tiles - 1) / tiles;
-    S = S < num_kb ? S : num_kb;
-    S = S < 32 ? S : 32;
-    const int per = (num_kb + S - 1) / S;
-    *kb_per = per;
-    *splits = (num_kb + per - 1) / per;
+    if ((M % 32) || (N % 4) || tiles >= kSplitSms || num_kb < 2) return;
+    const double prod = 2.0 * M * N * K / 1.0e15;  // seconds at ~1 PFLOP/s
+    const double part = 2.0 * 4.0 * M * N / 5.0e12;  // seconds per split of partial traffic
+    double best = 1e30;
+    int best_s = 1;
+    const int s_max = num_kb < 32 ? num_kb : 32;
+    for (int S = 1; S <= s_max; ++S) {
+        const int per = (num_kb + S - 1) / S;
+        const int Se = (num_kb + per - 1) / per;  // non-empty ranges
+        if (Se != S) continue;
+        const double waves = static_cast<double>((tiles * S + kSplitSms - 1) / kSplitSms);
+        const double t = prod * waves * kSplitSms / (static_cast<double>(S) * tiles) + (S > 1 ? part * S : 0.0);
+        if (t < best * 0.999) {
+            best = t;
+            best_s = S;
+        }
+    }
+    *splits = best_s;
+    *kb_per = (num_kb + best_s - 1) / best_s;
 }
 
 }  // namespace
