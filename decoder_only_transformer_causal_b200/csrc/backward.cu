@@ -410,16 +410,6 @@ __global__ void colsum_rows_kernel(const E* __restrict__ y, int rows, int C, flo
 
 // dpre = dh * gelu'(pre): erf form Phi(z) + z phi(z); tanh form 0.5 (1 + tanh a) +
 // 0.5 z (1 - tanh^2 a) sqrt(2/pi) (1 + 3 * 0.044715 z^2), a = sqrt(2/pi) (z + 0.044715 z^3).
-// d gelu(z) / dz for either form
-GPT_DEVINL float gelu_slope(float z, int tanh_form) {
-    if (tanh_form) {
-        const float c = 0.7978845608028654f;
-        const float th = tanhf(c * (z + 0.044715f * z * z * z));
-        return 0.5f * (1.f + th) + 0.5f * z * (1.f - th * th) * c * (1.f + 3.f * 0.044715f * z * z);
-    }
-    return 0.5f * (1.f + erff(z * 0.7071067811865476f)) + z * 0.3989422804014327f * __expf(-0.5f * z * z);
-}
-
 template <typename E>
 __global__ void gelu_backward_kernel(const float* __restrict__ dh, const E* __restrict__ pre, E* __restrict__ dpre,
                                      long long n, int tanh_form, int vec) {

@@ -444,6 +444,17 @@ GPT_DEVINL void st8(float* p, const float (&f)[8]) {
     reinterpret_cast<float4*>(p)[1] = make_float4(f[4], f[5], f[6], f[7]);
 }
 
+// d gelu(z) / dz (CUDA's erff / tanhf): erf form Phi(z) + z phi(z); tanh form 0.5 (1 + tanh a) +
+// 0.5 z (1 - tanh^2 a) sqrt(2/pi) (1 + 3 * 0.044715 z^2), a = sqrt(2/pi) (z + 0.044715 z^3).
+GPT_DEVINL float gelu_slope(float z, int tanh_form) {
+    if (tanh_form) {
+        const float c = 0.7978845608028654f;
+        const float th = tanhf(c * (z + 0.044715f * z * z * z));
+        return 0.5f * (1.f + th) + 0.5f * z * (1.f - th * th) * c * (1.f + 3.f * 0.044715f * z * z);
+    }
+    return 0.5f * (1.f + erff(z * 0.7071067811865476f)) + z * 0.3989422804014327f * __expf(-0.5f * z * z);
+}
+
 // Records a device-side status (first writer wins).
 GPT_DEVINL void set_status(int32_t* status, int32_t code) {
     if (status) atomicCAS(reinterpret_cast<int*>(status), 0, code);

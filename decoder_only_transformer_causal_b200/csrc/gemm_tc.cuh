@@ -37,10 +37,12 @@ constexpr int NEPI = 8;  // epilogue warps: two per TMEM lane quarter, each half
 
 // EPI_F32: out_fp32 = acc, plain store (a backward product, or the partial products of a split-K
 //          launch).
-// EPI_DGELU: out_bf16 = acc * gelu'(aux), aux the bf16 pre-activation [M, ld_aux] (the MLP's
-//          backward through GELU, fused into the product that yields d loss / d gelu output).
-// EPI_GELU2: pre = acc + b at rows [0, M) of out and gelu(acc + b) at rows [M, 2M) (the training
-//          forward keeps both for the backward; M % 32 == 0).
+// EPI_DGELU: out_bf16 = acc * aux, aux the bf16 GELU derivative [M, ld_aux] that the training
+//          forward stored (the MLP's backward through GELU, fused into the product that yields
+//          d loss / d gelu output).
+// EPI_GELU2: gelu'(acc + b) at rows [0, M) of out and gelu(acc + b) at rows [M, 2M) (the training
+//          forward keeps the GELU output for the weight gradient and its derivative for the
+//          backward through GELU; M % 32 == 0).
 enum Epi { EPI_STORE = 0, EPI_GELU = 1, EPI_RESID = 2, EPI_CE = 3, EPI_F32 = 4, EPI_DGELU = 5, EPI_GELU2 = 6 };
 
 struct Params {
@@ -95,19 +97,18 @@ GPT_DEVINL float rcp_approx(float x) {
     return y;
 }
 
-// d gelu(x) / dx with the same building blocks as gelu_f:
-//  erf form:  Phi(x) + x phi(x), phi(x) = exp(-x^2 / 2) / sqrt(2 pi) (the exponential the erf
-//             formula already takes);
-//  tanh form: 0.5 (1 + th) + 0.5 x (1 - th^2) sqrt(2/pi) (1 + 3 * 0.044715 x^2), th = tanh(u),
-//             tanh(u) = 1 - 2 / (1 + exp(2u)).
+// gelu(x) and gelu'(x) together, sharing the erf evaluation (or tanh's exponential).
 template <int TANH>
-GPT_DEVINL float gelu_grad_f(float x) {
+GPT_DEVINL void gelu_pair_f(float x, float& g, float& dg) {
     constexpr float kLog2e = 1.4426950408889634f;
     if (TANH) {
         const float c = 0.7978845608028654f;
         const float u = c * x * fmaf(0.044715f * x, x, 1.0f);
-        const float th = 1.0f - 2.0f * rcp_approx(1.0f + exp2_approx(2.0f * u * kLog2e));
-        return 0.5f * (1.0f + th) + 0.5f * x * (1.0f - th * th) * c * fmaf(3.0f * 0.044715f * x, x, 1.0f);
+        const float r = rcp_approx(1.0f + exp2_approx(2.0f * u * kLog2e));  // (1 - tanh u) / 2
+        const float th = 1.0f - 2.0f * r;
+        g = x * (1.0f - r);
+        dg = 0.5f * (1.0f + th) + 0.5f * x * (1.0f - th * th) * c * fmaf(3.0f * 0.044715f * x, x, 1.0f);
+        return;
     }
     const float z = fabsf(x) * 0.7071067811865476f;
     const float t = rcp_approx(fmaf(0.3275911f, z, 1.0f));
@@ -117,8 +118,9 @@ GPT_DEVINL float gelu_grad_f(float x) {
     q = fmaf(t, q, 0.254829592f);
     q *= t;
     const float e = exp2_approx(-z * z * kLog2e);  // exp(-x^2 / 2)
-    const float erf_abs = fmaf(-q, e, 1.0f);
-    return 0.5f * (1.0f + copysignf(erf_abs, x)) + x * 0.3989422804014327f * e;
+    const float phi_cdf = 0.5f * (1.0f + copysignf(fmaf(-q, e, 1.0f), x));
+    g = x * phi_cdf;
+    dg = phi_cdf + x * 0.3989422804014327f * e;
 }
 
 template <int TANH>
@@ -495,7 +497,7 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)  // 10 warps: <= 168 regi
                                 aux_ok = true;
                             }
 #pragma unroll
-                            for (int j = 0; j < 32; ++j) v[j] *= gelu_grad_f<GELU_TANH>(z[j]);
+                            for (int j = 0; j < 32; ++j) v[j] *= z[j];
                         }
                         if (EPI == EPI_CE) {
                             float cmax = -INFINITY;
@@ -532,10 +534,20 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)  // 10 warps: <= 168 regi
                         }
                         if (!band_ok) continue;  // warp-uniform: no row of this band exists
 #pragma unroll
+                        float vg[EPI == EPI_GELU2 ? 32 : 1];  // EPI_GELU2: the GELU outputs of pass 1
+                        if (EPI == EPI_GELU2) {
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) {
+                                float g, dg;
+                                gelu_pair_f<GELU_TANH>(v[j], g, dg);
+                                v[j] = dg;
+                                vg[j] = g;
+                            }
+                        }
                         for (int pass = 0; pass < (EPI == EPI_GELU2 ? 2 : 1); ++pass) {
                             if (EPI == EPI_GELU2 && pass == 1) {
 #pragma unroll
-                                for (int j = 0; j < 32; ++j) v[j] = gelu_f<GELU_TANH>(v[j]);
+                                for (int j = 0; j < 32; ++j) v[j] = vg[j];
                             }
                             if (lane == 0) bulk_wait_read_all();  // the buffer's previous tile was read
                             __syncwarp();

@@ -1192,8 +1192,10 @@ GPT_API int gpt_forward_train(const gpt_config_t* cfg, const void* weights, cons
                                       static_cast<const float*>(W.bias(l, W_PROJ_B)), x_mid, C, N, C, C, GPT_EPI_RESID,
                                       cfg->gelu, s));
         GPT_TRY(launch_layernorm(x_mid, W.layer(l, W_LN2_W), W.bias(l, W_LN2_B), u2, N, C, dt, s));
-        // c_fc keeps both its pre-activation (for the GELU derivative) and the GELU output: one
-        // product writing both when h directly follows pre (bf16), else a store and a GELU pass.
+        // c_fc keeps the GELU output (for the weight gradient) and, in the bf16 path, the GELU
+        // derivative at the pre-activation in `pre` (for the backward through GELU): one product
+        // writing both when h directly follows pre, else a store, a GELU pass and an in-place
+        // derivative pass.  The fp32 path keeps the pre-activation itself.
         const bool two_out = bf && (N % 32 == 0) &&
                              static_cast<uint8_t*>(hh) == static_cast<uint8_t*>(pre) + static_cast<size_t>(N) * 4 * C * es;
         if (two_out)
@@ -1208,8 +1210,12 @@ GPT_API int gpt_forward_train(const gpt_config_t* cfg, const void* weights, cons
             GPT_TRY(launch_linear_f32(static_cast<const float*>(u2), C, static_cast<const float*>(W.layer(l, W_FC_W)),
                                       static_cast<const float*>(W.bias(l, W_FC_B)), static_cast<float*>(pre), 4LL * C, N,
                                       4 * C, C, GPT_EPI_STORE, cfg->gelu, s));
-        if (!two_out)
+        if (!two_out) {
             GPT_TRY(launch_gelu_forward(pre, hh, static_cast<long long>(N) * 4 * C, dt, cfg->gelu == GPT_GELU_TANH, s));
+            if (bf)
+                GPT_TRY(launch_gelu_deriv_inplace(pre, static_cast<long long>(N) * 4 * C, dt,
+                                                  cfg->gelu == GPT_GELU_TANH, s));
+        }
         GPT_TRY(cuda_status(cudaMemcpyAsync(x_out, x_mid, static_cast<size_t>(N) * C * 4, cudaMemcpyDeviceToDevice, s)));
         if (bf)
             GPT_TRY(launch_gemm_bf16(static_cast<const bf16*>(hh), 4LL * C, static_cast<const bf16*>(W.layer(l, W_FC2_W)),
@@ -1328,8 +1334,9 @@ GPT_API int gpt_backward(const gpt_config_t* cfg, const void* weights, const int
                                       cfg->bias ? G(count - 1) : nullptr, 1, parts, N, C, s, dx16));
     for (int l = cfg->n_layer - 1; l >= 0; --l) {
         const uint8_t* L = ab + A.layer * l;
-        // mlp c_proj, then GELU: dpre = (dx W_fc2) * gelu'(pre) (bf16: one fused product; fp32: dh
-        // into d1, then the GELU backward); dW_fc2 += dx^T h; db_fc2 += sum dx
+        // mlp c_proj, then GELU: dpre = (dx W_fc2) * gelu'(pre) (bf16: one fused product reading the
+        // derivative the forward stored; fp32: dh into d1, then the GELU backward from the
+        // pre-activation); dW_fc2 += dx^T h; db_fc2 += sum dx
         if (bf) {
             GPT_TRY(linear_bwd(gx, C, L + A.h, 4LL * C, W.layer(l, W_FC2_W), C, 4 * C, dpre, GEMM_BWD_DGELU_BF16,
                                L + A.pre, GL(l, W_FC2_W), gT));

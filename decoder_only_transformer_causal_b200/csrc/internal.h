@@ -96,7 +96,8 @@ struct CeArgs {
     int n_part;
 };
 int gemm_ce_parts(int N);  // partial slots per row of the lm_head epilogue
-// launch_gemm_bf16 epilogue beyond GPT_EPI_*: out bf16 [2M, ldo] = {acc + b; gelu(acc + b)}, M % 32 == 0.
+// launch_gemm_bf16 epilogue beyond GPT_EPI_*: out bf16 [2M, ldo] = {gelu'(acc + b); gelu(acc + b)},
+// M % 32 == 0.
 constexpr int GEMM_EPI_GELU2 = 6;
 int launch_gemm_bf16(const bf16* A, long long lda, const bf16* W, long long ldw, const bf16* bias,
                      void* out, long long ldo, int M, int N, int K, int epilogue, int gelu,
@@ -115,7 +116,7 @@ size_t gemm_acc_split_bytes(int M, int N, int K);
 //   GEMM_BWD_ACC_F32     out fp32 += A B^T (a_mn allowed; split-K as launch_gemm_bf16_acc)
 //   GEMM_BWD_STORE_F32   out fp32  = A B^T
 //   GEMM_BWD_STORE_BF16  out bf16  = A B^T
-//   GEMM_BWD_DGELU_BF16  out bf16  = (A B^T) * gelu'(aux), aux bf16 [M, ld_aux] (gelu = GPT_GELU_*)
+//   GEMM_BWD_DGELU_BF16  out bf16  = (A B^T) * aux, aux bf16 [M, ld_aux] the stored GELU derivative
 enum { GEMM_BWD_ACC_F32 = 0, GEMM_BWD_STORE_F32 = 1, GEMM_BWD_STORE_BF16 = 2, GEMM_BWD_DGELU_BF16 = 3 };
 int launch_gemm_bf16_bwd(const bf16* A, long long lda, bool a_mn, const bf16* W, long long ldw, bool b_mn, void* out,
                          long long ldo, int M, int N, int K, int mode, const bf16* aux, long long ld_aux, int gelu,
@@ -215,6 +216,7 @@ int launch_transpose(const void* in, int in_dtype, long long ld_in, void* out, i
                      int Cc, cudaStream_t s);
 int launch_convert(const void* in, int in_dtype, void* out, int out_dtype, long long n, cudaStream_t s);
 int launch_gelu_forward(const void* pre, void* h, long long n, int dtype, int tanh_form, cudaStream_t s);
+int launch_gelu_deriv_inplace(void* pre, long long n, int dtype, int tanh_form, cudaStream_t s);
 // scratch: attn_bwd_scratch_bytes(B, nh, T) bytes, 16-byte aligned (D and lse2 padded to a multiple
 // of 128 rows per head).  Exactly one of Lb / Lf is non-null; hs 32 or 64.  status: optional device
 // word that records GPT_ERR_TIMEOUT from the tensor-core kernels.

@@ -88,6 +88,25 @@ __global__ void gelu_forward_kernel(const E* __restrict__ pre, E* __restrict__ h
     for (long long i = i0; i < n && i < i0 + 8; ++i) h[i] = stf<E>(gelu_value(ldf(pre + i), tanh_form));
 }
 
+// pre <- gelu'(pre) in place (the training forward's fallback when c_fc cannot write both outputs
+// in one epilogue: the backward reads the derivative, not the pre-activation).
+template <typename E>
+__global__ void gelu_deriv_inplace_kernel(E* __restrict__ pre, long long n, int tanh_form, int vec) {
+    griddep_launch_dependents();
+    griddep_wait();
+    const long long i0 = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) * 8;
+    if (i0 >= n) return;
+    if (vec && i0 + 8 <= n) {
+        float v[8];
+        ld8(pre + i0, v);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[e] = gelu_slope(v[e], tanh_form);
+        st8(pre + i0, v);
+        return;
+    }
+    for (long long i = i0; i < n && i < i0 + 8; ++i) pre[i] = stf<E>(gelu_slope(ldf(pre + i), tanh_form));
+}
+
 // ------------------------------------------------------------------ attention backward
 // Per (b, h) and query row i < Tp (Tp = T rounded up to 128): D[bh * Tp + i] = sum_d dO_i[d] O_i[d]
 // and L2[bh * Tp + i] = the forward's lse2_i; rows i >= T hold D = 0 and L2 = +inf (p = 0 there).
@@ -356,6 +375,17 @@ int launch_gelu_forward(const void* pre, void* h, long long n, int dtype, int ta
                                  static_cast<bf16*>(h), n, tanh_form, vec);
     return launch_overlapped(gelu_forward_kernel<float>, grid, block, 0, s, static_cast<const float*>(pre),
                              static_cast<float*>(h), n, tanh_form, vec);
+}
+
+int launch_gelu_deriv_inplace(void* pre, long long n, int dtype, int tanh_form, cudaStream_t s) {
+    if (n == 0) return GPT_OK;
+    const dim3 grid = grid8(n), block(256);
+    const int vec = al16(pre);
+    if (dtype == GPT_DTYPE_BF16)
+        return launch_overlapped(gelu_deriv_inplace_kernel<bf16>, grid, block, 0, s, static_cast<bf16*>(pre), n,
+                                 tanh_form, vec);
+    return launch_overlapped(gelu_deriv_inplace_kernel<float>, grid, block, 0, s, static_cast<float*>(pre), n,
+                             tanh_form, vec);
 }
 
 int launch_attention_backward(const AttnBwdLayout<bf16>* Lb, const AttnBwdLayout<float>* Lf, int B, int nh, int T,

@@ -410,7 +410,8 @@ int gpt_transpose(const void* in, int in_dtype, long long ld_in, void* out, int 
  * gpt_forward's computation and keeps what the backward needs in `acts`
  * (gpt_train_activation_bytes(cfg, B, T) bytes, 256-byte aligned; per layer the residual input,
  * both LayerNorm outputs, q/k/v, the attention output and its per-row log-sum-exp, the c_fc
- * pre-activation and the GELU output; then the final residual, ln_f's output, the logits and the
+ * pre-activation (bf16: GELU's derivative there, all the backward needs of it) and the GELU
+ * output; then the final residual, ln_f's output, the logits and the
  * {sum of row losses, counted rows} pair).  loss: device fp32 scalar.  workspace: as gpt_forward.
  * gpt_backward adds loss_scale * d(loss)/d(parameter) to grads (fp32, the flat element layout of
  * gpt_param_elems; zero it before the first micro-batch), reading acts; the tied head's and the
