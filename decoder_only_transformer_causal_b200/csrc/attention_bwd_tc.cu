@@ -16,9 +16,10 @@
 //   dQ kernel     outer = 128 queries, inner = the key tiles up to the diagonal.  S = Q K_n^T and
 //                 dP = dO V_n^T into TMEM; dS (bf16) goes back to TMEM and dQ += dS K_n takes it
 //                 as the A operand, K_n as an MN-major operand.
-// lse2 and D come from [B*nh, Tp] arrays (Tp = T rounded up to 128) whose padding holds
-// lse2 = +inf and D = 0, so queries past T get p = 0 with no test; the dK/dV kernel copies the
-// 64 entries of each query tile next to its Q / dO tiles with one bulk copy each.
+// -lse2 and D come from [B*nh, Tp] arrays (Tp = T rounded up to 128) whose padding holds
+// -lse2 = -inf and D = 0, so queries past T get p = 0 with no test; the dK/dV kernel copies the
+// 64 entries of each query tile next to its Q / dO tiles with one bulk copy each.  The row warps
+// form P and dS with packed f32x2 arithmetic.
 // Roles (192 threads, two CTAs per SM): warp 0 TMA producer, warp 1 MMA issuer (one thread),
 // warps 2-5 one outer row per thread.  TMEM (256 columns): dK/dV kernel S^T [0,64), dP^T
 // [64,128), dV [128,192), dK [192,256); dQ kernel S [0,64), dP [64,128), dQ [128,192),
@@ -62,7 +63,7 @@ struct Params {
     int qk_head_inner, o_head_inner;  // TMA coordinate order of the q/k/v maps and of the dO map
     bf16 *dq, *dk, *dv;
     long long sb, sh, st;             // element strides of dq / dk / dv (hs contiguous)
-    const float* lse2;                // [B*nh, Tp], padding +inf
+    const float* lse2;                // [B*nh, Tp]: -lse2 per query, padding -inf
     const float* D;                   // [B*nh, Tp], padding 0
     float scale_log2, inv_sqrt_hs;
     int32_t* status;
@@ -101,44 +102,50 @@ GPT_DEVINL void tmem_row_bf16(uint32_t taddr, float scale, uint32_t (&w)[32]) {
     }
 }
 
-// One 32-column half of a key row of the dK/dV kernel: P^T and dS^T for queries c0 + e.  MASK: the
-// tile touches the diagonal and columns c < cmin (queries before the key) are zero.
+// One 32-column half of a key row of the dK/dV kernel: P^T and dS^T for queries c0 + e, with packed
+// f32x2 arithmetic (one exponent FMA, one subtraction and one product per pair).  nl: the negated
+// lse2 per query; MASK: the tile touches the diagonal and columns c < cmin (queries before the key)
+// are zero.
 template <bool MASK>
-GPT_DEVINL void kv_half(const uint32_t (&su)[32], const uint32_t (&du)[32], const float* lv, const float* dv,
+GPT_DEVINL void kv_half(const uint32_t (&su)[32], const uint32_t (&du)[32], const float* nl, const float* dv,
                         float sc, int c0, int cmin, uint32_t* pw, uint32_t* dw) {
-    const float4* l4 = reinterpret_cast<const float4*>(lv + c0);
-    const float4* d4 = reinterpret_cast<const float4*>(dv + c0);
+    const uint64_t* nl2 = reinterpret_cast<const uint64_t*>(nl + c0);
+    const uint64_t* d2 = reinterpret_cast<const uint64_t*>(dv + c0);
+    const uint64_t SC = f2_pack(sc, sc);
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-        const float4 L = l4[q], Dq = d4[q];
-        const float ll[4] = {L.x, L.y, L.z, L.w}, dd[4] = {Dq.x, Dq.y, Dq.z, Dq.w};
-        float pp[4], ds[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int k = 4 * q + e;
-            pp[e] = exp2_approx(fmaf(__uint_as_float(su[k]), sc, -ll[e]));
-            if (MASK && c0 + k < cmin) pp[e] = 0.f;
-            ds[e] = pp[e] * (__uint_as_float(du[k]) - dd[e]);
-        }
-        pw[2 * q] = pack_bf16x2(pp[0], pp[1]);
-        pw[2 * q + 1] = pack_bf16x2(pp[2], pp[3]);
-        dw[2 * q] = pack_bf16x2(ds[0], ds[1]);
-        dw[2 * q + 1] = pack_bf16x2(ds[2], ds[3]);
+    for (int k = 0; k < 32; k += 2) {
+        float p0, p1;
+        f2_unpack(f2_fma(f2_pack(__uint_as_float(su[k]), __uint_as_float(su[k + 1])), SC, nl2[k / 2]), p0, p1);
+        p0 = exp2_approx(p0);
+        p1 = exp2_approx(p1);
+        if (MASK && c0 + k < cmin) p0 = 0.f;
+        if (MASK && c0 + k + 1 < cmin) p1 = 0.f;
+        const uint64_t pp = f2_pack(p0, p1);
+        float s0, s1;
+        f2_unpack(f2_mul(pp, f2_sub(f2_pack(__uint_as_float(du[k]), __uint_as_float(du[k + 1])), d2[k / 2])), s0, s1);
+        pw[k / 2] = pack_bf16x2(p0, p1);
+        dw[k / 2] = pack_bf16x2(s0, s1);
     }
 }
 
-// One 32-column half of a query row of the dQ kernel: dS for keys c0 + e.  MASK: columns c > cmax
-// (keys after the query) are zero.
+// One 32-column half of a query row of the dQ kernel: dS for keys c0 + e (packed f32x2).  nlse: the
+// row's negated lse2; MASK: columns c > cmax (keys after the query) are zero.
 template <bool MASK>
 GPT_DEVINL void q_half(const uint32_t (&su)[32], const uint32_t (&du)[32], float sc, float nlse, float Di, int c0,
                        int cmax, uint32_t* dw) {
+    const uint64_t SC = f2_pack(sc, sc), NL = f2_pack(nlse, nlse), DD = f2_pack(Di, Di);
 #pragma unroll
     for (int e = 0; e < 32; e += 2) {
-        float p0 = exp2_approx(fmaf(__uint_as_float(su[e]), sc, nlse));
-        float p1 = exp2_approx(fmaf(__uint_as_float(su[e + 1]), sc, nlse));
+        float p0, p1;
+        f2_unpack(f2_fma(f2_pack(__uint_as_float(su[e]), __uint_as_float(su[e + 1])), SC, NL), p0, p1);
+        p0 = exp2_approx(p0);
+        p1 = exp2_approx(p1);
         if (MASK && c0 + e > cmax) p0 = 0.f;
         if (MASK && c0 + e + 1 > cmax) p1 = 0.f;
-        dw[e / 2] = pack_bf16x2(p0 * (__uint_as_float(du[e]) - Di), p1 * (__uint_as_float(du[e + 1]) - Di));
+        float s0, s1;
+        f2_unpack(f2_mul(f2_pack(p0, p1), f2_sub(f2_pack(__uint_as_float(du[e]), __uint_as_float(du[e + 1])), DD)),
+                  s0, s1);
+        dw[e / 2] = pack_bf16x2(s0, s1);
     }
 }
 
@@ -295,7 +302,7 @@ __global__ void __launch_bounds__(THREADS, 2)
                 break;
             }
             tc_fence_after();
-            const float* lv = vlse + st * BN;
+            const float* lv = vlse + st * BN;  // negated lse2 of the tile's queries
             const float* dv = vD + st * BN;
             const int cmin = r - n * BN;  // key k0 + r sees query k0 + n*64 + c iff c >= cmin
             uint32_t pw[32], dw[32];
@@ -477,7 +484,7 @@ __global__ void __launch_bounds__(THREADS, 2)
         const uint32_t tS = tmem + lane_off, tdP = tmem + 64 + lane_off, tdS = tmem + 192 + lane_off;
         const float sc = p.scale_log2;
         const long long vi = static_cast<long long>(bh) * p.Tp + i;  // i < Tp: Tp is a multiple of 128
-        const float nlse = -__ldcg(p.lse2 + vi);
+        const float nlse = __ldcg(p.lse2 + vi);  // stored negated
         const float Di = __ldcg(p.D + vi);
         bool ok = true;
         for (int n = 0; n < nk; ++n) {

@@ -109,7 +109,8 @@ __global__ void gelu_deriv_inplace_kernel(E* __restrict__ pre, long long n, int 
 
 // ------------------------------------------------------------------ attention backward
 // Per (b, h) and query row i < Tp (Tp = T rounded up to 128): D[bh * Tp + i] = sum_d dO_i[d] O_i[d]
-// and L2[bh * Tp + i] = the forward's lse2_i; rows i >= T hold D = 0 and L2 = +inf (p = 0 there).
+// and L2[bh * Tp + i] = -lse2_i (the forward's, negated for the tensor-core kernels' exponent FMA);
+// rows i >= T hold D = 0 and L2 = -inf (p = 0 there).
 // hs / 8 threads per row, each with one 8-value slice of dO_i and O_i (16-byte loads when `vec`);
 // the slices meet in shuffles within the row's lane group.
 template <typename E>
@@ -142,7 +143,7 @@ __global__ void attn_bwd_rowdot_kernel(const AttnBwdLayout<E> L, int B, int nh, 
     for (int off = G / 2; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
     if (valid && part == 0) {
         D[row] = i < T ? s : 0.f;
-        L2[row] = i < T ? __ldcg(L.lse + static_cast<long long>(bh) * T + i) : INFINITY;
+        L2[row] = i < T ? -__ldcg(L.lse + static_cast<long long>(bh) * T + i) : -INFINITY;
     }
 }
 
