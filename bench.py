@@ -435,10 +435,10 @@ def adamw_bench(model, native, dev, stream, peaks, peak_src, steps: int = 20, wa
 
 
 def backward_pieces_bench(native, dev, stream, peaks, peak_src, reps: int = 10):
-    """The largest backward steps that are not matrix products, at the GPT-2 124M shapes
-    ("nanoGPT 全局流程图" 3.4): the cross-entropy gradient over the full logits [12288, 50304] bf16
-    (reads the logits twice, writes the gradient: 3 x 1.24 GB) and one LayerNorm backward
-    [12288, 768] (reads dy and x, reads and writes dx: 4 x 37.7 MB).  Inputs exceed the L2."""
+    """Backward steps at the GPT-2 124M shapes ("nanoGPT 全局流程图" 3.4): the cross-entropy gradient
+    over the full logits [12288, 50304] bf16 (reads the logits twice, writes the gradient:
+    3 x 1.24 GB), one LayerNorm backward [12288, 768] (reads dy and x, reads and writes dx:
+    4 x 37.7 MB) and the attention backward of one layer.  Inputs exceed the L2."""
     rows, V, C = 12 * 1024, 50304, 768
     g = torch.Generator(device=dev).manual_seed(3)
     z = (torch.randn((rows, V), device=dev, generator=g) * 1.5).to(torch.bfloat16)
@@ -451,11 +451,22 @@ def backward_pieces_bench(native, dev, stream, peaks, peak_src, reps: int = 10):
     dx = torch.zeros_like(x)
     dw = torch.empty(C, device=dev)
     db = torch.empty(C, device=dev)
+    # attention backward at the attention workload (B 12, 12 heads, T 1024, hs 64): algorithmic work
+    # = the five products of the flash backward (S recomputed, dP, dV, dQ, dK) over the causal pairs,
+    # 5 * 2 * hs * T (T + 1) / 2 per (b, h); the kernels run seven (S and dP in both passes).
+    Ba, nh, T, hs = 12, 12, 1024, 64
+    q, k, v, do_ = (torch.randn((Ba, nh, T, hs), device=dev, generator=g).to(torch.bfloat16) for _ in range(4))
+    y, lse = native.attention_train(q, k, v)
+    dqkv = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
+    aws = native.alloc_workspace(native.LIB.gpt_attention_backward_workspace_bytes(Ba, nh, T), dev)
+    attn_flops = 5 * 2 * hs * T * (T + 1) / 2 * Ba * nh
     out = {}
     for name, fn, nbytes in (
             ("cross_entropy_backward", lambda: native.cross_entropy_backward(z, tgt, sc, dlogits=dz), 3 * rows * V * 2),
             ("layernorm_backward", lambda: native.layernorm_backward(dy, x, w, dx=dx, accumulate=True, dw=dw, db=db),
-             4 * rows * C * 4)):
+             4 * rows * C * 4),
+            ("attention_backward", lambda: native.attention_backward(q, k, v, y, do_, lse, out=dqkv, workspace=aws),
+             None)):
         for _ in range(3):
             fn()
         torch.cuda.synchronize()
@@ -466,6 +477,13 @@ def backward_pieces_bench(native, dev, stream, peaks, peak_src, reps: int = 10):
         e1.record(stream)
         torch.cuda.synchronize()
         ms = e0.elapsed_time(e1) / reps
+        if nbytes is None:
+            tf = attn_flops / (ms / 1000.0) / 1e12
+            out[name] = {"ms": ms, "workload": "causal attention backward B 12, 12 heads, T 1024, hs 64, bf16",
+                         "roofline": {"bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"],
+                                      "unit": "TFLOP/s", "frac": tf / peaks["bf16_tflops"], "flops": attn_flops,
+                                      "peak_source": peak_src}}
+            continue
         gbs = nbytes / (ms / 1000.0) / 1e9
         out[name] = {"ms": ms, "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                                             "frac": gbs / peaks["hbm_gbs"], "bytes": nbytes, "peak_source": peak_src}}

@@ -575,11 +575,13 @@ def attention_train(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, status=No
     return y, lse
 
 
-def attention_backward(q, k, v, o, dout, lse, stream=None):
-    """gpt_attention_backward: returns (dq, dk, dv) for [B, nh, T, hs] tensors."""
+def attention_backward(q, k, v, o, dout, lse, stream=None, out=None, workspace=None):
+    """gpt_attention_backward: returns (dq, dk, dv) for [B, nh, T, hs] tensors (into `out`, a
+    (dq, dk, dv) triple, and `workspace` when given)."""
     B, nh, T, hs = q.shape
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    ws = alloc_workspace(LIB.gpt_attention_backward_workspace_bytes(B, nh, T), q.device)
+    dq, dk, dv = out if out is not None else (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
+    ws = workspace if workspace is not None else alloc_workspace(
+        LIB.gpt_attention_backward_workspace_bytes(B, nh, T), q.device)
     _check(LIB.gpt_attention_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
                                       _ptr(dv), B, nh, T, hs, _dt(q), _ptr(ws), ws.numel(), _stream(stream)),
            "gpt_attention_backward")
