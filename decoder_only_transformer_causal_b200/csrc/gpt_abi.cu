@@ -945,7 +945,8 @@ GPT_API size_t gpt_attention_backward_workspace_bytes(int B, int nh, int T) {
 
 GPT_API int gpt_attention_backward(const void* q, const void* k, const void* v, const void* o, const void* dout,
                                    const float* lse, void* dq, void* dk, void* dv, int B, int nh, int T, int hs,
-                                   int dtype, void* workspace, size_t workspace_bytes, void* stream) {
+                                   int dtype, void* workspace, size_t workspace_bytes, int32_t* status,
+                                   void* stream) {
     if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !workspace) return GPT_ERR_NULL;
     if (B < 0 || nh < 0 || T < 0 || hs <= 0) return GPT_ERR_BAD_SHAPE;
     if (dtype != GPT_DTYPE_BF16 && dtype != GPT_DTYPE_F32) return GPT_ERR_BAD_SHAPE;
@@ -958,12 +959,12 @@ GPT_API int gpt_attention_backward(const void* q, const void* k, const void* v, 
         AttnBwdLayout<bf16> L{static_cast<const bf16*>(q), static_cast<const bf16*>(k), static_cast<const bf16*>(v),
                               sb, sh, hs, static_cast<const bf16*>(o), static_cast<const bf16*>(dout), sb, sh, hs,
                               static_cast<bf16*>(dq), static_cast<bf16*>(dk), static_cast<bf16*>(dv), lse};
-        return launch_attention_backward(&L, nullptr, B, nh, T, hs, D, nullptr, s);
+        return launch_attention_backward(&L, nullptr, B, nh, T, hs, D, status, s);
     }
     AttnBwdLayout<float> L{static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v), sb,
                            sh, hs, static_cast<const float*>(o), static_cast<const float*>(dout), sb, sh, hs,
                            static_cast<float*>(dq), static_cast<float*>(dk), static_cast<float*>(dv), lse};
-    return launch_attention_backward(nullptr, &L, B, nh, T, hs, D, nullptr, s);
+    return launch_attention_backward(nullptr, &L, B, nh, T, hs, D, status, s);
 }
 
 GPT_API size_t gpt_linear_backward_workspace_bytes(int rows, int n_out, int n_in, int dtype) {

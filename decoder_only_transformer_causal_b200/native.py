@@ -108,7 +108,7 @@ def _load() -> ctypes.CDLL:
         "gpt_attention_backward_workspace_bytes": (Z, [I, I, I]),
         "gpt_linear_backward_workspace_bytes": (Z, [I, I, I, I]),
         "gpt_linear_backward": (I, [P, P, P, I, I, I, I, P, P, P, Z, P, P]),
-        "gpt_attention_backward": (I, [P, P, P, P, P, P, P, P, P, I, I, I, I, D, P, Z, P]),
+        "gpt_attention_backward": (I, [P, P, P, P, P, P, P, P, P, I, I, I, I, D, P, Z, P, P]),
         "gpt_transpose": (I, [P, D, L, P, D, L, I, I, P]),
         "gpt_train_activation_bytes": (Z, [CFG, I, I]),
         "gpt_backward_workspace_bytes": (Z, [CFG, I, I]),
@@ -575,15 +575,16 @@ def attention_train(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, status=No
     return y, lse
 
 
-def attention_backward(q, k, v, o, dout, lse, stream=None, out=None, workspace=None):
+def attention_backward(q, k, v, o, dout, lse, stream=None, out=None, workspace=None, status=None):
     """gpt_attention_backward: returns (dq, dk, dv) for [B, nh, T, hs] tensors (into `out`, a
-    (dq, dk, dv) triple, and `workspace` when given)."""
+    (dq, dk, dv) triple, and `workspace` when given; `status`: optional device int32)."""
     B, nh, T, hs = q.shape
     dq, dk, dv = out if out is not None else (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
     ws = workspace if workspace is not None else alloc_workspace(
         LIB.gpt_attention_backward_workspace_bytes(B, nh, T), q.device)
     _check(LIB.gpt_attention_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
-                                      _ptr(dv), B, nh, T, hs, _dt(q), _ptr(ws), ws.numel(), _stream(stream)),
+                                      _ptr(dv), B, nh, T, hs, _dt(q), _ptr(ws), ws.numel(), _ptr(status),
+                                      _stream(stream)),
            "gpt_attention_backward")
     return dq, dk, dv
 

@@ -380,11 +380,13 @@ int gpt_attention_train(const void* q, const void* k, const void* v, void* y, fl
  * (dK/dV per 128-key tile, dQ per 128-query tile; P and dS rounded to bf16 as MMA operands);
  * everything else runs SIMT kernels.  Results are bit-reproducible (fixed summation order).
  * workspace: gpt_attention_backward_workspace_bytes(B, nh, T) bytes, 256-byte aligned (D and a
- * padded copy of lse). */
+ * padded copy of lse).  status: optional device int32 that receives GPT_ERR_TIMEOUT if a pipeline
+ * wait of the tensor-core kernels expires (as gpt_linear). */
 size_t gpt_attention_backward_workspace_bytes(int B, int nh, int T);
 int gpt_attention_backward(const void* q, const void* k, const void* v, const void* o, const void* dout,
                            const float* lse, void* dq, void* dk, void* dv, int B, int nh, int T, int hs,
-                           int dtype, void* workspace, size_t workspace_bytes, void* stream);
+                           int dtype, void* workspace, size_t workspace_bytes, int32_t* status,
+                           void* stream);
 
 /* Backward of nn.Linear y = x W^T + b ("nanoGPT 全局流程图", 3.4 反向传播):
  *   dx = dy W       fp32 [rows, n_in], overwritten

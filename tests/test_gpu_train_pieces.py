@@ -41,9 +41,11 @@ def test_attention_lse_and_backward(B, nh, T, hs, dtype):
     m = s.max(-1)
     ref_lse = (m + np.log(np.exp(s - m[..., None]).sum(-1))) / math.log(2.0)
     assert np.abs(f64(lse) - ref_lse).max() < (2e-3 if dtype == torch.bfloat16 else 1e-5)
-    dq, dk, dv = native.attention_backward(qd, kd, vd, y, gd, lse)
-    dq2, dk2, dv2 = native.attention_backward(qd, kd, vd, y, gd, lse)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    dq, dk, dv = native.attention_backward(qd, kd, vd, y, gd, lse, status=status)
+    dq2, dk2, dv2 = native.attention_backward(qd, kd, vd, y, gd, lse, status=status)
     assert torch.equal(dq, dq2) and torch.equal(dk, dk2) and torch.equal(dv, dv2)
+    assert int(status) == native.GPT_OK  # no pipeline wait expired
     rdq, rdk, rdv = ob.attention_backward(f64(dout), f64(q), f64(k), f64(v))
     # bf16: inputs, the forward output o and the results are bf16 (2^-9 relative each); the
     # recomputed probabilities use the bf16-path lse; fp32: accumulation order only
