@@ -717,7 +717,9 @@ def main():
                              "tflops": a_tf, "ms": a["ms"], "frac_of_bf16_peak": a_tf / peaks["bf16_tflops"],
                              "flops": a["work"], "peak_source": peak_src}
         line["kernels_ms_per_forward"] = {k: round(v, 4) for k, v in share.items()}
-    if rank == 0 and not args.no_kernels:
+    # Single-GPU measurements (decode, optimizer, backward pieces) run in the N = 1 line only, so
+    # that the other ranks of an N > 1 run do not idle in a collective while rank 0 works alone.
+    if rank == 0 and world == 1 and not args.no_kernels:
         line["decode"] = decode_bench(model, native, dev, stream, peaks, peak_src)
         line["adamw"] = adamw_bench(model, native, dev, stream, peaks, peak_src)
         line["backward_pieces"] = backward_pieces_bench(native, dev, stream, peaks, peak_src)
