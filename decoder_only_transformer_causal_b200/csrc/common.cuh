@@ -182,7 +182,8 @@ GPT_DEVINL void bulk_load_1d(void* dst, const void* src, uint32_t bytes, uint64_
 }
 
 // 2-D tensor load by either CTA of a pair for a 2-SM MMA: data into this CTA's shared memory, the
-// bytes counted on the barrier at cluster address `bar` (the leader CTA's).  No multicast.
+// bytes counted on the barrier at cluster address `bar` (the leader CTA's).  Each CTA's copy
+// lands in that CTA's own shared memory only.
 GPT_DEVINL void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint32_t bar, int x, int y) {
     asm volatile(
         "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
