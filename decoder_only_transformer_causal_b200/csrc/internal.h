@@ -214,7 +214,6 @@ struct AttnBwdLayout {
 };
 int launch_transpose(const void* in, int in_dtype, long long ld_in, void* out, int out_dtype, long long ld_out, int R,
                      int Cc, cudaStream_t s);
-int launch_convert(const void* in, int in_dtype, void* out, int out_dtype, long long n, cudaStream_t s);
 int launch_gelu_forward(const void* pre, void* h, long long n, int dtype, int tanh_form, cudaStream_t s);
 int launch_gelu_deriv_inplace(void* pre, long long n, int dtype, int tanh_form, cudaStream_t s);
 // scratch: attn_bwd_scratch_bytes(B, nh, T) bytes, 16-byte aligned (D and lse2 padded to a multiple

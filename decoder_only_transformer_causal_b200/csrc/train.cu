@@ -1,7 +1,7 @@
 // Kernels the training step adds around the tensor-core GEMM ("nanoGPT 全局流程图", 3.4 反向传播):
-// transposes / conversions that turn the Linear layers' backward products into the GEMM's
-// A[M,K] B[N,K]^T form, the GELU applied to a stored pre-activation, and the causal attention's
-// backward.
+// the transpose that gives the fp32 path's backward products their A[M,K] B[N,K]^T operands (the
+// bf16 path reads MN-major operands in place), the GELU and its derivative applied to a stored
+// pre-activation, and the causal attention's backward.
 //
 // Attention backward (per batch b, head h; s_ij = q_i . k_j, p_ij = 2^(s_ij * scale_log2 - lse2_i)
 // with lse2 the forward's per-row log2-sum-exp, so P is recomputed, never stored):
@@ -51,21 +51,6 @@ __global__ void transpose_kernel(const Ti* __restrict__ in, long long ld_in, To*
 
 // Elementwise kernels: thread t takes values [8t, 8t + 8) with 16-byte accesses when `vec` (every
 // buffer 16-byte aligned) and the group is whole, one value at a time otherwise.
-template <typename Ti, typename To>
-__global__ void convert_kernel(const Ti* __restrict__ in, To* __restrict__ out, long long n, int vec) {
-    griddep_launch_dependents();
-    griddep_wait();
-    const long long i0 = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) * 8;
-    if (i0 >= n) return;
-    if (vec && i0 + 8 <= n) {
-        float v[8];
-        ld8(in + i0, v);
-        st8(out + i0, v);
-        return;
-    }
-    for (long long i = i0; i < n && i < i0 + 8; ++i) out[i] = stf<To>(ldf(in + i));
-}
-
 GPT_DEVINL float gelu_value(float z, int tanh_form) {
     return tanh_form ? 0.5f * z * (1.f + tanhf(0.7978845608028654f * (z + 0.044715f * z * z * z)))
                      : 0.5f * z * (1.f + erff(z * 0.7071067811865476f));
@@ -348,24 +333,6 @@ namespace {
 bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 dim3 grid8(long long n) { return dim3(static_cast<unsigned>((n + 8LL * 256 - 1) / (8LL * 256))); }
 }  // namespace
-
-int launch_convert(const void* in, int in_dtype, void* out, int out_dtype, long long n, cudaStream_t s) {
-    if (n == 0) return GPT_OK;
-    const dim3 grid = grid8(n), block(256);
-    const int vec = al16(in) && al16(out);
-    const bool ib = in_dtype == GPT_DTYPE_BF16, ob = out_dtype == GPT_DTYPE_BF16;
-    if (!ib && ob)
-        return launch_overlapped(convert_kernel<float, bf16>, grid, block, 0, s, static_cast<const float*>(in),
-                                 static_cast<bf16*>(out), n, vec);
-    if (ib && !ob)
-        return launch_overlapped(convert_kernel<bf16, float>, grid, block, 0, s, static_cast<const bf16*>(in),
-                                 static_cast<float*>(out), n, vec);
-    if (ib)
-        return launch_overlapped(convert_kernel<bf16, bf16>, grid, block, 0, s, static_cast<const bf16*>(in),
-                                 static_cast<bf16*>(out), n, vec);
-    return launch_overlapped(convert_kernel<float, float>, grid, block, 0, s, static_cast<const float*>(in),
-                             static_cast<float*>(out), n, vec);
-}
 
 int launch_gelu_forward(const void* pre, void* h, long long n, int dtype, int tanh_form, cudaStream_t s) {
     if (n == 0) return GPT_OK;
