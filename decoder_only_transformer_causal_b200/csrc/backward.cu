@@ -64,7 +64,8 @@ GPT_DEVINL float wsum(float v) {
 template <typename E>
 __global__ void __launch_bounds__(kBwdWarps * 32)
     ce_backward_kernel(const E* __restrict__ z, const int64_t* __restrict__ targets, const double* __restrict__ sum_count,
-                       E* __restrict__ dz, int rows, int V, float scale, int32_t* status) {
+                       E* __restrict__ dz, int rows, int V, float scale, int32_t* status,
+                       const float* __restrict__ row_lse) {
     griddep_launch_dependents();
     griddep_wait();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -83,42 +84,47 @@ __global__ void __launch_bounds__(kBwdWarps * 32)
         for (int v = lane; v < V; v += 32) dr[v] = st1<E>(0.f);
         return;
     }
-    float m = -INFINITY, s = 0.f;
     constexpr int VW = 16 / sizeof(E);  // elements per 16-byte access
     const bool vec = (V % VW) == 0;     // rows are then 16-byte aligned
-    if (vec) {
-        for (int v = lane * VW; v < V; v += 32 * VW) {
-            float f[VW];
-            ld_vec(zr + v, f);
-            float mx = f[0];
-#pragma unroll
-            for (int e = 1; e < VW; ++e) mx = fmaxf(mx, f[e]);
-            const float mn = fmaxf(m, mx);
-            float add = 0.f;
-#pragma unroll
-            for (int e = 0; e < VW; ++e) add += __expf(f[e] - mn);
-            s = (m == -INFINITY ? 0.f : s * __expf(m - mn)) + add;
-            m = mn;
-        }
+    float lse;
+    if (row_lse) {
+        lse = __ldcg(row_lse + r);  // the forward's logsumexp of the row: one pass below
     } else {
-        for (int v = lane; v < V; v += 32) {
-            const float x = ld1(zr + v);
-            if (x > m) {
-                s = s * __expf(m - x) + 1.f;
-                m = x;
-            } else {
-                s += __expf(x - m);
+        float m = -INFINITY, s = 0.f;
+        if (vec) {
+            for (int v = lane * VW; v < V; v += 32 * VW) {
+                float f[VW];
+                ld_vec(zr + v, f);
+                float mx = f[0];
+#pragma unroll
+                for (int e = 1; e < VW; ++e) mx = fmaxf(mx, f[e]);
+                const float mn = fmaxf(m, mx);
+                float add = 0.f;
+#pragma unroll
+                for (int e = 0; e < VW; ++e) add += __expf(f[e] - mn);
+                s = (m == -INFINITY ? 0.f : s * __expf(m - mn)) + add;
+                m = mn;
+            }
+        } else {
+            for (int v = lane; v < V; v += 32) {
+                const float x = ld1(zr + v);
+                if (x > m) {
+                    s = s * __expf(m - x) + 1.f;
+                    m = x;
+                } else {
+                    s += __expf(x - m);
+                }
             }
         }
-    }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        const float m2 = __shfl_xor_sync(0xffffffffu, m, o), s2 = __shfl_xor_sync(0xffffffffu, s, o);
-        const float mm = fmaxf(m, m2);
-        s = (m == -INFINITY ? 0.f : s * __expf(m - mm)) + (m2 == -INFINITY ? 0.f : s2 * __expf(m2 - mm));
-        m = mm;
+        for (int o = 16; o > 0; o >>= 1) {
+            const float m2 = __shfl_xor_sync(0xffffffffu, m, o), s2 = __shfl_xor_sync(0xffffffffu, s, o);
+            const float mm = fmaxf(m, m2);
+            s = (m == -INFINITY ? 0.f : s * __expf(m - mm)) + (m2 == -INFINITY ? 0.f : s2 * __expf(m2 - mm));
+            m = mm;
+        }
+        lse = m + __logf(s);
     }
-    const float lse = m + __logf(s);
     const float inv_n = static_cast<float>(static_cast<double>(scale) / n);
     if (vec) {
         for (int v = lane * VW; v < V; v += 32 * VW) {
@@ -516,13 +522,13 @@ __global__ void embed_wpe_kernel(const float* __restrict__ dx, int B, int T, int
 }  // namespace
 
 int launch_ce_backward(const void* logits, int dtype, const int64_t* targets, const double* sum_count, void* dlogits,
-                       int rows, int V, int32_t* status, cudaStream_t s, float scale) {
+                       int rows, int V, int32_t* status, cudaStream_t s, float scale, const float* row_lse) {
     const dim3 grid((rows + kBwdWarps - 1) / kBwdWarps), block(kBwdWarps * 32);
     if (dtype == GPT_DTYPE_BF16)
         return launch_overlapped(ce_backward_kernel<bf16>, grid, block, 0, s, static_cast<const bf16*>(logits),
-                                 targets, sum_count, static_cast<bf16*>(dlogits), rows, V, scale, status);
+                                 targets, sum_count, static_cast<bf16*>(dlogits), rows, V, scale, status, row_lse);
     return launch_overlapped(ce_backward_kernel<float>, grid, block, 0, s, static_cast<const float*>(logits), targets,
-                             sum_count, static_cast<float*>(dlogits), rows, V, scale, status);
+                             sum_count, static_cast<float*>(dlogits), rows, V, scale, status, row_lse);
 }
 
 int layernorm_backward_parts(int rows, int C) {

@@ -1025,7 +1025,7 @@ namespace {
 // Activations the backward needs, per layer and at the end (N = B * T rows, E = storage type).
 struct ActPlan {
     size_t x_in, u1, qkv, y, lse, x_mid, u2, pre, h, layer;  // offsets within a layer's block
-    size_t final_off, x_f, u_f, logits, sum_count, total;
+    size_t final_off, x_f, u_f, logits, sum_count, row_lse, total;
 };
 
 ActPlan plan_acts(const gpt_config_t* c, long long B, long long T) {
@@ -1048,6 +1048,7 @@ ActPlan plan_acts(const gpt_config_t* c, long long B, long long T) {
     A.u_f = f; f += a256(N * C * es);
     A.logits = f; f += a256(N * static_cast<size_t>(c->vocab_size) * es);
     A.sum_count = f; f += 256;
+    A.row_lse = f; f += a256(N * 4);  // bf16: each row's logsumexp from the head's fp32 accumulators
     A.total = f;
     return A;
 }
@@ -1236,7 +1237,8 @@ GPT_API int gpt_forward_train(const gpt_config_t* cfg, const void* weights, cons
         CeArgs ce{targets, reinterpret_cast<float2*>(ws + P.part), reinterpret_cast<float*>(ws + P.tlogit), P.n_part};
         GPT_TRY(launch_gemm_bf16(static_cast<const bf16*>(u_f), C, static_cast<const bf16*>(W.wte()), C, nullptr, logits, V,
                                  N, V, C, 3 /* EPI_CE */, cfg->gelu, &ce, status, s));
-        GPT_TRY(launch_ce_rows_from_parts(ce.part, P.n_part, ce.tlogit, targets, N, V, rl, status, s));
+        GPT_TRY(launch_ce_rows_from_parts(ce.part, P.n_part, ce.tlogit, targets, N, V, rl, status, s,
+                                          reinterpret_cast<float*>(ab + A.row_lse)));
     } else {
         GPT_TRY(launch_linear_f32(static_cast<const float*>(u_f), C, static_cast<const float*>(W.wte()), nullptr,
                                   static_cast<float*>(logits), V, N, V, C, GPT_EPI_STORE, cfg->gelu, s));
@@ -1328,8 +1330,9 @@ GPT_API int gpt_backward(const gpt_config_t* cfg, const void* weights, const int
     GPT_TRY(cuda_status(cudaMemsetAsync(status, 0, sizeof(int32_t), s)));
     // d loss / d logits, then the tied head: du_f = dz wte, dwte += dz^T u_f
     if (!(loss_scale > 0.f) || !isfinite(loss_scale)) return GPT_ERR_BAD_SHAPE;
+    // bf16: d(logits) in one pass with the row logsumexp the forward kept; fp32: reduced here
     GPT_TRY(launch_ce_backward(ab + A.logits, dt, targets, reinterpret_cast<const double*>(ab + A.sum_count), dz, N, V,
-                               status, s, loss_scale));
+                               status, s, loss_scale, bf ? reinterpret_cast<const float*>(ab + A.row_lse) : nullptr));
     GPT_TRY(linear_bwd(dz, V, ab + A.u_f, C, W.wte(), V, C, d1, F32_OUT, nullptr, G(0), dzT));
     GPT_TRY(launch_layernorm_backward(d1, reinterpret_cast<const float*>(ab + A.x_f), W.lnf_w(), dt, dx, 0, G(count - 2),
                                       cfg->bias ? G(count - 1) : nullptr, 1, parts, N, C, s, dx16));

@@ -80,7 +80,8 @@ int launch_layernorm(const float* x, const void* w, const void* b, void* out, in
 // bf16 path: combine the lm_head epilogue's partials into per-row losses.
 int launch_ce_rows_from_parts(const float2* part, int n_part, const float* tlogit,
                               const int64_t* targets, int rows, int V, float* row_loss,
-                              int32_t* status, cudaStream_t s);
+                              int32_t* status, cudaStream_t s,
+                              float* row_lse = nullptr);
 // fp32 path: per-row losses straight from fp32 logits.
 int launch_ce_rows_from_logits(const float* logits, const int64_t* targets, int rows, int V,
                                float* row_loss, int32_t* status, cudaStream_t s);
@@ -186,8 +187,10 @@ int launch_adamw(const OptTable& tab, int dtype, float* params, const float* gra
                  float* norm_out, void* ws, cudaStream_t s);
 
 // ---- backward kernels of the non-matmul pieces (backward.cu)
+// row_lse (optional): each row's logsumexp from the forward; the gradient then takes one pass.
 int launch_ce_backward(const void* logits, int dtype, const int64_t* targets, const double* sum_count, void* dlogits,
-                       int rows, int V, int32_t* status, cudaStream_t s, float scale = 1.f);
+                       int rows, int V, int32_t* status, cudaStream_t s, float scale = 1.f,
+                       const float* row_lse = nullptr);
 int layernorm_backward_parts(int rows, int C);  // part: [parts, 2C] floats
 // dx16 (optional): a bf16 copy of the dx rows as written (the next products' operand).
 int launch_layernorm_backward(const float* dy, const float* x, const void* w, int dtype, float* dx, int accumulate,

@@ -118,7 +118,8 @@ __global__ void layernorm_kernel(const float* __restrict__ x, const To* __restri
 __global__ void ce_rows_from_parts_kernel(const float2* __restrict__ part, int n_part,
                                           const float* __restrict__ tlogit,
                                           const int64_t* __restrict__ targets, int rows, int V,
-                                          float* __restrict__ row_loss, int32_t* status) {
+                                          float* __restrict__ row_loss, int32_t* status,
+                                          float* __restrict__ row_lse) {
     griddep_launch_dependents();
     griddep_wait();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -143,7 +144,11 @@ __global__ void ce_rows_from_parts_kernel(const float2* __restrict__ part, int n
         if (q.y > 0.f) s += q.y * expf(q.x - m);
     }
     s = warp_sum(s);
-    if (lane == 0) row_loss[row] = m + logf(s) - tlogit[row];
+    if (lane == 0) {
+        const float l = m + logf(s);
+        row_loss[row] = l - tlogit[row];
+        if (row_lse) row_lse[row] = l;
+    }
 }
 
 __global__ void ce_rows_from_logits_kernel(const float* __restrict__ logits,
@@ -250,11 +255,11 @@ int launch_layernorm(const float* x, const void* w, const void* b, void* out, in
 
 int launch_ce_rows_from_parts(const float2* part, int n_part, const float* tlogit,
                               const int64_t* targets, int rows, int V, float* row_loss,
-                              int32_t* status, cudaStream_t s) {
+                              int32_t* status, cudaStream_t s, float* row_lse) {
     if (rows == 0) return GPT_OK;
     const unsigned blocks = (rows + kWarpsPerBlock - 1) / kWarpsPerBlock;
     return launch_overlapped(ce_rows_from_parts_kernel, dim3(blocks), dim3(32 * kWarpsPerBlock), 0, s, part, n_part,
-                             tlogit, targets, rows, V, row_loss, status);
+                             tlogit, targets, rows, V, row_loss, status, row_lse);
 }
 
 int launch_ce_rows_from_logits(const float* logits, const int64_t* targets, int rows, int V,

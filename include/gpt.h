@@ -413,7 +413,8 @@ int gpt_transpose(const void* in, int in_dtype, long long ld_in, void* out, int 
  * (gpt_train_activation_bytes(cfg, B, T) bytes, 256-byte aligned; per layer the residual input,
  * both LayerNorm outputs, q/k/v, the attention output and its per-row log-sum-exp, the c_fc
  * pre-activation (bf16: GELU's derivative there, all the backward needs of it) and the GELU
- * output; then the final residual, ln_f's output, the logits and the
+ * output; then the final residual, ln_f's output, the logits, each row's logsumexp (bf16: from
+ * the head's fp32 accumulators; the backward's d(logits) then takes one pass) and the
  * {sum of row losses, counted rows} pair).  loss: device fp32 scalar.  workspace: as gpt_forward.
  * gpt_backward adds loss_scale * d(loss)/d(parameter) to grads (fp32, the flat element layout of
  * gpt_param_elems; zero it before the first micro-batch), reading acts; the tied head's and the
