@@ -237,3 +237,40 @@ def test_backward_pieces_host_validation():
     assert Lb.gpt_embedding_backward_workspace_bytes(16, 1025) == 0                   # > 16384 positions
     assert Lb.gpt_embedding_backward(FAKE, FAKE, 16, 1025, 8, 10, FAKE, FAKE, FAKE, 1 << 30, None, None) \
         == native.GPT_ERR_UNSUPPORTED
+
+
+def test_training_products_host_validation():
+    """Workspace sizes and argument checks of the Linear and attention backward entry points
+    (all return before touching a device)."""
+    Lb = native.LIB
+    bf, f32 = native.GPT_DTYPE_BF16, native.GPT_DTYPE_F32
+    # attention backward: D and the negated lse, both padded to 128 rows per (b, h)
+    for B, nh, T in ((12, 12, 1024), (2, 3, 300), (1, 1, 1)):
+        tp = (T + 127) // 128 * 128
+        assert Lb.gpt_attention_backward_workspace_bytes(B, nh, T) == (2 * B * nh * tp * 4 + 255) // 256 * 256
+    assert Lb.gpt_attention_backward_workspace_bytes(0, 1, 1) == 0
+    assert Lb.gpt_attention_backward(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 8, 48, bf, FAKE,
+                                     1 << 20, None, None) == native.GPT_ERR_UNSUPPORTED       # hs 48
+    assert Lb.gpt_attention_backward(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 8, 64, bf, FAKE,
+                                     16, None, None) == native.GPT_ERR_WS_TOO_SMALL
+    assert Lb.gpt_attention_backward(None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 8, 64, bf, FAKE,
+                                     1 << 20, None, None) == native.GPT_ERR_NULL
+    # Linear backward: bf16 needs room for the split-K partials of narrow weight gradients
+    # (GPT-2's attn c_proj: 768 x 768 over 12,288 rows splits its K range), fp32 for the transposes
+    ws_split = Lb.gpt_linear_backward_workspace_bytes(12288, 768, 768, bf)
+    assert ws_split > 256 and (ws_split - 256) % (768 * 768 * 4) == 0
+    assert Lb.gpt_linear_backward_workspace_bytes(12288, 50304, 768, bf) == 256      # the head: enough tiles
+    r, o, i = 77, 40, 24
+    a = lambda n: (n + 255) // 256 * 256
+    assert Lb.gpt_linear_backward_workspace_bytes(r, o, i, f32) == 256 + a(i * o * 4) + a(o * r * 4) + a(i * r * 4)
+    assert Lb.gpt_linear_backward_workspace_bytes(0, 8, 8, bf) == 0
+    assert Lb.gpt_linear_backward_workspace_bytes(8, 8, 8, 7) == 0
+    ws = 1 << 20
+    assert Lb.gpt_linear_backward(None, FAKE, FAKE, 8, 8, 8, bf, FAKE, FAKE, FAKE, ws, None, None) == native.GPT_ERR_NULL
+    assert Lb.gpt_linear_backward(FAKE, FAKE, FAKE, 8, 0, 8, bf, FAKE, FAKE, FAKE, ws, None, None) \
+        == native.GPT_ERR_BAD_SHAPE
+    assert Lb.gpt_linear_backward(FAKE, FAKE, FAKE, 8, 12, 8, bf, FAKE, FAKE, FAKE, ws, None, None) \
+        == native.GPT_ERR_UNSUPPORTED                                                     # n_out % 8
+    assert Lb.gpt_linear_backward(FAKE, FAKE, FAKE, 64, 64, 64, f32, FAKE, FAKE, FAKE, 16, None, None) \
+        == native.GPT_ERR_WS_TOO_SMALL
+    assert Lb.gpt_linear_backward(FAKE, FAKE, FAKE, 0, 8, 8, bf, FAKE, FAKE, FAKE, ws, None, None) == native.GPT_OK
