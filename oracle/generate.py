@@ -11,7 +11,7 @@ Pages (cited by title and section):
   [速查表] "nanoGPT 核心代码速查表" (pgsm.cn): 七、关键函数签名,
            generate(idx, max_new_tokens, temperature, top_k) -> tokens.
 
-Readings taken where the pages leave a step open (each is listed in the design doc):
+Readings taken where the pages leave a step open:
   * The multinomial draw is inverse-CDF sampling with a uniform u in [0, 1) supplied by the
     caller: the drawn index is the smallest i with p_0 + ... + p_i > u.  The pages call
     torch.multinomial, whose internal random stream they do not define; passing u in makes

@@ -15,7 +15,7 @@ Pages (cited by title and section):
   [速查表]   "nanoGPT 核心代码速查表" (pgsm.cn): 三、Attention 计算步骤.
   [DummyGPT] "DummyGPTModel" page (paozippq.com): 参数规模分析, DummyLayerNorm comment.
 
-Readings taken where the pages are silent or disagree (each is listed in the design doc):
+Readings taken where the pages are silent or disagree:
   * GELU is x*Phi(x) with the exact normal CDF ([逐步详解] 4. MLP; nn.GELU() in [流程图]
     §2.5 (C)); the tanh form is offered as an explicit alternative mode.
   * cross-entropy skips targets equal to -1 and averages over the rest ([流程图] §3.2,

@@ -12,7 +12,7 @@ Pages (cited by title and section):
            rest, torch.optim.AdamW with betas (0.9, 0.95)).
   [代码解析] "nanoGPT 代码解析" (liaow.com wiki): configure_optimizers (the same grouping).
 
-Readings taken where the pages leave a step open (each is listed in the design doc):
+Readings taken where the pages leave a step open:
   * get_lr after lr_decay_iters: the page's code stops at the cosine branch but its comment
     (阶段3) and its plot hold the rate at min_lr; that is what is computed here.
   * AdamW is torch.optim.AdamW's algorithm (the page calls it): decoupled decay
