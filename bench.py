@@ -599,7 +599,8 @@ def main():
 
     w = seeded.WORKLOADS[WORKLOAD]
     cfg = GPTConfig.from_dict(w.model_dict())
-    model = GPT(cfg, seeded.make_weights(w.model_dict(), seed=seeded.BASE_SEED + 17 * rank, device=str(dev)), dev)
+    # replicated weights (the same draw on every rank); each rank's batch shard is its own draw
+    model = GPT(cfg, seeded.make_weights(w.model_dict(), seed=seeded.BASE_SEED + 17, device=str(dev)), dev)
     idx_h, tgt_h = seeded.make_tokens(w.batch, w.seq_len, w.token_high, seed=seeded.BASE_SEED + 100_000 + rank)
     idx, tgt = idx_h.to(dev), tgt_h.to(dev)
     ws = model.workspace(w.batch, w.seq_len)

@@ -71,10 +71,11 @@ def allreduce_grads(grads: torch.Tensor, group=None) -> torch.Tensor:
     return grads
 
 
-def train_step_sharded(trainer, idx: torch.Tensor, targets: torch.Tensor, group=None) -> float:
+def train_step_sharded(trainer, idx: torch.Tensor, targets: torch.Tensor, group=None) -> torch.Tensor:
     """One data-parallel training step of a Trainer on this rank's shard [B_r, T] (already on the
     rank's device): training forward, all-reduce of the loss terms, backward against the global
-    count, SUM all-reduce of the gradients, AdamW.  Returns the global mean loss (host float)."""
+    count, SUM all-reduce of the gradients, AdamW.  Returns the global mean loss as a device fp64
+    scalar (NaN when no row is counted), so consecutive steps queue without a host round trip."""
     from . import native
     cfg, w = trainer.model.cfg, trainer.model.weights
     B, T = idx.shape
@@ -85,5 +86,5 @@ def train_step_sharded(trainer, idx: torch.Tensor, targets: torch.Tensor, group=
     native.backward(cfg, w, idx, targets, trainer.acts, trainer.grads, trainer.bws)
     allreduce_grads(trainer.grads, group)
     trainer.opt.step(trainer.grads)
-    return global_loss(lt)
+    return lt[0] / lt[1]
 
