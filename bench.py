@@ -149,26 +149,40 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- CPU oracle timing
-def oracle_sample(w, T_sample: int, budget_s: float, max_reps: int = 1000):
+def host_cores() -> int:
+    """CPU cores this process may run on (its affinity mask)."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover - non-Linux hosts
+        return os.cpu_count() or 1
+
+
+def oracle_sample(w, T_sample: int, budget_s: float, max_reps: int = 1000, threads: int | None = None, W=None):
     """Times the fp64 oracle on one sequence of T_sample tokens of the workload (full depth,
-    full width, full vocabulary), repeated until budget_s has passed."""
-    import numpy as np  # noqa: F401
+    full width, full vocabulary), repeated until budget_s has passed.  threads: BLAS thread limit
+    (None: the library's default, one per core of the affinity mask).  Returns (times, threads
+    used by BLAS)."""
     import oracle
-    from threadpoolctl import threadpool_info
+    from threadpoolctl import threadpool_info, threadpool_limits
     cfg = w.model_dict()
-    W = seeded.to_f64(seeded.make_weights(cfg))
+    if W is None:
+        W = seeded.to_f64(seeded.make_weights(cfg))
     idx, tgt = seeded.make_tokens(1, T_sample, w.token_high)
     idx, tgt = idx.numpy(), tgt.numpy()
     times = []
-    t_end = time.perf_counter() + budget_s
-    while len(times) < max_reps:
-        t0 = time.perf_counter()
-        oracle.forward(W, cfg, idx, tgt, keep_logits=False)
-        times.append(time.perf_counter() - t0)
-        if time.perf_counter() > t_end:
-            break
-    threads = max([d.get("num_threads", 1) for d in threadpool_info()] + [1])
-    return times, threads
+    with threadpool_limits(limits=threads):
+        used = max([d.get("num_threads", 1) for d in threadpool_info()] + [1])
+        t_end = time.perf_counter() + budget_s
+        while len(times) < max_reps:
+            t0 = time.perf_counter()
+            oracle.forward(W, cfg, idx, tgt, keep_logits=False)
+            times.append(time.perf_counter() - t0)
+            if time.perf_counter() > t_end:
+                break
+    return times, used
+
+
+CPU_SAMPLE_T = 256   # tokens of the one sequence each oracle repetition runs (both CPU arms)
 
 
 # ---------------------------------------------------------------- reference arm
@@ -177,7 +191,7 @@ def run_reference(args):
     if rank != 0:
         return 0
     w = seeded.WORKLOADS[WORKLOAD]
-    T_sample = 64
+    T_sample = CPU_SAMPLE_T
     import oracle
     from threadpoolctl import threadpool_info
     cfg = w.model_dict()
@@ -191,6 +205,7 @@ def run_reference(args):
         oracle.forward(W, cfg, idx, tgt, keep_logits=False)
     dt = time.perf_counter() - t0
     threads = max([d.get("num_threads", 1) for d in threadpool_info()] + [1])
+    threads = min(threads, host_cores())
     value = T_sample * args.steps / dt
     sample = (f"one sequence of {T_sample} tokens of the workload (all {w.n_layer} layers, width "
               f"{w.n_embd}, vocab {w.vocab_size}) per step, fp64 numpy oracle")
@@ -254,13 +269,35 @@ def kernel_ops(w, native, dev, stream, only=None):
         return lambda: native.lm_head_loss(u, wte, tgt, workspace=ws, logits=logits, loss=loss, stream=stream)
 
     def layernorm():
-        x = rnd((N, C), 1.0, torch.float32)
+        # four input / output pairs (226 MB, more than the 126 MB L2) used in turn, so every
+        # launch reads its input from HBM
+        xs = [rnd((N, C), 1.0, torch.float32) for _ in range(4)]
         lw, lb = torch.ones(C, device=dev, dtype=bf), torch.zeros(C, device=dev, dtype=bf)
-        out = torch.empty((N, C), device=dev, dtype=bf)
-        return lambda: native.layernorm(x, lw, lb, out=out, stream=stream)
+        outs = [torch.empty((N, C), device=dev, dtype=bf) for _ in range(4)]
+        turn = [0]
+
+        def run():
+            i = turn[0] = (turn[0] + 1) % 4
+            native.layernorm(xs[i], lw, lb, out=outs[i], stream=stream)
+        return run
+
+    def embed():
+        # three (wte, x) sets (~380 MB) used in turn, so every launch reads and writes HBM
+        _, wpe = None, rnd((w.seq_len, C), 0.02)
+        wtes = [rnd((V, C), 0.02) for _ in range(3)]
+        xs = [torch.empty((w.batch, w.seq_len, C), device=dev) for _ in range(3)]
+        idx, _ = seeded.make_tokens(w.batch, w.seq_len, w.token_high)
+        idx = idx.to(dev)
+        turn = [0]
+
+        def run():
+            i = turn[0] = (turn[0] + 1) % 3
+            native.embed(wtes[i], wpe, idx, x=xs[i], stream=stream)
+        return run
 
     # name -> (factory, work per launch, bound, launches per forward, kernel function)
     specs = {
+        "embed": (embed, float(N * 8 + N * C * 2 + w.seq_len * C * 2 + N * C * 4), "hbm", 1),
         "gemm_c_attn": (lambda: gemm(C, 3 * C, native.GPT_EPI_STORE, bf), 2.0 * N * 3 * C * C, "tensor", L),
         "attention": (attention, attention_flops(w.batch, w.n_head, w.seq_len, hs), "tensor", L),
         "gemm_attn_proj_resid": (lambda: gemm(C, C, native.GPT_EPI_RESID, torch.float32), 2.0 * N * C * C,
@@ -287,6 +324,7 @@ KERNEL_OF = {
     "lm_head_ce": "gemm_bf16_tc<256, 3, 0, 0, 0, 1> (+ ce_rows, loss_finalize)",
     "attention": "attention_fwd_tc",
     "layernorm": "layernorm_kernel<bf16>",
+    "embed": "embed_kernel<bf16>",
 }
 
 
@@ -387,6 +425,40 @@ def decode_bench(model, native, dev, stream, peaks, peak_src, steps: int = 64, w
                            "batch": B, "prompt": 1,
                            "note": "host wall clock around gpt_generate with pinned host copies in and out; "
                                    "launched eagerly (no graph), one launch sequence per token"}
+    return out
+
+
+def head_last_bench(native, dev, stream, peaks, peak_src, reps: int = 20):
+    """The inference branch's head ("nanoGPT 全局流程图", §3.2 ④, logits [B, 1, V]): gpt_lm_head_last,
+    ln_f of each sequence's last residual row and the product with the tied wte, at the GPT-2
+    124M (B 12) and XL (B 4, the [4, 1, 50304] output of the XL configuration) shapes.  HBM-bound:
+    algorithmic bytes = wte once (V C bf16) + the B fp32 rows + ln_f weight and bias + the bf16
+    logits.  Two wte copies are used in turn so that no launch finds its table in the L2."""
+    out = {}
+    V = 50304
+    for name, B, C in (("gpt2", 12, 768), ("gpt2-xl", 4, 1600)):
+        g = torch.Generator(device=dev).manual_seed(13)
+        x = torch.randn((B, 1024, C), device=dev, generator=g)
+        wtes = [(0.02 * torch.randn((V, C), device=dev, generator=g)).to(torch.bfloat16) for _ in range(2)]
+        lw = torch.ones(C, device=dev, dtype=torch.bfloat16)
+        lb = torch.zeros(C, device=dev, dtype=torch.bfloat16)
+        logits = torch.empty((B, V), device=dev, dtype=torch.bfloat16)
+        turn = [0]
+
+        def run():
+            i = turn[0] = (turn[0] + 1) % 2
+            native.lm_head_last(x, lw, lb, wtes[i], logits=logits, stream=stream)
+        for _ in range(4):
+            run()
+        ms = time_region(run, reps, stream)
+        nbytes = V * C * 2 + B * C * 4 + 2 * C * 2 + B * V * 2
+        gbs = nbytes / (ms / 1000.0) / 1e9
+        out[name] = {"workload": f"ln_f + tied head of the last position, B {B}, C {C}, V {V}, bf16",
+                     "us_per_launch": ms * 1000.0,
+                     "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                  "frac": gbs / peaks["hbm_gbs"], "bytes_per_launch": nbytes,
+                                  "peak_source": peak_src}}
+        del x, wtes
     return out
 
 
@@ -513,33 +585,37 @@ def train_bench(native, dev, stream, world, rank, dist, steps: int = 5, warmup: 
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(steps):
-        step()
+        last = step()
     e1.record(stream)
     torch.cuda.synchronize()
     t = torch.tensor([e0.elapsed_time(e1) / steps], device=dev)
     if dist is not None:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     ms = float(t)
-    # phase split of one more (single-GPU) step
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
-    cfg = model.cfg
-    ev[0].record(stream)
-    native.forward_train(cfg, model.weights, idx, tgt, tr.acts, tr.fws, loss=tr.loss)
-    ev[1].record(stream)
-    tr.grads.zero_()
-    native.backward(cfg, model.weights, idx, tgt, tr.acts, tr.grads, tr.bws)
-    ev[2].record(stream)
-    tr.opt.step(tr.grads)
-    ev[3].record(stream)
-    torch.cuda.synchronize()
-    loss = float(tr.loss)
+    out = {"workload": f"GPT-2 124M training step, B {w.batch} x T {w.seq_len} per GPU, bf16 weights/activations, "
+                       "fp32 master weights and Adam moments" + (f", data-parallel over {world} GPUs" if world > 1 else ""),
+           "tokens_per_s": world * w.batch * w.seq_len / (ms / 1000.0), "ms_per_step": ms}
+    if world == 1:
+        # phase split of one more step (single GPU only: with N > 1 a step without the two
+        # all-reduces would let the replicated weights of the ranks diverge)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        cfg = model.cfg
+        ev[0].record(stream)
+        native.forward_train(cfg, model.weights, idx, tgt, tr.acts, tr.fws, loss=tr.loss)
+        ev[1].record(stream)
+        tr.grads.zero_()
+        native.backward(cfg, model.weights, idx, tgt, tr.acts, tr.grads, tr.bws)
+        ev[2].record(stream)
+        tr.opt.step(tr.grads)
+        ev[3].record(stream)
+        torch.cuda.synchronize()
+        out["phase_ms"] = {"forward_train": ev[0].elapsed_time(ev[1]), "backward": ev[1].elapsed_time(ev[2]),
+                           "adamw": ev[2].elapsed_time(ev[3])}
+        out["loss_after"] = float(tr.loss)
+    else:
+        out["loss_after"] = float(last)
     del tr, model
-    return {"workload": f"GPT-2 124M training step, B {w.batch} x T {w.seq_len} per GPU, bf16 weights/activations, "
-                        "fp32 master weights and Adam moments" + (f", data-parallel over {world} GPUs" if world > 1 else ""),
-            "tokens_per_s": world * w.batch * w.seq_len / (ms / 1000.0), "ms_per_step": ms,
-            "phase_ms": {"forward_train": ev[0].elapsed_time(ev[1]), "backward": ev[1].elapsed_time(ev[2]),
-                         "adamw": ev[2].elapsed_time(ev[3])},
-            "loss_after": loss}
+    return out
 
 
 def adamw_only(args):
@@ -718,9 +794,17 @@ def main():
                              "tflops": a_tf, "ms": a["ms"], "frac_of_bf16_peak": a_tf / peaks["bf16_tflops"],
                              "flops": a["work"], "peak_source": peak_src}
         line["kernels_ms_per_forward"] = {k: round(v, 4) for k, v in share.items()}
+        # the HBM-bound kernels against the copy bandwidth (inputs rotated past the L2)
+        line["memory_bound"] = {
+            k: {"kernel": KERNEL_OF[k], "us_per_launch": v["ms"] * 1000.0,
+                "achieved_gbs": v["work"] / (v["ms"] / 1000.0) / 1e9, "peak_gbs": peaks["hbm_gbs"],
+                "frac": v["work"] / (v["ms"] / 1000.0) / 1e9 / peaks["hbm_gbs"], "bytes_per_launch": v["work"],
+                "peak_source": peak_src}
+            for k, v in kt.items() if v["bound"] == "hbm"}
     # Single-GPU measurements (decode, optimizer, backward pieces) run in the N = 1 line only, so
     # that the other ranks of an N > 1 run do not idle in a collective while rank 0 works alone.
     if rank == 0 and world == 1 and not args.no_kernels:
+        line["last_position"] = head_last_bench(native, dev, stream, peaks, peak_src)
         line["decode"] = decode_bench(model, native, dev, stream, peaks, peak_src)
         line["adamw"] = adamw_bench(model, native, dev, stream, peaks, peak_src)
         line["backward_pieces"] = backward_pieces_bench(native, dev, stream, peaks, peak_src)
@@ -729,11 +813,18 @@ def main():
         if rank == 0:
             line["train"] = tr
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        times, threads = oracle_sample(w, 256, budget_s=12.0)
-        tok_s = 256 * len(times) / sum(times)
-        line["cpu_baseline"] = {"value": tok_s, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-                                "sample": f"{len(times)} x one sequence of 256 tokens of the workload (all "
-                                          f"{w.n_layer} layers, full vocab), fp64 numpy oracle"}
+        W64 = seeded.to_f64(seeded.make_weights(w.model_dict()))
+        cores = host_cores()
+        times, threads = oracle_sample(w, CPU_SAMPLE_T, budget_s=12.0, threads=cores, W=W64)
+        tok_s = CPU_SAMPLE_T * len(times) / sum(times)
+        t1, _ = oracle_sample(w, 64, budget_s=6.0, threads=1, W=W64)
+        line["cpu_baseline"] = {"value": tok_s, "unit": "tokens/s", "cores": min(threads, cores), "kind": "oracle",
+                                "host_cores": cores,
+                                "sample": f"{len(times)} x one sequence of {CPU_SAMPLE_T} tokens of the workload (all "
+                                          f"{w.n_layer} layers, full vocab), fp64 numpy oracle",
+                                "one_core": {"value": 64 * len(t1) / sum(t1), "unit": "tokens/s", "cores": 1,
+                                             "sample": f"{len(t1)} x one sequence of 64 tokens, BLAS limited to "
+                                                       "one thread"}}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist is not None:

@@ -620,4 +620,7 @@ int launch_attention_backward_tc(const AttnBwdLayout<bf16>& L, int B, int nh, in
                              v128, q64, g64, p);
 }
 
+// Pipeline-wait limit of this file's kernels on the current device (0: the default).
+GPT_DEFINE_WAIT_LIMIT_SETTER(set_wait_limit_attention_bwd)
+
 }  // namespace gpt

@@ -53,4 +53,7 @@ int launch_attention_bf16(const AttnLayout& L, int B, int nh, int T, int32_t* st
                              attn::SMEM_BYTES, s, tq, tk, tv, p);
 }
 
+// Pipeline-wait limit of this file's kernels on the current device (0: the default).
+GPT_DEFINE_WAIT_LIMIT_SETTER(set_wait_limit_attention)
+
 }  // namespace gpt

@@ -149,7 +149,10 @@ __global__ void __launch_bounds__(THREADS, 2)
             constexpr uint32_t idesc_s = make_idesc_bf16(BQ, BKV, false);
             constexpr uint32_t idesc_o = make_idesc_bf16(BQ, HS, true);
             const uint32_t tS = tmem + COL_S, tP = tmem + COL_P, tO = tmem + COL_O;
-            bool ok = mbar_wait(q_full, 0, abort_flag);
+            // Testing aid: nothing arrives on `drain` before the commit below, so this wait can only
+            // give up, which sends the whole CTA down its time-out path.
+            if (g_force_timeout) mbar_wait(drain, 0, abort_flag);
+            bool ok = !g_force_timeout && mbar_wait(q_full, 0, abort_flag);
             tc_fence_after();
             const uint32_t q_addr = smem_addr(sQ);
             for (int j = 0; ok && j <= n_kv; ++j) {

@@ -20,6 +20,24 @@ typedef __nv_bfloat16 bf16;
 // drains what it has in flight and returns instead of hanging.
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s
 
+// The limit the pipeline waits (mbar_wait, mbar_wait_cluster) apply on this device: kWaitLimitNs
+// unless gpt_set_wait_limit_ns lowered it (to exercise the time-out path).  Internal linkage: each
+// translation unit with pipeline waits holds its own copy and defines a setter for it with
+// GPT_DEFINE_WAIT_LIMIT_SETTER.  The drains on the way out (mbar_drain) always keep kWaitLimitNs,
+// so no kernel leaves a copy or a product in flight because of a lowered limit.
+static __device__ uint64_t g_wait_limit_ns = kWaitLimitNs;
+// Testing aid (same linkage): when nonzero, the MMA-issuing thread of the attention kernel and of
+// the product kernel first waits for an event that never happens, so that the time-out path runs
+// on purpose: nothing has arrived on the kernel's drain barrier before its final commit.
+static __device__ int g_force_timeout = 0;
+#define GPT_DEFINE_WAIT_LIMIT_SETTER(name)                                                       \
+    int name(unsigned long long ns, int force) {                                                 \
+        const uint64_t v = ns ? static_cast<uint64_t>(ns) : kWaitLimitNs;                       \
+        const int f = force ? 1 : 0;                                                             \
+        if (cudaMemcpyToSymbol(g_wait_limit_ns, &v, sizeof(v)) != cudaSuccess) return GPT_ERR_CUDA; \
+        return cudaMemcpyToSymbol(g_force_timeout, &f, sizeof(f)) == cudaSuccess ? GPT_OK : GPT_ERR_CUDA; \
+    }
+
 GPT_DEVINL uint32_t smem_addr(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -68,11 +86,12 @@ GPT_DEVINL bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_fl
     const uint32_t a = smem_addr(bar);
     if (mbar_try_wait(a, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
+    const uint64_t limit = g_wait_limit_ns;
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(a, parity)) return true;
         if ((it & 63u) == 0u) {
             if (*abort_flag) return false;
-            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            if (globaltimer_ns() - t0 > limit) {
                 *abort_flag = 1;
                 return false;
             }
@@ -96,11 +115,12 @@ GPT_DEVINL bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* 
     };
     if (try_wait()) return true;
     const uint64_t t0 = globaltimer_ns();
+    const uint64_t limit = g_wait_limit_ns;
     for (uint32_t it = 1;; ++it) {
         if (try_wait()) return true;
         if ((it & 63u) == 0u) {
             if (*abort_flag) return false;
-            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            if (globaltimer_ns() - t0 > limit) {
                 *abort_flag = 1;
                 return false;
             }
@@ -147,6 +167,32 @@ GPT_DEVINL uint32_t map_to_rank(const void* p, uint32_t rank) {
 // Arrive on a barrier of another CTA of the cluster.
 GPT_DEVINL void mbar_arrive_remote(uint32_t cluster_addr) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+// Stores a 64-bit value into another CTA's shared memory (cluster address).
+GPT_DEVINL void st_cluster_u64(uint32_t cluster_addr, unsigned long long v) {
+    asm volatile("st.shared::cluster.u64 [%0], %1;" ::"r"(cluster_addr), "l"(v) : "memory");
+}
+// Counts `bytes` as arrived on the barrier's current phase without a copy (cancels an expected
+// transfer that will never be issued).
+GPT_DEVINL void mbar_complete_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.complete_tx.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes) : "memory");
+}
+// A wait with only a time bound (no abort flag), acquiring at cluster scope; false on time-out.
+GPT_DEVINL bool mbar_wait_cluster_bounded(uint64_t* bar, uint32_t parity) {
+    const uint32_t a = smem_addr(bar);
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
+        uint32_t ok;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(a), "r"(parity)
+            : "memory");
+        if (ok) return true;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    }
 }
 
 // ------------------------------------------------------------------ TMA

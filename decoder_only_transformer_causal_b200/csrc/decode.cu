@@ -157,6 +157,7 @@ enum DecodeEpi {
     DV_RESID = 2,   // out fp32 [rows, N] += .
     DV_F32 = 3,     // out fp32 [rows, N]
     DV_QKV = 4,     // columns [0, C) -> out E (q); [C, 3C) -> kv[row, *pos, :] (k then v)
+    DV_STORE = 5,   // out E [rows, N]
 };
 
 GPT_DEVINL void store4(bf16* p, float a, float b, float c, float d) {
@@ -181,7 +182,9 @@ template <typename E, int EPI, int KSPLIT, int CPW, bool LN, int ROWS>
 __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const GemvArgs<E> a) {
     griddep_launch_dependents();
     // the weights never change: start bringing them into L2 while the previous kernel finishes
-    if (threadIdx.x == 0) prefetch_l2_share(a.W, static_cast<size_t>(a.N) * a.K * sizeof(E));
+    // (when each CTA takes one column group, its share of the prefetch is exactly its rows of W)
+    if (threadIdx.x == 0 && static_cast<long long>(gridDim.x) * ((kGemvWarps / KSPLIT) * CPW) >= a.N)
+        prefetch_l2_share(a.W, static_cast<size_t>(a.N) * a.K * sizeof(E));
     griddep_wait();
     extern __shared__ __align__(16) uint8_t gemv_smem[];
     E* xs = reinterpret_cast<E*>(gemv_smem);  // [rows][K]
@@ -298,6 +301,8 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const GemvArgs<E> a)
                     *o = __ldcg(o) + v;
                 } else if (EPI == DV_F32) {
                     static_cast<float*>(a.out)[r * a.ldo + n] = v;
+                } else if (EPI == DV_STORE) {
+                    static_cast<E*>(a.out)[r * a.ldo + n] = from_f<E>(v);
                 } else {  // DV_QKV
                     if (n < a.C) {
                         static_cast<E*>(a.out)[r * a.ldo + n] = from_f<E>(v);
@@ -728,7 +733,11 @@ int launch_gemv_inst(const GemvArgs<E>& a, cudaStream_t s) {
     static size_t opted[kMaxDevices] = {};
     const int rc = opt_in_smem(reinterpret_cast<const void*>(kern), smem, opted);
     if (rc) return rc;
-    return launch_overlapped(kern, dim3((a.N + kCols - 1) / kCols), dim3(kGemvThreads), smem, s, a);
+    int grid = (a.N + kCols - 1) / kCols;
+    // With the LayerNorm prologue every CTA normalises all rows again: for the wide head product
+    // a few CTAs per SM, each looping over column groups, share that work among more columns.
+    if (LN && a.N >= 16384) grid = min(grid, 4 * num_sms());
+    return launch_overlapped(kern, dim3(grid), dim3(kGemvThreads), smem, s, a);
 }
 
 // Warps per column: enough CTAs for narrow outputs, four columns a warp for the head (two with
@@ -783,6 +792,7 @@ int gemv_typed(int epi, bool ln, const void* x, long long ldx, const E* ln_w, co
                 case DV_GELU: rc = launch_gemv_rows<E, DV_GELU, true>(a, s); break;
                 case DV_F32: rc = launch_gemv_rows<E, DV_F32, true>(a, s); break;
                 case DV_QKV: rc = launch_gemv_rows<E, DV_QKV, true>(a, s); break;
+                case DV_STORE: rc = launch_gemv_rows<E, DV_STORE, true>(a, s); break;
                 default: return GPT_ERR_UNSUPPORTED;
             }
         } else {
@@ -809,6 +819,11 @@ int launch_gemv(int epi, bool ln, int dtype, const void* x, long long ldx, const
     return gemv_typed<float>(epi, ln, x, ldx, static_cast<const float*>(ln_w), static_cast<const float*>(ln_b),
                              static_cast<const float*>(W), static_cast<const float*>(bias), out, ldo, B, N, K,
                              gelu_tanh, static_cast<float*>(kv), pos, C, block_size, bump_pos, s);
+}
+
+size_t gemv_smem_bytes(int B, int K, int dtype, bool ln) {
+    const size_t es = dtype == GPT_DTYPE_BF16 ? 2 : 4;
+    return static_cast<size_t>(min(B, kGemvRows)) * K * (es + (ln ? 4 : 0));
 }
 
 size_t decode_attn_part_floats(int B, int nh, int hs, int block_size) {

@@ -276,4 +276,7 @@ int launch_gemm_bf16_acc(const bf16* A, long long lda, bool a_mn, const bf16* W,
                                 s, split_ws);
 }
 
+// Pipeline-wait limit of this file's kernels on the current device (0: the default).
+GPT_DEFINE_WAIT_LIMIT_SETTER(set_wait_limit_gemm)
+
 }  // namespace gpt

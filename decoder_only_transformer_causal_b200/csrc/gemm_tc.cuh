@@ -167,7 +167,10 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)  // 10 warps: <= 168 regi
     uint64_t* tfull = empty + kStages;
     uint64_t* tempty = tfull + 2;
     uint64_t* drain = tempty + 2;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    uint64_t* peer_done = drain + 1;            // PAIR, leader: the peer's producer has finished
+    volatile unsigned long long* peer_issued =  // PAIR, leader: the peer's count of issued stage loads
+        reinterpret_cast<volatile unsigned long long*>(peer_done + 1);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(peer_done + 2);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5;
@@ -207,6 +210,8 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)  // 10 warps: <= 168 regi
             mbar_init(&tempty[a], (PAIR ? 2 : 1) * NEPI * 32);
         }
         mbar_init(drain, 1);
+        mbar_init(peer_done, 1);
+        *peer_issued = 0ull;
         *abort_flag = 0;
         fence_barrier_init();
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -283,10 +288,35 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)  // 10 warps: <= 168 regi
             }
             // Make sure no bulk copy is still writing shared memory when the CTA exits: wait
             // for the latest load issued into each stage (already complete on the normal path).
-            // The leader's `full` phases count the peer's bytes too.
-            const long long n_check = rank != 0 ? 0 : (issued < kStages ? issued : kStages);
+            // The leader's `full` phases count the peer's bytes too, so the leader drains for both
+            // CTAs.  After a time-out the two producers may have issued different numbers of
+            // stage loads: the peer reports its count, and the leader balances the byte count of
+            // every phase only one of them issued (the peer's bytes expected on a phase the leader
+            // never armed; a peer half that will never come completed by hand), so that every
+            // issued copy is waited for before the pair's final cluster barrier.
+            long long total = issued;
+            if (PAIR && rank != 0) {
+                st_cluster_u64(map_to_rank(const_cast<unsigned long long*>(peer_issued), 0),
+                               static_cast<unsigned long long>(issued));
+                mbar_arrive_remote(map_to_rank(peer_done, 0));
+            }
+            if (PAIR && rank == 0) {
+                const long long peer = mbar_wait_cluster_bounded(peer_done, 0)
+                                           ? static_cast<long long>(*peer_issued) : issued;
+                const long long lo = peer < issued ? peer : issued, hi = peer < issued ? issued : peer;
+                for (long long idx = lo; idx < hi; ++idx) {
+                    uint64_t* b = &full[idx % kStages];
+                    if (idx >= kStages) mbar_drain(b, static_cast<uint32_t>(((idx - kStages) / kStages) & 1));
+                    if (peer > issued)
+                        mbar_arrive_expect_tx(b, L::STAGE_BYTES);  // only the peer's half arrives
+                    else
+                        mbar_complete_tx(b, L::STAGE_BYTES);       // the peer's half never comes
+                }
+                total = hi;
+            }
+            const long long n_check = rank != 0 ? 0 : (total < kStages ? total : kStages);
             for (long long i = 1; i <= n_check; ++i) {
-                const long long idx = issued - i;
+                const long long idx = total - i;
                 mbar_drain(&full[idx % kStages], static_cast<uint32_t>((idx / kStages) & 1));
             }
         }
@@ -299,6 +329,13 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)  // 10 warps: <= 168 regi
             int acc = 0;
             uint32_t acc_ph = 0;
             bool ok = true;
+            // Testing aid: nothing arrives on `drain` before the commit below, so this wait can only
+            // give up, which sends the CTA (for a pair: the leader; the peer's own waits then give
+            // up too) down its time-out path.
+            if (g_force_timeout) {
+                mbar_wait(drain, 0, abort_flag);
+                ok = false;
+            }
             for (int tile = unit0; tile < num_tiles && ok; tile += n_units) {
                 if (!(PAIR ? mbar_wait_cluster(&tempty[acc], acc_ph ^ 1u, abort_flag)
                            : mbar_wait(&tempty[acc], acc_ph ^ 1u, abort_flag)))

@@ -122,6 +122,23 @@ size_t a256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// The fused last-position head: the tensor-core kernel for bf16 (C <= 2048), the LayerNorm-prologue
+// GEMV for fp32, which stages up to 16 rows of the normalised input and its fp32 source in shared
+// memory.
+bool head_last_supported(int C, int B, int dtype) {
+    if (dtype == GPT_DTYPE_BF16) return head_last_tc_supported(C);
+    return C % 8 == 0 && gemv_smem_bytes(B, C, dtype, true) <= 227u * 1024u;
+}
+
+int launch_head_last(const float* x, long long ldx, const void* lnw, const void* lnb, const void* wte, int B, int C,
+                     int V, int dtype, void* logits, int32_t* status, cudaStream_t s) {
+    if (dtype == GPT_DTYPE_BF16)
+        return launch_head_last_bf16(x, ldx, static_cast<const bf16*>(lnw), static_cast<const bf16*>(lnb),
+                                     static_cast<const bf16*>(wte), B, C, V, static_cast<bf16*>(logits), V, status, s);
+    return launch_gemv(kGemvEpiStore, true, dtype, x, ldx, lnw, lnb, wte, nullptr, logits, V, B, V, C, 0, nullptr,
+                       nullptr, C, 1, 0, s);
+}
+
 int elem_size(const gpt_config_t* c) { return c->dtype == GPT_DTYPE_BF16 ? 2 : 4; }
 
 int validate(const gpt_config_t* c) {
@@ -509,6 +526,13 @@ GPT_API size_t gpt_workspace_bytes(const gpt_config_t* cfg, int B, int T) {
     return plan_ws(cfg, B, T).total;
 }
 
+GPT_API int gpt_set_wait_limit_ns(unsigned long long ns, int force_timeout) {
+    GPT_TRY(set_wait_limit_attention(ns, force_timeout));
+    GPT_TRY(set_wait_limit_gemm(ns, force_timeout));
+    GPT_TRY(set_wait_limit_head(ns, force_timeout));
+    return set_wait_limit_attention_bwd(ns, force_timeout);
+}
+
 GPT_API int gpt_check_status(void* workspace, void* stream) {
     if (!workspace) return GPT_ERR_NULL;
     return sync_and_read_status(workspace, static_cast<cudaStream_t>(stream));
@@ -533,6 +557,15 @@ GPT_API int gpt_forward(const gpt_config_t* cfg, const void* weights, const int6
     GPT_TRY(cuda_status(cudaMemsetAsync(status, 0, sizeof(int32_t), s)));
     GPT_TRY(launch_embed(W.wte(), W.wpe(), idx, x, B, T, C, V, cfg->dtype, status, s));
     for (int l = 0; l < cfg->n_layer; ++l) GPT_TRY(run_block(cfg, W, l, x, B, T, ws, P, s));
+
+    if (!targets && head_last_supported(C, B, cfg->dtype)) {
+        // Inference branch: only the last position's logits, [B, 1, V] (§3.2 ④): ln_f of the B
+        // last residual rows fused into one HBM-bound pass over wte (per 16 rows).
+        GPT_TRY(launch_head_last(x + static_cast<long long>(T - 1) * C, static_cast<long long>(T) * C, W.lnf_w(),
+                                 W.lnf_b(), W.wte(), B, C, V, cfg->dtype, logits, status, s));
+        if (flags & GPT_FLAG_SYNC_CHECK) return sync_and_read_status(ws, s);
+        return GPT_OK;
+    }
     GPT_TRY(launch_layernorm(x, W.lnf_w(), W.lnf_b(), u, N, C, cfg->dtype, s));
 
     if (targets) {
@@ -550,7 +583,8 @@ GPT_API int gpt_forward(const gpt_config_t* cfg, const void* weights, const int6
         }
         GPT_TRY(launch_loss_finalize(rl, targets, N, V, loss, loss_sum_count, s));
     } else {
-        // Inference branch: only the last position's logits, [B, 1, V] (§3.2 ④).
+        // Inference branch for widths the fused head above does not take: ln_f over every row,
+        // then the product of the last rows.
         const long long lda = static_cast<long long>(T) * C;
         if (cfg->dtype == GPT_DTYPE_BF16) {
             const bf16* ulast = static_cast<const bf16*>(u) + static_cast<long long>(T - 1) * C;
@@ -564,6 +598,17 @@ GPT_API int gpt_forward(const gpt_config_t* cfg, const void* weights, const int6
     }
     if (flags & GPT_FLAG_SYNC_CHECK) return sync_and_read_status(ws, s);
     return GPT_OK;
+}
+
+GPT_API int gpt_lm_head_last(const float* x, long long ldx, const void* lnf_w, const void* lnf_b, const void* wte,
+                             int B, int C, int V, int dtype, void* logits, int32_t* status, void* stream) {
+    if (!x || !lnf_w || !wte || !logits) return GPT_ERR_NULL;
+    if (B < 1 || C < 1 || V < 1 || ldx < C) return GPT_ERR_BAD_SHAPE;
+    if (dtype != GPT_DTYPE_BF16 && dtype != GPT_DTYPE_F32) return GPT_ERR_BAD_SHAPE;
+    if (!head_last_supported(C, B, dtype)) return GPT_ERR_UNSUPPORTED;
+    if (!aligned(x, 16) || (ldx % 4) || !aligned(wte, 16)) return GPT_ERR_BAD_ALIGN;
+    return launch_head_last(x, ldx, lnf_w, lnf_b, wte, B, C, V, dtype, logits, status,
+                            static_cast<cudaStream_t>(stream));
 }
 
 GPT_API int gpt_block(const gpt_config_t* cfg, const void* weights, int layer, float* x, int B, int T,

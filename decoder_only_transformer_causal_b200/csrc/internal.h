@@ -133,6 +133,21 @@ struct AttnLayout {
 };
 int launch_attention_bf16(const AttnLayout& L, int B, int nh, int T, int32_t* status, cudaStream_t s);
 
+// Limit after which a pipeline wait of the tensor-core kernels gives up, on the current device,
+// one setter per file holding such kernels (ns 0: the default 1 s), and the forced time-out of
+// the testing aid (common.cuh, g_force_timeout).
+int set_wait_limit_attention(unsigned long long ns, int force);
+int set_wait_limit_gemm(unsigned long long ns, int force);
+int set_wait_limit_attention_bwd(unsigned long long ns, int force);
+int set_wait_limit_head(unsigned long long ns, int force);
+
+// ---- the inference branch's head (head_last.cu): logits[b, :] = LayerNorm(x_b; lnw, lnb) wte^T
+// for B rows x + b * ldx (fp32, 16-byte aligned rows); logits bf16 at out + b * ldo.  C % 8 == 0
+// and C <= 2048 (head_last_tc_supported).
+bool head_last_tc_supported(int C);
+int launch_head_last_bf16(const float* x, long long ldx, const bf16* lnw, const bf16* lnb, const bf16* wte, int B,
+                          int C, int V, bf16* out, long long ldo, int32_t* status, cudaStream_t s);
+
 // ---- fp32 SIMT path (simt_f32.cu)
 int launch_linear_f32(const float* A, long long lda, const float* W, const float* bias, float* out,
                       long long ldo, int M, int N, int K, int epilogue, int gelu, cudaStream_t s);
@@ -150,11 +165,15 @@ int launch_attention_f32(const AttnLayoutF32& L, int B, int nh, int T, int hs, c
 int launch_embed_pos(const void* wte, const void* wpe, const int64_t* tok, long long ld_tok, const int* pos, float* x,
                      int B, int C, int V, int block_size, int dtype, int32_t* status, cudaStream_t s);
 // Matrix-vector products of B rows against W [N, K]; epi 1 gelu -> E, 2 fp32 +=, 3 fp32
-// store, 4 qkv split (q -> out, k/v -> kv[b, *pos]).  ln: the input is the fp32 residual
-// stream and LayerNorm(ln_w, ln_b) is applied to it first.  bump_pos: advance *pos by one.
+// store, 4 qkv split (q -> out, k/v -> kv[b, *pos]), 5 store E.  ln: the input is the fp32
+// residual stream and LayerNorm(ln_w, ln_b) is applied to it first.  bump_pos: advance *pos by
+// one.  gemv_smem_bytes: the dynamic shared memory a launch with `B` rows needs (the library's
+// limit is 227 KB per CTA).
 int launch_gemv(int epi, bool ln, int dtype, const void* x, long long ldx, const void* ln_w, const void* ln_b,
                 const void* W, const void* bias, void* out, long long ldo, int B, int N, int K, int gelu_tanh,
                 void* kv, int* pos, int C, int block_size, int bump_pos, cudaStream_t s);
+size_t gemv_smem_bytes(int B, int K, int dtype, bool ln);
+constexpr int kGemvEpiStore = 5;
 size_t decode_attn_part_floats(int B, int nh, int hs, int block_size);
 // counter: B * nh ints, zero on entry and on return.
 int launch_decode_attention(int dtype, const void* q, const void* kv, const int* pos, float* part, int* counter,

@@ -28,7 +28,8 @@ std::mutex g_setup_mutex;
 void* g_scratch_on_device[kMaxDevices] = {nullptr};
 
 // Device address of g_lm_head_scratch on the current device.  In host code the array's name is
-// only a stand-in, so the address is looked up once per device with that device current.
+// only a stand-in, so the address is looked up once per device with that device current and kept
+// for the life of the process (a device reset invalidates it; the header says so).
 int scratch_for_current_device(void** out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return GPT_ERR_CUDA;

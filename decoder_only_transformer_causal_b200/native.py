@@ -76,6 +76,7 @@ def _load() -> ctypes.CDLL:
         "gpt_weights_layout": (I, [CFG, P, P, I]),
         "gpt_workspace_bytes": (Z, [CFG, I, I]),
         "gpt_check_status": (I, [P, P]),
+        "gpt_set_wait_limit_ns": (I, [ctypes.c_ulonglong, I]),
         "gpt_forward": (I, [CFG, P, P, P, I, I, P, P, P, P, P, Z, P, I]),
         "gpt_block": (I, [CFG, P, I, P, I, I, P, Z, P, I]),
         "gpt_attention": (I, [P, P, P, P, I, I, I, I, D, P, P]),
@@ -85,6 +86,7 @@ def _load() -> ctypes.CDLL:
         "gpt_lm_head_workspace_bytes": (Z, [I, I]),
         "gpt_lm_head_loss": (I, [P, P, P, I, I, I, D, P, P, P, P, P, Z, P, I]),
         "gpt_lm_head_loss_noalloc": (I, [P, P, P, I, I, I, D, P, P, P, P, P, I]),
+        "gpt_lm_head_last": (I, [P, L, P, P, P, I, I, I, D, P, P, P]),
         "gpt_kv_cache_bytes": (Z, [CFG, I]),
         "gpt_decode_workspace_bytes": (Z, [CFG, I, I]),
         "gpt_generate_workspace_bytes": (Z, [CFG, I, I, I]),
@@ -126,9 +128,9 @@ def _load() -> ctypes.CDLL:
 LIB = _load()
 
 EXPORTED = ("gpt_status_string", "gpt_abi_version", "gpt_last_cuda_error", "gpt_validate_config", "gpt_weights_bytes",
-            "gpt_weights_count", "gpt_weights_layout", "gpt_workspace_bytes", "gpt_check_status",
+            "gpt_weights_count", "gpt_weights_layout", "gpt_workspace_bytes", "gpt_check_status", "gpt_set_wait_limit_ns",
             "gpt_forward", "gpt_block", "gpt_attention", "gpt_embed", "gpt_layernorm", "gpt_linear",
-            "gpt_lm_head_workspace_bytes", "gpt_lm_head_loss", "gpt_lm_head_loss_noalloc",
+            "gpt_lm_head_workspace_bytes", "gpt_lm_head_loss", "gpt_lm_head_loss_noalloc", "gpt_lm_head_last",
             "gpt_kv_cache_bytes", "gpt_decode_workspace_bytes", "gpt_generate_workspace_bytes", "gpt_prefill",
             "gpt_decode_step", "gpt_sample", "gpt_generate", "gpt_lr_schedule", "gpt_param_elems",
             "gpt_adamw_workspace_bytes", "gpt_adamw_step", "gpt_cross_entropy_backward",
@@ -256,6 +258,12 @@ def check_status(workspace: torch.Tensor, stream=None) -> int:
     return LIB.gpt_check_status(_ptr(workspace), _stream(stream))
 
 
+def set_wait_limit_ns(ns: int, force_timeout: bool = False) -> None:
+    """gpt_set_wait_limit_ns: the pipeline-wait limit of the tensor-core kernels on the current
+    device (0 restores the default) and the forced time-out; a testing aid for the time-out path."""
+    _check(LIB.gpt_set_wait_limit_ns(int(ns), int(bool(force_timeout))), "gpt_set_wait_limit_ns")
+
+
 def forward(cfg: GPTConfig, weights: torch.Tensor, idx: torch.Tensor, targets: torch.Tensor | None,
             workspace: torch.Tensor, logits: torch.Tensor | None = None, loss: torch.Tensor | None = None,
             row_loss: torch.Tensor | None = None, loss_sum_count: torch.Tensor | None = None,
@@ -329,6 +337,27 @@ def linear(x, W, b=None, out=None, epilogue=GPT_EPI_STORE, gelu=GPT_GELU_ERF, st
     _check(LIB.gpt_linear(_ptr(x), _ptr(W), _ptr(b), _ptr(out), M, N, K, dtype, epilogue, gelu,
                           _ptr(status), _stream(stream)), "gpt_linear")
     return out
+
+
+def lm_head_last(x: torch.Tensor, lnf_w: torch.Tensor, lnf_b: torch.Tensor | None, wte: torch.Tensor,
+                 logits: torch.Tensor | None = None, status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """gpt_lm_head_last: ln_f and the tied head of the last position of each sequence.  x is the
+    fp32 residual stream [B, T, C] (only row T-1 of each sequence is read) or [B, C]; returns
+    logits [B, V] in wte's dtype."""
+    if x.dtype != torch.float32 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous float32 tensor")
+    if x.dim() == 3:
+        B, T, C = x.shape
+        base, ldx = x[:, T - 1].data_ptr(), T * C
+    else:
+        B, C = x.shape
+        base, ldx = x.data_ptr(), C
+    V = wte.shape[0]
+    if logits is None:
+        logits = torch.empty((B, V), dtype=wte.dtype, device=x.device)
+    _check(LIB.gpt_lm_head_last(base, ldx, _ptr(lnf_w), _ptr(lnf_b), _ptr(wte), B, C, V, _dt(wte), _ptr(logits),
+                                _ptr(status), _stream(stream)), "gpt_lm_head_last")
+    return logits
 
 
 def lm_head_workspace_bytes(rows: int, V: int) -> int:

@@ -122,6 +122,20 @@ size_t gpt_workspace_bytes(const gpt_config_t* cfg, int B, int T);
  * returns it (GPT_OK, GPT_ERR_INDEX or GPT_ERR_TIMEOUT), or GPT_ERR_CUDA. */
 int gpt_check_status(void* workspace, void* stream);
 
+/* Testing aid with no counterpart in the pages: sets, on the current device, the time after
+ * which a pipeline wait inside the tensor-core kernels (a thread waiting for a copy, a product or
+ * another warp's result) gives up, in nanoseconds; 0 restores the default of 1 s.  A kernel whose
+ * wait gives up records GPT_ERR_TIMEOUT in its status word, lets every copy and product it has
+ * already issued finish (those drains keep the default limit), releases its tensor memory and
+ * returns; its outputs are then invalid.
+ *   force_timeout != 0 makes the causal attention kernel and the product kernels (gpt_linear,
+ *   single CTAs for M < 256 and CTA pairs from M = 256) launched from then on wait first for an
+ *   event that never happens, so their time-out path runs on purpose after `ns`; 0 turns that
+ *   off.
+ * Call it with no kernel of this library running or queued on the device (it copies to the device
+ * synchronously).  Returns GPT_OK or GPT_ERR_CUDA. */
+int gpt_set_wait_limit_ns(unsigned long long ns, int force_timeout);
+
 /* ---- the forward pass ---------------------------------------------------------------
  * GPT.forward(idx, targets) ("nanoGPT 全局流程图", §3.2; "nanoGPT 代码解析", forward).
  *   weights  packed buffer described above.
@@ -186,6 +200,22 @@ int gpt_layernorm(const float* x, const void* w, const void* b, void* out,
 int gpt_linear(const void* x, const void* W, const void* b, void* out, int M, int N, int K,
                int dtype, int epilogue, int gelu, int32_t* status, void* stream);
 
+/* The inference branch of the head ("nanoGPT 全局流程图", §3.2 ④: with no targets only the last
+ * position goes through ln_f and lm_head, logits [B, 1, V]):
+ *   logits[b, :] = LayerNorm(x[b * ldx .. b * ldx + C); lnf_w, lnf_b) wte^T
+ *   x       fp32 residual rows, row b at element offset b * ldx (for a [B, T, C] residual stream,
+ *           pass &x[0, T-1, 0] and ldx = T * C); 16-byte aligned, ldx % 4 == 0.
+ *   lnf_w, lnf_b  [C] in `dtype` (lnf_b may be NULL); wte [V, C] in `dtype`, 16-byte aligned.
+ *   logits  [B, V] in `dtype` (rows V elements apart).
+ *   status  optional device int32 (NULL allowed): GPT_ERR_TIMEOUT if a pipeline wait of the
+ *           tensor-core kernel gave up (never cleared by the library).
+ *   Requires C % 8 == 0, and C <= 2048 for bf16 (for fp32, min(B, 16) * C * 8 <= 227 KB);
+ *   else GPT_ERR_UNSUPPORTED.  One read of wte per 16 rows: the product is bound by HBM.
+ *   gpt_forward with targets == NULL runs this on its final residual rows. */
+int gpt_lm_head_last(const float* x, long long ldx, const void* lnf_w, const void* lnf_b,
+                     const void* wte, int B, int C, int V, int dtype, void* logits, int32_t* status,
+                     void* stream);
+
 /* Tied head with fused cross-entropy ("nanoGPT 全局流程图", §3.2 ④ and §3.3):
  *   logits = u wte^T ([rows, V] in `dtype`), then per row logsumexp - logit[target] over all
  *   V columns, averaged over rows whose target != -1 (fixed-order reduction).
@@ -210,10 +240,16 @@ int gpt_lm_head_loss(const void* u, const void* wte, const int64_t* targets, int
  *   (gpt_lm_head_workspace_bytes(rows, V) > 16 MiB; about 5,300 rows at V = 50304) returns
  *   GPT_ERR_WS_TOO_SMALL before anything is enqueued.  Nothing is allocated or freed.
  *   The first call on each device looks up the array's device address (cudaGetSymbolAddress)
- *   with that device current; make that first call before any stream capture begins.
+ *   with that device current and keeps it for the life of the process; make that first call
+ *   before any stream capture begins.  cudaDeviceReset (or any other teardown of the device's
+ *   primary context) invalidates the kept address: do not call this entry point on a device
+ *   after resetting it.
  *   All calls on a device share the array and it keeps the last call's contents (the status
  *   word is cleared at the start of each call): calls whose work overlaps on the GPU race, so
- *   order them on one stream.  With GPT_FLAG_SYNC_CHECK the status word is read from the array. */
+ *   order them on one stream.  With GPT_FLAG_SYNC_CHECK the status word is read from the array.
+ *   Without that flag a call whose head product gave up on a bounded wait (GPT_ERR_TIMEOUT in
+ *   the status word) still returns GPT_OK, and its loss may then be built from partial sums an
+ *   earlier call left in the array: pass GPT_FLAG_SYNC_CHECK where that matters. */
 int gpt_lm_head_loss_noalloc(const void* u, const void* wte, const int64_t* targets, int rows,
                              int C, int V, int dtype, void* logits, float* loss, float* row_loss,
                              double* loss_sum_count, void* stream, int flags);

@@ -125,6 +125,18 @@ def test_kernel_entry_validation():
     assert L.gpt_lm_head_loss(FAKE, FAKE, FAKE, 4, 64, 128, native.GPT_DTYPE_BF16, FAKE, None, None, None,
                               FAKE, 16, None, 0) == native.GPT_ERR_WS_TOO_SMALL
     assert L.gpt_check_status(None, None) == native.GPT_ERR_NULL
+    bf = native.GPT_DTYPE_BF16
+    assert L.gpt_lm_head_last(None, 768, FAKE, None, FAKE, 4, 768, 50304, bf, FAKE, None, None) == native.GPT_ERR_NULL
+    assert L.gpt_lm_head_last(FAKE, 100, FAKE, None, FAKE, 4, 768, 50304, bf, FAKE, None, None) \
+        == native.GPT_ERR_BAD_SHAPE                                # ldx < C
+    assert L.gpt_lm_head_last(FAKE, 776, FAKE, None, FAKE, 4, 772, 50304, bf, FAKE, None, None) \
+        == native.GPT_ERR_UNSUPPORTED                              # C % 8
+    assert L.gpt_lm_head_last(FAKE, 4096, FAKE, None, FAKE, 16, 4096, 50304, bf, FAKE, None, None) \
+        == native.GPT_ERR_UNSUPPORTED                              # 16 staged rows of 4096 exceed shared memory
+    assert L.gpt_lm_head_last(FAKE + 4, 768, FAKE, None, FAKE, 4, 768, 50304, bf, FAKE, None, None) \
+        == native.GPT_ERR_BAD_ALIGN
+    assert L.gpt_lm_head_last(FAKE, 770, FAKE, None, FAKE, 4, 768, 50304, bf, FAKE, None, None) \
+        == native.GPT_ERR_BAD_ALIGN                                # row stride not a multiple of 16 bytes
 
 
 def test_generation_sizes():

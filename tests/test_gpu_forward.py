@@ -2,8 +2,8 @@
 against the fp64 oracle, from the tiny fp32 model to GPT-2 XL at full size.
 
 Full-size bf16 workloads run on the GPU exactly as the benchmark launches them; the oracle
-then recomputes sampled sequences (sequences are independent) and, for the two largest
-models, a prefix of one sequence (logits at position t depend only on positions <= t)."""
+then recomputes every sequence of GPT-2 124M and whole 1024-token sequences of GPT-2 medium and
+XL (sequences are independent, so each one is checked at every position and vocabulary entry)."""
 import math
 
 import numpy as np
@@ -113,18 +113,53 @@ def _full_size(name, sample_b, prefix=None, atol=BF16_ATOL, mean_tol=None):
 
 
 def test_gpt2_full_size():
-    _full_size("gpt2", sample_b=[0, 11])
+    _full_size("gpt2", sample_b=list(range(12)))
 
 
 def test_gpt2_medium_full_size():
-    _full_size("gpt2-medium", sample_b=[5], prefix=384)
+    _full_size("gpt2-medium", sample_b=[0, 5])
 
 
 def test_gpt2_xl_full_size_and_last_position():
-    m, idx, logits = _full_size("gpt2-xl", sample_b=[2], prefix=256, atol=XL_ATOL, mean_tol=XL_MEAN)
+    m, idx, logits = _full_size("gpt2-xl", sample_b=[2], atol=XL_ATOL, mean_tol=XL_MEAN)
     last, _ = m(idx.cuda(), None, sync_check=True)
     assert last.shape == (4, 1, 50304)
     assert max_abs(f64(last)[:, 0], f64(logits[:, -1])) <= BF16_ATOL
+
+
+# ------------------------------------------------------------------ inference branch (targets=None)
+# "nanoGPT 全局流程图", §3.2 ④: without targets only the last position goes through ln_f and the
+# head, logits [B, 1, V].  Every sequence's last row against the oracle's, full depth.
+@pytest.mark.parametrize("name,B,T,atol", [("gpt2", 2, 1024, BF16_ATOL), ("gpt2-xl", 4, 256, XL_ATOL)])
+def test_last_position_logits_vs_oracle(name, B, T, atol):
+    cfg, W, W64, idx, _ = model_inputs(name, B=B, T=T)
+    m = gpu_model(cfg, W)
+    last, none = m(idx.cuda(), None, sync_check=True)
+    assert none is None and last.shape == (B, 1, cfg["vocab_size"]) and last.dtype == torch.bfloat16
+    ref = oracle.forward(W64, cfg, idx.numpy(), None)["logits"]
+    err = max_abs(f64(last), ref)
+    assert err <= atol, err
+    assert float(np.mean(np.abs(f64(last) - ref))) <= XL_MEAN
+
+
+@pytest.mark.parametrize("B,C,dtype", [(4, 1600, torch.bfloat16), (1, 768, torch.bfloat16), (17, 768, torch.bfloat16),
+                                       (3, 128, torch.float32)])
+def test_lm_head_last_kernel(B, C, dtype):
+    """gpt_lm_head_last alone: ln_f of row T-1 of each sequence and the tied head, against the
+    oracle's LayerNorm and head on the same stored inputs (B 17 takes two passes over wte)."""
+    from decoder_only_transformer_causal_b200 import native
+    V, T = 50304 if dtype == torch.bfloat16 else 65, 5
+    g = torch.Generator().manual_seed(91)
+    x = torch.randn((B, T, C), generator=g) * 1.5 + 0.3
+    wte = (torch.randn((V, C), generator=g) * 0.02).to(dtype)
+    lw = (1 + 0.1 * torch.randn(C, generator=g)).to(dtype)
+    lb = (0.1 * torch.randn(C, generator=g)).to(dtype)
+    got = native.lm_head_last(x.cuda(), lw.cuda(), lb.cuda(), wte.cuda())
+    torch.cuda.synchronize()
+    u = oracle.layer_norm(f64(x[:, T - 1]), f64(lw), f64(lb))
+    ref = oracle.lm_head(u, {"wte": f64(wte)})
+    tol = F32_ATOL if dtype == torch.float32 else BF16_ATOL
+    assert max_abs(f64(got), ref) <= tol
 
 
 def test_loss_at_init_band():

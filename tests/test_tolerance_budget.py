@@ -58,17 +58,29 @@ def replay(W, cfg, idx):
     return bf16(u @ W["wte"].T)
 
 
-@pytest.mark.slow
-@pytest.mark.skipif(not os.environ.get("GPT_SLOW_TESTS"),
-                    reason="builds the 1.56B-parameter model in fp64 (~3 min); set GPT_SLOW_TESTS=1")
-def test_xl_bf16_replay_exceeds_2e2():
+def _xl_replay_error(positions):
     w = seeded.WORKLOADS["gpt2-xl"]
     cfg = w.model_dict()
     W = seeded.to_f64(seeded.make_weights(cfg))
     idx, _ = seeded.make_tokens(w.batch, w.seq_len, w.token_high)
-    seq = idx[2:3, :128].numpy()
+    seq = idx[2:3, :positions].numpy()
     exact = oracle.lm_head(oracle.final_hidden(W, cfg, seq), W)
-    err = np.abs(replay(W, cfg, seq) - exact)
+    return np.abs(replay(W, cfg, seq) - exact)
+
+
+def test_xl_bf16_replay_exceeds_2e2():
+    """32 positions of the XL parity test's sequence (~20 s, 13 GB of fp64 weights): already
+    there the bf16 storage points alone put the logits more than 2e-2 from the exact values."""
+    err = _xl_replay_error(32)
     assert err.max() > 2e-2          # the stated bar is out of reach for bf16 storage
     assert err.max() < 3e-2          # the derived XL bar holds for the replay itself
+    assert err.mean() < 5e-3
+
+
+@pytest.mark.slow
+@pytest.mark.skipif(not os.environ.get("GPT_SLOW_TESTS"),
+                    reason="the same replay over 128 positions (~1 min); set GPT_SLOW_TESTS=1")
+def test_xl_bf16_replay_exceeds_2e2_128_positions():
+    err = _xl_replay_error(128)
+    assert 2e-2 < err.max() < 3e-2
     assert err.mean() < 5e-3
