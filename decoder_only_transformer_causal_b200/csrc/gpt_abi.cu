@@ -1295,6 +1295,31 @@ GPT_API int gpt_forward_train(const gpt_config_t* cfg, const void* weights, cons
     return GPT_OK;
 }
 
+GPT_API int gpt_grad_buckets(const gpt_config_t* cfg, size_t* starts, size_t* stops, int n) {
+    const int rc = validate(cfg);
+    if (rc != GPT_OK) return rc;
+    const int L = cfg->n_layer, count = 2 + kTensorsPerLayer * L + 2;
+    if (count > kOptMaxTensors) return GPT_ERR_UNSUPPORTED;
+    size_t offs[kOptMaxTensors];
+    layout(cfg, offs, nullptr, count);
+    const size_t es = elem_size(cfg);
+    const size_t total = gpt_param_elems(cfg);
+    for (int i = 0; i <= L && i < n; ++i) {
+        size_t a, b;
+        if (i < L) {
+            const int l = L - 1 - i;  // buckets in the order the backward finishes them
+            a = offs[2 + kTensorsPerLayer * l] / es;
+            b = (i == 0) ? total : offs[2 + kTensorsPerLayer * (l + 1)] / es;
+        } else {
+            a = 0;
+            b = offs[2] / es;
+        }
+        if (starts) starts[i] = a;
+        if (stops) stops[i] = b;
+    }
+    return L + 1;
+}
+
 GPT_API size_t gpt_train_loss_terms_offset(const gpt_config_t* cfg, int B, int T) {
     if (validate(cfg) != GPT_OK || B < 1 || T < 1 || T > cfg->block_size) return 0;
     return plan_acts(cfg, B, T).sum_count;
@@ -1302,7 +1327,7 @@ GPT_API size_t gpt_train_loss_terms_offset(const gpt_config_t* cfg, int B, int T
 
 GPT_API int gpt_backward(const gpt_config_t* cfg, const void* weights, const int64_t* idx, const int64_t* targets, int B,
                          int T, const void* acts, size_t acts_bytes, float* grads, float loss_scale, void* workspace,
-                         size_t workspace_bytes, void* stream, int flags) {
+                         size_t workspace_bytes, void* stream, int flags, void* const* bucket_events) {
     ActPlan A;
     GPT_TRY(check_train(cfg, weights, idx, targets, B, T, acts, acts_bytes, &A));
     if (!grads || !workspace) return GPT_ERR_NULL;
@@ -1381,6 +1406,12 @@ GPT_API int gpt_backward(const gpt_config_t* cfg, const void* weights, const int
     GPT_TRY(linear_bwd(dz, V, ab + A.u_f, C, W.wte(), V, C, d1, F32_OUT, nullptr, G(0), dzT));
     GPT_TRY(launch_layernorm_backward(d1, reinterpret_cast<const float*>(ab + A.x_f), W.lnf_w(), dt, dx, 0, G(count - 2),
                                       cfg->bias ? G(count - 1) : nullptr, 1, parts, N, C, s, dx16));
+    // Event i marks the end of bucket i (gpt_grad_buckets): a caller may start reducing that range
+    // of grads on another stream while the rest of the backward runs.
+    auto mark = [&](int i) -> int {
+        if (!bucket_events || !bucket_events[i]) return GPT_OK;
+        return cuda_status(cudaEventRecord(static_cast<cudaEvent_t>(bucket_events[i]), s));
+    };
     for (int l = cfg->n_layer - 1; l >= 0; --l) {
         const uint8_t* L = ab + A.layer * l;
         // mlp c_proj, then GELU: dpre = (dx W_fc2) * gelu'(pre) (bf16: one fused product reading the
@@ -1432,9 +1463,11 @@ GPT_API int gpt_backward(const gpt_config_t* cfg, const void* weights, const int
         GPT_TRY(launch_layernorm_backward(d1, reinterpret_cast<const float*>(L + A.x_in), W.layer(l, W_LN1_W), dt, dx, 1,
                                           GL(l, W_LN1_W), cfg->bias ? GL(l, W_LN1_B) : nullptr, 1, parts, N, C, s,
                                           dx16));
+        GPT_TRY(mark(cfg->n_layer - 1 - l));  // every gradient of layer l (and, for the last layer, ln_f) is final
     }
     GPT_TRY(launch_embed_backward(idx, dx, B, T, C, V, G(0), G(1), reinterpret_cast<unsigned long long*>(ws + P.sort),
                                   status, s));
+    GPT_TRY(mark(cfg->n_layer));  // wte (the head's and the embedding's parts) and wpe
     if (flags & GPT_FLAG_SYNC_CHECK) return sync_and_read_status(ws, s);
     return GPT_OK;
 }

@@ -12,7 +12,10 @@ Data-parallel training ("nanoGPT 全局流程图" 3.4-3.7; "nanoGPT 核心代码
 each rank runs the training forward on its shard, the {sum, count} pair is all-reduced *before*
 the backward so every rank's cross-entropy gradient divides by the global count, and a SUM
 all-reduce of the flat fp32 gradients then gives exactly the whole batch's gradient (also when
-ignored targets are spread unevenly); every rank applies the same AdamW step.
+ignored targets are spread unevenly); every rank applies the same AdamW step.  The gradient
+reduction runs per layer bucket on a second stream, each bucket as soon as the backward has
+finished it (gpt_grad_buckets, gpt_backward's bucket events), overlapping the backward of the
+earlier layers.
 """
 from __future__ import annotations
 
@@ -71,11 +74,43 @@ def allreduce_grads(grads: torch.Tensor, group=None) -> torch.Tensor:
     return grads
 
 
-def train_step_sharded(trainer, idx: torch.Tensor, targets: torch.Tensor, group=None) -> torch.Tensor:
+def allreduce_grads_bucketed(grads: torch.Tensor, buckets, wait=None, group=None) -> torch.Tensor:
+    """SUM all-reduce of the flat fp32 gradient array one bucket (an element range) at a time, in
+    the given order; wait(i), when given, runs before bucket i is reduced (the GPU step makes the
+    communication stream wait there for the backward's event of that bucket)."""
+    if grads.dtype != torch.float32:
+        raise ValueError("grads must be float32")
+    for i, (a, b) in enumerate(buckets):
+        if wait is not None:
+            wait(i)
+        dist.all_reduce(grads[a:b], op=dist.ReduceOp.SUM, group=group)
+    return grads
+
+
+class _Overlap:
+    """Per-trainer state of the overlapped reduction: the gradient buckets, one CUDA event per
+    bucket (recorded by gpt_backward when the bucket is complete) and the communication stream."""
+
+    def __init__(self, trainer):
+        from . import native
+        dev = trainer.model.device
+        self.buckets = native.grad_buckets(trainer.model.cfg)
+        self.stream = torch.cuda.Stream(dev)
+        self.events = [torch.cuda.Event() for _ in self.buckets]
+        main = torch.cuda.current_stream(dev)
+        for e in self.events:      # the CUDA events exist from their first record on
+            e.record(main)
+
+
+def train_step_sharded(trainer, idx: torch.Tensor, targets: torch.Tensor, group=None,
+                       overlap: bool = True) -> torch.Tensor:
     """One data-parallel training step of a Trainer on this rank's shard [B_r, T] (already on the
     rank's device): training forward, all-reduce of the loss terms, backward against the global
-    count, SUM all-reduce of the gradients, AdamW.  Returns the global mean loss as a device fp64
-    scalar (NaN when no row is counted), so consecutive steps queue without a host round trip."""
+    count, SUM all-reduce of the gradients, AdamW.  With overlap (the default) the gradients are
+    reduced per layer on a second stream while the backward of the earlier layers still runs: each
+    bucket's all-reduce waits only for the event gpt_backward records when that bucket is complete,
+    and the optimizer waits for all of them.  Returns the global mean loss as a device fp64 scalar
+    (NaN when no row is counted), so consecutive steps queue without a host round trip."""
     from . import native
     cfg, w = trainer.model.cfg, trainer.model.weights
     B, T = idx.shape
@@ -83,8 +118,20 @@ def train_step_sharded(trainer, idx: torch.Tensor, targets: torch.Tensor, group=
     lt = native.loss_terms(cfg, trainer.acts, B, T)
     allreduce_loss_terms(lt, group)
     trainer.grads.zero_()
-    native.backward(cfg, w, idx, targets, trainer.acts, trainer.grads, trainer.bws)
-    allreduce_grads(trainer.grads, group)
+    if not overlap:
+        native.backward(cfg, w, idx, targets, trainer.acts, trainer.grads, trainer.bws)
+        allreduce_grads(trainer.grads, group)
+    else:
+        ov = getattr(trainer, "_dp_overlap", None)
+        if ov is None:
+            ov = trainer._dp_overlap = _Overlap(trainer)
+        main = torch.cuda.current_stream(trainer.model.device)
+        native.backward(cfg, w, idx, targets, trainer.acts, trainer.grads, trainer.bws, stream=main,
+                        bucket_events=ov.events)
+        with torch.cuda.stream(ov.stream):
+            allreduce_grads_bucketed(trainer.grads, ov.buckets, wait=lambda i: ov.stream.wait_event(ov.events[i]),
+                                     group=group)
+        main.wait_stream(ov.stream)
     trainer.opt.step(trainer.grads)
     return lt[0] / lt[1]
 

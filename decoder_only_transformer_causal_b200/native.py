@@ -115,7 +115,8 @@ def _load() -> ctypes.CDLL:
         "gpt_train_activation_bytes": (Z, [CFG, I, I]),
         "gpt_backward_workspace_bytes": (Z, [CFG, I, I]),
         "gpt_forward_train": (I, [CFG, P, P, P, I, I, P, Z, P, P, Z, P, I]),
-        "gpt_backward": (I, [CFG, P, P, P, I, I, P, Z, P, F, P, Z, P, I]),
+        "gpt_backward": (I, [CFG, P, P, P, I, I, P, Z, P, F, P, Z, P, I, P]),
+        "gpt_grad_buckets": (I, [CFG, P, P, I]),
         "gpt_train_loss_terms_offset": (Z, [CFG, I, I]),
     }
     for name, (res, args) in sig.items():
@@ -139,7 +140,7 @@ EXPORTED = ("gpt_status_string", "gpt_abi_version", "gpt_last_cuda_error", "gpt_
             "gpt_attention_train", "gpt_attention_backward_workspace_bytes", "gpt_attention_backward", "gpt_transpose",
             "gpt_linear_backward_workspace_bytes", "gpt_linear_backward",
             "gpt_train_activation_bytes", "gpt_backward_workspace_bytes", "gpt_forward_train", "gpt_backward",
-            "gpt_train_loss_terms_offset")
+            "gpt_grad_buckets", "gpt_train_loss_terms_offset")
 
 
 def status_string(status: int) -> str:
@@ -661,13 +662,34 @@ def forward_train(cfg, weights, idx, targets, acts, workspace, loss=None, stream
     return loss
 
 
-def backward(cfg, weights, idx, targets, acts, grads, workspace, loss_scale=1.0, stream=None, sync_check=False):
-    """gpt_backward: adds loss_scale * the gradients into grads (fp32 [param_elems])."""
+def backward(cfg, weights, idx, targets, acts, grads, workspace, loss_scale=1.0, stream=None, sync_check=False,
+             bucket_events=None):
+    """gpt_backward: adds loss_scale * the gradients into grads (fp32 [param_elems]).  bucket_events:
+    optional list of n_layer + 1 torch.cuda.Event (already recorded once, so that the CUDA event
+    exists); event i is recorded when gradient bucket i (grad_buckets) is complete."""
     B, T = idx.shape
+    evs = None
+    if bucket_events is not None:
+        if len(bucket_events) != cfg.n_layer + 1:
+            raise ValueError("bucket_events needs n_layer + 1 events")
+        handles = [e.cuda_event for e in bucket_events]
+        if not all(handles):
+            raise ValueError("record each event once before passing it (its CUDA event is created then)")
+        evs = (ctypes.c_void_p * len(handles))(*handles)
     _check(LIB.gpt_backward(ctypes.byref(cfg.c()), _ptr(weights), _ptr(idx), _ptr(targets), B, T, _ptr(acts),
                             acts.numel(), _ptr(grads), float(loss_scale), _ptr(workspace), workspace.numel(),
-                            _stream(stream), GPT_FLAG_SYNC_CHECK if sync_check else 0), "gpt_backward")
+                            _stream(stream), GPT_FLAG_SYNC_CHECK if sync_check else 0, evs), "gpt_backward")
     return grads
+
+
+def grad_buckets(cfg) -> list[tuple[int, int]]:
+    """gpt_grad_buckets: the [start, stop) element ranges of the flat gradient array in the order the
+    backward completes them (layer n_layer - 1 with ln_f first, ..., layer 0, then wte and wpe)."""
+    n = LIB.gpt_grad_buckets(ctypes.byref(cfg.c()), None, None, 0)
+    _check(n if n < 0 else GPT_OK, "gpt_grad_buckets")
+    a, b = (ctypes.c_size_t * n)(), (ctypes.c_size_t * n)()
+    LIB.gpt_grad_buckets(ctypes.byref(cfg.c()), a, b, n)
+    return [(int(a[i]), int(b[i])) for i in range(n)]
 
 
 def loss_terms(cfg, acts: torch.Tensor, B: int, T: int) -> torch.Tensor:

@@ -471,7 +471,19 @@ int gpt_forward_train(const gpt_config_t* cfg, const void* weights, const int64_
 size_t gpt_train_loss_terms_offset(const gpt_config_t* cfg, int B, int T);
 int gpt_backward(const gpt_config_t* cfg, const void* weights, const int64_t* idx, const int64_t* targets,
                  int B, int T, const void* acts, size_t acts_bytes, float* grads, float loss_scale,
-                 void* workspace, size_t workspace_bytes, void* stream, int flags);
+                 void* workspace, size_t workspace_bytes, void* stream, int flags,
+                 void* const* bucket_events);
+
+/* Gradient buckets for overlapping a data-parallel gradient reduction with the backward ("nanoGPT
+ * 全局流程图" 3.4 and the per-GPU batch of "nanoGPT 核心代码速查表" 七): n_layer + 1 element ranges
+ * [starts[i], stops[i]) of the flat fp32 gradient array, in the order gpt_backward finishes them:
+ * bucket i < n_layer holds every parameter of layer n_layer - 1 - i (bucket 0 also ln_f's), bucket
+ * n_layer holds wte and wpe (complete only after the embedding's gradient, the last step).  Together
+ * they cover the array once.  gpt_backward's bucket_events (NULL, or n_layer + 1 cudaEvent_t handles,
+ * entries may be NULL): event i is recorded on `stream` right after the last kernel that writes
+ * bucket i, so another stream may wait on it and reduce that range while the backward goes on.
+ * Returns n_layer + 1 (filling at most n entries; either array may be NULL) or a negative status. */
+int gpt_grad_buckets(const gpt_config_t* cfg, size_t* starts, size_t* stops, int n);
 
 #ifdef __cplusplus
 }

@@ -120,3 +120,84 @@ def test_sharded_gradients_match_full_batch(tmp_path, world, batch):
     mp.spawn(_grad_rank_main, args=(world, _free_port(), batch, str(out)), nprocs=world, join=True)
     err, scale = np.load(out)
     assert err <= 1e-6 * scale                     # fp32 transport of fp64 gradients
+
+
+def test_gradient_buckets_cover_the_array_in_backward_order():
+    """gpt_grad_buckets: n_layer + 1 disjoint ranges covering the flat gradient array once; bucket i
+    < n_layer holds every tensor of layer n_layer - 1 - i (bucket 0 also ln_f), the last one wte and
+    wpe -- the order in which the backward completes them."""
+    from decoder_only_transformer_causal_b200 import native
+    from decoder_only_transformer_causal_b200.native import GPTConfig
+    for name in ("tiny", "gpt2"):
+        cfg = GPTConfig.from_dict(seeded.WORKLOADS[name].model_dict())
+        buckets = native.grad_buckets(cfg)
+        L = cfg.n_layer
+        assert len(buckets) == L + 1
+        spans = sorted(buckets)
+        assert spans[0][0] == 0 and spans[-1][1] == native.param_elems(cfg)
+        assert all(spans[i][1] == spans[i + 1][0] for i in range(len(spans) - 1))
+        es = 2 if cfg.dtype == "bf16" else 4
+        entries, _ = native.weights_layout(cfg)
+        for tname, off, numel in entries:
+            a, b = off // es, off // es + numel
+            if tname.startswith("h."):
+                i = L - 1 - int(tname.split(".")[1])
+            elif tname.startswith("ln_f"):
+                i = 0
+            else:
+                i = L
+            assert buckets[i][0] <= a and b <= buckets[i][1], (tname, i)
+
+
+def _bucket_rank_main(rank, world, port, batch, out_path):
+    """The bucketed reduction of the packed flat gradient array (the layout gpt_backward writes),
+    with the buckets in the backward's order: equal to the whole batch's oracle gradient."""
+    import oracle.backward as ob
+    from decoder_only_transformer_causal_b200 import native
+    from decoder_only_transformer_causal_b200.data_parallel import allreduce_grads_bucketed
+    from decoder_only_transformer_causal_b200.native import GPTConfig
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        cfgd = dict(TINY, n_layer=2)
+        cfg = GPTConfig.from_dict(cfgd)
+        W = seeded.to_f64(seeded.make_weights(cfgd, stress=True))
+        idx, tgt = seeded.make_tokens(batch, 16, cfgd["vocab_size"], ignore_frac=0.3)
+        tgt[0, :12] = -1
+        a, b = shard_range(batch, world, rank)
+        entries, _ = native.weights_layout(cfg)
+
+        def flatten(g, scale):
+            flat = torch.zeros(native.param_elems(cfg), dtype=torch.float32)
+            for n, off, numel in entries:
+                flat[off // 4: off // 4 + numel] = torch.from_numpy((g[n] * scale).ravel().astype(np.float32))
+            return flat
+        sc = torch.zeros(2, dtype=torch.float64)
+        flat = torch.zeros(native.param_elems(cfg), dtype=torch.float32)
+        if b > a:
+            g, _ = ob.backward(W, cfgd, idx[a:b].numpy(), tgt[a:b].numpy())
+            n_r = float((tgt[a:b] != -1).sum())
+            sc[1] = n_r
+            allreduce_loss_terms(sc)
+            flat = flatten(g, n_r / float(sc[1]))
+        else:
+            allreduce_loss_terms(sc)
+        order = []
+        allreduce_grads_bucketed(flat, native.grad_buckets(cfg), wait=order.append)
+        if rank == 0:
+            g_full, _ = ob.backward(W, cfgd, idx.numpy(), tgt.numpy())
+            ref = flatten(g_full, 1.0).numpy()
+            np.save(out_path, np.array([np.abs(flat.numpy() - ref).max(), np.abs(ref).max(),
+                                        float(order == list(range(cfg.n_layer + 1)))]))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,batch", [(2, 3), (3, 4)])
+def test_bucketed_gradients_match_full_batch(tmp_path, world, batch):
+    out = tmp_path / "b.npy"
+    mp.spawn(_bucket_rank_main, args=(world, _free_port(), batch, str(out)), nprocs=world, join=True)
+    err, scale, in_order = np.load(out)
+    assert in_order == 1.0
+    assert err <= 1e-6 * scale

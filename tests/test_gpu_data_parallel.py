@@ -45,14 +45,17 @@ def single_rank_group():
         dist.destroy_process_group()
 
 
-def test_sharded_step_equals_single_gpu_step(single_rank_group):
+@pytest.mark.parametrize("overlap", [True, False])
+def test_sharded_step_equals_single_gpu_step(single_rank_group, overlap):
+    """With overlap, the gradient buckets are reduced on a second stream as gpt_backward's events
+    fire; the result must not depend on it."""
     from decoder_only_transformer_causal_b200.data_parallel import train_step_sharded
     B, T = 2, 128
     idx, tgt = _tokens(B, T)
     a, b = _trainer(B, T), _trainer(B, T)
     for _ in range(2):
         la = a.step(idx, tgt)
-        lb = train_step_sharded(b, idx, tgt)
+        lb = train_step_sharded(b, idx, tgt, overlap=overlap)
         torch.cuda.synchronize()
         assert torch.equal(a.loss, b.loss)
         assert abs(float(lb) - float(la)) <= 1e-6 * abs(float(la))
