@@ -444,6 +444,18 @@ int decode_step_impl(const gpt_config_t* c, const Weights& W, const int64_t* tok
     void* h = ws + P.h;
     float* part = reinterpret_cast<float*>(ws + D.part);
     int* counter = reinterpret_cast<int*>(ws + D.counter);
+    if (decode_persistent_supported(dt, B, C, hs, V, c->bias)) {
+        // the whole step in one cooperative launch with grid barriers between its phases
+        long long off[kTensorsPerLayer];
+        for (int i = 0; i < kTensorsPerLayer; ++i) off[i] = static_cast<long long>(W.in_layer[i]);
+        return launch_decode_persistent(W.wte(), W.wpe(), W.layer(0, 0), static_cast<long long>(W.layer_bytes), off,
+                                        c->bias, W.lnf_w(), W.lnf_b(), tok, ld_tok, kv,
+                                        static_cast<long long>(kv_layer_bytes(c, B) / 2), logits, ldl, pos, x, q, y,
+                                        h, part, counter,
+                                        static_cast<int>(decode_attn_part_floats(1, 1, hs, bs) / (hs + 2)),
+                                        reinterpret_cast<unsigned*>(ws + 8), status, B, C, nh, V, c->n_layer, bs, gt,
+                                        s);
+    }
     GPT_TRY(launch_embed_pos(W.wte(), W.wpe(), tok, ld_tok, pos, x, B, C, V, bs, dt, status, s));
     for (int l = 0; l < c->n_layer; ++l) {
         uint8_t* kvl = kv + kv_layer_bytes(c, B) * l;
@@ -530,6 +542,7 @@ GPT_API int gpt_set_wait_limit_ns(unsigned long long ns, int force_timeout) {
     GPT_TRY(set_wait_limit_attention(ns, force_timeout));
     GPT_TRY(set_wait_limit_gemm(ns, force_timeout));
     GPT_TRY(set_wait_limit_head(ns, force_timeout));
+    GPT_TRY(set_wait_limit_decode(ns, force_timeout));
     return set_wait_limit_attention_bwd(ns, force_timeout);
 }
 

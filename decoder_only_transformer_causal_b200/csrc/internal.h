@@ -140,6 +140,18 @@ int set_wait_limit_attention(unsigned long long ns, int force);
 int set_wait_limit_gemm(unsigned long long ns, int force);
 int set_wait_limit_attention_bwd(unsigned long long ns, int force);
 int set_wait_limit_head(unsigned long long ns, int force);
+int set_wait_limit_decode(unsigned long long ns, int force);
+
+// ---- one decode step as a single cooperative kernel (decode_persistent.cu): bf16, B <= 16,
+// C % 128 == 0 and C <= 1024, head size % 8 == 0 and <= 64, V % 8 == 0, and a shared-memory plan
+// that fits.  bar: a word zeroed per launch (set here).
+bool decode_persistent_supported(int dtype, int B, int C, int hs, int V, int has_bias);
+int launch_decode_persistent(const void* wte, const void* wpe, const void* layer0, long long layer_bytes,
+                             const long long (&off)[12], int has_bias, const void* lnf_w, const void* lnf_b,
+                             const int64_t* tok, long long ld_tok, void* kv, long long kv_layer_elems, float* logits,
+                             long long ldl, int* pos, float* x, void* q, void* y, void* h, float* part,
+                             int* counter, int n_split_max, unsigned* bar, int32_t* status, int B, int C, int nh,
+                             int V, int L, int block_size, int gelu_tanh, cudaStream_t s);
 
 // ---- the inference branch's head (head_last.cu): logits[b, :] = LayerNorm(x_b; lnw, lnb) wte^T
 // for B rows x + b * ldx (fp32, 16-byte aligned rows); logits bf16 at out + b * ldo.  C % 8 == 0

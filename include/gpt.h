@@ -128,10 +128,11 @@ int gpt_check_status(void* workspace, void* stream);
  * wait gives up records GPT_ERR_TIMEOUT in its status word, lets every copy and product it has
  * already issued finish (those drains keep the default limit), releases its tensor memory and
  * returns; its outputs are then invalid.
- *   force_timeout != 0 makes the causal attention kernel and the product kernels (gpt_linear,
- *   single CTAs for M < 256 and CTA pairs from M = 256) launched from then on wait first for an
- *   event that never happens, so their time-out path runs on purpose after `ns`; 0 turns that
- *   off.
+ *   force_timeout != 0 makes the causal attention kernel, the product kernels (gpt_linear,
+ *   single CTAs for M < 256 and CTA pairs from M = 256) and the single-launch decode step
+ *   (gpt_decode_step and gpt_generate in bf16, at its first grid barrier) launched from then on
+ *   wait first for an event that never happens, so their time-out path runs on purpose after
+ *   `ns`; 0 turns that off.  A decode step that timed out leaves the position where it was.
  * Call it with no kernel of this library running or queued on the device (it copies to the device
  * synchronously).  Returns GPT_OK or GPT_ERR_CUDA. */
 int gpt_set_wait_limit_ns(unsigned long long ns, int force_timeout);

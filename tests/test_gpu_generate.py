@@ -147,6 +147,28 @@ def test_decode_steps_match_forward(name, stress, layers, B, T0, n, steps, gelu)
         assert err <= tol, (s, err)
 
 
+PLAN_CASES = [
+    # workload, layers, B, T0, n_forced, bias, gelu: the single-launch decode step's shared-memory
+    # plans (four weight slots for GPT-2 124M; two for C = 1024 with B <= 8; one for C = 1024, B > 8)
+    ("gpt2-medium", 2, 2, 70, 3, True, "erf"),
+    ("gpt2-medium", 2, 12, 70, 2, True, "erf"),
+    ("gpt2", 2, 16, 63, 3, False, "tanh"),        # 16 sequences, no biases; 64 -> 65 keys: a new chunk
+]
+
+
+@pytest.mark.parametrize("name,layers,B,T0,n,bias,gelu", PLAN_CASES)
+def test_decode_step_plans_match_forward(name, layers, B, T0, n, bias, gelu):
+    cfg, W, W64, _, _ = model_inputs(name, stress=True, n_layer=layers, bias=bias)
+    V = cfg["vocab_size"]
+    prompt, _ = seeded.make_tokens(B, T0, min(V, 50257), seed=9011)
+    forced, _ = seeded.make_tokens(B, n, min(V, 50257), seed=9012)
+    got = decode_logits_gpu(cfg, W, prompt, forced, gelu)
+    ref = decode_logits_oracle(cfg, W64, prompt, forced, range(n + 1), gelu)
+    for s, r in ref.items():
+        err = max_abs(got[s], r)
+        assert err <= BF16_ATOL, (s, err)
+
+
 def test_decode_past_window_is_reported_and_writes_nothing():
     from decoder_only_transformer_causal_b200 import native
     cfg, W, _, _, _ = model_inputs("tiny", stress=True)

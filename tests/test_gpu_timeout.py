@@ -1,4 +1,5 @@
-"""The time-out path of the tensor-core kernels, made to run on purpose without faulting the GPU.
+"""The time-out path of the tensor-core kernels and of the single-launch decode step, made to run on
+purpose without faulting the GPU.
 
 Every pipeline wait in the tensor-core kernels is bounded: when a wait gives up, the kernel records
 GPT_ERR_TIMEOUT in its status word, lets the copies and products it already issued finish, frees
@@ -69,3 +70,35 @@ def test_gemm_wait_limit_gives_timeout_then_recovers(short_waits, M):
     assert int(st.item()) == native.GPT_OK
     ref = x.float() @ W.float().T + b.float()
     assert float((out.float() - ref).abs().max()) <= 2e-2
+
+
+def test_decode_step_wait_limit_gives_timeout_then_recovers():
+    """The single-launch decode step waits at its first grid barrier for an arrival that never
+    comes: every CTA gives up after 1 ms, lets its weight copies land and returns, the position stays
+    where it was, and the next step (limits restored) gives the logits of an undisturbed step."""
+    import seeded
+    from decoder_only_transformer_causal_b200 import GPT, GPTConfig, native
+    from gpu_helpers import model_inputs
+    cfg_d, W, _, _, _ = model_inputs("gpt2", stress=True, n_layer=2)
+    m = GPT(GPTConfig.from_dict(cfg_d), W)
+    B, T0 = 1, 40
+    prompt, _ = seeded.make_tokens(B, T0, 50257, seed=9021)
+    tok = torch.tensor([123], dtype=torch.int64, device="cuda")
+    runs = []
+    for forced in (False, True):
+        kv = native.alloc_kv_cache(m.cfg, B)
+        ws = native.alloc_workspace(native.decode_workspace_bytes(m.cfg, B, T0))
+        native.prefill(m.cfg, m.weights, prompt.cuda(), kv, ws, sync_check=True)
+        if forced:
+            torch.cuda.synchronize()
+            native.set_wait_limit_ns(1_000_000, force_timeout=True)
+            try:
+                native.decode_step(m.cfg, m.weights, tok, kv, ws)
+                assert native.check_status(ws) == native.GPT_ERR_TIMEOUT
+            finally:
+                torch.cuda.synchronize()
+                native.set_wait_limit_ns(0)
+        logits = native.decode_step(m.cfg, m.weights, tok, kv, ws, sync_check=True).clone()
+        assert native.check_status(ws) == native.GPT_OK
+        runs.append(logits)
+    assert torch.equal(runs[0], runs[1])
