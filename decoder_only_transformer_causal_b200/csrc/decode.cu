@@ -546,9 +546,9 @@ constexpr int kSampleMaxV = 52 * 1024;  // the row in shared memory: 208 KB (plu
 // One CTA per row stages the row in shared memory (V <= kSampleMaxV) and, in the same pass,
 // counts the order-preserving 32-bit keys by their top 11 bits.  A scan from the top bin finds
 // the bin holding the top_k-th largest key; its members (few, for a top-k of a spread-out
-// row) are gathered and the remaining 21 bits found by bisection over them: the largest t with
-// count(key >= t) >= top_k is the k-th largest key itself.  (A bin with more than
-// kSampleCand members is bisected over the whole row instead.)  For the draw, warp w owns the
+// row) are gathered and two more histogram levels over them (bits 20..10, then 9..0) give the
+// k-th largest key itself.  (A bin with more than kSampleCand members is bisected over the whole
+// row instead: the largest t with count(key >= t) >= top_k.)  For the draw, warp w owns the
 // contiguous segment [w*seg, (w+1)*seg): the exponentials are fp32 and their sums fp64 (one
 // entry's share of a flat distribution over tens of thousands of entries is not far above
 // fp32 accumulation error).  Every thread adds the 32 segment sums in the same order, so
@@ -569,6 +569,32 @@ GPT_DEVINL uint32_t block_count(uint32_t c, uint32_t* acc, int& phase) {
     __syncthreads();
     ++phase;
     return *cur;
+}
+
+// Scan of hist[0, 2048) from the top bin down: the bin that holds the need-th largest entry
+// (need >= 1 and at most the histogram's total), and that entry's rank inside the bin, into
+// *s_bin / *s_need.  kSampleThreads threads, two bins each.
+GPT_DEVINL void top_bin(const uint32_t* hist, uint32_t need, uint32_t* s_wtot, uint32_t* s_bin, uint32_t* s_need) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const uint32_t h0 = hist[kSampleBins - 1 - 2 * tid], h1 = hist[kSampleBins - 2 - 2 * tid];
+    uint32_t incl = h0 + h1;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t n = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += n;
+    }
+    if (lane == 31) s_wtot[warp] = incl;
+    __syncthreads();
+    uint32_t before = 0;
+    for (int w = 0; w < warp; ++w) before += s_wtot[w];
+    incl += before;
+    const uint32_t excl = incl - h0 - h1;
+    if (excl < need && incl >= need) {
+        const bool first = excl + h0 >= need;
+        *s_bin = first ? kSampleBins - 1 - 2 * tid : kSampleBins - 2 - 2 * tid;
+        *s_need = first ? need - excl : need - excl - h0;
+    }
+    __syncthreads();
 }
 
 __global__ void __launch_bounds__(kSampleThreads)
@@ -593,11 +619,23 @@ __global__ void __launch_bounds__(kSampleThreads)
     if (tid == 0) s_ncand = 0;
     __syncthreads();
     float mx = -INFINITY;
-    for (int i = tid; i < V; i += kSampleThreads) {
-        const float v = __ldcg(lg + i);
-        zs[i] = v;
-        mx = fmaxf(mx, v);
-        if (filter) atomicAdd(&hist[fkey(v) >> 21], 1u);
+    // eight loads in flight per thread (the row is ~50 loads per thread for V 50304)
+    for (int i0 = tid; i0 < V; i0 += 8 * kSampleThreads) {
+        float v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int i = i0 + j * kSampleThreads;
+            v[j] = i < V ? __ldcg(lg + i) : 0.f;
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int i = i0 + j * kSampleThreads;
+            if (i < V) {
+                zs[i] = v[j];
+                mx = fmaxf(mx, v[j]);
+                if (filter) atomicAdd(&hist[fkey(v[j]) >> 21], 1u);
+            }
+        }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
@@ -609,43 +647,30 @@ __global__ void __launch_bounds__(kSampleThreads)
 
     uint32_t thr_key = 0;  // key of the top_k-th largest logit
     if (filter) {
-        // bins from the top: thread t holds bins 2047-2t and 2046-2t
-        const uint32_t h0 = hist[kSampleBins - 1 - 2 * tid], h1 = hist[kSampleBins - 2 - 2 * tid];
-        uint32_t incl = h0 + h1;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t n = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += n;
-        }
-        if (lane == 31) s_wtot[warp] = incl;
-        __syncthreads();
-        uint32_t before = 0;
-        for (int w = 0; w < warp; ++w) before += s_wtot[w];
-        incl += before;
-        const uint32_t excl = incl - h0 - h1, need = static_cast<uint32_t>(top_k);
-        if (excl < need && incl >= need) {
-            const bool first = excl + h0 >= need;
-            s_bin = first ? kSampleBins - 1 - 2 * tid : kSampleBins - 2 - 2 * tid;
-            s_need = first ? need - excl : need - excl - h0;
-        }
-        __syncthreads();
+        top_bin(hist, static_cast<uint32_t>(top_k), s_wtot, &s_bin, &s_need);
         const uint32_t bin = s_bin, need2 = s_need;
         const uint32_t nbin = hist[bin];
         int phase = 0;
         uint32_t lo = bin << 21, hi = lo | ((1u << 21) - 1);  // invariant: count(key >= lo) >= need
         if (nbin <= kSampleCand) {
+            // the bin's members, then two more histogram levels over them: bits 20..10, 9..0
             for (int i = tid; i < V; i += kSampleThreads) {
                 const uint32_t key = fkey(zs[i]);
                 if ((key >> 21) == bin) cand[atomicAdd(&s_ncand, 1u)] = key;
             }
+            for (int i = tid; i < kSampleBins; i += kSampleThreads) hist[i] = 0;
             __syncthreads();
-            for (int it = 0; it < 22 && lo < hi; ++it) {  // the range halves: 21 steps suffice
-                const uint32_t mid = lo + (hi - lo + 1) / 2;
-                uint32_t c = 0;
-                for (uint32_t i = tid; i < nbin; i += kSampleThreads) c += cand[i] >= mid;
-                if (block_count(c, s_acc, phase) >= need2) lo = mid;
-                else hi = mid - 1;
-            }
+            for (uint32_t i = tid; i < nbin; i += kSampleThreads) atomicAdd(&hist[(cand[i] >> 10) & 2047u], 1u);
+            __syncthreads();
+            top_bin(hist, need2, s_wtot, &s_bin, &s_need);
+            const uint32_t bin2 = s_bin, need3 = s_need;
+            for (int i = tid; i < kSampleBins; i += kSampleThreads) hist[i] = 0;
+            __syncthreads();
+            for (uint32_t i = tid; i < nbin; i += kSampleThreads)
+                if (((cand[i] >> 10) & 2047u) == bin2) atomicAdd(&hist[cand[i] & 1023u], 1u);
+            __syncthreads();
+            top_bin(hist, need3, s_wtot, &s_bin, &s_need);  // bins 1024.. are empty
+            lo = (bin << 21) | (bin2 << 10) | s_bin;
         } else {
             for (int it = 0; it < 22 && lo < hi; ++it) {
                 const uint32_t mid = lo + (hi - lo + 1) / 2;
