@@ -22,7 +22,7 @@
 // and the LayerNorm weights that precede c_attn and c_fc) are copied into shared memory by bulk
 // copies (cp.async.bulk, one per row, rows padded by 16 bytes so that fragment loads are free of
 // bank conflicts).  A slot is refilled as soon as its product is done, between the CTA's arrival at
-// the barrier and its wait, by warp 1 while thread 0 waits: with S = 4 slots the next layer's
+// the barrier and its wait, one copy per thread: with S = 4 slots the next layer's
 // weights are in flight while this one runs; smaller shared-memory budgets (larger B or C) use S = 2
 // or 1.  The products are tensor-core mma.sync m16n8k16 (bf16 in, fp32 accumulate): up to 16 staged
 // rows are the A operand, 8 weight rows the B operand, K split over the CTA's warps when it owns
@@ -181,34 +181,34 @@ GPT_DEVINL void cp_async16(void* dst, const void* src, int src_bytes) {
 // Waits for every cp.async this thread has issued.
 GPT_DEVINL void cp_async_wait_all() { asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory"); }
 
-// Warp 1: bulk copies of this CTA's rows (and bias) of weight phase j into its slot.
+// Bulk copies of this CTA's rows (and bias, and the LayerNorm weights) of weight phase j into its
+// slot, one copy per thread (thread i: row i), so that their issue runs in parallel.
 GPT_DEVINL void issue_phase(Ctx& c, int j) {
     const StepArgs& a = c.a;
-    // warp 1 issues, so that thread 0 (warp 0) is free to wait at the grid barrier meanwhile
-    if (j >= 4 * a.L || (threadIdx.x >> 5) != 1) return;
-    const int lane = threadIdx.x & 31;
+    if (j >= 4 * a.L) return;
     int N, K, t0, t1;
     const bf16 *W, *bias;
     phase_shape(a, j & 3, j >> 2, N, K, W, bias);
     cta_tiles(N, t0, t1);
     const int nrows = (t1 - t0) * kTile;
     const int si = slot_of(a, j), x = j & 3, lnb = ln_bytes(a, x);
+    const int n_ln = lnb ? (a.has_bias ? 2 : 1) : 0;
+    const int n_copies = n_ln + nrows + (bias && nrows ? 1 : 0);
+    const int i = threadIdx.x;
     uint8_t* dst = c.smem + a.slot_off[si];
     const uint32_t row_bytes = static_cast<uint32_t>(K) * 2, ld_bytes = static_cast<uint32_t>(K + kPad) * 2;
-    fence_proxy_async_shared();  // this CTA's earlier reads of the slot, before the async writes
-    if (lane == 0) mbar_arrive_expect_tx(c.slot_bar + si, lnb + nrows * row_bytes + (bias ? nrows * 2 : 0));
-    __syncwarp();
-    if (lnb && lane < (a.has_bias ? 2 : 1)) {
-        const int t = (x == P_QKV ? T_LN1W : T_LN2W) + lane;
-        bulk_load_1d(dst + lane * a.C * 2, tensor(a, j >> 2, t), a.C * 2, c.slot_bar + si);
-    }
-    dst += lnb;
-#pragma unroll 1
-    for (int r = lane; r < nrows; r += 32)
-        bulk_load_1d(dst + static_cast<size_t>(r) * ld_bytes, W + static_cast<long long>(t0 * kTile + r) * K,
+    if (i == 0) mbar_arrive_expect_tx(c.slot_bar + si, lnb + nrows * row_bytes + (bias ? nrows * 2 : 0));
+    if (i >= n_copies) return;
+    fence_proxy_async_shared();  // this CTA's earlier reads of the slot (ordered by a CTA barrier)
+    if (i < n_ln) {
+        bulk_load_1d(dst + i * a.C * 2, tensor(a, j >> 2, (x == P_QKV ? T_LN1W : T_LN2W) + i), a.C * 2, c.slot_bar + si);
+    } else if (i < n_ln + nrows) {
+        const int r = i - n_ln;
+        bulk_load_1d(dst + lnb + static_cast<size_t>(r) * ld_bytes, W + static_cast<long long>(t0 * kTile + r) * K,
                      row_bytes, c.slot_bar + si);
-    if (bias && nrows && lane == 0)
-        bulk_load_1d(dst + static_cast<size_t>(nrows) * ld_bytes, bias + t0 * kTile, nrows * 2, c.slot_bar + si);
+    } else {
+        bulk_load_1d(dst + lnb + static_cast<size_t>(nrows) * ld_bytes, bias + t0 * kTile, nrows * 2, c.slot_bar + si);
+    }
 }
 
 // Waits until weight phase j has landed; the result is the same for every thread of the CTA.
@@ -468,7 +468,7 @@ GPT_DEVINL void product(const StepArgs& a, int out, const bf16* us, int ldu, con
 // 8, 4, 2 or 1 warps of one CTA, which take 64-key chunks in turn.
 GPT_DEVINL int attention_cpu(const StepArgs& a) {
     const int cpu = static_cast<int>(gridDim.x) / (a.B * a.nh);
-    return cpu >= 2 ? min(min(cpu, a.n_split_max), 16) : 1;
+    return cpu >= 2 ? min(min(cpu, a.n_split_max), 4) : 1;  // 4 measured best at B 1 (of 1, 4, 12)
 }
 GPT_DEVINL int attention_wpu(const StepArgs& a) {
     if (attention_cpu(a) > 1) return kWarps;
@@ -837,7 +837,9 @@ bool decode_persistent_supported(int dtype, int B, int C, int hs, int V, int has
         return false;
     const int grid = num_sms();
     SmemPlan sp;
-    return grid > 0 && (C / kTile + grid - 1) / grid * kTile <= kResidCols && plan_smem(B, C, has_bias != 0, grid, sp);
+    // residual columns per CTA fit the addend buffer; a phase's copies (rows + LayerNorm + bias) fit one per thread
+    return grid > 0 && (C / kTile + grid - 1) / grid * kTile <= kResidCols &&
+           (4 * C / kTile + grid - 1) / grid * kTile + 3 <= kThreads && plan_smem(B, C, has_bias != 0, grid, sp);
 }
 
 int launch_decode_persistent(const void* wte, const void* wpe, const void* layer0, long long layer_bytes,
