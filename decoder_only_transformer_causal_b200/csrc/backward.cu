@@ -201,12 +201,20 @@ __global__ void __launch_bounds__(kBwdWarps * 32)
 }
 
 // The same with each row held in registers (VEC float4 of x and of dy per lane, C <= 128 VEC):
-// x and dy are read once; each warp takes kLnRowsPerWarp consecutive rows.  Up to C = 768 (VEC 6)
+// x and dy are read once; each warp takes ln_rows_per_warp(rows) consecutive rows.  Up to C = 768 (VEC 6)
 // the next row's x, dy (and the dx it adds to) are loaded while the current one is reduced and
 // the lanes' dw / db column sums stay in registers; wider rows (whose registers would spill) load
 // row by row and add into per-warp sums in shared memory.  The warps' sums meet in warp order, so
-// a CTA leaves one partial per 32 rows.
-constexpr int kLnRowsPerWarp = 4;  // rows per warp in the register kernel: 32 per CTA
+// a CTA leaves one partial per kBwdWarps * ln_rows_per_warp(rows) rows.
+constexpr int kLnRowsPerWarp = 4;  // rows per warp in the register kernel, at least
+
+// Rows per warp of the register kernel: enough that the grid is one wave of CTAs (one per SM), so
+// no SM idles in a partial last wave and every warp's one-row lookahead runs over many rows.
+int ln_rows_per_warp(int rows) {
+    const int sms = num_sms() > 0 ? num_sms() : 148;
+    const int per = (rows + sms * kBwdWarps - 1) / (sms * kBwdWarps);
+    return per > kLnRowsPerWarp ? per : kLnRowsPerWarp;
+}
 
 template <int VEC>
 struct LnRow {
@@ -231,7 +239,7 @@ template <typename Tw, int VEC>
 __global__ void __launch_bounds__(kBwdWarps * 32)
     layernorm_backward_reg_kernel(const float* __restrict__ dy, const float* __restrict__ x, const Tw* __restrict__ w,
                                   float* __restrict__ dx, int accumulate, float* __restrict__ part, int rows, int C,
-                                  bf16* __restrict__ dx16) {
+                                  bf16* __restrict__ dx16, int rows_per_warp) {
     griddep_launch_dependents();
     griddep_wait();
     extern __shared__ float sm[];  // [kBwdWarps][2][C] per-warp column sums
@@ -251,8 +259,8 @@ __global__ void __launch_bounds__(kBwdWarps * 32)
         for (int c = lane; c < 2 * C; c += 32) my[c] = 0.f;
         __syncwarp();
     }
-    const int r0 = (blockIdx.x * kBwdWarps + warp) * kLnRowsPerWarp;
-    const int r1 = min(rows, r0 + kLnRowsPerWarp);
+    const int r0 = (blockIdx.x * kBwdWarps + warp) * rows_per_warp;
+    const int r1 = min(rows, r0 + rows_per_warp);
     LnRow<VEC> cur, nxt;
     if (kPipe && r0 < r1) {
         const long long o = static_cast<long long>(r0) * C;
@@ -532,7 +540,7 @@ int launch_ce_backward(const void* logits, int dtype, const int64_t* targets, co
 }
 
 int layernorm_backward_parts(int rows, int C) {
-    const int per = (C <= 2048 && C % 4 == 0) ? kBwdWarps * kLnRowsPerWarp : kBwdWarps;
+    const int per = (C <= 2048 && C % 4 == 0) ? kBwdWarps * ln_rows_per_warp(rows) : kBwdWarps;
     return (rows + per - 1) / per;
 }
 
@@ -548,7 +556,7 @@ int launch_ln_bwd_reg(const float* dy, const float* x, const void* w, float* dx,
     if (rc) return rc;
     return launch_overlapped(layernorm_backward_reg_kernel<Tw, VEC>, dim3(layernorm_backward_parts(rows, C)),
                              dim3(kBwdWarps * 32), smem, s, dy, x, static_cast<const Tw*>(w), dx, accumulate, part,
-                             rows, C, dx16);
+                             rows, C, dx16, ln_rows_per_warp(rows));
 }
 }  // namespace
 
