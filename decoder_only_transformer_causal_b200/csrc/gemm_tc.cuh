@@ -417,7 +417,20 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)  // 10 warps: <= 168 regi
             }
             long long tgt = -1;
             if (EPI == EPI_CE && row_ok) tgt = p.targets[row];
-            // EPI_DGELU: the first chunk's pre-activations, loaded before the accumulator wait
+            // EPI_DGELU: this row's slice of the next tile's GELU derivatives goes to L2 now (one
+            // tile ahead, so its chunk loads below hit L2), then the first chunk's values are loaded
+            // before the accumulator wait
+            if (EPI == EPI_DGELU && tile + n_units < num_tiles) {
+                int m_nx, n_nx;
+                tile_mn(tile + n_units, m_nx, n_nx);
+                const int row_nx = m_nx * TM + static_cast<int>(rank) * BM + quarter * 32 + lane;
+                const int n_first = n_nx * BN + half * COLS;
+                if (row_nx < p.M && n_first + COLS <= p.N)
+                    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(
+                                     p.aux + static_cast<long long>(row_nx) * p.ld_aux + n_first),
+                                 "r"(static_cast<uint32_t>(COLS * 2))
+                                 : "memory");
+            }
             uint32_t aux_next[EPI == EPI_DGELU ? 16 : 1];
             bool aux_ok = false;
             if (EPI == EPI_DGELU && row_ok && nw0 + 32 <= p.N) {
