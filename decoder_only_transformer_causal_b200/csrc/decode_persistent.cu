@@ -31,7 +31,8 @@
 //
 // Attention: with at least two CTAs per (sequence, head) unit, cpu CTAs share a unit (each an equal
 // share of the keys, split again over its 8 warps; the last CTA to finish, by a per-unit ticket,
-// merges their partials); otherwise a unit gets 8, 4, 2 or 1 warps of one CTA.  A warp copies up to
+// merges their partials); otherwise (larger batches) each unit's keys are split over single warps
+// anywhere in the grid, merged by the unit's last warp.  A warp copies up to
 // 32 key and value rows with cp.async, lane t scores key t, and lane l accumulates output
 // dimensions 2l, 2l + 1 (online softmax across chunks).  The cache rows are prefetched into L2 a
 // phase ahead.  Data written during the step (residual, q, the cache, y, h) is read through L2
@@ -476,6 +477,17 @@ GPT_DEVINL int attention_wpu(const StepArgs& a) {
     return per >= 8 ? 8 : per >= 4 ? 4 : per >= 2 ? 2 : 1;
 }
 
+// Warp-level split (used when attention_cpu is 1): every (sequence, head) unit is cut into `parts`
+// equal key ranges (parts <= 16, each at least one 32-key chunk, as many as the grid's warps
+// allow), and global warp
+// g takes items g, g + W, ... (item = unit * parts + part).  Each warp leaves its partial (m, l, O)
+// in global memory; the last warp of a unit to finish (a per-unit ticket) merges them.
+GPT_DEVINL int attention_parts(const StepArgs& a, int n_keys) {
+    const int per = static_cast<int>(gridDim.x) * kWarps / (a.B * a.nh);
+    const int by_keys = (n_keys + kChunk - 1) / kChunk;
+    return max(1, min(min(per, by_keys), min(a.n_split_max, 16)));
+}
+
 // L2 prefetch of [p, p + bytes) by the calling warp, in pieces of at most 32 KB spread over its
 // lanes.  p and bytes are multiples of 16.
 GPT_DEVINL void prefetch_span(const void* p, size_t bytes) {
@@ -524,7 +536,108 @@ GPT_DEVINL void prefetch_kv(const StepArgs& a, int layer, int p) {
     }
 }
 
-// Attention of the newest position over the cache [0, p] for every (sequence, head).
+// Attention when there are at least as many (sequence, head) units as CTAs (larger batches): the
+// units' key ranges are split over single warps (attention_parts).  A warp
+// copies up to 32 key and value rows of its range (lane t: key k0 + t) and the query into its
+// staging area with cp.async, lane t scores key t, the warp takes the chunk's max and sum, and lane
+// l accumulates output dimensions 2l, 2l + 1 (online softmax across chunks).
+GPT_DEVINL void attention_warps(const StepArgs& a, int layer, int p, uint8_t* stage) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int C = a.C, hs = a.hs, nh = a.nh, nv16 = hs / 8;
+    const int n_keys = min(p + 1, a.block_size);
+    const int parts = attention_parts(a, n_keys), units = a.B * nh, items = units * parts;
+    const bf16* kvl = a.kv + a.kv_layer * layer;
+    bf16* ks = reinterpret_cast<bf16*>(stage + warp * kAttnWarpBytes);
+    bf16* vs = ks + kChunk * kKld;
+    bf16* qs = vs + kChunk * kMaxHs;
+    const int d = 2 * lane;  // this lane's output dimensions d, d + 1 (hs <= 64)
+    for (int it = blockIdx.x * kWarps + warp; it < items; it += gridDim.x * kWarps) {
+        const int u = it / parts, sh = it % parts;
+        const int b = u / nh, h = u % nh;
+        const int kb = sh * n_keys / parts, ke = (sh + 1) * n_keys / parts;
+        const bf16* base = kvl + static_cast<long long>(b) * a.block_size * 2 * C + h * hs;
+        if (lane < nv16) cp_async16(qs + 8 * lane, a.q + static_cast<long long>(b) * C + h * hs + 8 * lane, 16);
+        float m = -INFINITY, l = 0.f, o0 = 0.f, o1 = 0.f;
+#pragma unroll 1
+        for (int k0 = kb; k0 < ke; k0 += kChunk) {
+            const int nk = min(kChunk, ke - k0);
+            const bool in = lane < nk;
+            const bf16* kr = base + static_cast<long long>(k0 + (in ? lane : 0)) * 2 * C;
+#pragma unroll 1
+            for (int i = 0; i < nv16; ++i) {
+                cp_async16(ks + lane * kKld + 8 * i, kr + 8 * i, in ? 16 : 0);
+                cp_async16(vs + lane * kMaxHs + 8 * i, kr + C + 8 * i, in ? 16 : 0);
+            }
+            cp_async_wait_all();
+            __syncwarp();
+            float sc = 0.f;
+#pragma unroll 1
+            for (int i = 0; i < nv16; ++i) {
+                float kf[8], qf[8];
+                unpack8(*reinterpret_cast<const uint4*>(ks + lane * kKld + 8 * i), kf);
+                unpack8(*reinterpret_cast<const uint4*>(qs + 8 * i), qf);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) sc = fmaf(qf[e], kf[e], sc);
+            }
+            sc = in ? sc * a.scale_log2 : -INFINITY;
+            float mc = sc;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) mc = fmaxf(mc, __shfl_xor_sync(0xffffffffu, mc, o));
+            const float mn = fmaxf(m, mc);    // finite: every chunk has a key (nk >= 1)
+            const float corr = exp2f(m - mn);  // 0 on the warp's first chunk (m = -inf)
+            const float pl = in ? exp2f(sc - mn) : 0.f;
+            l = l * corr + warp_sum(pl);
+            o0 *= corr;
+            o1 *= corr;
+            m = mn;
+            // lanes with 2 lane >= hs accumulate what lies past the copied dimensions and store nothing
+#pragma unroll 2
+            for (int t = 0; t < nk; ++t) {
+                const float pt = __shfl_sync(0xffffffffu, pl, t);
+                const __nv_bfloat162 v2 = *reinterpret_cast<const __nv_bfloat162*>(vs + t * kMaxHs + 2 * lane);
+                o0 = fmaf(pt, __low2float(v2), o0);
+                o1 = fmaf(pt, __high2float(v2), o1);
+            }
+            __syncwarp();  // the next chunk's copies overwrite the staging area
+        }
+        cp_async_wait_all();  // the query copy of a range without keys
+        __syncwarp();
+        bf16* yr = a.y + static_cast<long long>(b) * C + h * hs;
+        if (parts == 1) {
+            if (d < hs) *reinterpret_cast<__nv_bfloat162*>(yr + d) = __floats2bfloat162_rn(o0 / l, o1 / l);
+            continue;
+        }
+        // this warp's partial; the unit's last warp merges them:
+        // y = sum_i 2^(m_i - M) O_i / sum_i 2^(m_i - M) l_i
+        float* gp = a.part + (static_cast<long long>(u) * a.n_split_max + sh) * (hs + 2);
+        if (d < hs) __stcg(gp + 2 + d, o0), __stcg(gp + 3 + d, o1);
+        if (lane == 0) __stcg(gp, m), __stcg(gp + 1, l);
+        __threadfence();
+        __syncwarp();
+        int ticket = 0;
+        if (lane == 0) ticket = atomicAdd(a.counter + u, 1);
+        ticket = __shfl_sync(0xffffffffu, ticket, 0);
+        if (ticket != parts - 1) continue;
+        __threadfence();
+        const float* g0 = a.part + static_cast<long long>(u) * a.n_split_max * (hs + 2);
+        const float mine = lane < parts ? __ldcg(g0 + lane * (hs + 2)) : -INFINITY;  // parts <= 16
+        float M = mine;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        float L = 0.f, z0 = 0.f, z1 = 0.f;
+#pragma unroll 4
+        for (int i = 0; i < parts; ++i) {
+            const float mi = __shfl_sync(0xffffffffu, mine, i);
+            const float* gi = g0 + i * (hs + 2);
+            const float wgt = mi == -INFINITY ? 0.f : exp2f(mi - M);  // a range without keys: 0
+            L = fmaf(wgt, __ldcg(gi + 1), L);
+            if (d < hs) z0 = fmaf(wgt, __ldcg(gi + 2 + d), z0), z1 = fmaf(wgt, __ldcg(gi + 3 + d), z1);
+        }
+        if (d < hs) *reinterpret_cast<__nv_bfloat162*>(yr + d) = __floats2bfloat162_rn(z0 / L, z1 / L);
+        if (lane == 0) a.counter[u] = 0;
+    }
+}
+
 // Attention of the newest position over the cache [0, p] for every (sequence, head).  Per chunk of
 // up to 32 keys a warp copies the key and value rows (lane t: key k0 + t) and the query into its
 // staging area with cp.async, lane t scores key t, the warp takes the chunk's max and sum, and lane
@@ -719,7 +832,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const __grid_c
         }
         if (!(ok = grid_wait(c))) break;
         if (x == P_QKV) {
-            if (p >= 0) attention(a, l, p, red, smem + kFixedBytes);
+            if (p >= 0) {
+                if (attention_cpu(a) > 1)
+                    attention(a, l, p, red, smem + kFixedBytes);
+                else
+                    attention_warps(a, l, p, smem + kFixedBytes);
+            }
             if (!(ok = grid_sync(c))) break;
         }
     }
