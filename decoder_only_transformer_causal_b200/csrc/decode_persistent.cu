@@ -30,8 +30,8 @@
 // are sent to L2 while the last layer runs, and the next step's first weights at the end.
 //
 // Attention: with at least two CTAs per (sequence, head) unit, cpu CTAs share a unit (each an equal
-// share of the keys, split again over its 8 warps; the last CTA to finish, by a per-unit ticket,
-// merges their partials); otherwise (larger batches) each unit's keys are split over single warps
+// share of the keys, split again over its 8 warps; c_proj's staging merges their partials);
+// otherwise (larger batches) each unit's keys are split over single warps
 // anywhere in the grid, merged by the unit's last warp.  A warp copies up to
 // 32 key and value rows with cp.async, lane t scores key t, and lane l accumulates output
 // dimensions 2l, 2l + 1 (online softmax across chunks).  The cache rows are prefetched into L2 a
@@ -51,6 +51,7 @@ constexpr int kMaxRows = 16;     // sequences per launch (the mma's M)
 constexpr int kTile = 8;         // weight rows per tile (the mma's N)
 constexpr int kPad = 8;          // bf16 elements of padding per staged row
 constexpr int kChunk = 32;       // keys per attention chunk: a lane per key
+constexpr int kMaxCtaSplit = 4;  // CTAs sharing one (sequence, head): 4 measured best at B 1 (of 1, 4, 12)
 constexpr int kMaxHs = 64;       // head size (every GPT-2 size has 64)
 constexpr int kMaxC = 1024;      // a LayerNorm row lives in registers: C / 128 float4 per lane
 constexpr int kResidCols = 32;   // residual columns one CTA may own
@@ -469,7 +470,7 @@ GPT_DEVINL void product(const StepArgs& a, int out, const bf16* us, int ldu, con
 // 8, 4, 2 or 1 warps of one CTA, which take 64-key chunks in turn.
 GPT_DEVINL int attention_cpu(const StepArgs& a) {
     const int cpu = static_cast<int>(gridDim.x) / (a.B * a.nh);
-    return cpu >= 2 ? min(min(cpu, a.n_split_max), 4) : 1;  // 4 measured best at B 1 (of 1, 4, 12)
+    return cpu >= 2 ? min(min(cpu, a.n_split_max), kMaxCtaSplit) : 1;
 }
 GPT_DEVINL int attention_wpu(const StepArgs& a) {
     if (attention_cpu(a) > 1) return kWarps;
@@ -719,7 +720,7 @@ GPT_DEVINL void attention(const StepArgs& a, int layer, int p, float* part, uint
         }
         __syncthreads();
         // the unit's first warp merges its warps: y = sum_i 2^(m_i - M) O_i / sum_i 2^(m_i - M) l_i;
-        // with cpu > 1 the merged (M, L, O) is this CTA's partial
+        // with cpu > 1 the merged (M, L, O) is this CTA's partial, which c_proj's staging merges
         if (u < units && wi == 0) {
             const float* pw = part + warp * (2 + kMaxHs);
             float M = -INFINITY;
@@ -736,35 +737,49 @@ GPT_DEVINL void attention(const StepArgs& a, int layer, int p, float* part, uint
             if (cpu == 1) {
                 if (d < hs) *reinterpret_cast<__nv_bfloat162*>(yr + d) = __floats2bfloat162_rn(y0 / Ls, y1 / Ls);
             } else {
-                // this CTA's partial to global memory; the last CTA of the unit (a per-unit ticket)
-                // merges the cpu partials
+                // this CTA's partial to global memory, for c_proj's staging (the barrier orders it)
                 float* gp = a.part + (static_cast<long long>(u) * a.n_split_max + blockIdx.x % cpu) * (hs + 2);
                 if (d < hs) __stcg(gp + 2 + d, y0), __stcg(gp + 3 + d, y1);
                 if (lane == 0) __stcg(gp, M), __stcg(gp + 1, Ls);
-                __threadfence();
-                __syncwarp();
-                int ticket = 0;
-                if (lane == 0) ticket = atomicAdd(a.counter + u, 1);
-                ticket = __shfl_sync(0xffffffffu, ticket, 0);
-                if (ticket == cpu - 1) {
-                    __threadfence();
-                    const float* g0 = a.part + static_cast<long long>(u) * a.n_split_max * (hs + 2);
-                    float MM = -INFINITY;
-                    for (int i = 0; i < cpu; ++i) MM = fmaxf(MM, __ldcg(g0 + i * (hs + 2)));
-                    float LL = 0.f, z0 = 0.f, z1 = 0.f;
-                    for (int i = 0; i < cpu; ++i) {
-                        const float* gi = g0 + i * (hs + 2);
-                        const float mi = __ldcg(gi);
-                        const float wgt = mi == -INFINITY ? 0.f : exp2f(mi - MM);  // a CTA without keys: 0
-                        LL = fmaf(wgt, __ldcg(gi + 1), LL);
-                        if (d < hs) z0 = fmaf(wgt, __ldcg(gi + 2 + d), z0), z1 = fmaf(wgt, __ldcg(gi + 3 + d), z1);
-                    }
-                    if (d < hs) *reinterpret_cast<__nv_bfloat162*>(yr + d) = __floats2bfloat162_rn(z0 / LL, z1 / LL);
-                    if (lane == 0) a.counter[u] = 0;
-                }
             }
         }
         __syncthreads();
+    }
+}
+
+// c_proj's input rows when attention split its (sequence, head) units over cpu > 1 CTAs: y[b, h hs
+// + d] = sum_i 2^(m_i - M) O_i[d] / sum_i 2^(m_i - M) l_i over the unit's cpu partials (M the
+// largest m_i), rounded to bf16 into the staged rows (stride ldu).
+GPT_DEVINL void stage_y_merge(const StepArgs& a, bf16* us, int ldu) {
+    const int hs = a.hs, cpu = attention_cpu(a), lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    // a warp per (sequence, head) unit: lane l merges dimensions 2l, 2l + 1 over the cpu partials
+    for (int u = warp; u < a.B * a.nh; u += kWarps) {
+        const float* g0 = a.part + static_cast<long long>(u) * a.n_split_max * (hs + 2);
+        const int d = 2 * lane;
+        // every load of the unit's (at most kMaxCtaSplit) partials goes out at once
+        float mi[kMaxCtaSplit], li[kMaxCtaSplit];
+        float2 oi[kMaxCtaSplit];
+#pragma unroll
+        for (int i = 0; i < kMaxCtaSplit; ++i) {
+            const bool in = i < cpu;
+            mi[i] = in ? __ldcg(g0 + i * (hs + 2)) : -INFINITY;
+            li[i] = in ? __ldcg(g0 + i * (hs + 2) + 1) : 0.f;
+            oi[i] = (in && d < hs) ? __ldcg(reinterpret_cast<const float2*>(g0 + i * (hs + 2) + 2 + d)) : make_float2(0.f, 0.f);
+        }
+        float M = mi[0];
+#pragma unroll
+        for (int i = 1; i < kMaxCtaSplit; ++i) M = fmaxf(M, mi[i]);
+        float L = 0.f, z0 = 0.f, z1 = 0.f;
+#pragma unroll
+        for (int i = 0; i < kMaxCtaSplit; ++i) {
+            const float wgt = mi[i] == -INFINITY ? 0.f : exp2f(mi[i] - M);
+            L = fmaf(wgt, li[i], L);
+            z0 = fmaf(wgt, oi[i].x, z0);
+            z1 = fmaf(wgt, oi[i].y, z1);
+        }
+        if (d < hs)
+            *reinterpret_cast<__nv_bfloat162*>(us + (u / a.nh) * ldu + (u % a.nh) * hs + d) =
+                __floats2bfloat162_rn(z0 / L, z1 / L);
     }
 }
 
@@ -805,7 +820,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const __grid_c
         cta_tiles(N, t0, t1);
         if (x == P_PROJ || x == P_FC2) {
             // x += c_proj(y) or c_proj(h): the input rows, and the residual entries the epilogue adds to
-            stage_rows(x == P_PROJ ? a.y : a.h, B, K, us, K + kPad);
+            if (x == P_PROJ && attention_cpu(a) > 1)
+                stage_y_merge(a, us, K + kPad);
+            else
+                stage_rows(x == P_PROJ ? a.y : a.h, B, K, us, K + kPad);
             stage_resid(a, t0 * kTile, (t1 - t0) * kTile, xs);
             if (!(ok = wait_phase(c, j))) break;
         } else {
