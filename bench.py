@@ -324,7 +324,7 @@ KERNEL_OF = {
     "lm_head_ce": "gemm_bf16_tc<256, 3, 0, 0, 0, 1> (+ ce_rows, loss_finalize)",
     "attention": "attention_fwd_tc",
     "layernorm": "layernorm_kernel<bf16>",
-    "embed": "embed_kernel<bf16>",
+    "embed": "embed_rows_kernel<bf16, 6>",
 }
 
 

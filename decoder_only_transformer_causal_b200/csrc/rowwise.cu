@@ -60,6 +60,44 @@ __global__ void embed_kernel(const Tw* __restrict__ wte, const Tw* __restrict__ 
     store4(x + row * C + c, make_float4(a.x + p.x, a.y + p.y, a.z + p.z, a.w + p.w));
 }
 
+// The same with a warp per row: the token id once per row, then every 4-element chunk of the
+// row's wte and wpe slices loaded before any is added (VEC chunks per lane, C <= 128 VEC), so a
+// warp keeps a whole row's loads in flight instead of one chunk per thread.
+template <typename Tw, int VEC>
+__global__ void embed_rows_kernel(const Tw* __restrict__ wte, const Tw* __restrict__ wpe,
+                                  const int64_t* __restrict__ idx, float* __restrict__ x, int rows, int T, int C,
+                                  int V, int32_t* status) {
+    griddep_launch_dependents();
+    griddep_wait();
+    const int lane = threadIdx.x & 31;
+    const int nwarps = static_cast<int>((gridDim.x * blockDim.x) >> 5);
+    const int units = C >> 2;
+    for (int row = static_cast<int>((blockIdx.x * blockDim.x + threadIdx.x) >> 5); row < rows; row += nwarps) {
+        long long tok = idx[row];
+        if (tok < 0 || tok >= V) {
+            if (lane == 0) set_status(status, GPT_ERR_INDEX);
+            tok = 0;
+        }
+        const Tw* er = wte + tok * C;
+        const Tw* pr = wpe + static_cast<long long>(row % T) * C;
+        float4 a[VEC], p[VEC];
+#pragma unroll
+        for (int j = 0; j < VEC; ++j) {
+            const int u = lane + 32 * j;
+            if (u < units) {
+                a[j] = load4(er + 4 * u);
+                p[j] = load4(pr + 4 * u);
+            }
+        }
+        float* xr = x + static_cast<long long>(row) * C;
+#pragma unroll
+        for (int j = 0; j < VEC; ++j) {
+            const int u = lane + 32 * j;
+            if (u < units) store4(xr + 4 * u, make_float4(a[j].x + p[j].x, a[j].y + p[j].y, a[j].z + p[j].z, a[j].w + p[j].w));
+        }
+    }
+}
+
 // LayerNorm over rows of fp32 x, population variance, eps 1e-5 ("nanoGPT 全局流程图",
 // §2.5 (A)).  The row stays in registers: mean, then sum of squared deviations.
 constexpr int kLnMaxVec = 16;  // float4 per lane -> C <= 2048
@@ -215,10 +253,31 @@ __global__ void __launch_bounds__(kFinThreads)
 
 }  // namespace
 
+namespace {
+template <typename Tw, int VEC = 1>
+int launch_embed_rows(const Tw* wte, const Tw* wpe, const int64_t* idx, float* x, int rows, int T, int C, int V,
+                      int32_t* status, cudaStream_t s) {
+    if constexpr (VEC < 16) {
+        if (C > 128 * VEC) return launch_embed_rows<Tw, VEC + 1>(wte, wpe, idx, x, rows, T, C, V, status, s);
+    }
+    const int warps = rows < 148 * 64 ? rows : 148 * 64;  // enough warps to keep every SM's loads in flight
+    return launch_overlapped(embed_rows_kernel<Tw, VEC>, dim3((warps + 7) / 8), dim3(256), 0, s, wte, wpe, idx, x,
+                             rows, T, C, V, status);
+}
+}  // namespace
+
 int launch_embed(const void* wte, const void* wpe, const int64_t* idx, float* x, int B, int T, int C,
                  int V, int dtype, int32_t* status, cudaStream_t s) {
     const long long total4 = static_cast<long long>(B) * T * (C / 4);
     if (total4 == 0) return GPT_OK;
+    if (C % 4 == 0 && C <= 2048 && static_cast<long long>(B) * T < (1LL << 31)) {
+        const int rows = B * T;
+        return dtype == GPT_DTYPE_BF16
+                   ? launch_embed_rows(static_cast<const bf16*>(wte), static_cast<const bf16*>(wpe), idx, x, rows, T,
+                                       C, V, status, s)
+                   : launch_embed_rows(static_cast<const float*>(wte), static_cast<const float*>(wpe), idx, x, rows, T,
+                                       C, V, status, s);
+    }
     const int threads = 256;
     const unsigned blocks = static_cast<unsigned>((total4 + threads - 1) / threads);
     if (dtype == GPT_DTYPE_BF16)
