@@ -145,18 +145,21 @@ __global__ void __launch_bounds__(kBwdWarps * 32)
 // LayerNorm backward, one warp per row: y = xhat w + b, xhat = (x - mean) * rstd;
 // dx (+)= rstd (dxhat - mean(dxhat) - xhat mean(dxhat xhat)), dxhat = dy w.  Each CTA also
 // leaves its rows' sums of dy * xhat and dy per column in part[blockIdx.x] (the weight and bias
-// gradients after the column reduction).
+// gradients after the column reduction) and, with nsum 3, the column sums of dx as written: the
+// residual stream's gradient, which is also the bias gradient of the projection whose output
+// was added to the stream here (attn c_proj before ln_2, the previous Block's mlp c_proj before
+// ln_1 or ln_f).
 template <typename Tw>
 __global__ void __launch_bounds__(kBwdWarps * 32)
     layernorm_backward_kernel(const float* __restrict__ dy, const float* __restrict__ x, const Tw* __restrict__ w,
                               float* __restrict__ dx, int accumulate, float* __restrict__ part, int rows, int C,
-                              bf16* __restrict__ dx16) {
+                              bf16* __restrict__ dx16, int nsum) {
     griddep_launch_dependents();
     griddep_wait();
-    extern __shared__ float sm[];  // [kBwdWarps][2][C] per-warp column sums
+    extern __shared__ float sm[];  // [kBwdWarps][nsum][C] per-warp column sums
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    float* my = sm + static_cast<size_t>(warp) * 2 * C;
-    for (int c = lane; c < 2 * C; c += 32) my[c] = 0.f;
+    float* my = sm + static_cast<size_t>(warp) * nsum * C;
+    for (int c = lane; c < nsum * C; c += 32) my[c] = 0.f;
     __syncwarp();
     const int r = blockIdx.x * kBwdWarps + warp;
     if (r < rows) {
@@ -189,14 +192,15 @@ __global__ void __launch_bounds__(kBwdWarps * 32)
             const float o = accumulate ? __ldcg(dxr + c) + v : v;
             dxr[c] = o;
             if (dx16) dx16[static_cast<long long>(r) * C + c] = __float2bfloat16_rn(o);
+            if (nsum == 3) my[2 * C + c] += o;
         }
     }
     __syncthreads();
     // this CTA's column sums, warps added in order
-    for (int c = threadIdx.x; c < 2 * C; c += kBwdWarps * 32) {
+    for (int c = threadIdx.x; c < nsum * C; c += kBwdWarps * 32) {
         float v = 0.f;
-        for (int wp = 0; wp < kBwdWarps; ++wp) v += sm[static_cast<size_t>(wp) * 2 * C + c];
-        part[static_cast<long long>(blockIdx.x) * 2 * C + c] = v;
+        for (int wp = 0; wp < kBwdWarps; ++wp) v += sm[static_cast<size_t>(wp) * nsum * C + c];
+        part[static_cast<long long>(blockIdx.x) * nsum * C + c] = v;
     }
 }
 
@@ -239,10 +243,10 @@ template <typename Tw, int VEC>
 __global__ void __launch_bounds__(kBwdWarps * 32)
     layernorm_backward_reg_kernel(const float* __restrict__ dy, const float* __restrict__ x, const Tw* __restrict__ w,
                                   float* __restrict__ dx, int accumulate, float* __restrict__ part, int rows, int C,
-                                  bf16* __restrict__ dx16, int rows_per_warp) {
+                                  bf16* __restrict__ dx16, int rows_per_warp, int nsum) {
     griddep_launch_dependents();
     griddep_wait();
-    extern __shared__ float sm[];  // [kBwdWarps][2][C] per-warp column sums
+    extern __shared__ float sm[];  // [kBwdWarps][nsum][C] per-warp column sums
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     float4 wv[VEC], dwa[VEC], dba[VEC];
 #pragma unroll
@@ -254,11 +258,10 @@ __global__ void __launch_bounds__(kBwdWarps * 32)
         dba[j] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
     constexpr bool kPipe = VEC <= 6;
-    float* my = sm + static_cast<size_t>(warp) * 2 * C;
-    if constexpr (!kPipe) {
-        for (int c = lane; c < 2 * C; c += 32) my[c] = 0.f;
-        __syncwarp();
-    }
+    float* my = sm + static_cast<size_t>(warp) * nsum * C;
+    // dw / db sums: registers (kPipe) or shared memory; the dx sums (nsum 3) always shared memory
+    for (int c = kPipe ? 2 * C + lane : lane; c < nsum * C; c += 32) my[c] = 0.f;
+    __syncwarp();
     const int r0 = (blockIdx.x * kBwdWarps + warp) * rows_per_warp;
     const int r1 = min(rows, r0 + rows_per_warp);
     LnRow<VEC> cur, nxt;
@@ -326,6 +329,11 @@ __global__ void __launch_bounds__(kBwdWarps * 32)
                 if (dx16)
                     *reinterpret_cast<uint2*>(dx16 + static_cast<long long>(r) * C + c) =
                         make_uint2(pack_bf16x2(o.x, o.y), pack_bf16x2(o.z, o.w));
+                if (nsum == 3) {
+                    float4* ds = reinterpret_cast<float4*>(my + 2 * C + c);
+                    const float4 t = *ds;
+                    *ds = make_float4(t.x + o.x, t.y + o.y, t.z + o.z, t.w + o.w);
+                }
             }
         }
         if constexpr (kPipe) cur = nxt;
@@ -341,10 +349,37 @@ __global__ void __launch_bounds__(kBwdWarps * 32)
         }
     }
     __syncthreads();
-    for (int c = threadIdx.x; c < 2 * C; c += kBwdWarps * 32) {
+    for (int c = threadIdx.x; c < nsum * C; c += kBwdWarps * 32) {
         float v = 0.f;
-        for (int wp = 0; wp < kBwdWarps; ++wp) v += sm[static_cast<size_t>(wp) * 2 * C + c];
-        part[static_cast<long long>(blockIdx.x) * 2 * C + c] = v;
+        for (int wp = 0; wp < kBwdWarps; ++wp) v += sm[static_cast<size_t>(wp) * nsum * C + c];
+        part[static_cast<long long>(blockIdx.x) * nsum * C + c] = v;
+    }
+}
+
+// The second stage of the LayerNorm backward's column sums: column c of the [n_part, n_out * C]
+// partials goes to out_{c / C}[c % C] (+)= the sum over parts in order; a null out is skipped.
+__global__ void __launch_bounds__(256)
+    colsum_parts3_kernel(const float* __restrict__ part, int n_part, int C, int n_out, float* out0, float* out1,
+                         float* out2, int accumulate) {
+    griddep_launch_dependents();
+    griddep_wait();
+    __shared__ float red[8][33];
+    const int c = blockIdx.x * 32 + threadIdx.x;
+    const long long ld = static_cast<long long>(n_out) * C;
+    float v = 0.f;
+    if (c < ld) {
+#pragma unroll 4
+        for (int i = threadIdx.y; i < n_part; i += 8) v += __ldcg(part + i * ld + c);
+    }
+    red[threadIdx.y][threadIdx.x] = v;
+    __syncthreads();
+    if (threadIdx.y == 0 && c < ld) {
+        float t = red[0][threadIdx.x];
+#pragma unroll
+        for (int k = 1; k < 8; ++k) t += red[k][threadIdx.x];
+        const int which = c / C, cc = c - which * C;
+        float* out = which == 0 ? out0 : which == 1 ? out1 : out2;
+        if (out) out[cc] = accumulate ? __ldcg(out + cc) + t : t;
     }
 }
 
@@ -539,7 +574,7 @@ int launch_ce_backward(const void* logits, int dtype, const int64_t* targets, co
                              sum_count, static_cast<float*>(dlogits), rows, V, scale, status, row_lse);
 }
 
-int layernorm_backward_parts(int rows, int C) {
+int layernorm_backward_parts(int rows, int C) {  // partials of 2C (3C with dsum) floats each
     const int per = (C <= 2048 && C % 4 == 0) ? kBwdWarps * ln_rows_per_warp(rows) : kBwdWarps;
     return (rows + per - 1) / per;
 }
@@ -547,52 +582,49 @@ int layernorm_backward_parts(int rows, int C) {
 namespace {
 template <typename Tw, int VEC = 1>
 int launch_ln_bwd_reg(const float* dy, const float* x, const void* w, float* dx, bf16* dx16, int accumulate, float* part, int rows,
-                      int C, size_t smem, cudaStream_t s) {
+                      int C, int nsum, size_t smem, cudaStream_t s) {
     if constexpr (VEC < 16) {
-        if (C > 128 * VEC) return launch_ln_bwd_reg<Tw, VEC + 1>(dy, x, w, dx, dx16, accumulate, part, rows, C, smem, s);
+        if (C > 128 * VEC)
+            return launch_ln_bwd_reg<Tw, VEC + 1>(dy, x, w, dx, dx16, accumulate, part, rows, C, nsum, smem, s);
     }
     static size_t opted[kMaxDevices] = {};
     const int rc = opt_in_smem(reinterpret_cast<const void*>(layernorm_backward_reg_kernel<Tw, VEC>), smem, opted);
     if (rc) return rc;
     return launch_overlapped(layernorm_backward_reg_kernel<Tw, VEC>, dim3(layernorm_backward_parts(rows, C)),
                              dim3(kBwdWarps * 32), smem, s, dy, x, static_cast<const Tw*>(w), dx, accumulate, part,
-                             rows, C, dx16, ln_rows_per_warp(rows));
+                             rows, C, dx16, ln_rows_per_warp(rows), nsum);
 }
 }  // namespace
 
 int launch_layernorm_backward(const float* dy, const float* x, const void* w, int dtype, float* dx, int accumulate,
                               float* dw, float* db, int accumulate_wb, float* part, int rows, int C, cudaStream_t s,
-                              bf16* dx16) {
+                              bf16* dx16, float* dsum) {
     const int n_part = layernorm_backward_parts(rows, C);
-    const size_t smem = static_cast<size_t>(kBwdWarps) * 2 * C * sizeof(float);
+    const int nsum = dsum ? 3 : 2;
+    const size_t smem = static_cast<size_t>(kBwdWarps) * nsum * C * sizeof(float);
     int rc;
     if (C <= 2048 && C % 4 == 0) {
-        rc = dtype == GPT_DTYPE_BF16 ? launch_ln_bwd_reg<bf16>(dy, x, w, dx, dx16, accumulate, part, rows, C, smem, s)
-                                     : launch_ln_bwd_reg<float>(dy, x, w, dx, dx16, accumulate, part, rows, C, smem, s);
+        rc = dtype == GPT_DTYPE_BF16
+                 ? launch_ln_bwd_reg<bf16>(dy, x, w, dx, dx16, accumulate, part, rows, C, nsum, smem, s)
+                 : launch_ln_bwd_reg<float>(dy, x, w, dx, dx16, accumulate, part, rows, C, nsum, smem, s);
     } else if (dtype == GPT_DTYPE_BF16) {
         static size_t opted[kMaxDevices] = {};
         rc = opt_in_smem(reinterpret_cast<const void*>(layernorm_backward_kernel<bf16>), smem, opted);
         if (!rc)
             rc = launch_overlapped(layernorm_backward_kernel<bf16>, dim3(n_part), dim3(kBwdWarps * 32), smem, s, dy,
-                                   x, static_cast<const bf16*>(w), dx, accumulate, part, rows, C, dx16);
+                                   x, static_cast<const bf16*>(w), dx, accumulate, part, rows, C, dx16, nsum);
     } else {
         static size_t opted[kMaxDevices] = {};
         rc = opt_in_smem(reinterpret_cast<const void*>(layernorm_backward_kernel<float>), smem, opted);
         if (!rc)
             rc = launch_overlapped(layernorm_backward_kernel<float>, dim3(n_part), dim3(kBwdWarps * 32), smem, s, dy,
-                                   x, static_cast<const float*>(w), dx, accumulate, part, rows, C, dx16);
+                                   x, static_cast<const float*>(w), dx, accumulate, part, rows, C, dx16, nsum);
     }
     if (rc) return rc;
-    if (db == dw + C)  // adjacent gradients (the packed layout when C * 4 is a multiple of 256): one pass
-        return launch_overlapped(colsum_parts_kernel, dim3((2 * C + 31) / 32), dim3(32, 8), 0, s,
-                                 static_cast<const float*>(part), 2LL * C, n_part, 2 * C, dw, accumulate_wb);
-    const dim3 gp((C + 31) / 32), bp(32, 8);
-    rc = launch_overlapped(colsum_parts_kernel, gp, bp, 0, s, static_cast<const float*>(part), 2LL * C, n_part, C, dw,
-                           accumulate_wb);
-    if (rc) return rc;
-    if (!db) return GPT_OK;
-    return launch_overlapped(colsum_parts_kernel, gp, bp, 0, s, static_cast<const float*>(part + C), 2LL * C, n_part, C,
-                             db, accumulate_wb);
+    // dsum always accumulates (bias gradients add into the caller's gradient buffer)
+    if (dsum && !accumulate_wb) return GPT_ERR_UNSUPPORTED;
+    return launch_overlapped(colsum_parts3_kernel, dim3((nsum * C + 31) / 32), dim3(32, 8), 0, s,
+                             static_cast<const float*>(part), n_part, C, nsum, dw, db, dsum, accumulate_wb);
 }
 
 int colsum_parts(int rows) { return (rows + kColRows - 1) / kColRows; }

@@ -1137,7 +1137,7 @@ BwdPlan plan_bwd(const gpt_config_t* c, long long B, long long T) {
     P.dqkv = off; off += a256(N * 3 * C * es);
     P.dy = off; off += a256(N * C * es);
     P.D = off; off += a256(attn_bwd_scratch_bytes(B, c->n_head, T));
-    const size_t lnp = static_cast<size_t>(layernorm_backward_parts(static_cast<int>(N), static_cast<int>(C))) * 2 * C;
+    const size_t lnp = static_cast<size_t>(layernorm_backward_parts(static_cast<int>(N), static_cast<int>(C))) * 3 * C;
     const size_t csp = static_cast<size_t>(colsum_parts(static_cast<int>(N))) * 4 * C;
     P.parts = off; off += a256(std::max(lnp, csp) * 4);
     P.sort = off; off += a256(N * 8);
@@ -1417,8 +1417,13 @@ GPT_API int gpt_backward(const gpt_config_t* cfg, const void* weights, const int
     GPT_TRY(launch_ce_backward(ab + A.logits, dt, targets, reinterpret_cast<const double*>(ab + A.sum_count), dz, N, V,
                                status, s, loss_scale, bf ? reinterpret_cast<const float*>(ab + A.row_lse) : nullptr));
     GPT_TRY(linear_bwd(dz, V, ab + A.u_f, C, W.wte(), V, C, d1, F32_OUT, nullptr, G(0), dzT));
+    // The residual gradient each LayerNorm backward writes is also the bias gradient of the
+    // projection that added into the stream there: the last Block's mlp c_proj at ln_f, attn c_proj
+    // at ln_2, the previous Block's mlp c_proj at ln_1.  The LayerNorm backward sums it as it goes.
+    const int Lm1 = cfg->n_layer - 1;
     GPT_TRY(launch_layernorm_backward(d1, reinterpret_cast<const float*>(ab + A.x_f), W.lnf_w(), dt, dx, 0, G(count - 2),
-                                      cfg->bias ? G(count - 1) : nullptr, 1, parts, N, C, s, dx16));
+                                      cfg->bias ? G(count - 1) : nullptr, 1, parts, N, C, s, dx16,
+                                      cfg->bias ? GL(Lm1, W_FC2_B) : nullptr));
     // Event i marks the end of bucket i (gpt_grad_buckets): a caller may start reducing that range
     // of grads on another stream while the rest of the backward runs.
     auto mark = [&](int i) -> int {
@@ -1429,7 +1434,7 @@ GPT_API int gpt_backward(const gpt_config_t* cfg, const void* weights, const int
         const uint8_t* L = ab + A.layer * l;
         // mlp c_proj, then GELU: dpre = (dx W_fc2) * gelu'(pre) (bf16: one fused product reading the
         // derivative the forward stored; fp32: dh into d1, then the GELU backward from the
-        // pre-activation); dW_fc2 += dx^T h; db_fc2 += sum dx
+        // pre-activation); dW_fc2 += dx^T h (db_fc2 += sum dx came with the LayerNorm backward above)
         if (bf) {
             GPT_TRY(linear_bwd(gx, C, L + A.h, 4LL * C, W.layer(l, W_FC2_W), C, 4 * C, dpre, GEMM_BWD_DGELU_BF16,
                                L + A.pre, GL(l, W_FC2_W), gT));
@@ -1439,18 +1444,17 @@ GPT_API int gpt_backward(const gpt_config_t* cfg, const void* weights, const int
             GPT_TRY(launch_gelu_backward(d1, L + A.pre, dt, dpre, static_cast<long long>(nc) * 4,
                                          cfg->gelu == GPT_GELU_TANH, s));
         }
-        if (cfg->bias) GPT_TRY(launch_colsum(dx, F32, N, C, GL(l, W_FC2_B), 1, parts, s));
         // c_fc: du2 = dpre W_fc (into d1 [N, C]); dW_fc += dpre^T u2; db_fc += sum dpre
         GPT_TRY(linear_bwd(dpre, 4LL * C, L + A.u2, C, W.layer(l, W_FC_W), 4 * C, C, d1, F32_OUT, nullptr,
                            GL(l, W_FC_W), gT));
         if (cfg->bias) GPT_TRY(launch_colsum(dpre, dt, N, 4 * C, GL(l, W_FC_B), 1, parts, s));
         GPT_TRY(launch_layernorm_backward(d1, reinterpret_cast<const float*>(L + A.x_mid), W.layer(l, W_LN2_W), dt, dx, 1,
                                           GL(l, W_LN2_W), cfg->bias ? GL(l, W_LN2_B) : nullptr, 1, parts, N, C, s,
-                                          dx16));
-        // attn c_proj: dy = dx W_proj (straight into the config dtype); dW_proj += dx^T y; db_proj += sum dx
+                                          dx16, cfg->bias ? GL(l, W_PROJ_B) : nullptr));
+        // attn c_proj: dy = dx W_proj (straight into the config dtype); dW_proj += dx^T y (db_proj += sum dx
+        // came with ln_2's backward)
         GPT_TRY(linear_bwd(gx, C, L + A.y, C, W.layer(l, W_PROJ_W), C, C, dy, bf ? GEMM_BWD_STORE_BF16 : F32_OUT,
                            nullptr, GL(l, W_PROJ_W), gT));
-        if (cfg->bias) GPT_TRY(launch_colsum(dx, F32, N, C, GL(l, W_PROJ_B), 1, parts, s));
         // attention backward into dqkv (the qkv layout)
         const float* lse = reinterpret_cast<const float*>(L + A.lse);
         const long long qsb = 3LL * C * T, ysb = static_cast<long long>(C) * T;
@@ -1475,7 +1479,7 @@ GPT_API int gpt_backward(const gpt_config_t* cfg, const void* weights, const int
         if (cfg->bias) GPT_TRY(launch_colsum(dqkv, dt, N, 3 * C, GL(l, W_ATTN_B), 1, parts, s));
         GPT_TRY(launch_layernorm_backward(d1, reinterpret_cast<const float*>(L + A.x_in), W.layer(l, W_LN1_W), dt, dx, 1,
                                           GL(l, W_LN1_W), cfg->bias ? GL(l, W_LN1_B) : nullptr, 1, parts, N, C, s,
-                                          dx16));
+                                          dx16, cfg->bias && l > 0 ? GL(l - 1, W_FC2_B) : nullptr));
         GPT_TRY(mark(cfg->n_layer - 1 - l));  // every gradient of layer l (and, for the last layer, ln_f) is final
     }
     GPT_TRY(launch_embed_backward(idx, dx, B, T, C, V, G(0), G(1), reinterpret_cast<unsigned long long*>(ws + P.sort),

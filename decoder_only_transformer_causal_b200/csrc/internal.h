@@ -222,11 +222,13 @@ int launch_adamw(const OptTable& tab, int dtype, float* params, const float* gra
 int launch_ce_backward(const void* logits, int dtype, const int64_t* targets, const double* sum_count, void* dlogits,
                        int rows, int V, int32_t* status, cudaStream_t s, float scale = 1.f,
                        const float* row_lse = nullptr);
-int layernorm_backward_parts(int rows, int C);  // part: [parts, 2C] floats
+int layernorm_backward_parts(int rows, int C);  // part: [parts, 2C] floats ([parts, 3C] with dsum)
 // dx16 (optional): a bf16 copy of the dx rows as written (the next products' operand).
+// dsum (optional, needs accumulate_wb): dsum[c] += sum over rows of dx[r, c] as written, the bias
+// gradient of the projection that added into the residual stream at this LayerNorm's input.
 int launch_layernorm_backward(const float* dy, const float* x, const void* w, int dtype, float* dx, int accumulate,
                               float* dw, float* db, int accumulate_wb, float* part, int rows, int C, cudaStream_t s,
-                              bf16* dx16 = nullptr);
+                              bf16* dx16 = nullptr, float* dsum = nullptr);
 int colsum_parts(int rows);              // part: [parts, C] floats
 int launch_colsum(const void* y, int dtype, int rows, int C, float* out, int accumulate, float* part,
                   cudaStream_t s);

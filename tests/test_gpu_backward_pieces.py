@@ -66,9 +66,13 @@ def test_layernorm_backward(rows, C, wdtype):
     assert torch.equal(dx, dx2) and torch.equal(dw, dw2)
 
 
-@pytest.mark.parametrize("rows,C,dtype", [(12288, 3072, torch.bfloat16), (300, 768, torch.float32),
-                                          (129, 65, torch.float32)])
+@pytest.mark.parametrize("rows,C,dtype", [(12288, 3072, torch.bfloat16), (12288, 768, torch.float32),
+                                          (300, 768, torch.float32), (129, 65, torch.float32),
+                                          (77, 65, torch.bfloat16), (1, 100, torch.bfloat16),
+                                          (40, 8200, torch.bfloat16), (33, 4100, torch.float32)])
 def test_bias_grad(rows, C, dtype):
+    """Vector loads or, where C is not a multiple of the vector width, element loads; widths past
+    one CTA's column span; one row; a repeat must give the identical sums."""
     from decoder_only_transformer_causal_b200 import native
     dy = (torch.randn(rows, C, generator=torch.Generator().manual_seed(7)) * 0.01).to(dtype)
     start = torch.full((C,), 0.25, device="cuda")
