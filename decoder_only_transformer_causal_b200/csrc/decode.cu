@@ -619,8 +619,33 @@ __global__ void __launch_bounds__(kSampleThreads)
     if (tid == 0) s_ncand = 0;
     __syncthreads();
     float mx = -INFINITY;
-    // eight loads in flight per thread (the row is ~50 loads per thread for V 50304)
-    for (int i0 = tid; i0 < V; i0 += 8 * kSampleThreads) {
+    const bool vec = (V & 3) == 0 && (ld_logits & 3) == 0 && (reinterpret_cast<uintptr_t>(logits) & 15) == 0;
+    // 16-byte loads, eight in flight per thread (two rounds for V 50304)
+    const int V4 = vec ? V >> 2 : 0;
+    for (int i0 = tid; i0 < V4; i0 += 8 * kSampleThreads) {
+        float4 v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int i = i0 + j * kSampleThreads;
+            v[j] = i < V4 ? __ldcg(reinterpret_cast<const float4*>(lg) + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int i = i0 + j * kSampleThreads;
+            if (i < V4) {
+                reinterpret_cast<float4*>(zs)[i] = v[j];
+                mx = fmaxf(mx, fmaxf(fmaxf(v[j].x, v[j].y), fmaxf(v[j].z, v[j].w)));
+                if (filter) {
+                    atomicAdd(&hist[fkey(v[j].x) >> 21], 1u);
+                    atomicAdd(&hist[fkey(v[j].y) >> 21], 1u);
+                    atomicAdd(&hist[fkey(v[j].z) >> 21], 1u);
+                    atomicAdd(&hist[fkey(v[j].w) >> 21], 1u);
+                }
+            }
+        }
+    }
+    // element loads otherwise, eight in flight per thread
+    for (int i0 = vec ? V : tid; i0 < V; i0 += 8 * kSampleThreads) {
         float v[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
@@ -716,6 +741,8 @@ __global__ void __launch_bounds__(kSampleThreads)
             const float li = zs[i];
             if (fkey(li) >= thr_key) p = static_cast<double>(expf(li / temperature - m));
         }
+        const uint32_t nz = __ballot_sync(0xffffffffu, p > 0.0);
+        if (!nz) continue;  // nothing kept in these 32 entries: the running sum stays
         double c = p;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -728,8 +755,7 @@ __global__ void __launch_bounds__(kSampleThreads)
             if (lane == __ffs(hit) - 1) out[b * ld_out] = i;
             return;
         }
-        const uint32_t nz = __ballot_sync(0xffffffffu, p > 0.0);
-        if (nz) last = i0 + 31 - __clz(nz);
+        last = i0 + 31 - __clz(nz);
         cum = __shfl_sync(0xffffffffu, c, 31);
     }
     // rounding left the target past the segment's running sum: its last entry with p > 0
