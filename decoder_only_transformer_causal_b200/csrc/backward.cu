@@ -356,27 +356,29 @@ __global__ void __launch_bounds__(kBwdWarps * 32)
     }
 }
 
-// The second stage of the LayerNorm backward's column sums: column c of the [n_part, n_out * C]
-// partials goes to out_{c / C}[c % C] (+)= the sum over parts in order; a null out is skipped.
-__global__ void __launch_bounds__(256)
+// The second stage of a column reduction with up to three destinations: column c of the
+// [n_part, n_out * C] partials goes to out_{c / C}[c % C] (+)= the sum over parts in order; a
+// null out is skipped.  Block (32, 32): slice y adds parts y, y + 32, ... (eight loads in flight),
+// then the 32 slice sums are added in order.
+__global__ void __launch_bounds__(1024)
     colsum_parts3_kernel(const float* __restrict__ part, int n_part, int C, int n_out, float* out0, float* out1,
                          float* out2, int accumulate) {
     griddep_launch_dependents();
     griddep_wait();
-    __shared__ float red[8][33];
+    __shared__ float red[32][33];
     const int c = blockIdx.x * 32 + threadIdx.x;
     const long long ld = static_cast<long long>(n_out) * C;
     float v = 0.f;
     if (c < ld) {
-#pragma unroll 4
-        for (int i = threadIdx.y; i < n_part; i += 8) v += __ldcg(part + i * ld + c);
+#pragma unroll 8
+        for (int i = threadIdx.y; i < n_part; i += 32) v += __ldcg(part + i * ld + c);
     }
     red[threadIdx.y][threadIdx.x] = v;
     __syncthreads();
     if (threadIdx.y == 0 && c < ld) {
         float t = red[0][threadIdx.x];
 #pragma unroll
-        for (int k = 1; k < 8; ++k) t += red[k][threadIdx.x];
+        for (int k = 1; k < 32; ++k) t += red[k][threadIdx.x];
         const int which = c / C, cc = c - which * C;
         float* out = which == 0 ? out0 : which == 1 ? out1 : out2;
         if (out) out[cc] = accumulate ? __ldcg(out + cc) + t : t;
@@ -623,8 +625,14 @@ int launch_layernorm_backward(const float* dy, const float* x, const void* w, in
     if (rc) return rc;
     // dsum always accumulates (bias gradients add into the caller's gradient buffer)
     if (dsum && !accumulate_wb) return GPT_ERR_UNSUPPORTED;
-    return launch_overlapped(colsum_parts3_kernel, dim3((nsum * C + 31) / 32), dim3(32, 8), 0, s,
+    return launch_overlapped(colsum_parts3_kernel, dim3((nsum * C + 31) / 32), dim3(32, 32), 0, s,
                              static_cast<const float*>(part), n_part, C, nsum, dw, db, dsum, accumulate_wb);
+}
+
+int launch_colsum_bands(const float* part, int n_part, int C, float* out, int accumulate, cudaStream_t s) {
+    if (n_part < 1 || C < 1) return GPT_OK;
+    return launch_overlapped(colsum_parts3_kernel, dim3((C + 31) / 32), dim3(32, 32), 0, s, part, n_part, C, 1, out,
+                             static_cast<float*>(nullptr), static_cast<float*>(nullptr), accumulate);
 }
 
 int colsum_parts(int rows) { return (rows + kColRows - 1) / kColRows; }

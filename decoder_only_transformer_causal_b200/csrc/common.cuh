@@ -469,6 +469,25 @@ GPT_DEVINL uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// Column sums of a warp's 32 x 32 block (lane = row, v[c] = column c): lane l returns the sum of
+// v[l] over the 32 lanes.  A transposing butterfly: at distance k each lane keeps the half of its
+// live columns on its own side of bit k and adds its partner's copy of that half (31 exchanges
+// and adds per lane, in an order fixed by the lane index).  v is consumed.
+GPT_DEVINL float warp_colsum32(float (&v)[32]) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int k = 16; k >= 1; k >>= 1) {
+        const bool up = (lane & k) != 0;
+#pragma unroll
+        for (int j = 0; j < k; ++j) {
+            const float send = up ? v[j] : v[j + k];
+            const float keep = up ? v[j + k] : v[j];
+            v[j] = keep + __shfl_xor_sync(0xffffffffu, send, k);
+        }
+    }
+    return v[0];
+}
+
 // Programmatic dependent launch.  A kernel launched with programmatic stream serialisation may
 // start before its predecessor in the stream has finished: it must call griddep_wait() before
 // it reads or writes memory the predecessor touches (the wait returns once the predecessor has

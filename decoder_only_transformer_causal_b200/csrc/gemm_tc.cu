@@ -190,7 +190,7 @@ int launch_gemm_bf16(const bf16* A, long long lda, const bf16* W, long long ldw,
 
 int launch_gemm_bf16_bwd(const bf16* A, long long lda, bool a_mn, const bf16* W, long long ldw, bool b_mn, void* out,
                          long long ldo, int M, int N, int K, int mode, const bf16* aux, long long ld_aux, int gelu,
-                         int32_t* status, cudaStream_t s, float* split_ws) {
+                         int32_t* status, cudaStream_t s, float* split_ws, float* colsum) {
     if (M == 0 || N == 0) return GPT_OK;
     if (!b_mn || (a_mn && mode != GEMM_BWD_ACC_F32)) return GPT_ERR_UNSUPPORTED;
     CUtensorMap ta, tb, tc;
@@ -246,6 +246,8 @@ int launch_gemm_bf16_bwd(const bf16* A, long long lda, bool a_mn, const bf16* W,
         if ((reinterpret_cast<uintptr_t>(aux) & 15) || (ld_aux % 8)) return GPT_ERR_BAD_ALIGN;
         p.aux = aux;
         p.ld_aux = ld_aux;
+        p.colsum = colsum;
+        p.ld_colsum = N;
     }
     switch (mode) {
         case GEMM_BWD_ACC_F32:

@@ -62,6 +62,10 @@ struct Params {
     int kb_per_split;
     const bf16* aux;  // EPI_DGELU: [M, ld_aux]
     long long ld_aux;
+    // EPI_DGELU (optional): the output's column sums per 32-row band, [ceil(M / 32), ld_colsum]
+    // (the first stage of the bias gradient of the layer whose input gradient this is)
+    float* colsum;
+    long long ld_colsum;
 };
 
 // PAIR: a cluster of two CTAs computes one 256 x BN tile with the 2-SM MMA; each CTA stages its
@@ -613,6 +617,15 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)  // 10 warps: <= 168 regi
                                 tma_store_2d(&tmC, stg, n, row0 + pass * p.M);
                                 bulk_commit();
                             }
+                        }
+                        if (EPI == EPI_DGELU && p.colsum) {
+                            // this band's column sums of the 32 columns (rows past M add zero)
+                            if (!row_ok) {
+#pragma unroll
+                                for (int j = 0; j < 32; ++j) v[j] = 0.f;
+                            }
+                            const float cs = warp_colsum32(v);
+                            if (n + lane < p.N) p.colsum[static_cast<long long>(row0 >> 5) * p.ld_colsum + n + lane] = cs;
                         }
                     }
                 }

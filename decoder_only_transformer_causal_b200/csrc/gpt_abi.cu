@@ -1139,7 +1139,8 @@ BwdPlan plan_bwd(const gpt_config_t* c, long long B, long long T) {
     P.D = off; off += a256(attn_bwd_scratch_bytes(B, c->n_head, T));
     const size_t lnp = static_cast<size_t>(layernorm_backward_parts(static_cast<int>(N), static_cast<int>(C))) * 3 * C;
     const size_t csp = static_cast<size_t>(colsum_parts(static_cast<int>(N))) * 4 * C;
-    P.parts = off; off += a256(std::max(lnp, csp) * 4);
+    const size_t bands = (N + 31) / 32 * 4 * C;  // db_fc's per-band sums from the DGELU product
+    P.parts = off; off += a256(std::max({lnp, csp, bands}) * 4);
     P.sort = off; off += a256(N * 8);
     // split-K partial products of the weight-gradient GEMMs (bf16)
     size_t sk = 0;
@@ -1386,11 +1387,13 @@ GPT_API int gpt_backward(const gpt_config_t* cfg, const void* weights, const int
     // the GEMM the stored dY, X and W as MN-major operands where the product needs their transposes;
     // fp32 (GEMM_BWD_STORE_F32 only) forms the transposes in scratch first (yT: room for dY^T).
     auto linear_bwd = [&](const void* dYp, long long ldy, const void* Xp, long long ldx, const void* Wp, int n_out,
-                          int n_in, void* dIn, int mode, const void* aux, float* dW, void* yT) -> int {
+                          int n_in, void* dIn, int mode, const void* aux, float* dW, void* yT,
+                          float* colsum = nullptr) -> int {
         if (bf) {
             const bf16* y = static_cast<const bf16*>(dYp);
             GPT_TRY(launch_gemm_bf16_bwd(y, ldy, false, static_cast<const bf16*>(Wp), n_in, true, dIn, n_in, N, n_in,
-                                         n_out, mode, static_cast<const bf16*>(aux), n_in, cfg->gelu, status, s));
+                                         n_out, mode, static_cast<const bf16*>(aux), n_in, cfg->gelu, status, s,
+                                         nullptr, colsum));
             return launch_gemm_bf16_bwd(y, ldy, true, static_cast<const bf16*>(Xp), ldx, true, dW, n_in, n_out, n_in, N,
                                         GEMM_BWD_ACC_F32, nullptr, 0, 0, status, s,
                                         reinterpret_cast<float*>(ws + P.splitk));
@@ -1436,18 +1439,20 @@ GPT_API int gpt_backward(const gpt_config_t* cfg, const void* weights, const int
         // derivative the forward stored; fp32: dh into d1, then the GELU backward from the
         // pre-activation); dW_fc2 += dx^T h (db_fc2 += sum dx came with the LayerNorm backward above)
         if (bf) {
+            // the product's epilogue also leaves dpre's column sums per 32-row band (db_fc)
             GPT_TRY(linear_bwd(gx, C, L + A.h, 4LL * C, W.layer(l, W_FC2_W), C, 4 * C, dpre, GEMM_BWD_DGELU_BF16,
-                               L + A.pre, GL(l, W_FC2_W), gT));
+                               L + A.pre, GL(l, W_FC2_W), gT, cfg->bias ? parts : nullptr));
+            if (cfg->bias) GPT_TRY(launch_colsum_bands(parts, (N + 31) / 32, 4 * C, GL(l, W_FC_B), 1, s));
         } else {
             GPT_TRY(linear_bwd(gx, C, L + A.h, 4LL * C, W.layer(l, W_FC2_W), C, 4 * C, d1, F32_OUT, nullptr,
                                GL(l, W_FC2_W), gT));
             GPT_TRY(launch_gelu_backward(d1, L + A.pre, dt, dpre, static_cast<long long>(nc) * 4,
                                          cfg->gelu == GPT_GELU_TANH, s));
         }
-        // c_fc: du2 = dpre W_fc (into d1 [N, C]); dW_fc += dpre^T u2; db_fc += sum dpre
+        // c_fc: du2 = dpre W_fc (into d1 [N, C]); dW_fc += dpre^T u2; db_fc += sum dpre (bf16: above)
         GPT_TRY(linear_bwd(dpre, 4LL * C, L + A.u2, C, W.layer(l, W_FC_W), 4 * C, C, d1, F32_OUT, nullptr,
                            GL(l, W_FC_W), gT));
-        if (cfg->bias) GPT_TRY(launch_colsum(dpre, dt, N, 4 * C, GL(l, W_FC_B), 1, parts, s));
+        if (cfg->bias && !bf) GPT_TRY(launch_colsum(dpre, dt, N, 4 * C, GL(l, W_FC_B), 1, parts, s));
         GPT_TRY(launch_layernorm_backward(d1, reinterpret_cast<const float*>(L + A.x_mid), W.layer(l, W_LN2_W), dt, dx, 1,
                                           GL(l, W_LN2_W), cfg->bias ? GL(l, W_LN2_B) : nullptr, 1, parts, N, C, s,
                                           dx16, cfg->bias ? GL(l, W_PROJ_B) : nullptr));

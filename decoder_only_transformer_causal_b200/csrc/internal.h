@@ -117,11 +117,13 @@ size_t gemm_acc_split_bytes(int M, int N, int K);
 //   GEMM_BWD_ACC_F32     out fp32 += A B^T (a_mn allowed; split-K as launch_gemm_bf16_acc)
 //   GEMM_BWD_STORE_F32   out fp32  = A B^T
 //   GEMM_BWD_STORE_BF16  out bf16  = A B^T
-//   GEMM_BWD_DGELU_BF16  out bf16  = (A B^T) * aux, aux bf16 [M, ld_aux] the stored GELU derivative
+//   GEMM_BWD_DGELU_BF16  out bf16  = (A B^T) * aux, aux bf16 [M, ld_aux] the stored GELU derivative;
+//                        with colsum, also its column sums per 32-row band into colsum
+//                        [ceil(M / 32), N] (launch_colsum_bands finishes the bias gradient)
 enum { GEMM_BWD_ACC_F32 = 0, GEMM_BWD_STORE_F32 = 1, GEMM_BWD_STORE_BF16 = 2, GEMM_BWD_DGELU_BF16 = 3 };
 int launch_gemm_bf16_bwd(const bf16* A, long long lda, bool a_mn, const bf16* W, long long ldw, bool b_mn, void* out,
                          long long ldo, int M, int N, int K, int mode, const bf16* aux, long long ld_aux, int gelu,
-                         int32_t* status, cudaStream_t s, float* split_ws = nullptr);
+                         int32_t* status, cudaStream_t s, float* split_ws = nullptr, float* colsum = nullptr);
 
 // ---- tensor-core attention (attention_tc.cu); strides in elements
 struct AttnLayout {
@@ -230,6 +232,9 @@ int launch_layernorm_backward(const float* dy, const float* x, const void* w, in
                               float* dw, float* db, int accumulate_wb, float* part, int rows, int C, cudaStream_t s,
                               bf16* dx16 = nullptr, float* dsum = nullptr);
 int colsum_parts(int rows);              // part: [parts, C] floats
+// out[c] (+)= sum over i < n_part of part[i * C + c], in order of i (the second stage of the
+// per-band column sums a producer kernel leaves).
+int launch_colsum_bands(const float* part, int n_part, int C, float* out, int accumulate, cudaStream_t s);
 int launch_colsum(const void* y, int dtype, int rows, int C, float* out, int accumulate, float* part,
                   cudaStream_t s);
 int launch_gelu_backward(const float* dh, const void* pre, int dtype, void* dpre, long long n, int tanh_form,
