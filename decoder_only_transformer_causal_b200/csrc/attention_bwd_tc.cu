@@ -67,6 +67,12 @@ struct Params {
     const float* D;                   // [B*nh, Tp], padding 0
     float scale_log2, inv_sqrt_hs;
     int32_t* status;
+    // Optional: column sums of dq / dk / dv per 32-row band of each sequence (the first stage of the
+    // bias gradient of the layer that produced q, k, v): row b * bands + t / 32 of colsum
+    // [B * bands, cs_ld]; head h's columns of q, k, v start at cs_q, cs_k, cs_v + h * HS.
+    float* colsum;
+    long long cs_ld;
+    int cs_q, cs_k, cs_v, bands;
 };
 
 // Rows [t, t + box) of head h, batch b in a 4-D map {hs, head, t, b} or {hs, t, head, b}.
@@ -100,6 +106,36 @@ GPT_DEVINL void tmem_row_bf16(uint32_t taddr, float scale, uint32_t (&w)[32]) {
         for (int e = 0; e < 16; ++e)
             w[half * 16 + e] = pack_bf16x2(__uint_as_float(u[2 * e]) * scale, __uint_as_float(u[2 * e + 1]) * scale);
     }
+}
+
+// As tmem_row_bf16, and with cs (warp-uniform) the column sums of the warp's 32 rows of the scaled
+// fp32 values (rows with !valid add zero) into cs[0, 64): lane l writes columns l and 32 + l.
+GPT_DEVINL void tmem_row_bf16_colsum(uint32_t taddr, float scale, uint32_t (&w)[32], bool valid, float* cs) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+        uint32_t u[32];
+        tmem_ld32(taddr + half * 32, u);
+        float v[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(u[e]) * scale;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) w[half * 16 + e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
+        if (cs) {
+            if (!valid) {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) v[e] = 0.f;
+            }
+            cs[half * 32 + lane] = warp_colsum32(v);
+        }
+    }
+}
+
+// The band row of this warp's 32 rows [t0, t0 + 32) of sequence b in p.colsum, or null (no sums
+// asked for, or a band entirely past T).
+GPT_DEVINL float* colsum_band(const Params& p, int b, int t0) {
+    if (!p.colsum || t0 >= p.T) return nullptr;
+    return p.colsum + (static_cast<long long>(b) * p.bands + t0 / 32) * p.cs_ld;
 }
 
 // One 32-column half of a key row of the dK/dV kernel: P^T and dS^T for queries c0 + e, with packed
@@ -341,9 +377,10 @@ __global__ void __launch_bounds__(THREADS, 2)
             uint32_t w[32];
             const int j = k0 + r;
             const long long off = b * p.sb + h * p.sh + static_cast<long long>(j) * p.st;
-            tmem_row_bf16(tmem + 128 + lane_off, 1.f, w);
+            float* cs = colsum_band(p, b, k0 + quarter * 32);
+            tmem_row_bf16_colsum(tmem + 128 + lane_off, 1.f, w, j < p.T, cs ? cs + p.cs_v + h * HS : nullptr);
             if (j < p.T) store_row_bf16(p.dv + off, w);
-            tmem_row_bf16(tmem + 192 + lane_off, p.inv_sqrt_hs, w);
+            tmem_row_bf16_colsum(tmem + 192 + lane_off, p.inv_sqrt_hs, w, j < p.T, cs ? cs + p.cs_k + h * HS : nullptr);
             if (j < p.T) store_row_bf16(p.dk + off, w);
         }
     }
@@ -531,7 +568,8 @@ __global__ void __launch_bounds__(THREADS, 2)
         if (__all_sync(0xffffffffu, last)) {
             tc_fence_after();
             uint32_t w[32];
-            tmem_row_bf16(tmem + 128 + lane_off, p.inv_sqrt_hs, w);
+            float* cs = colsum_band(p, b, q0 + quarter * 32);
+            tmem_row_bf16_colsum(tmem + 128 + lane_off, p.inv_sqrt_hs, w, i < p.T, cs ? cs + p.cs_q + h * HS : nullptr);
             if (i < p.T) store_row_bf16(p.dq + b * p.sb + h * p.sh + static_cast<long long>(i) * p.st, w);
         }
     }
@@ -573,7 +611,7 @@ size_t attn_bwd_scratch_bytes(long long B, long long nh, long long T) {
 }
 
 int launch_attention_backward_tc(const AttnBwdLayout<bf16>& L, int B, int nh, int T, const float* D,
-                                 const float* lse2, int32_t* status, cudaStream_t s) {
+                                 const float* lse2, int32_t* status, cudaStream_t s, const AttnBwdColsum* cs) {
     using namespace attn_bwd;
     // Results are stored as 16-byte rows: 16-byte aligned bases and strides that are multiples of 8.
     auto aligned = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15) == 0; };
@@ -607,6 +645,14 @@ int launch_attention_backward_tc(const AttnBwdLayout<bf16>& L, int B, int nh, in
     p.scale_log2 = static_cast<float>(1.4426950408889634 / sqrt(static_cast<double>(HS)));
     p.inv_sqrt_hs = static_cast<float>(1.0 / sqrt(static_cast<double>(HS)));
     p.status = status;
+    if (cs) {
+        p.colsum = cs->part;
+        p.cs_ld = cs->ld;
+        p.cs_q = cs->col_q;
+        p.cs_k = cs->col_k;
+        p.cs_v = cs->col_v;
+        p.bands = (T + 31) / 32;
+    }
     static size_t opted_q[kMaxDevices] = {}, opted_kv[kMaxDevices] = {};
     rc = opt_in_smem(reinterpret_cast<const void*>(attn_bwd_dq_tc), Q_SMEM, opted_q);
     if (!rc) rc = opt_in_smem(reinterpret_cast<const void*>(attn_bwd_dkdv_tc), KV_SMEM, opted_kv);

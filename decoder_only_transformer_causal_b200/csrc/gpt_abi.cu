@@ -1139,7 +1139,8 @@ BwdPlan plan_bwd(const gpt_config_t* c, long long B, long long T) {
     P.D = off; off += a256(attn_bwd_scratch_bytes(B, c->n_head, T));
     const size_t lnp = static_cast<size_t>(layernorm_backward_parts(static_cast<int>(N), static_cast<int>(C))) * 3 * C;
     const size_t csp = static_cast<size_t>(colsum_parts(static_cast<int>(N))) * 4 * C;
-    const size_t bands = (N + 31) / 32 * 4 * C;  // db_fc's per-band sums from the DGELU product
+    // per-band column sums: db_fc's from the DGELU product, db_attn's from the attention backward
+    const size_t bands = std::max((N + 31) / 32 * 4 * C, static_cast<size_t>(B * ((T + 31) / 32)) * 3 * C);
     P.parts = off; off += a256(std::max({lnp, csp, bands}) * 4);
     P.sort = off; off += a256(N * 8);
     // split-K partial products of the weight-gradient GEMMs (bf16)
@@ -1462,6 +1463,7 @@ GPT_API int gpt_backward(const gpt_config_t* cfg, const void* weights, const int
                            nullptr, GL(l, W_PROJ_W), gT));
         // attention backward into dqkv (the qkv layout)
         const float* lse = reinterpret_cast<const float*>(L + A.lse);
+        bool attn_bias_done = false;
         const long long qsb = 3LL * C * T, ysb = static_cast<long long>(C) * T;
         if (bf) {
             const bf16* q = reinterpret_cast<const bf16*>(L + A.qkv);
@@ -1469,7 +1471,13 @@ GPT_API int gpt_backward(const gpt_config_t* cfg, const void* weights, const int
             AttnBwdLayout<bf16> AL{q, q + C, q + 2 * C, qsb, hs, 3LL * C,
                                    reinterpret_cast<const bf16*>(L + A.y), static_cast<const bf16*>(dy), ysb, hs, C,
                                    dq, dq + C, dq + 2 * C, lse};
-            GPT_TRY(launch_attention_backward(&AL, nullptr, B, nh, T, hs, D, status, s));
+            // the tensor-core kernels also leave dqkv's column sums per 32-row band (db_attn)
+            const AttnBwdColsum cs{parts, 3LL * C, 0, C, 2 * C};
+            bool cs_done = false;
+            GPT_TRY(launch_attention_backward(&AL, nullptr, B, nh, T, hs, D, status, s, cfg->bias ? &cs : nullptr,
+                                              &cs_done));
+            if (cs_done) GPT_TRY(launch_colsum_bands(parts, B * ((T + 31) / 32), 3 * C, GL(l, W_ATTN_B), 1, s));
+            attn_bias_done = cs_done;
         } else {
             const float* q = reinterpret_cast<const float*>(L + A.qkv);
             float* dq = static_cast<float*>(dqkv);
@@ -1478,10 +1486,11 @@ GPT_API int gpt_backward(const gpt_config_t* cfg, const void* weights, const int
                                     dq, dq + C, dq + 2 * C, lse};
             GPT_TRY(launch_attention_backward(nullptr, &AL, B, nh, T, hs, D, status, s));
         }
-        // c_attn: du1 = dqkv W_attn (into d1 [N, C]); dW_attn += dqkv^T u1; db_attn += sum dqkv
+        // c_attn: du1 = dqkv W_attn (into d1 [N, C]); dW_attn += dqkv^T u1; db_attn += sum dqkv (unless the
+        // attention backward's band sums gave it above)
         GPT_TRY(linear_bwd(dqkv, 3LL * C, L + A.u1, C, W.layer(l, W_ATTN_W), 3 * C, C, d1, F32_OUT, nullptr,
                            GL(l, W_ATTN_W), gT));
-        if (cfg->bias) GPT_TRY(launch_colsum(dqkv, dt, N, 3 * C, GL(l, W_ATTN_B), 1, parts, s));
+        if (cfg->bias && !attn_bias_done) GPT_TRY(launch_colsum(dqkv, dt, N, 3 * C, GL(l, W_ATTN_B), 1, parts, s));
         GPT_TRY(launch_layernorm_backward(d1, reinterpret_cast<const float*>(L + A.x_in), W.layer(l, W_LN1_W), dt, dx, 1,
                                           GL(l, W_LN1_W), cfg->bias ? GL(l, W_LN1_B) : nullptr, 1, parts, N, C, s,
                                           dx16, cfg->bias && l > 0 ? GL(l - 1, W_FC2_B) : nullptr));

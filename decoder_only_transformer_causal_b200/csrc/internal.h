@@ -261,11 +261,22 @@ int launch_gelu_deriv_inplace(void* pre, long long n, int dtype, int tanh_form, 
 // of 128 rows per head).  Exactly one of Lb / Lf is non-null; hs 32 or 64.  status: optional device
 // word that records GPT_ERR_TIMEOUT from the tensor-core kernels.
 size_t attn_bwd_scratch_bytes(long long B, long long nh, long long T);
+// Column sums of dq / dk / dv per 32-row band of each sequence, left by the tensor-core kernels:
+// part [B * ceil(T / 32), ld] floats; head h's columns of q, k, v start at col_q, col_k, col_v +
+// h * hs (finish with launch_colsum_bands).
+struct AttnBwdColsum {
+    float* part;
+    long long ld;
+    int col_q, col_k, col_v;
+};
+// cs (optional): *cs_done says whether the band sums were written (the tensor-core kernels ran).
 int launch_attention_backward(const AttnBwdLayout<bf16>* Lb, const AttnBwdLayout<float>* Lf, int B, int nh, int T,
-                              int hs, float* scratch, int32_t* status, cudaStream_t s);
+                              int hs, float* scratch, int32_t* status, cudaStream_t s,
+                              const AttnBwdColsum* cs = nullptr, bool* cs_done = nullptr);
 // bf16, head size 64: returns GPT_ERR_BAD_ALIGN (nothing launched) when an operand cannot be
 // described by a TMA map.
 int launch_attention_backward_tc(const AttnBwdLayout<bf16>& L, int B, int nh, int T, const float* D,
-                                 const float* lse2, int32_t* status, cudaStream_t s);
+                                 const float* lse2, int32_t* status, cudaStream_t s,
+                                 const AttnBwdColsum* cs = nullptr);
 
 }  // namespace gpt

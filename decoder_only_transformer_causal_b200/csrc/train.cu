@@ -285,7 +285,7 @@ __global__ void __launch_bounds__(2 * kBwdRows)
 // D / L2: the padded [B*nh, Tp] arrays of attn_bwd_rowdot_kernel.
 template <typename E, int HS>
 int attn_bwd_typed(const AttnBwdLayout<E>& L, int B, int nh, int T, float* D, float* L2, int32_t* status,
-                   cudaStream_t s) {
+                   cudaStream_t s, const AttnBwdColsum* cs, bool* cs_done) {
     const int Tp = (T + 127) / 128 * 128;
     const long long threads = static_cast<long long>(B) * nh * Tp * (HS / 8);
     const int vec = ((reinterpret_cast<uintptr_t>(L.o) | reinterpret_cast<uintptr_t>(L.dout)) & 15) == 0 &&
@@ -296,8 +296,11 @@ int attn_bwd_typed(const AttnBwdLayout<E>& L, int B, int nh, int T, float* D, fl
     if constexpr (sizeof(E) == 2 && HS == 64) {
         // Tensor-core kernels whenever the operands can be described by TMA maps (16-byte
         // aligned bases and strides); the SIMT kernels below otherwise.
-        rc = launch_attention_backward_tc(L, B, nh, T, D, L2, status, s);
-        if (rc != GPT_ERR_BAD_ALIGN) return rc;
+        rc = launch_attention_backward_tc(L, B, nh, T, D, L2, status, s, cs);
+        if (rc != GPT_ERR_BAD_ALIGN) {
+            if (cs_done) *cs_done = cs != nullptr && rc == GPT_OK;
+            return rc;
+        }
     }
     const float scale_log2 = static_cast<float>(1.4426950408889634 / sqrt(static_cast<double>(HS)));
     const float inv = static_cast<float>(1.0 / sqrt(static_cast<double>(HS)));
@@ -357,17 +360,19 @@ int launch_gelu_deriv_inplace(void* pre, long long n, int dtype, int tanh_form, 
 }
 
 int launch_attention_backward(const AttnBwdLayout<bf16>* Lb, const AttnBwdLayout<float>* Lf, int B, int nh, int T,
-                              int hs, float* scratch, int32_t* status, cudaStream_t s) {
+                              int hs, float* scratch, int32_t* status, cudaStream_t s, const AttnBwdColsum* cs,
+                              bool* cs_done) {
+    if (cs_done) *cs_done = false;
     if (B == 0 || nh == 0 || T == 0) return GPT_OK;
     float* D = scratch;
     float* L2 = scratch + static_cast<long long>(B) * nh * ((T + 127) / 128 * 128);
     if (Lb) {
-        if (hs == 64) return attn_bwd_typed<bf16, 64>(*Lb, B, nh, T, D, L2, status, s);
-        if (hs == 32) return attn_bwd_typed<bf16, 32>(*Lb, B, nh, T, D, L2, status, s);
+        if (hs == 64) return attn_bwd_typed<bf16, 64>(*Lb, B, nh, T, D, L2, status, s, cs, cs_done);
+        if (hs == 32) return attn_bwd_typed<bf16, 32>(*Lb, B, nh, T, D, L2, status, s, cs, cs_done);
         return GPT_ERR_UNSUPPORTED;
     }
-    if (hs == 64) return attn_bwd_typed<float, 64>(*Lf, B, nh, T, D, L2, status, s);
-    if (hs == 32) return attn_bwd_typed<float, 32>(*Lf, B, nh, T, D, L2, status, s);
+    if (hs == 64) return attn_bwd_typed<float, 64>(*Lf, B, nh, T, D, L2, status, s, cs, cs_done);
+    if (hs == 32) return attn_bwd_typed<float, 32>(*Lf, B, nh, T, D, L2, status, s, cs, cs_done);
     return GPT_ERR_UNSUPPORTED;
 }
 
