@@ -19,7 +19,9 @@
 // -lse2 and D come from [B*nh, Tp] arrays (Tp = T rounded up to 128) whose padding holds
 // -lse2 = -inf and D = 0, so queries past T get p = 0 with no test; the dK/dV kernel copies the
 // 64 entries of each query tile next to its Q / dO tiles with one bulk copy each.  The row warps
-// form P and dS with packed f32x2 arithmetic.
+// form P and dS with packed f32x2 arithmetic.  The inner tiles stream through a ring: two stages in
+// the dK/dV kernel (its P^T and dS^T operands take the rest of the shared memory two CTAs per SM
+// allow), four in the dQ kernel (three tiles in flight ahead of the one being used).
 // Roles (192 threads, two CTAs per SM): warp 0 TMA producer, warp 1 MMA issuer (one thread),
 // warps 2-5 one outer row per thread.  TMEM (256 columns): dK/dV kernel S^T [0,64), dP^T
 // [64,128), dV [128,192), dK [192,256); dQ kernel S [0,64), dP [64,128), dQ [128,192),
@@ -43,6 +45,8 @@ constexpr int ROWS_BYTES = BM * BN * 2;   // 16 KB: a bf16 [128 x 64] operand wr
 constexpr int VEC_BYTES = BN * 4;         // 64 fp32
 constexpr uint32_t TMEM_COLS = 256;
 constexpr int kNumBars = 11;
+constexpr int QNST = 4;  // dQ kernel: stages of the key / value tiles (prefetch three tiles ahead)
+constexpr int kQBars = 7 + 2 * QNST;
 
 // dK/dV kernel: K, V | Q[2], dO[2] | P^T, dS^T | lse2[2], D[2] | barriers
 constexpr int KV_OFF_Q = 2 * OUTER_BYTES;
@@ -52,10 +56,10 @@ constexpr int KV_OFF_DS = KV_OFF_P + ROWS_BYTES;
 constexpr int KV_OFF_VEC = KV_OFF_DS + ROWS_BYTES;
 constexpr int KV_OFF_BAR = KV_OFF_VEC + 4 * VEC_BYTES;
 constexpr int KV_SMEM = KV_OFF_BAR + 256 + 1024;
-// dQ kernel: Q, dO | K[2], V[2] | barriers
+// dQ kernel: Q, dO | K[QNST], V[QNST] | barriers
 constexpr int Q_OFF_K = 2 * OUTER_BYTES;
-constexpr int Q_OFF_V = Q_OFF_K + 2 * INNER_BYTES;
-constexpr int Q_OFF_BAR = Q_OFF_V + 2 * INNER_BYTES;
+constexpr int Q_OFF_V = Q_OFF_K + QNST * INNER_BYTES;
+constexpr int Q_OFF_BAR = Q_OFF_V + QNST * INNER_BYTES;
 constexpr int Q_SMEM = Q_OFF_BAR + 256 + 1024;
 
 struct Params {
@@ -408,15 +412,15 @@ __global__ void __launch_bounds__(THREADS, 2)
     uint8_t* sV = smem + Q_OFF_V;  // 2 stages
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Q_OFF_BAR);
     uint64_t* a_full = bars + 0;
-    uint64_t* b_full = bars + 1;   // [2]
-    uint64_t* b_empty = bars + 3;  // [2]
-    uint64_t* s_full = bars + 5;
-    uint64_t* s_free = bars + 6;   // 128 arrivals
-    uint64_t* p_full = bars + 7;   // dS in TMEM (128 arrivals)
-    uint64_t* ds_free = bars + 8;  // the dQ MMA has read dS
-    uint64_t* acc_done = bars + 9;
-    uint64_t* drain = bars + 10;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
+    uint64_t* b_full = bars + 1;
+    uint64_t* b_empty = bars + 1 + QNST;
+    uint64_t* s_full = bars + 1 + 2 * QNST;
+    uint64_t* s_free = s_full + 1;
+    uint64_t* p_full = s_full + 2;
+    uint64_t* ds_free = s_full + 3;
+    uint64_t* acc_done = s_full + 4;
+    uint64_t* drain = s_full + 5;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kQBars);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5;
@@ -430,7 +434,7 @@ __global__ void __launch_bounds__(THREADS, 2)
     const int nk = (min(q0 + BM, p.T) + BN - 1) / BN;  // key tiles n * 64, n < nk
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kNumBars; ++i) mbar_init(&bars[i], (i == 6 || i == 7) ? 128u : 1u);
+        for (int i = 0; i < kQBars; ++i) mbar_init(&bars[i], (i == 2 + 2 * QNST || i == 3 + 2 * QNST) ? 128u : 1u);
         *abort_flag = 0;
         fence_barrier_init();
         fence_proxy_async_shared();
@@ -457,16 +461,16 @@ __global__ void __launch_bounds__(THREADS, 2)
             load_rows(sG, &tmG, a_full, p.o_head_inner, h, q0, b);
             int issued = 0;
             for (int n = 0; n < nk; ++n) {
-                const int st = n & 1;
-                if (!mbar_wait(&b_empty[st], ((n >> 1) & 1) ^ 1u, abort_flag)) break;
+                const int st = n % QNST;
+                if (!mbar_wait(&b_empty[st], ((n / QNST) & 1) ^ 1u, abort_flag)) break;
                 mbar_arrive_expect_tx(&b_full[st], 2 * INNER_BYTES);
                 load_rows(sK + st * INNER_BYTES, &tmK, &b_full[st], p.qk_head_inner, h, n * BN, b);
                 load_rows(sV + st * INNER_BYTES, &tmV, &b_full[st], p.qk_head_inner, h, n * BN, b);
                 ++issued;
             }
             mbar_drain(a_full, 0);
-            for (int i = 1; i <= 2; ++i)
-                if (issued - i >= 0) mbar_drain(&b_full[(issued - i) & 1], ((issued - i) >> 1) & 1);
+            for (int i = 1; i <= QNST; ++i)
+                if (issued - i >= 0) mbar_drain(&b_full[(issued - i) % QNST], ((issued - i) / QNST) & 1);
         }
     } else if (warp == 1) {
         if (lane == 0) {
@@ -478,8 +482,8 @@ __global__ void __launch_bounds__(THREADS, 2)
             tc_fence_after();
             for (int n = 0; ok && n <= nk; ++n) {
                 if (n < nk) {
-                    const int st = n & 1;
-                    if (!mbar_wait(&b_full[st], (n >> 1) & 1, abort_flag)) break;
+                    const int st = n % QNST;
+                    if (!mbar_wait(&b_full[st], (n / QNST) & 1, abort_flag)) break;
                     if (n > 0 && !mbar_wait(s_free, (n - 1) & 1, abort_flag)) break;
                     tc_fence_after();
                     const uint32_t k_addr = smem_addr(sK + st * INNER_BYTES);
@@ -496,7 +500,7 @@ __global__ void __launch_bounds__(THREADS, 2)
                 }
                 if (n > 0) {
                     // dQ += dS_m K_m
-                    const int m = n - 1, st = m & 1;
+                    const int m = n - 1, st = m % QNST;
                     if (!mbar_wait(p_full, m & 1, abort_flag)) break;
                     tc_fence_after();
                     const uint32_t k_addr = smem_addr(sK + st * INNER_BYTES);
