@@ -258,10 +258,8 @@ GPT_DEVINL void issue_head_tile(const StepArgs& a, int tile, uint8_t* buf, uint6
 GPT_DEVINL void grid_arrive(Ctx& c) {
     __syncthreads();
     c.target += gridDim.x;
-    if (threadIdx.x == 0) {
-        __threadfence();  // this CTA's writes of the phase, before its arrival
-        atomicAdd(c.a.bar, 1u);
-    }
+    if (threadIdx.x == 0)  // release: this CTA's writes of the phase (ordered by the barrier above) first
+        asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(c.a.bar) : "memory");
 }
 
 // The wait, bounded.  Returns false (every thread) once any wait has given up.
@@ -271,11 +269,11 @@ GPT_DEVINL bool grid_wait(Ctx& c) {
         const uint64_t limit = g_wait_limit_ns;
         // the testing aid: a forced time-out waits for one arrival more than there will be
         const unsigned target = c.target + (g_force_timeout ? 1u : 0u);
-        for (;;) {
+        for (uint32_t it = 1;; ++it) {
             unsigned v;
             asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(c.a.bar) : "memory");
             if (v >= target) break;
-            if (globaltimer_ns() - t0 > limit) {
+            if ((it & 15u) == 0u && globaltimer_ns() - t0 > limit) {  // the clock read every 16 polls
                 *c.abort = 1;
                 set_status(c.a.status, GPT_ERR_TIMEOUT);
                 break;
