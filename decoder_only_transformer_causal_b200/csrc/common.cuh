@@ -168,6 +168,28 @@ GPT_DEVINL uint32_t map_to_rank(const void* p, uint32_t rank) {
 GPT_DEVINL void mbar_arrive_remote(uint32_t cluster_addr) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
+// Loads, stores and adds on another CTA's shared memory (cluster addresses from map_to_rank).
+GPT_DEVINL uint32_t ld_cluster_u32(uint32_t cluster_addr) {
+    uint32_t v;
+    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(cluster_addr) : "memory");
+    return v;
+}
+GPT_DEVINL double ld_cluster_f64(uint32_t cluster_addr) {
+    double v;
+    asm volatile("ld.shared::cluster.f64 %0, [%1];" : "=d"(v) : "r"(cluster_addr) : "memory");
+    return v;
+}
+GPT_DEVINL void st_cluster_u32(uint32_t cluster_addr, uint32_t v) {
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+GPT_DEVINL void red_cluster_add_u32(uint32_t cluster_addr, uint32_t v) {
+    asm volatile("red.shared::cluster.add.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+GPT_DEVINL uint32_t atom_cluster_add_u32(uint32_t cluster_addr, uint32_t v) {
+    uint32_t old;
+    asm volatile("atom.shared::cluster.add.u32 %0, [%1], %2;" : "=r"(old) : "r"(cluster_addr), "r"(v) : "memory");
+    return old;
+}
 // Stores a 64-bit value into another CTA's shared memory (cluster address).
 GPT_DEVINL void st_cluster_u64(uint32_t cluster_addr, unsigned long long v) {
     asm volatile("st.shared::cluster.u64 [%0], %1;" ::"r"(cluster_addr), "l"(v) : "memory");

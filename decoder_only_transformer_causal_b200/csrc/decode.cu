@@ -762,6 +762,268 @@ __global__ void __launch_bounds__(kSampleThreads)
     if (lane == 0) out[b * ld_out] = last;
 }
 
+// The same draw with a row spread over a cluster of kSampleCtas CTAs (V >= kSampleClusterMinV): one
+// CTA's instruction rate bounds the single-CTA kernel (three passes over the row by one SM).
+// CTA rank r stages entries [r S, min(V, (r + 1) S)) of the row (S = ceil(V / kSampleCtas) rounded up
+// to a multiple of 4) and counts their keys' top 11 bits; the counts meet in CTA 0's histogram
+// (distributed shared memory), from which every CTA finds the bin of the top_k-th largest key; the
+// bin's members are gathered into CTA 0, copied back by every CTA and resolved there (bits 20..10,
+// 9..0), so each CTA knows the threshold key without another barrier.  (A bin of more than
+// kSampleCand members is bisected: each step's count is summed across the cluster in CTA 0.)  The
+// draw: each CTA sums its kept exponentials per warp segment in fp64; every CTA adds the CTAs'
+// totals in rank order, so the interval [lo, hi) of warp w of CTA r has the same computed bounds in
+// every CTA and the intervals tile [0, total) exactly; the one warp whose interval holds u * total
+// walks its segment as in the single-CTA kernel.
+constexpr int kSampleCtas = 8;
+constexpr int kSampleClusterMinV = 4096;
+constexpr int kCThreads = 512;
+constexpr int kCWarps = kCThreads / 32;
+
+// top_bin for kCThreads threads, four bins each.
+GPT_DEVINL void top_bin_c(const uint32_t* hist, uint32_t need, uint32_t* s_wtot, uint32_t* s_bin, uint32_t* s_need) {
+    constexpr int PER = kSampleBins / kCThreads;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    uint32_t h[PER], sum = 0;
+#pragma unroll
+    for (int k = 0; k < PER; ++k) {
+        h[k] = hist[kSampleBins - 1 - (PER * tid + k)];
+        sum += h[k];
+    }
+    uint32_t incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t nb = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += nb;
+    }
+    if (lane == 31) s_wtot[warp] = incl;
+    __syncthreads();
+    uint32_t before = 0;
+    for (int w = 0; w < warp; ++w) before += s_wtot[w];
+    incl += before;
+    uint32_t acc = incl - sum;
+    if (acc < need && incl >= need) {
+        bool found = false;
+#pragma unroll
+        for (int k = 0; k < PER; ++k) {
+            if (!found && acc + h[k] >= need) {
+                *s_bin = kSampleBins - 1 - (PER * tid + k);
+                *s_need = need - acc;
+                found = true;
+            }
+            acc += h[k];
+        }
+    }
+    __syncthreads();
+}
+
+__global__ void __launch_bounds__(kCThreads)
+    sample_cluster_kernel(const float* __restrict__ logits, long long ld_logits, int V, float temperature, int top_k,
+                          const float* __restrict__ u, int64_t* __restrict__ out, long long ld_out) {
+    griddep_launch_dependents();
+    griddep_wait();
+    extern __shared__ __align__(16) float zs[];  // this CTA's slice of the row
+    __shared__ uint32_t hist[kSampleBins];       // this slice's counts; CTA 0's become the row's
+    __shared__ uint32_t hist2[kSampleBins];      // the row's counts, then the finer levels
+    __shared__ uint32_t cand[kSampleCand];       // the bin's members (gathered in CTA 0, copied by the rest)
+    __shared__ uint32_t s_acc[3], s_ncand, s_bin, s_need;
+    __shared__ uint32_t s_wtot[kCWarps];
+    __shared__ float s_wmax[kCWarps];
+    __shared__ double s_wsum[kCWarps];
+    __shared__ uint32_t s_max;  // this slice's largest logit (float bits)
+    __shared__ double s_tot;    // this slice's sum of kept exponentials
+    const uint32_t rank = cluster_ctarank();
+    const int b = static_cast<int>(blockIdx.x) / kSampleCtas;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const float* lg = logits + b * ld_logits;
+    const bool filter = top_k > 0 && top_k < V;
+    const int S = ((V + kSampleCtas - 1) / kSampleCtas + 3) & ~3;
+    const int c0 = min(V, static_cast<int>(rank) * S);
+    const int n = min(V, c0 + S) - c0;
+
+    for (int i = tid; i < kSampleBins; i += kCThreads) hist[i] = 0;
+    if (tid < 3) s_acc[tid] = 0;
+    if (tid == 0) s_ncand = 0;
+    cluster_sync();  // every CTA of the cluster runs, its counters zero, before any remote access
+
+    // 1. the slice: shared memory, its maximum, the histogram of its keys' top 11 bits
+    float mx = -INFINITY;
+    const bool vec = ((ld_logits | c0) & 3) == 0 && (reinterpret_cast<uintptr_t>(logits) & 15) == 0;
+    const int n4 = vec ? n >> 2 : 0;
+    for (int i0 = tid; i0 < n4; i0 += 4 * kCThreads) {
+        float4 v[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int i = i0 + j * kCThreads;
+            v[j] = i < n4 ? __ldcg(reinterpret_cast<const float4*>(lg + c0) + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int i = i0 + j * kCThreads;
+            if (i < n4) {
+                reinterpret_cast<float4*>(zs)[i] = v[j];
+                mx = fmaxf(mx, fmaxf(fmaxf(v[j].x, v[j].y), fmaxf(v[j].z, v[j].w)));
+                if (filter) {
+                    atomicAdd(&hist[fkey(v[j].x) >> 21], 1u);
+                    atomicAdd(&hist[fkey(v[j].y) >> 21], 1u);
+                    atomicAdd(&hist[fkey(v[j].z) >> 21], 1u);
+                    atomicAdd(&hist[fkey(v[j].w) >> 21], 1u);
+                }
+            }
+        }
+    }
+    for (int i = 4 * n4 + tid; i < n; i += kCThreads) {
+        const float v = __ldcg(lg + c0 + i);
+        zs[i] = v;
+        mx = fmaxf(mx, v);
+        if (filter) atomicAdd(&hist[fkey(v) >> 21], 1u);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if (lane == 0) s_wmax[warp] = mx;
+    __syncthreads();
+    if (tid == 0) {
+        float m0 = s_wmax[0];
+        for (int w = 1; w < kCWarps; ++w) m0 = fmaxf(m0, s_wmax[w]);
+        s_max = __float_as_uint(m0);
+    }
+    // 2. the slice's counts into CTA 0's histogram
+    if (filter && rank != 0) {
+        const uint32_t h0 = map_to_rank(hist, 0);
+        for (int t = tid; t < kSampleBins; t += kCThreads)
+            if (hist[t]) red_cluster_add_u32(h0 + 4u * t, hist[t]);
+    }
+    cluster_sync();  // CTA 0 holds the row's counts; every slice maximum is written
+
+    // 3. the row's maximum; the bin of the top_k-th largest key, found by every CTA
+    float lmax = -INFINITY;
+    for (int r = 0; r < kSampleCtas; ++r) lmax = fmaxf(lmax, __uint_as_float(ld_cluster_u32(map_to_rank(&s_max, r))));
+    const float m = lmax / temperature;  // the largest z (division is monotone)
+    uint32_t thr_key = 0;                // key of the top_k-th largest logit
+    if (filter) {
+        const uint32_t h0 = map_to_rank(hist, 0);
+        for (int t = tid; t < kSampleBins; t += kCThreads) hist2[t] = rank == 0 ? hist[t] : ld_cluster_u32(h0 + 4u * t);
+        __syncthreads();
+        top_bin_c(hist2, static_cast<uint32_t>(top_k), s_wtot, &s_bin, &s_need);
+        const uint32_t bin = s_bin, need2 = s_need;
+        const uint32_t nbin = hist2[bin];
+        uint32_t lo = bin << 21, hi = lo | ((1u << 21) - 1);  // invariant: count(key >= lo) >= need
+        if (nbin <= kSampleCand) {
+            // 4. the slice's members of the bin appended to CTA 0's list (one remote add per warp and pass)
+            const uint32_t cnt0 = map_to_rank(&s_ncand, 0), cand0 = map_to_rank(cand, 0);
+            for (int base = 0; base < n; base += kCThreads) {
+                const int i = base + tid;
+                const uint32_t key = i < n ? fkey(zs[i]) : 0u;
+                const bool hit = i < n && (key >> 21) == bin;
+                const uint32_t mask = __ballot_sync(0xffffffffu, hit);
+                if (mask) {
+                    uint32_t pos = 0;
+                    if (lane == 0) pos = atom_cluster_add_u32(cnt0, static_cast<uint32_t>(__popc(mask)));
+                    pos = __shfl_sync(0xffffffffu, pos, 0);
+                    if (hit) st_cluster_u32(cand0 + 4u * (pos + __popc(mask & ((1u << lane) - 1u))), key);
+                }
+            }
+            cluster_sync();  // CTA 0 holds the bin's nbin members
+            // 5. every CTA resolves bits 20..10, then 9..0, from its own copy of the members
+            if (rank != 0)
+                for (uint32_t i = tid; i < nbin; i += kCThreads) cand[i] = ld_cluster_u32(cand0 + 4u * i);
+            for (int i = tid; i < kSampleBins; i += kCThreads) hist2[i] = 0;
+            __syncthreads();
+            for (uint32_t i = tid; i < nbin; i += kCThreads) atomicAdd(&hist2[(cand[i] >> 10) & 2047u], 1u);
+            __syncthreads();
+            top_bin_c(hist2, need2, s_wtot, &s_bin, &s_need);
+            const uint32_t bin2 = s_bin, need3 = s_need;
+            for (int i = tid; i < kSampleBins; i += kCThreads) hist2[i] = 0;
+            __syncthreads();
+            for (uint32_t i = tid; i < nbin; i += kCThreads)
+                if (((cand[i] >> 10) & 2047u) == bin2) atomicAdd(&hist2[cand[i] & 1023u], 1u);
+            __syncthreads();
+            top_bin_c(hist2, need3, s_wtot, &s_bin, &s_need);  // bins 1024.. are empty
+            lo = (bin << 21) | (bin2 << 10) | s_bin;
+        } else {
+            // the bin bisected over the row; each step's count summed in CTA 0 (three rotating
+            // counters: step k adds into s_acc[k % 3] and CTA 0 clears s_acc[(k + 1) % 3], which no CTA
+            // can still be reading)
+            const uint32_t acc0 = map_to_rank(s_acc, 0);
+            for (int it = 0; it < 22 && lo < hi; ++it) {  // lo, hi agree in every CTA
+                const uint32_t mid = lo + (hi - lo + 1) / 2;
+                uint32_t c = 0;
+                for (int i = tid; i < n; i += kCThreads) {
+                    const uint32_t key = fkey(zs[i]);
+                    c += (key >> 21) == bin && key >= mid;
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+                if (lane == 0 && c) red_cluster_add_u32(acc0 + 4u * (it % 3), c);
+                if (rank == 0 && tid == 0) s_acc[(it + 1) % 3] = 0;
+                cluster_sync();
+                if (ld_cluster_u32(acc0 + 4u * (it % 3)) >= need2) lo = mid;
+                else hi = mid - 1;
+            }
+        }
+        thr_key = lo;
+    }
+
+    // 6. the slice's kept exponentials summed per warp segment (fp64), then the CTAs' totals in order
+    const int seg = ((n + kCWarps * 32 - 1) / (kCWarps * 32)) * 32;
+    const int s0 = min(n, warp * seg), s1 = min(n, s0 + seg);
+    double part = 0.0;
+    for (int i = s0 + lane; i < s1; i += 32) {
+        const float li = zs[i];
+        if (fkey(li) >= thr_key) part += static_cast<double>(expf(li / temperature - m));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+    if (lane == 0) s_wsum[warp] = part;
+    __syncthreads();
+    double wlo = 0.0, whi = 0.0, ctot = 0.0;
+    for (int w = 0; w < kCWarps; ++w) {
+        if (w == warp) wlo = ctot;
+        ctot += s_wsum[w];
+        if (w == warp) whi = ctot;
+    }
+    if (tid == 0) s_tot = ctot;
+    cluster_sync();  // every slice total written
+    double before = 0.0, after = 0.0, total = 0.0;
+    for (int r = 0; r < kSampleCtas; ++r) {
+        if (r == static_cast<int>(rank)) before = total;
+        total += ld_cluster_f64(map_to_rank(&s_tot, r));
+        if (r == static_cast<int>(rank)) after = total;
+    }
+    cluster_sync();  // no CTA leaves while another may still read its shared memory
+    // this warp's interval: [before + wlo, before + whi), its last warp's upper end the next slice's start
+    const double target = static_cast<double>(__ldcg(u + b)) * total;
+    const double lo_b = before + wlo, hi_b = warp + 1 < kCWarps ? before + whi : after;
+    const double seg_sum = s_wsum[warp];
+    if (!(seg_sum > 0.0 && lo_b <= target && target < hi_b)) return;
+    double cum = lo_b;
+    long long last = -1;
+    for (int i0 = s0; i0 < s1; i0 += 32) {
+        const int i = i0 + lane;
+        double p = 0.0;
+        if (i < s1) {
+            const float li = zs[i];
+            if (fkey(li) >= thr_key) p = static_cast<double>(expf(li / temperature - m));
+        }
+        const uint32_t nz = __ballot_sync(0xffffffffu, p > 0.0);
+        if (!nz) continue;
+        double c = p;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const double nb = __shfl_up_sync(0xffffffffu, c, o);
+            if (lane >= o) c += nb;
+        }
+        c += cum;
+        const uint32_t hit = __ballot_sync(0xffffffffu, p > 0.0 && c > target);
+        if (hit) {
+            if (lane == __ffs(hit) - 1) out[b * ld_out] = c0 + i;
+            return;
+        }
+        last = c0 + i0 + 31 - __clz(nz);
+        cum = __shfl_sync(0xffffffffu, c, 31);
+    }
+    if (lane == 0) out[b * ld_out] = last;
+}
+
 }  // namespace
 
 // ------------------------------------------------------------------ launchers
@@ -926,6 +1188,17 @@ int sample_max_vocab() { return kSampleMaxV; }
 int launch_sample(const float* logits, long long ld_logits, int B, int V, float temperature, int top_k,
                   const float* u, int64_t* out, long long ld_out, cudaStream_t s) {
     if (V > kSampleMaxV) return GPT_ERR_UNSUPPORTED;
+    if (V >= kSampleClusterMinV) {
+        const int S = ((V + kSampleCtas - 1) / kSampleCtas + 3) & ~3;
+        // static + dynamic shared memory pass 48 KB: the dynamic part needs the opt-in
+        static size_t opted_c[kMaxDevices] = {};
+        const int rc = opt_in_smem(reinterpret_cast<const void*>(sample_cluster_kernel),
+                                   ((kSampleMaxV + kSampleCtas - 1) / kSampleCtas + 3) / 4 * 4 * sizeof(float), opted_c);
+        if (rc) return rc;
+        return launch_overlapped_cluster(sample_cluster_kernel, kSampleCtas, dim3(B * kSampleCtas), dim3(kCThreads),
+                                         static_cast<size_t>(S) * sizeof(float), s, logits, ld_logits, V, temperature,
+                                         top_k, u, out, ld_out);
+    }
     static size_t opted[kMaxDevices] = {};
     const int smem = V * static_cast<int>(sizeof(float));
     const int rc = opt_in_smem(reinterpret_cast<const void*>(sample_kernel), kSampleMaxV * sizeof(float), opted);

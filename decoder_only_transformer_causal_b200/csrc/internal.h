@@ -42,10 +42,10 @@ int launch_overlapped(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem
     return cuda_status(cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...));
 }
 
-// The same in clusters of two CTAs (the 2-SM MMA's pairs); grid.x must be even.
+// The same in clusters of `cluster_x` CTAs along x; grid.x must be a multiple of it.
 template <typename... KArgs, typename... Args>
-int launch_overlapped_pairs(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
-                            Args&&... args) {
+int launch_overlapped_cluster(void (*kern)(KArgs...), unsigned cluster_x, dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t s, Args&&... args) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = block;
@@ -55,12 +55,19 @@ int launch_overlapped_pairs(void (*kern)(KArgs...), dim3 grid, dim3 block, size_
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     attr[1].id = cudaLaunchAttributeClusterDimension;
-    attr[1].val.clusterDim.x = 2;
+    attr[1].val.clusterDim.x = cluster_x;
     attr[1].val.clusterDim.y = 1;
     attr[1].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
     return cuda_status(cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...));
+}
+
+// Clusters of two CTAs (the 2-SM MMA's pairs); grid.x must be even.
+template <typename... KArgs, typename... Args>
+int launch_overlapped_pairs(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                            Args&&... args) {
+    return launch_overlapped_cluster(kern, 2u, grid, block, smem, s, static_cast<Args&&>(args)...);
 }
 
 // ---- TMA descriptors (cuTensorMapEncodeTiled through the runtime's driver entry point)

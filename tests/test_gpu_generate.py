@@ -85,6 +85,26 @@ def test_sample_matches_oracle(V, B, temperature, top_k, ties):
         assert np.array_equal(got, logits.argmax(-1).numpy())
 
 
+@pytest.mark.parametrize("V,top_k", [(3000, 100), (8192, 100), (50304, 3000)])
+def test_sample_crowded_bin(V, top_k):
+    """Every logit in [1, 1.2): one bin of the top-11-bit histogram holds the whole row, more
+    members than the candidate buffer, so the threshold is found by bisection (over one CTA's row
+    for V < 4096, over a cluster's slices otherwise)."""
+    from decoder_only_transformer_causal_b200 import native
+    g = torch.Generator().manual_seed(V)
+    base = 1.0 + 0.2 * torch.rand(3, V, generator=g)
+    reps = 8
+    logits = base.repeat(reps, 1)
+    u = seeded.make_uniforms(1, 3 * reps)[0]
+    got = native.sample(logits.cuda(), u.cuda(), 0.9, top_k).cpu().numpy()
+    ref = oracle.gen.sample(f64(logits), 0.9, top_k, f64(u))
+    bad = [i for i in np.nonzero(got != ref)[0]
+           if not allowed_pick(f64(logits[i]), float(u[i]), int(got[i]), 0.9, top_k, 0.0)]
+    assert not bad, [(i, got[i], ref[i], float(u[i])) for i in bad[:5]]
+    kth = np.sort(logits.numpy(), axis=1)[:, -top_k]
+    assert all(logits[i, got[i]].item() >= kth[i] for i in range(len(got)))
+
+
 def test_sample_strided_output():
     from decoder_only_transformer_causal_b200 import native
     logits = seeded.make_logits(4, 777).cuda()
