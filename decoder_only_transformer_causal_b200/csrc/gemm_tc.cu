@@ -35,10 +35,12 @@ int max_pairs(const void* kern, int threads, size_t smem, int* cache) {
 
 // PAIR: 256-row tiles on CTA pairs (the 2-SM MMA); the B map's box must then be 128 rows
 // (K-major B) — see b_box_rows().
+// tx: EPI_DGELU's derivative map (any map otherwise; it is not read).
 template <int EPI, int GELU_TANH, int A_MN = 0, int B_MN = 0, int PAIR = 0>
 int launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, const gemm::Params& p,
-               cudaStream_t s) {
-    using L = gemm::Cfg<kBN, PAIR>;
+               cudaStream_t s, const CUtensorMap* tx = nullptr) {
+    using L = gemm::Cfg<kBN, PAIR, EPI == gemm::EPI_DGELU>;
+    const CUtensorMap& txr = tx ? *tx : tc;
     auto kern = gemm::gemm_bf16_tc<kBN, EPI, GELU_TANH, A_MN, B_MN, PAIR>;
     static size_t opted[kMaxDevices] = {};
     const int rc = opt_in_smem(reinterpret_cast<const void*>(kern), L::SMEM_BYTES, opted);
@@ -50,10 +52,10 @@ int launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& 
         int units = max_pairs(reinterpret_cast<const void*>(kern), L::THREADS, L::SMEM_BYTES, cache);
         if (units <= 0) units = num_sms() / 2;
         units = tiles < units ? tiles : units;
-        return launch_overlapped_pairs(kern, dim3(2 * units), dim3(L::THREADS), L::SMEM_BYTES, s, ta, tb, tc, p);
+        return launch_overlapped_pairs(kern, dim3(2 * units), dim3(L::THREADS), L::SMEM_BYTES, s, ta, tb, tc, txr, p);
     }
     const int grid = tiles < num_sms() ? tiles : num_sms();
-    return launch_overlapped(kern, dim3(grid), dim3(L::THREADS), L::SMEM_BYTES, s, ta, tb, tc, p);
+    return launch_overlapped(kern, dim3(grid), dim3(L::THREADS), L::SMEM_BYTES, s, ta, tb, tc, txr, p);
 }
 
 // 2-SM pairs pay off once there are two 128-row blocks to pair.
@@ -241,9 +243,14 @@ int launch_gemm_bf16_bwd(const bf16* A, long long lda, bool a_mn, const bf16* W,
     // The input-gradient products (K-major A, M = token rows) run on CTA pairs; MN-major B boxes are
     // 64 columns wide either way.
     const bool pair = !a_mn && use_pairs(M);
+    CUtensorMap tx;
     if (mode == GEMM_BWD_DGELU_BF16) {
         if (!aux) return GPT_ERR_NULL;
         if ((reinterpret_cast<uintptr_t>(aux) & 15) || (ld_aux % 8)) return GPT_ERR_BAD_ALIGN;
+        // the epilogue warps' 64-column x 32-row boxes of the derivatives
+        rc = make_tmap_bf16_2d(&tx, aux, static_cast<uint64_t>(N), static_cast<uint64_t>(M),
+                               static_cast<uint64_t>(ld_aux) * 2, 64, 32);
+        if (rc) return rc;
         p.aux = aux;
         p.ld_aux = ld_aux;
         p.colsum = colsum;
@@ -262,10 +269,10 @@ int launch_gemm_bf16_bwd(const bf16* A, long long lda, bool a_mn, const bf16* W,
                         : launch_one<gemm::EPI_STORE, 0, 0, 1>(ta, tb, tc, p, s);
         case GEMM_BWD_DGELU_BF16:
             if (gelu == GPT_GELU_TANH)
-                return pair ? launch_one<gemm::EPI_DGELU, 1, 0, 1, 1>(ta, tb, tc, p, s)
-                            : launch_one<gemm::EPI_DGELU, 1, 0, 1>(ta, tb, tc, p, s);
-            return pair ? launch_one<gemm::EPI_DGELU, 0, 0, 1, 1>(ta, tb, tc, p, s)
-                        : launch_one<gemm::EPI_DGELU, 0, 0, 1>(ta, tb, tc, p, s);
+                return pair ? launch_one<gemm::EPI_DGELU, 1, 0, 1, 1>(ta, tb, tc, p, s, &tx)
+                            : launch_one<gemm::EPI_DGELU, 1, 0, 1>(ta, tb, tc, p, s, &tx);
+            return pair ? launch_one<gemm::EPI_DGELU, 0, 0, 1, 1>(ta, tb, tc, p, s, &tx)
+                        : launch_one<gemm::EPI_DGELU, 0, 0, 1>(ta, tb, tc, p, s, &tx);
         default: return GPT_ERR_UNSUPPORTED;
     }
 }

@@ -39,7 +39,8 @@ constexpr int NEPI = 8;  // epilogue warps: two per TMEM lane quarter, each half
 //          launch).
 // EPI_DGELU: out_bf16 = acc * aux, aux the bf16 GELU derivative [M, ld_aux] that the training
 //          forward stored (the MLP's backward through GELU, fused into the product that yields
-//          d loss / d gelu output).
+//          d loss / d gelu output).  Each epilogue warp's 32 x 128 slice of aux is copied by TMA into
+//          shared memory when the warp starts the tile, so it arrives while the products run.
 // EPI_GELU2: gelu'(acc + b) at rows [0, M) of out and gelu(acc + b) at rows [M, 2M) (the training
 //          forward keeps the GELU output for the weight gradient and its derivative for the
 //          backward through GELU; M % 32 == 0).
@@ -69,16 +70,20 @@ struct Params {
 };
 
 // PAIR: a cluster of two CTAs computes one 256 x BN tile with the 2-SM MMA; each CTA stages its
-// own 128 rows of A and half of B's BN rows, so a stage is 32 KB and six fit.
-template <int BN, int PAIR = 0>
+// own 128 rows of A and half of B's BN rows, so a stage is 32 KB and six fit.  AUX (EPI_DGELU):
+// each epilogue warp also stages its 32 x 128 slice of the tile's GELU derivatives (two 64-column
+// TMA boxes, 128-byte swizzle, 8 KB), which costs two stages of the ring.
+template <int BN, int PAIR = 0, int AUX = 0>
 struct Cfg {
     static_assert(BN == 256, "BN");
-    static constexpr int STAGES = PAIR ? 6 : kStages;
+    static constexpr int STAGES = PAIR ? (AUX ? 4 : 6) : (AUX ? 2 : kStages);
     static constexpr int B_ROWS = PAIR ? BN / 2 : BN;         // rows of B this CTA stages
     static constexpr int A_BYTES = BM * BK * 2;
     static constexpr int B_BYTES = B_ROWS * BK * 2;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-    static constexpr int BIAS_OFF = STAGES * STAGE_BYTES;     // one bias slice per epilogue warp
+    static constexpr int AUX_OFF = STAGES * STAGE_BYTES;      // AUX: [NEPI][2 boxes][32 rows][64]
+    static constexpr int AUX_WARP_BYTES = 32 * (BN / (NEPI / 4)) * 2;
+    static constexpr int BIAS_OFF = AUX_OFF + (AUX ? NEPI * AUX_WARP_BYTES : 0);  // a bias slice per epilogue warp
     static constexpr int STG_OFF = BIAS_OFF + NEPI * (BN / (NEPI / 4)) * 4;
     static constexpr int STG_BYTES = 32 * 64;                 // 32 rows x 64 bytes per warp
     static constexpr int BAR_OFF = STG_OFF + NEPI * STG_BYTES;
@@ -154,11 +159,14 @@ GPT_DEVINL float gelu_f(float x) {
 // CTA's TMA loads count on the leader's `full`, the leader's one MMA thread issues the 2-SM MMAs
 // (M = 256) and its commits arrive on `empty` and `tfull` in both CTAs, and both CTAs' epilogue
 // threads arrive on the leader's `tempty`.  Each CTA's epilogue drains its own 128 rows.
+// tmX: EPI_DGELU's map of the GELU derivatives ([M, N] bf16, 64 x 32 boxes, 128-byte swizzle);
+// unused otherwise.
 template <int BN, int EPI, int GELU_TANH, int A_MN = 0, int B_MN = 0, int PAIR = 0>
 __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)  // 10 warps: <= 168 registers per thread
     gemm_bf16_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                 const __grid_constant__ CUtensorMap tmC, const Params p) {
-    using L = Cfg<BN, PAIR>;
+                 const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmX,
+                 const Params p) {
+    using L = Cfg<BN, PAIR, EPI == EPI_DGELU>;
     constexpr int kStages = L::STAGES;
     constexpr int TM = PAIR ? 2 * BM : BM;  // output rows per tile
     constexpr int COLS = L::COLS_PER_WARP;
@@ -172,9 +180,10 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)  // 10 warps: <= 168 regi
     uint64_t* tempty = tfull + 2;
     uint64_t* drain = tempty + 2;
     uint64_t* peer_done = drain + 1;            // PAIR, leader: the peer's producer has finished
+    uint64_t* aux_full = peer_done + 1;         // EPI_DGELU: [NEPI] a warp's derivative slice landed
     volatile unsigned long long* peer_issued =  // PAIR, leader: the peer's count of issued stage loads
-        reinterpret_cast<volatile unsigned long long*>(peer_done + 1);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(peer_done + 2);
+        reinterpret_cast<volatile unsigned long long*>(aux_full + NEPI);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(aux_full + NEPI + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5;
@@ -215,6 +224,7 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)  // 10 warps: <= 168 regi
         }
         mbar_init(drain, 1);
         mbar_init(peer_done, 1);
+        for (int w = 0; w < NEPI; ++w) mbar_init(&aux_full[w], 1);
         *peer_issued = 0ull;
         *abort_flag = 0;
         fence_barrier_init();
@@ -222,6 +232,7 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)  // 10 warps: <= 168 regi
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
         tma_prefetch_desc(&tmC);
+        if (EPI == EPI_DGELU) tma_prefetch_desc(&tmX);
     }
     if (warp == 1) {
         if (PAIR) {
@@ -400,6 +411,9 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)  // 10 warps: <= 168 regi
         const int half = ew >> 2;            // which BN/2 columns of the tile
         int acc = 0;
         uint32_t acc_ph = 0;
+        uint32_t aux_ph = 0;
+        bool aux_pending = false;  // EPI_DGELU: a derivative load of this warp not yet waited for
+        uint8_t* abuf = smem + L::AUX_OFF + ew * L::AUX_WARP_BYTES;  // EPI_DGELU: this warp's slice
         for (int tile = unit0; tile < num_tiles; tile += n_units) {
             int m_blk, n_blk;
             tile_mn(tile, m_blk, n_blk);
@@ -409,6 +423,19 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)  // 10 warps: <= 168 regi
             const int nw0 = n0 + half * COLS;  // first column of this warp's slice
             float* sb = sbias + ew * COLS;  // this warp's private bias slice
             uint8_t* stg = smem + L::STG_OFF + ew * L::STG_BYTES;  // this warp's staging tile
+
+            // EPI_DGELU: this warp's 32 x 128 slice of the GELU derivatives is copied into shared
+            // memory while the tile's products run (rows past M and columns past N read as zero).
+            if (EPI == EPI_DGELU) {
+                __syncwarp();  // every lane's reads of the previous tile's slice are done
+                if (lane == 0) {
+                    fence_proxy_async_shared();
+                    mbar_arrive_expect_tx(&aux_full[ew], static_cast<uint32_t>(L::AUX_WARP_BYTES));
+                    tma_load_2d(abuf, &tmX, &aux_full[ew], nw0, m0 + quarter * 32);
+                    tma_load_2d(abuf + L::AUX_WARP_BYTES / 2, &tmX, &aux_full[ew], nw0 + 64, m0 + quarter * 32);
+                }
+                aux_pending = true;
+            }
 
             // Before the accumulator is ready: this warp's bias slice into shared memory.
             if (EPI != EPI_CE) {
@@ -421,35 +448,17 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)  // 10 warps: <= 168 regi
             }
             long long tgt = -1;
             if (EPI == EPI_CE && row_ok) tgt = p.targets[row];
-            // EPI_DGELU: this row's slice of the next tile's GELU derivatives goes to L2 now (one
-            // tile ahead, so its chunk loads below hit L2), then the first chunk's values are loaded
-            // before the accumulator wait
-            if (EPI == EPI_DGELU && tile + n_units < num_tiles) {
-                int m_nx, n_nx;
-                tile_mn(tile + n_units, m_nx, n_nx);
-                const int row_nx = m_nx * TM + static_cast<int>(rank) * BM + quarter * 32 + lane;
-                const int n_first = n_nx * BN + half * COLS;
-                if (row_nx < p.M && n_first + COLS <= p.N)
-                    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(
-                                     p.aux + static_cast<long long>(row_nx) * p.ld_aux + n_first),
-                                 "r"(static_cast<uint32_t>(COLS * 2))
-                                 : "memory");
-            }
-            uint32_t aux_next[EPI == EPI_DGELU ? 16 : 1];
-            bool aux_ok = false;
-            if (EPI == EPI_DGELU && row_ok && nw0 + 32 <= p.N) {
-                const uint4* an = reinterpret_cast<const uint4*>(p.aux + static_cast<long long>(row) * p.ld_aux + nw0);
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const uint4 w = __ldcg(an + q);
-                    aux_next[4 * q] = w.x, aux_next[4 * q + 1] = w.y, aux_next[4 * q + 2] = w.z, aux_next[4 * q + 3] = w.w;
-                }
-                aux_ok = true;
-            }
 
             const bool got = mbar_wait(&tfull[acc], acc_ph, abort_flag);
             __syncwarp();  // tcgen05.ld below is warp-collective
             if (!__all_sync(0xffffffffu, got)) break;
+            if (EPI == EPI_DGELU) {
+                const bool ag = mbar_wait(&aux_full[ew], aux_ph, abort_flag);
+                __syncwarp();
+                if (!__all_sync(0xffffffffu, ag)) break;
+                aux_ph ^= 1u;
+                aux_pending = false;
+            }
             tc_fence_after();
             const uint32_t tbase = tmem_base + static_cast<uint32_t>(acc * BN + half * COLS) +
                                    (static_cast<uint32_t>(quarter * 32) << 16);
@@ -521,37 +530,21 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)  // 10 warps: <= 168 regi
 #pragma unroll
                             for (int j = 0; j < 32; ++j) v[j] = gelu_f<GELU_TANH>(v[j]);
                         }
-                        if (EPI == EPI_DGELU && row_ok) {
-                            // this row's 32 pre-activations of the chunk: from the registers loaded
-                            // one chunk ahead (whole chunks), else element by element
-                            float z[32];
-                            if (full_chunk && aux_ok) {
+                        if (EPI == EPI_DGELU) {
+                            // this row's 32 derivatives of the chunk from the staged slice: row `lane`
+                            // of box cc / 64, 16-byte chunks (cc % 64) / 8 .. + 3, swizzled by row % 8
+                            const uint8_t* rp = abuf + (cc >> 6) * (L::AUX_WARP_BYTES / 2) + lane * 128;
+                            const int c16 = (cc & 63) >> 3;
 #pragma unroll
-                                for (int q = 0; q < 16; ++q) {
-                                    z[2 * q] = __uint_as_float(aux_next[q] << 16);
-                                    z[2 * q + 1] = __uint_as_float(aux_next[q] & 0xffff0000u);
+                            for (int q = 0; q < 4; ++q) {
+                                const uint4 w = *reinterpret_cast<const uint4*>(rp + (((c16 + q) ^ (lane & 7)) << 4));
+                                const uint32_t u4[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) {
+                                    v[8 * q + 2 * e] *= __uint_as_float(u4[e] << 16);
+                                    v[8 * q + 2 * e + 1] *= __uint_as_float(u4[e] & 0xffff0000u);
                                 }
-                            } else {
-                                const bf16* ap = p.aux + static_cast<long long>(row) * p.ld_aux + n;
-#pragma unroll
-                                for (int j = 0; j < 32; ++j)
-                                    z[j] = n + j < p.N ? __bfloat162float(ap[j]) : 0.f;
                             }
-                            // the next chunk's pre-activations, loaded while this one is finished
-                            aux_ok = false;
-                            if (cc + 32 < COLS && nw0 + cc + 64 <= p.N) {
-                                const uint4* an = reinterpret_cast<const uint4*>(
-                                    p.aux + static_cast<long long>(row) * p.ld_aux + n + 32);
-#pragma unroll
-                                for (int q = 0; q < 4; ++q) {
-                                    const uint4 w = __ldcg(an + q);
-                                    aux_next[4 * q] = w.x, aux_next[4 * q + 1] = w.y;
-                                    aux_next[4 * q + 2] = w.z, aux_next[4 * q + 3] = w.w;
-                                }
-                                aux_ok = true;
-                            }
-#pragma unroll
-                            for (int j = 0; j < 32; ++j) v[j] *= z[j];
                         }
                         if (EPI == EPI_CE) {
                             float cmax = -INFINITY;
@@ -587,7 +580,6 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)  // 10 warps: <= 168 regi
                             }
                         }
                         if (!band_ok) continue;  // warp-uniform: no row of this band exists
-#pragma unroll
                         float vg[EPI == EPI_GELU2 ? 32 : 1];  // EPI_GELU2: the GELU outputs of pass 1
                         if (EPI == EPI_GELU2) {
 #pragma unroll
@@ -643,6 +635,9 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)  // 10 warps: <= 168 regi
             if (acc == 0) acc_ph ^= 1u;
         }
         if (lane == 0) bulk_wait_all();  // this warp's stores and reduce-adds have completed
+        // a derivative load issued for a tile this warp did not finish (time-out) lands before exit
+        if (EPI == EPI_DGELU && aux_pending && lane == 0) mbar_drain(&aux_full[ew], aux_ph);
+        __syncwarp();
     }
 
     __syncthreads();
