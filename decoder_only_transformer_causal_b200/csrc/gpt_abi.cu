@@ -1226,7 +1226,8 @@ GPT_API int gpt_forward_train(const gpt_config_t* cfg, const void* weights, cons
         void* u2 = L + A.u2;
         void* pre = L + A.pre;
         void* hh = L + A.h;
-        GPT_TRY(launch_layernorm(x_in, W.layer(l, W_LN1_W), W.bias(l, W_LN1_B), u1, N, C, dt, s));
+        // ln_1 also copies x_in to x_mid, which attn c_proj then adds into (x_in stays for the backward)
+        GPT_TRY(launch_layernorm(x_in, W.layer(l, W_LN1_W), W.bias(l, W_LN1_B), u1, N, C, dt, s, x_mid));
         if (bf) {
             GPT_TRY(launch_gemm_bf16(static_cast<const bf16*>(u1), C, static_cast<const bf16*>(W.layer(l, W_ATTN_W)), C,
                                      static_cast<const bf16*>(W.bias(l, W_ATTN_B)), qkv, 3LL * C, N, 3 * C, C,
@@ -1244,7 +1245,6 @@ GPT_API int gpt_forward_train(const gpt_config_t* cfg, const void* weights, cons
                              static_cast<long long>(C) * T, hs, C, lse};
             GPT_TRY(launch_attention_f32(AL, B, nh, T, hs, s));
         }
-        GPT_TRY(cuda_status(cudaMemcpyAsync(x_mid, x_in, static_cast<size_t>(N) * C * 4, cudaMemcpyDeviceToDevice, s)));
         if (bf)
             GPT_TRY(launch_gemm_bf16(static_cast<const bf16*>(y), C, static_cast<const bf16*>(W.layer(l, W_PROJ_W)), C,
                                      static_cast<const bf16*>(W.bias(l, W_PROJ_B)), x_mid, C, N, C, C, GPT_EPI_RESID,
@@ -1253,7 +1253,8 @@ GPT_API int gpt_forward_train(const gpt_config_t* cfg, const void* weights, cons
             GPT_TRY(launch_linear_f32(static_cast<const float*>(y), C, static_cast<const float*>(W.layer(l, W_PROJ_W)),
                                       static_cast<const float*>(W.bias(l, W_PROJ_B)), x_mid, C, N, C, C, GPT_EPI_RESID,
                                       cfg->gelu, s));
-        GPT_TRY(launch_layernorm(x_mid, W.layer(l, W_LN2_W), W.bias(l, W_LN2_B), u2, N, C, dt, s));
+        // ln_2 also copies x_mid to the next layer's x_in (x_out), which mlp c_proj adds into
+        GPT_TRY(launch_layernorm(x_mid, W.layer(l, W_LN2_W), W.bias(l, W_LN2_B), u2, N, C, dt, s, x_out));
         // c_fc keeps the GELU output (for the weight gradient) and, in the bf16 path, the GELU
         // derivative at the pre-activation in `pre` (for the backward through GELU): one product
         // writing both when h directly follows pre, else a store, a GELU pass and an in-place
@@ -1278,7 +1279,6 @@ GPT_API int gpt_forward_train(const gpt_config_t* cfg, const void* weights, cons
                 GPT_TRY(launch_gelu_deriv_inplace(pre, static_cast<long long>(N) * 4 * C, dt,
                                                   cfg->gelu == GPT_GELU_TANH, s));
         }
-        GPT_TRY(cuda_status(cudaMemcpyAsync(x_out, x_mid, static_cast<size_t>(N) * C * 4, cudaMemcpyDeviceToDevice, s)));
         if (bf)
             GPT_TRY(launch_gemm_bf16(static_cast<const bf16*>(hh), 4LL * C, static_cast<const bf16*>(W.layer(l, W_FC2_W)),
                                      4LL * C, static_cast<const bf16*>(W.bias(l, W_FC2_B)), x_out, C, N, C, 4 * C,

@@ -82,8 +82,9 @@ int make_tmap_bf16_4d(CUtensorMap* m, const void* base, const uint64_t dims[4],
 // ---- row-wise kernels (rowwise.cu)
 int launch_embed(const void* wte, const void* wpe, const int64_t* idx, float* x, int B, int T,
                  int C, int V, int dtype, int32_t* status, cudaStream_t s);
+// xcopy (optional, 16-byte aligned): also writes the input rows there unchanged.
 int launch_layernorm(const float* x, const void* w, const void* b, void* out, int rows, int C,
-                     int dtype, cudaStream_t s);
+                     int dtype, cudaStream_t s, float* xcopy = nullptr);
 // bf16 path: combine the lm_head epilogue's partials into per-row losses.
 int launch_ce_rows_from_parts(const float2* part, int n_part, const float* tlogit,
                               const int64_t* targets, int rows, int V, float* row_loss,

@@ -102,9 +102,12 @@ __global__ void embed_rows_kernel(const Tw* __restrict__ wte, const Tw* __restri
 // §2.5 (A)).  The row stays in registers: mean, then sum of squared deviations.
 constexpr int kLnMaxVec = 16;  // float4 per lane -> C <= 2048
 
+// xcopy (optional): the input rows are also written there unchanged (the training forward keeps
+// each residual stream state for the backward while the next projection adds into the copy).
 template <typename To, int VEC>  // VEC = float4 per lane, ceil(C / 128): registers sized to the row
 __global__ void layernorm_kernel(const float* __restrict__ x, const To* __restrict__ w,
-                                 const To* __restrict__ bias, To* __restrict__ out, int rows, int C) {
+                                 const To* __restrict__ bias, To* __restrict__ out, int rows, int C,
+                                 float* __restrict__ xcopy) {
     griddep_launch_dependents();
     griddep_wait();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -123,6 +126,14 @@ __global__ void layernorm_kernel(const float* __restrict__ x, const To* __restri
         }
     }
     const float mean = warp_sum(s) / C;
+    if (xcopy) {
+        float* cr = xcopy + static_cast<long long>(row) * C;
+#pragma unroll
+        for (int k = 0; k < VEC; ++k) {
+            const int j = lane + 32 * k;
+            if (j < nv) store4(cr + 4 * j, v[k]);
+        }
+    }
     float ss = 0.f;
 #pragma unroll
     for (int k = 0; k < VEC; ++k) {
@@ -289,27 +300,30 @@ int launch_embed(const void* wte, const void* wpe, const int64_t* idx, float* x,
 
 namespace {
 template <typename To, int VEC>
-int launch_ln_vec(const float* x, const void* w, const void* b, void* out, int rows, int C, cudaStream_t s) {
+int launch_ln_vec(const float* x, const void* w, const void* b, void* out, int rows, int C, float* xcopy,
+                  cudaStream_t s) {
     const unsigned blocks = (rows + kWarpsPerBlock - 1) / kWarpsPerBlock;
     return launch_overlapped(layernorm_kernel<To, VEC>, dim3(blocks), dim3(32 * kWarpsPerBlock), 0, s, x,
-                             static_cast<const To*>(w), static_cast<const To*>(b), static_cast<To*>(out), rows, C);
+                             static_cast<const To*>(w), static_cast<const To*>(b), static_cast<To*>(out), rows, C,
+                             xcopy);
 }
 
 template <typename To, int VEC = 1>
-int launch_ln(const float* x, const void* w, const void* b, void* out, int rows, int C, cudaStream_t s) {
+int launch_ln(const float* x, const void* w, const void* b, void* out, int rows, int C, float* xcopy,
+              cudaStream_t s) {
     if constexpr (VEC < kLnMaxVec) {
-        if (C > 128 * VEC) return launch_ln<To, VEC + 1>(x, w, b, out, rows, C, s);
+        if (C > 128 * VEC) return launch_ln<To, VEC + 1>(x, w, b, out, rows, C, xcopy, s);
     }
-    return launch_ln_vec<To, VEC>(x, w, b, out, rows, C, s);
+    return launch_ln_vec<To, VEC>(x, w, b, out, rows, C, xcopy, s);
 }
 }  // namespace
 
 int launch_layernorm(const float* x, const void* w, const void* b, void* out, int rows, int C,
-                     int dtype, cudaStream_t s) {
+                     int dtype, cudaStream_t s, float* xcopy) {
     if (C > 4 * 32 * kLnMaxVec || (C & 3)) return GPT_ERR_UNSUPPORTED;
     if (rows == 0) return GPT_OK;
-    if (dtype == GPT_DTYPE_BF16) return launch_ln<bf16>(x, w, b, out, rows, C, s);
-    return launch_ln<float>(x, w, b, out, rows, C, s);
+    if (dtype == GPT_DTYPE_BF16) return launch_ln<bf16>(x, w, b, out, rows, C, xcopy, s);
+    return launch_ln<float>(x, w, b, out, rows, C, xcopy, s);
 }
 
 int launch_ce_rows_from_parts(const float2* part, int n_part, const float* tlogit,
