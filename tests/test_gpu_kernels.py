@@ -86,6 +86,24 @@ def test_linear_bf16(M, N, K, epi):
     assert err <= tol, err
 
 
+def test_linear_bf16_gelu_wide_range():
+    """Pre-activations spread over about [-60, 60]: the erf-form GELU epilogue must give x for large
+    x and 0 for large negative x (its polynomial's argument is clamped) and stay within bf16's
+    relative step everywhere."""
+    from decoder_only_transformer_causal_b200 import native
+    M, N, K = 512, 512, 64
+    x = gen((M, K), 1.0, 16)
+    W = gen((N, K), 20.0 / math.sqrt(K), 17)
+    b = gen((N,), 1.0, 18)
+    ref = oracle.gelu(oracle.linear(f64(x), f64(W), f64(b)), "erf")
+    out = native.linear(x.cuda(), W.cuda(), b.cuda(), epilogue=native.GPT_EPI_GELU, gelu=native.GELUS["erf"])
+    torch.cuda.synchronize()
+    got = f64(out)
+    assert float(np.abs(ref).max()) > 40.0
+    err = np.abs(got - ref)
+    assert float((err - (4e-3 * np.abs(ref) + 1e-4)).max()) <= 0.0, float(err.max())
+
+
 @pytest.mark.parametrize("M,N,K", [(64, 96, 40), (300, 200, 136), (512, 1536, 128)])
 @pytest.mark.parametrize("epi", [0, 1, 2])
 def test_linear_f32(M, N, K, epi):
