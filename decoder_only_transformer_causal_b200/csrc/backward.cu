@@ -483,11 +483,99 @@ __global__ void gelu_backward_kernel(const float* __restrict__ dh, const E* __re
 
 // ------------------------------------------------------------------ embedding backward
 // dwte[v] += sum of dx[r] over rows r with idx[r] = v, in row order; dwpe[t] += sum over the
-// batch of dx[b, t].  The rows are ordered by (token, row) with a bitonic sort of 64-bit keys in
-// one CTA's shared memory (N <= kEmbSortMax rows), then each run of equal tokens is summed by one
-// warp in row order.
+// batch of dx[b, t].  The rows are ordered by (token, row) in one CTA's shared memory (N <=
+// kEmbSortMax rows), then each run of equal tokens is summed by one warp in row order.  The order
+// comes from a stable radix sort of 32-bit keys token << 14 | row on the token bits, 8 at a time
+// from the least significant (rows start in order and every pass keeps equal digits in order),
+// when the tokens fit 18 bits; else from a bitonic sort of 64-bit keys.
 constexpr int kEmbSortMax = 16384;
 constexpr int kEmbSortThreads = 1024;
+constexpr int kEmbRowBits = 14;  // rows < kEmbSortMax
+constexpr int kEmbRadixMaxV = (1 << (32 - kEmbRowBits)) - 1;  // tokens 0..V (V: a bad index) in 18 bits
+
+__global__ void __launch_bounds__(kEmbSortThreads)
+    embed_radix_sort_kernel(const int64_t* __restrict__ idx, int N, int V, unsigned long long* __restrict__ sorted,
+                            int32_t* status) {
+    griddep_launch_dependents();
+    griddep_wait();
+    extern __shared__ uint32_t sbuf[];  // two buffers of N keys
+    __shared__ uint32_t whist[32][257];  // per warp: digit counts, then running offsets
+    __shared__ uint32_t s_dbase[256];
+    uint32_t* ka = sbuf;
+    uint32_t* kb = sbuf + N;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int i = threadIdx.x; i < N; i += kEmbSortThreads) {
+        long long t = __ldcg(idx + i);
+        if (t < 0 || t >= V) {
+            set_status(status, GPT_ERR_INDEX);
+            t = V;  // sorts after every valid token; skipped by the run kernel
+        }
+        ka[i] = (static_cast<uint32_t>(t) << kEmbRowBits) | static_cast<uint32_t>(i);
+    }
+    const int nb = 32 - __clz(V);  // bits of the largest key token, V
+    const int E = (N + 31) / 32;   // each warp's contiguous chunk
+    const int w0 = min(N, warp * E), w1 = min(N, w0 + E);
+    for (int shift = kEmbRowBits; shift < kEmbRowBits + nb; shift += 8) {
+        for (int d = lane; d < 256; d += 32) whist[warp][d] = 0;
+        __syncthreads();  // the keys (first pass: their construction) and the zeroed counts
+        for (int i = w0 + lane; i < w1; i += 32) atomicAdd(&whist[warp][(ka[i] >> shift) & 255u], 1u);
+        __syncthreads();
+        // digit d's slots: after every smaller digit, then warp by warp
+        uint32_t tot = 0;
+        if (threadIdx.x < 256) {
+            const int d = threadIdx.x;
+            for (int w = 0; w < 32; ++w) {
+                const uint32_t c = whist[w][d];
+                whist[w][d] = tot;
+                tot += c;
+            }
+            s_dbase[d] = tot;
+        }
+        __syncthreads();
+        if (warp == 0) {  // exclusive scan of the 256 digit totals, eight digits a lane
+            uint32_t v[8], sum = 0;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                v[k] = s_dbase[8 * lane + k];
+                sum += v[k];
+            }
+            uint32_t incl = sum;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t n = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += n;
+            }
+            uint32_t run = incl - sum;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                s_dbase[8 * lane + k] = run;
+                run += v[k];
+            }
+        }
+        __syncthreads();
+        // stable scatter: each warp walks its chunk in order, lanes with equal digits in lane order
+        for (int base = w0; base < w1; base += 32) {
+            const int i = base + lane;
+            const bool ok = i < w1;
+            const uint32_t k = ok ? ka[i] : 0u;
+            const uint32_t d = ok ? (k >> shift) & 255u : 256u + static_cast<uint32_t>(lane);
+            const uint32_t peers = __match_any_sync(0xffffffffu, d);
+            const uint32_t rank = __popc(peers & ((1u << lane) - 1u));
+            if (ok) kb[s_dbase[d] + whist[warp][d] + rank] = k;
+            __syncwarp();
+            if (ok && rank == 0) whist[warp][d] += __popc(peers);
+            __syncwarp();
+        }
+        __syncthreads();
+        uint32_t* t = ka;
+        ka = kb;
+        kb = t;
+    }
+    for (int i = threadIdx.x; i < N; i += kEmbSortThreads) {
+        const uint32_t k = ka[i];
+        sorted[i] = (static_cast<unsigned long long>(k >> kEmbRowBits) << 32) | (k & ((1u << kEmbRowBits) - 1u));
+    }
+}
 
 __global__ void __launch_bounds__(kEmbSortThreads)
     embed_sort_kernel(const int64_t* __restrict__ idx, int N, int V, unsigned long long* __restrict__ sorted,
@@ -544,13 +632,26 @@ __global__ void embed_runs_kernel(const unsigned long long* __restrict__ sorted,
     int end = warp + 1;
     while (end < N && static_cast<unsigned>(__ldcg(sorted + end) >> 32) == tok) ++end;
     float* out = dwte + static_cast<long long>(tok) * C;
-    for (int c = lane; c < C; c += 32) {
-        float v = 0.f;
+    // lane l owns columns c0 + l + 32 j, j < 8: a row's eight loads are issued together
+    for (int c0 = 0; c0 < C; c0 += 256) {
+        float v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[j] = 0.f;
         for (int s = warp; s < end; ++s) {
             const unsigned r = static_cast<unsigned>(__ldcg(sorted + s) & 0xffffffffull);
-            v += __ldcg(dx + static_cast<long long>(r) * C + c);
+            const float* xr = dx + static_cast<long long>(r) * C + c0 + lane;
+            float t[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) t[j] = c0 + lane + 32 * j < C ? __ldcg(xr + 32 * j) : 0.f;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) v[j] += t[j];
         }
-        out[c] = __ldcg(out + c) + v;
+        float o[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) o[j] = c0 + lane + 32 * j < C ? __ldcg(out + c0 + lane + 32 * j) : 0.f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            if (c0 + lane + 32 * j < C) out[c0 + lane + 32 * j] = o[j] + v[j];
     }
 }
 
@@ -672,13 +773,23 @@ int launch_embed_backward(const int64_t* idx, const float* dx, int B, int T, int
                           unsigned long long* sorted, int32_t* status, cudaStream_t s) {
     const int N = B * T;
     if (N > kEmbSortMax) return GPT_ERR_UNSUPPORTED;
-    int n2 = 1;
-    while (n2 < N) n2 <<= 1;
-    const size_t smem = static_cast<size_t>(n2) * sizeof(unsigned long long);
-    static size_t opted[kMaxDevices] = {};
-    int rc = opt_in_smem(reinterpret_cast<const void*>(embed_sort_kernel), smem, opted);
-    if (rc) return rc;
-    rc = launch_overlapped(embed_sort_kernel, dim3(1), dim3(kEmbSortThreads), smem, s, idx, N, V, sorted, status);
+    int rc;
+    if (V <= kEmbRadixMaxV) {
+        const size_t smem = static_cast<size_t>(2) * N * sizeof(uint32_t);
+        static size_t opted_r[kMaxDevices] = {};
+        rc = opt_in_smem(reinterpret_cast<const void*>(embed_radix_sort_kernel), smem, opted_r);
+        if (rc) return rc;
+        rc = launch_overlapped(embed_radix_sort_kernel, dim3(1), dim3(kEmbSortThreads), smem, s, idx, N, V, sorted,
+                               status);
+    } else {
+        int n2 = 1;
+        while (n2 < N) n2 <<= 1;
+        const size_t smem = static_cast<size_t>(n2) * sizeof(unsigned long long);
+        static size_t opted[kMaxDevices] = {};
+        rc = opt_in_smem(reinterpret_cast<const void*>(embed_sort_kernel), smem, opted);
+        if (rc) return rc;
+        rc = launch_overlapped(embed_sort_kernel, dim3(1), dim3(kEmbSortThreads), smem, s, idx, N, V, sorted, status);
+    }
     if (rc) return rc;
     rc = launch_overlapped(embed_runs_kernel, dim3((N * 32 + 255) / 256), dim3(256), 0, s,
                            static_cast<const unsigned long long*>(sorted), N, V, dx, C, dwte);
