@@ -15,11 +15,11 @@
 //   warps 2-5   softmax, one query row per thread: load the S row from TMEM, mask the
 //               diagonal tile, update the running maximum / sum, write P (bf16) to TMEM,
 //               rescale O in TMEM when the maximum moved by more than 2^8, and finally
-//               write y = O / l.  3-input maxima cut the issue count; off the diagonal the
-//               exponent is one scalar FMA per score (scalar math measured ~1% faster than packed
-//               f32x2 there, whose register pairs cost moves); on the diagonal tile the 32-column
-//               chunks right of a warp's last row are fully masked and skip the exponential.  The exponential (MUFU ex2, 16 per clock
-//               per SM) is the unit this kernel is bound by at head size 64.
+//               write y = O / l.  3-input maxima cut the issue count; the exponents' arguments
+//               and the row sums are packed f32x2 FMAs and adds (one instruction per two
+//               scores); on the diagonal tile the 32-column chunks right of a warp's last row are
+//               fully masked and skip the exponential, one branch per chunk.  The exponential
+//               (MUFU ex2, 16 per clock per SM) bounds this kernel at head size 64.
 // TMEM columns: S [0,128), P [128,192) (bf16 pairs), O [192,256).  256 columns and 80 KB of
 // shared memory let two CTAs share an SM, so one CTA's softmax overlaps the other's MMAs.
 //
@@ -247,7 +247,6 @@ __global__ void __launch_bounds__(THREADS, 2)
             }
             const bool diag = (j == n_kv - 1);
             const float SCs = p.scale_log2, NMs = -m_used;
-            float accs[4] = {0.f, 0.f, 0.f, 0.f};
             uint64_t acc4[4] = {0, 0, 0, 0};
             uint32_t pk0[32], pk1[32];
             // Off the diagonal every column is live (a loop with no per-column test).  On the
@@ -255,32 +254,42 @@ __global__ void __launch_bounds__(THREADS, 2)
             // every lane: P is 0 there and no exponential is evaluated.
             const int live_cols = diag ? (quarter + 1) * 32 : BKV;  // warp-uniform
             if (!diag) {
+                const uint64_t SC2 = f2_pack(SCs, SCs), NM2 = f2_pack(NMs, NMs);
 #pragma unroll
                 for (int c = 0; c < BKV; c += 2) {
-                    const float p0 = exp2_approx(fmaf(s[c], SCs, NMs)), p1 = exp2_approx(fmaf(s[c + 1], SCs, NMs));
-                    accs[(c >> 1) & 3] += p0 + p1;
+                    float x0, x1;
+                    f2_unpack(f2_fma(f2_pack(s[c], s[c + 1]), SC2, NM2), x0, x1);
+                    const float p0 = exp2_approx(x0), p1 = exp2_approx(x1);
+                    acc4[(c >> 1) & 3] = f2_add(acc4[(c >> 1) & 3], f2_pack(p0, p1));
                     if (c < 64) pk0[c / 2] = pack_bf16x2(p0, p1);
                     else pk1[(c - 64) / 2] = pack_bf16x2(p0, p1);
                 }
             } else {
                 const uint64_t SC = f2_pack(p.scale_log2, p.scale_log2), NM = f2_pack(-m_used, -m_used);
 #pragma unroll
-                for (int c = 0; c < BKV; c += 2) {
-                    float p0 = 0.f, p1 = 0.f;
-                    if (c < live_cols) {
-                        float x0, x1;
-                        f2_unpack(f2_fma(f2_pack(s[c], s[c + 1]), SC, NM), x0, x1);
-                        p0 = exp2_approx(x0);
-                        p1 = exp2_approx(x1);
-                        acc4[(c >> 1) & 3] = f2_add(acc4[(c >> 1) & 3], f2_pack(p0, p1));
+                for (int ch = 0; ch < BKV / 32; ++ch) {
+                    if (ch * 32 < live_cols) {  // warp-uniform: one branch per 32-column chunk
+#pragma unroll
+                        for (int c = ch * 32; c < ch * 32 + 32; c += 2) {
+                            float x0, x1;
+                            f2_unpack(f2_fma(f2_pack(s[c], s[c + 1]), SC, NM), x0, x1);
+                            const float p0 = exp2_approx(x0), p1 = exp2_approx(x1);
+                            acc4[(c >> 1) & 3] = f2_add(acc4[(c >> 1) & 3], f2_pack(p0, p1));
+                            if (c < 64) pk0[c / 2] = pack_bf16x2(p0, p1);
+                            else pk1[(c - 64) / 2] = pack_bf16x2(p0, p1);
+                        }
+                    } else {
+#pragma unroll
+                        for (int c = ch * 32; c < ch * 32 + 32; c += 2) {
+                            if (c < 64) pk0[c / 2] = 0u;
+                            else pk1[(c - 64) / 2] = 0u;
+                        }
                     }
-                    if (c < 64) pk0[c / 2] = pack_bf16x2(p0, p1);
-                    else pk1[(c - 64) / 2] = pack_bf16x2(p0, p1);
                 }
             }
             float a0, a1, b0, b1, c0, c1, d0, d1;
             f2_unpack(acc4[0], a0, a1); f2_unpack(acc4[1], b0, b1); f2_unpack(acc4[2], c0, c1); f2_unpack(acc4[3], d0, d1);
-            const float rs = ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1)) + ((accs[0] + accs[1]) + (accs[2] + accs[3]));
+            const float rs = ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
             l = l * alpha + rs;
             // P_j may overwrite P_{j-1} and O may be rescaled only after O += P_{j-1} V_{j-1}.
             if (j > 0) {
