@@ -51,7 +51,7 @@ constexpr int kMaxRows = 16;     // sequences per launch (the mma's M)
 constexpr int kTile = 8;         // weight rows per tile (the mma's N)
 constexpr int kPad = 8;          // bf16 elements of padding per staged row
 constexpr int kChunk = 32;       // keys per attention chunk: a lane per key
-constexpr int kMaxCtaSplit = 4;  // CTAs sharing one (sequence, head): 4 measured best at B 1 (of 1, 4, 12)
+constexpr int kMaxCtaSplit = 4;  // CTAs sharing one (sequence, head): 4 measured best at B 1 (of 1, 4, 6, 8, 12)
 constexpr int kMaxHs = 64;       // head size (every GPT-2 size has 64)
 constexpr int kMaxC = 1024;      // a LayerNorm row lives in registers: C / 128 float4 per lane
 constexpr int kResidCols = 32;   // residual columns one CTA may own
